@@ -1,0 +1,504 @@
+"""Benchmark of the paged-KV-cache decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload llama13b_mix|long_fp8|...] [--also long_fp8] [--no-e2e]
+
+A step is one pass of the whole hot path over the batch: host block bookkeeping
+(C++), one metadata upload, block-table patch, copy-on-write block copies, the
+KV-cache write of every sequence's new token, and paged decode attention (plan,
+partition kernel, log-sum-exp merge). Each sequence appends one token per step,
+so contexts grow by one token per step, as in serving.
+
+Metric: KV-read GB/s = the bytes a decode step must move at minimum (every
+context token's K and V row once per kv head, q, out, block-table entries,
+context lengths) / device time of the whole step; also sequence-tokens/s
+(context tokens attended per second). The KV read per step (10.5 GB for the 13B
+mix, 2.1 GB for the 32K fp8 case) is far larger than the 126 MB L2, so no flush
+is needed between steps.
+
+N > 1 (torchrun): replicas. Each rank runs the same workload on its own GPU with
+no collective on the data path (sequences are independent); the step time is the
+max over ranks and `value` is the sum of all ranks' bytes over that time.
+
+--impl reference times the float64 CPU oracle (the correctness reference) on a
+bounded sample of the same workload, on the host's cores, on rank 0 only.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "paged decode attention KV-read GB/s (% of B200 HBM peak); seq-tokens/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def decode_bytes(lens, hkv, hq, d, kv_bytes, q_bytes, bs) -> int:
+    """Algorithmic bytes of one decode step: K and V of every context token once per
+    kv head, q in, out back, the block-table entries read, the context lengths."""
+    lens = np.asarray(lens, dtype=np.int64)
+    kv = int(2 * lens.sum() * hkv * d * kv_bytes)
+    s = len(lens)
+    return kv + 2 * s * hq * d * q_bytes + int(4 * ((lens + bs - 1) // bs).sum()) + 4 * s
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (replicas: only timing is reduced across ranks)
+# ---------------------------------------------------------------------------
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world, backend):
+    if world <= 1:
+        return None
+    import datetime
+    import torch.distributed as dist
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def reduce_max(x: float, dist, device=None) -> float:
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def reduce_sum(x: float, dist, device=None) -> float:
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier(dist, device=None):
+    if dist is not None:
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# our implementation
+# ---------------------------------------------------------------------------
+
+def build_engine(w, growth, device):
+    """Engine for workload `w` with room for `growth` more tokens per sequence; the
+    cache is filled with seeded N(0,1) draws on the device; every sequence holds its
+    history (L - 1 tokens), so the timed steps append from position L - 1."""
+    import torch
+    import synthetic
+    from paged_kv_cache_436_b200.engine import DecodeEngine
+    eng = DecodeEngine(num_seqs=w.num_seqs, num_q_heads=w.num_q_heads, num_kv_heads=w.num_kv_heads,
+                       head_dim=w.head_dim, block_size=w.block_size, kv_dtype=w.kv_dtype, q_dtype=w.q_dtype,
+                       num_blocks=w.num_blocks, initial_order=w.initial_order,
+                       max_blocks_per_seq=w.max_blocks_per_seq(growth),
+                       max_context_len=w.max_context_len + growth, device=device)
+    if w.kv_dtype == "e4m3":
+        kc, ks = synthetic.normal_e4m3_codes(tuple(eng.k_cache.shape), w.seed * 10 + 1, device)
+        eng.k_cache.copy_(kc)
+        del kc
+        vc, vs = synthetic.normal_e4m3_codes(tuple(eng.v_cache.shape), w.seed * 10 + 2, device)
+        eng.v_cache.copy_(vc)
+        del vc
+        eng.cache.desc.k_scale, eng.cache.desc.v_scale = ks, vs
+    else:
+        synthetic.fill_normal_(eng.k_cache, w.kv_dtype, w.seed * 10 + 1)
+        synthetic.fill_normal_(eng.v_cache, w.kv_dtype, w.seed * 10 + 2)
+    for s, L in enumerate(w.context_lens):
+        eng.extend(s, L - 1)
+    eng.upload_tables()
+    torch.cuda.synchronize(device)
+    return eng
+
+
+class StepRunner:
+    """Runs engine steps with events around the partition kernel (decode stage 1)."""
+
+    def __init__(self, eng, w, n_inputs, device):
+        import torch
+        import synthetic
+        import paged_kv_cache_436_b200 as pa
+        self.pa, self.torch = pa, torch
+        self.eng, self.w, self.device = eng, w, device
+        self.inputs = []
+        for i in range(n_inputs):
+            q, k, v = synthetic.step_inputs(w, i, device=device)
+            self.inputs.append((q, k, v))
+        self.out = torch.empty_like(self.inputs[0][0])
+        self.stream = torch.cuda.current_stream(device)
+        self.kv_bytes = 1 if w.kv_dtype == "e4m3" else 2
+        self.q_bytes = 2
+
+    def step(self, i, ev_pair=None, host=None):
+        """One step. Returns (decode bytes, kernel launches). With `host`, the step's
+        q/k/v come from pinned host buffers and `out` goes back to a pinned buffer."""
+        pa, eng, w = self.pa, self.eng, self.w
+        if host is None:
+            q, k, v = self.inputs[i % len(self.inputs)]
+        else:
+            hq, hk, hv, hout, dq, dk, dv = host
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            q, k, v = dq, dk, dv
+        slots, cows, lens, upd = eng.bookkeeping()
+        launches = 0
+        if upd.shape[0]:
+            pa.block_table_update(upd, eng.bt_dev)
+            launches += 1
+        if cows.shape[0]:
+            pa.copy_blocks(cows, eng.cache)
+            launches += 1
+        pa.reshape_and_cache(k, v, slots, eng.cache)
+        eng.lens_dev = lens
+        launches += 1
+        eng.run_decode(q, self.out, w.scale, stage=0)
+        if ev_pair is not None:
+            ev_pair[0].record(self.stream)
+        eng.run_decode(q, self.out, w.scale, stage=1)
+        if ev_pair is not None:
+            ev_pair[1].record(self.stream)
+        eng.run_decode(q, self.out, w.scale, stage=2)
+        launches += 3 if eng.max_context_len > 512 else 2
+        if host is not None:
+            hout.copy_(self.out, non_blocking=True)
+        nbytes = decode_bytes(eng.lens, w.num_kv_heads, w.num_q_heads, w.head_dim, self.kv_bytes,
+                              self.q_bytes, w.block_size)
+        return nbytes, launches
+
+
+def time_ours(w, steps, warmup, device, dist, e2e=True, clocks=True, local_rank=0):
+    import torch
+    n_e2e = steps if e2e else 0
+    growth = warmup + steps + (warmup + n_e2e if e2e else 0) + 2
+    eng = build_engine(w, growth, device)
+    run = StepRunner(eng, w, 4, device)
+    for i in range(warmup):
+        run.step(i)
+    torch.cuda.synchronize(device)
+    barrier(dist, device)
+    sampler = ClockSampler(local_rank) if clocks else None
+    if sampler:
+        sampler.start()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    torch.cuda.synchronize(device)
+    barrier(dist, device)
+    total_bytes, launches, lens_sum, kbytes = 0, 0, 0, []
+    t0.record()
+    for i in range(steps):
+        nb, nl = run.step(i, kev[i])
+        total_bytes += nb
+        launches += nl
+        lens_sum += int(eng.lens.sum())
+        kbytes.append(nb)
+    t1.record()
+    torch.cuda.synchronize(device)
+    clk = sampler.stop() if sampler else None
+    ms = t0.elapsed_time(t1)
+    kernel_ms = [a.elapsed_time(b) for a, b in kev]
+    ms_max = reduce_max(ms, dist, device)
+    res = {"ms_total": ms_max, "bytes": total_bytes, "launches": launches, "seq_tokens": lens_sum,
+           "kernel_ms_mean": float(np.mean(kernel_ms)), "kernel_bytes_mean": float(np.mean(kbytes)),
+           "clocks": clk, "num_cow": eng.last_num_cow}
+    if e2e:
+        S, Hq, Hkv, D = w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim
+        q0, k0, v0 = run.inputs[0]
+        host = (q0.cpu().pin_memory(), k0.cpu().pin_memory(), v0.cpu().pin_memory(),
+                torch.empty_like(run.out, device="cpu").pin_memory(),
+                torch.empty_like(q0), torch.empty_like(k0), torch.empty_like(v0))
+        for i in range(warmup):
+            run.step(i, host=host)
+        torch.cuda.synchronize(device)
+        barrier(dist, device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        eb = 0
+        e0.record()
+        for i in range(n_e2e):
+            nb, _ = run.step(i, host=host)
+            eb += nb
+        e1.record()
+        torch.cuda.synchronize(device)
+        ems = reduce_max(e0.elapsed_time(e1), dist, device)
+        h2d = sum(t.numel() * t.element_size() for t in host[:3]) + eng._meta_bytes
+        d2h = host[3].numel() * host[3].element_size()
+        res["e2e"] = {"ms_total": ems, "bytes": eb, "h2d": h2d, "d2h": d2h, "steps": n_e2e}
+    del eng, run
+    torch.cuda.empty_cache()
+    return res
+
+
+# ---------------------------------------------------------------------------
+# the oracle on the host cores (cpu_baseline and --impl reference)
+# ---------------------------------------------------------------------------
+
+def oracle_sample_inputs(w, budget_s):
+    """A bounded sample of the workload for the float64 oracle: whole sequences
+    (all heads) in a seeded order, as many as fit in about `budget_s` of CPU time
+    at a first estimate; their blocks are drawn fresh on the host, laid out 0..n-1."""
+    import synthetic
+    rng = np.random.default_rng(w.seed + 7)
+    order = rng.permutation(w.num_seqs)
+    q = synthetic.normal_codes((w.num_seqs, w.num_q_heads, w.head_dim), w.q_dtype, w.seed + 9).numpy()
+    q = q.view(np.uint16)
+    # first estimate: ~0.7 us of oracle time per (token, kv head) on one core
+    est, chosen = 0.0, []
+    for s in order:
+        chosen.append(int(s))
+        est += 0.7e-6 * w.context_lens[s] * w.num_q_heads
+        if est >= budget_s:
+            break
+    items = []
+    for s in chosen:
+        L = w.context_lens[s]
+        nbk = -(-L // w.block_size)
+        shape = (nbk, w.num_kv_heads, w.block_size, w.head_dim)
+        if w.kv_dtype == "e4m3":
+            kc = rng.integers(0, 0x7E, size=shape, dtype=np.uint8)
+            vc = rng.integers(0, 0x7E, size=shape, dtype=np.uint8)
+            ks = vs = 6.0 / 448
+        else:
+            kc = synthetic.normal_codes(shape, w.kv_dtype, s + 1).numpy().view(np.uint16)
+            vc = synthetic.normal_codes(shape, w.kv_dtype, s + 2).numpy().view(np.uint16)
+            ks = vs = 1.0
+        items.append((s, L, kc, vc, ks, vs, np.arange(nbk, dtype=np.int64)[None, :]))
+    return q, items
+
+
+def oracle_run(w, q, items):
+    """One pass of the oracle over the sample; returns (bytes, tokens, cpu seconds)."""
+    from threadpoolctl import threadpool_limits
+    from oracle import attention as oatt
+    kvb = 1 if w.kv_dtype == "e4m3" else 2
+    nbytes, ntok = 0, 0
+    with threadpool_limits(limits=1):
+        t0 = time.process_time()
+        for s, L, kc, vc, ks, vs, bt in items:
+            oatt.paged_decode(q[s:s + 1], w.q_dtype, kc, vc, w.kv_dtype, ks, vs, bt, [L], w.scale)
+            nbytes += decode_bytes([L], w.num_kv_heads, w.num_q_heads, w.head_dim, kvb, 2, w.block_size)
+            ntok += L
+        dt = time.process_time() - t0
+    return nbytes, ntok, dt
+
+
+def sample_text(w, items, seconds, passes=1):
+    lens = [it[1] for it in items]
+    return (f"float64 numpy oracle on 1 thread (BLAS limited to 1): {len(items)} whole sequences of the "
+            f"{w.name} workload (context lengths {min(lens)}..{max(lens)}, all {w.num_q_heads} q heads), "
+            f"{passes} pass(es), {seconds:.1f} s of CPU time")
+
+
+def cpu_baseline_obj(w, budget_s):
+    q, items = oracle_sample_inputs(w, budget_s)
+    nb, nt, dt = oracle_run(w, q, items)
+    return {"value": nb / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "seq_tokens_per_s": nt / dt, "sample": sample_text(w, items, dt)}
+
+
+def reference_arm(w, args):
+    """--impl reference: the oracle, each step one pass over a bounded sample."""
+    per_step = max(0.2, min(2.0, 120.0 / (args.steps + args.warmup)))
+    q, items = oracle_sample_inputs(w, per_step)
+    for _ in range(args.warmup):
+        oracle_run(w, q, items)
+    tb, tt, ts = 0, 0, 0.0
+    for _ in range(args.steps):
+        nb, nt, dt = oracle_run(w, q, items)
+        tb, tt, ts = tb + nb, tt + nt, ts + dt
+    gbs = tb / ts / 1e9
+    return {"metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ts / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": workload_config(w, 1), "seq_tokens_per_s": tt / ts,
+            "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": sample_text(w, items, ts, args.steps) +
+                             "; ms_per_step is the time of one pass over this sample"},
+            "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# ---------------------------------------------------------------------------
+
+def workload_config(w, n_gpus):
+    return {"workload": w.name, "num_seqs": w.num_seqs, "num_q_heads": w.num_q_heads,
+            "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim, "block_size": w.block_size,
+            "kv_dtype": w.kv_dtype, "q_dtype": w.q_dtype, "sum_context_tokens": int(sum(w.context_lens)),
+            "max_context_len": int(max(w.context_lens)), "partition_tokens": 512,
+            "l2": "no flush: KV read per step far above the 126 MB L2",
+            "parallelism": f"replicas{n_gpus}" if n_gpus > 1 else "single GPU"}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="llama13b_mix")
+    ap.add_argument("--also", default="long_fp8", help="second workload reported in the same line ('' = none)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    args = ap.parse_args(argv)
+    args.warmup = max(args.warmup, 3)
+
+    import synthetic
+    world, rank, local = dist_env()
+    w = synthetic.make(args.workload)
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(reference_arm(w, args)))
+        return 0
+
+    import torch
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the product path has no CPU fallback)")
+    import paged_kv_cache_436_b200 as pa
+    pa.lib()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    dist = init_dist(world, "nccl")
+    try:
+        res = time_ours(w, args.steps, args.warmup, device, dist, e2e=not args.no_e2e,
+                        clocks=True, local_rank=local)
+        also = None
+        if args.also:
+            wa = synthetic.make(args.also)
+            also = time_ours(wa, args.steps, args.warmup, device, dist, e2e=False, clocks=False,
+                             local_rank=local)
+        peak, peak_src = peaks()
+        all_bytes = reduce_sum(res["bytes"], dist, device)
+        value = all_bytes / (res["ms_total"] / 1e3) / 1e9
+        tokens = reduce_sum(res["seq_tokens"], dist, device) / (res["ms_total"] / 1e3)
+        kern_gbs = res["kernel_bytes_mean"] / (res["kernel_ms_mean"] / 1e3) / 1e9
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": res["ms_total"] / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": w.kv_dtype, "data": "synthetic",
+            "config": workload_config(w, world),
+            "seq_tokens_per_s": tokens,
+            "pct_of_hbm": {"measured_copy": value / world / peak, "nominal_8tbs": value / world / NOMINAL_HBM_GBS},
+            "roofline": {"bound": "hbm", "kernel": "partition_kernel (pa_decode stage 1)",
+                         "achieved": kern_gbs, "peak": peak, "unit": "GB/s", "frac": kern_gbs / peak,
+                         "peak_source": peak_src + " HBM copy bandwidth (MEASURED_PEAKS hbm_gbs)",
+                         "frac_of_nominal_8tbs": kern_gbs / NOMINAL_HBM_GBS,
+                         "bytes_per_launch": res["kernel_bytes_mean"], "ms_per_launch": res["kernel_ms_mean"],
+                         "traffic": None},
+            "gpu_launches": res["launches"],
+            "clocks": res["clocks"],
+        }
+        if "e2e" in res:
+            e = res["e2e"]
+            line["e2e"] = {"value": reduce_sum(e["bytes"], dist, device) / (e["ms_total"] / 1e3) / 1e9,
+                           "unit": "GB/s", "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"],
+                           "ms_per_step": e["ms_total"] / e["steps"]}
+        if also is not None:
+            line["also"] = {"workload": args.also,
+                            "value": reduce_sum(also["bytes"], dist, device) / (also["ms_total"] / 1e3) / 1e9,
+                            "unit": "GB/s", "ms_per_step": also["ms_total"] / args.steps,
+                            "seq_tokens_per_s": reduce_sum(also["seq_tokens"], dist, device) / (also["ms_total"] / 1e3),
+                            "roofline": {"bound": "hbm",
+                                         "achieved": also["kernel_bytes_mean"] / (also["kernel_ms_mean"] / 1e3) / 1e9,
+                                         "peak": peak, "unit": "GB/s",
+                                         "frac": also["kernel_bytes_mean"] / (also["kernel_ms_mean"] / 1e3) / 1e9 / peak,
+                                         "ms_per_launch": also["kernel_ms_mean"]}}
+        if rank == 0 and world == 1:
+            line["cpu_baseline"] = cpu_baseline_obj(w, args.cpu_budget)
+        if rank == 0:
+            print(json.dumps(line))
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,287 @@
+/*
+ * pa.h -- C ABI of libpa: paged KV-cache decode attention for NVIDIA B200 (sm_100a).
+ *
+ * The method (PagedAttention as three web pages describe it):
+ *   page 1 "突破GPU内存瓶颈：vLLM与PagedAttention技术深度解析", section
+ *          "2. PagedAttention的革命性设计" -- fixed-size blocks, a per-sequence block
+ *          table mapping logical to physical blocks, blocks shared between sequences;
+ *   page 2 (untitled; first section "1. 为什么vLLM能实现24倍推理加速"), section
+ *          "1.1 PagedAttention的内存管理革命" -- the op
+ *          paged_attention(queries, key_cache, value_cache, block_tables); section
+ *          "2.2 关键数据结构剖析" -- the metadata (block_tables, context_lens,
+ *          num_heads, head_size); section "3.3 常见问题排查" -- the v2 kernel for long
+ *          text; section "4.2 混合精度策略" -- an FP8 KV cache;
+ *   page 3 "内存优化：KV Cache管理、PagedAttention原理与内存池配置", section
+ *          "PagedAttention原理" -- blocks of 16 or 32 tokens, refcounted sharing, a free
+ *          list with O(1) alloc/free and no device allocation per request.
+ *
+ * Conventions for every call below.
+ *   - Device pointers are plain CUDA device addresses owned by the caller; the
+ *     library never allocates, frees or retains device memory. Host pointers are
+ *     plain host memory owned by the caller.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *     stream). GPU calls only enqueue work and return; results are ready when the
+ *     stream reaches them.
+ *   - Argument checks that need no device data (null pointers, shapes, dtype
+ *     combinations, 16-byte alignment, supported head_dim / block_size / group
+ *     size) run on the host before anything is enqueued and return PA_ERR_ARG;
+ *     nothing is launched then.
+ *   - Checks of device data (block ids in [0, num_blocks), context lengths within
+ *     the block table and the declared maximum, slots and copy pairs in range)
+ *     run inside the kernels. A violation never touches memory out of range: the
+ *     offending item is skipped (or its length clamped), and a sticky device error
+ *     word records the first violation; read it with pa_last_device_error().
+ *   - A CUDA launch error returns PA_ERR_CUDA.
+ *
+ * Cache layout (both K and V): [num_blocks][num_kv_heads][block_size][head_dim],
+ * row-major, contiguous. Token position j of a sequence s lives at
+ *   cache[block_tables[s][j / block_size]][h][j % block_size][:].
+ */
+#ifndef PA_H
+#define PA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_ARG = -1,          /* invalid argument (host-side check); nothing enqueued */
+  PA_ERR_OOM = -2,          /* block pool has no free block */
+  PA_ERR_STATE = -3,        /* refcount of a free block taken or dropped */
+  PA_ERR_CUDA = -4,         /* a CUDA runtime call failed */
+  PA_ERR_DEVICE_CHECK = -5  /* a kernel found invalid device data (see pa_last_device_error) */
+} pa_status;
+
+typedef enum { PA_F16 = 0, PA_BF16 = 1, PA_E4M3 = 2 } pa_dtype;
+
+/* Device error codes recorded by the kernels (first one wins until read). */
+enum {
+  PA_DEV_OK = 0,
+  PA_DEV_BAD_BLOCK_ID = 1,     /* info: seq, logical block, value */
+  PA_DEV_BAD_CONTEXT_LEN = 2,  /* info: seq, value, limit */
+  PA_DEV_BAD_SLOT = 3,         /* info: token, value, limit */
+  PA_DEV_BAD_COPY_PAIR = 4,    /* info: pair, src, dst */
+  PA_DEV_BAD_TABLE_UPDATE = 5, /* info: update, seq, col */
+  PA_DEV_WAIT_TIMEOUT = 6      /* info: kernel id, unit, stage */
+};
+
+/*
+ * One KV cache (K and V of one attention layer).
+ *   num_blocks    physical blocks in the pool
+ *   num_kv_heads  kv heads (Hkv)
+ *   block_size    tokens per block: 8, 16 or 32 (page 3, section "内存池配置": 8..32;
+ *                 16 the default, 32 for sequences beyond 4K tokens)
+ *   head_dim      64 or 128
+ *   kv_dtype      PA_F16, PA_BF16 or PA_E4M3 (OCP E4M3, saturating, one scale per tensor)
+ *   k_scale, v_scale  per-tensor dequantisation scales: stored code c means c * scale.
+ *                 Must be 1.0 for 16-bit caches.
+ *   k_cache, v_cache  device pointers, 16-byte aligned.
+ */
+typedef struct {
+  int32_t num_blocks;
+  int32_t num_kv_heads;
+  int32_t block_size;
+  int32_t head_dim;
+  int32_t kv_dtype;
+  float k_scale;
+  float v_scale;
+  void* k_cache;
+  void* v_cache;
+} pa_cache_desc;
+
+/* ------------------------------------------------------------------------- */
+/* KV-cache write                                                             */
+/* ------------------------------------------------------------------------- */
+/*
+ * pa_reshape_and_cache -- write each new token's K and V rows into its slot.
+ * The slot of logical position j of a sequence is block_table[j / BS] * BS + j % BS
+ * (page 1, section "2. PagedAttention的革命性设计", the block table).
+ *   k, v          device [num_tokens][num_kv_heads][head_dim] of in_dtype; consecutive
+ *                 tokens are k_token_stride (v_token_stride) elements apart, heads and
+ *                 dims contiguous inside a token; 16-byte aligned rows.
+ *   in_dtype      PA_F16 or PA_BF16. For 16-bit caches it must equal kv_dtype and the
+ *                 codes are copied bit for bit. For an E4M3 cache each value x is stored
+ *                 as e4m3_rne_satfinite(x / scale), the division in binary32.
+ *   slot_mapping  device int64 [num_tokens]; a negative slot skips the token; a slot
+ *                 >= num_blocks * block_size is skipped and recorded (PA_DEV_BAD_SLOT).
+ * Two tokens with the same slot race; callers give distinct slots.
+ */
+pa_status pa_reshape_and_cache(const void* k, const void* v, int32_t in_dtype, int32_t num_tokens,
+                               int64_t k_token_stride, int64_t v_token_stride,
+                               const int64_t* slot_mapping, const pa_cache_desc* cache,
+                               void* stream);
+
+/* ------------------------------------------------------------------------- */
+/* Block copy (copy-on-write)                                                 */
+/* ------------------------------------------------------------------------- */
+/*
+ * pa_copy_blocks -- for each pair (src, dst): block dst of K and of V becomes a bit
+ * copy of block src (all kv heads, all slots). This is the copy that copy-on-write
+ * needs when a sequence appends into a block it shares (page 3, section
+ * "PagedAttention原理": blocks shared between requests through reference counts;
+ * page 1, section "5. 高级应用场景": parallel sampling and beam search).
+ *   src_dst_pairs device int64 [num_pairs][2].
+ * Pairs are copied concurrently: no block may be the destination of one pair and
+ * the source or destination of another. Out-of-range ids skip the pair and are
+ * recorded (PA_DEV_BAD_COPY_PAIR). num_pairs == 0 enqueues nothing.
+ */
+pa_status pa_copy_blocks(const int64_t* src_dst_pairs, int32_t num_pairs,
+                         const pa_cache_desc* cache, void* stream);
+
+/* ------------------------------------------------------------------------- */
+/* Decode attention                                                           */
+/* ------------------------------------------------------------------------- */
+/*
+ * pa_decode -- one query token per sequence attends over its whole paged context:
+ *   out[s,h,:] = sum_j softmax_j(scale * <q[s,h,:], K_s[j]>) * V_s[j],  j < context_lens[s]
+ * with K_s[j] = k_scale * cache_k[block_tables[s][j / BS]][h / G][j % BS][:] (V likewise),
+ * G = num_q_heads / num_kv_heads (query head h reads kv head h / G).
+ * Page 2, section "1.1 PagedAttention的内存管理革命" (the paged op beside
+ * matmul(q, k^T)/sqrt(d)); page 3, section "核心原理" (one query against all cached keys).
+ * Long contexts are split into partitions of 512 tokens whose partial results
+ * (running max, sum of exponentials, unnormalised output) are merged by a second,
+ * log-sum-exp kernel (page 2, section "3.3 常见问题排查": the v2 kernel for long text).
+ * All softmax and accumulation arithmetic is binary32.
+ *   q              device [num_seqs][num_q_heads][head_dim] of q_dtype (PA_F16 / PA_BF16);
+ *                  for 16-bit caches q_dtype must equal kv_dtype.
+ *   block_tables   device int32 [num_seqs][max_blocks_per_seq].
+ *   context_lens   device int32 [num_seqs]; 0 gives an all-zero output row.
+ *   max_context_len host upper bound of context_lens (sizes the partition grid).
+ *   scale          softmax scale (e.g. 1/sqrt(head_dim)).
+ *   out            device [num_seqs][num_q_heads][head_dim] of q_dtype, rounded to
+ *                  nearest even from binary32.
+ *   workspace      device scratch of at least pa_decode_workspace_size() bytes,
+ *                  256-byte aligned; owned by the caller; contents need not be
+ *                  initialised and are undefined afterwards. Two pa_decode calls that
+ *                  run at the same time need separate workspaces.
+ * Supported: head_dim 64 or 128; block_size 8, 16, 32; G in {1, 2, 4, 8}.
+ */
+pa_status pa_decode(const void* q, int32_t q_dtype, int32_t num_seqs, int32_t num_q_heads,
+                    const pa_cache_desc* cache, const int32_t* block_tables,
+                    int32_t max_blocks_per_seq, const int32_t* context_lens,
+                    int32_t max_context_len, float scale, void* out, void* workspace,
+                    size_t workspace_bytes, void* stream);
+
+/* Bytes of workspace pa_decode needs for these sizes (0 on invalid sizes). */
+size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,
+                                int32_t max_context_len);
+
+/*
+ * pa_decode_stage -- run one of pa_decode's three launches alone, with the same
+ * arguments: stage 0 plans the partitions (and zeroes rows of empty sequences),
+ * stage 1 runs the partition kernel, stage 2 merges partitions. Running 0, 1, 2 in
+ * order on one stream is exactly pa_decode. For timing one kernel in isolation.
+ */
+pa_status pa_decode_stage(int32_t stage, const void* q, int32_t q_dtype, int32_t num_seqs,
+                          int32_t num_q_heads, const pa_cache_desc* cache,
+                          const int32_t* block_tables, int32_t max_blocks_per_seq,
+                          const int32_t* context_lens, int32_t max_context_len, float scale,
+                          void* out, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * pa_last_device_error -- synchronise `stream`, then read and clear the device error
+ * word of the current device. *code receives a PA_DEV_* value; info (may be NULL)
+ * receives 3 int32 details. Returns PA_ERR_DEVICE_CHECK when *code != 0.
+ */
+pa_status pa_last_device_error(void* stream, int32_t* code, int32_t* info);
+
+/* ------------------------------------------------------------------------- */
+/* Device mirror of the block tables                                          */
+/* ------------------------------------------------------------------------- */
+/*
+ * pa_block_table_update -- apply table entries produced by the host bookkeeping
+ * (pa_batch_append's updates) to the device copy of the block tables:
+ *   block_tables[u.seq * max_blocks_per_seq + u.col] = u.block for every update u.
+ *   updates  device int32 [num_updates][3] = (seq, col, block).
+ * Out-of-range (seq, col) skips the update and is recorded (PA_DEV_BAD_TABLE_UPDATE).
+ */
+pa_status pa_block_table_update(const int32_t* updates, int32_t num_updates, int32_t* block_tables,
+                                int32_t num_seqs, int32_t max_blocks_per_seq, void* stream);
+
+/* ------------------------------------------------------------------------- */
+/* Host block pool: O(1) free list + reference counts                         */
+/* ------------------------------------------------------------------------- */
+/*
+ * Page 3, section "PagedAttention原理": free blocks form a linked list, alloc and free
+ * are O(1), blocks are shared through reference counts; a sequence takes a block
+ * only when it grows into one and returns all of them when it finishes; waste is
+ * confined to a sequence's last block (page 1, section "2. PagedAttention的革命性设计").
+ * The free list is a LIFO stack threaded through an array; initial_order seeds it
+ * so that successive allocations return initial_order[0], [1], ...; a block whose
+ * count reaches zero is pushed on top. Not thread-safe: one pool per engine thread.
+ */
+typedef struct pa_pool pa_pool;
+
+/* initial_order: host int32 permutation of 0..num_blocks-1, or NULL for 0..N-1. */
+pa_status pa_pool_create(int32_t num_blocks, const int32_t* initial_order, pa_pool** out);
+void pa_pool_destroy(pa_pool* pool);
+pa_status pa_pool_alloc(pa_pool* pool, int32_t* block);      /* refcount := 1; PA_ERR_OOM if empty */
+pa_status pa_pool_incref(pa_pool* pool, int32_t block);      /* PA_ERR_STATE if block is free */
+pa_status pa_pool_decref(pa_pool* pool, int32_t block);      /* at 0 the block is freed;
+                                                                PA_ERR_STATE if already free */
+int32_t pa_pool_refcount(const pa_pool* pool, int32_t block); /* -1 if out of range */
+int32_t pa_pool_num_free(const pa_pool* pool);
+int32_t pa_pool_num_blocks(const pa_pool* pool);
+/* The free list in allocation order (first = next to be handed out); writes
+ * min(capacity, num_free) ids and returns how many it wrote. */
+int32_t pa_pool_free_list(const pa_pool* pool, int32_t* blocks, int32_t capacity);
+
+/*
+ * pa_seq_append -- host bookkeeping for appending logical position `pos` to one
+ * sequence. block_table_row (host, max_blocks entries) holds ceil(pos / BS) valid
+ * entries before the call. If pos % BS == 0 a new block is allocated into entry
+ * pos / BS. Otherwise, if the last block is shared (refcount > 1), a fresh block is
+ * allocated, (old, new) is reported through *cow_src / *cow_dst for pa_copy_blocks,
+ * the old block loses one reference and the entry is replaced (copy-on-write).
+ * *slot = row[pos / BS] * BS + pos % BS. *cow_src = *cow_dst = -1 when no copy.
+ * On PA_ERR_OOM nothing has changed.
+ */
+pa_status pa_seq_append(pa_pool* pool, int32_t* block_table_row, int32_t max_blocks, int32_t pos,
+                        int32_t block_size, int64_t* slot, int32_t* cow_src, int32_t* cow_dst);
+
+/*
+ * pa_seq_extend -- append positions start_pos .. start_pos + n_tokens - 1 (a prompt).
+ * slots (host int64 [n_tokens]) may be NULL. At most the first position can need a
+ * copy; it is reported through *cow_src / *cow_dst (-1 when none). On PA_ERR_OOM the
+ * positions before the failing one have been appended; *n_done (may be NULL) says
+ * how many.
+ */
+pa_status pa_seq_extend(pa_pool* pool, int32_t* block_table_row, int32_t max_blocks,
+                        int32_t start_pos, int32_t n_tokens, int32_t block_size, int64_t* slots,
+                        int32_t* cow_src, int32_t* cow_dst, int32_t* n_done);
+
+/* pa_seq_fork -- a sequence sharing the first n_blocks blocks of row: each gets one
+ * more reference; the caller copies the row. */
+pa_status pa_seq_fork(pa_pool* pool, const int32_t* block_table_row, int32_t n_blocks);
+
+/* pa_seq_free -- a finished sequence drops one reference of each of its n_blocks blocks. */
+pa_status pa_seq_free(pa_pool* pool, const int32_t* block_table_row, int32_t n_blocks);
+
+/*
+ * pa_batch_append -- one decode step's bookkeeping for a batch: pa_seq_append for
+ * sequences 0..num_seqs-1 in order, at positions[s].
+ *   block_tables  host int32 [num_seqs][max_blocks] (updated in place)
+ *   slots         host int64 [num_seqs] out
+ *   cow_pairs     host int64 [num_seqs][2] out; *num_cow pairs written
+ *   updates       host int32 [num_seqs][3] out; (seq, col, block) for every table
+ *                 entry written, *num_updates of them (for pa_block_table_update)
+ *   n_done        sequences fully processed (== num_seqs on success)
+ * On an error the sequences before *n_done have been appended and reported.
+ */
+pa_status pa_batch_append(pa_pool* pool, int32_t* block_tables, int32_t num_seqs, int32_t max_blocks,
+                          const int32_t* positions, int32_t block_size, int64_t* slots,
+                          int64_t* cow_pairs, int32_t* num_cow, int32_t* updates,
+                          int32_t* num_updates, int32_t* n_done);
+
+/* Library version string and the device architecture it was built for. */
+const char* pa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H */

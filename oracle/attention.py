@@ -35,20 +35,20 @@ import numpy as np
 from . import codecs
 
 
-def gather_sequence(cache_f64: np.ndarray, block_table_row, context_len: int,
+def gather_sequence(cache: np.ndarray, block_table_row, context_len: int,
                     kv_head: int) -> np.ndarray:
     """Rows 0..L-1 of one sequence for one kv head, in logical order.
 
-    ``cache_f64`` is a decoded cache of shape [NB, Hkv, BS, D]. Token j lives in
-    physical block ``block_table_row[j // BS]`` at offset ``j % BS``.
+    ``cache`` is a cache of shape [NB, Hkv, BS, D] (decoded values or raw codes).
+    Token j lives in physical block ``block_table_row[j // BS]`` at offset ``j % BS``.
     """
-    bs = cache_f64.shape[2]
+    bs = cache.shape[2]
     rows = []
     for j in range(context_len):
         phys = int(block_table_row[j // bs])
-        rows.append(cache_f64[phys, kv_head, j % bs, :])
+        rows.append(cache[phys, kv_head, j % bs, :])
     if not rows:
-        return np.zeros((0, cache_f64.shape[3]), dtype=np.float64)
+        return np.zeros((0, cache.shape[3]), dtype=cache.dtype)
     return np.stack(rows)
 
 
@@ -91,25 +91,26 @@ def paged_decode(q_codes: np.ndarray, q_dtype: str, k_codes: np.ndarray, v_codes
                  context_lens, scale: float, heads=None) -> np.ndarray:
     """Decode attention from raw element codes (what the device buffers hold).
 
-    Decodes with the oracle's own bit-level codecs, multiplies K by ``k_scale``
-    and V by ``v_scale`` (per-tensor scales; 1.0 for 16-bit caches) and calls
-    :func:`paged_decode_f64`. Only the blocks the sequences reference are decoded.
+    For each (s, h): gathers the sequence's K and V codes of kv head h // G through
+    its block table, decodes them with the oracle's own bit-level codecs,
+    multiplies by the per-tensor scales (1.0 for 16-bit caches) and evaluates
+    :func:`softmax_weighted_sum`. Decoding is elementwise, so gathering first
+    gives the same values as decoding the whole cache first.
     """
     q = codecs.decode(q_codes, q_dtype)
-    used = sorted({int(b) for s in range(block_tables.shape[0])
-                   for b in block_tables[s, :_nblocks(int(context_lens[s]), k_codes.shape[2])]})
-    remap = {b: i for i, b in enumerate(used)}
-    bt = np.zeros_like(block_tables)
-    for s in range(block_tables.shape[0]):
-        n = _nblocks(int(context_lens[s]), k_codes.shape[2])
-        for j in range(n):
-            bt[s, j] = remap[int(block_tables[s, j])]
-    idx = np.array(used, dtype=np.int64)
-    k = codecs.decode(k_codes[idx], kv_dtype) * float(k_scale) if len(idx) else \
-        np.zeros((0,) + k_codes.shape[1:])
-    v = codecs.decode(v_codes[idx], kv_dtype) * float(v_scale) if len(idx) else \
-        np.zeros((0,) + v_codes.shape[1:])
-    return paged_decode_f64(q, k, v, bt, context_lens, scale, heads=heads)
+    S, Hq, D = q.shape
+    Hkv = k_codes.shape[1]
+    assert Hq % Hkv == 0
+    G = Hq // Hkv
+    out = np.zeros((S, Hq, D), dtype=np.float64)
+    pairs = heads if heads is not None else [(s, h) for s in range(S) for h in range(Hq)]
+    for s, h in pairs:
+        g = h // G
+        L = int(context_lens[s])
+        K = codecs.decode(gather_sequence(k_codes, block_tables[s], L, g), kv_dtype) * float(k_scale)
+        V = codecs.decode(gather_sequence(v_codes, block_tables[s], L, g), kv_dtype) * float(v_scale)
+        out[s, h] = softmax_weighted_sum(q[s, h], K, V, scale)
+    return out
 
 
 def _nblocks(context_len: int, block_size: int) -> int:

@@ -1,0 +1,306 @@
+"""Python binding of libpa: paged KV-cache decode attention for B200 (sm_100a).
+
+Argument marshalling only. Every step of the path -- the block bookkeeping, the
+KV-cache write, the block copy and the decode attention -- runs inside libpa (C++
+on the host, CUDA kernels on the device). PyTorch provides device memory and
+streams; this module passes ``tensor.data_ptr()`` and the current stream.
+
+There is no fallback: if ``lib/libpa.so`` is missing or cannot be loaded every
+call raises :class:`LibraryMissing`.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "lib", "libpa.so")
+
+PA_OK, PA_ERR_ARG, PA_ERR_OOM, PA_ERR_STATE, PA_ERR_CUDA, PA_ERR_DEVICE_CHECK = 0, -1, -2, -3, -4, -5
+PA_F16, PA_BF16, PA_E4M3 = 0, 1, 2
+DTYPES = {"f16": PA_F16, "bf16": PA_BF16, "e4m3": PA_E4M3}
+DEVICE_ERRORS = {0: "ok", 1: "bad block id", 2: "bad context length", 3: "bad slot",
+                 4: "bad copy pair", 5: "bad table update", 6: "wait timeout"}
+STATUS = {PA_OK: "ok", PA_ERR_ARG: "invalid argument", PA_ERR_OOM: "out of blocks",
+          PA_ERR_STATE: "refcount state", PA_ERR_CUDA: "CUDA error", PA_ERR_DEVICE_CHECK: "device check"}
+
+
+class LibraryMissing(RuntimeError):
+    pass
+
+
+class PaError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {STATUS.get(status, status)} ({status})")
+        self.status = status
+
+
+class CacheDesc(ctypes.Structure):
+    _fields_ = [("num_blocks", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
+                ("block_size", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("kv_dtype", ctypes.c_int32), ("k_scale", ctypes.c_float),
+                ("v_scale", ctypes.c_float), ("k_cache", ctypes.c_void_p),
+                ("v_cache", ctypes.c_void_p)]
+
+
+_lib = None
+
+_P = ctypes.c_void_p
+_I32 = ctypes.c_int32
+_I64 = ctypes.c_int64
+_PI32 = ctypes.POINTER(ctypes.c_int32)
+_PI64 = ctypes.POINTER(ctypes.c_int64)
+_PDESC = ctypes.POINTER(CacheDesc)
+
+_SIGNATURES = {
+    "pa_reshape_and_cache": (_I32, [_P, _P, _I32, _I32, _I64, _I64, _P, _PDESC, _P]),
+    "pa_copy_blocks": (_I32, [_P, _I32, _PDESC, _P]),
+    "pa_decode": (_I32, [_P, _I32, _I32, _I32, _PDESC, _P, _I32, _P, _I32, ctypes.c_float, _P, _P,
+                         ctypes.c_size_t, _P]),
+    "pa_decode_stage": (_I32, [_I32, _P, _I32, _I32, _I32, _PDESC, _P, _I32, _P, _I32, ctypes.c_float,
+                               _P, _P, ctypes.c_size_t, _P]),
+    "pa_decode_workspace_size": (ctypes.c_size_t, [_I32, _I32, _I32, _I32]),
+    "pa_last_device_error": (_I32, [_P, _PI32, _PI32]),
+    "pa_block_table_update": (_I32, [_P, _I32, _P, _I32, _I32, _P]),
+    "pa_pool_create": (_I32, [_I32, _PI32, ctypes.POINTER(_P)]),
+    "pa_pool_destroy": (None, [_P]),
+    "pa_pool_alloc": (_I32, [_P, _PI32]),
+    "pa_pool_incref": (_I32, [_P, _I32]),
+    "pa_pool_decref": (_I32, [_P, _I32]),
+    "pa_pool_refcount": (_I32, [_P, _I32]),
+    "pa_pool_num_free": (_I32, [_P]),
+    "pa_pool_num_blocks": (_I32, [_P]),
+    "pa_pool_free_list": (_I32, [_P, _PI32, _I32]),
+    "pa_seq_append": (_I32, [_P, _PI32, _I32, _I32, _I32, _PI64, _PI32, _PI32]),
+    "pa_seq_extend": (_I32, [_P, _PI32, _I32, _I32, _I32, _I32, _PI64, _PI32, _PI32, _PI32]),
+    "pa_seq_fork": (_I32, [_P, _PI32, _I32]),
+    "pa_seq_free": (_I32, [_P, _PI32, _I32]),
+    "pa_batch_append": (_I32, [_P, _PI32, _I32, _I32, _PI32, _I32, _PI64, _PI64, _PI32, _PI32, _PI32,
+                               _PI32]),
+    "pa_version": (ctypes.c_char_p, []),
+}
+
+
+def lib():
+    """The loaded libpa (raises LibraryMissing when it is not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise LibraryMissing(f"{LIB_PATH} not built: run `python -m paged_kv_cache_436_b200.build`")
+        try:
+            L = ctypes.CDLL(LIB_PATH)
+        except OSError as e:
+            raise LibraryMissing(f"cannot load {LIB_PATH}: {e}") from e
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(status: int, what: str) -> None:
+    if status != PA_OK:
+        raise PaError(status, what)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _stream(stream=None):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _i32p(a):
+    """Pointer into a contiguous host int32 buffer (numpy array or CPU tensor)."""
+    if hasattr(a, "ctypes"):
+        return a.ctypes.data_as(_PI32)
+    return ctypes.cast(a.data_ptr(), _PI32)
+
+
+def _i64p(a):
+    if hasattr(a, "ctypes"):
+        return a.ctypes.data_as(_PI64)
+    return ctypes.cast(a.data_ptr(), _PI64)
+
+
+# ---------------------------------------------------------------------------
+# device ops
+# ---------------------------------------------------------------------------
+
+def dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.float16:
+        return PA_F16
+    if t.dtype == torch.bfloat16:
+        return PA_BF16
+    if t.dtype in (torch.uint8, torch.float8_e4m3fn):
+        return PA_E4M3
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+class KVCache:
+    """K and V caches [num_blocks, num_kv_heads, block_size, head_dim] plus their scales."""
+
+    def __init__(self, k_cache, v_cache, kv_dtype: str, k_scale: float = 1.0, v_scale: float = 1.0):
+        assert k_cache.shape == v_cache.shape and k_cache.dim() == 4
+        assert k_cache.is_contiguous() and v_cache.is_contiguous()
+        self.k_cache, self.v_cache = k_cache, v_cache
+        self.kv_dtype = kv_dtype
+        nb, hkv, bs, d = k_cache.shape
+        self.desc = CacheDesc(nb, hkv, bs, d, DTYPES[kv_dtype], float(k_scale), float(v_scale),
+                              k_cache.data_ptr(), v_cache.data_ptr())
+
+    @property
+    def num_blocks(self):
+        return self.desc.num_blocks
+
+    @property
+    def block_size(self):
+        return self.desc.block_size
+
+
+def reshape_and_cache(k, v, slot_mapping, cache: KVCache, stream=None) -> None:
+    """Write each token's K/V rows ([T, Hkv, D], fp16/bf16) into its slot (int64 [T])."""
+    T = k.shape[0]
+    st = lib().pa_reshape_and_cache(_ptr(k), _ptr(v), dtype_code(k), T, k.stride(0), v.stride(0),
+                                    _ptr(slot_mapping), ctypes.byref(cache.desc), _stream(stream))
+    _check(st, "pa_reshape_and_cache")
+
+
+def copy_blocks(pairs, cache: KVCache, stream=None) -> None:
+    """Copy whole blocks src -> dst for each row of the device int64 [n, 2] ``pairs``."""
+    n = 0 if pairs is None else pairs.shape[0]
+    st = lib().pa_copy_blocks(_ptr(pairs), n, ctypes.byref(cache.desc), _stream(stream))
+    _check(st, "pa_copy_blocks")
+
+
+def decode_workspace_size(num_seqs, num_q_heads, head_dim, max_context_len) -> int:
+    return int(lib().pa_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_context_len))
+
+
+def decode(q, cache: KVCache, block_tables, context_lens, max_context_len: int, scale: float, out,
+           workspace, stream=None, stage=None) -> None:
+    """Paged decode attention: out[s, h] = softmax(scale q K^T) V over each context.
+
+    q, out: [S, Hq, D] fp16/bf16; block_tables int32 [S, MB]; context_lens int32 [S];
+    workspace: uint8 device buffer of at least decode_workspace_size(...) bytes.
+    ``stage`` (0, 1 or 2) runs one of the three launches alone.
+    """
+    S, Hq, _ = q.shape
+    args = (_ptr(q), dtype_code(q), S, Hq, ctypes.byref(cache.desc), _ptr(block_tables),
+            block_tables.shape[1], _ptr(context_lens), int(max_context_len), float(scale), _ptr(out),
+            _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    if stage is None:
+        _check(lib().pa_decode(*args), "pa_decode")
+    else:
+        _check(lib().pa_decode_stage(int(stage), *args), f"pa_decode_stage({stage})")
+
+
+def block_table_update(updates, block_tables, stream=None) -> None:
+    """Apply (seq, col, block) int32 [n, 3] device updates to the device block tables."""
+    n = 0 if updates is None else updates.shape[0]
+    st = lib().pa_block_table_update(_ptr(updates), n, _ptr(block_tables), block_tables.shape[0],
+                                     block_tables.shape[1], _stream(stream))
+    _check(st, "pa_block_table_update")
+
+
+def last_device_error(stream=None):
+    """(code, info) of the sticky device error word, cleared by the read (synchronises)."""
+    code = ctypes.c_int32(0)
+    info = (ctypes.c_int32 * 3)()
+    st = lib().pa_last_device_error(_stream(stream), ctypes.byref(code), info)
+    if st not in (PA_OK, PA_ERR_DEVICE_CHECK):
+        raise PaError(st, "pa_last_device_error")
+    return code.value, tuple(info)
+
+
+# ---------------------------------------------------------------------------
+# host block pool
+# ---------------------------------------------------------------------------
+
+class Pool:
+    """O(1) free-list block pool with reference counts (host memory only)."""
+
+    def __init__(self, num_blocks: int, initial_order=None):
+        import numpy as np
+        self._h = ctypes.c_void_p()
+        order = None
+        if initial_order is not None:
+            self._order = np.ascontiguousarray(np.asarray(initial_order, dtype=np.int32))
+            order = _i32p(self._order)
+        _check(lib().pa_pool_create(int(num_blocks), order, ctypes.byref(self._h)), "pa_pool_create")
+
+    def close(self):
+        if self._h:
+            lib().pa_pool_destroy(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def alloc(self) -> int:
+        b = ctypes.c_int32()
+        _check(lib().pa_pool_alloc(self._h, ctypes.byref(b)), "pa_pool_alloc")
+        return b.value
+
+    def incref(self, b: int):
+        _check(lib().pa_pool_incref(self._h, int(b)), "pa_pool_incref")
+
+    def decref(self, b: int):
+        _check(lib().pa_pool_decref(self._h, int(b)), "pa_pool_decref")
+
+    def refcount(self, b: int) -> int:
+        return lib().pa_pool_refcount(self._h, int(b))
+
+    def num_free(self) -> int:
+        return lib().pa_pool_num_free(self._h)
+
+    def free_list(self):
+        import numpy as np
+        n = self.num_free()
+        buf = np.zeros(max(n, 1), dtype=np.int32)
+        got = lib().pa_pool_free_list(self._h, _i32p(buf), n)
+        return buf[:got].tolist()
+
+    def seq_append(self, row, pos: int, block_size: int):
+        """row: host int32 array (numpy), updated in place. Returns (slot, cow_src, cow_dst)."""
+        slot = ctypes.c_int64()
+        cs, cd = ctypes.c_int32(), ctypes.c_int32()
+        _check(lib().pa_seq_append(self._h, _i32p(row), row.shape[-1], int(pos), int(block_size),
+                                   ctypes.byref(slot), ctypes.byref(cs), ctypes.byref(cd)), "pa_seq_append")
+        return slot.value, cs.value, cd.value
+
+    def seq_extend(self, row, start_pos: int, n_tokens: int, block_size: int, slots=None):
+        cs, cd, done = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+        st = lib().pa_seq_extend(self._h, _i32p(row), row.shape[-1], int(start_pos), int(n_tokens),
+                                 int(block_size), _i64p(slots) if slots is not None else None,
+                                 ctypes.byref(cs), ctypes.byref(cd), ctypes.byref(done))
+        _check(st, "pa_seq_extend")
+        return cs.value, cd.value
+
+    def seq_fork(self, row, n_blocks: int):
+        _check(lib().pa_seq_fork(self._h, _i32p(row), int(n_blocks)), "pa_seq_fork")
+
+    def seq_free(self, row, n_blocks: int):
+        _check(lib().pa_seq_free(self._h, _i32p(row), int(n_blocks)), "pa_seq_free")
+
+    def batch_append(self, block_tables, positions, block_size: int, slots, cow_pairs, updates):
+        """One step's bookkeeping. All buffers are contiguous host arrays; returns (n_cow, n_updates)."""
+        ncow, nupd, done = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+        st = lib().pa_batch_append(self._h, _i32p(block_tables), block_tables.shape[0], block_tables.shape[1],
+                                   _i32p(positions), int(block_size), _i64p(slots), _i64p(cow_pairs),
+                                   ctypes.byref(ncow), _i32p(updates), ctypes.byref(nupd), ctypes.byref(done))
+        _check(st, "pa_batch_append")
+        return ncow.value, nupd.value
+
+
+def version() -> str:
+    return lib().pa_version().decode()

@@ -1,0 +1,4 @@
+// Single translation unit for the device code of libpa: the kernels share one
+// device error word, so they are compiled together (no relocatable device code).
+#include "pa_decode.cu"
+#include "pa_cache.cu"

@@ -189,3 +189,30 @@ def normal_e4m3_codes(shape, seed: int, device="cpu", chunk=1 << 26):
         y = (x / scale).clamp_(-448.0, 448.0)
         out[start:start + m] = y.to(torch.float8_e4m3fn).view(torch.uint8)
     return out.view(*shape), float(scale)
+
+
+def fill_normal_(t, dtype: str, seed: int, chunk=1 << 26):
+    """Fill a contiguous fp16/bf16 tensor (any device) with seeded N(0, 1) values,
+    chunk by chunk (bounded temporary memory)."""
+    torch = _torch()
+    g = torch.Generator(device=t.device)
+    g.manual_seed(seed)
+    flat = t.view(-1)
+    target = getattr(torch, _TORCH_DT[dtype])
+    for start in range(0, flat.numel(), chunk):
+        m = min(chunk, flat.numel() - start)
+        x = torch.randn(m, generator=g, device=t.device, dtype=torch.float32)
+        flat[start:start + m].copy_(x.to(target).view(t.dtype))
+    return t
+
+
+def step_inputs(w: Workload, step: int, device="cpu"):
+    """The query and the new token's K/V of every sequence at a given step.
+
+    q: [S, Hq, D] (q dtype); k_new, v_new: [S, Hkv, D] (q dtype; an E4M3 cache is
+    written from the query dtype)."""
+    base = w.seed * 1000 + 17 * step
+    q = normal_values((w.num_seqs, w.num_q_heads, w.head_dim), w.q_dtype, base + 1, device)
+    k = normal_values((w.num_seqs, w.num_kv_heads, w.head_dim), w.q_dtype, base + 2, device)
+    v = normal_values((w.num_seqs, w.num_kv_heads, w.head_dim), w.q_dtype, base + 3, device)
+    return q, k, v

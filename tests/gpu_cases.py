@@ -1,0 +1,153 @@
+"""Shared set-up for the GPU parity tests: a workload is built twice, once through
+the CUDA library (engine, C++ pool, kernels) and once through the oracle (its own
+pool model, its own cache ops, float64 attention); the inputs come only from the
+seeded generators in ``synthetic``."""
+
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import synthetic
+from oracle import attention as oatt
+from oracle import cache_ops as oops
+from oracle.pool import BlockPool
+import paged_kv_cache_436_b200 as pa
+from paged_kv_cache_436_b200.engine import DecodeEngine
+
+# parity tolerances of the decode output: |err| <= atol + rtol * |ref|
+TOL = {"f16": (2e-3, 1e-2), "bf16": (2e-3, 1e-2), "e4m3": (3e-2, 3e-2)}
+
+
+def codes_np(t):
+    """Raw element codes of a tensor as an unsigned numpy array."""
+    t = t.detach().cpu().contiguous()
+    if t.element_size() == 1:
+        return t.view(torch.uint8).numpy()
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def assert_close(got, ref, kv_dtype, what=""):
+    atol, rtol = TOL[kv_dtype]
+    got = np.asarray(got, dtype=np.float64)
+    err = np.abs(got - ref)
+    bound = atol + rtol * np.abs(ref)
+    bad = err > bound
+    assert np.all(np.isfinite(got)), f"{what}: non-finite output"
+    assert not bad.any(), (f"{what}: {bad.sum()} of {bad.size} outside tolerance; "
+                           f"max err {err.max():.3e}, worst ratio {(err / bound).max():.2f}")
+    return float(err.max())
+
+
+def make_engine(w, device="cuda", growth=0, k_scale=1.0, v_scale=1.0):
+    """Engine sized for the workload's context lengths plus `growth` more tokens each."""
+    MB = w.max_blocks_per_seq(growth)
+    return DecodeEngine(num_seqs=w.num_seqs, num_q_heads=w.num_q_heads, num_kv_heads=w.num_kv_heads,
+                        head_dim=w.head_dim, block_size=w.block_size, kv_dtype=w.kv_dtype,
+                        q_dtype=w.q_dtype, num_blocks=w.num_blocks, initial_order=w.initial_order,
+                        max_blocks_per_seq=MB, max_context_len=w.max_context_len + growth,
+                        k_scale=k_scale, v_scale=v_scale, device=device)
+
+
+def fill_cache(w, eng):
+    """Seeded N(0,1) cache contents, drawn on the engine's device."""
+    if w.kv_dtype == "e4m3":
+        kc, ks = synthetic.normal_e4m3_codes(tuple(eng.k_cache.shape), w.seed * 10 + 1, eng.device)
+        vc, vs = synthetic.normal_e4m3_codes(tuple(eng.v_cache.shape), w.seed * 10 + 2, eng.device)
+        eng.k_cache.copy_(kc)
+        eng.v_cache.copy_(vc)
+        del kc, vc
+        eng.cache.desc.k_scale = ks
+        eng.cache.desc.v_scale = vs
+    else:
+        synthetic.fill_normal_(eng.k_cache, w.kv_dtype, w.seed * 10 + 1)
+        synthetic.fill_normal_(eng.v_cache, w.kv_dtype, w.seed * 10 + 2)
+
+
+class OracleMirror:
+    """The oracle's own view of the same workload: pool model, tables, cache codes
+    of the blocks it needs, and float64 attention."""
+
+    def __init__(self, w):
+        self.w = w
+        self.pool = BlockPool(w.num_blocks, w.initial_order)
+        self.rows = [[] for _ in range(w.num_seqs)]
+        self.lens = [0] * w.num_seqs
+
+    def extend(self, s, n):
+        slots, cows = self.pool.seq_extend(self.rows[s], self.lens[s], n, self.w.block_size)
+        self.lens[s] += n
+        return slots, cows
+
+    def fork(self, parent, child):
+        self.rows[child] = self.pool.fork(self.rows[parent])
+        self.lens[child] = self.lens[parent]
+
+    def step_bookkeeping(self):
+        pos = list(self.lens)
+        slots, cows, upd = self.pool.batch_append(self.rows, pos, self.w.block_size)
+        self.lens = [L + 1 for L in self.lens]
+        return slots, cows, upd
+
+    def table(self, MB):
+        bt = np.zeros((self.w.num_seqs, MB), dtype=np.int32)
+        for s, r in enumerate(self.rows):
+            bt[s, :len(r)] = r
+        return bt
+
+
+def check_tables(eng, mirror):
+    """Host block tables, lengths and reference counts of the C++ pool equal the oracle's."""
+    w = mirror.w
+    for s in range(w.num_seqs):
+        n = len(mirror.rows[s])
+        assert eng.bt_host[s, :n].tolist() == mirror.rows[s], f"block table of seq {s}"
+        assert int(eng.lens[s]) == mirror.lens[s]
+    assert eng.pool.num_free() == mirror.pool.num_free()
+    assert eng.pool.free_list() == mirror.pool.free_list()
+    for b in range(w.num_blocks):
+        assert eng.pool.refcount(b) == mirror.pool.refcnt[b]
+
+
+def run_decode_step(w, sample_heads=None, sample_seqs=None, growth=0, device="cuda"):
+    """History of L-1 tokens per sequence, then one full step that appends the
+    last token and decodes over L. Returns (max error, engine)."""
+    eng = make_engine(w, device, growth=growth)
+    fill_cache(w, eng)
+    mir = OracleMirror(w)
+    for s, L in enumerate(w.context_lens):
+        eng.extend(s, L - 1)
+        mir.extend(s, L - 1)
+    check_tables(eng, mir)
+    eng.upload_tables()
+    slots_o, cows_o, _ = mir.step_bookkeeping()
+    assert cows_o == []
+    seqs = range(w.num_seqs) if sample_seqs is None else sample_seqs
+    blocks = sorted({b for s in seqs for b in mir.rows[s]})
+    idx = torch.tensor(blocks, dtype=torch.int64, device=device)
+    k0 = codes_np(eng.k_cache.index_select(0, idx))          # the oracle's copy, before the step
+    v0 = codes_np(eng.v_cache.index_select(0, idx))
+    q, k, v = synthetic.step_inputs(w, 0)
+    qd, kd, vd = q.to(device), k.to(device), v.to(device)
+    out = torch.full_like(qd, float("nan"))
+    eng.step(qd, kd, vd, out, w.scale)
+    torch.cuda.synchronize()
+    assert pa.last_device_error()[0] == 0
+    check_tables(eng, mir)
+    # the oracle writes the new tokens into its copy (slots remapped to the copied blocks)
+    remap = {b: i for i, b in enumerate(blocks)}
+    BS = w.block_size
+    sl = np.array([remap[s_ // BS] * BS + s_ % BS if (s_ // BS) in remap else -1 for s_ in slots_o])
+    ks, vs = eng.cache.desc.k_scale, eng.cache.desc.v_scale
+    ek, ev = oops.reshape_and_cache(codes_np(k), codes_np(v), w.q_dtype, sl, k0, v0, w.kv_dtype, ks, vs)
+    assert np.array_equal(codes_np(eng.k_cache.index_select(0, idx)), ek), "K cache after the step"
+    assert np.array_equal(codes_np(eng.v_cache.index_select(0, idx)), ev), "V cache after the step"
+    bt = np.zeros((w.num_seqs, eng.MB), np.int64)
+    for s in seqs:
+        bt[s, :len(mir.rows[s])] = [remap[b] for b in mir.rows[s]]
+    heads = [(s, h) for s in seqs for h in (range(w.num_q_heads) if sample_heads is None else sample_heads)]
+    ref = oatt.paged_decode(codes_np(q), w.q_dtype, ek, ev, w.kv_dtype, ks, vs, bt, mir.lens, w.scale,
+                            heads=heads)
+    got = out.double().cpu().numpy()
+    hs = tuple(np.array(heads).T)
+    return assert_close(got[hs], ref[hs], w.kv_dtype, w.name), eng

@@ -1,0 +1,229 @@
+"""CPU tests of the C-ABI library: it loads, exports every symbol the header
+declares, and its host block pool matches the oracle's pool model bit for bit.
+No GPU call is made here."""
+
+import ctypes
+import os
+import re
+import time
+
+import numpy as np
+import pytest
+
+import paged_kv_cache_436_b200 as pa
+from oracle.pool import BlockPool, PoolError
+from paged_kv_cache_436_b200 import build as pa_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built_library():
+    if pa_build.stale():
+        pa_build.build()
+    return pa.lib()
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "pa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pa_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = header_functions()
+    assert len(names) >= 20
+    L = ctypes.CDLL(pa.LIB_PATH)
+    missing = [n for n in names if not hasattr(L, n)]
+    assert not missing, missing
+    assert set(names) == set(pa._SIGNATURES), "binding and header disagree"
+
+
+def test_version_and_sizes():
+    assert "sm_100a" in pa.version()
+    # plan (S+1 ints) + (m, l) + acc per (seq, q head, partition), each 256-byte aligned
+    assert pa.decode_workspace_size(8, 32, 128, 32768) == 256 + 8 * 32 * 64 * 2 * 4 + 8 * 32 * 64 * 128 * 4
+    assert pa.decode_workspace_size(-1, 32, 128, 10) == 0
+
+
+def test_host_argument_checks_launch_nothing():
+    L = pa.lib()
+    desc = pa.CacheDesc(16, 2, 16, 128, pa.PA_BF16, 1.0, 1.0, 0, 0)      # null cache pointers
+    assert L.pa_copy_blocks(None, 1, ctypes.byref(desc), None) == pa.PA_ERR_ARG
+    desc = pa.CacheDesc(16, 2, 16, 96, pa.PA_BF16, 1.0, 1.0, 256, 256)  # unsupported head_dim
+    assert L.pa_reshape_and_cache(None, None, pa.PA_BF16, 1, 256, 256, None, ctypes.byref(desc), None) == pa.PA_ERR_ARG
+    desc = pa.CacheDesc(16, 2, 16, 128, pa.PA_BF16, 2.0, 1.0, 256, 256)  # scale on a 16-bit cache
+    assert L.pa_copy_blocks(None, 0, ctypes.byref(desc), None) == pa.PA_ERR_ARG
+    desc = pa.CacheDesc(16, 2, 12, 128, pa.PA_BF16, 1.0, 1.0, 256, 256)  # block size 12
+    assert L.pa_copy_blocks(None, 0, ctypes.byref(desc), None) == pa.PA_ERR_ARG
+    desc = pa.CacheDesc(16, 2, 16, 128, pa.PA_BF16, 1.0, 1.0, 256, 256)
+    # 6 q heads over 2 kv heads: G = 3 is not supported
+    assert L.pa_decode(256, pa.PA_BF16, 1, 6, ctypes.byref(desc), 256, 1, 256, 16, 1.0, 256, 256, 1 << 20,
+                       None) == pa.PA_ERR_ARG
+    # q dtype must match a 16-bit cache
+    assert L.pa_decode(256, pa.PA_F16, 1, 2, ctypes.byref(desc), 256, 1, 256, 16, 1.0, 256, 256, 1 << 20,
+                       None) == pa.PA_ERR_ARG
+    # workspace too small
+    assert L.pa_decode(256, pa.PA_BF16, 4, 2, ctypes.byref(desc), 256, 4, 256, 2048, 1.0, 256, 256, 64,
+                       None) == pa.PA_ERR_ARG
+    # no sequences: nothing to do
+    assert L.pa_decode(None, pa.PA_BF16, 0, 2, ctypes.byref(desc), None, 1, None, 0, 1.0, None, None, 0,
+                       None) == pa.PA_OK
+
+
+def _oracle_equal(native: pa.Pool, model: BlockPool):
+    assert native.num_free() == model.num_free()
+    assert native.free_list() == model.free_list()
+    for b in range(model.num_blocks):
+        assert native.refcount(b) == model.refcnt[b]
+
+
+def test_native_pool_fixtures_match_oracle():
+    order = [0, 1, 2, 4, 3, 7, 8, 9, 5, 6, 10, 11]
+    native, model = pa.Pool(12, order), BlockPool(12, order)
+    rows_n = {r: np.zeros(4, np.int32) for r in "ABC"}
+    rows_m = {r: [] for r in "ABC"}
+    lens = {"A": 3, "B": 3, "C": 2}
+    for lb in range(3):
+        for r in "ABC":
+            if lb < lens[r]:
+                sn = native.seq_append(rows_n[r], lb * 16, 16)
+                sm = model.seq_append(rows_m[r], lb * 16, 16)
+                assert sn == sm
+    assert {r: rows_n[r][:lens[r]].tolist() for r in "ABC"} == {"A": [0, 4, 8], "B": [1, 3, 9], "C": [2, 7]}
+    _oracle_equal(native, model)
+
+
+def test_native_pool_errors():
+    p = pa.Pool(2)
+    assert [p.alloc(), p.alloc()] == [0, 1]
+    with pytest.raises(pa.PaError) as e:
+        p.alloc()
+    assert e.value.status == pa.PA_ERR_OOM
+    p.decref(1)
+    with pytest.raises(pa.PaError) as e:
+        p.decref(1)
+    assert e.value.status == pa.PA_ERR_STATE
+    with pytest.raises(pa.PaError) as e:
+        p.incref(1)
+    assert e.value.status == pa.PA_ERR_STATE
+    with pytest.raises(pa.PaError) as e:
+        pa.Pool(3, [0, 2, 2])
+    assert e.value.status == pa.PA_ERR_ARG
+    row = np.zeros(1, np.int32)
+    with pytest.raises(pa.PaError):
+        p.seq_append(row, 16, 16)          # logical block 1 is beyond the 1-entry row
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_native_pool_random_ops_match_oracle(seed):
+    rng = np.random.default_rng(100 + seed)
+    NB, BS, MB = 96, 8, 64
+    order = rng.permutation(NB)
+    native, model = pa.Pool(NB, order), BlockPool(NB, order)
+    seqs = []    # [native row, model row, length]
+    for _ in range(1500):
+        op = int(rng.integers(0, 5))
+        if op == 0 or not seqs:
+            n = int(rng.integers(1, 40))
+            rn, rm = np.zeros(MB, np.int32), []
+            slots_n = np.zeros(n, np.int64)
+            try:
+                model.seq_extend(rm, 0, n, BS)
+                ok_m = True
+            except PoolError:
+                ok_m = False
+            try:
+                native.seq_extend(rn, 0, n, BS, slots_n)
+                ok_n = True
+            except pa.PaError as e:
+                assert e.status == pa.PA_ERR_OOM
+                ok_n = False
+            assert ok_m == ok_n
+            if ok_m:
+                seqs.append([rn, rm, n])
+            else:
+                # both stranded the same partial allocation; keep the pools comparable
+                pass
+        elif op == 1:
+            i = int(rng.integers(len(seqs)))
+            rn, rm, n = seqs[i]
+            try:
+                a = model.seq_append(rm, n, BS)
+            except PoolError:
+                a = None
+            try:
+                b = native.seq_append(rn, n, BS)
+            except pa.PaError:
+                b = None
+            assert a == b
+            if a is not None:
+                seqs[i][2] = n + 1
+        elif op == 2:
+            i = int(rng.integers(len(seqs)))
+            rn, rm, n = seqs[i]
+            nb = -(-n // BS)
+            native.seq_fork(rn, nb)
+            seqs.append([rn.copy(), model.fork(rm), n])
+        elif op == 3:
+            i = int(rng.integers(len(seqs)))
+            rn, rm, n = seqs.pop(i)
+            native.seq_free(rn, -(-n // BS))
+            model.free_seq(rm)
+        else:
+            # a batched decode step over all live sequences
+            if not seqs:
+                continue
+            S = len(seqs)
+            bt = np.zeros((S, MB), np.int32)
+            for s, (rn, _, _) in enumerate(seqs):
+                bt[s] = rn
+            pos = np.array([n for _, _, n in seqs], np.int32)
+            snap = (model.free_list(), list(model.refcnt), [list(r) for _, r, _ in seqs])
+            try:
+                slots_m, cows_m, upd_m = model.batch_append([r for _, r, _ in seqs], list(pos), BS)
+                ok = True
+            except PoolError:
+                ok = False
+            slots = np.zeros(S, np.int64)
+            cows = np.zeros((S, 2), np.int64)
+            upd = np.zeros((S, 3), np.int32)
+            try:
+                ncow, nupd = native.batch_append(bt, pos, BS, slots, cows, upd)
+                ok_n = True
+            except pa.PaError:
+                ok_n = False
+            assert ok == ok_n
+            if not ok:
+                # partial batch on both sides: rebuild the comparison from scratch
+                return
+            assert slots.tolist() == slots_m
+            assert [tuple(x) for x in cows[:ncow].tolist()] == cows_m
+            assert [tuple(x) for x in upd[:nupd].tolist()] == upd_m
+            for s in range(S):
+                seqs[s][0] = bt[s].copy()
+                seqs[s][2] += 1
+        for rn, rm, n in seqs:
+            assert rn[:len(rm)].tolist() == rm
+        _oracle_equal(native, model)
+
+
+def test_alloc_free_cost_is_flat_in_pool_size():
+    """O(1) alloc/free: the time per operation does not grow with the pool (page 3,
+    section "PagedAttention原理")."""
+    L = pa.lib()
+
+    def per_op(nb):
+        p = pa.Pool(nb)
+        row = np.zeros(4096, np.int32)
+        cs, cd, done = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+        t0 = time.perf_counter()
+        for _ in range(20):
+            assert L.pa_seq_extend(p._h, pa._i32p(row), 4096, 0, 4096 * 16, 16, None,
+                                   ctypes.byref(cs), ctypes.byref(cd), ctypes.byref(done)) == 0
+            assert L.pa_seq_free(p._h, pa._i32p(row), 4096) == 0
+        return (time.perf_counter() - t0) / (20 * 4096 * 16)
+
+    small = min(per_op(4096) for _ in range(3))
+    big = min(per_op(1 << 22) for _ in range(3))
+    assert big < 4 * small + 2e-8, (small, big)

@@ -1,0 +1,210 @@
+"""GPU parity of the decode step against the float64 oracle.
+
+Each case builds the workload twice from the same seeded inputs -- through the
+CUDA library (C++ pool, device tables, kernels) and through the oracle (its own
+pool model, cache ops and attention) -- and compares block tables and cache
+bytes exactly and attention outputs within the tolerance of the KV format:
+|err| <= 2e-3 + 1e-2 |ref| for fp16/bf16 caches, 3e-2 + 3e-2 |ref| for E4M3.
+"""
+
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import paged_kv_cache_436_b200 as pa
+import synthetic
+from oracle import attention as oatt
+from oracle import cache_ops as oops
+from tests.gpu_cases import (OracleMirror, assert_close, check_tables, codes_np, fill_cache, make_engine,
+                              run_decode_step)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def test_tiny_config():
+    w = synthetic.make("tiny")
+    run_decode_step(w)
+
+
+def test_tiny_extra_slots_into_free_blocks():
+    """4 new tokens written into slots of blocks no sequence holds: rows exact, rest untouched."""
+    w = synthetic.make("tiny")
+    eng = make_engine(w, DEV)
+    fill_cache(w, eng)
+    for s, L in enumerate(w.context_lens):
+        eng.extend(s, L)
+    held = {int(b) for s in range(4) for b in eng.bt_host[s, :-(-w.context_lens[s] // 16)]}
+    assert not held & {sl // 16 for sl in w.extra_slots}
+    k0, v0 = codes_np(eng.k_cache), codes_np(eng.v_cache)
+    _, k, v = synthetic.step_inputs(w, 5)
+    slots = np.array(w.extra_slots, np.int64)
+    pa.reshape_and_cache(k.to(DEV), v.to(DEV), torch.from_numpy(slots).to(DEV), eng.cache)
+    ek, ev = oops.reshape_and_cache(codes_np(k), codes_np(v), "f16", slots, k0, v0, "f16")
+    assert np.array_equal(codes_np(eng.k_cache), ek) and np.array_equal(codes_np(eng.v_cache), ev)
+
+
+def test_llama7b_step_config():
+    run_decode_step(synthetic.make("llama7b_step"))
+
+
+def test_gqa_prefix_config():
+    """1000-token prefix written once and shared by 64 sequences; 63 copy-on-write
+    block copies; private tokens written; decode with 32 q / 8 kv heads."""
+    w = synthetic.make("gqa_prefix")
+    eng = make_engine(w, DEV)
+    fill_cache(w, eng)
+    mir = OracleMirror(w)
+    P = w.prefix_len
+    pre_slots = np.zeros(P, np.int64)
+    eng.extend(0, P, pre_slots)
+    sl_o, _ = mir.extend(0, P)
+    assert pre_slots.tolist() == sl_o
+    for s in range(1, w.num_seqs):
+        eng.fork(0, s)
+        mir.fork(0, s)
+    pairs, priv_slots, pairs_o, priv_o = [], [], [], []
+    for s, p in enumerate(w.private_lens):
+        sl = np.zeros(p, np.int64)
+        cs, cd = eng.extend(s, p, sl)
+        if cs >= 0:
+            pairs.append((cs, cd))
+        priv_slots.append(sl)
+        so, co = mir.extend(s, p)
+        pairs_o += co
+        priv_o += so
+    assert pairs == pairs_o and len(pairs) == w.num_seqs - 1
+    priv_slots = np.concatenate(priv_slots)
+    assert priv_slots.tolist() == priv_o
+    check_tables(eng, mir)
+    eng.upload_tables()
+    k0, v0 = codes_np(eng.k_cache), codes_np(eng.v_cache)
+    n_priv = int(sum(w.private_lens))
+    kp = synthetic.normal_values((P, w.num_kv_heads, w.head_dim), "bf16", w.seed + 101)
+    vp = synthetic.normal_values((P, w.num_kv_heads, w.head_dim), "bf16", w.seed + 102)
+    kq = synthetic.normal_values((n_priv, w.num_kv_heads, w.head_dim), "bf16", w.seed + 103)
+    vq = synthetic.normal_values((n_priv, w.num_kv_heads, w.head_dim), "bf16", w.seed + 104)
+    q = synthetic.normal_values((w.num_seqs, w.num_q_heads, w.head_dim), "bf16", w.seed + 105)
+    pa.reshape_and_cache(kp.to(DEV), vp.to(DEV), torch.from_numpy(pre_slots).to(DEV), eng.cache)
+    pa.copy_blocks(torch.tensor(pairs, dtype=torch.int64, device=DEV), eng.cache)
+    pa.reshape_and_cache(kq.to(DEV), vq.to(DEV), torch.from_numpy(priv_slots).to(DEV), eng.cache)
+    out = torch.full((w.num_seqs, w.num_q_heads, w.head_dim), float("nan"), dtype=torch.bfloat16, device=DEV)
+    eng.run_decode(q.to(DEV), out, w.scale)
+    torch.cuda.synchronize()
+    assert pa.last_device_error()[0] == 0
+    ek, ev = oops.reshape_and_cache(codes_np(kp), codes_np(vp), "bf16", pre_slots, k0, v0, "bf16")
+    ek, ev = oops.copy_blocks(ek, ev, pairs_o)
+    ek, ev = oops.reshape_and_cache(codes_np(kq), codes_np(vq), "bf16", priv_slots, ek, ev, "bf16")
+    assert np.array_equal(codes_np(eng.k_cache), ek) and np.array_equal(codes_np(eng.v_cache), ev)
+    ref = oatt.paged_decode(codes_np(q), "bf16", ek, ev, "bf16", 1.0, 1.0, mir.table(eng.MB), mir.lens, w.scale)
+    assert_close(out.double().cpu().numpy(), ref, "bf16", "gqa_prefix")
+
+
+# partition edges (512), block edges, and a long tail
+EDGE_LENS = [1, 2, 15, 16, 17, 511, 512, 513, 1023, 1024, 1025, 1537, 2100]
+
+
+@pytest.mark.parametrize("kv,q,D,BS,G", [
+    ("bf16", "bf16", 128, 16, 1), ("f16", "f16", 128, 16, 1), ("bf16", "bf16", 128, 16, 4),
+    ("f16", "f16", 64, 16, 2), ("bf16", "bf16", 64, 8, 8), ("f16", "f16", 128, 32, 4),
+    ("bf16", "bf16", 128, 8, 2), ("e4m3", "bf16", 128, 32, 1), ("e4m3", "f16", 64, 16, 4),
+    ("e4m3", "bf16", 128, 16, 8), ("e4m3", "bf16", 64, 8, 1), ("bf16", "bf16", 128, 32, 8)])
+def test_fuzz_shapes_and_partition_edges(kv, q, D, BS, G):
+    Hkv = 2
+    seed = zlib.crc32(repr((kv, q, D, BS, G)).encode()) % 100000
+    w = synthetic.custom(len(EDGE_LENS), Hkv * G, Hkv, D, BS, kv, q, EDGE_LENS, seed)
+    run_decode_step(w)
+
+
+def test_single_token_context_returns_value_row():
+    w = synthetic.custom(3, 4, 4, 128, 16, "bf16", "bf16", [1, 1, 1], 77)
+    err, eng = run_decode_step(w)
+    assert err == 0.0      # the softmax of one score is exactly 1: out = V row, rounded once
+
+
+def test_empty_context_gives_zero_rows():
+    w = synthetic.custom(3, 8, 2, 128, 16, "bf16", "bf16", [40, 1, 700], 78)
+    eng = make_engine(w, DEV)
+    fill_cache(w, eng)
+    for s, L in enumerate(w.context_lens):
+        eng.extend(s, L)
+    eng.upload_tables()
+    eng.lens_dev.copy_(torch.tensor([40, 0, 700], dtype=torch.int32))
+    q = synthetic.normal_values((3, 8, 128), "bf16", 5).to(DEV)
+    out = torch.full_like(q, float("nan"))
+    eng.run_decode(q, out, w.scale)
+    o = out.float().cpu()
+    assert torch.all(o[1] == 0) and torch.isfinite(o).all()
+
+
+def test_block_permutation_gives_identical_bits():
+    """Moving every physical block (and its table entries) leaves the output bits unchanged."""
+    w = synthetic.custom(4, 8, 8, 128, 16, "bf16", "bf16", [100, 600, 1300, 31], 79)
+    eng = make_engine(w, DEV)
+    fill_cache(w, eng)
+    for s, L in enumerate(w.context_lens):
+        eng.extend(s, L)
+    eng.upload_tables()
+    q = synthetic.normal_values((4, 8, 128), "bf16", 6).to(DEV)
+    out1 = torch.empty_like(q)
+    eng.run_decode(q, out1, w.scale)
+    perm = torch.from_numpy(np.random.default_rng(9).permutation(w.num_blocks)).to(DEV)
+    kc2, vc2 = torch.empty_like(eng.k_cache), torch.empty_like(eng.v_cache)
+    kc2[perm] = eng.k_cache
+    vc2[perm] = eng.v_cache
+    cache2 = pa.KVCache(kc2, vc2, "bf16")
+    bt2 = perm.to(torch.int32)[eng.bt_dev.long()]
+    out2 = torch.empty_like(q)
+    pa.decode(q, cache2, bt2, eng.lens_dev, eng.max_context_len, w.scale, out2, eng.ws)
+    assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
+
+
+def test_gqa_equals_mha_with_duplicated_kv_heads():
+    """G query heads sharing a kv head give the bits of MHA over G copies of it."""
+    w = synthetic.custom(3, 8, 2, 128, 16, "bf16", "bf16", [77, 530, 1200], 80)
+    eng = make_engine(w, DEV)
+    fill_cache(w, eng)
+    for s, L in enumerate(w.context_lens):
+        eng.extend(s, L)
+    eng.upload_tables()
+    q = synthetic.normal_values((3, 8, 128), "bf16", 7).to(DEV)
+    out_g = torch.empty_like(q)
+    eng.run_decode(q, out_g, w.scale)
+    kc = eng.k_cache.repeat_interleave(4, dim=1).contiguous()
+    vc = eng.v_cache.repeat_interleave(4, dim=1).contiguous()
+    out_m = torch.empty_like(q)
+    pa.decode(q, pa.KVCache(kc, vc, "bf16"), eng.bt_dev, eng.lens_dev, eng.max_context_len, w.scale,
+              out_m, eng.ws)
+    assert torch.equal(out_g.view(torch.int16), out_m.view(torch.int16))
+
+
+def test_bad_block_id_is_recorded_not_faulting():
+    w = synthetic.custom(2, 4, 4, 128, 16, "bf16", "bf16", [40, 20], 81)
+    eng = make_engine(w, DEV)
+    fill_cache(w, eng)
+    for s, L in enumerate(w.context_lens):
+        eng.extend(s, L)
+    eng.bt_host[1, 1] = w.num_blocks + 7
+    eng.upload_tables()
+    q = synthetic.normal_values((2, 4, 128), "bf16", 8).to(DEV)
+    out = torch.empty_like(q)
+    eng.run_decode(q, out, w.scale)
+    code, info = pa.last_device_error()
+    assert code == 1 and info == (1, 1, w.num_blocks + 7)
+
+
+def test_context_beyond_table_is_clamped_and_recorded():
+    w = synthetic.custom(2, 4, 4, 128, 16, "bf16", "bf16", [40, 20], 82)
+    eng = make_engine(w, DEV)
+    fill_cache(w, eng)
+    for s, L in enumerate(w.context_lens):
+        eng.extend(s, L)
+    eng.upload_tables()
+    eng.lens_dev.copy_(torch.tensor([40, 10 ** 6], dtype=torch.int32))
+    q = synthetic.normal_values((2, 4, 128), "bf16", 9).to(DEV)
+    out = torch.empty_like(q)
+    eng.run_decode(q, out, w.scale)
+    code, info = pa.last_device_error()
+    assert code == 2 and info[0] == 1 and info[1] == 10 ** 6
