@@ -54,6 +54,25 @@ def peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def kernel_traffic(workload: str, bytes_per_launch: float):
+    """DRAM bytes per partition-kernel launch, scaled from the committed ncu capture's
+    traffic / algorithmic-byte ratio; None when the kernel source changed since."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "partition_kernel_traffic.json")) as f:
+            rec = json.load(f)
+        h = hashlib.sha256()
+        for name in ("pa_decode.cu", "pa_device.cuh"):
+            with open(os.path.join(ROOT, "paged_kv_cache_436_b200", "csrc", name), "rb") as f:
+                h.update(f.read())
+        if h.hexdigest() != rec["source_sha256"]:
+            return None
+        base = workload.split("[")[0]
+        return rec["traffic_per_algorithmic_byte"][base] * bytes_per_launch
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def decode_bytes(lens, hkv, hq, d, kv_bytes, q_bytes, bs) -> int:
     """Algorithmic bytes of one decode step: K and V of every context token once per
     kv head, q in, out back, the block-table entries read, the context lengths."""
@@ -115,7 +134,7 @@ def barrier(dist, device=None):
 # ---------------------------------------------------------------------------
 
 class ClockSampler:
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    QUERY = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -135,7 +154,10 @@ class ClockSampler:
         except Exception:
             self.proc = None
 
-    def stop(self):
+    def stop(self, window=None):
+        """Median SM clock, max clock and throttle reasons of the samples taken inside
+        `window` = (t_start, t_end) host wall-clock seconds (all samples if None)."""
+        import datetime
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
         time.sleep(0.25)
@@ -149,14 +171,18 @@ class ClockSampler:
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in open(self.path):
             parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
+            if len(parts) < 10:
                 continue
             try:
-                sm.append(float(parts[1]))
-                smax.append(float(parts[2]))
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                clk, cmax = float(parts[2]), float(parts[3])
             except ValueError:
                 continue
-            for n, v in zip(names, parts[5:9]):
+            if window is not None and not (window[0] - 0.05 <= ts <= window[1] + 0.05):
+                continue
+            sm.append(clk)
+            smax.append(cmax)
+            for n, v in zip(names, parts[6:10]):
                 if v.lower() == "active":
                     reasons.add(n)
         if not sm:
@@ -176,6 +202,7 @@ def build_engine(w, growth, device):
     import torch
     import synthetic
     from paged_kv_cache_436_b200.engine import DecodeEngine
+    w = synthetic.grown(w, growth)
     eng = DecodeEngine(num_seqs=w.num_seqs, num_q_heads=w.num_q_heads, num_kv_heads=w.num_kv_heads,
                        head_dim=w.head_dim, block_size=w.block_size, kv_dtype=w.kv_dtype, q_dtype=w.q_dtype,
                        num_blocks=w.num_blocks, initial_order=w.initial_order,
@@ -273,6 +300,7 @@ def time_ours(w, steps, warmup, device, dist, e2e=True, clocks=True, local_rank=
     torch.cuda.synchronize(device)
     barrier(dist, device)
     total_bytes, launches, lens_sum, kbytes = 0, 0, 0, []
+    wall0 = time.time()
     t0.record()
     for i in range(steps):
         nb, nl = run.step(i, kev[i])
@@ -282,7 +310,8 @@ def time_ours(w, steps, warmup, device, dist, e2e=True, clocks=True, local_rank=
         kbytes.append(nb)
     t1.record()
     torch.cuda.synchronize(device)
-    clk = sampler.stop() if sampler else None
+    wall1 = time.time()
+    clk = sampler.stop((wall0, wall1)) if sampler else None
     ms = t0.elapsed_time(t1)
     kernel_ms = [a.elapsed_time(b) for a, b in kev]
     ms_max = reduce_max(ms, dist, device)
@@ -320,36 +349,39 @@ def time_ours(w, steps, warmup, device, dist, e2e=True, clocks=True, local_rank=
 # the oracle on the host cores (cpu_baseline and --impl reference)
 # ---------------------------------------------------------------------------
 
+def _sample_item(w, s, rng):
+    """Blocks of sequence s for the oracle, drawn fresh on the host, laid out 0..n-1."""
+    import synthetic
+    L = w.context_lens[s]
+    nbk = -(-L // w.block_size)
+    shape = (nbk, w.num_kv_heads, w.block_size, w.head_dim)
+    if w.kv_dtype == "e4m3":
+        kc = rng.integers(0, 0x7E, size=shape, dtype=np.uint8)
+        vc = rng.integers(0, 0x7E, size=shape, dtype=np.uint8)
+        ks = vs = 6.0 / 448
+    else:
+        kc = synthetic.normal_codes(shape, w.kv_dtype, s + 1).numpy().view(np.uint16)
+        vc = synthetic.normal_codes(shape, w.kv_dtype, s + 2).numpy().view(np.uint16)
+        ks = vs = 1.0
+    return (s, L, kc, vc, ks, vs, np.arange(nbk, dtype=np.int64)[None, :])
+
+
 def oracle_sample_inputs(w, budget_s):
-    """A bounded sample of the workload for the float64 oracle: whole sequences
-    (all heads) in a seeded order, as many as fit in about `budget_s` of CPU time
-    at a first estimate; their blocks are drawn fresh on the host, laid out 0..n-1."""
+    """A bounded sample of the workload for the float64 oracle: whole sequences (all
+    heads) in a seeded order, added one at a time until the oracle has spent about
+    `budget_s` seconds of CPU time on them."""
     import synthetic
     rng = np.random.default_rng(w.seed + 7)
     order = rng.permutation(w.num_seqs)
     q = synthetic.normal_codes((w.num_seqs, w.num_q_heads, w.head_dim), w.q_dtype, w.seed + 9).numpy()
     q = q.view(np.uint16)
-    # first estimate: ~0.7 us of oracle time per (token, kv head) on one core
-    est, chosen = 0.0, []
+    items, spent = [], 0.0
     for s in order:
-        chosen.append(int(s))
-        est += 0.7e-6 * w.context_lens[s] * w.num_q_heads
-        if est >= budget_s:
+        item = _sample_item(w, int(s), rng)
+        spent += oracle_run(w, q, [item])[2]
+        items.append(item)
+        if spent >= budget_s:
             break
-    items = []
-    for s in chosen:
-        L = w.context_lens[s]
-        nbk = -(-L // w.block_size)
-        shape = (nbk, w.num_kv_heads, w.block_size, w.head_dim)
-        if w.kv_dtype == "e4m3":
-            kc = rng.integers(0, 0x7E, size=shape, dtype=np.uint8)
-            vc = rng.integers(0, 0x7E, size=shape, dtype=np.uint8)
-            ks = vs = 6.0 / 448
-        else:
-            kc = synthetic.normal_codes(shape, w.kv_dtype, s + 1).numpy().view(np.uint16)
-            vc = synthetic.normal_codes(shape, w.kv_dtype, s + 2).numpy().view(np.uint16)
-            ks = vs = 1.0
-        items.append((s, L, kc, vc, ks, vs, np.arange(nbk, dtype=np.int64)[None, :]))
     return q, items
 
 
@@ -418,19 +450,24 @@ def workload_config(w, n_gpus):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="llama13b_mix")
     ap.add_argument("--also", default="long_fp8", help="second workload reported in the same line ('' = none)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--no-cpu", action="store_true", help="skip the oracle's cpu_baseline leg")
+    ap.add_argument("--subset", type=int, default=0,
+                    help="only the first N sequences (a smaller case of the same shapes, for profiling)")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)
 
     import synthetic
     world, rank, local = dist_env()
     w = synthetic.make(args.workload)
+    if args.subset:
+        w = synthetic.subset(w, args.subset)
 
     if args.impl == "reference":
         if rank != 0:
@@ -452,6 +489,8 @@ def main(argv=None):
         also = None
         if args.also:
             wa = synthetic.make(args.also)
+            if args.subset:
+                wa = synthetic.subset(wa, max(1, args.subset * wa.num_seqs // 256))
             also = time_ours(wa, args.steps, args.warmup, device, dist, e2e=False, clocks=False,
                              local_rank=local)
         peak, peak_src = peaks()
@@ -471,7 +510,7 @@ def main(argv=None):
                          "peak_source": peak_src + " HBM copy bandwidth (MEASURED_PEAKS hbm_gbs)",
                          "frac_of_nominal_8tbs": kern_gbs / NOMINAL_HBM_GBS,
                          "bytes_per_launch": res["kernel_bytes_mean"], "ms_per_launch": res["kernel_ms_mean"],
-                         "traffic": None},
+                         "traffic": kernel_traffic(w.name, res["kernel_bytes_mean"])},
             "gpu_launches": res["launches"],
             "clocks": res["clocks"],
         }
@@ -489,8 +528,9 @@ def main(argv=None):
                                          "achieved": also["kernel_bytes_mean"] / (also["kernel_ms_mean"] / 1e3) / 1e9,
                                          "peak": peak, "unit": "GB/s",
                                          "frac": also["kernel_bytes_mean"] / (also["kernel_ms_mean"] / 1e3) / 1e9 / peak,
-                                         "ms_per_launch": also["kernel_ms_mean"]}}
-        if rank == 0 and world == 1:
+                                         "ms_per_launch": also["kernel_ms_mean"],
+                                         "traffic": kernel_traffic(wa.name, also["kernel_bytes_mean"])}}
+        if rank == 0 and world == 1 and not args.no_cpu:
             line["cpu_baseline"] = cpu_baseline_obj(w, args.cpu_budget)
         if rank == 0:
             print(json.dumps(line))

@@ -216,3 +216,30 @@ def step_inputs(w: Workload, step: int, device="cpu"):
     k = normal_values((w.num_seqs, w.num_kv_heads, w.head_dim), w.q_dtype, base + 2, device)
     v = normal_values((w.num_seqs, w.num_kv_heads, w.head_dim), w.q_dtype, base + 3, device)
     return q, k, v
+
+
+def subset(w: Workload, n_seqs: int) -> Workload:
+    """The first n_seqs sequences of a workload, with a pool re-sized to 1.1x their
+    need and a fresh seeded permutation (smaller device footprint, same shapes)."""
+    if n_seqs >= w.num_seqs:
+        return w
+    rng = np.random.default_rng(w.seed + 1000 * n_seqs)
+    lens = list(w.context_lens[:n_seqs])
+    nb = _pool_size(lens, w.block_size)
+    return Workload(f"{w.name}[:{n_seqs}]", w.index, n_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim,
+                    w.block_size, w.kv_dtype, w.q_dtype, lens, nb, rng.permutation(nb).tolist(), w.scale,
+                    w.seed, w.prefix_len, list(w.private_lens[:n_seqs]), [])
+
+
+def grown(w: Workload, tokens: int) -> Workload:
+    """The same workload with room for `tokens` more tokens per sequence: the pool
+    gains S * ceil(tokens / BS) blocks, handed out (in a seeded order) after the
+    recipe's own blocks."""
+    extra = w.num_seqs * (-(-tokens // w.block_size))
+    if extra == 0:
+        return w
+    rng = np.random.default_rng(w.seed + 77)
+    order = list(w.initial_order) + (w.num_blocks + rng.permutation(extra)).tolist()
+    return Workload(w.name, w.index, w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size,
+                    w.kv_dtype, w.q_dtype, list(w.context_lens), w.num_blocks + extra, order, w.scale,
+                    w.seed, w.prefix_len, list(w.private_lens), list(w.extra_slots))
