@@ -17,7 +17,8 @@
  *
  * Conventions for every call below.
  *   - Device pointers are plain CUDA device addresses owned by the caller; the
- *     library never allocates, frees or retains device memory. Host pointers are
+ *     library never allocates or frees device memory, and the only device memory it
+ *     holds is the fixed scratch array of pa_decode_no_alloc. Host pointers are
  *     plain host memory owned by the caller.
  *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
  *     stream). GPU calls only enqueue work and return; results are ready when the
@@ -181,6 +182,33 @@ pa_status pa_decode_stage(int32_t stage, const void* q, int32_t q_dtype, int32_t
                           const int32_t* block_tables, int32_t max_blocks_per_seq,
                           const int32_t* context_lens, int32_t max_context_len, float scale,
                           void* out, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * pa_decode_no_alloc -- pa_decode for callers that may not allocate device memory.
+ * The source pages have no counterpart; this entry point exists for integration.
+ * Who needs it: code that is not allowed to call cudaMalloc/cudaFree, e.g. a plugin
+ * inside a host framework that owns all device memory through its own caching
+ * allocator (raw allocations would escape its accounting, and cudaFree synchronises
+ * the device), or a serving loop that forbids allocation calls because they can
+ * stall other streams. Same arguments and results as pa_decode, minus the
+ * workspace: the split-K scratch is a fixed array of PA_NO_ALLOC_WORKSPACE_BYTES
+ * (16 MiB) inside the library's device image, present on every GPU that loads the
+ * library until the process exits. The call allocates nothing.
+ *   - Sizes whose pa_decode_workspace_size() exceeds PA_NO_ALLOC_WORKSPACE_BYTES are
+ *     rejected with PA_ERR_ARG before anything is enqueued (e.g. 8 sequences x 32 q
+ *     heads x 32K tokens x head_dim 128 fit; 256 x 40 heads x 8K do not).
+ *   - The first call on a device looks up the array's device address (once per
+ *     device, with that device current); make that first call before any stream
+ *     capture.
+ *   - Every call on a device shares the one array and leaves its contents behind;
+ *     nothing in it needs to start at zero. Calls that may overlap on the GPU (on
+ *     different streams, or from different host threads) race on it: serialise them.
+ */
+#define PA_NO_ALLOC_WORKSPACE_BYTES ((size_t)16 << 20)
+pa_status pa_decode_no_alloc(const void* q, int32_t q_dtype, int32_t num_seqs, int32_t num_q_heads,
+                             const pa_cache_desc* cache, const int32_t* block_tables,
+                             int32_t max_blocks_per_seq, const int32_t* context_lens,
+                             int32_t max_context_len, float scale, void* out, void* stream);
 
 /*
  * pa_last_device_error -- synchronise `stream`, then read and clear the device error

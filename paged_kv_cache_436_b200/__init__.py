@@ -61,6 +61,7 @@ _SIGNATURES = {
     "pa_decode_stage": (_I32, [_I32, _P, _I32, _I32, _I32, _PDESC, _P, _I32, _P, _I32, ctypes.c_float,
                                _P, _P, ctypes.c_size_t, _P]),
     "pa_decode_workspace_size": (ctypes.c_size_t, [_I32, _I32, _I32, _I32]),
+    "pa_decode_no_alloc": (_I32, [_P, _I32, _I32, _I32, _PDESC, _P, _I32, _P, _I32, ctypes.c_float, _P, _P]),
     "pa_last_device_error": (_I32, [_P, _PI32, _PI32]),
     "pa_block_table_update": (_I32, [_P, _I32, _P, _I32, _I32, _P]),
     "pa_pool_create": (_I32, [_I32, _PI32, ctypes.POINTER(_P)]),
@@ -199,6 +200,22 @@ def decode(q, cache: KVCache, block_tables, context_lens, max_context_len: int, 
         _check(lib().pa_decode(*args), "pa_decode")
     else:
         _check(lib().pa_decode_stage(int(stage), *args), f"pa_decode_stage({stage})")
+
+
+NO_ALLOC_WORKSPACE_BYTES = 16 << 20
+
+
+def decode_no_alloc(q, cache: KVCache, block_tables, context_lens, max_context_len: int, scale: float, out,
+                    stream=None) -> None:
+    """pa_decode without a caller workspace: for callers that may not allocate device
+    memory. The split-K scratch is a fixed 16 MiB array inside the library, shared by
+    every call on a device (serialise calls that could overlap); sizes needing more
+    raise PaError(PA_ERR_ARG)."""
+    S, Hq, _ = q.shape
+    st = lib().pa_decode_no_alloc(_ptr(q), dtype_code(q), S, Hq, ctypes.byref(cache.desc), _ptr(block_tables),
+                                  block_tables.shape[1], _ptr(context_lens), int(max_context_len), float(scale),
+                                  _ptr(out), _stream(stream))
+    _check(st, "pa_decode_no_alloc")
 
 
 def block_table_update(updates, block_tables, stream=None) -> None:

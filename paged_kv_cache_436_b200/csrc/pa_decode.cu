@@ -620,6 +620,41 @@ pa_status decode_impl(int stage_mask, const void* q, int32_t q_dtype, int32_t nu
   return PA_OK;
 }
 
+// ---------------------------------------------------------------------------
+// Allocation-free decode: the workspace lives in a fixed device array
+// ---------------------------------------------------------------------------
+// Some callers may not allocate device memory at all: a plugin running inside a
+// host framework that owns every device byte through its own caching allocator
+// (a raw cudaMalloc would bypass that allocator's accounting, and cudaFree
+// synchronises the whole device), or a latency-critical serving loop that forbids
+// allocation calls because they can stall other streams. For them
+// pa_decode_no_alloc uses this array as its workspace. It is part of the
+// library's device image, so every GPU that loads the library holds these
+// PA_NO_ALLOC_WORKSPACE_BYTES until the process exits.
+static __device__ __align__(256) unsigned char g_no_alloc_ws[PA_NO_ALLOC_WORKSPACE_BYTES];
+
+std::mutex g_no_alloc_mu;
+void* g_no_alloc_ptr[kMaxDevices];
+
+// Device address of g_no_alloc_ws on the current device. In host code the array's
+// name only stands in for the symbol, so the address is looked up once per device
+// (with that device current) and cached.
+cudaError_t no_alloc_workspace(void** ptr) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_no_alloc_mu);
+  if (!g_no_alloc_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_no_alloc_ws);
+    if (e != cudaSuccess) return e;
+    g_no_alloc_ptr[dev] = p;
+  }
+  *ptr = g_no_alloc_ptr[dev];
+  return cudaSuccess;
+}
+
 }  // namespace pa
 
 extern "C" {
@@ -668,6 +703,22 @@ pa_status pa_last_device_error(void* stream, int32_t* code, int32_t* info) {
     info[2] = host[3];
   }
   return host[0] ? PA_ERR_DEVICE_CHECK : PA_OK;
+}
+
+pa_status pa_decode_no_alloc(const void* q, int32_t q_dtype, int32_t num_seqs, int32_t num_q_heads,
+                             const pa_cache_desc* cache, const int32_t* block_tables,
+                             int32_t max_blocks_per_seq, const int32_t* context_lens,
+                             int32_t max_context_len, float scale, void* out, void* stream) {
+  if (!cache) return PA_ERR_ARG;
+  const size_t need = pa_decode_workspace_size(num_seqs, num_q_heads, cache->head_dim, max_context_len);
+  if (need == 0 || need > PA_NO_ALLOC_WORKSPACE_BYTES) return PA_ERR_ARG;
+  void* ws = nullptr;
+  if (pa::no_alloc_workspace(&ws) != cudaSuccess) return PA_ERR_CUDA;
+  // Nothing in the workspace has to start at zero: every call rewrites the plan
+  // and writes each partial result before reading it.
+  return pa::decode_impl(7, q, q_dtype, num_seqs, num_q_heads, cache, block_tables, max_blocks_per_seq,
+                         context_lens, max_context_len, scale, out, ws, PA_NO_ALLOC_WORKSPACE_BYTES,
+                         stream);
 }
 
 const char* pa_version(void) { return "libpa 0.1 (sm_100a)"; }
