@@ -151,7 +151,8 @@ pa_status pa_copy_blocks(const int64_t* src_dst_pairs, int32_t num_pairs,
  *                  for 16-bit caches q_dtype must equal kv_dtype.
  *   block_tables   device int32 [num_seqs][max_blocks_per_seq].
  *   context_lens   device int32 [num_seqs]; 0 gives an all-zero output row.
- *   max_context_len host upper bound of context_lens (sizes the partition grid).
+ *   max_context_len host upper bound of context_lens (sizes the partition grid);
+ *                  at most 6,291,456 (12288 partitions).
  *   scale          softmax scale (e.g. 1/sqrt(head_dim)).
  *   out            device [num_seqs][num_q_heads][head_dim] of q_dtype, rounded to
  *                  nearest even from binary32.

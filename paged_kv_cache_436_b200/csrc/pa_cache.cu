@@ -20,8 +20,8 @@
 
 namespace pa {
 
-// One CTA per token; threads stride over the token's Hkv * D elements in vectors
-// of 8 input elements (16 bytes).
+// grid (tokens, 2, chunks): y = 0 writes K, y = 1 writes V; each thread moves one
+// vector of 8 input elements (16 bytes) of the token's Hkv * D row.
 template <int KV, int IN>
 __global__ void __launch_bounds__(128) reshape_kernel(const uint8_t* __restrict__ k,
                                                       const uint8_t* __restrict__ v,
@@ -31,50 +31,50 @@ __global__ void __launch_bounds__(128) reshape_kernel(const uint8_t* __restrict_
                                                       int Hkv, int BS, int D, int num_blocks,
                                                       float k_scale, float v_scale) {
   using IT = typename Q<IN>::T;
-  const int t = blockIdx.x;
+  const int t = blockIdx.x, which = blockIdx.y;
+  const int i = blockIdx.z * blockDim.x + threadIdx.x;
+  const int nvec = Hkv * D / 8;
+  if (i >= nvec) return;
   const int64_t slot = slots[t];
   if (slot < 0) return;
   const int64_t limit = int64_t(num_blocks) * BS;
   if (slot >= limit) {
-    if (threadIdx.x == 0) record_error(PA_DEV_BAD_SLOT, t, int(slot > 0x7fffffff ? 0x7fffffff : slot), int(limit > 0x7fffffff ? 0x7fffffff : limit));
+    if (i == 0 && which == 0)
+      record_error(PA_DEV_BAD_SLOT, t, int(slot > 0x7fffffff ? 0x7fffffff : slot),
+                   int(limit > 0x7fffffff ? 0x7fffffff : limit));
     return;
   }
   const int64_t blk = slot / BS;
   const int off = int(slot - blk * BS);
   constexpr int EB = Kv<KV>::kBytes;
-  const int nvec = Hkv * D / 8;
-  for (int which = 0; which < 2; ++which) {
-    const uint8_t* src = (which ? v : k) + int64_t(t) * (which ? v_stride_bytes : k_stride_bytes);
-    uint8_t* dst_base = which ? vc : kc;
+  const uint8_t* src = (which ? v : k) + int64_t(t) * (which ? v_stride_bytes : k_stride_bytes);
+  uint8_t* dst_base = which ? vc : kc;
+  const int e0 = i * 8;
+  const int h = e0 / D, d = e0 - h * D;
+  const uint4 raw = *reinterpret_cast<const uint4*>(src + size_t(e0) * 2);
+  uint8_t* dst = dst_base + (((size_t(blk) * Hkv + h) * BS + off) * D + d) * EB;
+  if constexpr (KV != PA_E4M3) {
+    *reinterpret_cast<uint4*>(dst) = raw;
+  } else {
+    // x / scale in binary32 (round to nearest), then E4M3 round-to-nearest-even,
+    // saturating to +-448
     const float sc = which ? v_scale : k_scale;
-    for (int i = threadIdx.x; i < nvec; i += blockDim.x) {
-      const int e0 = i * 8;
-      const int h = e0 / D, d = e0 - h * D;
-      const uint4 raw = *reinterpret_cast<const uint4*>(src + size_t(e0) * 2);
-      uint8_t* dst = dst_base + (((size_t(blk) * Hkv + h) * BS + off) * D + d) * EB;
-      if constexpr (KV != PA_E4M3) {
-        *reinterpret_cast<uint4*>(dst) = raw;
-      } else {
-        // x / scale in binary32 (round to nearest), then E4M3 round-to-nearest-even,
-        // saturating to +-448
-        const IT* e = reinterpret_cast<const IT*>(&raw);
-        uint32_t packed[2];
+    const IT* e = reinterpret_cast<const IT*>(&raw);
+    uint32_t packed[2];
 #pragma unroll
-        for (int w = 0; w < 2; ++w) {
-          uint32_t word = 0;
+    for (int w = 0; w < 2; ++w) {
+      uint32_t word = 0;
 #pragma unroll
-          for (int pr = 0; pr < 2; ++pr) {
-            const float a = __fdiv_rn(Q<IN>::to_float(e[4 * w + 2 * pr]), sc);
-            const float b = __fdiv_rn(Q<IN>::to_float(e[4 * w + 2 * pr + 1]), sc);
-            const __nv_fp8x2_storage_t two =
-                __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
-            word |= uint32_t(two) << (16 * pr);
-          }
-          packed[w] = word;
-        }
-        *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
+      for (int pr = 0; pr < 2; ++pr) {
+        const float a = __fdiv_rn(Q<IN>::to_float(e[4 * w + 2 * pr]), sc);
+        const float b = __fdiv_rn(Q<IN>::to_float(e[4 * w + 2 * pr + 1]), sc);
+        const __nv_fp8x2_storage_t two =
+            __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+        word |= uint32_t(two) << (16 * pr);
       }
+      packed[w] = word;
     }
+    *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
   }
 }
 
@@ -137,7 +137,8 @@ pa_status pa_reshape_and_cache(const void* k, const void* v, int32_t in_dtype, i
   const auto* kb = static_cast<const uint8_t*>(k);
   const auto* vb = static_cast<const uint8_t*>(v);
   const int64_t ks = k_token_stride * 2, vs = v_token_stride * 2;
-  const dim3 grid(num_tokens), block(128);
+  const int nvec = c->num_kv_heads * c->head_dim / 8;
+  const dim3 grid(num_tokens, 2, (nvec + 127) / 128), block(128);
   if (c->kv_dtype == PA_F16)
     pa::reshape_kernel<PA_F16, PA_F16><<<grid, block, 0, s>>>(kb, vb, ks, vs, slot_mapping, kc, vc, c->num_kv_heads,
                                                               c->block_size, c->head_dim, c->num_blocks, 1.f, 1.f);

@@ -116,10 +116,18 @@ struct Cfg {
   static constexpr int kIters = BS / kRPI;        // iterations per block
   static constexpr int kChunk = BS * kRow;        // one (block, kv head) chunk of K (or V)
   static constexpr int kStage = 2 * kChunk;       // K + V
-  static constexpr int kWarps = 4;
-  static constexpr int kStages = kStage >= 16384 ? 2 : (kStage >= 8192 ? 3 : 4);
-  static constexpr int kBPP = kPartitionTokens / BS;             // blocks per partition
-  static constexpr int kMaxPerWarp = (kBPP + kWarps - 1) / kWarps;
+  static constexpr int kBlocksPerPartition = kPartitionTokens / BS;
+  // each warp streams about 8 blocks of a partition: 4 warps for BS 16, 2 for BS 32
+  static constexpr int kWarps = kBlocksPerPartition / 8 < 2 ? 2 : (kBlocksPerPartition / 8 > 8 ? 8 : kBlocksPerPartition / 8);
+  // 2 stages of K+V per warp: with 8 KB stages, 3 CTAs of 4 warps (or 6 of 2) share an
+  // SM: 12 warps and 192 KB in flight per SM
+  static constexpr int kStages = kStage >= 8192 ? 2 : 4;
+  // the producer may run ahead into the warp's next unit. Measured on B200: +1-2 %
+  // for E4M3 (more work per byte: the pipeline must stay full), -2 % for 16-bit
+  // caches (already at the DRAM limit: more requests in flight only add queueing)
+  static constexpr bool kLookahead = (KV == PA_E4M3);
+  static constexpr int kThreads = kWarps * 32;
+  static constexpr int kMaxPerWarp = (kBlocksPerPartition + kWarps - 1) / kWarps;
   static constexpr int kStageBytes = kWarps * kStages * kStage;
   static constexpr int kBarBytes = kWarps * kStages * 8;
   static constexpr int kMergeFloats = kWarps * G * (D + 2);
@@ -129,12 +137,55 @@ struct Cfg {
   static_assert(kMaxPerWarp <= 32, "block ids per warp must fit the lanes");
 };
 
+// One work unit (sequence, kv head, partition) as one warp of the CTA sees it.
+struct Unit {
+  int u;                 // unit index; >= total when there is no unit
+  int s, hk, part;
+  int L, nparts, b0;     // context length, partitions of the sequence, first block
+  int mine;              // blocks of this unit this warp streams
+  int bid;               // lane i: physical block of the warp's i-th block (i < mine)
+};
+
+template <int BS, int NW>
+__device__ __forceinline__ Unit make_unit(const DecodeParams& p, int u, int total, int warp, int lane) {
+  constexpr int BPP = kPartitionTokens / BS;
+  Unit x;
+  x.u = u;
+  x.mine = 0;
+  x.bid = 0;
+  if (u >= total) return x;
+  const int pair = u / p.num_kv_heads;
+  x.hk = u - pair * p.num_kv_heads;
+  int lo = 0, hi = p.num_seqs;       // plan[lo] <= pair < plan[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (p.plan[mid] <= pair) lo = mid; else hi = mid;
+  }
+  x.s = lo;
+  x.part = pair - p.plan[lo];
+  x.L = clamp_len(p.context_lens[lo], p.len_limit);
+  x.nparts = (x.L + kPartitionTokens - 1) / kPartitionTokens;
+  x.b0 = x.part * BPP;
+  const int nblk = min(BPP, (x.L + BS - 1) / BS - x.b0);
+  x.mine = nblk > warp ? (nblk - warp + NW - 1) / NW : 0;
+  if (lane < x.mine) {
+    const int lb = x.b0 + warp + lane * NW;
+    int v = p.block_tables[size_t(x.s) * p.max_blocks + lb];
+    if (v < 0 || v >= p.num_blocks) {
+      record_error(PA_DEV_BAD_BLOCK_ID, x.s, lb, v);
+      v = 0;
+    }
+    x.bid = v;
+  }
+  return x;
+}
+
 template <int QD, int KV, int D, int BS, int G>
-__global__ void __launch_bounds__(128) partition_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(Cfg<KV, D, BS, G>::kThreads) partition_kernel(const DecodeParams p) {
   using C = Cfg<KV, D, BS, G>;
   using QT = typename Q<QD>::T;
   constexpr int EPL = C::kEPL, LPR = C::kLPR, RPI = C::kRPI, IT = C::kIters;
-  constexpr int NS = C::kStages, NW = C::kWarps;
+  constexpr int NS = C::kStages, NW = C::kWarps, QV = EPL / 8;
 
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kStageBytes);
@@ -151,72 +202,70 @@ __global__ void __launch_bounds__(128) partition_kernel(const DecodeParams p) {
   __syncthreads();
 
   const int Hkv = p.num_kv_heads, Hq = p.num_q_heads;
-  const int total_units = p.plan[p.num_seqs] * Hkv;
+  const int total = p.plan[p.num_seqs] * Hkv;
   const uint64_t pol = l2_policy_evict_first();
   uint8_t* my_stage = smem + warp * NS * C::kStage;
   uint64_t* my_bar = bars + warp * NS;
-  uint32_t seq_no = 0;          // items this warp has consumed so far (all units)
+  const size_t block_stride = size_t(Hkv) * C::kChunk;
+
+  // The warp's blocks form one stream across its units: item g (a global count)
+  // lives in stage g % NS and completes phase (g / NS) & 1 of that stage's barrier.
+  // The producer (lane 0) keeps up to NS items in flight and runs ahead into the
+  // next unit, so a unit boundary does not drain the pipeline.
+  uint32_t consumed = 0;   // items consumed so far
+  uint32_t issued = 0;     // items issued so far
+  uint32_t base = 0;       // global number of cur's first item
   bool aborted = false;
 
-  for (int u = blockIdx.x; u < total_units; u += gridDim.x) {
-    // ---- unit -> (sequence, kv head, partition) -------------------------------
-    const int pair = u / Hkv, hk = u - pair * Hkv;
-    int lo = 0, hi = p.num_seqs;
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (p.plan[mid] <= pair) lo = mid; else hi = mid;
+  auto load_q = [&](const Unit& un, uint4 (&raw)[G][QV]) {
+    const QT* qp = static_cast<const QT*>(p.q) + (size_t(un.s) * Hq + size_t(un.hk) * G) * D + j * EPL;
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+      for (int v = 0; v < QV; ++v) raw[g][v] = *reinterpret_cast<const uint4*>(qp + size_t(g) * D + v * 8);
+  };
+  auto issue = [&](const Unit& un, int idx, uint32_t g) {
+    const int bid = __shfl_sync(kFull, un.bid, idx);
+    if (lane == 0) {
+      const int st = g % NS;
+      uint8_t* dst = my_stage + st * C::kStage;
+      mbar_arrive_expect_tx(&my_bar[st], C::kStage);
+      const size_t off = size_t(bid) * block_stride + size_t(un.hk) * C::kChunk;
+      bulk_g2s(dst, p.k_cache + off, C::kChunk, &my_bar[st], pol);
+      bulk_g2s(dst + C::kChunk, p.v_cache + off, C::kChunk, &my_bar[st], pol);
     }
-    const int s = lo, part = pair - p.plan[s];
-    const int L = clamp_len(p.context_lens[s], p.len_limit);
-    const int nparts = (L + kPartitionTokens - 1) / kPartitionTokens;
-    const int nblk_seq = (L + BS - 1) / BS;
-    const int b0 = part * C::kBPP;
-    const int nblk = min(C::kBPP, nblk_seq - b0);
-    const int mine = nblk > warp ? (nblk - warp + NW - 1) / NW : 0;
-
-    // this warp's block ids, one per lane, checked against the pool
-    int bid_reg = 0;
-    if (lane < mine) {
-      const int lb = b0 + warp + lane * NW;
-      int v = p.block_tables[size_t(s) * p.max_blocks + lb];
-      if (v < 0 || v >= p.num_blocks) {
-        record_error(PA_DEV_BAD_BLOCK_ID, s, lb, v);
-        v = 0;
-      }
-      bid_reg = v;
+  };
+  // issue every item whose stage is free: those of cur first, then of nxt
+  auto top_up = [&](const Unit& cur, const Unit& nxt) {
+    while (issued < consumed + NS) {
+      const int k = int(issued - base);
+      if (k < cur.mine) issue(cur, k, issued);
+      else if (C::kLookahead && k - cur.mine < nxt.mine) issue(nxt, k - cur.mine, issued);
+      else break;
+      ++issued;
     }
+  };
 
-    // q for the G heads of this kv head, pre-multiplied by scale * k_scale * log2 e
+  Unit cur = make_unit<BS, NW>(p, blockIdx.x, total, warp, lane);
+  uint4 qraw[G][QV];
+  if (cur.u < total) load_q(cur, qraw);
+
+  while (cur.u < total) {
+    const Unit nxt = make_unit<BS, NW>(p, cur.u + gridDim.x, total, warp, lane);
+    top_up(cur, nxt);
+    uint4 qraw_next[G][QV];
+    if (nxt.u < total) load_q(nxt, qraw_next);
+
+    // q of the G heads, binary32, pre-multiplied by scale * k_scale * log2 e
     float qf[G][EPL];
-    {
-      const QT* qp = static_cast<const QT*>(p.q) + (size_t(s) * Hq + size_t(hk) * G) * D + j * EPL;
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
+    for (int g = 0; g < G; ++g)
 #pragma unroll
-        for (int v = 0; v < EPL / 8; ++v) {
-          const uint4 raw = *reinterpret_cast<const uint4*>(qp + size_t(g) * D + v * 8);
-          const QT* e = reinterpret_cast<const QT*>(&raw);
+      for (int v = 0; v < QV; ++v) {
+        const QT* e = reinterpret_cast<const QT*>(&qraw[g][v]);
 #pragma unroll
-          for (int t = 0; t < 8; ++t) qf[g][v * 8 + t] = Q<QD>::to_float(e[t]) * p.q_mul;
-        }
+        for (int x = 0; x < 8; ++x) qf[g][v * 8 + x] = Q<QD>::to_float(e[x]) * p.q_mul;
       }
-    }
-
-    const size_t head_off = size_t(hk) * C::kChunk;
-    const size_t block_stride = size_t(Hkv) * C::kChunk;
-    auto issue = [&](int i) {
-      const int bid = __shfl_sync(kFull, bid_reg, i);
-      if (lane == 0) {
-        const int st = (seq_no + i) % NS;
-        uint8_t* dst = my_stage + st * C::kStage;
-        mbar_arrive_expect_tx(&my_bar[st], C::kStage);
-        const size_t off = size_t(bid) * block_stride + head_off;
-        bulk_g2s(dst, p.k_cache + off, C::kChunk, &my_bar[st], pol);
-        bulk_g2s(dst + C::kChunk, p.v_cache + off, C::kChunk, &my_bar[st], pol);
-      }
-    };
-    const int pre = mine < NS ? mine : NS;
-    for (int i = 0; i < pre; ++i) issue(i);
 
     float m[G], l[G], acc[G][EPL];
 #pragma unroll
@@ -227,22 +276,19 @@ __global__ void __launch_bounds__(128) partition_kernel(const DecodeParams p) {
       for (int e = 0; e < EPL; ++e) acc[g][e] = 0.f;
     }
 
-    int consumed = 0;
-    for (int i = 0; i < mine && !aborted; ++i) {
-      const int n = seq_no + i;
+    for (int i = 0; i < cur.mine; ++i) {
+      const uint32_t n = consumed;
       const int st = n % NS;
-      const uint32_t parity = (n / NS) & 1;
-      const bool ok = mbar_wait_bounded(&my_bar[st], parity);
+      const bool ok = mbar_wait_bounded(&my_bar[st], (n / NS) & 1);
       if (!__all_sync(kFull, ok)) {
-        if (lane == 0) record_error(PA_DEV_WAIT_TIMEOUT, 1, u, st);
+        if (lane == 0) record_error(PA_DEV_WAIT_TIMEOUT, 1, cur.u, st);
         aborted = true;
         break;
       }
-      consumed = i + 1;
       const uint8_t* Ks = my_stage + st * C::kStage;
       const uint8_t* Vs = Ks + C::kChunk;
-      const int lb = b0 + warp + i * NW;
-      const int valid = min(BS, L - lb * BS);   // >= 1
+      const int lb = cur.b0 + warp + i * NW;
+      const int valid = min(BS, cur.L - lb * BS);   // >= 1
 
       // scores of this lane's rows for the G heads
       float sc[G][IT];
@@ -269,7 +315,8 @@ __global__ void __launch_bounds__(128) partition_kernel(const DecodeParams p) {
           if (it * RPI + r >= valid) sc[g][it] = -INFINITY;
         }
       }
-      // online softmax update (base 2)
+      // online softmax update (base 2); the accumulator is rescaled only when the
+      // running maximum moves (a warp-uniform branch)
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         float mx = sc[g][0];
@@ -277,18 +324,20 @@ __global__ void __launch_bounds__(128) partition_kernel(const DecodeParams p) {
         for (int it = 1; it < IT; ++it) mx = fmaxf(mx, sc[g][it]);
 #pragma unroll
         for (int off = LPR; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, off));
-        const float mnew = fmaxf(m[g], mx);
-        const float corr = exp2f(m[g] - mnew);
-        m[g] = mnew;
+        if (mx > m[g]) {
+          const float corr = exp2f(m[g] - mx);
+          m[g] = mx;
+          l[g] *= corr;
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) acc[g][e] *= corr;
+        }
         float ps = 0.f;
 #pragma unroll
         for (int it = 0; it < IT; ++it) {
-          sc[g][it] = exp2f(sc[g][it] - mnew);
+          sc[g][it] = exp2f(sc[g][it] - m[g]);
           ps += sc[g][it];
         }
-        l[g] = l[g] * corr + ps;
-#pragma unroll
-        for (int e = 0; e < EPL; ++e) acc[g][e] *= corr;
+        l[g] += ps;
       }
       // P . V over this lane's rows
 #pragma unroll
@@ -305,20 +354,13 @@ __global__ void __launch_bounds__(128) partition_kernel(const DecodeParams p) {
           }
         }
       }
-      __syncwarp();
-      if (i + NS < mine) issue(i + NS);
+      __syncwarp();          // every lane is done with this stage before it is refilled
+      ++consumed;
+      top_up(cur, nxt);
     }
-    if (aborted) {
-      // let the copies this warp still has in flight land before leaving
-      for (int i = consumed; i < mine && i < consumed + NS; ++i) {
-        const int n = seq_no + i;
-        mbar_wait_bounded(&my_bar[n % NS], (n / NS) & 1, 100000000ull);
-      }
-      if (lane == 0) s_abort = 1;
-    }
-    seq_no += mine;
+    if (aborted && lane == 0) s_abort = 1;
 
-    // combine the row groups of the warp, then stage the warp's state for the merge
+    // combine the warp's row groups, then stage the warp's state for the merge
 #pragma unroll
     for (int g = 0; g < G; ++g) {
 #pragma unroll
@@ -343,7 +385,7 @@ __global__ void __launch_bounds__(128) partition_kernel(const DecodeParams p) {
     __syncthreads();
 
     // merge the warps: out = sum_w acc_w 2^(m_w - M) / sum_w l_w 2^(m_w - M)
-    for (int idx = threadIdx.x; idx < G * D; idx += NW * 32) {
+    for (int idx = threadIdx.x; idx < G * D; idx += C::kThreads) {
       const int g = idx / D, d = idx - g * D;
       float M = -INFINITY;
 #pragma unroll
@@ -356,12 +398,12 @@ __global__ void __launch_bounds__(128) partition_kernel(const DecodeParams p) {
         ls += ww[1] * f;
         a += ww[2 + d] * f;
       }
-      const int h = hk * G + g;
-      if (nparts == 1) {
-        QT* o = static_cast<QT*>(p.out) + (size_t(s) * Hq + h) * D + d;
+      const int h = cur.hk * G + g;
+      if (cur.nparts == 1) {
+        QT* o = static_cast<QT*>(p.out) + (size_t(cur.s) * Hq + h) * D + d;
         *o = Q<QD>::from_float(a * p.v_scale / ls);
       } else {
-        const size_t slot = (size_t(s) * Hq + h) * p.max_parts + part;
+        const size_t slot = (size_t(cur.s) * Hq + h) * p.max_parts + cur.part;
         p.part_acc[slot * D + d] = a * p.v_scale;
         if (d == 0) {
           p.part_ml[slot * 2] = M;
@@ -371,57 +413,86 @@ __global__ void __launch_bounds__(128) partition_kernel(const DecodeParams p) {
     }
     __syncthreads();
     if (s_abort) break;
+    base += cur.mine;
+    cur = nxt;
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+      for (int v = 0; v < QV; ++v) qraw[g][v] = qraw_next[g][v];
   }
+  // leave no copy in flight into this CTA's shared memory (bounded waits)
+  for (uint32_t n = consumed; n < issued; ++n) mbar_wait_bounded(&my_bar[n % NS], (n / NS) & 1, 100000000ull);
 }
 
 // --------------------------------------------------------------------------
 // log-sum-exp merge of partitions
 // --------------------------------------------------------------------------
+// One CTA of D threads per (sequence, q head); thread d owns output dim d. The
+// partition weights 2^(m_p - M) go through shared memory, the P partial rows are
+// read coalesced (512 B per partition for D = 128) with independent loads.
 template <int QD, int D>
-__global__ void __launch_bounds__(256) reduce_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(D) reduce_kernel(const DecodeParams p) {
   using QT = typename Q<QD>::T;
-  constexpr int DPL = D / 32;   // dims per lane
-  const int gw = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-  if (gw >= p.num_seqs * p.num_q_heads) return;
-  const int s = gw / p.num_q_heads, h = gw - s * p.num_q_heads;
+  extern __shared__ float wsm[];             // [max_parts] weights
+  __shared__ float red[D / 32];
+  __shared__ float s_M, s_ls;
+  const int sh = blockIdx.x;
+  const int s = sh / p.num_q_heads;
   const int L = clamp_len(p.context_lens[s], p.len_limit);
   const int P = (L + kPartitionTokens - 1) / kPartitionTokens;
-  if (P <= 1) return;
-  const size_t base = (size_t(s) * p.num_q_heads + h) * p.max_parts;
+  if (P <= 1) return;                        // one partition: the partition kernel wrote out
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const size_t base = size_t(sh) * p.max_parts;
   const float* ml = p.part_ml + base * 2;
   float M = -INFINITY;
-  for (int i = lane; i < P; i += 32) M = fmaxf(M, ml[2 * i]);
+  for (int i = t; i < P; i += D) M = fmaxf(M, ml[2 * i]);
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, off));
+  if (lane == 0) red[warp] = M;
+  __syncthreads();
+  if (t == 0) {
+    float v = red[0];
+    for (int w = 1; w < D / 32; ++w) v = fmaxf(v, red[w]);
+    s_M = v;
+  }
+  __syncthreads();
+  M = s_M;
   float ls = 0.f;
-  for (int i = lane; i < P; i += 32) ls += ml[2 * i + 1] * exp2f(ml[2 * i] - M);
+  for (int i = t; i < P; i += D) {
+    const float w = exp2f(ml[2 * i] - M);
+    wsm[i] = w;
+    ls += ml[2 * i + 1] * w;
+  }
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) ls += __shfl_xor_sync(kFull, ls, off);
-  float a[DPL];
-#pragma unroll
-  for (int k = 0; k < DPL; ++k) a[k] = 0.f;
-  const float* accp = p.part_acc + base * D + lane * DPL;
-  for (int i = 0; i < P; ++i) {
-    const float w = exp2f(ml[2 * i] - M);
-    if constexpr (DPL == 4) {
-      const float4 v = *reinterpret_cast<const float4*>(accp + size_t(i) * D);
-      a[0] = fmaf(w, v.x, a[0]);
-      a[1] = fmaf(w, v.y, a[1]);
-      a[2] = fmaf(w, v.z, a[2]);
-      a[3] = fmaf(w, v.w, a[3]);
-    } else {
-#pragma unroll
-      for (int k = 0; k < DPL; ++k) a[k] = fmaf(w, accp[size_t(i) * D + k], a[k]);
-    }
+  __syncthreads();                           // red[] reuse and wsm[] ready
+  if (lane == 0) red[warp] = ls;
+  __syncthreads();
+  if (t == 0) {
+    float v = 0.f;
+    for (int w = 0; w < D / 32; ++w) v += red[w];
+    s_ls = v;
   }
-  QT* o = static_cast<QT*>(p.out) + (size_t(s) * p.num_q_heads + h) * D + lane * DPL;
-#pragma unroll
-  for (int k = 0; k < DPL; ++k) o[k] = Q<QD>::from_float(a[k] / ls);
+  __syncthreads();
+  const float* accp = p.part_acc + base * D + t;
+  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+  int i = 0;
+  for (; i + 4 <= P; i += 4) {
+    a0 = fmaf(wsm[i], accp[size_t(i) * D], a0);
+    a1 = fmaf(wsm[i + 1], accp[size_t(i + 1) * D], a1);
+    a2 = fmaf(wsm[i + 2], accp[size_t(i + 2) * D], a2);
+    a3 = fmaf(wsm[i + 3], accp[size_t(i + 3) * D], a3);
+  }
+  for (; i < P; ++i) a0 = fmaf(wsm[i], accp[size_t(i) * D], a0);
+  QT* o = static_cast<QT*>(p.out) + size_t(sh) * D + t;
+  *o = Q<QD>::from_float(((a0 + a1) + (a2 + a3)) / s_ls);
 }
 
 // --------------------------------------------------------------------------
 // host side
 // --------------------------------------------------------------------------
+constexpr int kMaxPartitions = 12288;   // max_context_len <= 12288 * 512 = 6,291,456 tokens
+
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct WsLayout {
@@ -442,6 +513,7 @@ using KernelFn = void (*)(const DecodeParams);
 struct Launch {
   KernelFn fn = nullptr;
   int smem = 0;
+  int threads = 0;
 };
 
 template <int QD, int KV, int D, int BS, int G>
@@ -449,6 +521,7 @@ Launch get_partition() {
   Launch l;
   l.fn = partition_kernel<QD, KV, D, BS, G>;
   l.smem = Cfg<KV, D, BS, G>::kSmem;
+  l.threads = Cfg<KV, D, BS, G>::kThreads;
   return l;
 }
 
@@ -526,7 +599,7 @@ cudaError_t occupancy(const Launch& l, int* grid_cap) {
   e = cudaFuncSetAttribute(l.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, l.smem);
   if (e != cudaSuccess) return e;
   int blocks = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, l.fn, 128, l.smem);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, l.fn, l.threads, l.smem);
   if (e != cudaSuccess) return e;
   if (blocks < 1) blocks = 1;
   if (g_occ_n[dev] < 128) g_occ[dev][g_occ_n[dev]++] = OccEntry{l.fn, blocks};
@@ -570,6 +643,7 @@ pa_status decode_impl(int stage_mask, const void* q, int32_t q_dtype, int32_t nu
   if (!aligned16(q) || !aligned16(out) || (reinterpret_cast<uintptr_t>(workspace) & 255)) return PA_ERR_ARG;
   const int D = c->head_dim, BS = c->block_size;
   const int max_parts = max_context_len > 0 ? (max_context_len + kPartitionTokens - 1) / kPartitionTokens : 1;
+  if (max_parts > kMaxPartitions) return PA_ERR_ARG;   // merge weights live in 48 KB of smem
   const WsLayout ws = ws_layout(num_seqs, num_q_heads, D, max_parts);
   if (workspace_bytes < ws.total) return PA_ERR_ARG;
   const Launch part = pick_partition(q_dtype, c->kv_dtype, D, BS, G);
@@ -608,13 +682,12 @@ pa_status decode_impl(int stage_mask, const void* q, int32_t q_dtype, int32_t nu
     if (occupancy(part, &cap) != cudaSuccess) return PA_ERR_CUDA;
     const long long units = (long long)num_seqs * c->num_kv_heads * max_parts;
     const int grid = int(units < cap ? units : cap);
-    part.fn<<<grid, 128, part.smem, s>>>(p);
+    part.fn<<<grid, part.threads, part.smem, s>>>(p);
     if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
   }
   if ((stage_mask & 4) && max_parts > 1) {
-    const long long warps = (long long)num_seqs * num_q_heads;
-    const int grid = int((warps + 7) / 8);
-    pick_reduce(q_dtype, D)<<<grid, 256, 0, s>>>(p);
+    const long long rows = (long long)num_seqs * num_q_heads;
+    pick_reduce(q_dtype, D)<<<unsigned(rows), D, size_t(max_parts) * 4, s>>>(p);
     if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
   }
   return PA_OK;
