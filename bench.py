@@ -319,26 +319,30 @@ def time_ours(w, steps, warmup, device, dist, e2e=True, clocks=True, local_rank=
            "kernel_ms_mean": float(np.mean(kernel_ms)), "kernel_bytes_mean": float(np.mean(kbytes)),
            "clocks": clk, "num_cow": eng.last_num_cow}
     if e2e:
-        S, Hq, Hkv, D = w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim
+        # the same steps through the host-buffer API: pinned inputs copied in and the
+        # output copied out every step, overlapped with the kernels of adjacent steps
+        from paged_kv_cache_436_b200.engine import HostPipeline
         q0, k0, v0 = run.inputs[0]
-        host = (q0.cpu().pin_memory(), k0.cpu().pin_memory(), v0.cpu().pin_memory(),
-                torch.empty_like(run.out, device="cpu").pin_memory(),
-                torch.empty_like(q0), torch.empty_like(k0), torch.empty_like(v0))
+        hq, hk, hv = q0.cpu().pin_memory(), k0.cpu().pin_memory(), v0.cpu().pin_memory()
+        hout = [torch.empty_like(run.out, device="cpu").pin_memory() for _ in range(2)]
+        pipe = HostPipeline(eng, w.scale)
         for i in range(warmup):
-            run.step(i, host=host)
-        torch.cuda.synchronize(device)
+            pipe.submit(hq, hk, hv, hout[i & 1])
+        pipe.sync()
         barrier(dist, device)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         eb = 0
-        e0.record()
+        e0.record(pipe.compute)
+        pipe.h2d.wait_event(e0)
         for i in range(n_e2e):
-            nb, _ = run.step(i, host=host)
-            eb += nb
-        e1.record()
-        torch.cuda.synchronize(device)
+            pipe.submit(hq, hk, hv, hout[i & 1])
+            eb += decode_bytes(eng.lens, w.num_kv_heads, w.num_q_heads, w.head_dim, run.kv_bytes,
+                               run.q_bytes, w.block_size)
+        e1.record(pipe.d2h)
+        pipe.sync()
         ems = reduce_max(e0.elapsed_time(e1), dist, device)
-        h2d = sum(t.numel() * t.element_size() for t in host[:3]) + eng._meta_bytes
-        d2h = host[3].numel() * host[3].element_size()
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv)) + eng._meta_bytes
+        d2h = hout[0].numel() * hout[0].element_size()
         res["e2e"] = {"ms_total": ems, "bytes": eb, "h2d": h2d, "d2h": d2h, "steps": n_e2e}
     del eng, run
     torch.cuda.empty_cache()

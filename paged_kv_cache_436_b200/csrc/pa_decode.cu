@@ -60,6 +60,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const DecodeParams p) {
   __shared__ int warp_tot[32];
   __shared__ int carry;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  grid_dependency_launch_dependents();       // the partition kernel may be scheduled now
   if (threadIdx.x == 0) carry = 0;
   __syncthreads();
   for (int base = 0; base < p.num_seqs; base += blockDim.x) {
@@ -200,6 +201,8 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, G>::kThreads) partition_kernel(
     fence_mbar_init();
   }
   __syncthreads();
+  grid_dependency_launch_dependents();       // the merge kernel may be scheduled early
+  grid_dependency_wait();                    // the plan (and all earlier work) is complete
 
   const int Hkv = p.num_kv_heads, Hq = p.num_q_heads;
   const int total = p.plan[p.num_seqs] * Hkv;
@@ -427,38 +430,45 @@ __global__ void __launch_bounds__(Cfg<KV, D, BS, G>::kThreads) partition_kernel(
 // --------------------------------------------------------------------------
 // log-sum-exp merge of partitions
 // --------------------------------------------------------------------------
-// One CTA of D threads per (sequence, q head); thread d owns output dim d. The
-// partition weights 2^(m_p - M) go through shared memory, the P partial rows are
-// read coalesced (512 B per partition for D = 128) with independent loads.
+// One CTA of 4 warps per (sequence, q head); a row with one partition exits at once
+// (the partition kernel wrote its output). Warp w merges partitions w, w + 4, ...;
+// lane l owns D/32 consecutive output dims and keeps 8 partial rows in flight
+// (coalesced: a warp reads one 4 B * D row per partition). The weights 2^(m_p - M)
+// go through shared memory; the four warp sums meet in shared memory.
+constexpr int kMergeWarps = 4;
+
 template <int QD, int D>
-__global__ void __launch_bounds__(D) reduce_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(kMergeWarps * 32) reduce_kernel(const DecodeParams p) {
   using QT = typename Q<QD>::T;
+  constexpr int NT = kMergeWarps * 32, DPL = D / 32;
   extern __shared__ float wsm[];             // [max_parts] weights
-  __shared__ float red[D / 32];
-  __shared__ float s_M, s_ls;
+  __shared__ float red[kMergeWarps];
+  __shared__ float wsum[kMergeWarps][D];
+  __shared__ float s_M;
+  grid_dependency_wait();                    // partials of the partition kernel are complete
   const int sh = blockIdx.x;
   const int s = sh / p.num_q_heads;
   const int L = clamp_len(p.context_lens[s], p.len_limit);
   const int P = (L + kPartitionTokens - 1) / kPartitionTokens;
-  if (P <= 1) return;                        // one partition: the partition kernel wrote out
+  if (P <= 1) return;
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const size_t base = size_t(sh) * p.max_parts;
   const float* ml = p.part_ml + base * 2;
   float M = -INFINITY;
-  for (int i = t; i < P; i += D) M = fmaxf(M, ml[2 * i]);
+  for (int i = t; i < P; i += NT) M = fmaxf(M, ml[2 * i]);
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, off));
   if (lane == 0) red[warp] = M;
   __syncthreads();
   if (t == 0) {
     float v = red[0];
-    for (int w = 1; w < D / 32; ++w) v = fmaxf(v, red[w]);
+    for (int w = 1; w < kMergeWarps; ++w) v = fmaxf(v, red[w]);
     s_M = v;
   }
   __syncthreads();
   M = s_M;
   float ls = 0.f;
-  for (int i = t; i < P; i += D) {
+  for (int i = t; i < P; i += NT) {
     const float w = exp2f(ml[2 * i] - M);
     wsm[i] = w;
     ls += ml[2 * i + 1] * w;
@@ -467,25 +477,45 @@ __global__ void __launch_bounds__(D) reduce_kernel(const DecodeParams p) {
   for (int off = 16; off >= 1; off >>= 1) ls += __shfl_xor_sync(kFull, ls, off);
   __syncthreads();                           // red[] reuse and wsm[] ready
   if (lane == 0) red[warp] = ls;
-  __syncthreads();
-  if (t == 0) {
-    float v = 0.f;
-    for (int w = 0; w < D / 32; ++w) v += red[w];
-    s_ls = v;
+  const float* accp = p.part_acc + base * D + lane * DPL;
+  float a[DPL];
+#pragma unroll
+  for (int k = 0; k < DPL; ++k) a[k] = 0.f;
+  int i = warp;
+  for (; i + 7 * kMergeWarps < P; i += 8 * kMergeWarps) {
+    float x[8][DPL];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const float* src = accp + size_t(i + u * kMergeWarps) * D;
+      if constexpr (DPL == 4) {
+        const float4 v = *reinterpret_cast<const float4*>(src);
+        x[u][0] = v.x; x[u][1] = v.y; x[u][2] = v.z; x[u][3] = v.w;
+      } else {
+#pragma unroll
+        for (int k = 0; k < DPL; ++k) x[u][k] = src[k];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+#pragma unroll
+      for (int k = 0; k < DPL; ++k) a[k] = fmaf(wsm[i + u * kMergeWarps], x[u][k], a[k]);
   }
+  for (; i < P; i += kMergeWarps)
+#pragma unroll
+    for (int k = 0; k < DPL; ++k) a[k] = fmaf(wsm[i], accp[size_t(i) * D + k], a[k]);
+#pragma unroll
+  for (int k = 0; k < DPL; ++k) wsum[warp][lane * DPL + k] = a[k];
   __syncthreads();
-  const float* accp = p.part_acc + base * D + t;
-  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-  int i = 0;
-  for (; i + 4 <= P; i += 4) {
-    a0 = fmaf(wsm[i], accp[size_t(i) * D], a0);
-    a1 = fmaf(wsm[i + 1], accp[size_t(i + 1) * D], a1);
-    a2 = fmaf(wsm[i + 2], accp[size_t(i + 2) * D], a2);
-    a3 = fmaf(wsm[i + 3], accp[size_t(i + 3) * D], a3);
+  for (int d = t; d < D; d += NT) {
+    float tot = 0.f, lsum = 0.f;
+#pragma unroll
+    for (int w = 0; w < kMergeWarps; ++w) {
+      tot += wsum[w][d];
+      lsum += red[w];
+    }
+    QT* o = static_cast<QT*>(p.out) + size_t(sh) * D + d;
+    *o = Q<QD>::from_float(tot / lsum);
   }
-  for (; i < P; ++i) a0 = fmaf(wsm[i], accp[size_t(i) * D], a0);
-  QT* o = static_cast<QT*>(p.out) + size_t(sh) * D + t;
-  *o = Q<QD>::from_float(((a0 + a1) + (a2 + a3)) / s_ls);
 }
 
 // --------------------------------------------------------------------------
@@ -607,6 +637,25 @@ cudaError_t occupancy(const Launch& l, int* grid_cap) {
   return cudaSuccess;
 }
 
+// Launch a kernel that may start while the previous kernel on the stream finishes
+// (programmatic dependent launch). The kernel itself calls grid_dependency_wait()
+// before it touches anything the earlier work produced; since every kernel launched
+// this way waits on its predecessor, completion order stays transitive.
+cudaError_t launch_dependent(KernelFn fn, int grid, int threads, size_t smem, cudaStream_t s,
+                             const DecodeParams& p) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, fn, p);
+}
+
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 pa_status validate_cache(const pa_cache_desc* c) {
@@ -682,13 +731,13 @@ pa_status decode_impl(int stage_mask, const void* q, int32_t q_dtype, int32_t nu
     if (occupancy(part, &cap) != cudaSuccess) return PA_ERR_CUDA;
     const long long units = (long long)num_seqs * c->num_kv_heads * max_parts;
     const int grid = int(units < cap ? units : cap);
-    part.fn<<<grid, part.threads, part.smem, s>>>(p);
-    if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+    if (launch_dependent(part.fn, grid, part.threads, part.smem, s, p) != cudaSuccess) return PA_ERR_CUDA;
   }
   if ((stage_mask & 4) && max_parts > 1) {
     const long long rows = (long long)num_seqs * num_q_heads;
-    pick_reduce(q_dtype, D)<<<unsigned(rows), D, size_t(max_parts) * 4, s>>>(p);
-    if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+    if (launch_dependent(pick_reduce(q_dtype, D), int(rows), kMergeWarps * 32, size_t(max_parts) * 4, s, p) !=
+        cudaSuccess)
+      return PA_ERR_CUDA;
   }
   return PA_OK;
 }

@@ -129,3 +129,60 @@ class DecodeEngine:
         """pa_decode alone over the current device tables and lengths."""
         decode(q, self.cache, self.bt_dev, self.lens_dev, self.max_context_len, scale, out, self.ws,
                stream, stage=stage)
+
+
+class HostPipeline:
+    """Decode steps whose inputs and outputs live in pinned host memory.
+
+    Each step copies its q and new K/V rows host->device and its output
+    device->host, every step. The copies run on their own streams (one per
+    direction) into double-buffered device tensors, ordered by events, so the
+    copies of step i+1 / i-1 overlap the kernels of step i. The caller must not
+    modify a step's host inputs, or read its host output, before ``sync()``.
+    """
+
+    def __init__(self, engine: DecodeEngine, scale: float):
+        self.eng, self.scale = engine, scale
+        dev = engine.device
+        S, Hq, Hkv, D = engine.S, engine.Hq, engine.Hkv, engine.D
+        qt = _TORCH[engine.q_dtype]
+        self.dq = [torch.empty((S, Hq, D), dtype=qt, device=dev) for _ in range(2)]
+        self.dk = [torch.empty((S, Hkv, D), dtype=qt, device=dev) for _ in range(2)]
+        self.dv = [torch.empty((S, Hkv, D), dtype=qt, device=dev) for _ in range(2)]
+        self.dout = [torch.empty((S, Hq, D), dtype=qt, device=dev) for _ in range(2)]
+        self.compute = torch.cuda.current_stream(dev)
+        self.h2d = torch.cuda.Stream(dev)
+        self.d2h = torch.cuda.Stream(dev)
+        self.free_in = [None, None]     # step that last read buffer b has finished
+        self.free_out = [None, None]    # the output copy that last read dout[b] has finished
+        self.n = 0
+
+    def submit(self, hq, hk, hv, hout):
+        b = self.n & 1
+        self.n += 1
+        with torch.cuda.stream(self.h2d):
+            if self.free_in[b] is not None:
+                self.h2d.wait_event(self.free_in[b])
+            self.dq[b].copy_(hq, non_blocking=True)
+            self.dk[b].copy_(hk, non_blocking=True)
+            self.dv[b].copy_(hv, non_blocking=True)
+            landed = torch.cuda.Event()
+            landed.record(self.h2d)
+        self.compute.wait_event(landed)
+        if self.free_out[b] is not None:
+            self.compute.wait_event(self.free_out[b])
+        self.eng.step(self.dq[b], self.dk[b], self.dv[b], self.dout[b], self.scale, stream=self.compute)
+        done = torch.cuda.Event()
+        done.record(self.compute)
+        self.free_in[b] = done
+        with torch.cuda.stream(self.d2h):
+            self.d2h.wait_event(done)
+            hout.copy_(self.dout[b], non_blocking=True)
+            copied = torch.cuda.Event()
+            copied.record(self.d2h)
+        self.free_out[b] = copied
+        return copied
+
+    def sync(self):
+        self.d2h.synchronize()
+        self.compute.synchronize()
