@@ -207,7 +207,7 @@ def build_engine(w, growth, device):
                        head_dim=w.head_dim, block_size=w.block_size, kv_dtype=w.kv_dtype, q_dtype=w.q_dtype,
                        num_blocks=w.num_blocks, initial_order=w.initial_order,
                        max_blocks_per_seq=w.max_blocks_per_seq(growth),
-                       max_context_len=w.max_context_len + growth, device=device)
+                       max_context_len=w.max_context_len + growth, scale=w.scale, device=device)
     if w.kv_dtype == "e4m3":
         kc, ks = synthetic.normal_e4m3_codes(tuple(eng.k_cache.shape), w.seed * 10 + 1, device)
         eng.k_cache.copy_(kc)
@@ -219,8 +219,23 @@ def build_engine(w, growth, device):
     else:
         synthetic.fill_normal_(eng.k_cache, w.kv_dtype, w.seed * 10 + 1)
         synthetic.fill_normal_(eng.v_cache, w.kv_dtype, w.seed * 10 + 2)
-    for s, L in enumerate(w.context_lens):
-        eng.extend(s, L - 1)
+    if w.prefix_len:
+        # one sequence holds the shared prefix, the others fork it; each then takes
+        # its private tokens but the last (copy-on-write of the shared partial block)
+        import paged_kv_cache_436_b200 as pa
+        eng.extend(0, w.prefix_len)
+        for s in range(1, w.num_seqs):
+            eng.fork(0, s)
+        pairs = []
+        for s, priv in enumerate(w.private_lens):
+            cs, cd = eng.extend(s, priv - 1)
+            if cs >= 0:
+                pairs.append((cs, cd))
+        if pairs:
+            pa.copy_blocks(torch.tensor(pairs, dtype=torch.int64, device=device), eng.cache)
+    else:
+        for s, L in enumerate(w.context_lens):
+            eng.extend(s, L - 1)
     eng.upload_tables()
     torch.cuda.synchronize(device)
     return eng
@@ -244,42 +259,14 @@ class StepRunner:
         self.kv_bytes = 1 if w.kv_dtype == "e4m3" else 2
         self.q_bytes = 2
 
-    def step(self, i, ev_pair=None, host=None):
-        """One step. Returns (decode bytes, kernel launches). With `host`, the step's
-        q/k/v come from pinned host buffers and `out` goes back to a pinned buffer."""
-        pa, eng, w = self.pa, self.eng, self.w
-        if host is None:
-            q, k, v = self.inputs[i % len(self.inputs)]
-        else:
-            hq, hk, hv, hout, dq, dk, dv = host
-            dq.copy_(hq, non_blocking=True)
-            dk.copy_(hk, non_blocking=True)
-            dv.copy_(hv, non_blocking=True)
-            q, k, v = dq, dk, dv
-        slots, cows, lens, upd = eng.bookkeeping()
-        launches = 0
-        if upd.shape[0]:
-            pa.block_table_update(upd, eng.bt_dev)
-            launches += 1
-        if cows.shape[0]:
-            pa.copy_blocks(cows, eng.cache)
-            launches += 1
-        pa.reshape_and_cache(k, v, slots, eng.cache)
-        eng.lens_dev = lens
-        launches += 1
-        eng.run_decode(q, self.out, w.scale, stage=0)
-        if ev_pair is not None:
-            ev_pair[0].record(self.stream)
-        eng.run_decode(q, self.out, w.scale, stage=1)
-        if ev_pair is not None:
-            ev_pair[1].record(self.stream)
-        eng.run_decode(q, self.out, w.scale, stage=2)
-        launches += 3 if eng.max_context_len > 512 else 2
-        if host is not None:
-            hout.copy_(self.out, non_blocking=True)
-        nbytes = decode_bytes(eng.lens, w.num_kv_heads, w.num_q_heads, w.head_dim, self.kv_bytes,
-                              self.q_bytes, w.block_size)
-        return nbytes, launches
+    def step(self, i, ev_pair=None):
+        """One native engine step on device-resident inputs; CUDA events around the
+        partition kernel. Returns (decode bytes, kernel launches)."""
+        q, k, v = self.inputs[i % len(self.inputs)]
+        self.eng.step(q, k, v, self.out, events=ev_pair)
+        nbytes = decode_bytes(self.eng.lens, self.w.num_kv_heads, self.w.num_q_heads, self.w.head_dim,
+                              self.kv_bytes, self.q_bytes, self.w.block_size)
+        return nbytes, self.eng.last_step()[2]
 
 
 def time_ours(w, steps, warmup, device, dist, e2e=True, clocks=True, local_rank=0):
@@ -297,6 +284,9 @@ def time_ours(w, steps, warmup, device, dist, e2e=True, clocks=True, local_rank=
         sampler.start()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for a, b in kev:            # torch creates the CUDA events at their first record
+        a.record()
+        b.record()
     torch.cuda.synchronize(device)
     barrier(dist, device)
     total_bytes, launches, lens_sum, kbytes = 0, 0, 0, []
@@ -317,7 +307,7 @@ def time_ours(w, steps, warmup, device, dist, e2e=True, clocks=True, local_rank=
     ms_max = reduce_max(ms, dist, device)
     res = {"ms_total": ms_max, "bytes": total_bytes, "launches": launches, "seq_tokens": lens_sum,
            "kernel_ms_mean": float(np.mean(kernel_ms)), "kernel_bytes_mean": float(np.mean(kbytes)),
-           "clocks": clk, "num_cow": eng.last_num_cow}
+           "clocks": clk, "num_cow": eng.last_step()[0]}
     if e2e:
         # the same steps through the host-buffer API: pinned inputs copied in and the
         # output copied out every step, overlapped with the kernels of adjacent steps
@@ -325,7 +315,7 @@ def time_ours(w, steps, warmup, device, dist, e2e=True, clocks=True, local_rank=
         q0, k0, v0 = run.inputs[0]
         hq, hk, hv = q0.cpu().pin_memory(), k0.cpu().pin_memory(), v0.cpu().pin_memory()
         hout = [torch.empty_like(run.out, device="cpu").pin_memory() for _ in range(2)]
-        pipe = HostPipeline(eng, w.scale)
+        pipe = HostPipeline(eng)
         for i in range(warmup):
             pipe.submit(hq, hk, hv, hout[i & 1])
         pipe.sync()
@@ -341,7 +331,7 @@ def time_ours(w, steps, warmup, device, dist, e2e=True, clocks=True, local_rank=
         e1.record(pipe.d2h)
         pipe.sync()
         ems = reduce_max(e0.elapsed_time(e1), dist, device)
-        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv)) + eng._meta_bytes
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv)) + eng.meta_bytes
         d2h = hout[0].numel() * hout[0].element_size()
         res["e2e"] = {"ms_total": ems, "bytes": eb, "h2d": h2d, "d2h": d2h, "steps": n_e2e}
     del eng, run
@@ -490,13 +480,13 @@ def main(argv=None):
     try:
         res = time_ours(w, args.steps, args.warmup, device, dist, e2e=not args.no_e2e,
                         clocks=True, local_rank=local)
-        also = None
-        if args.also:
-            wa = synthetic.make(args.also)
+        also = []
+        for name in [a for a in args.also.split(",") if a]:
+            wa = synthetic.make(name)
             if args.subset:
                 wa = synthetic.subset(wa, max(1, args.subset * wa.num_seqs // 256))
-            also = time_ours(wa, args.steps, args.warmup, device, dist, e2e=False, clocks=False,
-                             local_rank=local)
+            also.append((wa, time_ours(wa, args.steps, args.warmup, device, dist, e2e=False, clocks=False,
+                                       local_rank=local)))
         peak, peak_src = peaks()
         all_bytes = reduce_sum(res["bytes"], dist, device)
         value = all_bytes / (res["ms_total"] / 1e3) / 1e9
@@ -523,17 +513,19 @@ def main(argv=None):
             line["e2e"] = {"value": reduce_sum(e["bytes"], dist, device) / (e["ms_total"] / 1e3) / 1e9,
                            "unit": "GB/s", "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"],
                            "ms_per_step": e["ms_total"] / e["steps"]}
-        if also is not None:
-            line["also"] = {"workload": args.also,
-                            "value": reduce_sum(also["bytes"], dist, device) / (also["ms_total"] / 1e3) / 1e9,
-                            "unit": "GB/s", "ms_per_step": also["ms_total"] / args.steps,
-                            "seq_tokens_per_s": reduce_sum(also["seq_tokens"], dist, device) / (also["ms_total"] / 1e3),
-                            "roofline": {"bound": "hbm",
-                                         "achieved": also["kernel_bytes_mean"] / (also["kernel_ms_mean"] / 1e3) / 1e9,
-                                         "peak": peak, "unit": "GB/s",
-                                         "frac": also["kernel_bytes_mean"] / (also["kernel_ms_mean"] / 1e3) / 1e9 / peak,
-                                         "ms_per_launch": also["kernel_ms_mean"],
-                                         "traffic": kernel_traffic(wa.name, also["kernel_bytes_mean"])}}
+        for wa, ra in also:
+            kg = ra["kernel_bytes_mean"] / (ra["kernel_ms_mean"] / 1e3) / 1e9
+            entry = {"workload": wa.name,
+                     "value": reduce_sum(ra["bytes"], dist, device) / (ra["ms_total"] / 1e3) / 1e9,
+                     "unit": "GB/s", "ms_per_step": ra["ms_total"] / args.steps,
+                     "seq_tokens_per_s": reduce_sum(ra["seq_tokens"], dist, device) / (ra["ms_total"] / 1e3),
+                     "roofline": {"bound": "hbm", "achieved": kg, "peak": peak, "unit": "GB/s",
+                                  "frac": kg / peak, "ms_per_launch": ra["kernel_ms_mean"],
+                                  "traffic": kernel_traffic(wa.name, ra["kernel_bytes_mean"])}}
+            if wa.prefix_len:
+                entry["note"] = ("logical bytes: the shared prefix is counted once per sequence; "
+                                 "it is read from HBM about once and from L2 after that")
+            line.setdefault("also", []).append(entry)
         if rank == 0 and world == 1 and not args.no_cpu:
             line["cpu_baseline"] = cpu_baseline_obj(w, args.cpu_budget)
         if rank == 0:

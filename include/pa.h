@@ -306,6 +306,76 @@ pa_status pa_batch_append(pa_pool* pool, int32_t* block_tables, int32_t num_seqs
                           int64_t* cow_pairs, int32_t* num_cow, int32_t* updates,
                           int32_t* num_updates, int32_t* n_done);
 
+/* ------------------------------------------------------------------------- */
+/* Native decode step                                                         */
+/* ------------------------------------------------------------------------- */
+/*
+ * pa_engine -- one call per decode step: host bookkeeping for every sequence and
+ * the step's device work, with no interpreter in between (page 3, section
+ * "PagedAttention原理": blocks taken on demand, shared by reference count; page 2,
+ * section "2.2 关键数据结构剖析": block tables and context lengths reach the kernels as
+ * attention metadata). The engine owns two CUDA events and nothing else; every
+ * buffer below is the caller's and must outlive the engine.
+ *   pool                  the block pool (borrowed; not thread-safe, see above)
+ *   block_tables_host     host int32 [num_seqs][max_blocks_per_seq], the pool's tables
+ *   context_lens_host     host int32 [num_seqs]: tokens each sequence holds; a step
+ *                         appends one token to every sequence and increments them
+ *   block_tables_dev      device int32 [num_seqs][max_blocks_per_seq], the mirror the
+ *                         kernels read (patched every step with the updates)
+ *   meta_host[2]          two pinned host buffers of meta_bytes (double-buffered)
+ *   meta_dev              device buffer of meta_bytes, 16-byte aligned
+ *   meta_bytes            >= pa_engine_meta_bytes(num_seqs)
+ *   workspace             device scratch for pa_decode (>= pa_decode_workspace_size)
+ *   cache, q_dtype, num_q_heads, max_context_len, scale   as for pa_decode
+ */
+typedef struct {
+  pa_pool* pool;
+  int32_t num_seqs;
+  int32_t num_q_heads;
+  int32_t max_blocks_per_seq;
+  int32_t max_context_len;
+  int32_t q_dtype;
+  float scale;
+  pa_cache_desc cache;
+  int32_t* block_tables_host;
+  int32_t* context_lens_host;
+  int32_t* block_tables_dev;
+  void* meta_host[2];
+  void* meta_dev;
+  size_t meta_bytes;
+  void* workspace;
+  size_t workspace_bytes;
+} pa_engine_config;
+
+typedef struct pa_engine pa_engine;
+
+/* Bytes of one metadata buffer for num_seqs sequences (slots, copy pairs, lengths,
+ * table updates, each 16-byte aligned). */
+size_t pa_engine_meta_bytes(int32_t num_seqs);
+pa_status pa_engine_create(const pa_engine_config* config, pa_engine** out);
+void pa_engine_destroy(pa_engine* engine);
+
+/*
+ * pa_engine_step -- append one token to every sequence and decode:
+ *   1. pa_batch_append on the host (slots, copy-on-write pairs, table updates);
+ *   2. one cudaMemcpyAsync of the packed metadata (waits first, on the host, for the
+ *      copy of two steps ago that read the same pinned buffer);
+ *   3. pa_block_table_update, pa_copy_blocks (only when there are updates / pairs),
+ *      pa_reshape_and_cache of k_new / v_new, pa_decode.
+ *   q, out        device [num_seqs][num_q_heads][head_dim] of q_dtype
+ *   k_new, v_new  device [num_seqs][num_kv_heads][head_dim] of q_dtype, contiguous
+ *   ev_partition_begin / _end  optional cudaEvent_t (NULL = none), recorded on the
+ *                 stream right before and after the partition kernel (for timing it)
+ * On PA_ERR_OOM the sequences before the failing one have been appended (their
+ * context_lens_host entries incremented) and nothing has been enqueued.
+ */
+pa_status pa_engine_step(pa_engine* engine, const void* q, const void* k_new, const void* v_new, void* out,
+                         void* stream, void* ev_partition_begin, void* ev_partition_end);
+
+/* Copy pairs, table updates and kernel launches of the last step. */
+pa_status pa_engine_last_step(const pa_engine* engine, int32_t* num_cow, int32_t* num_updates,
+                              int32_t* launches);
+
 /* Library version string and the device architecture it was built for. */
 const char* pa_version(void);
 

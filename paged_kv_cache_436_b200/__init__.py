@@ -44,6 +44,16 @@ class CacheDesc(ctypes.Structure):
                 ("v_cache", ctypes.c_void_p)]
 
 
+class EngineConfig(ctypes.Structure):
+    _fields_ = [("pool", ctypes.c_void_p), ("num_seqs", ctypes.c_int32), ("num_q_heads", ctypes.c_int32),
+                ("max_blocks_per_seq", ctypes.c_int32), ("max_context_len", ctypes.c_int32),
+                ("q_dtype", ctypes.c_int32), ("scale", ctypes.c_float), ("cache", CacheDesc),
+                ("block_tables_host", ctypes.c_void_p), ("context_lens_host", ctypes.c_void_p),
+                ("block_tables_dev", ctypes.c_void_p), ("meta_host", ctypes.c_void_p * 2),
+                ("meta_dev", ctypes.c_void_p), ("meta_bytes", ctypes.c_size_t),
+                ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)]
+
+
 _lib = None
 
 _P = ctypes.c_void_p
@@ -79,6 +89,11 @@ _SIGNATURES = {
     "pa_seq_free": (_I32, [_P, _PI32, _I32]),
     "pa_batch_append": (_I32, [_P, _PI32, _I32, _I32, _PI32, _I32, _PI64, _PI64, _PI32, _PI32, _PI32,
                                _PI32]),
+    "pa_engine_meta_bytes": (ctypes.c_size_t, [_I32]),
+    "pa_engine_create": (_I32, [ctypes.POINTER(EngineConfig), ctypes.POINTER(_P)]),
+    "pa_engine_destroy": (None, [_P]),
+    "pa_engine_step": (_I32, [_P, _P, _P, _P, _P, _P, _P, _P]),
+    "pa_engine_last_step": (_I32, [_P, _PI32, _PI32, _PI32]),
     "pa_version": (ctypes.c_char_p, []),
 }
 

@@ -1,41 +1,41 @@
 """One decode step of the paged-KV-cache path, end to end, on one GPU.
 
-A step, for a batch of S sequences that each append one token:
+A step appends one token to every sequence of the batch and decodes:
 
 1. host bookkeeping (C++ ``pa_batch_append``): the slot of each new token, a
    new block when a sequence crosses a block boundary, a copy-on-write pair when
    it appends into a shared block (page 3 «内存优化：KV Cache管理、PagedAttention原理与
    内存池配置», section "PagedAttention原理");
-2. one host->device copy of the step's metadata (slots, copy pairs, block-table
-   updates) from a pinned buffer; the block-table mirror is patched on the device
-   (``pa_block_table_update``) -- page 2 (untitled, first section "1. 为什么vLLM能
-   实现24倍推理加速"), section "2.2 关键数据结构剖析": block tables and context lengths
-   travel with the attention metadata;
-3. ``pa_copy_blocks`` for the copy-on-write pairs;
-4. ``pa_reshape_and_cache`` of the new tokens' K and V;
-5. ``pa_decode``.
+2. one host->device copy of the step's metadata from a pinned buffer (page 2,
+   untitled, first section "1. 为什么vLLM能实现24倍推理加速", section "2.2 关键数据结构
+   剖析": block tables and context lengths travel with the attention metadata);
+3. ``pa_block_table_update``, ``pa_copy_blocks``, ``pa_reshape_and_cache``,
+   ``pa_decode``.
 
-Every computation happens in libpa; this class only owns buffers and orders calls.
+All of it runs in one native call (``pa_engine_step``); this class owns the
+buffers the native engine borrows and the set-up helpers.
 """
 
 from __future__ import annotations
 
+import ctypes
+
 import numpy as np
 import torch
 
-from . import (KVCache, Pool, block_table_update, copy_blocks, decode, decode_workspace_size,
-               reshape_and_cache)
+from . import (EngineConfig, KVCache, Pool, _check, _stream, decode, decode_workspace_size, dtype_code, lib)
 
 _TORCH = {"f16": torch.float16, "bf16": torch.bfloat16}
 
 
 class DecodeEngine:
     def __init__(self, *, num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, kv_dtype,
-                 q_dtype, num_blocks, initial_order, max_blocks_per_seq, max_context_len,
+                 q_dtype, num_blocks, initial_order, max_blocks_per_seq, max_context_len, scale=None,
                  k_scale=1.0, v_scale=1.0, device="cuda", k_cache=None, v_cache=None):
         self.S, self.Hq, self.Hkv, self.D = num_seqs, num_q_heads, num_kv_heads, head_dim
         self.BS, self.kv_dtype, self.q_dtype = block_size, kv_dtype, q_dtype
         self.MB = max_blocks_per_seq
+        self.scale = float(scale) if scale is not None else 1.0 / float(np.sqrt(head_dim))
         self.device = torch.device(device)
         self.pool = Pool(num_blocks, initial_order)
         cache_t = torch.uint8 if kv_dtype == "e4m3" else _TORCH[kv_dtype]
@@ -50,17 +50,11 @@ class DecodeEngine:
         self.max_context_len = int(max_context_len)
         self.ws = torch.empty(decode_workspace_size(num_seqs, num_q_heads, head_dim, self.max_context_len),
                               dtype=torch.uint8, device=self.device)
-        # packed per-step metadata: slots (int64 S) | cow pairs (int64 2S) | lens (int32 S) | updates (int32 3S)
-        self._off_cow = 8 * num_seqs
-        self._off_lens = self._off_cow + 16 * num_seqs
-        self._off_upd = self._off_lens + 4 * num_seqs
-        self._meta_bytes = self._off_upd + 12 * num_seqs
-        self._meta_host = [torch.empty(self._meta_bytes, dtype=torch.uint8).pin_memory() for _ in range(2)]
-        self._meta_event = [None, None]
-        self._meta_dev = torch.empty(self._meta_bytes, dtype=torch.uint8, device=self.device)
-        self._flip = 0
-        self.last_num_cow = 0
-        self.last_num_updates = 0
+        self.meta_bytes = int(lib().pa_engine_meta_bytes(num_seqs))
+        self._meta_host = [torch.empty(self.meta_bytes, dtype=torch.uint8).pin_memory() for _ in range(2)]
+        self._meta_dev = torch.empty(self.meta_bytes, dtype=torch.uint8, device=self.device)
+        self._native = None
+        self._native_key = None
 
     # ------------------------------------------------------------------ set-up
     def extend(self, s: int, n_tokens: int, slots: np.ndarray | None = None):
@@ -83,52 +77,67 @@ class DecodeEngine:
         self.lens_dev.copy_(torch.from_numpy(self.lens))
 
     # ------------------------------------------------------------------ step
-    def bookkeeping(self, stream=None):
-        """Step parts 1-2: host bookkeeping for one token per sequence and the
-        metadata upload. Returns device views (slots, cow_pairs, updates)."""
-        i = self._flip
-        self._flip ^= 1
-        if self._meta_event[i] is not None:
-            self._meta_event[i].synchronize()      # the copy that last read this buffer is done
-        host = self._meta_host[i]
-        S = self.S
-        slots = host[:self._off_cow].view(torch.int64).numpy()
-        cows = host[self._off_cow:self._off_lens].view(torch.int64).numpy().reshape(S, 2)
-        lens = host[self._off_lens:self._off_upd].view(torch.int32).numpy()
-        upd = host[self._off_upd:].view(torch.int32).numpy().reshape(S, 3)
-        positions = self.lens.copy()
-        ncow, nupd = self.pool.batch_append(self.bt_host, positions, self.BS, slots, cows, upd)
-        self.lens += 1
-        lens[:] = self.lens
-        self.last_num_cow, self.last_num_updates = ncow, nupd
-        s = stream if stream is not None else torch.cuda.current_stream(self.device)
-        with torch.cuda.stream(s):
-            self._meta_dev.copy_(host, non_blocking=True)
-            ev = torch.cuda.Event()
-            ev.record(s)
-        self._meta_event[i] = ev
-        d = self._meta_dev
-        return (d[:self._off_cow].view(torch.int64),
-                d[self._off_cow:self._off_lens].view(torch.int64).view(S, 2)[:ncow],
-                d[self._off_lens:self._off_upd].view(torch.int32),
-                d[self._off_upd:].view(torch.int32).view(S, 3)[:nupd])
+    def _engine(self):
+        d = self.cache.desc
+        key = (self.scale, d.k_scale, d.v_scale)
+        if self._native is not None and self._native_key == key:
+            return self._native
+        self.close()
+        cfg = EngineConfig()
+        cfg.pool = self.pool._h
+        cfg.num_seqs, cfg.num_q_heads, cfg.max_blocks_per_seq = self.S, self.Hq, self.MB
+        cfg.max_context_len, cfg.q_dtype, cfg.scale = self.max_context_len, dtype_code(
+            torch.empty(0, dtype=_TORCH[self.q_dtype])), self.scale
+        cfg.cache = d
+        cfg.block_tables_host = self.bt_host.ctypes.data
+        cfg.context_lens_host = self.lens.ctypes.data
+        cfg.block_tables_dev = self.bt_dev.data_ptr()
+        cfg.meta_host[0], cfg.meta_host[1] = self._meta_host[0].data_ptr(), self._meta_host[1].data_ptr()
+        cfg.meta_dev, cfg.meta_bytes = self._meta_dev.data_ptr(), self.meta_bytes
+        cfg.workspace, cfg.workspace_bytes = self.ws.data_ptr(), self.ws.numel()
+        h = ctypes.c_void_p()
+        _check(lib().pa_engine_create(ctypes.byref(cfg), ctypes.byref(h)), "pa_engine_create")
+        self._native, self._native_key = h, key
+        return h
 
-    def step(self, q, k_new, v_new, out, scale: float, stream=None):
-        """One full decode step: bookkeeping, table patch, CoW copies, cache write, decode."""
-        slots, cows, lens, upd = self.bookkeeping(stream)
-        if upd.shape[0]:
-            block_table_update(upd, self.bt_dev, stream)
-        if cows.shape[0]:
-            copy_blocks(cows, self.cache, stream)
-        reshape_and_cache(k_new, v_new, slots, self.cache, stream)
-        self.lens_dev = lens
-        decode(q, self.cache, self.bt_dev, lens, self.max_context_len, scale, out, self.ws, stream)
+    def close(self):
+        if self._native is not None:
+            lib().pa_engine_destroy(self._native)
+            self._native = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def step(self, q, k_new, v_new, out, scale=None, stream=None, events=None):
+        """One full decode step (native): bookkeeping, metadata upload, table patch,
+        copy-on-write copies, cache write of k_new / v_new, decode into out.
+        `events` = (begin, end) torch.cuda.Events recorded around the partition kernel
+        (they must exist already: torch creates an event at its first record)."""
+        if scale is not None and float(scale) != self.scale:
+            raise ValueError("the softmax scale is fixed when the engine is created")
+        h = self._engine()
+        e0 = ctypes.c_void_p(events[0].cuda_event) if events else None
+        e1 = ctypes.c_void_p(events[1].cuda_event) if events else None
+        st = lib().pa_engine_step(h, ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k_new.data_ptr()),
+                                  ctypes.c_void_p(v_new.data_ptr()), ctypes.c_void_p(out.data_ptr()),
+                                  _stream(stream), e0, e1)
+        _check(st, "pa_engine_step")
         return out
 
-    def run_decode(self, q, out, scale: float, stream=None, stage=None):
-        """pa_decode alone over the current device tables and lengths."""
-        decode(q, self.cache, self.bt_dev, self.lens_dev, self.max_context_len, scale, out, self.ws,
-               stream, stage=stage)
+    def last_step(self):
+        """(copy pairs, table updates, kernel launches) of the last step."""
+        a, b, c = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+        _check(lib().pa_engine_last_step(self._native, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)),
+               "pa_engine_last_step")
+        return a.value, b.value, c.value
+
+    def run_decode(self, q, out, scale=None, stream=None, stage=None):
+        """pa_decode alone over the current device tables and `lens_dev`."""
+        decode(q, self.cache, self.bt_dev, self.lens_dev, self.max_context_len,
+               self.scale if scale is None else scale, out, self.ws, stream, stage=stage)
 
 
 class HostPipeline:
@@ -141,8 +150,8 @@ class HostPipeline:
     modify a step's host inputs, or read its host output, before ``sync()``.
     """
 
-    def __init__(self, engine: DecodeEngine, scale: float):
-        self.eng, self.scale = engine, scale
+    def __init__(self, engine: DecodeEngine, scale=None):
+        self.eng = engine
         dev = engine.device
         S, Hq, Hkv, D = engine.S, engine.Hq, engine.Hkv, engine.D
         qt = _TORCH[engine.q_dtype]
@@ -171,7 +180,7 @@ class HostPipeline:
         self.compute.wait_event(landed)
         if self.free_out[b] is not None:
             self.compute.wait_event(self.free_out[b])
-        self.eng.step(self.dq[b], self.dk[b], self.dv[b], self.dout[b], self.scale, stream=self.compute)
+        self.eng.step(self.dq[b], self.dk[b], self.dv[b], self.dout[b], stream=self.compute)
         done = torch.cuda.Event()
         done.record(self.compute)
         self.free_in[b] = done

@@ -45,7 +45,7 @@ def make_engine(w, device="cuda", growth=0, k_scale=1.0, v_scale=1.0):
     return DecodeEngine(num_seqs=w.num_seqs, num_q_heads=w.num_q_heads, num_kv_heads=w.num_kv_heads,
                         head_dim=w.head_dim, block_size=w.block_size, kv_dtype=w.kv_dtype,
                         q_dtype=w.q_dtype, num_blocks=w.num_blocks, initial_order=w.initial_order,
-                        max_blocks_per_seq=MB, max_context_len=w.max_context_len + growth,
+                        max_blocks_per_seq=MB, max_context_len=w.max_context_len + growth, scale=w.scale,
                         k_scale=k_scale, v_scale=v_scale, device=device)
 
 

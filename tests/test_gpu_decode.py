@@ -245,3 +245,24 @@ def test_host_pipeline_matches_device_steps():
         outs.append(res)
     for a, b in zip(*outs):
         assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_engine_step_out_of_blocks_reports_and_keeps_state_consistent():
+    """A step that runs out of blocks mid-batch returns PA_ERR_OOM; the sequences
+    before the failing one hold their new token, nothing is enqueued."""
+    w = synthetic.custom(3, 4, 4, 64, 16, "f16", "f16", [16, 16, 16], 84, pool_factor=1.0)
+    eng = make_engine(w, DEV, growth=16)
+    fill_cache(w, eng)
+    for s in range(3):
+        eng.extend(s, 16)                      # every sequence fills its block exactly
+    while eng.pool.num_free() > 1:             # leave one free block: only sequence 0 can grow
+        eng.pool.alloc()
+    eng.upload_tables()
+    q, k, v = (t.to(DEV) for t in synthetic.step_inputs(w, 0))
+    out = torch.zeros_like(q)
+    with pytest.raises(pa.PaError) as e:
+        eng.step(q, k, v, out, w.scale)
+    assert e.value.status == pa.PA_ERR_OOM
+    assert eng.lens.tolist() == [17, 16, 16] and eng.pool.num_free() == 0
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(out) == 0
