@@ -220,19 +220,26 @@ def build_engine(w, growth, device):
         synthetic.fill_normal_(eng.k_cache, w.kv_dtype, w.seed * 10 + 1)
         synthetic.fill_normal_(eng.v_cache, w.kv_dtype, w.seed * 10 + 2)
     if w.prefix_len:
-        # one sequence holds the shared prefix, the others fork it; each then takes
-        # its private tokens but the last (copy-on-write of the shared partial block)
+        # requests admitted through the prefix cache: all carry the same history, so
+        # every request after the first reuses its full blocks and allocates only its
+        # partial block and private tokens (the step appends each request's last token)
         import paged_kv_cache_436_b200 as pa
-        eng.extend(0, w.prefix_len)
-        for s in range(1, w.num_seqs):
-            eng.fork(0, s)
-        pairs = []
+        rng = np.random.default_rng(w.seed + 5)
+        hist = rng.integers(0, 32000, size=w.prefix_len).tolist()
+        cache = pa.PrefixCache(w.block_size)
+        t0 = time.perf_counter()
         for s, priv in enumerate(w.private_lens):
-            cs, cd = eng.extend(s, priv - 1)
-            if cs >= 0:
-                pairs.append((cs, cd))
-        if pairs:
-            pa.copy_blocks(torch.tensor(pairs, dtype=torch.int64, device=device), eng.cache)
+            prompt = hist + rng.integers(0, 32000, size=priv - 1).tolist()
+            n = cache.match(eng.pool, prompt, eng.bt_host[s])
+            eng.lens[s] = n * w.block_size
+            eng.extend(s, len(prompt) - n * w.block_size)
+            cache.insert(eng.pool, prompt, eng.bt_host[s])
+        eng.prefix_report = {"host_us_per_request": (time.perf_counter() - t0) / w.num_seqs * 1e6,
+                             "kv_blocks_held": w.num_blocks - eng.pool.num_free(),
+                             "kv_blocks_without_prefix_cache": int(sum(-(-(w.prefix_len + p - 1) // w.block_size)
+                                                                       for p in w.private_lens)),
+                             "cached_blocks": len(cache)}
+        eng.prefix_cache = cache
     else:
         for s, L in enumerate(w.context_lens):
             eng.extend(s, L - 1)
@@ -307,7 +314,8 @@ def time_ours(w, steps, warmup, device, dist, e2e=True, clocks=True, local_rank=
     ms_max = reduce_max(ms, dist, device)
     res = {"ms_total": ms_max, "bytes": total_bytes, "launches": launches, "seq_tokens": lens_sum,
            "kernel_ms_mean": float(np.mean(kernel_ms)), "kernel_bytes_mean": float(np.mean(kbytes)),
-           "clocks": clk, "num_cow": eng.last_step()[0]}
+           "clocks": clk, "num_cow": eng.last_step()[0],
+           "prefix_report": getattr(eng, "prefix_report", None)}
     if e2e:
         # the same steps through the host-buffer API: pinned inputs copied in and the
         # output copied out every step, overlapped with the kernels of adjacent steps
@@ -482,7 +490,15 @@ def main(argv=None):
                         clocks=True, local_rank=local)
         also = []
         for name in [a for a in args.also.split(",") if a]:
-            wa = synthetic.make(name)
+            if name == "gqa_noshare":
+                # the GQA-prefix shapes with every sequence holding its own blocks
+                g = synthetic.make("gqa_prefix")
+                wa = synthetic.custom(g.num_seqs, g.num_q_heads, g.num_kv_heads, g.head_dim, g.block_size,
+                                      g.kv_dtype, g.q_dtype, g.context_lens, g.seed, pool_factor=1.1,
+                                      scale=g.scale)
+                wa.name = "gqa_noshare"
+            else:
+                wa = synthetic.make(name)
             if args.subset:
                 wa = synthetic.subset(wa, max(1, args.subset * wa.num_seqs // 256))
             also.append((wa, time_ours(wa, args.steps, args.warmup, device, dist, e2e=False, clocks=False,
@@ -525,6 +541,7 @@ def main(argv=None):
             if wa.prefix_len:
                 entry["note"] = ("logical bytes: the shared prefix is counted once per sequence; "
                                  "it is read from HBM about once and from L2 after that")
+                entry["prefix_cache"] = ra.get("prefix_report")
             line.setdefault("also", []).append(entry)
         if rank == 0 and world == 1 and not args.no_cpu:
             line["cpu_baseline"] = cpu_baseline_obj(w, args.cpu_budget)

@@ -307,6 +307,39 @@ pa_status pa_batch_append(pa_pool* pool, int32_t* block_tables, int32_t num_seqs
                           int32_t* num_updates, int32_t* n_done);
 
 /* ------------------------------------------------------------------------- */
+/* Prefix cache (host)                                                        */
+/* ------------------------------------------------------------------------- */
+/*
+ * A host index from the token content of full KV blocks to the physical blocks that
+ * hold them (page 3, section "案例与场景": a global hash index over the KV blocks of a
+ * common prefix; a matching request reuses those blocks and allocates only for its
+ * new tokens; section "误区与复盘" (误区3): only exactly equal prefixes hit).
+ * Full block k of a prompt is reusable iff the prompt's tokens [0, (k+1)*BS) equal
+ * those of the sequence that filled the cached block. Keys chain a 64-bit FNV-1a hash
+ * over the previous block's key and the block's token ids; every hit is verified
+ * against the stored parent key and tokens, so a reuse is always exact. The index
+ * holds one pool reference on every block it lists. Not thread-safe.
+ */
+typedef struct pa_prefix_cache pa_prefix_cache;
+pa_status pa_prefix_cache_create(int32_t block_size, pa_prefix_cache** out);
+/* Frees the index only; call pa_prefix_cache_clear first to return its references. */
+void pa_prefix_cache_destroy(pa_prefix_cache* cache);
+int32_t pa_prefix_cache_size(const pa_prefix_cache* cache);
+/* Walks the prompt's full blocks in order; each hit takes a reference and is written
+ * to block_table_row[k]; stops at the first miss. *n_matched = blocks reused. */
+pa_status pa_prefix_cache_match(pa_prefix_cache* cache, pa_pool* pool, const int32_t* tokens, int32_t n_tokens,
+                                int32_t* block_table_row, int32_t max_blocks, int32_t* n_matched);
+/* Lists every full block of a sequence (tokens from position 0, blocks in
+ * block_table_row) that the index does not hold yet, taking a reference on each. */
+pa_status pa_prefix_cache_insert(pa_prefix_cache* cache, pa_pool* pool, const int32_t* tokens, int32_t n_tokens,
+                                 const int32_t* block_table_row, int32_t* n_inserted);
+/* Drops, oldest insertion first, up to max_blocks entries whose block only the index
+ * holds (refcount 1); those blocks return to the free list. */
+pa_status pa_prefix_cache_evict(pa_prefix_cache* cache, pa_pool* pool, int32_t max_blocks, int32_t* n_evicted);
+/* Drops every entry and its reference. */
+pa_status pa_prefix_cache_clear(pa_prefix_cache* cache, pa_pool* pool, int32_t* n_released);
+
+/* ------------------------------------------------------------------------- */
 /* Native decode step                                                         */
 /* ------------------------------------------------------------------------- */
 /*

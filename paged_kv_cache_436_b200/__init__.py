@@ -94,6 +94,13 @@ _SIGNATURES = {
     "pa_engine_destroy": (None, [_P]),
     "pa_engine_step": (_I32, [_P, _P, _P, _P, _P, _P, _P, _P]),
     "pa_engine_last_step": (_I32, [_P, _PI32, _PI32, _PI32]),
+    "pa_prefix_cache_create": (_I32, [_I32, ctypes.POINTER(_P)]),
+    "pa_prefix_cache_destroy": (None, [_P]),
+    "pa_prefix_cache_size": (_I32, [_P]),
+    "pa_prefix_cache_match": (_I32, [_P, _P, _PI32, _I32, _PI32, _I32, _PI32]),
+    "pa_prefix_cache_insert": (_I32, [_P, _P, _PI32, _I32, _PI32, _PI32]),
+    "pa_prefix_cache_evict": (_I32, [_P, _P, _I32, _PI32]),
+    "pa_prefix_cache_clear": (_I32, [_P, _P, _PI32]),
     "pa_version": (ctypes.c_char_p, []),
 }
 
@@ -332,6 +339,52 @@ class Pool:
                                    ctypes.byref(ncow), _i32p(updates), ctypes.byref(nupd), ctypes.byref(done))
         _check(st, "pa_batch_append")
         return ncow.value, nupd.value
+
+
+class PrefixCache:
+    """Host index from the content of full KV blocks to cached physical blocks."""
+
+    def __init__(self, block_size: int):
+        self._h = ctypes.c_void_p()
+        _check(lib().pa_prefix_cache_create(int(block_size), ctypes.byref(self._h)), "pa_prefix_cache_create")
+
+    def __len__(self):
+        return lib().pa_prefix_cache_size(self._h)
+
+    def __del__(self):
+        try:
+            if self._h:
+                lib().pa_prefix_cache_destroy(self._h)
+        except Exception:
+            pass
+
+    def match(self, pool: Pool, tokens, row) -> int:
+        """Reuse the leading cached full blocks of `tokens` into `row` (host int32)."""
+        import numpy as np
+        t = np.ascontiguousarray(tokens, dtype=np.int32)
+        n = ctypes.c_int32()
+        _check(lib().pa_prefix_cache_match(self._h, pool._h, _i32p(t), t.size, _i32p(row), row.shape[-1],
+                                           ctypes.byref(n)), "pa_prefix_cache_match")
+        return n.value
+
+    def insert(self, pool: Pool, tokens, row) -> int:
+        import numpy as np
+        t = np.ascontiguousarray(tokens, dtype=np.int32)
+        n = ctypes.c_int32()
+        _check(lib().pa_prefix_cache_insert(self._h, pool._h, _i32p(t), t.size, _i32p(row), ctypes.byref(n)),
+               "pa_prefix_cache_insert")
+        return n.value
+
+    def evict(self, pool: Pool, max_blocks: int) -> int:
+        n = ctypes.c_int32()
+        _check(lib().pa_prefix_cache_evict(self._h, pool._h, int(max_blocks), ctypes.byref(n)),
+               "pa_prefix_cache_evict")
+        return n.value
+
+    def clear(self, pool: Pool) -> int:
+        n = ctypes.c_int32()
+        _check(lib().pa_prefix_cache_clear(self._h, pool._h, ctypes.byref(n)), "pa_prefix_cache_clear")
+        return n.value
 
 
 def version() -> str:

@@ -266,3 +266,66 @@ def test_engine_step_out_of_blocks_reports_and_keeps_state_consistent():
     assert eng.lens.tolist() == [17, 16, 16] and eng.pool.num_free() == 0
     torch.cuda.synchronize()
     assert torch.count_nonzero(out) == 0
+
+
+def test_decode_over_prefix_cache_built_batch():
+    """Requests sharing a 1000-token history, admitted through the prefix cache: the
+    first writes the history's K/V, the others reuse its 62 full blocks and write only
+    their unmatched tokens. Tables, cache bytes and outputs against the oracle running
+    its own pool, prefix cache and cache ops."""
+    from oracle.pool import BlockPool
+    from oracle.prefix_cache import PrefixCache as OPrefix
+    S, Hq, Hkv, D, BS, hist_len = 12, 32, 8, 128, 16, 1000
+    rng = np.random.default_rng(91)
+    priv = rng.integers(1, 60, size=S).tolist()
+    lens = [hist_len + p for p in priv]
+    w = synthetic.custom(S, Hq, Hkv, D, BS, "bf16", "bf16", lens, 92, pool_factor=0.3)
+    w.num_blocks = 62 + sum(-(-L // BS) - 62 for L in lens) + 4
+    w.initial_order = rng.permutation(w.num_blocks).tolist()
+    hist = rng.integers(0, 32000, size=hist_len).tolist()
+    prompts = [hist + rng.integers(0, 32000, size=p).tolist() for p in priv]
+    # K/V of every (position, token): history rows are the same for every request
+    kh = synthetic.normal_values((hist_len, Hkv, D), "bf16", 93)
+    vh = synthetic.normal_values((hist_len, Hkv, D), "bf16", 94)
+    eng = make_engine(w, DEV)
+    fill_cache(w, eng)
+    ncache = pa.PrefixCache(BS)
+    opool, ocache = BlockPool(w.num_blocks, w.initial_order), OPrefix(BS)
+    k0, v0 = codes_np(eng.k_cache), codes_np(eng.v_cache)
+    ek, ev = k0, v0
+    orows = []
+    for s, prompt in enumerate(prompts):
+        n = ncache.match(eng.pool, prompt, eng.bt_host[s])
+        eng.lens[s] = n * BS
+        start = n * BS
+        slots = np.zeros(len(prompt) - start, np.int64)
+        eng.extend(s, len(prompt) - start, slots)
+        ncache.insert(eng.pool, prompt, eng.bt_host[s])
+        orow = []
+        on = ocache.match(opool, prompt, orow)
+        opool.seq_extend(orow, on * BS, len(prompt) - on * BS, BS)
+        ocache.insert(opool, prompt, orow)
+        orows.append(orow)
+        assert n == on == (0 if s == 0 else 62)
+        assert eng.bt_host[s, :len(orow)].tolist() == orow
+        # this request's unmatched tokens: history rows from the shared table, then private rows
+        m = len(prompt) - start
+        kp = synthetic.normal_values((len(prompt) - hist_len, Hkv, D), "bf16", 1000 + s)
+        vp = synthetic.normal_values((len(prompt) - hist_len, Hkv, D), "bf16", 2000 + s)
+        kt = torch.cat([kh[start:], kp])[-m:] if start < hist_len else kp[start - hist_len:]
+        vt = torch.cat([vh[start:], vp])[-m:] if start < hist_len else vp[start - hist_len:]
+        pa.reshape_and_cache(kt.to(DEV), vt.to(DEV), torch.from_numpy(slots).to(DEV), eng.cache)
+        ek, ev = oops.reshape_and_cache(codes_np(kt), codes_np(vt), "bf16", slots, ek, ev, "bf16")
+    assert eng.pool.num_free() == opool.num_free() and len(ncache) == len(ocache) >= 62
+    eng.upload_tables()
+    q = synthetic.normal_values((S, Hq, D), "bf16", 95).to(DEV)
+    out = torch.full_like(q, float("nan"))
+    eng.run_decode(q, out, w.scale)
+    torch.cuda.synchronize()
+    assert pa.last_device_error()[0] == 0
+    assert np.array_equal(codes_np(eng.k_cache), ek) and np.array_equal(codes_np(eng.v_cache), ev)
+    bt = np.zeros((S, eng.MB), np.int64)
+    for s, r in enumerate(orows):
+        bt[s, :len(r)] = r
+    ref = oatt.paged_decode(codes_np(q), "bf16", ek, ev, "bf16", 1.0, 1.0, bt, lens, w.scale)
+    assert_close(out.double().cpu().numpy(), ref, "bf16", "prefix-cache batch")
