@@ -219,7 +219,14 @@ def build_engine(w, growth, device):
     else:
         synthetic.fill_normal_(eng.k_cache, w.kv_dtype, w.seed * 10 + 1)
         synthetic.fill_normal_(eng.v_cache, w.kv_dtype, w.seed * 10 + 2)
-    if w.prefix_len:
+    if getattr(w, "beam_width", 0):
+        # each request's prompt is written once; its other beams fork it
+        W = w.beam_width
+        for r in range(w.num_seqs // W):
+            eng.extend(r * W, w.context_lens[r * W] - 1)
+            for j in range(1, W):
+                eng.fork(r * W, r * W + j)
+    elif w.prefix_len:
         # requests admitted through the prefix cache: all carry the same history, so
         # every request after the first reuses its full blocks and allocates only its
         # partial block and private tokens (the step appends each request's last token)
@@ -268,8 +275,13 @@ class StepRunner:
 
     def step(self, i, ev_pair=None):
         """One native engine step on device-resident inputs; CUDA events around the
-        partition kernel. Returns (decode bytes, kernel launches)."""
+        partition kernel. Beam workloads re-select their beams first (host reorder +
+        table upload). Returns (decode bytes, kernel launches)."""
         q, k, v = self.inputs[i % len(self.inputs)]
+        width = getattr(self.w, "beam_width", 0)
+        if width:
+            import synthetic
+            self.eng.reorder(synthetic.beam_parents(self.w.num_seqs // width, width, i, self.w.seed))
         self.eng.step(q, k, v, self.out, events=ev_pair)
         nbytes = decode_bytes(self.eng.lens, self.w.num_kv_heads, self.w.num_q_heads, self.w.head_dim,
                               self.kv_bytes, self.q_bytes, self.w.block_size)
@@ -490,7 +502,9 @@ def main(argv=None):
                         clocks=True, local_rank=local)
         also = []
         for name in [a for a in args.also.split(",") if a]:
-            if name == "gqa_noshare":
+            if name == "beam5":
+                wa = synthetic.beam_workload()
+            elif name == "gqa_noshare":
                 # the GQA-prefix shapes with every sequence holding its own blocks
                 g = synthetic.make("gqa_prefix")
                 wa = synthetic.custom(g.num_seqs, g.num_q_heads, g.num_kv_heads, g.head_dim, g.block_size,
@@ -538,6 +552,10 @@ def main(argv=None):
                      "roofline": {"bound": "hbm", "achieved": kg, "peak": peak, "unit": "GB/s",
                                   "frac": kg / peak, "ms_per_launch": ra["kernel_ms_mean"],
                                   "traffic": kernel_traffic(wa.name, ra["kernel_bytes_mean"])}}
+            if getattr(wa, "beam_width", 0):
+                entry["note"] = ("logical bytes: each beam's whole context is counted; the beams of a "
+                                 "request share their prompt blocks")
+                entry["copy_on_write_pairs_last_step"] = ra["num_cow"]
             if wa.prefix_len:
                 entry["note"] = ("logical bytes: the shared prefix is counted once per sequence; "
                                  "it is read from HBM about once and from L2 after that")

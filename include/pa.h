@@ -409,6 +409,21 @@ pa_status pa_engine_step(pa_engine* engine, const void* q, const void* k_new, co
 pa_status pa_engine_last_step(const pa_engine* engine, int32_t* num_cow, int32_t* num_updates,
                               int32_t* launches);
 
+/*
+ * pa_batch_reorder -- beam re-selection: new sequence i continues old sequence
+ * parents[i] (page 1, section "5. 高级应用场景": beams share their common blocks).
+ * Row i of block_tables (host int32 [num_seqs][max_blocks]) becomes a copy of old row
+ * parents[i] and context_lens[i] (host, tokens held) its length; every new row takes
+ * one reference per block before any old row drops its references, so a beam chosen
+ * k times holds its blocks k times and a beam chosen 0 times frees its private
+ * blocks. The next pa_seq_append / pa_batch_append into a shared partial block then
+ * reports the copy-on-write pair. O(total blocks). The caller refreshes the device
+ * mirror of the tables (e.g. a full upload). PA_ERR_ARG / PA_ERR_STATE leave
+ * everything unchanged.
+ */
+pa_status pa_batch_reorder(pa_pool* pool, int32_t* block_tables, int32_t* context_lens, int32_t num_seqs,
+                           int32_t max_blocks, int32_t block_size, const int32_t* parents);
+
 /* Library version string and the device architecture it was built for. */
 const char* pa_version(void);
 

@@ -147,3 +147,23 @@ class BlockPool:
             if pos % block_size == 0 or cs >= 0:
                 updates.append((s, pos // block_size, row[pos // block_size]))
         return slots, cows, updates
+
+
+def reorder(pool: BlockPool, rows: list, lens: list, parents) -> tuple:
+    """Beam re-selection: new sequence i continues old sequence parents[i].
+
+    Page 1 «突破GPU内存瓶颈：vLLM与PagedAttention技术深度解析», section "5. 高级应用场景"
+    (beam search: the beams share their common blocks). Reading: every new row is a
+    copy of its parent's row and takes one reference per block; then every old row
+    drops its references, so a beam chosen k times holds its blocks k times and a
+    beam chosen 0 times returns its private blocks. Returns (new rows, new lens).
+    """
+    new_rows = [list(rows[p]) for p in parents]
+    new_lens = [lens[p] for p in parents]
+    for r in new_rows:
+        for b in r:
+            pool.incref(b)
+    for r in rows:
+        for b in r:
+            pool.decref(b)
+    return new_rows, new_lens

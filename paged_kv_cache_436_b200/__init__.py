@@ -101,6 +101,7 @@ _SIGNATURES = {
     "pa_prefix_cache_insert": (_I32, [_P, _P, _PI32, _I32, _PI32, _PI32]),
     "pa_prefix_cache_evict": (_I32, [_P, _P, _I32, _PI32]),
     "pa_prefix_cache_clear": (_I32, [_P, _P, _PI32]),
+    "pa_batch_reorder": (_I32, [_P, _PI32, _PI32, _I32, _I32, _I32, _PI32]),
     "pa_version": (ctypes.c_char_p, []),
 }
 
@@ -330,6 +331,13 @@ class Pool:
 
     def seq_free(self, row, n_blocks: int):
         _check(lib().pa_seq_free(self._h, _i32p(row), int(n_blocks)), "pa_seq_free")
+
+    def batch_reorder(self, block_tables, context_lens, block_size: int, parents):
+        """Beam re-selection in place: row i continues old row parents[i] (host int32 arrays)."""
+        import numpy as np
+        par = np.ascontiguousarray(parents, dtype=np.int32)
+        _check(lib().pa_batch_reorder(self._h, _i32p(block_tables), _i32p(context_lens), block_tables.shape[0],
+                                      block_tables.shape[1], int(block_size), _i32p(par)), "pa_batch_reorder")
 
     def batch_append(self, block_tables, positions, block_size: int, slots, cow_pairs, updates):
         """One step's bookkeeping. All buffers are contiguous host arrays; returns (n_cow, n_updates)."""

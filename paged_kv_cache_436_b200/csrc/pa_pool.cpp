@@ -209,4 +209,42 @@ pa_status pa_batch_append(pa_pool* pool, int32_t* block_tables, int32_t num_seqs
   return PA_OK;
 }
 
+pa_status pa_batch_reorder(pa_pool* pool, int32_t* block_tables, int32_t* context_lens, int32_t num_seqs,
+                           int32_t max_blocks, int32_t block_size, const int32_t* parents) {
+  if (!pool || !block_tables || !context_lens || !parents || num_seqs < 0 || max_blocks <= 0 || block_size <= 0)
+    return PA_ERR_ARG;
+  for (int32_t i = 0; i < num_seqs; ++i) {
+    if (parents[i] < 0 || parents[i] >= num_seqs) return PA_ERR_ARG;
+    if (context_lens[i] < 0 || ceil_div(context_lens[i], block_size) > max_blocks) return PA_ERR_ARG;
+  }
+  const size_t n = size_t(num_seqs) * max_blocks;
+  std::vector<int32_t> old_tables(block_tables, block_tables + n);
+  std::vector<int32_t> old_lens(context_lens, context_lens + num_seqs);
+  for (int32_t i = 0; i < num_seqs; ++i) {
+    const int32_t p = parents[i];
+    const int32_t nb = ceil_div(old_lens[p], block_size);
+    for (int32_t k = 0; k < nb; ++k)
+      if (!in_range(pool, old_tables[size_t(p) * max_blocks + k]) ||
+          pool->refcnt[old_tables[size_t(p) * max_blocks + k]] == 0)
+        return PA_ERR_STATE;
+  }
+  // every new row takes its references before any old row drops its own
+  for (int32_t i = 0; i < num_seqs; ++i) {
+    const int32_t p = parents[i];
+    const int32_t nb = ceil_div(old_lens[p], block_size);
+    std::memcpy(block_tables + size_t(i) * max_blocks, old_tables.data() + size_t(p) * max_blocks,
+                size_t(max_blocks) * sizeof(int32_t));
+    context_lens[i] = old_lens[p];
+    for (int32_t k = 0; k < nb; ++k) ++pool->refcnt[old_tables[size_t(p) * max_blocks + k]];
+  }
+  for (int32_t i = 0; i < num_seqs; ++i) {
+    const int32_t nb = ceil_div(old_lens[i], block_size);
+    for (int32_t k = 0; k < nb; ++k) {
+      const int32_t b = old_tables[size_t(i) * max_blocks + k];
+      if (--pool->refcnt[b] == 0) push(pool, b);
+    }
+  }
+  return PA_OK;
+}
+
 }  // extern "C"

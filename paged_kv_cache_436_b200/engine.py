@@ -55,6 +55,10 @@ class DecodeEngine:
         self._meta_dev = torch.empty(self.meta_bytes, dtype=torch.uint8, device=self.device)
         self._native = None
         self._native_key = None
+        self._stage = [(torch.empty((num_seqs, max_blocks_per_seq), dtype=torch.int32).pin_memory(),
+                        torch.empty(num_seqs, dtype=torch.int32).pin_memory()) for _ in range(2)]
+        self._stage_event = [None, None]
+        self._stage_flip = 0
 
     # ------------------------------------------------------------------ set-up
     def extend(self, s: int, n_tokens: int, slots: np.ndarray | None = None):
@@ -70,6 +74,26 @@ class DecodeEngine:
         self.pool.seq_fork(self.bt_host[parent], nb)
         self.bt_host[child] = self.bt_host[parent]
         self.lens[child] = self.lens[parent]
+
+    def reorder(self, parents, stream=None):
+        """Beam re-selection: sequence i continues old sequence parents[i] (host
+        bookkeeping in C++), then the device mirror of the tables and lengths is
+        refreshed from a pinned staging buffer (double-buffered, asynchronous)."""
+        self.pool.batch_reorder(self.bt_host, self.lens, self.BS, parents)
+        i = self._stage_flip
+        self._stage_flip ^= 1
+        if self._stage_event[i] is not None:
+            self._stage_event[i].synchronize()      # the copy that last read this buffer is done
+        bt_h, lens_h = self._stage[i]
+        bt_h.numpy()[:] = self.bt_host
+        lens_h.numpy()[:] = self.lens
+        s = stream if stream is not None else torch.cuda.current_stream(self.device)
+        with torch.cuda.stream(s):
+            self.bt_dev.copy_(bt_h, non_blocking=True)
+            self.lens_dev.copy_(lens_h, non_blocking=True)
+            ev = torch.cuda.Event()
+            ev.record(s)
+        self._stage_event[i] = ev
 
     def upload_tables(self):
         """Copy the whole host block table and lengths to the device (set-up only)."""

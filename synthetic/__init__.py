@@ -53,6 +53,7 @@ class Workload:
     prefix_len: int = 0         # tokens shared by every sequence (gqa_prefix)
     private_lens: list = field(default_factory=list)   # gqa_prefix: tokens after the prefix
     extra_slots: list = field(default_factory=list)    # tiny: slots in blocks no sequence holds
+    beam_width: int = 0         # beam workloads: sequences r*width .. r*width+width-1 are one request
 
     @property
     def group(self) -> int:
@@ -228,7 +229,7 @@ def subset(w: Workload, n_seqs: int) -> Workload:
     nb = _pool_size(lens, w.block_size)
     return Workload(f"{w.name}[:{n_seqs}]", w.index, n_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim,
                     w.block_size, w.kv_dtype, w.q_dtype, lens, nb, rng.permutation(nb).tolist(), w.scale,
-                    w.seed, w.prefix_len, list(w.private_lens[:n_seqs]), [])
+                    w.seed, w.prefix_len, list(w.private_lens[:n_seqs]), [], w.beam_width)
 
 
 def grown(w: Workload, tokens: int) -> Workload:
@@ -242,4 +243,38 @@ def grown(w: Workload, tokens: int) -> Workload:
     order = list(w.initial_order) + (w.num_blocks + rng.permutation(extra)).tolist()
     return Workload(w.name, w.index, w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size,
                     w.kv_dtype, w.q_dtype, list(w.context_lens), w.num_blocks + extra, order, w.scale,
-                    w.seed, w.prefix_len, list(w.private_lens), list(w.extra_slots))
+                    w.seed, w.prefix_len, list(w.private_lens), list(w.extra_slots), w.beam_width)
+
+
+# --------------------------------------------------------------------------
+# beam search (page 1, section "5. 高级应用场景": width-5 beam search)
+# --------------------------------------------------------------------------
+
+BEAM_PARENT_WEIGHTS = (0.40, 0.25, 0.15, 0.12, 0.08)
+
+
+def beam_workload(num_requests=16, width=5, prompt=1024, num_heads=40, head_dim=128, block_size=16,
+                  kv_dtype="bf16", growth=256, seed=4369) -> Workload:
+    """`num_requests` prompts of `prompt` + U[0,15] tokens, each decoded by `width`
+    beams (sequence r * width + j is beam j of request r). The pool holds one copy of
+    every prompt plus room for `growth` private tokens per beam."""
+    rng = np.random.default_rng(seed)
+    plens = (prompt + rng.integers(0, 16, size=num_requests)).tolist()
+    lens = [L for L in plens for _ in range(width)]
+    need = sum(-(-L // block_size) for L in plens) + num_requests * width * (-(-growth // block_size) + 1)
+    nb = int(math.ceil(1.1 * need))
+    return Workload("beam%d" % width, 0, num_requests * width, num_heads, num_heads, head_dim, block_size,
+                    kv_dtype, kv_dtype, lens, nb, rng.permutation(nb).tolist(), 1.0 / math.sqrt(head_dim), seed,
+                    beam_width=width)
+
+
+def beam_parents(num_requests: int, width: int, step: int, seed: int):
+    """Seeded beam re-selection of one step: new beam j of request r continues old
+    beam parents[r * width + j] (same request; beams ranked by index, the better
+    ones chosen more often; sorted, as a top-k selection would list them)."""
+    rng = np.random.default_rng(seed * 7919 + step)
+    out = []
+    for r in range(num_requests):
+        picks = np.sort(rng.choice(width, size=width, p=BEAM_PARENT_WEIGHTS[:width]))
+        out += (r * width + picks).tolist()
+    return out

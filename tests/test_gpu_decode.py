@@ -329,3 +329,54 @@ def test_decode_over_prefix_cache_built_batch():
         bt[s, :len(r)] = r
     ref = oatt.paged_decode(codes_np(q), "bf16", ek, ev, "bf16", 1.0, 1.0, bt, lens, w.scale)
     assert_close(out.double().cpu().numpy(), ref, "bf16", "prefix-cache batch")
+
+
+def test_beam_search_steps():
+    """Width-5 beams: each step re-selects beams (fork/free), appends one token per beam
+    (copy-on-write of shared partial blocks), writes the tokens and decodes. Tables,
+    copy pairs, cache bytes and outputs against the oracle over several steps."""
+    from oracle import pool as opool_mod
+    from oracle.pool import BlockPool
+    R, W = 3, 5
+    w = synthetic.beam_workload(num_requests=R, width=W, prompt=90, num_heads=4, head_dim=128,
+                                block_size=16, growth=40, seed=4242)
+    S = R * W
+    eng = make_engine(w, DEV, growth=40)
+    fill_cache(w, eng)
+    opool = BlockPool(w.num_blocks, w.initial_order)
+    orows, olens = [[] for _ in range(S)], [0] * S
+    for r in range(R):
+        L = w.context_lens[r * W]
+        eng.extend(r * W, L)
+        opool.seq_extend(orows[r * W], 0, L, w.block_size)
+        for j in range(1, W):
+            eng.fork(r * W, r * W + j)
+            orows[r * W + j] = opool.fork(orows[r * W])
+        olens[r * W:(r + 1) * W] = [L] * W
+    eng.upload_tables()
+    ek, ev = codes_np(eng.k_cache), codes_np(eng.v_cache)
+    cows_seen = 0
+    for step in range(6):
+        parents = synthetic.beam_parents(R, W, step, w.seed)
+        eng.reorder(parents)
+        orows, olens = opool_mod.reorder(opool, orows, olens, parents)
+        q, k, v = synthetic.step_inputs(w, step)
+        out = torch.full(q.shape, float("nan"), dtype=q.dtype, device=DEV)
+        eng.step(q.to(DEV), k.to(DEV), v.to(DEV), out, w.scale)
+        torch.cuda.synchronize()
+        assert pa.last_device_error()[0] == 0
+        oslots, ocows, _ = opool.batch_append(orows, olens, w.block_size)
+        olens = [L + 1 for L in olens]
+        assert eng.last_step()[0] == len(ocows)
+        cows_seen += len(ocows)
+        for s in range(S):
+            assert eng.bt_host[s, :len(orows[s])].tolist() == orows[s]
+        ek, ev = oops.copy_blocks(ek, ev, ocows)
+        ek, ev = oops.reshape_and_cache(codes_np(k), codes_np(v), w.q_dtype, oslots, ek, ev, w.kv_dtype)
+        assert np.array_equal(codes_np(eng.k_cache), ek) and np.array_equal(codes_np(eng.v_cache), ev)
+        bt = np.zeros((S, eng.MB), np.int64)
+        for s, r in enumerate(orows):
+            bt[s, :len(r)] = r
+        ref = oatt.paged_decode(codes_np(q), w.q_dtype, ek, ev, w.kv_dtype, 1.0, 1.0, bt, olens, w.scale)
+        assert_close(out.double().cpu().numpy(), ref, w.kv_dtype, f"beam step {step}")
+    assert cows_seen > 0
