@@ -115,3 +115,42 @@ def paged_decode(q_codes: np.ndarray, q_dtype: str, k_codes: np.ndarray, v_codes
 
 def _nblocks(context_len: int, block_size: int) -> int:
     return -(-context_len // block_size)
+
+
+def paged_extend(q_codes: np.ndarray, q_dtype: str, k_codes: np.ndarray, v_codes: np.ndarray,
+                 kv_dtype: str, k_scale: float, v_scale: float, block_tables: np.ndarray,
+                 context_lens, query_start, scale: float, rows=None) -> np.ndarray:
+    """Several new tokens per sequence attend causally over the paged context.
+
+    Page 2 (untitled; first section "1. 为什么vLLM能实现24倍推理加速"), section
+    "2.1 核心组件交互流程": the execution engine runs prefill, decode and "extend"
+    (long-context extension) modes; section "2.2 关键数据结构剖析": the attention
+    metadata carries per-sequence query lengths beside the context lengths.
+
+    Reading: sequence s owns query rows query_start[s] .. query_start[s+1]-1 (Q_s of
+    them); its context_lens[s] = L_s tokens include the Q_s new ones, whose K/V are
+    already in the cache. Query i of s sits at position L_s - Q_s + i and attends to
+    tokens 0 .. L_s - Q_s + i (itself and everything before it). With Q_s = 1 this is
+    :func:`paged_decode`. ``rows`` optionally restricts the work to (query row, q head)
+    pairs. Returns out [T, Hq, D] float64.
+    """
+    q = codecs.decode(q_codes, q_dtype)
+    T, Hq, D = q.shape
+    Hkv = k_codes.shape[1]
+    G = Hq // Hkv
+    out = np.zeros((T, Hq, D), dtype=np.float64)
+    owner = {}
+    for s in range(len(context_lens)):
+        for t in range(int(query_start[s]), int(query_start[s + 1])):
+            owner[t] = s
+    pairs = rows if rows is not None else [(t, h) for t in range(T) for h in range(Hq)]
+    for t, h in pairs:
+        s = owner[t]
+        L = int(context_lens[s])
+        Qs = int(query_start[s + 1]) - int(query_start[s])
+        pos = L - Qs + (t - int(query_start[s]))
+        g = h // G
+        K = codecs.decode(gather_sequence(k_codes, block_tables[s], pos + 1, g), kv_dtype) * float(k_scale)
+        V = codecs.decode(gather_sequence(v_codes, block_tables[s], pos + 1, g), kv_dtype) * float(v_scale)
+        out[t, h] = softmax_weighted_sum(q[t, h], K, V, scale)
+    return out
