@@ -212,6 +212,33 @@ pa_status pa_decode_no_alloc(const void* q, int32_t q_dtype, int32_t num_seqs, i
                              int32_t max_context_len, float scale, void* out, void* stream);
 
 /*
+ * pa_extend -- several new tokens per sequence attend causally over the paged context
+ * (speculative verification, chunked prefill). Page 2, section "2.1 核心组件交互流程":
+ * the engine runs prefill, decode and extend modes; section "2.2 关键数据结构剖析": the
+ * metadata carries query lengths beside the context lengths.
+ *   query_start    device int32 [num_seqs + 1]: sequence s owns query rows
+ *                  query_start[s] .. query_start[s+1]-1 (Q_s rows), query_start[0] = 0
+ *   num_tokens     host: query_start[num_seqs] (rows of q and out)
+ *   context_lens   device int32 [num_seqs]: L_s, including the Q_s new tokens, whose K/V
+ *                  are already in the cache (pa_reshape_and_cache)
+ *   q, out         device [num_tokens][num_q_heads][head_dim] of q_dtype
+ * Query i of sequence s sits at position L_s - Q_s + i and attends to tokens
+ * 0 .. L_s - Q_s + i; out = softmax(scale * q K^T) V over them. Q_s > L_s is recorded
+ * (PA_DEV_BAD_CONTEXT_LEN) and its rows are zero. Runs on the tensor cores (16-bit
+ * inputs, binary32 accumulation; P rounded to the cache's 16-bit type); 512-token
+ * partitions merged by a log-sum-exp kernel as in pa_decode.
+ * Supported: 16-bit caches with q_dtype == kv_dtype, head_dim 64 or 128, block_size 16
+ * or 32, G in {1, 2, 4, 8}. workspace >= pa_extend_workspace_size(...), 256-byte aligned.
+ */
+pa_status pa_extend(const void* q, int32_t q_dtype, int32_t num_seqs, int32_t num_q_heads,
+                    const int32_t* query_start, int32_t num_tokens, const pa_cache_desc* cache,
+                    const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
+                    int32_t max_context_len, float scale, void* out, void* workspace, size_t workspace_bytes,
+                    void* stream);
+size_t pa_extend_workspace_size(int32_t num_seqs, int32_t num_tokens, int32_t num_q_heads, int32_t head_dim,
+                                int32_t max_context_len);
+
+/*
  * pa_last_device_error -- synchronise `stream`, then read and clear the device error
  * word of the current device. *code receives a PA_DEV_* value; info (may be NULL)
  * receives 3 int32 details. Returns PA_ERR_DEVICE_CHECK when *code != 0.

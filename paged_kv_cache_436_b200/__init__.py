@@ -102,6 +102,9 @@ _SIGNATURES = {
     "pa_prefix_cache_evict": (_I32, [_P, _P, _I32, _PI32]),
     "pa_prefix_cache_clear": (_I32, [_P, _P, _PI32]),
     "pa_batch_reorder": (_I32, [_P, _PI32, _PI32, _I32, _I32, _I32, _PI32]),
+    "pa_extend": (_I32, [_P, _I32, _I32, _I32, _P, _I32, _PDESC, _P, _I32, _P, _I32, ctypes.c_float, _P, _P,
+                         ctypes.c_size_t, _P]),
+    "pa_extend_workspace_size": (ctypes.c_size_t, [_I32, _I32, _I32, _I32, _I32]),
     "pa_version": (ctypes.c_char_p, []),
 }
 
@@ -223,6 +226,22 @@ def decode(q, cache: KVCache, block_tables, context_lens, max_context_len: int, 
         _check(lib().pa_decode(*args), "pa_decode")
     else:
         _check(lib().pa_decode_stage(int(stage), *args), f"pa_decode_stage({stage})")
+
+
+def extend_workspace_size(num_seqs, num_tokens, num_q_heads, head_dim, max_context_len) -> int:
+    return int(lib().pa_extend_workspace_size(num_seqs, num_tokens, num_q_heads, head_dim, max_context_len))
+
+
+def extend(q, cache: KVCache, query_start, block_tables, context_lens, max_context_len: int, scale: float, out,
+           workspace, stream=None) -> None:
+    """Multi-query causal attention: q, out [T, Hq, D]; query_start int32 [S + 1] (device)."""
+    T, Hq, _ = q.shape
+    S = query_start.shape[0] - 1
+    st = lib().pa_extend(_ptr(q), dtype_code(q), S, Hq, _ptr(query_start), T, ctypes.byref(cache.desc),
+                         _ptr(block_tables), block_tables.shape[1], _ptr(context_lens), int(max_context_len),
+                         float(scale), _ptr(out), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                         _stream(stream))
+    _check(st, "pa_extend")
 
 
 NO_ALLOC_WORKSPACE_BYTES = 16 << 20

@@ -1,0 +1,645 @@
+// Multi-query causal attention over the paged cache ("extend": several new tokens per
+// sequence -- speculative verification, chunked prefill -- attend to the whole context).
+//
+// Page 2 (untitled; first section "1. 为什么vLLM能实现24倍推理加速"), section
+// "2.1 核心组件交互流程": the execution engine runs prefill, decode and extend modes;
+// section "2.2 关键数据结构剖析": the attention metadata carries query lengths beside
+// the context lengths. Query i of sequence s sits at position L_s - Q_s + i and
+// attends to tokens 0 .. L_s - Q_s + i.
+//
+// With 16 query rows per K/V byte the work is a real contraction, so it runs on the
+// tensor cores (mma.sync m16n8k16, 16-bit inputs, binary32 accumulation):
+//   * a work unit is (sequence, kv head, tile of 16 rows, 512-token partition); a row
+//     is a (query, q head of the kv head's group) pair, so a tile holds 16 / G queries;
+//   * each warp is an independent persistent worker with a 2-stage ring of K/V blocks;
+//     every token row arrives by its own 1-D bulk copy (TMA engine, no multicast) into
+//     a padded shared-memory row (head_dim * 2 + 16 bytes), which keeps the ldmatrix
+//     reads of 8 rows free of bank conflicts without a tensor map;
+//   * S = Q K^T and O += P V per 16-token slice; the S accumulators are reused as the
+//     P operand (rounded to the cache's 16-bit type; the running sum adds the same
+//     rounded values); causal mask per row; online softmax in base 2;
+//   * one partition writes the output row, several write (max, sum, unnormalised row)
+//     for the log-sum-exp merge kernel, as in decode.
+#include <cuda_runtime.h>
+
+#include "pa.h"
+#include "pa_device.cuh"
+
+namespace pa {
+
+struct ExtendParams {
+  const void* q;
+  void* out;
+  const uint8_t* k_cache;
+  const uint8_t* v_cache;
+  const int32_t* block_tables;
+  const int32_t* context_lens;
+  const int32_t* query_start;   // [S + 1]
+  int32_t* plan;                // [S + 1] exclusive scan of units per sequence (one kv head)
+  float* part_ml;               // [T][Hq][Pmax][2]
+  float* part_acc;              // [T][Hq][Pmax][D]
+  int num_seqs, num_tokens, num_q_heads, num_kv_heads, num_blocks, max_blocks, max_parts;
+  int len_limit;
+  float s_mul;                  // scale * log2(e)
+  int out_row_bytes;            // Hq * D * 2
+};
+
+constexpr int kTileRows = 16;
+
+__device__ __forceinline__ int ext_clamp(int x, int lo, int hi) { return x < lo ? lo : (x > hi ? hi : x); }
+
+// Query count and position of query 0 of sequence s (validated the same way everywhere).
+__device__ __forceinline__ void ext_seq(const ExtendParams& p, int s, int& Q, int& base) {
+  const int L = ext_clamp(p.context_lens[s], 0, p.len_limit);
+  Q = p.query_start[s + 1] - p.query_start[s];
+  if (Q < 0 || Q > L) Q = 0;               // invalid: recorded by the plan, no work
+  base = L - Q;
+}
+
+// Partitions tile t of a sequence touches: its last query sits at base + last index.
+__device__ __forceinline__ int ext_tile_parts(int base, int Q, int qpt, int t) {
+  const int last = min((t + 1) * qpt, Q) - 1;
+  return (base + last + 1 + kPartitionTokens - 1) / kPartitionTokens;
+}
+
+__global__ void __launch_bounds__(1024) extend_plan_kernel(const ExtendParams p, int qpt) {
+  __shared__ int warp_tot[32];
+  __shared__ int carry;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  grid_dependency_launch_dependents();
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  for (int b = 0; b < p.num_seqs; b += blockDim.x) {
+    const int s = b + threadIdx.x;
+    int units = 0;
+    if (s < p.num_seqs) {
+      const int Lraw = p.context_lens[s];
+      const int Qraw = p.query_start[s + 1] - p.query_start[s];
+      if (Lraw < 0 || Lraw > p.len_limit) record_error(PA_DEV_BAD_CONTEXT_LEN, s, Lraw, p.len_limit);
+      int Q, base;
+      ext_seq(p, s, Q, base);
+      if (Qraw != Q) {
+        record_error(PA_DEV_BAD_CONTEXT_LEN, s, Qraw, Lraw);
+        // the rows of an invalid sequence are zero
+        const int t0 = ext_clamp(p.query_start[s], 0, p.num_tokens);
+        const int t1 = ext_clamp(p.query_start[s + 1], t0, p.num_tokens);
+        for (int t = t0; t < t1; ++t) {
+          uint4* row = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.out) + size_t(t) * p.out_row_bytes);
+          for (int i = 0; i < p.out_row_bytes / 16; ++i) row[i] = make_uint4(0, 0, 0, 0);
+        }
+      }
+      const int tiles = (Q + qpt - 1) / qpt;
+      for (int t = 0; t < tiles; ++t) units += ext_tile_parts(base, Q, qpt, t);
+    }
+    int incl = units;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(kFull, incl, off);
+      if (lane >= off) incl += v;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      const int nw = blockDim.x >> 5;
+      int v = lane < nw ? warp_tot[lane] : 0;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int x = __shfl_up_sync(kFull, v, off);
+        if (lane >= off) v += x;
+      }
+      if (lane < nw) warp_tot[lane] = v;
+    }
+    __syncthreads();
+    const int before = carry + (warp > 0 ? warp_tot[warp - 1] : 0) + incl - units;
+    if (s < p.num_seqs) p.plan[s] = before;
+    __syncthreads();
+    if (threadIdx.x == blockDim.x - 1) carry = before + units;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) p.plan[p.num_seqs] = carry;
+}
+
+// --------------------------------------------------------------------------
+// tensor-core helpers
+// --------------------------------------------------------------------------
+template <int QD>
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  if constexpr (QD == PA_BF16) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  } else {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  }
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_addr(p)));
+}
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_addr(p)));
+}
+
+template <int QD>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi, float& lo_r, float& hi_r) {
+  using T = typename Q<QD>::T;
+  const T a = Q<QD>::from_float(lo), b = Q<QD>::from_float(hi);
+  lo_r = Q<QD>::to_float(a);
+  hi_r = Q<QD>::to_float(b);
+  const uint16_t ua = *reinterpret_cast<const uint16_t*>(&a), ub = *reinterpret_cast<const uint16_t*>(&b);
+  return uint32_t(ua) | (uint32_t(ub) << 16);
+}
+
+template <int D, int BS>
+struct ExtCfg {
+  static constexpr int kRowBytes = D * 2;
+  static constexpr int kRowPad = kRowBytes + 16;        // padded row: conflict-free ldmatrix
+  static constexpr int kStage = 2 * BS * kRowPad;       // K rows then V rows
+  static constexpr int kStages = 2;
+  static constexpr int kWarps = 4;
+  static constexpr int kThreads = kWarps * 32;
+  static constexpr int kSmem = kWarps * kStages * kStage + kWarps * kStages * 8;
+  static constexpr int kBlocksPerPartition = kPartitionTokens / BS;
+  static_assert(BS % 16 == 0, "blocks hold whole 16-token slices");
+  static_assert(kBlocksPerPartition <= 32, "block ids of a partition fit the lanes");
+};
+
+struct ExtUnit {
+  int u;
+  int s, hk, t, part;
+  int Q, base, row0;        // row0: query row index of the sequence's first query
+  int b0, nblk;             // first block and block count of the partition (causal)
+  int bid;                  // lane i: physical block of the unit's i-th block
+};
+
+template <int BS>
+__device__ __forceinline__ ExtUnit ext_make_unit(const ExtendParams& p, int u, int total, int qpt, int lane) {
+  constexpr int BPP = kPartitionTokens / BS;
+  ExtUnit x;
+  x.u = u;
+  x.nblk = 0;
+  x.bid = 0;
+  if (u >= total) return x;
+  const int pair = u / p.num_kv_heads;
+  x.hk = u - pair * p.num_kv_heads;
+  int lo = 0, hi = p.num_seqs;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (p.plan[mid] <= pair) lo = mid; else hi = mid;
+  }
+  x.s = lo;
+  ext_seq(p, lo, x.Q, x.base);
+  x.row0 = p.query_start[lo];
+  int k = pair - p.plan[lo];
+  const int tiles = (x.Q + qpt - 1) / qpt;
+  x.t = 0;
+  for (int t = 0; t < tiles; ++t) {
+    const int P = ext_tile_parts(x.base, x.Q, qpt, t);
+    if (k < P) {
+      x.t = t;
+      break;
+    }
+    k -= P;
+  }
+  x.part = k;
+  const int last = x.base + min((x.t + 1) * qpt, x.Q) - 1;     // last position the tile sees
+  x.b0 = x.part * BPP;
+  x.nblk = min(BPP, (last + 1 + BS - 1) / BS - x.b0);
+  if (lane < x.nblk) {
+    const int lb = x.b0 + lane;
+    int v = p.block_tables[size_t(x.s) * p.max_blocks + lb];
+    if (v < 0 || v >= p.num_blocks) {
+      record_error(PA_DEV_BAD_BLOCK_ID, x.s, lb, v);
+      v = 0;
+    }
+    x.bid = v;
+  }
+  return x;
+}
+
+template <int QD, int D, int BS, int G>
+__global__ void __launch_bounds__(ExtCfg<D, BS>::kThreads) extend_kernel(const ExtendParams p) {
+  using C = ExtCfg<D, BS>;
+  using QT = typename Q<QD>::T;
+  constexpr int NS = C::kStages, NW = C::kWarps, KK = D / 16, NT = D / 8;
+  constexpr int QPT = kTileRows / G;                      // queries per tile
+
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + NW * NS * C::kStage);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint8_t* ring = smem + warp * NS * C::kStage;
+  uint64_t* bar = bars + warp * NS;
+  if (lane == 0) {
+    for (int i = 0; i < NS; ++i) mbar_init(&bar[i], 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  grid_dependency_launch_dependents();
+  grid_dependency_wait();
+
+  const int Hq = p.num_q_heads, Hkv = p.num_kv_heads;
+  const int total = p.plan[p.num_seqs] * Hkv;
+  const uint64_t pol = l2_policy_evict_first();
+  const size_t head_stride = size_t(BS) * C::kRowBytes;           // one (block, kv head) chunk
+  const size_t block_stride = size_t(Hkv) * head_stride;
+  uint32_t consumed = 0;
+
+  // rows of this lane: r0 = lane / 4 and r0 + 8 of the tile
+  const int r0 = lane >> 2, cq = (lane & 3) * 2;
+
+  for (int u = blockIdx.x * NW + warp; u < total; u += gridDim.x * NW) {
+    const ExtUnit x = ext_make_unit<BS>(p, u, total, QPT, lane);
+    // query index, position and output row of the lane's two rows (-1: no such query)
+    int qpos[2], tok[2], head[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int r = r0 + 8 * h;
+      const int qi = x.t * QPT + r / G;
+      head[h] = x.hk * G + r % G;
+      if (qi < x.Q) {
+        qpos[h] = x.base + qi;
+        tok[h] = x.row0 + qi;
+      } else {
+        qpos[h] = -1;
+        tok[h] = -1;
+      }
+    }
+    // Q fragments (A operand, 16 rows x D), zero for missing rows
+    uint32_t qa[KK][4];
+#pragma unroll
+    for (int kk = 0; kk < KK; ++kk)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int h = e & 1, dim = kk * 16 + cq + (e >> 1) * 8;
+        qa[kk][e] = tok[h] >= 0 ? *reinterpret_cast<const uint32_t*>(
+                                      static_cast<const QT*>(p.q) + (size_t(tok[h]) * Hq + head[h]) * D + dim)
+                                : 0u;
+      }
+
+    auto issue = [&](int i, uint32_t g) {
+      const int bid = __shfl_sync(kFull, x.bid, i);
+      const int st = g % NS;
+      uint8_t* dst = ring + st * C::kStage;
+      if (lane == 0) mbar_arrive_expect_tx(&bar[st], 2 * BS * C::kRowBytes);
+      __syncwarp();
+      const size_t off = size_t(bid) * block_stride + size_t(x.hk) * head_stride;
+      for (int j = lane; j < 2 * BS; j += 32) {
+        const int which = j / BS, row = j - which * BS;
+        const uint8_t* src = (which ? p.v_cache : p.k_cache) + off + size_t(row) * C::kRowBytes;
+        bulk_g2s(dst + which * BS * C::kRowPad + row * C::kRowPad, src, C::kRowBytes, &bar[st], pol);
+      }
+    };
+    for (int i = 0; i < NS && i < x.nblk; ++i) issue(i, consumed + i);
+
+    float o[NT][4];
+#pragma unroll
+    for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+    float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+    bool failed = false;
+
+    for (int i = 0; i < x.nblk; ++i) {
+      const uint32_t n = consumed;
+      const int st = n % NS;
+      if (!__all_sync(kFull, mbar_wait_bounded(&bar[st], (n / NS) & 1))) {
+        if (lane == 0) record_error(PA_DEV_WAIT_TIMEOUT, 2, u, st);
+        failed = true;
+        break;
+      }
+      const uint8_t* Ks = ring + st * C::kStage;
+      const uint8_t* Vs = Ks + BS * C::kRowPad;
+      const int tok0 = (x.b0 + i) * BS;
+#pragma unroll
+      for (int sb = 0; sb < BS / 16; ++sb) {
+        // S = Q K^T for 16 tokens (two n-tiles of 8)
+        float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+        for (int kk = 0; kk < KK; ++kk) {
+          uint32_t b[4];
+          const int trow = sb * 16 + (lane >> 4) * 8 + (lane & 7);
+          ldsm_x4(b, Ks + trow * C::kRowPad + (kk * 16 + ((lane >> 3) & 1) * 8) * 2);
+          mma16816<QD>(sc[0], qa[kk], b[0], b[1]);
+          mma16816<QD>(sc[1], qa[kk], b[2], b[3]);
+        }
+        // scale, causal mask, online softmax per row
+        float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int h = e >> 1;
+            const int tp = tok0 + sb * 16 + nt * 8 + cq + (e & 1);
+            float v = sc[nt][e] * p.s_mul;
+            if (tp > qpos[h]) v = -INFINITY;
+            sc[nt][e] = v;
+            mx[h] = fmaxf(mx[h], v);
+          }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          mx[h] = fmaxf(mx[h], __shfl_xor_sync(kFull, mx[h], 1));
+          mx[h] = fmaxf(mx[h], __shfl_xor_sync(kFull, mx[h], 2));
+        }
+        float base_m[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if (mx[h] > m[h]) {
+            const float corr = exp2f(m[h] - mx[h]);     // 0 while nothing was accumulated
+            m[h] = mx[h];
+            l[h] *= corr;
+#pragma unroll
+            for (int nn = 0; nn < NT; ++nn) {
+              o[nn][2 * h] *= corr;
+              o[nn][2 * h + 1] *= corr;
+            }
+          }
+          base_m[h] = m[h] == -INFINITY ? 0.f : m[h];
+        }
+        // P (rounded to the 16-bit type) as the A operand of P V; l adds the rounded p
+        uint32_t pa[4];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            float r_lo, r_hi;
+            pa[nt * 2 + h] = pack2<QD>(exp2f(sc[nt][2 * h] - base_m[h]), exp2f(sc[nt][2 * h + 1] - base_m[h]),
+                                       r_lo, r_hi);
+            l[h] += r_lo + r_hi;
+          }
+        // O += P V (V rows through ldmatrix.trans: two n-tiles of 8 dims per x4)
+#pragma unroll
+        for (int np = 0; np < NT / 2; ++np) {
+          uint32_t b[4];
+          const int trow = sb * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
+          ldsm_x4_trans(b, Vs + trow * C::kRowPad + (np * 16 + (lane >> 4) * 8) * 2);
+          mma16816<QD>(o[2 * np], pa, b[0], b[1]);
+          mma16816<QD>(o[2 * np + 1], pa, b[2], b[3]);
+        }
+      }
+      __syncwarp();
+      ++consumed;
+      if (i + NS < x.nblk) issue(i + NS, consumed + NS - 1);
+    }
+    if (failed) {
+      // let this unit's copies still in flight land before leaving
+      for (uint32_t k = consumed; k < consumed + NS; ++k) mbar_wait_bounded(&bar[k % NS], (k / NS) & 1, 100000000ull);
+      break;
+    }
+
+    // row sums over the quad, then the output row or the partition's partial
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      l[h] += __shfl_xor_sync(kFull, l[h], 1);
+      l[h] += __shfl_xor_sync(kFull, l[h], 2);
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      if (tok[h] < 0) continue;
+      const int P = (qpos[h] + 1 + kPartitionTokens - 1) / kPartitionTokens;
+      if (x.part >= P) continue;
+      if (P == 1) {
+        QT* orow = static_cast<QT*>(p.out) + (size_t(tok[h]) * Hq + head[h]) * D;
+        const float inv = 1.f / l[h];
+#pragma unroll
+        for (int nn = 0; nn < NT; ++nn) {
+          float a, b2;
+          const uint32_t w = pack2<QD>(o[nn][2 * h] * inv, o[nn][2 * h + 1] * inv, a, b2);
+          *reinterpret_cast<uint32_t*>(orow + nn * 8 + cq) = w;
+        }
+      } else {
+        const size_t slot = (size_t(tok[h]) * Hq + head[h]) * p.max_parts + x.part;
+        float* acc = p.part_acc + slot * D;
+#pragma unroll
+        for (int nn = 0; nn < NT; ++nn)
+          *reinterpret_cast<float2*>(acc + nn * 8 + cq) = make_float2(o[nn][2 * h], o[nn][2 * h + 1]);
+        if ((lane & 3) == 0) {
+          p.part_ml[slot * 2] = m[h];
+          p.part_ml[slot * 2 + 1] = l[h];
+        }
+      }
+    }
+  }
+}
+
+// Log-sum-exp merge of a query row's partitions: one 4-warp CTA per (query row, q head).
+template <int QD, int D>
+__global__ void __launch_bounds__(128) extend_reduce_kernel(const ExtendParams p) {
+  using QT = typename Q<QD>::T;
+  constexpr int NWARP = 4, NT = NWARP * 32, DPL = D / 32;
+  extern __shared__ float wsm[];
+  __shared__ float red[NWARP];
+  __shared__ float wsum[NWARP][D];
+  __shared__ float s_M;
+  grid_dependency_wait();
+  const int th = blockIdx.x;
+  const int t = th / p.num_q_heads;
+  int lo = 0, hi = p.num_seqs;                        // sequence owning query row t
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (p.query_start[mid] <= t) lo = mid; else hi = mid;
+  }
+  int Qn, base;
+  ext_seq(p, lo, Qn, base);
+  const int qi = t - p.query_start[lo];
+  if (qi < 0 || qi >= Qn) return;
+  const int P = (base + qi + 1 + kPartitionTokens - 1) / kPartitionTokens;
+  if (P <= 1) return;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const size_t sbase = size_t(th) * p.max_parts;
+  const float* ml = p.part_ml + sbase * 2;
+  float M = -INFINITY;
+  for (int i = tid; i < P; i += NT) M = fmaxf(M, ml[2 * i]);
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, off));
+  if (lane == 0) red[warp] = M;
+  __syncthreads();
+  if (tid == 0) s_M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  __syncthreads();
+  M = s_M;
+  float ls = 0.f;
+  for (int i = tid; i < P; i += NT) {
+    const float w = exp2f(ml[2 * i] - M);
+    wsm[i] = w;
+    ls += ml[2 * i + 1] * w;
+  }
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) ls += __shfl_xor_sync(kFull, ls, off);
+  __syncthreads();
+  if (lane == 0) red[warp] = ls;
+  const float* accp = p.part_acc + sbase * D + lane * DPL;
+  float a[DPL];
+#pragma unroll
+  for (int k = 0; k < DPL; ++k) a[k] = 0.f;
+  for (int i = warp; i < P; i += NWARP)
+#pragma unroll
+    for (int k = 0; k < DPL; ++k) a[k] = fmaf(wsm[i], accp[size_t(i) * D + k], a[k]);
+#pragma unroll
+  for (int k = 0; k < DPL; ++k) wsum[warp][lane * DPL + k] = a[k];
+  __syncthreads();
+  for (int d = tid; d < D; d += NT) {
+    const float tot = (wsum[0][d] + wsum[1][d]) + (wsum[2][d] + wsum[3][d]);
+    const float lsum = (red[0] + red[1]) + (red[2] + red[3]);
+    static_cast<QT*>(p.out)[size_t(th) * D + d] = Q<QD>::from_float(tot / lsum);
+  }
+}
+
+// --------------------------------------------------------------------------
+// host side
+// --------------------------------------------------------------------------
+struct ExtWs {
+  size_t plan, ml, acc, total;
+};
+
+inline ExtWs ext_ws(int S, int T, int Hq, int D, int max_parts) {
+  ExtWs w;
+  w.plan = 0;
+  w.ml = align256(size_t(S + 1) * 4);
+  w.acc = w.ml + align256(size_t(T) * Hq * max_parts * 2 * 4);
+  w.total = w.acc + align256(size_t(T) * Hq * max_parts * D * 4);
+  return w;
+}
+
+using ExtKernel = void (*)(const ExtendParams);
+struct ExtLaunch {
+  ExtKernel fn = nullptr;
+  int smem = 0, threads = 0;
+};
+
+template <int QD, int D, int BS, int G>
+ExtLaunch ext_get() {
+  return ExtLaunch{extend_kernel<QD, D, BS, G>, ExtCfg<D, BS>::kSmem, ExtCfg<D, BS>::kThreads};
+}
+template <int QD, int D, int BS>
+ExtLaunch ext_pick_g(int G) {
+  switch (G) {
+    case 1: return ext_get<QD, D, BS, 1>();
+    case 2: return ext_get<QD, D, BS, 2>();
+    case 4: return ext_get<QD, D, BS, 4>();
+    case 8: return ext_get<QD, D, BS, 8>();
+  }
+  return ExtLaunch{};
+}
+template <int QD, int D>
+ExtLaunch ext_pick_bs(int BS, int G) {
+  if (BS == 16) return ext_pick_g<QD, D, 16>(G);
+  if (BS == 32) return ext_pick_g<QD, D, 32>(G);
+  return ExtLaunch{};
+}
+template <int QD>
+ExtLaunch ext_pick_d(int D, int BS, int G) {
+  if (D == 64) return ext_pick_bs<QD, 64>(BS, G);
+  if (D == 128) return ext_pick_bs<QD, 128>(BS, G);
+  return ExtLaunch{};
+}
+
+cudaError_t ext_launch(ExtKernel fn, int grid, int threads, size_t smem, cudaStream_t s, const ExtendParams& p) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, fn, p);
+}
+
+}  // namespace pa
+
+extern "C" {
+
+size_t pa_extend_workspace_size(int32_t num_seqs, int32_t num_tokens, int32_t num_q_heads, int32_t head_dim,
+                                int32_t max_context_len) {
+  if (num_seqs < 0 || num_tokens < 0 || num_q_heads <= 0 || head_dim <= 0 || max_context_len < 0) return 0;
+  const int mp = max_context_len > 0 ? (max_context_len + pa::kPartitionTokens - 1) / pa::kPartitionTokens : 1;
+  return pa::ext_ws(num_seqs, num_tokens, num_q_heads, head_dim, mp).total;
+}
+
+pa_status pa_extend(const void* q, int32_t q_dtype, int32_t num_seqs, int32_t num_q_heads,
+                    const int32_t* query_start, int32_t num_tokens, const pa_cache_desc* c,
+                    const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
+                    int32_t max_context_len, float scale, void* out, void* workspace, size_t workspace_bytes,
+                    void* stream) {
+  using namespace pa;
+  pa_status st = validate_cache(c);
+  if (st != PA_OK) return st;
+  if (c->kv_dtype == PA_E4M3 || q_dtype != c->kv_dtype) return PA_ERR_ARG;   // 16-bit caches only
+  if (c->block_size != 16 && c->block_size != 32) return PA_ERR_ARG;
+  if (num_seqs < 0 || num_tokens < 0 || num_q_heads <= 0 || max_blocks_per_seq <= 0 || max_context_len < 0)
+    return PA_ERR_ARG;
+  if (num_q_heads % c->num_kv_heads != 0) return PA_ERR_ARG;
+  const int G = num_q_heads / c->num_kv_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return PA_ERR_ARG;
+  if (!std::isfinite(scale)) return PA_ERR_ARG;
+  if (num_seqs == 0 || num_tokens == 0) return PA_OK;
+  if (!q || !out || !query_start || !block_tables || !context_lens || !workspace) return PA_ERR_ARG;
+  if (!aligned16(q) || !aligned16(out) || (reinterpret_cast<uintptr_t>(workspace) & 255)) return PA_ERR_ARG;
+  const int D = c->head_dim, BS = c->block_size;
+  const int max_parts = max_context_len > 0 ? (max_context_len + kPartitionTokens - 1) / kPartitionTokens : 1;
+  if (max_parts > kMaxPartitions) return PA_ERR_ARG;
+  const ExtWs ws = ext_ws(num_seqs, num_tokens, num_q_heads, D, max_parts);
+  if (workspace_bytes < ws.total) return PA_ERR_ARG;
+  const ExtLaunch k = q_dtype == PA_BF16 ? ext_pick_d<PA_BF16>(D, BS, G) : ext_pick_d<PA_F16>(D, BS, G);
+  if (!k.fn) return PA_ERR_ARG;
+
+  ExtendParams p;
+  p.q = q;
+  p.out = out;
+  p.k_cache = static_cast<const uint8_t*>(c->k_cache);
+  p.v_cache = static_cast<const uint8_t*>(c->v_cache);
+  p.block_tables = block_tables;
+  p.context_lens = context_lens;
+  p.query_start = query_start;
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  p.plan = reinterpret_cast<int32_t*>(w + ws.plan);
+  p.part_ml = reinterpret_cast<float*>(w + ws.ml);
+  p.part_acc = reinterpret_cast<float*>(w + ws.acc);
+  p.num_seqs = num_seqs;
+  p.num_tokens = num_tokens;
+  p.num_q_heads = num_q_heads;
+  p.num_kv_heads = c->num_kv_heads;
+  p.num_blocks = c->num_blocks;
+  p.max_blocks = max_blocks_per_seq;
+  p.max_parts = max_parts;
+  const long long lim_a = (long long)max_blocks_per_seq * BS, lim_b = (long long)max_parts * kPartitionTokens;
+  p.len_limit = int(lim_a < lim_b ? lim_a : lim_b);
+  p.s_mul = scale * 1.4426950408889634f;
+  p.out_row_bytes = num_q_heads * D * 2;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  extend_plan_kernel<<<1, 1024, 0, s>>>(p, kTileRows / G);
+  if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+  int cap = 0;
+  Launch as_launch;
+  as_launch.fn = reinterpret_cast<KernelFn>(k.fn);
+  as_launch.smem = k.smem;
+  as_launch.threads = k.threads;
+  if (occupancy(as_launch, &cap) != cudaSuccess) return PA_ERR_CUDA;
+  // upper bound of the units: every tile of every sequence in every partition
+  const long long tiles = ((long long)num_tokens * G + kTileRows - 1) / kTileRows + num_seqs;
+  const long long units = tiles * c->num_kv_heads * max_parts;
+  const long long warps_needed = units;
+  const long long ctas = (warps_needed + ExtCfg<128, 16>::kWarps - 1) / ExtCfg<128, 16>::kWarps;
+  const int grid = int(ctas < cap ? ctas : cap);
+  if (ext_launch(k.fn, grid > 0 ? grid : 1, k.threads, k.smem, s, p) != cudaSuccess) return PA_ERR_CUDA;
+  if (max_parts > 1) {
+    const long long rows = (long long)num_tokens * num_q_heads;
+    ExtKernel red = q_dtype == PA_BF16 ? (D == 64 ? extend_reduce_kernel<PA_BF16, 64> : extend_reduce_kernel<PA_BF16, 128>)
+                                       : (D == 64 ? extend_reduce_kernel<PA_F16, 64> : extend_reduce_kernel<PA_F16, 128>);
+    if (ext_launch(red, int(rows), 128, size_t(max_parts) * 4, s, p) != cudaSuccess) return PA_ERR_CUDA;
+  }
+  return PA_OK;
+}
+
+}  // extern "C"

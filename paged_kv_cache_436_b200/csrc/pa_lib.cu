@@ -2,3 +2,4 @@
 // device error word, so they are compiled together (no relocatable device code).
 #include "pa_decode.cu"
 #include "pa_cache.cu"
+#include "pa_extend.cu"

@@ -1,0 +1,99 @@
+"""GPU parity of pa_extend (several new tokens per sequence, causal over the paged
+context) against the float64 oracle: |err| <= 2e-3 + 1e-2 |ref| for 16-bit caches."""
+
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import paged_kv_cache_436_b200 as pa
+import synthetic
+from oracle import attention as oatt
+from tests.gpu_cases import assert_close, codes_np, fill_cache, make_engine
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _setup(lens, qlens, Hq, Hkv, D, BS, dt, seed):
+    w = synthetic.custom(len(lens), Hq, Hkv, D, BS, dt, dt, lens, seed)
+    eng = make_engine(w, DEV)
+    fill_cache(w, eng)
+    for s, L in enumerate(lens):
+        eng.extend(s, L)
+    eng.upload_tables()
+    qs = np.concatenate([[0], np.cumsum(qlens)]).astype(np.int32)
+    T = int(qs[-1])
+    q = synthetic.normal_values((T, Hq, D), dt, seed + 7).to(DEV)
+    return w, eng, torch.from_numpy(qs).to(DEV), q, qs
+
+
+def _run(w, eng, qs_dev, q, qs_host):
+    T, Hq, D = q.shape
+    out = torch.full_like(q, float("nan"))
+    ws = torch.empty(pa.extend_workspace_size(w.num_seqs, T, Hq, D, eng.max_context_len), dtype=torch.uint8,
+                     device=DEV)
+    pa.extend(q, eng.cache, qs_dev, eng.bt_dev, eng.lens_dev, eng.max_context_len, w.scale, out, ws)
+    torch.cuda.synchronize()
+    return out
+
+
+def _ref(w, eng, q, qs_host, rows=None):
+    bt = eng.bt_host.astype(np.int64)
+    return oatt.paged_extend(codes_np(q), w.q_dtype, codes_np(eng.k_cache), codes_np(eng.v_cache), w.kv_dtype,
+                             1.0, 1.0, bt, list(eng.lens), qs_host, w.scale, rows=rows)
+
+
+@pytest.mark.parametrize("dt,D,BS,G", [("bf16", 128, 16, 1), ("f16", 128, 16, 1), ("bf16", 128, 32, 4),
+                                       ("f16", 64, 16, 2), ("bf16", 64, 32, 8), ("bf16", 128, 16, 8)])
+def test_extend_matches_oracle(dt, D, BS, G):
+    lens = [1, 5, 17, 511, 512, 513, 530, 1030, 1600]
+    qlens = [1, 5, 3, 8, 2, 7, 1, 16, 13]
+    seed = zlib.crc32(repr((dt, D, BS, G)).encode()) % 10000
+    w, eng, qs_dev, q, qs = _setup(lens, qlens, 2 * G, 2, D, BS, dt, seed)
+    out = _run(w, eng, qs_dev, q, qs)
+    assert pa.last_device_error()[0] == 0
+    ref = _ref(w, eng, q, qs)
+    assert_close(out.double().cpu().numpy(), ref, dt, f"extend {dt} D{D} BS{BS} G{G}")
+
+
+def test_chunked_prefill_matches_oracle():
+    """A whole 700-token prompt as queries (prefill), and a 150-token chunk over a
+    1300-token context (chunked prefill), with GQA."""
+    lens, qlens = [700, 1300], [700, 150]
+    w, eng, qs_dev, q, qs = _setup(lens, qlens, 8, 2, 128, 16, "bf16", 31)
+    out = _run(w, eng, qs_dev, q, qs)
+    assert pa.last_device_error()[0] == 0
+    rng = np.random.default_rng(5)
+    rows = [(int(t), int(h)) for t in rng.choice(850, size=120, replace=False) for h in (0, 3, 7)]
+    rows += [(0, h) for h in range(8)] + [(699, 1), (700, 2), (849, 5)]
+    ref = _ref(w, eng, q, qs, rows=rows)
+    got = out.double().cpu().numpy()
+    idx = tuple(np.array(rows).T)
+    assert_close(got[idx], ref[idx], "bf16", "chunked prefill")
+    # query 0 of the prompt sees token 0 only: out = that V row, rounded once
+    v0 = eng.v_cache[int(eng.bt_host[0, 0]), :, 0, :].float().cpu()
+    for h in range(8):
+        assert torch.equal(out[0, h].float().cpu(), v0[h // 4])
+
+
+def test_single_query_extend_agrees_with_decode():
+    lens = [40, 600, 1500, 3]
+    w, eng, qs_dev, q, qs = _setup(lens, [1, 1, 1, 1], 8, 2, 128, 16, "bf16", 41)
+    ext = _run(w, eng, qs_dev, q, qs)
+    dec = torch.empty_like(q)
+    eng.run_decode(q, dec)
+    torch.cuda.synchronize()
+    a, b = ext.double().cpu().numpy(), dec.double().cpu().numpy()
+    assert np.all(np.abs(a - b) <= 2e-3 + 1e-2 * np.abs(b))
+
+
+def test_more_queries_than_context_is_recorded_and_zero():
+    lens, qlens = [10, 20], [3, 4]
+    w, eng, qs_dev, q, qs = _setup(lens, qlens, 4, 4, 64, 16, "f16", 51)
+    eng.lens_dev.copy_(torch.tensor([2, 20], dtype=torch.int32))     # sequence 0: 3 queries, 2 tokens
+    out = _run(w, eng, qs_dev, q, qs)
+    code, info = pa.last_device_error()
+    assert code == 2 and info[0] == 0
+    assert torch.count_nonzero(out[:3]) == 0 and torch.isfinite(out[3:].float()).all()
