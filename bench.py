@@ -359,6 +359,58 @@ def time_ours(w, steps, warmup, device, dist, e2e=True, clocks=True, local_rank=
     return res
 
 
+def time_extend(name, steps, warmup, device):
+    """pa_extend alone (the tensor-core multi-query kernel and its merge), timed with
+    CUDA events: `spec4_mix` = 4 draft tokens per sequence over the 13B mix contexts
+    (speculative verification; HBM-bound), `prefill_8x2k` = 8 whole 2048-token prompts
+    (prefill from an empty context; compute-bound)."""
+    import torch
+    import synthetic
+    import paged_kv_cache_436_b200 as pa
+    if name == "spec4_mix":
+        base = synthetic.make("llama13b_mix")
+        w, qlen = base, 4
+    else:
+        w = synthetic.custom(8, 32, 32, 128, 16, "bf16", "bf16", [2048] * 8, 4371, pool_factor=1.05)
+        qlen = 2048
+    eng = build_engine(w, 1, device)                            # every sequence holds L - 1 tokens
+    for s in range(w.num_seqs):
+        eng.extend(s, 1)                                        # ... and now all L
+    eng.upload_tables()
+    qlens = [min(qlen, L) for L in w.context_lens]
+    qs = np.concatenate([[0], np.cumsum(qlens)]).astype(np.int32)
+    T = int(qs[-1])
+    q = synthetic.normal_values((T, w.num_q_heads, w.head_dim), w.q_dtype, w.seed + 11, device)
+    out = torch.empty_like(q)
+    ws = torch.empty(pa.extend_workspace_size(w.num_seqs, T, w.num_q_heads, w.head_dim, eng.max_context_len),
+                     dtype=torch.uint8, device=device)
+    qs_dev = torch.from_numpy(qs).to(device)
+
+    def call():
+        pa.extend(q, eng.cache, qs_dev, eng.bt_dev, eng.lens_dev, eng.max_context_len, w.scale, out, ws)
+
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        call()
+    e1.record()
+    torch.cuda.synchronize(device)
+    ms = e0.elapsed_time(e1) / steps
+    lens = np.asarray(w.context_lens, dtype=np.int64)
+    kv_bytes = int(2 * lens.sum() * w.num_kv_heads * w.head_dim * 2) + 2 * T * w.num_q_heads * w.head_dim * 2
+    flops = 0
+    for L, Qn in zip(lens, qlens):
+        pos = L - Qn + np.arange(Qn, dtype=np.int64)
+        flops += int(4 * w.num_q_heads * w.head_dim * (pos + 1).sum())
+    del eng
+    torch.cuda.empty_cache()
+    return {"workload": name, "ms_per_call": ms, "kv_gbs": kv_bytes / (ms / 1e3) / 1e9,
+            "tflops": flops / (ms / 1e3) / 1e12, "query_rows": T, "kv_bytes": kv_bytes, "flops": flops}
+
+
 # ---------------------------------------------------------------------------
 # the oracle on the host cores (cpu_baseline and --impl reference)
 # ---------------------------------------------------------------------------
@@ -501,7 +553,11 @@ def main(argv=None):
         res = time_ours(w, args.steps, args.warmup, device, dist, e2e=not args.no_e2e,
                         clocks=True, local_rank=local)
         also = []
+        extend_entries = []
         for name in [a for a in args.also.split(",") if a]:
+            if name in ("spec4_mix", "prefill_8x2k"):
+                extend_entries.append(time_extend(name, max(3, args.steps // 5), args.warmup, device))
+                continue
             if name == "beam5":
                 wa = synthetic.beam_workload()
             elif name == "gqa_noshare":
@@ -561,6 +617,17 @@ def main(argv=None):
                                  "it is read from HBM about once and from L2 after that")
                 entry["prefix_cache"] = ra.get("prefix_report")
             line.setdefault("also", []).append(entry)
+        if extend_entries:
+            import json as _json
+            with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+                bf16_peak = float(_json.load(f).get("bf16_tflops", 1645.7))
+            for e in extend_entries:
+                e["roofline"] = {"bound": "hbm" if e["workload"].startswith("spec") else "tensor",
+                                 "achieved": e["kv_gbs"] if e["workload"].startswith("spec") else e["tflops"],
+                                 "peak": peak if e["workload"].startswith("spec") else bf16_peak,
+                                 "unit": "GB/s" if e["workload"].startswith("spec") else "TFLOP/s"}
+                e["roofline"]["frac"] = e["roofline"]["achieved"] / e["roofline"]["peak"]
+                line.setdefault("extend", []).append(e)
         if rank == 0 and world == 1 and not args.no_cpu:
             line["cpu_baseline"] = cpu_baseline_obj(w, args.cpu_budget)
         if rank == 0:
