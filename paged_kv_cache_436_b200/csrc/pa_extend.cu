@@ -430,6 +430,242 @@ __global__ void __launch_bounds__(ExtCfg<D, BS>::kThreads) extend_kernel(const E
   }
 }
 
+// --------------------------------------------------------------------------
+// cooperative variant for long query runs (prefill, long extends)
+// --------------------------------------------------------------------------
+// A unit covers 64 rows (4 consumer warps x 16 rows) so that each K/V block is
+// streamed once per 64 rows instead of once per 16. A fifth warp only produces: it
+// walks the same unit sequence as the consumers and keeps the 2-stage ring full,
+// running ahead into the next unit; full[st] completes when a block has landed,
+// empty[st] when all four consumers are done with it. Every wait is bounded.
+constexpr int kCoopRows = 64;
+
+template <int D, int BS>
+struct CoopCfg {
+  static constexpr int kRowBytes = D * 2;
+  static constexpr int kRowPad = kRowBytes + 16;
+  static constexpr int kStage = 2 * BS * kRowPad;
+  static constexpr int kStages = 2;
+  static constexpr int kConsumers = 4;
+  static constexpr int kThreads = (kConsumers + 1) * 32;
+  static constexpr int kSmem = kStages * kStage + 2 * kStages * 8;
+  static constexpr int kBlocksPerPartition = kPartitionTokens / BS;
+};
+
+template <int QD, int D, int BS, int G>
+__global__ void __launch_bounds__(CoopCfg<D, BS>::kThreads) extend_coop_kernel(const ExtendParams p) {
+  using C = CoopCfg<D, BS>;
+  using QT = typename Q<QD>::T;
+  constexpr int NS = C::kStages, NC = C::kConsumers, KK = D / 16, NT = D / 8;
+  constexpr int QPT = kCoopRows / G;                   // queries per unit tile
+
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + NS * C::kStage);
+  uint64_t* empty = full + NS;
+  __shared__ int s_abort;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], NC);
+    }
+    s_abort = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  grid_dependency_launch_dependents();
+  grid_dependency_wait();
+
+  const int Hq = p.num_q_heads, Hkv = p.num_kv_heads;
+  const int total = p.plan[p.num_seqs] * Hkv;
+  const size_t head_stride = size_t(BS) * C::kRowBytes;
+  const size_t block_stride = size_t(Hkv) * head_stride;
+
+  if (warp == NC) {
+    // ---------------- producer warp ----------------
+    const uint64_t pol = l2_policy_evict_first();
+    uint32_t g = 0;
+    volatile int* abort_flag = &s_abort;
+    for (int u = blockIdx.x; u < total && !*abort_flag; u += gridDim.x) {
+      const ExtUnit x = ext_make_unit<BS>(p, u, total, QPT, lane);
+      for (int i = 0; i < x.nblk; ++i, ++g) {
+        const int st = g % NS;
+        // the consumers released this stage (a fresh barrier passes parity 1 at once)
+        if (!__all_sync(kFull, mbar_wait_bounded(&empty[st], ((g / NS) & 1) ^ 1))) {
+          if (lane == 0) {
+            record_error(PA_DEV_WAIT_TIMEOUT, 3, u, st);
+            s_abort = 1;
+          }
+          return;
+        }
+        const int bid = __shfl_sync(kFull, x.bid, i);
+        uint8_t* dst = smem + st * C::kStage;
+        if (lane == 0) mbar_arrive_expect_tx(&full[st], 2 * BS * C::kRowBytes);
+        __syncwarp();
+        const size_t off = size_t(bid) * block_stride + size_t(x.hk) * head_stride;
+        for (int j = lane; j < 2 * BS; j += 32) {
+          const int which = j / BS, row = j - which * BS;
+          const uint8_t* src = (which ? p.v_cache : p.k_cache) + off + size_t(row) * C::kRowBytes;
+          bulk_g2s(dst + which * BS * C::kRowPad + row * C::kRowPad, src, C::kRowBytes, &full[st], pol);
+        }
+      }
+    }
+    return;
+  }
+
+  // ---------------- consumer warps: 16 rows each ----------------
+  const int r0 = lane >> 2, cq = (lane & 3) * 2;
+  uint32_t g = 0;
+  for (int u = blockIdx.x; u < total; u += gridDim.x) {
+    const ExtUnit x = ext_make_unit<BS>(p, u, total, QPT, lane);
+    int qpos[2], tok[2], head[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int r = warp * 16 + r0 + 8 * h;              // row of the 64-row tile
+      const int qi = x.t * QPT + r / G;
+      head[h] = x.hk * G + r % G;
+      if (qi < x.Q) {
+        qpos[h] = x.base + qi;
+        tok[h] = x.row0 + qi;
+      } else {
+        qpos[h] = -1;
+        tok[h] = -1;
+      }
+    }
+    uint32_t qa[KK][4];
+#pragma unroll
+    for (int kk = 0; kk < KK; ++kk)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int h = e & 1, dim = kk * 16 + cq + (e >> 1) * 8;
+        qa[kk][e] = tok[h] >= 0 ? *reinterpret_cast<const uint32_t*>(
+                                      static_cast<const QT*>(p.q) + (size_t(tok[h]) * Hq + head[h]) * D + dim)
+                                : 0u;
+      }
+    float o[NT][4];
+#pragma unroll
+    for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+    float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+    // a warp whose rows all lie before this partition's first token still consumes the
+    // blocks (it must release the stages) but skips the math
+    const bool active = max(qpos[0], qpos[1]) >= x.b0 * BS;
+    const bool warp_active = __any_sync(kFull, active);
+
+    for (int i = 0; i < x.nblk; ++i, ++g) {
+      const int st = g % NS;
+      if (!__all_sync(kFull, mbar_wait_bounded(&full[st], (g / NS) & 1))) {
+        if (lane == 0) {
+          record_error(PA_DEV_WAIT_TIMEOUT, 4, u, st);
+          s_abort = 1;
+        }
+        return;
+      }
+      const uint8_t* Ks = smem + st * C::kStage;
+      const uint8_t* Vs = Ks + BS * C::kRowPad;
+      const int tok0 = (x.b0 + i) * BS;
+      if (warp_active) {
+#pragma unroll
+        for (int sb = 0; sb < BS / 16; ++sb) {
+          float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+          for (int kk = 0; kk < KK; ++kk) {
+            uint32_t b[4];
+            const int trow = sb * 16 + (lane >> 4) * 8 + (lane & 7);
+            ldsm_x4(b, Ks + trow * C::kRowPad + (kk * 16 + ((lane >> 3) & 1) * 8) * 2);
+            mma16816<QD>(sc[0], qa[kk], b[0], b[1]);
+            mma16816<QD>(sc[1], qa[kk], b[2], b[3]);
+          }
+          float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int h = e >> 1;
+              const int tp = tok0 + sb * 16 + nt * 8 + cq + (e & 1);
+              float v = sc[nt][e] * p.s_mul;
+              if (tp > qpos[h]) v = -INFINITY;
+              sc[nt][e] = v;
+              mx[h] = fmaxf(mx[h], v);
+            }
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            mx[h] = fmaxf(mx[h], __shfl_xor_sync(kFull, mx[h], 1));
+            mx[h] = fmaxf(mx[h], __shfl_xor_sync(kFull, mx[h], 2));
+          }
+          float base_m[2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            if (mx[h] > m[h]) {
+              const float corr = exp2f(m[h] - mx[h]);
+              m[h] = mx[h];
+              l[h] *= corr;
+#pragma unroll
+              for (int nn = 0; nn < NT; ++nn) {
+                o[nn][2 * h] *= corr;
+                o[nn][2 * h + 1] *= corr;
+              }
+            }
+            base_m[h] = m[h] == -INFINITY ? 0.f : m[h];
+          }
+          uint32_t pa[4];
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              float r_lo, r_hi;
+              pa[nt * 2 + h] = pack2<QD>(exp2f(sc[nt][2 * h] - base_m[h]), exp2f(sc[nt][2 * h + 1] - base_m[h]),
+                                         r_lo, r_hi);
+              l[h] += r_lo + r_hi;
+            }
+#pragma unroll
+          for (int np = 0; np < NT / 2; ++np) {
+            uint32_t b[4];
+            const int trow = sb * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
+            ldsm_x4_trans(b, Vs + trow * C::kRowPad + (np * 16 + (lane >> 4) * 8) * 2);
+            mma16816<QD>(o[2 * np], pa, b[0], b[1]);
+            mma16816<QD>(o[2 * np + 1], pa, b[2], b[3]);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);          // this warp is done with the stage
+    }
+    if (*static_cast<volatile int*>(&s_abort)) return;
+
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      l[h] += __shfl_xor_sync(kFull, l[h], 1);
+      l[h] += __shfl_xor_sync(kFull, l[h], 2);
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      if (tok[h] < 0) continue;
+      const int P = (qpos[h] + 1 + kPartitionTokens - 1) / kPartitionTokens;
+      if (x.part >= P) continue;
+      if (P == 1) {
+        QT* orow = static_cast<QT*>(p.out) + (size_t(tok[h]) * Hq + head[h]) * D;
+        const float inv = 1.f / l[h];
+#pragma unroll
+        for (int nn = 0; nn < NT; ++nn) {
+          float a, b2;
+          *reinterpret_cast<uint32_t*>(orow + nn * 8 + cq) =
+              pack2<QD>(o[nn][2 * h] * inv, o[nn][2 * h + 1] * inv, a, b2);
+        }
+      } else {
+        const size_t slot = (size_t(tok[h]) * Hq + head[h]) * p.max_parts + x.part;
+        float* acc = p.part_acc + slot * D;
+#pragma unroll
+        for (int nn = 0; nn < NT; ++nn)
+          *reinterpret_cast<float2*>(acc + nn * 8 + cq) = make_float2(o[nn][2 * h], o[nn][2 * h + 1]);
+        if ((lane & 3) == 0) {
+          p.part_ml[slot * 2] = m[h];
+          p.part_ml[slot * 2 + 1] = l[h];
+        }
+      }
+    }
+  }
+}
+
 // Log-sum-exp merge of a query row's partitions: one 4-warp CTA per (query row, q head).
 template <int QD, int D>
 __global__ void __launch_bounds__(128) extend_reduce_kernel(const ExtendParams p) {
@@ -515,29 +751,30 @@ struct ExtLaunch {
 };
 
 template <int QD, int D, int BS, int G>
-ExtLaunch ext_get() {
+ExtLaunch ext_get(bool coop) {
+  if (coop) return ExtLaunch{extend_coop_kernel<QD, D, BS, G>, CoopCfg<D, BS>::kSmem, CoopCfg<D, BS>::kThreads};
   return ExtLaunch{extend_kernel<QD, D, BS, G>, ExtCfg<D, BS>::kSmem, ExtCfg<D, BS>::kThreads};
 }
 template <int QD, int D, int BS>
-ExtLaunch ext_pick_g(int G) {
+ExtLaunch ext_pick_g(int G, bool coop) {
   switch (G) {
-    case 1: return ext_get<QD, D, BS, 1>();
-    case 2: return ext_get<QD, D, BS, 2>();
-    case 4: return ext_get<QD, D, BS, 4>();
-    case 8: return ext_get<QD, D, BS, 8>();
+    case 1: return ext_get<QD, D, BS, 1>(coop);
+    case 2: return ext_get<QD, D, BS, 2>(coop);
+    case 4: return ext_get<QD, D, BS, 4>(coop);
+    case 8: return ext_get<QD, D, BS, 8>(coop);
   }
   return ExtLaunch{};
 }
 template <int QD, int D>
-ExtLaunch ext_pick_bs(int BS, int G) {
-  if (BS == 16) return ext_pick_g<QD, D, 16>(G);
-  if (BS == 32) return ext_pick_g<QD, D, 32>(G);
+ExtLaunch ext_pick_bs(int BS, int G, bool coop) {
+  if (BS == 16) return ext_pick_g<QD, D, 16>(G, coop);
+  if (BS == 32) return ext_pick_g<QD, D, 32>(G, coop);
   return ExtLaunch{};
 }
 template <int QD>
-ExtLaunch ext_pick_d(int D, int BS, int G) {
-  if (D == 64) return ext_pick_bs<QD, 64>(BS, G);
-  if (D == 128) return ext_pick_bs<QD, 128>(BS, G);
+ExtLaunch ext_pick_d(int D, int BS, int G, bool coop) {
+  if (D == 64) return ext_pick_bs<QD, 64>(BS, G, coop);
+  if (D == 128) return ext_pick_bs<QD, 128>(BS, G, coop);
   return ExtLaunch{};
 }
 
@@ -590,7 +827,10 @@ pa_status pa_extend(const void* q, int32_t q_dtype, int32_t num_seqs, int32_t nu
   if (max_parts > kMaxPartitions) return PA_ERR_ARG;
   const ExtWs ws = ext_ws(num_seqs, num_tokens, num_q_heads, D, max_parts);
   if (workspace_bytes < ws.total) return PA_ERR_ARG;
-  const ExtLaunch k = q_dtype == PA_BF16 ? ext_pick_d<PA_BF16>(D, BS, G) : ext_pick_d<PA_F16>(D, BS, G);
+  // long query runs (more than one 16-row tile per sequence on average) share each K/V
+  // block among 64 rows; short ones (speculative drafts, decode) use 16-row warp tiles
+  const bool coop = (long long)num_tokens * G > (long long)kTileRows * num_seqs;
+  const ExtLaunch k = q_dtype == PA_BF16 ? ext_pick_d<PA_BF16>(D, BS, G, coop) : ext_pick_d<PA_F16>(D, BS, G, coop);
   if (!k.fn) return PA_ERR_ARG;
 
   ExtendParams p;
@@ -618,7 +858,7 @@ pa_status pa_extend(const void* q, int32_t q_dtype, int32_t num_seqs, int32_t nu
   p.out_row_bytes = num_q_heads * D * 2;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
-  extend_plan_kernel<<<1, 1024, 0, s>>>(p, kTileRows / G);
+  extend_plan_kernel<<<1, 1024, 0, s>>>(p, (coop ? kCoopRows : kTileRows) / G);
   if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
   int cap = 0;
   Launch as_launch;
@@ -627,10 +867,11 @@ pa_status pa_extend(const void* q, int32_t q_dtype, int32_t num_seqs, int32_t nu
   as_launch.threads = k.threads;
   if (occupancy(as_launch, &cap) != cudaSuccess) return PA_ERR_CUDA;
   // upper bound of the units: every tile of every sequence in every partition
-  const long long tiles = ((long long)num_tokens * G + kTileRows - 1) / kTileRows + num_seqs;
+  const int rows_per_unit = coop ? kCoopRows : kTileRows;
+  const long long tiles = ((long long)num_tokens * G + rows_per_unit - 1) / rows_per_unit + num_seqs;
   const long long units = tiles * c->num_kv_heads * max_parts;
-  const long long warps_needed = units;
-  const long long ctas = (warps_needed + ExtCfg<128, 16>::kWarps - 1) / ExtCfg<128, 16>::kWarps;
+  // the warp kernel runs 4 independent units per CTA, the cooperative one a unit per CTA
+  const long long ctas = coop ? units : (units + ExtCfg<128, 16>::kWarps - 1) / ExtCfg<128, 16>::kWarps;
   const int grid = int(ctas < cap ? ctas : cap);
   if (ext_launch(k.fn, grid > 0 ? grid : 1, k.threads, k.smem, s, p) != cudaSuccess) return PA_ERR_CUDA;
   if (max_parts > 1) {
