@@ -42,6 +42,7 @@ struct ExtendParams {
   int len_limit;
   float s_mul;                  // scale * log2(e)
   int out_row_bytes;            // Hq * D * 2
+  int chunk;                    // context tokens per unit: a multiple of kPartitionTokens
 };
 
 constexpr int kTileRows = 16;
@@ -56,10 +57,10 @@ __device__ __forceinline__ void ext_seq(const ExtendParams& p, int s, int& Q, in
   base = L - Q;
 }
 
-// Partitions tile t of a sequence touches: its last query sits at base + last index.
-__device__ __forceinline__ int ext_tile_parts(int base, int Q, int qpt, int t) {
+// Chunks tile t of a sequence touches: its last query sits at base + last index.
+__device__ __forceinline__ int ext_tile_parts(int base, int Q, int qpt, int t, int chunk) {
   const int last = min((t + 1) * qpt, Q) - 1;
-  return (base + last + 1 + kPartitionTokens - 1) / kPartitionTokens;
+  return (base + last + 1 + chunk - 1) / chunk;
 }
 
 __global__ void __launch_bounds__(1024) extend_plan_kernel(const ExtendParams p, int qpt) {
@@ -89,7 +90,7 @@ __global__ void __launch_bounds__(1024) extend_plan_kernel(const ExtendParams p,
         }
       }
       const int tiles = (Q + qpt - 1) / qpt;
-      for (int t = 0; t < tiles; ++t) units += ext_tile_parts(base, Q, qpt, t);
+      for (int t = 0; t < tiles; ++t) units += ext_tile_parts(base, Q, qpt, t, p.chunk);
     }
     int incl = units;
 #pragma unroll
@@ -151,6 +152,8 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], const void* p) {
                : "r"(smem_addr(p)));
 }
 
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
 template <int QD>
 __device__ __forceinline__ uint32_t pack2(float lo, float hi, float& lo_r, float& hi_r) {
   using T = typename Q<QD>::T;
@@ -180,6 +183,7 @@ struct ExtUnit {
   int s, hk, t, part;
   int Q, base, row0;        // row0: query row index of the sequence's first query
   int b0, nblk;             // first block and block count of the partition (causal)
+  int last;                 // last position any row of the tile sees
   int bid;                  // lane i: physical block of the unit's i-th block
 };
 
@@ -205,7 +209,7 @@ __device__ __forceinline__ ExtUnit ext_make_unit(const ExtendParams& p, int u, i
   const int tiles = (x.Q + qpt - 1) / qpt;
   x.t = 0;
   for (int t = 0; t < tiles; ++t) {
-    const int P = ext_tile_parts(x.base, x.Q, qpt, t);
+    const int P = ext_tile_parts(x.base, x.Q, qpt, t, p.chunk);
     if (k < P) {
       x.t = t;
       break;
@@ -214,6 +218,7 @@ __device__ __forceinline__ ExtUnit ext_make_unit(const ExtendParams& p, int u, i
   }
   x.part = k;
   const int last = x.base + min((x.t + 1) * qpt, x.Q) - 1;     // last position the tile sees
+  x.last = last;
   x.b0 = x.part * BPP;
   x.nblk = min(BPP, (last + 1 + BS - 1) / BS - x.b0);
   if (lane < x.nblk) {
@@ -244,6 +249,11 @@ __global__ void __launch_bounds__(ExtCfg<D, BS>::kThreads) extend_kernel(const E
     for (int i = 0; i < NS; ++i) mbar_init(&bar[i], 1);
     fence_mbar_init();
   }
+  // rows past a tile's last visible token are never copied: they keep zeros or an
+  // earlier visible row, so a 0-weighted row cannot bring cache bytes beyond the
+  // context (possibly NaN) into P V
+  for (int i = lane; i < NS * C::kStage / 16; i += 32) reinterpret_cast<uint4*>(ring)[i] = make_uint4(0, 0, 0, 0);
+  fence_async_smem();
   __syncwarp();
   grid_dependency_launch_dependents();
   grid_dependency_wait();
@@ -291,11 +301,12 @@ __global__ void __launch_bounds__(ExtCfg<D, BS>::kThreads) extend_kernel(const E
       const int bid = __shfl_sync(kFull, x.bid, i);
       const int st = g % NS;
       uint8_t* dst = ring + st * C::kStage;
-      if (lane == 0) mbar_arrive_expect_tx(&bar[st], 2 * BS * C::kRowBytes);
+      const int nrows = min(BS, x.last + 1 - (x.b0 + i) * BS);
+      if (lane == 0) mbar_arrive_expect_tx(&bar[st], 2 * nrows * C::kRowBytes);
       __syncwarp();
       const size_t off = size_t(bid) * block_stride + size_t(x.hk) * head_stride;
-      for (int j = lane; j < 2 * BS; j += 32) {
-        const int which = j / BS, row = j - which * BS;
+      for (int j = lane; j < 2 * nrows; j += 32) {
+        const int which = j / nrows, row = j - which * nrows;
         const uint8_t* src = (which ? p.v_cache : p.k_cache) + off + size_t(row) * C::kRowBytes;
         bulk_g2s(dst + which * BS * C::kRowPad + row * C::kRowPad, src, C::kRowBytes, &bar[st], pol);
       }
@@ -404,7 +415,7 @@ __global__ void __launch_bounds__(ExtCfg<D, BS>::kThreads) extend_kernel(const E
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       if (tok[h] < 0) continue;
-      const int P = (qpos[h] + 1 + kPartitionTokens - 1) / kPartitionTokens;
+      const int P = (qpos[h] + 1 + p.chunk - 1) / p.chunk;
       if (x.part >= P) continue;
       if (P == 1) {
         QT* orow = static_cast<QT*>(p.out) + (size_t(tok[h]) * Hq + head[h]) * D;
@@ -472,6 +483,9 @@ __global__ void __launch_bounds__(CoopCfg<D, BS>::kThreads) extend_coop_kernel(c
     s_abort = 0;
     fence_mbar_init();
   }
+  for (int i = threadIdx.x; i < NS * C::kStage / 16; i += blockDim.x)
+    reinterpret_cast<uint4*>(smem)[i] = make_uint4(0, 0, 0, 0);
+  fence_async_smem();
   __syncthreads();
   grid_dependency_launch_dependents();
   grid_dependency_wait();
@@ -500,11 +514,12 @@ __global__ void __launch_bounds__(CoopCfg<D, BS>::kThreads) extend_coop_kernel(c
         }
         const int bid = __shfl_sync(kFull, x.bid, i);
         uint8_t* dst = smem + st * C::kStage;
-        if (lane == 0) mbar_arrive_expect_tx(&full[st], 2 * BS * C::kRowBytes);
+        const int nrows = min(BS, x.last + 1 - (x.b0 + i) * BS);   // rows past it stay finite
+        if (lane == 0) mbar_arrive_expect_tx(&full[st], 2 * nrows * C::kRowBytes);
         __syncwarp();
         const size_t off = size_t(bid) * block_stride + size_t(x.hk) * head_stride;
-        for (int j = lane; j < 2 * BS; j += 32) {
-          const int which = j / BS, row = j - which * BS;
+        for (int j = lane; j < 2 * nrows; j += 32) {
+          const int which = j / nrows, row = j - which * nrows;
           const uint8_t* src = (which ? p.v_cache : p.k_cache) + off + size_t(row) * C::kRowBytes;
           bulk_g2s(dst + which * BS * C::kRowPad + row * C::kRowPad, src, C::kRowBytes, &full[st], pol);
         }
@@ -640,7 +655,7 @@ __global__ void __launch_bounds__(CoopCfg<D, BS>::kThreads) extend_coop_kernel(c
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       if (tok[h] < 0) continue;
-      const int P = (qpos[h] + 1 + kPartitionTokens - 1) / kPartitionTokens;
+      const int P = (qpos[h] + 1 + p.chunk - 1) / p.chunk;
       if (x.part >= P) continue;
       if (P == 1) {
         QT* orow = static_cast<QT*>(p.out) + (size_t(tok[h]) * Hq + head[h]) * D;
@@ -687,7 +702,7 @@ __global__ void __launch_bounds__(128) extend_reduce_kernel(const ExtendParams p
   ext_seq(p, lo, Qn, base);
   const int qi = t - p.query_start[lo];
   if (qi < 0 || qi >= Qn) return;
-  const int P = (base + qi + 1 + kPartitionTokens - 1) / kPartitionTokens;
+  const int P = (base + qi + 1 + p.chunk - 1) / p.chunk;
   if (P <= 1) return;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const size_t sbase = size_t(th) * p.max_parts;
@@ -792,6 +807,12 @@ cudaError_t ext_launch(ExtKernel fn, int grid, int threads, size_t smem, cudaStr
   return cudaLaunchKernelEx(&cfg, fn, p);
 }
 
+// tcgen05 path for long query runs (pa_extend_tc.cu)
+bool extend_tc_supported(int qd, int D, int BS, int G);
+cudaError_t extend_tc_grid_cap(int qd, int BS, int G, int* cap);
+pa_status extend_tc_launch(const ExtendParams& p, const pa_cache_desc* c, int qd, int G, int grid, cudaStream_t s);
+constexpr int kTcUnitRows = 128;
+
 }  // namespace pa
 
 extern "C" {
@@ -827,11 +848,17 @@ pa_status pa_extend(const void* q, int32_t q_dtype, int32_t num_seqs, int32_t nu
   if (max_parts > kMaxPartitions) return PA_ERR_ARG;
   const ExtWs ws = ext_ws(num_seqs, num_tokens, num_q_heads, D, max_parts);
   if (workspace_bytes < ws.total) return PA_ERR_ARG;
-  // long query runs (more than one 16-row tile per sequence on average) share each K/V
-  // block among 64 rows; short ones (speculative drafts, decode) use 16-row warp tiles
-  const bool coop = (long long)num_tokens * G > (long long)kTileRows * num_seqs;
-  const ExtLaunch k = q_dtype == PA_BF16 ? ext_pick_d<PA_BF16>(D, BS, G, coop) : ext_pick_d<PA_F16>(D, BS, G, coop);
-  if (!k.fn) return PA_ERR_ARG;
+  // Long query runs (at least half a 128-row tile per sequence on average) go to the
+  // tcgen05 kernel (head_dim 128) or, otherwise, the cooperative 64-row kernel; short
+  // ones (speculative drafts, decode) to the 16-row warp kernel.
+  const long long rows_total = (long long)num_tokens * G;
+  const bool tc = rows_total * 2 >= (long long)kTcUnitRows * num_seqs && extend_tc_supported(q_dtype, D, BS, G);
+  const bool coop = !tc && rows_total > (long long)kTileRows * num_seqs;
+  ExtLaunch k;
+  if (!tc) {
+    k = q_dtype == PA_BF16 ? ext_pick_d<PA_BF16>(D, BS, G, coop) : ext_pick_d<PA_F16>(D, BS, G, coop);
+    if (!k.fn) return PA_ERR_ARG;
+  }
 
   ExtendParams p;
   p.q = q;
@@ -858,23 +885,45 @@ pa_status pa_extend(const void* q, int32_t q_dtype, int32_t num_seqs, int32_t nu
   p.out_row_bytes = num_q_heads * D * 2;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
-  extend_plan_kernel<<<1, 1024, 0, s>>>(p, (coop ? kCoopRows : kTileRows) / G);
+  const int rows_per_unit = tc ? kTcUnitRows : coop ? kCoopRows : kTileRows;
+  // upper bound of the row tiles: every sequence's queries plus one ragged tile each
+  const long long tiles = (rows_total + rows_per_unit - 1) / rows_per_unit + num_seqs;
+  int grid = 1;
+  p.chunk = kPartitionTokens;
+  if (tc) {
+    // the whole context per unit when that already gives two units per SM; otherwise
+    // the largest multiple of the partition length that does (split-K + merge)
+    int cap = 0;
+    if (extend_tc_grid_cap(q_dtype, BS, G, &cap) != cudaSuccess) return PA_ERR_CUDA;
+    int nchunks = 1;
+    while (nchunks < max_parts && tiles * c->num_kv_heads * nchunks < 2LL * cap) ++nchunks;
+    const int parts_per_chunk = (max_parts + nchunks - 1) / nchunks;
+    p.chunk = parts_per_chunk * kPartitionTokens;
+    const long long units = tiles * c->num_kv_heads * ((max_parts + parts_per_chunk - 1) / parts_per_chunk);
+    grid = int(units < cap ? units : cap);
+  } else {
+    int cap = 0;
+    Launch as_launch;
+    as_launch.fn = reinterpret_cast<KernelFn>(k.fn);
+    as_launch.smem = k.smem;
+    as_launch.threads = k.threads;
+    if (occupancy(as_launch, &cap) != cudaSuccess) return PA_ERR_CUDA;
+    const long long units = tiles * c->num_kv_heads * max_parts;
+    // the warp kernel runs 4 independent units per CTA, the cooperative one a unit per CTA
+    const long long ctas = coop ? units : (units + ExtCfg<128, 16>::kWarps - 1) / ExtCfg<128, 16>::kWarps;
+    grid = int(ctas < cap ? ctas : cap);
+  }
+  if (grid < 1) grid = 1;
+
+  extend_plan_kernel<<<1, 1024, 0, s>>>(p, rows_per_unit / G);
   if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
-  int cap = 0;
-  Launch as_launch;
-  as_launch.fn = reinterpret_cast<KernelFn>(k.fn);
-  as_launch.smem = k.smem;
-  as_launch.threads = k.threads;
-  if (occupancy(as_launch, &cap) != cudaSuccess) return PA_ERR_CUDA;
-  // upper bound of the units: every tile of every sequence in every partition
-  const int rows_per_unit = coop ? kCoopRows : kTileRows;
-  const long long tiles = ((long long)num_tokens * G + rows_per_unit - 1) / rows_per_unit + num_seqs;
-  const long long units = tiles * c->num_kv_heads * max_parts;
-  // the warp kernel runs 4 independent units per CTA, the cooperative one a unit per CTA
-  const long long ctas = coop ? units : (units + ExtCfg<128, 16>::kWarps - 1) / ExtCfg<128, 16>::kWarps;
-  const int grid = int(ctas < cap ? ctas : cap);
-  if (ext_launch(k.fn, grid > 0 ? grid : 1, k.threads, k.smem, s, p) != cudaSuccess) return PA_ERR_CUDA;
-  if (max_parts > 1) {
+  if (tc) {
+    st = extend_tc_launch(p, c, q_dtype, G, grid, s);
+    if (st != PA_OK) return st;
+  } else if (ext_launch(k.fn, grid, k.threads, k.smem, s, p) != cudaSuccess) {
+    return PA_ERR_CUDA;
+  }
+  if (max_parts * kPartitionTokens > p.chunk) {   // some row spans several chunks
     const long long rows = (long long)num_tokens * num_q_heads;
     ExtKernel red = q_dtype == PA_BF16 ? (D == 64 ? extend_reduce_kernel<PA_BF16, 64> : extend_reduce_kernel<PA_BF16, 128>)
                                        : (D == 64 ? extend_reduce_kernel<PA_F16, 64> : extend_reduce_kernel<PA_F16, 128>);

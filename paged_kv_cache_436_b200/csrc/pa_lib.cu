@@ -3,3 +3,4 @@
 #include "pa_decode.cu"
 #include "pa_cache.cu"
 #include "pa_extend.cu"
+#include "pa_extend_tc.cu"

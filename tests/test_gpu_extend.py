@@ -97,3 +97,90 @@ def test_more_queries_than_context_is_recorded_and_zero():
     code, info = pa.last_device_error()
     assert code == 2 and info[0] == 0
     assert torch.count_nonzero(out[:3]) == 0 and torch.isfinite(out[3:].float()).all()
+
+
+def _nan_tails(w, eng):
+    """Cache bytes past each context in its last block set to NaN: memory that was never
+    written may hold anything, and no output may depend on it."""
+    BS = w.block_size
+    for s, L in enumerate(eng.lens):
+        if L % BS:
+            b = int(eng.bt_host[s, (L - 1) // BS])
+            eng.k_cache[b, :, L % BS:, :] = float("nan")
+            eng.v_cache[b, :, L % BS:, :] = float("nan")
+
+
+def _sample_rows(qs, Hq, n, seed):
+    """Random (token, head) rows plus the first and last query of every sequence."""
+    T = int(qs[-1])
+    rng = np.random.default_rng(seed)
+    rows = {(int(t), int(h)) for t, h in zip(rng.integers(0, T, n), rng.integers(0, Hq, n))}
+    for s in range(len(qs) - 1):
+        if qs[s + 1] > qs[s]:
+            for t in (int(qs[s]), int(qs[s + 1]) - 1):
+                rows.update((t, h) for h in range(Hq))
+    return sorted(rows)
+
+
+def _check_rows(w, eng, q, qs, out, rows, what):
+    ref = _ref(w, eng, q, qs, rows=rows)
+    idx = tuple(np.array(rows).T)
+    got = out.double().cpu().numpy()
+    assert np.isfinite(got[idx]).all(), what
+    assert_close(got[idx], ref[idx], w.kv_dtype, what)
+
+
+@pytest.mark.parametrize("dt,BS,G", [("bf16", 16, 1), ("f16", 16, 2), ("bf16", 32, 4), ("f16", 32, 8),
+                                     ("bf16", 16, 8), ("f16", 16, 1)])
+def test_long_runs_split_context(dt, BS, G):
+    """Long query runs (the 128-row tensor-core path): whole prompts, a chunk over a
+    longer context, a single query and a two-token draft in one batch; few units, so
+    the context is split into chunks merged by log-sum-exp. NaN past every context."""
+    lens = [130, 700, 1025, 257, 1, 1500]
+    qlens = [130, 700, 300, 257, 1, 2]
+    seed = zlib.crc32(repr(("long", dt, BS, G)).encode()) % 10000
+    w, eng, qs_dev, q, qs = _setup(lens, qlens, 2 * G, 2, 128, BS, dt, seed)
+    _nan_tails(w, eng)
+    out = _run(w, eng, qs_dev, q, qs)
+    assert pa.last_device_error()[0] == 0
+    _check_rows(w, eng, q, qs, out, _sample_rows(qs, 2 * G, 160, seed), f"long runs {dt} BS{BS} G{G}")
+
+
+def test_long_runs_whole_context_per_unit():
+    """Enough 128-row tiles to fill the GPU: every unit covers its rows' whole context
+    and writes the output directly (no merge pass)."""
+    lens = [1200, 1100, 1000, 1200]
+    w, eng, qs_dev, q, qs = _setup(lens, lens, 8, 8, 128, 16, "bf16", 77)
+    _nan_tails(w, eng)
+    out = _run(w, eng, qs_dev, q, qs)
+    assert pa.last_device_error()[0] == 0
+    _check_rows(w, eng, q, qs, out, _sample_rows(qs, 8, 200, 77), "whole-context units")
+    # query 0 of each prompt sees its token 0 only: the output is that V row exactly
+    for s in range(len(lens)):
+        v0 = eng.v_cache[int(eng.bt_host[s, 0]), :, 0, :]
+        assert torch.equal(out[int(qs[s])], v0)
+
+
+def test_prefill_8x2k_sampled():
+    """The benchmarked prefill shapes (8 prompts of 2048 tokens, 32 heads, head_dim 128,
+    bf16, 16-token blocks), checked on sampled rows."""
+    w, eng, qs_dev, q, qs = _setup([2048] * 8, [2048] * 8, 32, 32, 128, 16, "bf16", 4371)
+    out = _run(w, eng, qs_dev, q, qs)
+    assert pa.last_device_error()[0] == 0
+    _check_rows(w, eng, q, qs, out, _sample_rows(qs, 32, 120, 4371), "prefill 8x2k")
+
+
+def test_short_runs_ignore_bytes_past_the_context():
+    """The 16- and 64-row kernels never let cache bytes past the context reach P V."""
+    lens, qlens = [37, 530, 1031], [3, 5, 2]                 # 16-row warp kernel
+    w, eng, qs_dev, q, qs = _setup(lens, qlens, 4, 2, 128, 16, "bf16", 91)
+    _nan_tails(w, eng)
+    out = _run(w, eng, qs_dev, q, qs)
+    assert pa.last_device_error()[0] == 0
+    _check_rows(w, eng, q, qs, out, _sample_rows(qs, 4, 0, 91) + [(1, 1), (6, 3)], "warp kernel tails")
+    lens, qlens = [300, 77], [200, 60]                       # 64-row cooperative kernel (head_dim 64)
+    w, eng, qs_dev, q, qs = _setup(lens, qlens, 4, 2, 64, 16, "f16", 92)
+    _nan_tails(w, eng)
+    out = _run(w, eng, qs_dev, q, qs)
+    assert pa.last_device_error()[0] == 0
+    _check_rows(w, eng, q, qs, out, _sample_rows(qs, 4, 80, 92), "cooperative kernel tails")
