@@ -513,6 +513,38 @@ def workload_config(w, n_gpus):
             "parallelism": f"replicas{n_gpus}" if n_gpus > 1 else "single GPU"}
 
 
+EXTEND_WORKLOADS = ("spec4_mix", "prefill_8x2k")
+
+
+def extend_roofline(e, hbm_peak):
+    import json as _json
+    with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+        bf16_peak = float(_json.load(f).get("bf16_tflops", 1645.7))
+    spec = e["workload"].startswith("spec")
+    r = {"bound": "hbm" if spec else "tensor", "achieved": e["kv_gbs"] if spec else e["tflops"],
+         "peak": hbm_peak if spec else bf16_peak, "unit": "GB/s" if spec else "TFLOP/s"}
+    r["frac"] = r["achieved"] / r["peak"]
+    return r
+
+
+def extend_only(args, world, rank, local):
+    """`--workload spec4_mix|prefill_8x2k`: pa_extend alone on one GPU (a profiling and
+    tuning entry; the default line reports these under "extend")."""
+    import torch
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the product path has no CPU fallback)")
+    import paged_kv_cache_436_b200 as pa
+    pa.lib()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    e = time_extend(args.workload, args.steps, args.warmup, device)
+    peak, _ = peaks()
+    e["roofline"] = extend_roofline(e, peak)
+    if rank == 0:
+        print(json.dumps(e))
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -531,6 +563,8 @@ def main(argv=None):
 
     import synthetic
     world, rank, local = dist_env()
+    if args.workload in EXTEND_WORKLOADS:
+        return extend_only(args, world, rank, local)
     w = synthetic.make(args.workload)
     if args.subset:
         w = synthetic.subset(w, args.subset)
@@ -555,7 +589,7 @@ def main(argv=None):
         also = []
         extend_entries = []
         for name in [a for a in args.also.split(",") if a]:
-            if name in ("spec4_mix", "prefill_8x2k"):
+            if name in EXTEND_WORKLOADS:
                 extend_entries.append(time_extend(name, max(3, args.steps // 5), args.warmup, device))
                 continue
             if name == "beam5":
@@ -617,17 +651,9 @@ def main(argv=None):
                                  "it is read from HBM about once and from L2 after that")
                 entry["prefix_cache"] = ra.get("prefix_report")
             line.setdefault("also", []).append(entry)
-        if extend_entries:
-            import json as _json
-            with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
-                bf16_peak = float(_json.load(f).get("bf16_tflops", 1645.7))
-            for e in extend_entries:
-                e["roofline"] = {"bound": "hbm" if e["workload"].startswith("spec") else "tensor",
-                                 "achieved": e["kv_gbs"] if e["workload"].startswith("spec") else e["tflops"],
-                                 "peak": peak if e["workload"].startswith("spec") else bf16_peak,
-                                 "unit": "GB/s" if e["workload"].startswith("spec") else "TFLOP/s"}
-                e["roofline"]["frac"] = e["roofline"]["achieved"] / e["roofline"]["peak"]
-                line.setdefault("extend", []).append(e)
+        for e in extend_entries:
+            e["roofline"] = extend_roofline(e, peak)
+            line.setdefault("extend", []).append(e)
         if rank == 0 and world == 1 and not args.no_cpu:
             line["cpu_baseline"] = cpu_baseline_obj(w, args.cpu_budget)
         if rank == 0:

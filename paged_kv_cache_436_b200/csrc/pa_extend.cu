@@ -852,7 +852,8 @@ pa_status pa_extend(const void* q, int32_t q_dtype, int32_t num_seqs, int32_t nu
   // tcgen05 kernel (head_dim 128) or, otherwise, the cooperative 64-row kernel; short
   // ones (speculative drafts, decode) to the 16-row warp kernel.
   const long long rows_total = (long long)num_tokens * G;
-  const bool tc = rows_total * 2 >= (long long)kTcUnitRows * num_seqs && extend_tc_supported(q_dtype, D, BS, G);
+  const bool tc = rows_total * 2 >= (long long)kTcUnitRows * num_seqs && scale > 0.f &&
+                  extend_tc_supported(q_dtype, D, BS, G);
   const bool coop = !tc && rows_total > (long long)kTileRows * num_seqs;
   ExtLaunch k;
   if (!tc) {

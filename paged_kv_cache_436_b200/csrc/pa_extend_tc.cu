@@ -34,16 +34,18 @@ namespace pa {
 constexpr int kTcRows = 128;            // query rows per unit (TMEM lanes)
 constexpr int kTcTok = 128;             // tokens per K/V tile
 constexpr int kTcD = 128;               // head_dim of this path
-constexpr uint32_t kTcTmemCols = 256;   // S and O
+constexpr uint32_t kTcTmemCols = 512;   // S double buffer [0, 256), O double buffer [256, 512)
+constexpr int kTcSoftmaxWarps = 4;      // + one MMA-issue warp + one TMA producer warp
+constexpr int kTcThreads = (kTcSoftmaxWarps + 2) * 32;
 constexpr float kTcRescale = 8.f;       // log2 units
 
 struct TcSmem {
   static constexpr int kTile = kTcRows * kTcD * 2;   // 32 KB: two 64-column halves of 16 KB
   static constexpr int kQ = 0;
-  static constexpr int kP = kQ + kTile;
-  static constexpr int kK = kP + kTile;              // K buffers 0, 1
+  static constexpr int kP = kQ + kTile;              // P buffers 0, 1
+  static constexpr int kK = kP + 2 * kTile;          // K buffers 0, 1
   static constexpr int kV = kK + 2 * kTile;          // V buffers 0, 1
-  static constexpr int kBytes = kV + 2 * kTile + 1024;   // + alignment slack
+  static constexpr int kBytes = kV + 2 * kTile + 1024;   // 225 KB with the alignment slack
 };
 static_assert(kTcRows == kTcTok, "Q, P, K and V tiles share one swizzled layout");
 
@@ -99,6 +101,24 @@ __device__ __forceinline__ void tc_ld32(uint32_t addr, float* v) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// The same load without its wait: issue several, then one tc_wait_ld(), then read the
+// registers through pin_after_wait() so that no use is scheduled before the wait.
+__device__ __forceinline__ void tc_ld32_async(uint32_t addr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(addr));
+}
+__device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ uint32_t pin_after_wait(uint32_t x) {
+  asm volatile("" : "+r"(x));
+  return x;
+}
+
 __device__ __forceinline__ void tc_st32(uint32_t addr, const float* v) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
@@ -116,6 +136,23 @@ __device__ __forceinline__ void tc_st32(uint32_t addr, const float* v) {
       "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
       : "memory");
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// Two values rounded to the 16-bit type and packed (lo in the low half); `sum` adds the
+// rounded values.
+template <int QD>
+__device__ __forceinline__ uint32_t pack2_sum(float lo, float hi, float& sum) {
+  if constexpr (QD == PA_BF16) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    const uint32_t w = *reinterpret_cast<const uint32_t*>(&v);
+    sum += __uint_as_float(w << 16) + __uint_as_float(w & 0xffff0000u);
+    return w;
+  } else {
+    __half2 v = __floats2half2_rn(lo, hi);
+    const float2 f = __half22float2(v);
+    sum += f.x + f.y;
+    return *reinterpret_cast<const uint32_t*>(&v);
+  }
 }
 
 // 2^x on the special-function unit (flushes subnormal results to zero).
@@ -140,21 +177,66 @@ __device__ __forceinline__ uint32_t tc_swz(int r, int c) {
   return uint32_t((c >> 3) * (kTcRows * 128) + (r >> 3) * 1024 + (r & 7) * 128 + (((c & 7) ^ (r & 7)) << 4));
 }
 
+// Geometry of one work unit as every role of the CTA computes it.
+struct TcUnit {
+  int s, hk, t, part;
+  int Q, base, row0;
+  int t0, nvis, ntiles;     // first context token of the chunk, visible tokens, K/V tiles
+};
+
+__device__ __forceinline__ TcUnit tc_unit(const ExtendParams& p, int u, int total, int qpt) {
+  const ExtUnit x = ext_make_unit<16>(p, u, total, qpt, 64);   // no block-id reads
+  TcUnit t;
+  t.s = x.s;
+  t.hk = x.hk;
+  t.t = x.t;
+  t.part = x.part;
+  t.Q = x.Q;
+  t.base = x.base;
+  t.row0 = x.row0;
+  t.t0 = x.part * p.chunk;
+  t.nvis = min(p.chunk, x.last + 1 - t.t0);
+  t.ntiles = (t.nvis + kTcTok - 1) / kTcTok;
+  return t;
+}
+
+// Bounded wait that also gives up as soon as another role of the CTA has aborted.
+__device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int where, int u) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if (global_timer_ns() - t0 > 2000000000ull) {
+      record_error(PA_DEV_WAIT_TIMEOUT, where, u, int(parity));
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
+// Warp-uniform form: true only if every lane's wait succeeded.
+__device__ __forceinline__ bool tc_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort, int where, int u) {
+  return __all_sync(kFull, tc_wait(bar, parity, abort, where, u));
+}
+
 template <int QD, int BS, int G>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(192, 1)
     extend_tc_kernel(const ExtendParams p, const __grid_constant__ CUtensorMap tk,
                      const __grid_constant__ CUtensorMap tv) {
   using QT = typename Q<QD>::T;
-  constexpr int QPT = kTcRows / G;             // queries per unit
-  constexpr int BPT = kTcTok / BS;             // cache blocks per K/V tile
-  constexpr uint32_t kBlockTx = 2u * BS * kTcD * 2;   // K and V bytes of one cache block
+  constexpr int QPT = kTcRows / G;                    // queries per unit
+  constexpr int BPT = kTcTok / BS;                    // cache blocks per K/V tile
+  constexpr uint32_t kBlockTx = BS * kTcD * 2;        // bytes of one cache block of K (or V)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = sm + TcSmem::kQ;
-  uint8_t* sP = sm + TcSmem::kP;
-  __shared__ uint64_t bar_kv[2], bar_s, bar_o, bar_fin;
+  // per-tile ring barriers (index = tile & 1); per-unit ones (q_full, o_full/o_empty by unit & 1)
+  __shared__ uint64_t k_full[2], v_full[2], k_empty[2], pv_done[2], s_full[2], s_empty[2], p_full[2];
+  __shared__ uint64_t q_full, o_full[2], o_empty[2], bar_fin;
   __shared__ uint32_t tmem_slot;
-  __shared__ int s_fail;
+  __shared__ int s_abort;
+  volatile int* abort = &s_abort;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   if (warp == 0) {
@@ -163,13 +245,21 @@ __global__ void __launch_bounds__(128, 1)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
-  if (tid == 0) {
-    mbar_init(&bar_kv[0], 1);
-    mbar_init(&bar_kv[1], 1);
-    mbar_init(&bar_s, 1);
-    mbar_init(&bar_o, 1);
+  if (tid == 32) {
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&k_full[b], 1);
+      mbar_init(&v_full[b], 1);
+      mbar_init(&k_empty[b], 1);
+      mbar_init(&pv_done[b], 1);
+      mbar_init(&s_full[b], 1);
+      mbar_init(&s_empty[b], kTcSoftmaxWarps);
+      mbar_init(&p_full[b], kTcSoftmaxWarps);
+      mbar_init(&o_full[b], 1);
+      mbar_init(&o_empty[b], kTcSoftmaxWarps);
+    }
+    mbar_init(&q_full, kTcSoftmaxWarps);
     mbar_init(&bar_fin, 1);
-    s_fail = 0;
+    s_abort = 0;
     fence_mbar_init();
   }
   tc_fence_before();
@@ -179,229 +269,272 @@ __global__ void __launch_bounds__(128, 1)
   grid_dependency_wait();
 
   const uint32_t tmem = tmem_slot;
-  const uint32_t t_row = tmem + (uint32_t(warp * 32) << 16);   // this warp's 32 lanes, column 0
   const int Hq = p.num_q_heads, Hkv = p.num_kv_heads;
   const int total = p.plan[p.num_seqs] * Hkv;
-  const uint32_t idS = tc_idesc<QD>(0), idO = tc_idesc<QD>(1);
-  uint32_t it = 0;                          // K/V tiles this CTA has used (buffer it & 1)
-  uint32_t pending = 0, par[2] = {0, 0};    // thread 0: loads issued and not yet waited for
+  uint32_t last_load = 0;           // producer: tiles issued (for the drain after an abort)
 
-  for (int u = blockIdx.x; u < total; u += gridDim.x) {
-    const ExtUnit x = ext_make_unit<16>(p, u, total, QPT, 64);   // geometry only (no block ids)
-    const int qi = x.t * QPT + tid / G;
-    const int head = x.hk * G + tid % G;
-    const bool has_q = qi < x.Q;
-    const int qpos = has_q ? x.base + qi : -1;
-    const int tok = has_q ? x.row0 + qi : -1;
-    const int last = x.base + min((x.t + 1) * QPT, x.Q) - 1;   // last position the unit's rows see
-    const int t0 = x.part * p.chunk;
-    const int nvis = min(p.chunk, last + 1 - t0);                // visible tokens of the chunk (>= 1)
-    const int ntiles = (nvis + kTcTok - 1) / kTcTok;
-
-    {   // this thread's Q row -> swizzled K-major tile (zero for rows without a query)
-      const uint4* qrow =
-          reinterpret_cast<const uint4*>(static_cast<const QT*>(p.q) + (size_t(has_q ? tok : 0) * Hq + head) * kTcD);
-#pragma unroll
-      for (int c = 0; c < 16; ++c)
-        *reinterpret_cast<uint4*>(sQ + tc_swz(tid, c)) = has_q ? qrow[c] : make_uint4(0, 0, 0, 0);
-    }
-    fence_async_smem();
-    __syncthreads();
-
-    // K/V tile j of the unit into buffer g & 1, issued by warp 0: lane i loads cache
-    // block i of the tile (only the blocks with visible tokens). The block ids are read
-    // one tile ahead so that their latency hides behind the current tile's S = Q K^T.
-    const int32_t* trow = p.block_tables + size_t(x.s) * p.max_blocks;
-    auto tile_blocks = [&](int j) { return min(BPT, (nvis - j * kTcTok + BS - 1) / BS); };
-    auto fetch_id = [&](int j) {
-      const int lb = (t0 + j * kTcTok) / BS + lane;
-      int id = 0;
-      if (lane < tile_blocks(j)) {
-        id = trow[lb];
-        if (id < 0 || id >= p.num_blocks) {
-          record_error(PA_DEV_BAD_BLOCK_ID, x.s, lb, id);
-          id = 0;
+  if (warp == kTcSoftmaxWarps + 1) {
+    // ---------------- producer: K and V tiles by 2-D TMA, lane i loads cache block i ----------------
+    uint32_t g = 0;
+    for (int u = blockIdx.x; u < total && !*abort; u += gridDim.x) {
+      const TcUnit x = tc_unit(p, u, total, QPT);
+      const int32_t* trow = p.block_tables + size_t(x.s) * p.max_blocks;
+      auto blocks = [&](int j) { return min(BPT, (x.nvis - j * kTcTok + BS - 1) / BS); };
+      auto fetch = [&](int j) {   // block id of this lane's block of tile j
+        const int lb = (x.t0 + j * kTcTok) / BS + lane;
+        int id = 0;
+        if (lane < blocks(j)) {
+          id = trow[lb];
+          if (id < 0 || id >= p.num_blocks) {
+            record_error(PA_DEV_BAD_BLOCK_ID, x.s, lb, id);
+            id = 0;
+          }
         }
+        return id;
+      };
+      int id = fetch(0);
+      for (int j = 0; j < x.ntiles; ++j, ++g) {
+        const int b = g & 1, nb = blocks(j);
+        const int next = j + 1 < x.ntiles ? fetch(j + 1) : 0;   // read ahead of its use
+        const int y = (id * Hkv + x.hk) * BS;
+        const uint32_t off = b * TcSmem::kTile + lane * (BS * 128);
+        if (!tc_wait_warp(&k_empty[b], ((g >> 1) & 1) ^ 1, abort, 10, u)) break;
+        if (lane == 0) mbar_arrive_expect_tx(&k_full[b], uint32_t(nb) * kBlockTx);
+        __syncwarp();
+        if (lane < nb) {
+          tma_load_2d(sm + TcSmem::kK + off, &tk, 0, y, &k_full[b]);
+          tma_load_2d(sm + TcSmem::kK + off + kTcTok * 128, &tk, 64, y, &k_full[b]);
+        }
+        if (!tc_wait_warp(&pv_done[b], ((g >> 1) & 1) ^ 1, abort, 11, u)) {
+          last_load = g + 1;
+          break;
+        }
+        if (lane == 0) mbar_arrive_expect_tx(&v_full[b], uint32_t(nb) * kBlockTx);
+        __syncwarp();
+        if (lane < nb) {
+          tma_load_2d(sm + TcSmem::kV + off, &tv, 0, y, &v_full[b]);
+          tma_load_2d(sm + TcSmem::kV + off + kTcTok * 128, &tv, 64, y, &v_full[b]);
+        }
+        last_load = g + 1;
+        id = next;
       }
-      return id;
-    };
-    auto issue_tile = [&](int j, uint32_t g, int id) {
-      const int b = g & 1;
-      const int nb = tile_blocks(j);
+    }
+  } else if (warp == kTcSoftmaxWarps) {
+    // ---------------- MMA issue: S(g) then O += P(g-1) V(g-1) ----------------
+    const uint32_t idS = tc_idesc<QD>(0), idO = tc_idesc<QD>(1);
+    uint32_t g = 0, k = 0;
+    auto pv = [&](uint32_t h, bool first, uint32_t ob, int u) {
+      const int b = h & 1;
+      if (!tc_wait_warp(&p_full[b], (h >> 1) & 1, abort, 12, u)) return false;
+      if (!tc_wait_warp(&v_full[b], (h >> 1) & 1, abort, 13, u)) return false;
       if (lane == 0) {
-        mbar_arrive_expect_tx(&bar_kv[b], uint32_t(nb) * kBlockTx);
-        pending |= 1u << b;
-        par[b] = (g >> 1) & 1;
+        tc_fence_after();
+        const uint32_t pa_ = smem_addr(sm + TcSmem::kP + b * TcSmem::kTile);
+        const uint32_t va = smem_addr(sm + TcSmem::kV + b * TcSmem::kTile);
+#pragma unroll
+        for (int kk = 0; kk < kTcTok / 16; ++kk) {
+          const uint32_t aoff = (kk >> 2) * (kTcRows * 128) + (kk & 3) * 32;
+          tc_mma(tmem + 256 + ob * 128, tc_desc(pa_ + aoff, 1024, 16), tc_desc(va + kk * 2048, 1024, kTcTok * 128),
+                 idO, (first && kk == 0) ? 0u : 1u);
+        }
+        tc_commit(&pv_done[b]);
       }
       __syncwarp();
-      if (lane < nb) {
-        uint8_t* dk = sm + TcSmem::kK + b * TcSmem::kTile + lane * (BS * 128);
-        uint8_t* dv = sm + TcSmem::kV + b * TcSmem::kTile + lane * (BS * 128);
-        const int y = (id * Hkv + x.hk) * BS;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          tma_load_2d(dk + h * (kTcTok * 128), &tk, h * 64, y, &bar_kv[b]);
-          tma_load_2d(dv + h * (kTcTok * 128), &tv, h * 64, y, &bar_kv[b]);
-        }
-      }
+      return true;
     };
-    if (warp == 0) issue_tile(0, it, fetch_id(0));
-
-    float m_ref = -INFINITY, l = 0.f;
-    for (int j = 0; j < ntiles; ++j, ++it) {
-      const int b = it & 1;
-      int next_id = 0;
-      if (warp == 0 && j + 1 < ntiles) next_id = fetch_id(j + 1);
-      if (tid == 0) {   // S = Q K^T into columns [0, 128)
-        if (!mbar_wait_bounded(&bar_kv[b], (it >> 1) & 1)) {
-          record_error(PA_DEV_WAIT_TIMEOUT, 5, u, j);
-          s_fail = 1;
-        } else {
-          pending &= ~(1u << b);
+    for (int u = blockIdx.x; u < total && !*abort; u += gridDim.x, ++k) {
+      const TcUnit x = tc_unit(p, u, total, QPT);
+      const uint32_t ob = k & 1;
+      if (!tc_wait_warp(&q_full, k & 1, abort, 14, u)) break;
+      if (!tc_wait_warp(&o_empty[ob], ((k >> 1) & 1) ^ 1, abort, 15, u)) break;
+      bool ok = true;
+      for (int j = 0; j < x.ntiles && ok; ++j, ++g) {
+        const int b = g & 1;
+        ok = tc_wait_warp(&k_full[b], (g >> 1) & 1, abort, 16, u) &&
+             tc_wait_warp(&s_empty[b], ((g >> 1) & 1) ^ 1, abort, 17, u);
+        if (!ok) break;
+        if (lane == 0) {
           tc_fence_after();
           const uint32_t qa = smem_addr(sQ), ka = smem_addr(sm + TcSmem::kK + b * TcSmem::kTile);
 #pragma unroll
           for (int kk = 0; kk < kTcD / 16; ++kk) {
             const uint32_t off = (kk >> 2) * (kTcRows * 128) + (kk & 3) * 32;
-            tc_mma(tmem, tc_desc(qa + off, 1024, 16), tc_desc(ka + off, 1024, 16), idS, kk > 0);
+            tc_mma(tmem + b * 128, tc_desc(qa + off, 1024, 16), tc_desc(ka + off, 1024, 16), idS, kk > 0);
           }
-          tc_commit(&bar_s);
+          tc_commit(&s_full[b]);
+          tc_commit(&k_empty[b]);
         }
+        __syncwarp();
+        if (j > 0) ok = pv(g - 1, j == 1, ob, u);
       }
-      __syncthreads();
-      if (s_fail) break;
-      // S is in TMEM; the previous tile's P V is done too (P, O and that K/V buffer are free)
-      bool ok = mbar_wait_bounded(&bar_s, it & 1);
-      if (it > 0) ok = ok && mbar_wait_bounded(&bar_o, (it - 1) & 1);
-      if (!__all_sync(kFull, ok) && (tid & 31) == 0) {
-        record_error(PA_DEV_WAIT_TIMEOUT, 6, u, j);
-        s_fail = 1;
-      }
-      __syncthreads();
-      if (s_fail) break;
-      tc_fence_after();
-      if (warp == 0 && j + 1 < ntiles) issue_tile(j + 1, it + 1, next_id);
-
-      // V rows past the visible tokens (cache bytes beyond the context, or stale rows of
-      // blocks not loaded) are zeroed so that 0-weighted rows cannot carry a NaN into O
-      const int rem = nvis - j * kTcTok;
-      if (tid >= rem) {
-        uint8_t* vrow = sm + TcSmem::kV + b * TcSmem::kTile + (tid >> 3) * 1024 + (tid & 7) * 128;
+      if (!ok || !pv(g - 1, x.ntiles == 1, ob, u)) break;
+      if (lane == 0) tc_commit(&o_full[ob]);
+      __syncwarp();
+    }
+  } else {
+    // ---------------- softmax warps: thread tid owns row tid of the unit ----------------
+    const uint32_t t_row = tmem + (uint32_t(warp * 32) << 16);
+    auto write_q = [&](const TcUnit& x) {
+      const int qi = x.t * QPT + tid / G;
+      const bool has_q = qi < x.Q;
+      const uint4* qrow = reinterpret_cast<const uint4*>(
+          static_cast<const QT*>(p.q) + (size_t(has_q ? x.row0 + qi : 0) * Hq + x.hk * G + tid % G) * kTcD);
 #pragma unroll
-        for (int h = 0; h < 2; ++h)
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<uint4*>(vrow + h * (kTcTok * 128) + c * 16) = make_uint4(0, 0, 0, 0);
-      }
-
-      // softmax of this thread's row (base 2; scale * log2(e) applied here)
-      float s[kTcTok];
-#pragma unroll
-      for (int c = 0; c < kTcTok / 32; ++c) tc_ld32(t_row + c * 32, s + c * 32);
-      const int tp0 = t0 + j * kTcTok;
-      float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < kTcTok; ++c) {
-        const float v = tp0 + c > qpos ? -INFINITY : s[c] * p.s_mul;
-        s[c] = v;
-        mx = fmaxf(mx, v);
-      }
-      const bool up = mx > m_ref + kTcRescale;
-      const float corr = up ? ex2(m_ref - mx) : 1.f;   // 0 while nothing was accumulated
-      if (up) {
-        l *= corr;
-        m_ref = mx;
-      }
-      if (j > 0 && __any_sync(kFull, up)) {   // rescale the O rows of this warp that moved
-#pragma unroll 1
-        for (int c = 0; c < kTcD / 32; ++c) {
-          float o[32];
-          tc_ld32(t_row + 128 + c * 32, o);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] *= corr;
-          tc_st32(t_row + 128 + c * 32, o);
-        }
-      }
-      const float mb = m_ref == -INFINITY ? 0.f : m_ref;
-#pragma unroll
-      for (int c = 0; c < kTcTok / 8; ++c) {
-        uint32_t w[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          float r0, r1;
-          w[e] = pack2<QD>(ex2(s[c * 8 + 2 * e] - mb), ex2(s[c * 8 + 2 * e + 1] - mb), r0, r1);
-          l += r0 + r1;
-        }
-        *reinterpret_cast<uint4*>(sP + tc_swz(tid, c)) = make_uint4(w[0], w[1], w[2], w[3]);
-      }
+      for (int c = 0; c < 16; ++c)
+        *reinterpret_cast<uint4*>(sQ + tc_swz(tid, c)) = has_q ? qrow[c] : make_uint4(0, 0, 0, 0);
       fence_async_smem();
-      tc_fence_before();
-      __syncthreads();
-      if (tid == 0) {   // O += P V into columns [128, 256)
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&q_full);
+    };
+    uint32_t g = 0, k = 0;
+    if (blockIdx.x < total) write_q(tc_unit(p, blockIdx.x, total, QPT));
+    for (int u = blockIdx.x; u < total; u += gridDim.x, ++k) {
+      const TcUnit x = tc_unit(p, u, total, QPT);
+      const uint32_t ob = k & 1, t_o = t_row + 256 + ob * 128;
+      const int qi = x.t * QPT + tid / G;
+      const int head = x.hk * G + tid % G;
+      const bool has_q = qi < x.Q;
+      const int qpos = has_q ? x.base + qi : -1;
+      const int tok = has_q ? x.row0 + qi : -1;
+      float m_ref = -INFINITY, l = 0.f;
+      bool ok = true;
+      for (int j = 0; j < x.ntiles; ++j, ++g) {
+        const int b = g & 1;
+        if (!(ok = tc_wait_warp(&s_full[b], (g >> 1) & 1, abort, 18, u))) break;
         tc_fence_after();
-        const uint32_t pa_ = smem_addr(sP), va = smem_addr(sm + TcSmem::kV + b * TcSmem::kTile);
+        float s[kTcTok];
+        {
+          uint32_t r[kTcTok];
 #pragma unroll
-        for (int kk = 0; kk < kTcTok / 16; ++kk) {
-          const uint32_t aoff = (kk >> 2) * (kTcRows * 128) + (kk & 3) * 32;
-          tc_mma(tmem + 128, tc_desc(pa_ + aoff, 1024, 16), tc_desc(va + kk * 2048, 1024, kTcTok * 128), idO,
-                 (j > 0 || kk > 0) ? 1u : 0u);
+          for (int c = 0; c < kTcTok / 32; ++c) tc_ld32_async(t_row + b * 128 + c * 32, r + c * 32);
+          tc_wait_ld();
+#pragma unroll
+          for (int c = 0; c < kTcTok; ++c) s[c] = __uint_as_float(pin_after_wait(r[c]));
         }
-        tc_commit(&bar_o);
-      }
-    }
-    if (s_fail) break;
-    {
-      const bool ok = mbar_wait_bounded(&bar_o, (it - 1) & 1);
-      if (!__all_sync(kFull, ok) && (tid & 31) == 0) {
-        record_error(PA_DEV_WAIT_TIMEOUT, 7, u, 0);
-        s_fail = 1;
-      }
-    }
-    __syncthreads();
-    if (s_fail) break;
-    tc_fence_after();
-
-    // the output row (whole context in this unit) or this chunk's partial
-    const int P = has_q ? (qpos + 1 + p.chunk - 1) / p.chunk : 0;
-    const bool wr = has_q && x.part < P;
-    const bool fin = wr && P == 1;
-    const float inv = fin ? 1.f / l : 0.f;
-    const size_t slot = (size_t(has_q ? tok : 0) * Hq + head) * p.max_parts + x.part;
-#pragma unroll 1
-    for (int c = 0; c < kTcD / 32; ++c) {
-      float o[32];
-      tc_ld32(t_row + 128 + c * 32, o);
-      if (fin) {
-        uint4* orow = reinterpret_cast<uint4*>(static_cast<QT*>(p.out) + (size_t(tok) * Hq + head) * kTcD + c * 32);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_empty[b]);
+        // causal mask, row maximum (8 independent chains)
+        const int tp0 = x.t0 + j * kTcTok;
+        if (tp0 + kTcTok - 1 > qpos) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+          for (int c = 0; c < kTcTok; ++c) s[c] = tp0 + c > qpos ? -INFINITY : s[c];
+        }
+        float m8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) m8[e] = s[e];
+#pragma unroll
+        for (int c = 8; c < kTcTok; ++c) m8[c & 7] = fmaxf(m8[c & 7], s[c]);
+        const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) *
+                         p.s_mul;
+        const bool up = mx > m_ref + kTcRescale;
+        const float corr = up ? ex2(m_ref - mx) : 1.f;   // 0 while nothing was accumulated
+        if (up) {
+          l *= corr;
+          m_ref = mx;
+        }
+        if (j > 0 && __any_sync(kFull, up)) {
+          // O must hold P(g-1) V(g-1) before it is rescaled
+          if (!(ok = tc_wait_warp(&pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1, abort, 19, u))) break;
+          tc_fence_after();
+#pragma unroll 1
+          for (int c = 0; c < kTcD / 32; ++c) {
+            float o[32];
+            tc_ld32(t_o + c * 32, o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] *= corr;
+            tc_st32(t_o + c * 32, o);
+          }
+        }
+        // P(g) into its buffer once P(g-2) V(g-2) has finished reading it
+        if (!(ok = tc_wait_warp(&pv_done[b], ((g >> 1) & 1) ^ 1, abort, 20, u))) break;
+        uint8_t* sP = sm + TcSmem::kP + b * TcSmem::kTile;
+        const float nmb = m_ref == -INFINITY ? 0.f : -m_ref;
+        float l8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < kTcTok / 8; ++c) {
           uint32_t w[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            float a, b2;
-            w[e] = pack2<QD>(o[i * 8 + 2 * e] * inv, o[i * 8 + 2 * e + 1] * inv, a, b2);
+          for (int e = 0; e < 4; ++e)
+            w[e] = pack2_sum<QD>(ex2(fmaf(s[c * 8 + 2 * e], p.s_mul, nmb)),
+                                 ex2(fmaf(s[c * 8 + 2 * e + 1], p.s_mul, nmb)), l8[(c & 1) * 4 + e]);
+          *reinterpret_cast<uint4*>(sP + tc_swz(tid, c)) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        l += ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
+        // V rows past the visible tokens (cache bytes beyond the context, or stale rows
+        // of blocks not loaded) are zeroed so that 0-weighted rows cannot bring a NaN
+        const int rem = x.nvis - j * kTcTok;
+        if (rem < kTcTok) {
+          if (!(ok = tc_wait_warp(&v_full[b], (g >> 1) & 1, abort, 21, u))) break;
+          if (tid >= rem) {
+            uint8_t* vrow = sm + TcSmem::kV + b * TcSmem::kTile + (tid >> 3) * 1024 + (tid & 7) * 128;
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+              for (int c = 0; c < 8; ++c)
+                *reinterpret_cast<uint4*>(vrow + h * (kTcTok * 128) + c * 16) = make_uint4(0, 0, 0, 0);
           }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[b]);
+      }
+      if (!ok) break;
+      // the next unit's Q (every S of this unit has completed), then this unit's O
+      if (u + (int)gridDim.x < total) write_q(tc_unit(p, u + gridDim.x, total, QPT));
+      if (!tc_wait_warp(&o_full[ob], (k >> 1) & 1, abort, 22, u)) break;
+      tc_fence_after();
+      const int P = has_q ? (qpos + 1 + p.chunk - 1) / p.chunk : 0;
+      const bool wr = has_q && x.part < P;
+      const bool fin = wr && P == 1;
+      const float inv = fin ? 1.f / l : 0.f;
+      const size_t slot = (size_t(has_q ? tok : 0) * Hq + head) * p.max_parts + x.part;
+      float o[kTcD];
+      {
+        uint32_t r[kTcD];
+#pragma unroll
+        for (int c = 0; c < kTcD / 32; ++c) tc_ld32_async(t_o + c * 32, r + c * 32);
+        tc_wait_ld();
+#pragma unroll
+        for (int c = 0; c < kTcD; ++c) o[c] = __uint_as_float(pin_after_wait(r[c]));
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&o_empty[ob]);
+      if (fin) {
+        uint4* orow = reinterpret_cast<uint4*>(static_cast<QT*>(p.out) + (size_t(tok) * Hq + head) * kTcD);
+#pragma unroll
+        for (int i = 0; i < kTcD / 8; ++i) {
+          float dummy = 0.f;
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) w[e] = pack2_sum<QD>(o[i * 8 + 2 * e] * inv, o[i * 8 + 2 * e + 1] * inv, dummy);
           orow[i] = make_uint4(w[0], w[1], w[2], w[3]);
         }
       } else if (wr) {
-        float4* acc = reinterpret_cast<float4*>(p.part_acc + slot * kTcD + c * 32);
+        float4* acc = reinterpret_cast<float4*>(p.part_acc + slot * kTcD);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+        for (int i = 0; i < kTcD / 4; ++i) acc[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+        p.part_ml[slot * 2] = m_ref;
+        p.part_ml[slot * 2 + 1] = l;
       }
     }
-    if (wr && !fin) {
-      p.part_ml[slot * 2] = m_ref;
-      p.part_ml[slot * 2 + 1] = l;
-    }
-    tc_fence_before();
-    __syncthreads();
   }
 
-  if (s_fail && tid == 0) {   // drain: MMAs issued so far, then outstanding loads
-    tc_commit(&bar_fin);
-    mbar_wait_bounded(&bar_fin, 0);
-    for (int b = 0; b < 2; ++b)
-      if (pending & (1u << b)) mbar_wait_bounded(&bar_kv[b], par[b]);
+  __syncthreads();
+  if (*abort) {   // drain what this CTA issued: MMAs (their thread), then loads (their warp)
+    if (warp == kTcSoftmaxWarps && lane == 0) {
+      tc_commit(&bar_fin);
+      mbar_wait_bounded(&bar_fin, 0);
+    }
+    if (warp == kTcSoftmaxWarps + 1 && lane == 0) {
+      for (uint32_t h = last_load >= 2 ? last_load - 2 : 0; h < last_load; ++h) {
+        mbar_wait_bounded(&k_full[h & 1], (h >> 1) & 1, 100000000ull);
+        mbar_wait_bounded(&v_full[h & 1], (h >> 1) & 1, 100000000ull);
+      }
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -469,7 +602,7 @@ cudaError_t extend_tc_grid_cap(int qd, int BS, int G, int* cap) {
   Launch l;
   l.fn = reinterpret_cast<KernelFn>(tc_pick(qd, BS, G));
   l.smem = TcSmem::kBytes;
-  l.threads = 128;
+  l.threads = kTcThreads;
   return occupancy(l, cap);
 }
 
@@ -487,7 +620,7 @@ pa_status extend_tc_launch(const ExtendParams& p, const pa_cache_desc* c, int qd
     return PA_ERR_ARG;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(128);
+  cfg.blockDim = dim3(kTcThreads);
   cfg.dynamicSmemBytes = TcSmem::kBytes;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
