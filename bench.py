@@ -359,7 +359,7 @@ def time_ours(w, steps, warmup, device, dist, e2e=True, clocks=True, local_rank=
     return res
 
 
-def time_extend(name, steps, warmup, device):
+def time_extend(name, steps, warmup, device, subset=0):
     """pa_extend alone (the tensor-core multi-query kernel and its merge), timed with
     CUDA events: `spec4_mix` = 4 draft tokens per sequence over the 13B mix contexts
     (speculative verification; HBM-bound), `prefill_8x2k` = 8 whole 2048-token prompts
@@ -369,7 +369,7 @@ def time_extend(name, steps, warmup, device):
     import paged_kv_cache_436_b200 as pa
     if name == "spec4_mix":
         base = synthetic.make("llama13b_mix")
-        w, qlen = base, 4
+        w, qlen = (synthetic.subset(base, subset) if subset else base), 4
     else:
         w = synthetic.custom(8, 32, 32, 128, 16, "bf16", "bf16", [2048] * 8, 4371, pool_factor=1.05)
         qlen = 2048
@@ -537,7 +537,7 @@ def extend_only(args, world, rank, local):
     pa.lib()
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
-    e = time_extend(args.workload, args.steps, args.warmup, device)
+    e = time_extend(args.workload, args.steps, args.warmup, device, subset=args.subset)
     peak, _ = peaks()
     e["roofline"] = extend_roofline(e, peak)
     if rank == 0:
