@@ -35,7 +35,7 @@ constexpr int kTcRows = 128;            // query rows per unit (TMEM lanes)
 constexpr int kTcTok = 128;             // tokens per K/V tile
 constexpr int kTcD = 128;               // head_dim of this path
 constexpr uint32_t kTcTmemCols = 512;   // S double buffer [0, 256), O double buffer [256, 512)
-constexpr int kTcSoftmaxWarps = 4;      // + one MMA-issue warp + one TMA producer warp
+constexpr int kTcSoftmaxWarps = 8;      // two per row group; + one MMA-issue warp + one TMA producer warp
 constexpr int kTcThreads = (kTcSoftmaxWarps + 2) * 32;
 constexpr float kTcRescale = 8.f;       // log2 units
 
@@ -162,6 +162,18 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// One 32-bit column of this warp's 32 lanes (warp-collective), with its wait.
+__device__ __forceinline__ void tc_st1(uint32_t addr, uint32_t v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(addr), "r"(v) : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t tc_ld1(uint32_t addr) {
+  uint32_t v;
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(v) : "r"(addr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+  return pin_after_wait(v);
+}
+
 // 2-D tiled TMA load (box given by the tensor map) signalling `bar` with its bytes.
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
   asm volatile(
@@ -221,7 +233,7 @@ __device__ __forceinline__ bool tc_wait_warp(uint64_t* bar, uint32_t parity, vol
 }
 
 template <int QD, int BS, int G>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kTcThreads, 1)
     extend_tc_kernel(const ExtendParams p, const __grid_constant__ CUtensorMap tk,
                      const __grid_constant__ CUtensorMap tv) {
   using QT = typename Q<QD>::T;
@@ -233,7 +245,7 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* sQ = sm + TcSmem::kQ;
   // per-tile ring barriers (index = tile & 1); per-unit ones (q_full, o_full/o_empty by unit & 1)
   __shared__ uint64_t k_full[2], v_full[2], k_empty[2], pv_done[2], s_full[2], s_empty[2], p_full[2];
-  __shared__ uint64_t q_full, o_full[2], o_empty[2], bar_fin;
+  __shared__ uint64_t q_full, o_full[2], o_empty[2], bar_fin, pair_bar[4];
   __shared__ uint32_t tmem_slot;
   __shared__ int s_abort;
   volatile int* abort = &s_abort;
@@ -258,6 +270,7 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&o_empty[b], kTcSoftmaxWarps);
     }
     mbar_init(&q_full, kTcSoftmaxWarps);
+    for (int i = 0; i < 4; ++i) mbar_init(&pair_bar[i], 2);
     mbar_init(&bar_fin, 1);
     s_abort = 0;
     fence_mbar_init();
@@ -372,16 +385,34 @@ __global__ void __launch_bounds__(192, 1)
       __syncwarp();
     }
   } else {
-    // ---------------- softmax warps: thread tid owns row tid of the unit ----------------
-    const uint32_t t_row = tmem + (uint32_t(warp * 32) << 16);
-    auto write_q = [&](const TcUnit& x) {
-      const int qi = x.t * QPT + tid / G;
+    // ---------------- softmax warps ----------------
+    // Warps w and w + 4 share TMEM lanes 32 (w % 4) .. + 31 (rows of the tile) and split
+    // the columns: half hf = w / 4 holds score / P / O columns [64 hf, 64 hf + 64). The
+    // pair combines its row maxima and sums through one TMEM column each has already read
+    // (its own first column of the S or O buffer) and a 2-arrival mbarrier.
+    const int hf = warp >> 2, rw = warp & 3, row = rw * 32 + lane;
+    const uint32_t t_row = tmem + (uint32_t(rw * 32) << 16);
+    uint32_t xc = 0;   // pair exchanges so far
+    auto exchange = [&](uint32_t col_own, uint32_t col_other, float v, int u, float* other) {
+      tc_st1(t_row + col_own, __float_as_uint(v));
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&pair_bar[rw]);
+      const bool ok = tc_wait_warp(&pair_bar[rw], xc & 1, abort, 23, u);
+      ++xc;
+      if (!ok) return false;
+      tc_fence_after();
+      *other = __uint_as_float(tc_ld1(t_row + col_other));
+      return true;
+    };
+    auto write_q = [&](const TcUnit& x) {   // this half of the row's q
+      const int qi = x.t * QPT + row / G;
       const bool has_q = qi < x.Q;
       const uint4* qrow = reinterpret_cast<const uint4*>(
-          static_cast<const QT*>(p.q) + (size_t(has_q ? x.row0 + qi : 0) * Hq + x.hk * G + tid % G) * kTcD);
+          static_cast<const QT*>(p.q) + (size_t(has_q ? x.row0 + qi : 0) * Hq + x.hk * G + row % G) * kTcD);
 #pragma unroll
-      for (int c = 0; c < 16; ++c)
-        *reinterpret_cast<uint4*>(sQ + tc_swz(tid, c)) = has_q ? qrow[c] : make_uint4(0, 0, 0, 0);
+      for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<uint4*>(sQ + tc_swz(row, hf * 8 + c)) = has_q ? qrow[hf * 8 + c] : make_uint4(0, 0, 0, 0);
       fence_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&q_full);
@@ -390,44 +421,47 @@ __global__ void __launch_bounds__(192, 1)
     if (blockIdx.x < total) write_q(tc_unit(p, blockIdx.x, total, QPT));
     for (int u = blockIdx.x; u < total; u += gridDim.x, ++k) {
       const TcUnit x = tc_unit(p, u, total, QPT);
-      const uint32_t ob = k & 1, t_o = t_row + 256 + ob * 128;
-      const int qi = x.t * QPT + tid / G;
-      const int head = x.hk * G + tid % G;
+      const uint32_t ob = k & 1, c_o = 256 + ob * 128 + hf * 64;   // this half of the O buffer
+      const int qi = x.t * QPT + row / G;
+      const int head = x.hk * G + row % G;
       const bool has_q = qi < x.Q;
       const int qpos = has_q ? x.base + qi : -1;
       const int tok = has_q ? x.row0 + qi : -1;
-      float m_ref = -INFINITY, l = 0.f;
+      float m_ref = -INFINITY, l = 0.f;   // l: this half's share of the row sum
       bool ok = true;
       for (int j = 0; j < x.ntiles; ++j, ++g) {
         const int b = g & 1;
+        const uint32_t c_s = b * 128 + hf * 64;                      // this half of S(g)
         if (!(ok = tc_wait_warp(&s_full[b], (g >> 1) & 1, abort, 18, u))) break;
         tc_fence_after();
-        float s[kTcTok];
+        float s[64];
         {
-          uint32_t r[kTcTok];
-#pragma unroll
-          for (int c = 0; c < kTcTok / 32; ++c) tc_ld32_async(t_row + b * 128 + c * 32, r + c * 32);
+          uint32_t r[64];
+          tc_ld32_async(t_row + c_s, r);
+          tc_ld32_async(t_row + c_s + 32, r + 32);
           tc_wait_ld();
 #pragma unroll
-          for (int c = 0; c < kTcTok; ++c) s[c] = __uint_as_float(pin_after_wait(r[c]));
+          for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(pin_after_wait(r[c]));
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s_empty[b]);
-        // causal mask, row maximum (8 independent chains)
-        const int tp0 = x.t0 + j * kTcTok;
-        if (tp0 + kTcTok - 1 > qpos) {
+        // causal mask, this half's maximum (8 independent chains), then the pair's
+        const int tp0 = x.t0 + j * kTcTok + hf * 64;
+        if (tp0 + 63 > qpos) {
 #pragma unroll
-          for (int c = 0; c < kTcTok; ++c) s[c] = tp0 + c > qpos ? -INFINITY : s[c];
+          for (int c = 0; c < 64; ++c) s[c] = tp0 + c > qpos ? -INFINITY : s[c];
         }
         float m8[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) m8[e] = s[e];
 #pragma unroll
-        for (int c = 8; c < kTcTok; ++c) m8[c & 7] = fmaxf(m8[c & 7], s[c]);
-        const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) *
-                         p.s_mul;
+        for (int c = 8; c < 64; ++c) m8[c & 7] = fmaxf(m8[c & 7], s[c]);
+        const float pm = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+        float po;
+        if (!(ok = exchange(c_s, b * 128 + (hf ^ 1) * 64, pm, u, &po))) break;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_empty[b]);
+        const float mx = fmaxf(pm, po) * p.s_mul;
         const bool up = mx > m_ref + kTcRescale;
         const float corr = up ? ex2(m_ref - mx) : 1.f;   // 0 while nothing was accumulated
         if (up) {
@@ -439,12 +473,12 @@ __global__ void __launch_bounds__(192, 1)
           if (!(ok = tc_wait_warp(&pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1, abort, 19, u))) break;
           tc_fence_after();
 #pragma unroll 1
-          for (int c = 0; c < kTcD / 32; ++c) {
+          for (int c = 0; c < 2; ++c) {
             float o[32];
-            tc_ld32(t_o + c * 32, o);
+            tc_ld32(t_row + c_o + c * 32, o);
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] *= corr;
-            tc_st32(t_o + c * 32, o);
+            tc_st32(t_row + c_o + c * 32, o);
           }
         }
         // P(g) into its buffer once P(g-2) V(g-2) has finished reading it
@@ -453,27 +487,26 @@ __global__ void __launch_bounds__(192, 1)
         const float nmb = m_ref == -INFINITY ? 0.f : -m_ref;
         float l8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int c = 0; c < kTcTok / 8; ++c) {
+        for (int c = 0; c < 8; ++c) {
           uint32_t w[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e)
             w[e] = pack2_sum<QD>(ex2(fmaf(s[c * 8 + 2 * e], p.s_mul, nmb)),
                                  ex2(fmaf(s[c * 8 + 2 * e + 1], p.s_mul, nmb)), l8[(c & 1) * 4 + e]);
-          *reinterpret_cast<uint4*>(sP + tc_swz(tid, c)) = make_uint4(w[0], w[1], w[2], w[3]);
+          *reinterpret_cast<uint4*>(sP + tc_swz(row, hf * 8 + c)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
         l += ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
         // V rows past the visible tokens (cache bytes beyond the context, or stale rows
-        // of blocks not loaded) are zeroed so that 0-weighted rows cannot bring a NaN
+        // of blocks not loaded) are zeroed, this half of each, so that 0-weighted rows
+        // cannot bring a NaN into O
         const int rem = x.nvis - j * kTcTok;
         if (rem < kTcTok) {
           if (!(ok = tc_wait_warp(&v_full[b], (g >> 1) & 1, abort, 21, u))) break;
-          if (tid >= rem) {
-            uint8_t* vrow = sm + TcSmem::kV + b * TcSmem::kTile + (tid >> 3) * 1024 + (tid & 7) * 128;
+          if (row >= rem) {
+            uint8_t* vrow = sm + TcSmem::kV + b * TcSmem::kTile + hf * (kTcTok * 128) + (row >> 3) * 1024 +
+                            (row & 7) * 128;
 #pragma unroll
-            for (int h = 0; h < 2; ++h)
-#pragma unroll
-              for (int c = 0; c < 8; ++c)
-                *reinterpret_cast<uint4*>(vrow + h * (kTcTok * 128) + c * 16) = make_uint4(0, 0, 0, 0);
+            for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(vrow + c * 16) = make_uint4(0, 0, 0, 0);
           }
         }
         fence_async_smem();
@@ -486,27 +519,30 @@ __global__ void __launch_bounds__(192, 1)
       if (u + (int)gridDim.x < total) write_q(tc_unit(p, u + gridDim.x, total, QPT));
       if (!tc_wait_warp(&o_full[ob], (k >> 1) & 1, abort, 22, u)) break;
       tc_fence_after();
-      const int P = has_q ? (qpos + 1 + p.chunk - 1) / p.chunk : 0;
-      const bool wr = has_q && x.part < P;
-      const bool fin = wr && P == 1;
-      const float inv = fin ? 1.f / l : 0.f;
-      const size_t slot = (size_t(has_q ? tok : 0) * Hq + head) * p.max_parts + x.part;
-      float o[kTcD];
+      float o[64];
       {
-        uint32_t r[kTcD];
-#pragma unroll
-        for (int c = 0; c < kTcD / 32; ++c) tc_ld32_async(t_o + c * 32, r + c * 32);
+        uint32_t r[64];
+        tc_ld32_async(t_row + c_o, r);
+        tc_ld32_async(t_row + c_o + 32, r + 32);
         tc_wait_ld();
 #pragma unroll
-        for (int c = 0; c < kTcD; ++c) o[c] = __uint_as_float(pin_after_wait(r[c]));
+        for (int c = 0; c < 64; ++c) o[c] = __uint_as_float(pin_after_wait(r[c]));
       }
+      float lo;
+      if (!exchange(c_o, 256 + ob * 128 + (hf ^ 1) * 64, l, u, &lo)) break;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&o_empty[ob]);
+      const float lsum = hf == 0 ? l + lo : lo + l;   // same order in both halves
+      const int P = has_q ? (qpos + 1 + p.chunk - 1) / p.chunk : 0;
+      const bool wr = has_q && x.part < P;
+      const bool fin = wr && P == 1;
       if (fin) {
-        uint4* orow = reinterpret_cast<uint4*>(static_cast<QT*>(p.out) + (size_t(tok) * Hq + head) * kTcD);
+        const float inv = 1.f / lsum;
+        uint4* orow =
+            reinterpret_cast<uint4*>(static_cast<QT*>(p.out) + (size_t(tok) * Hq + head) * kTcD + hf * 64);
 #pragma unroll
-        for (int i = 0; i < kTcD / 8; ++i) {
+        for (int i = 0; i < 8; ++i) {
           float dummy = 0.f;
           uint32_t w[4];
 #pragma unroll
@@ -514,11 +550,14 @@ __global__ void __launch_bounds__(192, 1)
           orow[i] = make_uint4(w[0], w[1], w[2], w[3]);
         }
       } else if (wr) {
-        float4* acc = reinterpret_cast<float4*>(p.part_acc + slot * kTcD);
+        const size_t slot = (size_t(tok) * Hq + head) * p.max_parts + x.part;
+        float4* acc = reinterpret_cast<float4*>(p.part_acc + slot * kTcD + hf * 64);
 #pragma unroll
-        for (int i = 0; i < kTcD / 4; ++i) acc[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
-        p.part_ml[slot * 2] = m_ref;
-        p.part_ml[slot * 2 + 1] = l;
+        for (int i = 0; i < 16; ++i) acc[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+        if (hf == 0) {
+          p.part_ml[slot * 2] = m_ref;
+          p.part_ml[slot * 2 + 1] = lsum;
+        }
       }
     }
   }
