@@ -223,10 +223,13 @@ pa_status pa_decode_no_alloc(const void* q, int32_t q_dtype, int32_t num_seqs, i
  *                  are already in the cache (pa_reshape_and_cache)
  *   q, out         device [num_tokens][num_q_heads][head_dim] of q_dtype
  * Query i of sequence s sits at position L_s - Q_s + i and attends to tokens
- * 0 .. L_s - Q_s + i; out = softmax(scale * q K^T) V over them. Q_s > L_s is recorded
- * (PA_DEV_BAD_CONTEXT_LEN) and its rows are zero. Runs on the tensor cores (16-bit
- * inputs, binary32 accumulation; P rounded to the cache's 16-bit type); 512-token
- * partitions merged by a log-sum-exp kernel as in pa_decode.
+ * 0 .. L_s - Q_s + i; out = softmax(scale * q K^T) V over them. Q_s > L_s, or a range
+ * outside [0, num_tokens], is recorded (PA_DEV_BAD_CONTEXT_LEN) and its rows are zero.
+ * Runs on the tensor cores (16-bit inputs, binary32 accumulation; P rounded to the
+ * cache's 16-bit type): mma.sync for short query runs, tcgen05 with TMEM accumulators
+ * for long ones (head_dim 128, scale > 0); context chunks (multiples of 512 tokens)
+ * merged by a log-sum-exp kernel as in pa_decode. Cache bytes past a context never
+ * affect the output.
  * Supported: 16-bit caches with q_dtype == kv_dtype, head_dim 64 or 128, block_size 16
  * or 32, G in {1, 2, 4, 8}. workspace >= pa_extend_workspace_size(...), 256-byte aligned.
  */

@@ -43,6 +43,9 @@ struct ExtendParams {
   float s_mul;                  // scale * log2(e)
   int out_row_bytes;            // Hq * D * 2
   int chunk;                    // context tokens per unit: a multiple of kPartitionTokens
+  int4* units;                  // optional: two int4 per (seq, tile, chunk) pair, written by the plan
+                                //   {s, tile, chunk index, row0}, {Q, base, first token, visible tokens}
+  long long units_cap;          // pairs the records can hold
 };
 
 constexpr int kTileRows = 16;
@@ -52,8 +55,9 @@ __device__ __forceinline__ int ext_clamp(int x, int lo, int hi) { return x < lo 
 // Query count and position of query 0 of sequence s (validated the same way everywhere).
 __device__ __forceinline__ void ext_seq(const ExtendParams& p, int s, int& Q, int& base) {
   const int L = ext_clamp(p.context_lens[s], 0, p.len_limit);
-  Q = p.query_start[s + 1] - p.query_start[s];
-  if (Q < 0 || Q > L) Q = 0;               // invalid: recorded by the plan, no work
+  const int q0 = p.query_start[s], q1 = p.query_start[s + 1];
+  Q = q1 - q0;
+  if (Q < 0 || Q > L || q0 < 0 || q1 > p.num_tokens) Q = 0;   // invalid: recorded by the plan, no work
   base = L - Q;
 }
 
@@ -112,12 +116,34 @@ __global__ void __launch_bounds__(1024) extend_plan_kernel(const ExtendParams p,
     }
     __syncthreads();
     const int before = carry + (warp > 0 ? warp_tot[warp - 1] : 0) + incl - units;
-    if (s < p.num_seqs) p.plan[s] = before;
+    if (s < p.num_seqs) {
+      p.plan[s] = before;
+      if (p.units && units > 0) {   // the pair records of this sequence, in plan order
+        int Q, base;
+        ext_seq(p, s, Q, base);
+        const int row0 = p.query_start[s];
+        int idx = before;
+        const int tiles = (Q + qpt - 1) / qpt;
+        for (int t = 0; t < tiles; ++t) {
+          const int last = base + min((t + 1) * qpt, Q) - 1;
+          const int P = ext_tile_parts(base, Q, qpt, t, p.chunk);
+          for (int part = 0; part < P && idx < p.units_cap; ++part, ++idx) {
+            const int t0 = part * p.chunk;
+            p.units[2 * size_t(idx)] = make_int4(s, t, part, row0);
+            p.units[2 * size_t(idx) + 1] = make_int4(Q, base, t0, min(p.chunk, last + 1 - t0));
+          }
+        }
+      }
+    }
     __syncthreads();
     if (threadIdx.x == blockDim.x - 1) carry = before + units;
     __syncthreads();
   }
-  if (threadIdx.x == 0) p.plan[p.num_seqs] = carry;
+  if (threadIdx.x == 0) {
+    // pairs past the records' capacity (only from inconsistent query_start) are dropped
+    if (p.units && carry > p.units_cap) record_error(PA_DEV_BAD_CONTEXT_LEN, -1, carry, int(p.units_cap));
+    p.plan[p.num_seqs] = p.units && carry > p.units_cap ? int(p.units_cap) : carry;
+  }
 }
 
 // --------------------------------------------------------------------------
@@ -747,15 +773,22 @@ __global__ void __launch_bounds__(128) extend_reduce_kernel(const ExtendParams p
 // host side
 // --------------------------------------------------------------------------
 struct ExtWs {
-  size_t plan, ml, acc, total;
+  size_t plan, ml, acc, units, total;
 };
+
+// Pair records of the 128-row path: it runs only when 2 T G >= 128 S, so its tiles are at
+// most T G / 128 + 1 + S <= 3 T Hq / 128 + 1, each with at most max_parts chunks.
+inline size_t ext_units_bound(int T, int Hq, int max_parts) {
+  return (3 * size_t(T) * Hq / 128 + 2) * size_t(max_parts);
+}
 
 inline ExtWs ext_ws(int S, int T, int Hq, int D, int max_parts) {
   ExtWs w;
   w.plan = 0;
   w.ml = align256(size_t(S + 1) * 4);
   w.acc = w.ml + align256(size_t(T) * Hq * max_parts * 2 * 4);
-  w.total = w.acc + align256(size_t(T) * Hq * max_parts * D * 4);
+  w.units = w.acc + align256(size_t(T) * Hq * max_parts * D * 4);
+  w.total = w.units + align256(ext_units_bound(T, Hq, max_parts) * 32);
   return w;
 }
 
@@ -873,6 +906,8 @@ pa_status pa_extend(const void* q, int32_t q_dtype, int32_t num_seqs, int32_t nu
   p.plan = reinterpret_cast<int32_t*>(w + ws.plan);
   p.part_ml = reinterpret_cast<float*>(w + ws.ml);
   p.part_acc = reinterpret_cast<float*>(w + ws.acc);
+  p.units = tc ? reinterpret_cast<int4*>(w + ws.units) : nullptr;
+  p.units_cap = (long long)ext_units_bound(num_tokens, num_q_heads, max_parts);
   p.num_seqs = num_seqs;
   p.num_tokens = num_tokens;
   p.num_q_heads = num_q_heads;

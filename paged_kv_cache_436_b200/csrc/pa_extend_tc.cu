@@ -196,18 +196,20 @@ struct TcUnit {
   int t0, nvis, ntiles;     // first context token of the chunk, visible tokens, K/V tiles
 };
 
-__device__ __forceinline__ TcUnit tc_unit(const ExtendParams& p, int u, int total, int qpt) {
-  const ExtUnit x = ext_make_unit<16>(p, u, total, qpt, 64);   // no block-id reads
+// Unit u = pair * Hkv + kv head; the pair's record was written by the plan kernel.
+__device__ __forceinline__ TcUnit tc_unit(const ExtendParams& p, int u) {
+  const int pair = u / p.num_kv_heads;
+  const int4 a = __ldg(p.units + 2 * size_t(pair)), b = __ldg(p.units + 2 * size_t(pair) + 1);
   TcUnit t;
-  t.s = x.s;
-  t.hk = x.hk;
-  t.t = x.t;
-  t.part = x.part;
-  t.Q = x.Q;
-  t.base = x.base;
-  t.row0 = x.row0;
-  t.t0 = x.part * p.chunk;
-  t.nvis = min(p.chunk, x.last + 1 - t.t0);
+  t.s = a.x;
+  t.hk = u - pair * p.num_kv_heads;
+  t.t = a.y;
+  t.part = a.z;
+  t.row0 = a.w;
+  t.Q = b.x;
+  t.base = b.y;
+  t.t0 = b.z;
+  t.nvis = b.w;
   t.ntiles = (t.nvis + kTcTok - 1) / kTcTok;
   return t;
 }
@@ -290,7 +292,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // ---------------- producer: K and V tiles by 2-D TMA, lane i loads cache block i ----------------
     uint32_t g = 0;
     for (int u = blockIdx.x; u < total && !*abort; u += gridDim.x) {
-      const TcUnit x = tc_unit(p, u, total, QPT);
+      const TcUnit x = tc_unit(p, u);
       const int32_t* trow = p.block_tables + size_t(x.s) * p.max_blocks;
       auto blocks = [&](int j) { return min(BPT, (x.nvis - j * kTcTok + BS - 1) / BS); };
       auto fetch = [&](int j) {   // block id of this lane's block of tile j
@@ -356,7 +358,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       return true;
     };
     for (int u = blockIdx.x; u < total && !*abort; u += gridDim.x, ++k) {
-      const TcUnit x = tc_unit(p, u, total, QPT);
+      const TcUnit x = tc_unit(p, u);
       const uint32_t ob = k & 1;
       if (!tc_wait_warp(&q_full, k & 1, abort, 14, u)) break;
       if (!tc_wait_warp(&o_empty[ob], ((k >> 1) & 1) ^ 1, abort, 15, u)) break;
@@ -418,9 +420,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (lane == 0) mbar_arrive(&q_full);
     };
     uint32_t g = 0, k = 0;
-    if (blockIdx.x < total) write_q(tc_unit(p, blockIdx.x, total, QPT));
+    TcUnit x;
+    if (blockIdx.x < total) {
+      x = tc_unit(p, blockIdx.x);
+      write_q(x);
+    }
     for (int u = blockIdx.x; u < total; u += gridDim.x, ++k) {
-      const TcUnit x = tc_unit(p, u, total, QPT);
+      const bool more = u + (int)gridDim.x < total;
+      const TcUnit xn = more ? tc_unit(p, u + gridDim.x) : x;   // read now, used after the first tile
       const uint32_t ob = k & 1, c_o = 256 + ob * 128 + hf * 64;   // this half of the O buffer
       const int qi = x.t * QPT + row / G;
       const int head = x.hk * G + row % G;
@@ -513,10 +520,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[b]);
+        if (j == 0 && more) {   // the next unit's q half-row towards L2
+          const int nqi = xn.t * QPT + row / G;
+          if (nqi < xn.Q) {
+            const QT* nq = static_cast<const QT*>(p.q) + (size_t(xn.row0 + nqi) * Hq + xn.hk * G + row % G) * kTcD + hf * 64;
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(nq));
+          }
+        }
       }
       if (!ok) break;
       // the next unit's Q (every S of this unit has completed), then this unit's O
-      if (u + (int)gridDim.x < total) write_q(tc_unit(p, u + gridDim.x, total, QPT));
+      if (more) write_q(xn);
       if (!tc_wait_warp(&o_full[ob], (k >> 1) & 1, abort, 22, u)) break;
       tc_fence_after();
       float o[64];
@@ -559,6 +573,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           p.part_ml[slot * 2 + 1] = lsum;
         }
       }
+      x = xn;
     }
   }
 
