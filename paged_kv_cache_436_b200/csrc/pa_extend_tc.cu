@@ -35,8 +35,8 @@ constexpr int kTcRows = 128;            // query rows per unit (TMEM lanes)
 constexpr int kTcTok = 128;             // tokens per K/V tile
 constexpr int kTcD = 128;               // head_dim of this path
 constexpr uint32_t kTcTmemCols = 512;   // S double buffer [0, 256), O double buffer [256, 512)
-constexpr int kTcSoftmaxWarps = 8;      // two per row group; + one MMA-issue warp + one TMA producer warp
-constexpr int kTcThreads = (kTcSoftmaxWarps + 2) * 32;
+constexpr int kTcSoftmaxWarps = 8;      // two per row group; + an MMA-issue warp + K and V producer warps
+constexpr int kTcThreads = (kTcSoftmaxWarps + 3) * 32;
 constexpr float kTcRescale = 8.f;       // log2 units
 
 struct TcSmem {
@@ -288,8 +288,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int total = p.plan[p.num_seqs] * Hkv;
   uint32_t last_load = 0;           // producer: tiles issued (for the drain after an abort)
 
-  if (warp == kTcSoftmaxWarps + 1) {
-    // ---------------- producer: K and V tiles by 2-D TMA, lane i loads cache block i ----------------
+  if (warp > kTcSoftmaxWarps) {
+    // ---------------- producers: warp kTcSoftmaxWarps + 1 streams K, the next one V, by 2-D
+    // TMA, lane i loading cache block i of a tile; separate warps, so that a K tile never
+    // waits behind the V tile before it (which waits for an older P V) ----------------
+    const bool is_v = warp == kTcSoftmaxWarps + 2;
+    uint64_t* full = is_v ? v_full : k_full;
+    uint64_t* empty = is_v ? pv_done : k_empty;   // V(g) after P(g-2) V(g-2); K(g) after S(g-2)
+    const CUtensorMap* map = is_v ? &tv : &tk;
+    uint8_t* ring = sm + (is_v ? TcSmem::kV : TcSmem::kK);
     uint32_t g = 0;
     for (int u = blockIdx.x; u < total && !*abort; u += gridDim.x) {
       const TcUnit x = tc_unit(p, u);
@@ -301,7 +308,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (lane < blocks(j)) {
           id = trow[lb];
           if (id < 0 || id >= p.num_blocks) {
-            record_error(PA_DEV_BAD_BLOCK_ID, x.s, lb, id);
+            if (!is_v) record_error(PA_DEV_BAD_BLOCK_ID, x.s, lb, id);
             id = 0;
           }
         }
@@ -312,23 +319,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int b = g & 1, nb = blocks(j);
         const int next = j + 1 < x.ntiles ? fetch(j + 1) : 0;   // read ahead of its use
         const int y = (id * Hkv + x.hk) * BS;
-        const uint32_t off = b * TcSmem::kTile + lane * (BS * 128);
-        if (!tc_wait_warp(&k_empty[b], ((g >> 1) & 1) ^ 1, abort, 10, u)) break;
-        if (lane == 0) mbar_arrive_expect_tx(&k_full[b], uint32_t(nb) * kBlockTx);
+        uint8_t* dst = ring + b * TcSmem::kTile + lane * (BS * 128);
+        if (!tc_wait_warp(&empty[b], ((g >> 1) & 1) ^ 1, abort, is_v ? 11 : 10, u)) break;
+        if (lane == 0) mbar_arrive_expect_tx(&full[b], uint32_t(nb) * kBlockTx);
         __syncwarp();
         if (lane < nb) {
-          tma_load_2d(sm + TcSmem::kK + off, &tk, 0, y, &k_full[b]);
-          tma_load_2d(sm + TcSmem::kK + off + kTcTok * 128, &tk, 64, y, &k_full[b]);
-        }
-        if (!tc_wait_warp(&pv_done[b], ((g >> 1) & 1) ^ 1, abort, 11, u)) {
-          last_load = g + 1;
-          break;
-        }
-        if (lane == 0) mbar_arrive_expect_tx(&v_full[b], uint32_t(nb) * kBlockTx);
-        __syncwarp();
-        if (lane < nb) {
-          tma_load_2d(sm + TcSmem::kV + off, &tv, 0, y, &v_full[b]);
-          tma_load_2d(sm + TcSmem::kV + off + kTcTok * 128, &tv, 64, y, &v_full[b]);
+          tma_load_2d(dst, map, 0, y, &full[b]);
+          tma_load_2d(dst + kTcTok * 128, map, 64, y, &full[b]);
         }
         last_load = g + 1;
         id = next;
@@ -583,11 +580,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc_commit(&bar_fin);
       mbar_wait_bounded(&bar_fin, 0);
     }
-    if (warp == kTcSoftmaxWarps + 1 && lane == 0) {
-      for (uint32_t h = last_load >= 2 ? last_load - 2 : 0; h < last_load; ++h) {
-        mbar_wait_bounded(&k_full[h & 1], (h >> 1) & 1, 100000000ull);
-        mbar_wait_bounded(&v_full[h & 1], (h >> 1) & 1, 100000000ull);
-      }
+    if (warp > kTcSoftmaxWarps && lane == 0) {
+      uint64_t* full = warp == kTcSoftmaxWarps + 2 ? v_full : k_full;
+      for (uint32_t h = last_load >= 2 ? last_load - 2 : 0; h < last_load; ++h)
+        mbar_wait_bounded(&full[h & 1], (h >> 1) & 1, 100000000ull);
     }
   }
   tc_fence_before();
