@@ -6,25 +6,33 @@
 //   * a work unit is (sequence, kv head, tile of 128 rows, chunk of the context); a row
 //     is a (query, q head of the kv head's group) pair; the chunk is a multiple of the
 //     512-token partition, chosen by the host so that there are enough units to fill
-//     the GPU (the whole context when there are, then no merge pass at all);
-//   * one CTA of 4 warps per unit (persistent); TMEM lane r holds row r and thread r
-//     owns it; TMEM columns [0, 128) hold S of the current 128-token K/V tile,
-//     [128, 256) the output accumulator O;
-//   * Q rows are stored by their threads into a 128B-swizzled K-major shared tile;
-//     K and V tiles come by 2-D TMA (cp.async.bulk.tensor, 128B swizzle, no
-//     multicast) straight from the paged cache, one box per (cache block, 64-column
-//     half); two K/V buffers, so tile j + 1 loads while tile j is in use;
-//   * thread 0 issues S = Q K^T (both K-major) and O += P V (P K-major; V MN-major,
-//     i.e. left in its [token][dim] cache layout) and commits each to an mbarrier;
-//   * the softmax reads its S row from TMEM, masks causally and keeps a reference
-//     maximum that moves only when the row maximum passes it by more than 2^8 (O and
-//     the running sum are then rescaled; every p stays below 2^8, so nothing is lost);
-//     P goes to a swizzled K-major shared tile in the query's 16-bit type and the
-//     running sum adds those same rounded values;
+//     the GPU (the whole context when there are, then no merge pass at all); the plan
+//     kernel writes one record per (sequence, tile, chunk);
+//   * one persistent CTA per SM with warp-specialised roles: 8 softmax warps (warps w
+//     and w + 4 share TMEM lanes 32 (w % 4) .. + 31, i.e. rows of the tile, and split
+//     the 128 columns into halves), one MMA-issue warp, one K and one V producer warp;
+//   * TMEM: S of two consecutive 128-token K/V tiles in columns [0, 256), the output
+//     accumulators O of two consecutive units in [256, 512);
+//   * the unit's Q rows come by one 3-D TMA box per 64-column half (64 dims x G heads x
+//     128 / G queries: the rows in (query, head) order) into a 128B-swizzled K-major
+//     tile, loaded as soon as the previous unit's last S has completed; K and V tiles
+//     come by 2-D TMA (cp.async.bulk.tensor, 128B swizzle, no multicast) straight from
+//     the paged cache, one box per (cache block, 64-column half), into 2-deep K and V
+//     rings;
+//   * S = Q K^T (both K-major) and O += P V (P K-major; V MN-major, i.e. left in its
+//     [token][dim] cache layout) are issued by one thread; order S(g), P(g-1) V(g-1),
+//     S(g+1), ... so that the next S runs while the softmax works on the current one;
+//   * the softmax reads its half of the S row from TMEM, masks causally and keeps a
+//     reference maximum that moves only when the row maximum passes it by more than 2^8
+//     (O and the running sum are then rescaled; every p stays below 2^8, so nothing is
+//     lost). The pair's maximum is combined through a TMEM column and a 2-arrival
+//     mbarrier; P is computed speculatively with the current reference meanwhile and
+//     recomputed only when the reference moves. P goes to a swizzled K-major shared
+//     tile in the query's 16-bit type and the running sum adds those rounded values;
 //   * a unit that covers a row's whole context writes the output row; otherwise it
 //     writes (max, sum, unnormalised row) for the log-sum-exp merge kernel.
-// Every wait is bounded; on a timeout the kernel records it, drains what it issued,
-// frees its TMEM and returns.
+// Every wait is bounded; on a timeout the kernel records it, every role stops, the MMA
+// and load issuers drain what they issued, and the TMEM is freed.
 #include <cuda.h>
 
 #include <mutex>
@@ -183,6 +191,15 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
       : "memory");
 }
 
+// 3-D tiled TMA load.
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_addr(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(z), "r"(smem_addr(bar))
+      : "memory");
+}
+
 // Byte offset of 16-byte chunk c (0..15) of row r in a [128 x 128] 16-bit tile kept
 // as two 128B-swizzled K-major halves of 64 columns (8-row atoms of 1 KB).
 __device__ __forceinline__ uint32_t tc_swz(int r, int c) {
@@ -237,7 +254,7 @@ __device__ __forceinline__ bool tc_wait_warp(uint64_t* bar, uint32_t parity, vol
 template <int QD, int BS, int G>
 __global__ void __launch_bounds__(kTcThreads, 1)
     extend_tc_kernel(const ExtendParams p, const __grid_constant__ CUtensorMap tk,
-                     const __grid_constant__ CUtensorMap tv) {
+                     const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tq) {
   using QT = typename Q<QD>::T;
   constexpr int QPT = kTcRows / G;                    // queries per unit
   constexpr int BPT = kTcTok / BS;                    // cache blocks per K/V tile
@@ -247,7 +264,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint8_t* sQ = sm + TcSmem::kQ;
   // per-tile ring barriers (index = tile & 1); per-unit ones (q_full, o_full/o_empty by unit & 1)
   __shared__ uint64_t k_full[2], v_full[2], k_empty[2], pv_done[2], s_full[2], s_empty[2], p_full[2];
-  __shared__ uint64_t q_full, o_full[2], o_empty[2], bar_fin, pair_bar[4];
+  __shared__ uint64_t q_full, q_empty, o_full[2], o_empty[2], bar_fin, pair_bar[4];
   __shared__ uint32_t tmem_slot;
   __shared__ int s_abort;
   volatile int* abort = &s_abort;
@@ -271,7 +288,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&o_full[b], 1);
       mbar_init(&o_empty[b], kTcSoftmaxWarps);
     }
-    mbar_init(&q_full, kTcSoftmaxWarps);
+    mbar_init(&q_full, 1);
+    mbar_init(&q_empty, 1);
     for (int i = 0; i < 4; ++i) mbar_init(&pair_bar[i], 2);
     mbar_init(&bar_fin, 1);
     s_abort = 0;
@@ -297,9 +315,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint64_t* empty = is_v ? pv_done : k_empty;   // V(g) after P(g-2) V(g-2); K(g) after S(g-2)
     const CUtensorMap* map = is_v ? &tv : &tk;
     uint8_t* ring = sm + (is_v ? TcSmem::kV : TcSmem::kK);
-    uint32_t g = 0;
-    for (int u = blockIdx.x; u < total && !*abort; u += gridDim.x) {
+    uint32_t g = 0, k = 0;
+    for (int u = blockIdx.x; u < total && !*abort; u += gridDim.x, ++k) {
       const TcUnit x = tc_unit(p, u);
+      if (is_v) {   // the unit's q rows: box {64 dims, G heads, QPT queries} per 64-dim half
+        if (k > 0 && !tc_wait_warp(&q_empty, (k - 1) & 1, abort, 26, u)) break;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&q_full, TcSmem::kTile);
+          tma_load_3d(sQ, &tq, 0, x.hk * G, x.row0 + x.t * QPT, &q_full);
+          tma_load_3d(sQ + kTcRows * 128, &tq, 64, x.hk * G, x.row0 + x.t * QPT, &q_full);
+        }
+        __syncwarp();
+      }
       const int32_t* trow = p.block_tables + size_t(x.s) * p.max_blocks;
       auto blocks = [&](int j) { return min(BPT, (x.nvis - j * kTcTok + BS - 1) / BS); };
       auto fetch = [&](int j) {   // block id of this lane's block of tile j
@@ -375,6 +402,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
           tc_commit(&s_full[b]);
           tc_commit(&k_empty[b]);
+          if (j + 1 == x.ntiles) tc_commit(&q_empty);   // sQ is free once this S completes
         }
         __syncwarp();
         if (j > 0) ok = pv(g - 1, j == 1, ob, u);
@@ -404,27 +432,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       *other = __uint_as_float(tc_ld1(t_row + col_other));
       return true;
     };
-    auto write_q = [&](const TcUnit& x) {   // this half of the row's q
-      const int qi = x.t * QPT + row / G;
-      const bool has_q = qi < x.Q;
-      const uint4* qrow = reinterpret_cast<const uint4*>(
-          static_cast<const QT*>(p.q) + (size_t(has_q ? x.row0 + qi : 0) * Hq + x.hk * G + row % G) * kTcD);
-#pragma unroll
-      for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<uint4*>(sQ + tc_swz(row, hf * 8 + c)) = has_q ? qrow[hf * 8 + c] : make_uint4(0, 0, 0, 0);
-      fence_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&q_full);
-    };
     uint32_t g = 0, k = 0;
-    TcUnit x;
-    if (blockIdx.x < total) {
-      x = tc_unit(p, blockIdx.x);
-      write_q(x);
-    }
     for (int u = blockIdx.x; u < total; u += gridDim.x, ++k) {
-      const bool more = u + (int)gridDim.x < total;
-      const TcUnit xn = more ? tc_unit(p, u + gridDim.x) : x;   // read now, used after the first tile
+      const TcUnit x = tc_unit(p, u);
       const uint32_t ob = k & 1, c_o = 256 + ob * 128 + hf * 64;   // this half of the O buffer
       const int qi = x.t * QPT + row / G;
       const int head = x.hk * G + row % G;
@@ -460,8 +470,37 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int c = 8; c < 64; ++c) m8[c & 7] = fmaxf(m8[c & 7], s[c]);
         const float pm = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
                                fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-        float po;
-        if (!(ok = exchange(c_s, b * 128 + (hf ^ 1) * 64, pm, u, &po))) break;
+        // publish this half's maximum to the partner warp (own first S column, already read)
+        tc_st1(t_row + c_s, __float_as_uint(pm));
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&pair_bar[rw]);
+        // P(g) goes into buffer b once P(g-2) V(g-2) has finished reading it
+        if (!(ok = tc_wait_warp(&pv_done[b], ((g >> 1) & 1) ^ 1, abort, 20, u))) break;
+        uint8_t* sP = sm + TcSmem::kP + b * TcSmem::kTile;
+        auto make_p = [&](float ref) {   // P = 2^(s * scale - ref) into sP; returns its rounded sum
+          const float nmb = -ref;
+          float l8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              w[e] = pack2_sum<QD>(ex2(fmaf(s[c * 8 + 2 * e], p.s_mul, nmb)),
+                                   ex2(fmaf(s[c * 8 + 2 * e + 1], p.s_mul, nmb)), l8[(c & 1) * 4 + e]);
+            *reinterpret_cast<uint4*>(sP + tc_swz(row, hf * 8 + c)) = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+          return ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
+        };
+        // speculatively with the current reference while the partner's maximum is in flight:
+        // it stands unless the pair's maximum passes the reference by more than 2^8
+        const bool spec = m_ref != -INFINITY && pm * p.s_mul <= m_ref + kTcRescale;
+        float lt = spec ? make_p(m_ref) : 0.f;
+        const bool okp = tc_wait_warp(&pair_bar[rw], xc & 1, abort, 23, u);
+        ++xc;
+        if (!(ok = okp)) break;
+        tc_fence_after();
+        const float po = __uint_as_float(tc_ld1(t_row + b * 128 + (hf ^ 1) * 64));
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_empty[b]);
@@ -485,21 +524,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             tc_st32(t_row + c_o + c * 32, o);
           }
         }
-        // P(g) into its buffer once P(g-2) V(g-2) has finished reading it
-        if (!(ok = tc_wait_warp(&pv_done[b], ((g >> 1) & 1) ^ 1, abort, 20, u))) break;
-        uint8_t* sP = sm + TcSmem::kP + b * TcSmem::kTile;
-        const float nmb = m_ref == -INFINITY ? 0.f : -m_ref;
-        float l8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint32_t w[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            w[e] = pack2_sum<QD>(ex2(fmaf(s[c * 8 + 2 * e], p.s_mul, nmb)),
-                                 ex2(fmaf(s[c * 8 + 2 * e + 1], p.s_mul, nmb)), l8[(c & 1) * 4 + e]);
-          *reinterpret_cast<uint4*>(sP + tc_swz(row, hf * 8 + c)) = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-        l += ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
+        if (!spec || up) lt = make_p(m_ref == -INFINITY ? 0.f : m_ref);
+        l += lt;
         // V rows past the visible tokens (cache bytes beyond the context, or stale rows
         // of blocks not loaded) are zeroed, this half of each, so that 0-weighted rows
         // cannot bring a NaN into O
@@ -517,17 +543,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[b]);
-        if (j == 0 && more) {   // the next unit's q half-row towards L2
-          const int nqi = xn.t * QPT + row / G;
-          if (nqi < xn.Q) {
-            const QT* nq = static_cast<const QT*>(p.q) + (size_t(xn.row0 + nqi) * Hq + xn.hk * G + row % G) * kTcD + hf * 64;
-            asm volatile("prefetch.global.L2 [%0];" ::"l"(nq));
-          }
-        }
       }
       if (!ok) break;
-      // the next unit's Q (every S of this unit has completed), then this unit's O
-      if (more) write_q(xn);
+      // this unit's O
       if (!tc_wait_warp(&o_full[ob], (k >> 1) & 1, abort, 22, u)) break;
       tc_fence_after();
       float o[64];
@@ -570,7 +588,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           p.part_ml[slot * 2 + 1] = lsum;
         }
       }
-      x = xn;
     }
   }
 
@@ -624,7 +641,19 @@ bool cache_tmap(TmapEncodeFn enc, CUtensorMap* m, const void* base, int qd, long
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-using TcKernel = void (*)(const ExtendParams, const CUtensorMap, const CUtensorMap);
+// q viewed as [tokens][q heads][head_dim]; box = 64 dims x G heads x 128 / G queries,
+// i.e. one 64-column half of a unit's 128 rows in (query, head) order.
+bool q_tmap(TmapEncodeFn enc, CUtensorMap* m, const void* q, int qd, int num_tokens, int Hq, int G) {
+  const cuuint64_t dims[3] = {cuuint64_t(kTcD), cuuint64_t(Hq), cuuint64_t(num_tokens)};
+  const cuuint64_t strides[2] = {cuuint64_t(kTcD) * 2, cuuint64_t(Hq) * kTcD * 2};
+  const cuuint32_t box[3] = {64, cuuint32_t(G), cuuint32_t(kTcRows / G)};
+  const cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, qd == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+             const_cast<void*>(q), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+using TcKernel = void (*)(const ExtendParams, const CUtensorMap, const CUtensorMap, const CUtensorMap);
 
 template <int QD, int BS>
 TcKernel tc_pick_g(int G) {
@@ -663,10 +692,11 @@ pa_status extend_tc_launch(const ExtendParams& p, const pa_cache_desc* c, int qd
   TcKernel fn = tc_pick(qd, c->block_size, G);
   TmapEncodeFn enc = tmap_encoder();
   if (!fn || !enc) return PA_ERR_ARG;
-  CUtensorMap tk, tv;
+  CUtensorMap tk, tv, tq;
   const long long rows = (long long)c->num_blocks * c->num_kv_heads * c->block_size;
   if (!cache_tmap(enc, &tk, c->k_cache, qd, rows, c->block_size) ||
-      !cache_tmap(enc, &tv, c->v_cache, qd, rows, c->block_size))
+      !cache_tmap(enc, &tv, c->v_cache, qd, rows, c->block_size) ||
+      !q_tmap(enc, &tq, p.q, qd, p.num_tokens, p.num_q_heads, G))
     return PA_ERR_ARG;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
@@ -678,7 +708,7 @@ pa_status extend_tc_launch(const ExtendParams& p, const pa_cache_desc* c, int qd
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, fn, p, tk, tv) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  return cudaLaunchKernelEx(&cfg, fn, p, tk, tv, tq) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 }  // namespace pa
