@@ -182,6 +182,44 @@ __device__ __forceinline__ uint32_t tc_ld1(uint32_t addr) {
   return pin_after_wait(v);
 }
 
+// Packed binary32 pairs (sm_100 f32x2 arithmetic): a * b + c and a + b, lane-wise.
+__device__ __forceinline__ float2 fma2(float2 a, float b, float c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %4};\n\t"
+      "mov.b64 rc, {%5, %5};\n\tfma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+// p = 2^a for a pair, rounded to the 16-bit type and packed (lo in the low half); the
+// rounded values are added to `sum` as a pair.
+template <int QD>
+__device__ __forceinline__ uint32_t exp2_pack(float2 a, float2& sum) {
+  const float p0 = ex2(a.x), p1 = ex2(a.y);
+  uint32_t w;
+  float2 r;
+  if constexpr (QD == PA_BF16) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(p0, p1);
+    w = *reinterpret_cast<const uint32_t*>(&v);
+    r = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+  } else {
+    __half2 v = __floats2half2_rn(p0, p1);
+    w = *reinterpret_cast<const uint32_t*>(&v);
+    r = __half22float2(v);
+  }
+  sum = add2(sum, r);
+  return w;
+}
+
 // 2-D tiled TMA load (box given by the tensor map) signalling `bar` with its bytes.
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
   asm volatile(
@@ -480,17 +518,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         uint8_t* sP = sm + TcSmem::kP + b * TcSmem::kTile;
         auto make_p = [&](float ref) {   // P = 2^(s * scale - ref) into sP; returns its rounded sum
           const float nmb = -ref;
-          float l8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+          float2 l2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             uint32_t w[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e)
-              w[e] = pack2_sum<QD>(ex2(fmaf(s[c * 8 + 2 * e], p.s_mul, nmb)),
-                                   ex2(fmaf(s[c * 8 + 2 * e + 1], p.s_mul, nmb)), l8[(c & 1) * 4 + e]);
+              w[e] = exp2_pack<QD>(fma2(make_float2(s[c * 8 + 2 * e], s[c * 8 + 2 * e + 1]), p.s_mul, nmb), l2[e]);
             *reinterpret_cast<uint4*>(sP + tc_swz(row, hf * 8 + c)) = make_uint4(w[0], w[1], w[2], w[3]);
           }
-          return ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
+          return ((l2[0].x + l2[0].y) + (l2[1].x + l2[1].y)) + ((l2[2].x + l2[2].y) + (l2[3].x + l2[3].y));
         };
         // speculatively with the current reference while the partner's maximum is in flight:
         // it stands unless the pair's maximum passes the reference by more than 2^8
@@ -566,19 +603,30 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int P = has_q ? (qpos + 1 + p.chunk - 1) / p.chunk : 0;
       const bool wr = has_q && x.part < P;
       const bool fin = wr && P == 1;
-      if (fin) {
+      if (fin) {   // this half of the row, rounded, staged in P buffer 0 (every P V has completed)
         const float inv = 1.f / lsum;
-        uint4* orow =
-            reinterpret_cast<uint4*>(static_cast<QT*>(p.out) + (size_t(tok) * Hq + head) * kTcD + hf * 64);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           float dummy = 0.f;
           uint32_t w[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) w[e] = pack2_sum<QD>(o[i * 8 + 2 * e] * inv, o[i * 8 + 2 * e + 1] * inv, dummy);
-          orow[i] = make_uint4(w[0], w[1], w[2], w[3]);
+          *reinterpret_cast<uint4*>(sm + TcSmem::kP + tc_swz(row, hf * 8 + i)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
-      } else if (wr) {
+      }
+      __syncwarp();
+      // coalesced: each store instruction writes 4 rows x 128 contiguous bytes
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int rr = rw * 32 + i * 4 + (lane >> 3), c = lane & 7;
+        const int rqi = x.t * QPT + rr / G;
+        if (x.part == 0 && rqi < x.Q && x.base + rqi + 1 <= p.chunk) {   // that row's whole context is here
+          QT* orow = static_cast<QT*>(p.out) + (size_t(x.row0 + rqi) * Hq + x.hk * G + rr % G) * kTcD + hf * 64;
+          *reinterpret_cast<uint4*>(orow + c * 8) = *reinterpret_cast<const uint4*>(sm + TcSmem::kP + tc_swz(rr, hf * 8 + c));
+        }
+      }
+      __syncwarp();
+      if (wr && !fin) {   // this chunk's partial: unnormalised half row, (max, sum) once
         const size_t slot = (size_t(tok) * Hq + head) * p.max_parts + x.part;
         float4* acc = reinterpret_cast<float4*>(p.part_acc + slot * kTcD + hf * 64);
 #pragma unroll
