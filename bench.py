@@ -389,16 +389,39 @@ def time_extend(name, steps, warmup, device, subset=0):
     def call():
         pa.extend(q, eng.cache, qs_dev, eng.bt_dev, eng.lens_dev, eng.max_context_len, w.scale, out, ws)
 
-    for _ in range(warmup):
-        call()
-    torch.cuda.synchronize(device)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(steps):
-        call()
-    e1.record()
-    torch.cuda.synchronize(device)
-    ms = e0.elapsed_time(e1) / steps
+    def timed(fn):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize(device)
+        return e0.elapsed_time(e1) / steps
+
+    ms = timed(call)
+    prefill = None
+    if name == "prefill_8x2k":
+        # the whole prefill step: the prompts' K / V into the cache plus the attention, as
+        # one fused pa_prefill and as pa_reshape_and_cache followed by pa_extend
+        k_new = synthetic.normal_values((T, w.num_kv_heads, w.head_dim), w.kv_dtype, w.seed + 12, device)
+        v_new = synthetic.normal_values((T, w.num_kv_heads, w.head_dim), w.kv_dtype, w.seed + 13, device)
+        BS = w.block_size
+        slots = np.concatenate([eng.bt_host[s, np.arange(L) // BS].astype(np.int64) * BS + np.arange(L) % BS
+                                for s, L in enumerate(w.context_lens)])
+        slots_dev = torch.from_numpy(slots).to(device)
+
+        def fused():
+            pa.prefill(q, k_new, v_new, eng.cache, qs_dev, eng.bt_dev, eng.lens_dev, eng.max_context_len, w.scale,
+                       out, ws)
+
+        def two_pass():
+            pa.reshape_and_cache(k_new, v_new, slots_dev, eng.cache)
+            call()
+
+        prefill = {"fused_ms": timed(fused), "reshape_then_extend_ms": timed(two_pass)}
     lens = np.asarray(w.context_lens, dtype=np.int64)
     kv_bytes = int(2 * lens.sum() * w.num_kv_heads * w.head_dim * 2) + 2 * T * w.num_q_heads * w.head_dim * 2
     flops = 0
@@ -407,8 +430,14 @@ def time_extend(name, steps, warmup, device, subset=0):
         flops += int(4 * w.num_q_heads * w.head_dim * (pos + 1).sum())
     del eng
     torch.cuda.empty_cache()
-    return {"workload": name, "ms_per_call": ms, "kv_gbs": kv_bytes / (ms / 1e3) / 1e9,
-            "tflops": flops / (ms / 1e3) / 1e12, "query_rows": T, "kv_bytes": kv_bytes, "flops": flops}
+    res = {"workload": name, "ms_per_call": ms, "kv_gbs": kv_bytes / (ms / 1e3) / 1e9,
+           "tflops": flops / (ms / 1e3) / 1e12, "query_rows": T, "kv_bytes": kv_bytes, "flops": flops}
+    if prefill is not None:
+        prefill["fused_tflops"] = flops / (prefill["fused_ms"] / 1e3) / 1e12
+        prefill["note"] = ("whole prefill step = the prompts' K/V written to the cache + attention; "
+                           "ms_per_call / tflops above time the attention alone (pa_extend)")
+        res["prefill_step"] = prefill
+    return res
 
 
 # ---------------------------------------------------------------------------

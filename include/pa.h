@@ -242,6 +242,35 @@ size_t pa_extend_workspace_size(int32_t num_seqs, int32_t num_tokens, int32_t nu
                                 int32_t max_context_len);
 
 /*
+ * pa_prefill -- causal attention of whole prompts over themselves, writing the prompts'
+ * K / V into the paged cache in the same pass. Page 2, section "2.1 核心组件交互流程":
+ * the engine's prefill mode processes the prompt and fills the KV cache that decode then
+ * reads (paged layout of page 3, section "PagedAttention原理").
+ *   q              device [num_tokens][num_q_heads][head_dim], dtype
+ *   k, v           device [num_tokens][num_kv_heads][head_dim], dtype: the prompts' keys
+ *                  and values, rows in query order (as pa_reshape_and_cache takes them)
+ *   query_start    device int32 [num_seqs + 1]: sequence s owns rows query_start[s] ..
+ *                  query_start[s+1]-1 (its prompt of Q_s tokens), query_start[0] = 0
+ *   context_lens   device int32 [num_seqs]: must equal Q_s (a prompt attends to itself);
+ *                  otherwise the sequence is recorded (PA_DEV_BAD_CONTEXT_LEN) and its rows
+ *                  are zero
+ *   block_tables   device int32 [num_seqs][max_blocks_per_seq]: blocks that belong to the
+ *                  sequence alone (freshly allocated), covering its Q_s tokens
+ *   out            device [num_tokens][num_q_heads][head_dim], dtype
+ * Afterwards cache slot bt[s][i / BS] * BS + i % BS holds k / v of prompt token i, bit for
+ * bit, for every i < Q_s; the slots past Q_s in a prompt's last block hold unspecified
+ * values. out is as pa_extend computes it with those cache contents.
+ * Supported: dtype = the cache's kv_dtype = PA_F16 or PA_BF16, head_dim 128, block_size 16
+ * or 32, G in {1, 2, 4, 8}, scale > 0 (the tcgen05 path); PA_ERR_ARG otherwise. workspace
+ * >= pa_extend_workspace_size(...), 256-byte aligned; k, v, q and out 16-byte aligned.
+ */
+pa_status pa_prefill(const void* q, const void* k, const void* v, int32_t dtype, int32_t num_seqs,
+                     int32_t num_q_heads, const int32_t* query_start, int32_t num_tokens, const pa_cache_desc* cache,
+                     const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
+                     int32_t max_context_len, float scale, void* out, void* workspace, size_t workspace_bytes,
+                     void* stream);
+
+/*
  * pa_last_device_error -- synchronise `stream`, then read and clear the device error
  * word of the current device. *code receives a PA_DEV_* value; info (may be NULL)
  * receives 3 int32 details. Returns PA_ERR_DEVICE_CHECK when *code != 0.

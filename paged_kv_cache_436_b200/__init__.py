@@ -105,6 +105,8 @@ _SIGNATURES = {
     "pa_extend": (_I32, [_P, _I32, _I32, _I32, _P, _I32, _PDESC, _P, _I32, _P, _I32, ctypes.c_float, _P, _P,
                          ctypes.c_size_t, _P]),
     "pa_extend_workspace_size": (ctypes.c_size_t, [_I32, _I32, _I32, _I32, _I32]),
+    "pa_prefill": (_I32, [_P, _P, _P, _I32, _I32, _I32, _P, _I32, _PDESC, _P, _I32, _P, _I32, ctypes.c_float, _P,
+                          _P, ctypes.c_size_t, _P]),
     "pa_version": (ctypes.c_char_p, []),
 }
 
@@ -242,6 +244,19 @@ def extend(q, cache: KVCache, query_start, block_tables, context_lens, max_conte
                          float(scale), _ptr(out), _ptr(workspace), workspace.numel() * workspace.element_size(),
                          _stream(stream))
     _check(st, "pa_extend")
+
+
+def prefill(q, k, v, cache: KVCache, query_start, block_tables, context_lens, max_context_len: int, scale: float,
+            out, workspace, stream=None) -> None:
+    """Whole prompts: q, out [T, Hq, D]; k, v [T, Hkv, D] (the prompts' keys and values, written
+    into the cache by the same kernel); query_start int32 [S + 1]; context_lens = prompt lengths."""
+    T, Hq, _ = q.shape
+    S = query_start.shape[0] - 1
+    st = lib().pa_prefill(_ptr(q), _ptr(k), _ptr(v), dtype_code(q), S, Hq, _ptr(query_start), T,
+                          ctypes.byref(cache.desc), _ptr(block_tables), block_tables.shape[1], _ptr(context_lens),
+                          int(max_context_len), float(scale), _ptr(out), _ptr(workspace),
+                          workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "pa_prefill")
 
 
 NO_ALLOC_WORKSPACE_BYTES = 16 << 20

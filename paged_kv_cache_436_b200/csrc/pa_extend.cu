@@ -46,6 +46,7 @@ struct ExtendParams {
   int4* units;                  // optional: two int4 per (seq, tile, chunk) pair, written by the plan
                                 //   {s, tile, chunk index, row0}, {Q, base, first token, visible tokens}
   long long units_cap;          // pairs the records can hold
+  int fresh;                    // whole prompts (pa_prefill): every L_s must equal Q_s
 };
 
 constexpr int kTileRows = 16;
@@ -57,7 +58,7 @@ __device__ __forceinline__ void ext_seq(const ExtendParams& p, int s, int& Q, in
   const int L = ext_clamp(p.context_lens[s], 0, p.len_limit);
   const int q0 = p.query_start[s], q1 = p.query_start[s + 1];
   Q = q1 - q0;
-  if (Q < 0 || Q > L || q0 < 0 || q1 > p.num_tokens) Q = 0;   // invalid: recorded by the plan, no work
+  if (Q < 0 || Q > L || q0 < 0 || q1 > p.num_tokens || (p.fresh && Q != L)) Q = 0;   // invalid: recorded, no work
   base = L - Q;
 }
 
@@ -843,7 +844,8 @@ cudaError_t ext_launch(ExtKernel fn, int grid, int threads, size_t smem, cudaStr
 // tcgen05 path for long query runs (pa_extend_tc.cu)
 bool extend_tc_supported(int qd, int D, int BS, int G);
 cudaError_t extend_tc_grid_cap(int qd, int BS, int G, int* cap);
-pa_status extend_tc_launch(const ExtendParams& p, const pa_cache_desc* c, int qd, int G, int grid, cudaStream_t s);
+pa_status extend_tc_launch(const ExtendParams& p, const pa_cache_desc* c, int qd, int G, int grid, cudaStream_t s,
+                           const void* k_new, const void* v_new);
 constexpr int kTcUnitRows = 128;
 
 }  // namespace pa
@@ -857,12 +859,17 @@ size_t pa_extend_workspace_size(int32_t num_seqs, int32_t num_tokens, int32_t nu
   return pa::ext_ws(num_seqs, num_tokens, num_q_heads, head_dim, mp).total;
 }
 
-pa_status pa_extend(const void* q, int32_t q_dtype, int32_t num_seqs, int32_t num_q_heads,
-                    const int32_t* query_start, int32_t num_tokens, const pa_cache_desc* c,
-                    const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
-                    int32_t max_context_len, float scale, void* out, void* workspace, size_t workspace_bytes,
-                    void* stream) {
-  using namespace pa;
+}  // extern "C"
+
+namespace pa {
+
+// pa_extend (k_new = v_new = null) and pa_prefill (fresh: the prompts' K / V in k_new,
+// v_new, written into the cache by the same kernel).
+static pa_status extend_impl(const void* q, int32_t q_dtype, int32_t num_seqs, int32_t num_q_heads,
+                             const int32_t* query_start, int32_t num_tokens, const pa_cache_desc* c,
+                             const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
+                             int32_t max_context_len, float scale, void* out, void* workspace,
+                             size_t workspace_bytes, void* stream, const void* k_new, const void* v_new, bool fresh) {
   pa_status st = validate_cache(c);
   if (st != PA_OK) return st;
   if (c->kv_dtype == PA_E4M3 || q_dtype != c->kv_dtype) return PA_ERR_ARG;   // 16-bit caches only
@@ -885,8 +892,9 @@ pa_status pa_extend(const void* q, int32_t q_dtype, int32_t num_seqs, int32_t nu
   // tcgen05 kernel (head_dim 128) or, otherwise, the cooperative 64-row kernel; short
   // ones (speculative drafts, decode) to the 16-row warp kernel.
   const long long rows_total = (long long)num_tokens * G;
-  const bool tc = rows_total * 2 >= (long long)kTcUnitRows * num_seqs && scale > 0.f &&
+  const bool tc = (fresh || rows_total * 2 >= (long long)kTcUnitRows * num_seqs) && scale > 0.f &&
                   extend_tc_supported(q_dtype, D, BS, G);
+  if (fresh && (!tc || !k_new || !v_new || !aligned16(k_new) || !aligned16(v_new))) return PA_ERR_ARG;
   const bool coop = !tc && rows_total > (long long)kTileRows * num_seqs;
   ExtLaunch k;
   if (!tc) {
@@ -908,6 +916,7 @@ pa_status pa_extend(const void* q, int32_t q_dtype, int32_t num_seqs, int32_t nu
   p.part_acc = reinterpret_cast<float*>(w + ws.acc);
   p.units = tc ? reinterpret_cast<int4*>(w + ws.units) : nullptr;
   p.units_cap = (long long)ext_units_bound(num_tokens, num_q_heads, max_parts);
+  p.fresh = fresh ? 1 : 0;
   p.num_seqs = num_seqs;
   p.num_tokens = num_tokens;
   p.num_q_heads = num_q_heads;
@@ -954,7 +963,7 @@ pa_status pa_extend(const void* q, int32_t q_dtype, int32_t num_seqs, int32_t nu
   extend_plan_kernel<<<1, 1024, 0, s>>>(p, rows_per_unit / G);
   if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
   if (tc) {
-    st = extend_tc_launch(p, c, q_dtype, G, grid, s);
+    st = extend_tc_launch(p, c, q_dtype, G, grid, s, k_new, v_new);
     if (st != PA_OK) return st;
   } else if (ext_launch(k.fn, grid, k.threads, k.smem, s, p) != cudaSuccess) {
     return PA_ERR_CUDA;
@@ -966,6 +975,30 @@ pa_status pa_extend(const void* q, int32_t q_dtype, int32_t num_seqs, int32_t nu
     if (ext_launch(red, int(rows), 128, size_t(max_parts) * 4, s, p) != cudaSuccess) return PA_ERR_CUDA;
   }
   return PA_OK;
+}
+
+}  // namespace pa
+
+extern "C" {
+
+pa_status pa_extend(const void* q, int32_t q_dtype, int32_t num_seqs, int32_t num_q_heads,
+                    const int32_t* query_start, int32_t num_tokens, const pa_cache_desc* c,
+                    const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
+                    int32_t max_context_len, float scale, void* out, void* workspace, size_t workspace_bytes,
+                    void* stream) {
+  return pa::extend_impl(q, q_dtype, num_seqs, num_q_heads, query_start, num_tokens, c, block_tables,
+                         max_blocks_per_seq, context_lens, max_context_len, scale, out, workspace, workspace_bytes,
+                         stream, nullptr, nullptr, false);
+}
+
+pa_status pa_prefill(const void* q, const void* k, const void* v, int32_t dtype, int32_t num_seqs,
+                     int32_t num_q_heads, const int32_t* query_start, int32_t num_tokens, const pa_cache_desc* c,
+                     const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
+                     int32_t max_context_len, float scale, void* out, void* workspace, size_t workspace_bytes,
+                     void* stream) {
+  return pa::extend_impl(q, dtype, num_seqs, num_q_heads, query_start, num_tokens, c, block_tables,
+                         max_blocks_per_seq, context_lens, max_context_len, scale, out, workspace, workspace_bytes,
+                         stream, k, v, true);
 }
 
 }  // extern "C"

@@ -238,6 +238,16 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, i
       : "memory");
 }
 
+// 2-D tiled TMA store shared -> global (bulk async-group of the issuing thread).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, int x, int y, const void* src) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(map), "r"(x),
+               "r"(y), "r"(smem_addr(src))
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // Byte offset of 16-byte chunk c (0..15) of row r in a [128 x 128] 16-bit tile kept
 // as two 128B-swizzled K-major halves of 64 columns (8-row atoms of 1 KB).
 __device__ __forceinline__ uint32_t tc_swz(int r, int c) {
@@ -292,7 +302,8 @@ __device__ __forceinline__ bool tc_wait_warp(uint64_t* bar, uint32_t parity, vol
 template <int QD, int BS, int G>
 __global__ void __launch_bounds__(kTcThreads, 1)
     extend_tc_kernel(const ExtendParams p, const __grid_constant__ CUtensorMap tk,
-                     const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tq) {
+                     const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tq,
+                     const __grid_constant__ CUtensorMap tkn, const __grid_constant__ CUtensorMap tvn) {
   using QT = typename Q<QD>::T;
   constexpr int QPT = kTcRows / G;                    // queries per unit
   constexpr int BPT = kTcTok / BS;                    // cache blocks per K/V tile
@@ -353,6 +364,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint64_t* empty = is_v ? pv_done : k_empty;   // V(g) after P(g-2) V(g-2); K(g) after S(g-2)
     const CUtensorMap* map = is_v ? &tv : &tk;
     uint8_t* ring = sm + (is_v ? TcSmem::kV : TcSmem::kK);
+    const CUtensorMap* in_map = is_v ? &tvn : &tkn;   // whole prompts: the prompt's K or V rows
+    int pend_g = -1, pend_nbw = 0, pend_y = 0;        // a loaded tile still to be written to the cache
+    auto flush_store = [&]() {
+      if (pend_g < 0) return true;
+      const int b = pend_g & 1;
+      if (!tc_wait_warp(&full[b], (uint32_t(pend_g) >> 1) & 1, abort, 27, pend_g)) return false;
+      if (lane < pend_nbw) {
+        const uint8_t* src = ring + b * TcSmem::kTile + lane * (BS * 128);
+        tma_store_2d(map, 0, pend_y, src);
+        tma_store_2d(map, 64, pend_y, src + kTcTok * 128);
+        bulk_commit();
+      }
+      pend_g = -1;
+      return true;
+    };
     uint32_t g = 0, k = 0;
     for (int u = blockIdx.x; u < total && !*abort; u += gridDim.x, ++k) {
       const TcUnit x = tc_unit(p, u);
@@ -367,22 +393,47 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       const int32_t* trow = p.block_tables + size_t(x.s) * p.max_blocks;
       auto blocks = [&](int j) { return min(BPT, (x.nvis - j * kTcTok + BS - 1) / BS); };
-      auto fetch = [&](int j) {   // block id of this lane's block of tile j
-        const int lb = (x.t0 + j * kTcTok) / BS + lane;
+      auto fetch = [&](int lb, int n) {   // block id of this lane's block (lane < n), checked
         int id = 0;
-        if (lane < blocks(j)) {
-          id = trow[lb];
+        if (lane < n) {
+          id = trow[lb + lane];
           if (id < 0 || id >= p.num_blocks) {
-            if (!is_v) record_error(PA_DEV_BAD_BLOCK_ID, x.s, lb, id);
+            if (!is_v) record_error(PA_DEV_BAD_BLOCK_ID, x.s, lb + lane, id);
             id = 0;
           }
         }
         return id;
       };
-      int id = fetch(0);
+      if (p.fresh) {
+        // whole prompts: tiles come from the prompt's own K / V rows, 128 rows per box;
+        // the row tile that sees all of a K/V tile's prompt positions also writes that
+        // tile into its cache blocks (TMA stores, once its load has landed)
+        bool ok = true;
+        for (int j = 0; j < x.ntiles; ++j, ++g) {
+          const int b = g & 1, p0 = x.t0 + j * kTcTok;
+          if (!(ok = tc_wait_warp(&empty[b], ((g >> 1) & 1) ^ 1, abort, is_v ? 11 : 10, u))) break;
+          bulk_wait_read_all();   // the stores that read this buffer two tiles ago
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&full[b], TcSmem::kTile);
+            tma_load_3d(ring + b * TcSmem::kTile, in_map, 0, x.hk, x.row0 + p0, &full[b]);
+            tma_load_3d(ring + b * TcSmem::kTile + kTcTok * 128, in_map, 64, x.hk, x.row0 + p0, &full[b]);
+          }
+          __syncwarp();
+          last_load = g + 1;
+          if (!(ok = flush_store())) break;
+          if (x.t == min((p0 + kTcTok - 1) / QPT, (x.Q - 1) / QPT)) {
+            pend_nbw = (min(p0 + kTcTok, x.Q) - p0 + BS - 1) / BS;
+            pend_y = (fetch(p0 / BS, pend_nbw) * Hkv + x.hk) * BS;
+            pend_g = int(g);
+          }
+        }
+        if (!ok) break;
+        continue;
+      }
+      int id = fetch(x.t0 / BS, blocks(0));
       for (int j = 0; j < x.ntiles; ++j, ++g) {
         const int b = g & 1, nb = blocks(j);
-        const int next = j + 1 < x.ntiles ? fetch(j + 1) : 0;   // read ahead of its use
+        const int next = j + 1 < x.ntiles ? fetch((x.t0 + (j + 1) * kTcTok) / BS, blocks(j + 1)) : 0;
         const int y = (id * Hkv + x.hk) * BS;
         uint8_t* dst = ring + b * TcSmem::kTile + lane * (BS * 128);
         if (!tc_wait_warp(&empty[b], ((g >> 1) & 1) ^ 1, abort, is_v ? 11 : 10, u)) break;
@@ -396,6 +447,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         id = next;
       }
     }
+    if (p.fresh && !*abort) flush_store();
+    bulk_wait_all();   // this thread's cache stores are complete before the kernel ends
   } else if (warp == kTcSoftmaxWarps) {
     // ---------------- MMA issue: S(g) then O += P(g-1) V(g-1) ----------------
     const uint32_t idS = tc_idesc<QD>(0), idO = tc_idesc<QD>(1);
@@ -701,7 +754,19 @@ bool q_tmap(TmapEncodeFn enc, CUtensorMap* m, const void* q, int qd, int num_tok
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-using TcKernel = void (*)(const ExtendParams, const CUtensorMap, const CUtensorMap, const CUtensorMap);
+// The prompts' own K / V ([tokens][kv heads][head_dim]); box = 64 dims x 1 head x 128 tokens.
+bool kv_in_tmap(TmapEncodeFn enc, CUtensorMap* m, const void* kv, int qd, int num_tokens, int Hkv) {
+  const cuuint64_t dims[3] = {cuuint64_t(kTcD), cuuint64_t(Hkv), cuuint64_t(num_tokens)};
+  const cuuint64_t strides[2] = {cuuint64_t(kTcD) * 2, cuuint64_t(Hkv) * kTcD * 2};
+  const cuuint32_t box[3] = {64, 1, cuuint32_t(kTcTok)};
+  const cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, qd == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+             const_cast<void*>(kv), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+using TcKernel = void (*)(const ExtendParams, const CUtensorMap, const CUtensorMap, const CUtensorMap,
+                          const CUtensorMap, const CUtensorMap);
 
 template <int QD, int BS>
 TcKernel tc_pick_g(int G) {
@@ -736,7 +801,7 @@ cudaError_t extend_tc_grid_cap(int qd, int BS, int G, int* cap) {
 // Launch after the plan kernel (programmatic dependent launch). The cache base pointers
 // are 16-byte aligned and the rows 256 bytes, as the tensor maps require.
 pa_status extend_tc_launch(const ExtendParams& p, const pa_cache_desc* c, int qd, int G, int grid,
-                           cudaStream_t s) {
+                           cudaStream_t s, const void* k_new, const void* v_new) {
   TcKernel fn = tc_pick(qd, c->block_size, G);
   TmapEncodeFn enc = tmap_encoder();
   if (!fn || !enc) return PA_ERR_ARG;
@@ -745,6 +810,10 @@ pa_status extend_tc_launch(const ExtendParams& p, const pa_cache_desc* c, int qd
   if (!cache_tmap(enc, &tk, c->k_cache, qd, rows, c->block_size) ||
       !cache_tmap(enc, &tv, c->v_cache, qd, rows, c->block_size) ||
       !q_tmap(enc, &tq, p.q, qd, p.num_tokens, p.num_q_heads, G))
+    return PA_ERR_ARG;
+  CUtensorMap tkn = tk, tvn = tv;   // used only for whole prompts
+  if (p.fresh && (!kv_in_tmap(enc, &tkn, k_new, qd, p.num_tokens, c->num_kv_heads) ||
+                  !kv_in_tmap(enc, &tvn, v_new, qd, p.num_tokens, c->num_kv_heads)))
     return PA_ERR_ARG;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
@@ -756,7 +825,7 @@ pa_status extend_tc_launch(const ExtendParams& p, const pa_cache_desc* c, int qd
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, fn, p, tk, tv, tq) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  return cudaLaunchKernelEx(&cfg, fn, p, tk, tv, tq, tkn, tvn) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 }  // namespace pa
