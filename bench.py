@@ -581,7 +581,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="llama13b_mix")
-    ap.add_argument("--also", default="long_fp8", help="second workload reported in the same line ('' = none)")
+    ap.add_argument("--also", default="long_fp8,prefill_8x2k,spec4_mix",
+                    help="further workloads reported in the same line ('' = none)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle's cpu_baseline leg")
