@@ -8,9 +8,10 @@
 //     512-token partition, chosen by the host so that there are enough units to fill
 //     the GPU (the whole context when there are, then no merge pass at all); the plan
 //     kernel writes one record per (sequence, tile, chunk);
-//   * one persistent CTA per SM with warp-specialised roles: 8 softmax warps (warps w
-//     and w + 4 share TMEM lanes 32 (w % 4) .. + 31, i.e. rows of the tile, and split
-//     the 128 columns into halves), one MMA-issue warp, one K and one V producer warp;
+//   * one persistent CTA per SM with warp-specialised roles: 8 softmax warps (warps w and
+//     w + 4 share TMEM lanes 32 (w % 4) .. + 31, i.e. rows of the tile, and split the 128
+//     columns into slices of 64: more slices put more warps in lockstep on the same SM
+//     sub-partition and measured slower), one MMA-issue warp, one K and one V producer warp;
 //   * TMEM: S of two consecutive 128-token K/V tiles in columns [0, 256), the output
 //     accumulators O of two consecutive units in [256, 512);
 //   * the unit's Q rows come by one 3-D TMA box per 64-column half (64 dims x G heads x
@@ -25,7 +26,7 @@
 //   * the softmax reads its half of the S row from TMEM, masks causally and keeps a
 //     reference maximum that moves only when the row maximum passes it by more than 2^8
 //     (O and the running sum are then rescaled; every p stays below 2^8, so nothing is
-//     lost). The pair's maximum is combined through a TMEM column and a 2-arrival
+//     lost). The group's maximum is combined through TMEM columns and a kTcSplit-arrival
 //     mbarrier; P is computed speculatively with the current reference meanwhile and
 //     recomputed only when the reference moves. P goes to a swizzled K-major shared
 //     tile in the query's 16-bit type and the running sum adds those rounded values;
@@ -43,7 +44,8 @@ constexpr int kTcRows = 128;            // query rows per unit (TMEM lanes)
 constexpr int kTcTok = 128;             // tokens per K/V tile
 constexpr int kTcD = 128;               // head_dim of this path
 constexpr uint32_t kTcTmemCols = 512;   // S double buffer [0, 256), O double buffer [256, 512)
-constexpr int kTcSoftmaxWarps = 8;      // two per row group; + an MMA-issue warp + K and V producer warps
+constexpr int kTcSplit = 2;             // softmax warps per 32-row group (column slices)
+constexpr int kTcSoftmaxWarps = 4 * kTcSplit;   // + an MMA-issue warp + K and V producer warps
 constexpr int kTcThreads = (kTcSoftmaxWarps + 3) * 32;
 constexpr float kTcRescale = 8.f;       // log2 units
 
@@ -313,7 +315,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint8_t* sQ = sm + TcSmem::kQ;
   // per-tile ring barriers (index = tile & 1); per-unit ones (q_full, o_full/o_empty by unit & 1)
   __shared__ uint64_t k_full[2], v_full[2], k_empty[2], pv_done[2], s_full[2], s_empty[2], p_full[2];
-  __shared__ uint64_t q_full, q_empty, o_full[2], o_empty[2], bar_fin, pair_bar[4];
+  __shared__ uint64_t q_full, q_empty, o_full[2], o_empty[2], bar_fin, grp_bar[4];
   __shared__ uint32_t tmem_slot;
   __shared__ int s_abort;
   volatile int* abort = &s_abort;
@@ -339,7 +341,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     mbar_init(&q_full, 1);
     mbar_init(&q_empty, 1);
-    for (int i = 0; i < 4; ++i) mbar_init(&pair_bar[i], 2);
+    for (int i = 0; i < 4; ++i) mbar_init(&grp_bar[i], kTcSplit);
     mbar_init(&bar_fin, 1);
     s_abort = 0;
     fence_mbar_init();
@@ -504,68 +506,70 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   } else {
     // ---------------- softmax warps ----------------
-    // Warps w and w + 4 share TMEM lanes 32 (w % 4) .. + 31 (rows of the tile) and split
-    // the columns: half hf = w / 4 holds score / P / O columns [64 hf, 64 hf + 64). The
-    // pair combines its row maxima and sums through one TMEM column each has already read
-    // (its own first column of the S or O buffer) and a 2-arrival mbarrier.
-    const int hf = warp >> 2, rw = warp & 3, row = rw * 32 + lane;
+    // Warps w, w + 4, w + 8, ... share TMEM lanes 32 (w % 4) .. + 31 (rows of the tile) and
+    // split the columns: slice q = w / 4 holds score / P / O columns [kCW q, kCW q + kCW).
+    // The group combines its row maxima and sums through one TMEM column each has already
+    // read (its own first column of the S or O buffer) and a kTcSplit-arrival mbarrier.
+    constexpr int kCW = kTcTok / kTcSplit;             // columns per warp
+    const int qs_ = warp >> 2, rw = warp & 3, row = rw * 32 + lane;
     const uint32_t t_row = tmem + (uint32_t(rw * 32) << 16);
-    uint32_t xc = 0;   // pair exchanges so far
-    auto exchange = [&](uint32_t col_own, uint32_t col_other, float v, int u, float* other) {
+    uint32_t xc = 0;   // group exchanges so far
+    auto publish = [&](uint32_t col_own, float v) {
       tc_st1(t_row + col_own, __float_as_uint(v));
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&pair_bar[rw]);
-      const bool ok = tc_wait_warp(&pair_bar[rw], xc & 1, abort, 23, u);
+      if (lane == 0) mbar_arrive(&grp_bar[rw]);
+    };
+    // all slices' values in slice order (identical in every warp of the group)
+    auto gather = [&](uint32_t col0, float own, int u, float* all) {
+      const bool ok = tc_wait_warp(&grp_bar[rw], xc & 1, abort, 23, u);
       ++xc;
       if (!ok) return false;
       tc_fence_after();
-      *other = __uint_as_float(tc_ld1(t_row + col_other));
+#pragma unroll
+      for (int q = 0; q < kTcSplit; ++q)
+        all[q] = q == qs_ ? own : __uint_as_float(tc_ld1(t_row + col0 + q * kCW));
       return true;
     };
     uint32_t g = 0, k = 0;
     for (int u = blockIdx.x; u < total; u += gridDim.x, ++k) {
       const TcUnit x = tc_unit(p, u);
-      const uint32_t ob = k & 1, c_o = 256 + ob * 128 + hf * 64;   // this half of the O buffer
+      const uint32_t ob = k & 1, c_o = 256 + ob * 128 + qs_ * kCW;   // this slice of the O buffer
       const int qi = x.t * QPT + row / G;
       const int head = x.hk * G + row % G;
       const bool has_q = qi < x.Q;
       const int qpos = has_q ? x.base + qi : -1;
       const int tok = has_q ? x.row0 + qi : -1;
-      float m_ref = -INFINITY, l = 0.f;   // l: this half's share of the row sum
+      float m_ref = -INFINITY, l = 0.f;   // l: this slice's share of the row sum
       bool ok = true;
       for (int j = 0; j < x.ntiles; ++j, ++g) {
         const int b = g & 1;
-        const uint32_t c_s = b * 128 + hf * 64;                      // this half of S(g)
+        const uint32_t c_s = b * 128 + qs_ * kCW;                    // this slice of S(g)
         if (!(ok = tc_wait_warp(&s_full[b], (g >> 1) & 1, abort, 18, u))) break;
         tc_fence_after();
-        float s[64];
+        float s[kCW];
         {
-          uint32_t r[64];
-          tc_ld32_async(t_row + c_s, r);
-          tc_ld32_async(t_row + c_s + 32, r + 32);
+          uint32_t r[kCW];
+#pragma unroll
+          for (int c = 0; c < kCW / 32; ++c) tc_ld32_async(t_row + c_s + c * 32, r + c * 32);
           tc_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(pin_after_wait(r[c]));
+          for (int c = 0; c < kCW; ++c) s[c] = __uint_as_float(pin_after_wait(r[c]));
         }
-        // causal mask, this half's maximum (8 independent chains), then the pair's
-        const int tp0 = x.t0 + j * kTcTok + hf * 64;
-        if (tp0 + 63 > qpos) {
+        // causal mask, this slice's maximum (8 independent chains)
+        const int tp0 = x.t0 + j * kTcTok + qs_ * kCW;
+        if (tp0 + kCW - 1 > qpos) {
 #pragma unroll
-          for (int c = 0; c < 64; ++c) s[c] = tp0 + c > qpos ? -INFINITY : s[c];
+          for (int c = 0; c < kCW; ++c) s[c] = tp0 + c > qpos ? -INFINITY : s[c];
         }
         float m8[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) m8[e] = s[e];
 #pragma unroll
-        for (int c = 8; c < 64; ++c) m8[c & 7] = fmaxf(m8[c & 7], s[c]);
+        for (int c = 8; c < kCW; ++c) m8[c & 7] = fmaxf(m8[c & 7], s[c]);
         const float pm = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
                                fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-        // publish this half's maximum to the partner warp (own first S column, already read)
-        tc_st1(t_row + c_s, __float_as_uint(pm));
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&pair_bar[rw]);
+        publish(c_s, pm);
         // P(g) goes into buffer b once P(g-2) V(g-2) has finished reading it
         if (!(ok = tc_wait_warp(&pv_done[b], ((g >> 1) & 1) ^ 1, abort, 20, u))) break;
         uint8_t* sP = sm + TcSmem::kP + b * TcSmem::kTile;
@@ -573,28 +577,28 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const float nmb = -ref;
           float2 l2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
+          for (int c = 0; c < kCW / 8; ++c) {
             uint32_t w[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e)
               w[e] = exp2_pack<QD>(fma2(make_float2(s[c * 8 + 2 * e], s[c * 8 + 2 * e + 1]), p.s_mul, nmb), l2[e]);
-            *reinterpret_cast<uint4*>(sP + tc_swz(row, hf * 8 + c)) = make_uint4(w[0], w[1], w[2], w[3]);
+            *reinterpret_cast<uint4*>(sP + tc_swz(row, qs_ * (kCW / 8) + c)) = make_uint4(w[0], w[1], w[2], w[3]);
           }
           return ((l2[0].x + l2[0].y) + (l2[1].x + l2[1].y)) + ((l2[2].x + l2[2].y) + (l2[3].x + l2[3].y));
         };
-        // speculatively with the current reference while the partner's maximum is in flight:
-        // it stands unless the pair's maximum passes the reference by more than 2^8
+        // speculatively with the current reference while the others' maxima are in flight:
+        // it stands unless the row maximum passes the reference by more than 2^8
         const bool spec = m_ref != -INFINITY && pm * p.s_mul <= m_ref + kTcRescale;
         float lt = spec ? make_p(m_ref) : 0.f;
-        const bool okp = tc_wait_warp(&pair_bar[rw], xc & 1, abort, 23, u);
-        ++xc;
-        if (!(ok = okp)) break;
-        tc_fence_after();
-        const float po = __uint_as_float(tc_ld1(t_row + b * 128 + (hf ^ 1) * 64));
+        float pms[kTcSplit];
+        if (!(ok = gather(b * 128, pm, u, pms))) break;
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_empty[b]);
-        const float mx = fmaxf(pm, po) * p.s_mul;
+        float rmax = pms[0];
+#pragma unroll
+        for (int q = 1; q < kTcSplit; ++q) rmax = fmaxf(rmax, pms[q]);
+        const float mx = rmax * p.s_mul;
         const bool up = mx > m_ref + kTcRescale;
         const float corr = up ? ex2(m_ref - mx) : 1.f;   // 0 while nothing was accumulated
         if (up) {
@@ -606,7 +610,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           if (!(ok = tc_wait_warp(&pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1, abort, 19, u))) break;
           tc_fence_after();
 #pragma unroll 1
-          for (int c = 0; c < 2; ++c) {
+          for (int c = 0; c < kCW / 32; ++c) {
             float o[32];
             tc_ld32(t_row + c_o + c * 32, o);
 #pragma unroll
@@ -617,16 +621,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (!spec || up) lt = make_p(m_ref == -INFINITY ? 0.f : m_ref);
         l += lt;
         // V rows past the visible tokens (cache bytes beyond the context, or stale rows
-        // of blocks not loaded) are zeroed, this half of each, so that 0-weighted rows
+        // of blocks not loaded) are zeroed, this slice of each, so that 0-weighted rows
         // cannot bring a NaN into O
         const int rem = x.nvis - j * kTcTok;
         if (rem < kTcTok) {
           if (!(ok = tc_wait_warp(&v_full[b], (g >> 1) & 1, abort, 21, u))) break;
           if (row >= rem) {
-            uint8_t* vrow = sm + TcSmem::kV + b * TcSmem::kTile + hf * (kTcTok * 128) + (row >> 3) * 1024 +
-                            (row & 7) * 128;
+            uint8_t* vt = sm + TcSmem::kV + b * TcSmem::kTile;
 #pragma unroll
-            for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(vrow + c * 16) = make_uint4(0, 0, 0, 0);
+            for (int c = 0; c < kCW / 8; ++c)
+              *reinterpret_cast<uint4*>(vt + tc_swz(row, qs_ * (kCW / 8) + c)) = make_uint4(0, 0, 0, 0);
           }
         }
         fence_async_smem();
@@ -638,53 +642,62 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       // this unit's O
       if (!tc_wait_warp(&o_full[ob], (k >> 1) & 1, abort, 22, u)) break;
       tc_fence_after();
-      float o[64];
+      float o[kCW];
       {
-        uint32_t r[64];
-        tc_ld32_async(t_row + c_o, r);
-        tc_ld32_async(t_row + c_o + 32, r + 32);
+        uint32_t r[kCW];
+#pragma unroll
+        for (int c = 0; c < kCW / 32; ++c) tc_ld32_async(t_row + c_o + c * 32, r + c * 32);
         tc_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 64; ++c) o[c] = __uint_as_float(pin_after_wait(r[c]));
+        for (int c = 0; c < kCW; ++c) o[c] = __uint_as_float(pin_after_wait(r[c]));
       }
-      float lo;
-      if (!exchange(c_o, 256 + ob * 128 + (hf ^ 1) * 64, l, u, &lo)) break;
+      publish(c_o, l);
+      float ls[kTcSplit];
+      if (!gather(256 + ob * 128, l, u, ls)) break;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&o_empty[ob]);
-      const float lsum = hf == 0 ? l + lo : lo + l;   // same order in both halves
+      float lsum = ls[0];   // slice order: the same sum in every warp of the group
+#pragma unroll
+      for (int q = 1; q < kTcSplit; ++q) lsum += ls[q];
       const int P = has_q ? (qpos + 1 + p.chunk - 1) / p.chunk : 0;
       const bool wr = has_q && x.part < P;
       const bool fin = wr && P == 1;
-      if (fin) {   // this half of the row, rounded, staged in P buffer 0 (every P V has completed)
+      if (fin) {   // this slice of the row, rounded, staged in P buffer 0 (every P V has completed)
         const float inv = 1.f / lsum;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < kCW / 8; ++i) {
           float dummy = 0.f;
           uint32_t w[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) w[e] = pack2_sum<QD>(o[i * 8 + 2 * e] * inv, o[i * 8 + 2 * e + 1] * inv, dummy);
-          *reinterpret_cast<uint4*>(sm + TcSmem::kP + tc_swz(row, hf * 8 + i)) = make_uint4(w[0], w[1], w[2], w[3]);
+          *reinterpret_cast<uint4*>(sm + TcSmem::kP + tc_swz(row, qs_ * (kCW / 8) + i)) =
+              make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
       __syncwarp();
-      // coalesced: each store instruction writes 4 rows x 128 contiguous bytes
+      {   // coalesced: each store instruction writes (32 / kLPR) rows x kCW * 2 contiguous bytes
+        constexpr int kLPR = kCW / 8;               // lanes per row (16 bytes each)
+        constexpr int kRPI = 32 / kLPR;             // rows per instruction
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int rr = rw * 32 + i * 4 + (lane >> 3), c = lane & 7;
-        const int rqi = x.t * QPT + rr / G;
-        if (x.part == 0 && rqi < x.Q && x.base + rqi + 1 <= p.chunk) {   // that row's whole context is here
-          QT* orow = static_cast<QT*>(p.out) + (size_t(x.row0 + rqi) * Hq + x.hk * G + rr % G) * kTcD + hf * 64;
-          *reinterpret_cast<uint4*>(orow + c * 8) = *reinterpret_cast<const uint4*>(sm + TcSmem::kP + tc_swz(rr, hf * 8 + c));
+        for (int i = 0; i < 32 / kRPI; ++i) {
+          const int rr = rw * 32 + i * kRPI + lane / kLPR, c = lane % kLPR;
+          const int rqi = x.t * QPT + rr / G;
+          if (x.part == 0 && rqi < x.Q && x.base + rqi + 1 <= p.chunk) {   // that row's whole context is here
+            QT* orow =
+                static_cast<QT*>(p.out) + (size_t(x.row0 + rqi) * Hq + x.hk * G + rr % G) * kTcD + qs_ * kCW;
+            *reinterpret_cast<uint4*>(orow + c * 8) =
+                *reinterpret_cast<const uint4*>(sm + TcSmem::kP + tc_swz(rr, qs_ * kLPR + c));
+          }
         }
       }
       __syncwarp();
-      if (wr && !fin) {   // this chunk's partial: unnormalised half row, (max, sum) once
+      if (wr && !fin) {   // this chunk's partial: unnormalised row slice, (max, sum) once
         const size_t slot = (size_t(tok) * Hq + head) * p.max_parts + x.part;
-        float4* acc = reinterpret_cast<float4*>(p.part_acc + slot * kTcD + hf * 64);
+        float4* acc = reinterpret_cast<float4*>(p.part_acc + slot * kTcD + qs_ * kCW);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) acc[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
-        if (hf == 0) {
+        for (int i = 0; i < kCW / 4; ++i) acc[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+        if (qs_ == 0) {
           p.part_ml[slot * 2] = m_ref;
           p.part_ml[slot * 2 + 1] = lsum;
         }
