@@ -271,6 +271,17 @@ pa_status pa_prefill(const void* q, const void* k, const void* v, int32_t dtype,
                      void* stream);
 
 /*
+ * pa_selftest_wait_timeout -- failure-detection self-test (the pages have no counterpart:
+ * it exercises this library's own guard). Enqueues one CTA on `stream` whose thread
+ * waits, through the same bounded mbarrier wait every kernel here uses, on a barrier that
+ * nothing ever arrives at. After limit_us microseconds the wait gives up, records
+ * PA_DEV_WAIT_TIMEOUT with info = {0x7E57, elapsed microseconds, 0} and the kernel
+ * returns: nothing faults, nothing hangs, the context stays usable. Read the result with
+ * pa_last_device_error. limit_us in 1 .. 2000000, else PA_ERR_ARG.
+ */
+pa_status pa_selftest_wait_timeout(uint32_t limit_us, void* stream);
+
+/*
  * pa_last_device_error -- synchronise `stream`, then read and clear the device error
  * word of the current device. *code receives a PA_DEV_* value; info (may be NULL)
  * receives 3 int32 details. Returns PA_ERR_DEVICE_CHECK when *code != 0.

@@ -105,6 +105,7 @@ _SIGNATURES = {
     "pa_extend": (_I32, [_P, _I32, _I32, _I32, _P, _I32, _PDESC, _P, _I32, _P, _I32, ctypes.c_float, _P, _P,
                          ctypes.c_size_t, _P]),
     "pa_extend_workspace_size": (ctypes.c_size_t, [_I32, _I32, _I32, _I32, _I32]),
+    "pa_selftest_wait_timeout": (_I32, [ctypes.c_uint32, _P]),
     "pa_prefill": (_I32, [_P, _P, _P, _I32, _I32, _I32, _P, _I32, _PDESC, _P, _I32, _P, _I32, ctypes.c_float, _P,
                           _P, ctypes.c_size_t, _P]),
     "pa_version": (ctypes.c_char_p, []),
@@ -257,6 +258,12 @@ def prefill(q, k, v, cache: KVCache, query_start, block_tables, context_lens, ma
                           int(max_context_len), float(scale), _ptr(out), _ptr(workspace),
                           workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "pa_prefill")
+
+
+def selftest_wait_timeout(limit_us: int, stream=None) -> None:
+    """Enqueue the bounded-wait self-test (a wait on a barrier nothing arrives at); read the
+    recorded timeout with last_device_error()."""
+    _check(lib().pa_selftest_wait_timeout(int(limit_us), _stream(stream)), "pa_selftest_wait_timeout")
 
 
 NO_ALLOC_WORKSPACE_BYTES = 16 << 20

@@ -115,6 +115,23 @@ inline bool aligned16_(const void* p) { return (reinterpret_cast<uintptr_t>(p) &
 
 }  // namespace pa
 
+namespace pa {
+
+// One thread waits on an mbarrier that nothing arrives at, through the bounded wait every
+// kernel of the library uses; when the limit runs out it records the timeout in the device
+// error word and returns, leaving the context usable.
+__global__ void __launch_bounds__(32) selftest_wait_kernel(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  fence_mbar_init();
+  const uint64_t t0 = global_timer_ns();
+  if (!mbar_wait_bounded(&bar, 0, limit_ns))
+    record_error(PA_DEV_WAIT_TIMEOUT, kSelftestKernelId, int((global_timer_ns() - t0) / 1000), 0);
+}
+
+}  // namespace pa
+
 extern "C" {
 
 pa_status pa_reshape_and_cache(const void* k, const void* v, int32_t in_dtype, int32_t num_tokens,
@@ -176,6 +193,12 @@ pa_status pa_block_table_update(const int32_t* updates, int32_t num_updates, int
   if (!updates || !block_tables) return PA_ERR_ARG;
   pa::table_update_kernel<<<(num_updates + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(
       updates, num_updates, block_tables, num_seqs, max_blocks_per_seq);
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status pa_selftest_wait_timeout(uint32_t limit_us, void* stream) {
+  if (limit_us == 0 || limit_us > 2000000) return PA_ERR_ARG;
+  pa::selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(uint64_t(limit_us) * 1000ull);
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 

@@ -13,6 +13,7 @@ namespace pa {
 
 constexpr int kPartitionTokens = 512;      // split-K partition length of the v2-style decode
 constexpr unsigned kFull = 0xffffffffu;
+constexpr int kSelftestKernelId = 0x7E57;   // kernel id the wait self-test records
 
 // ---------------------------------------------------------------------------
 // sticky device error word: [code, info0, info1, info2]; the first error wins
