@@ -184,3 +184,55 @@ def test_short_runs_ignore_bytes_past_the_context():
     out = _run(w, eng, qs_dev, q, qs)
     assert pa.last_device_error()[0] == 0
     _check_rows(w, eng, q, qs, out, _sample_rows(qs, 4, 80, 92), "cooperative kernel tails")
+
+
+def _compact(eng, seqs, BS):
+    """The oracle's copy of the blocks of `seqs` (host codes) and block tables remapped to it."""
+    lens = list(eng.lens)
+    blocks = sorted({int(b) for s in seqs for b in eng.bt_host[s, :-(-lens[s] // BS)]})
+    idx = torch.tensor(blocks, dtype=torch.int64, device=DEV)
+    kc, vc = codes_np(eng.k_cache.index_select(0, idx)), codes_np(eng.v_cache.index_select(0, idx))
+    remap = {b: i for i, b in enumerate(blocks)}
+    bt = np.zeros(eng.bt_host.shape, np.int64)
+    for s in seqs:
+        nb = -(-lens[s] // BS)
+        bt[s, :nb] = [remap[int(b)] for b in eng.bt_host[s, :nb]]
+    return kc, vc, bt, lens
+
+
+def test_spec4_mix_full_size_sampled():
+    """The benchmarked speculative-verification shapes: 4 draft tokens per sequence over the
+    13B mixed-length contexts (256 sequences, 40/40 heads, bf16), on sampled rows."""
+    w = synthetic.make("llama13b_mix")
+    eng = make_engine(w, DEV)
+    fill_cache(w, eng)
+    for s, L in enumerate(w.context_lens):
+        eng.extend(s, L)
+    eng.upload_tables()
+    qlens = [min(4, L) for L in w.context_lens]
+    qs = np.concatenate([[0], np.cumsum(qlens)]).astype(np.int32)
+    q = synthetic.normal_values((int(qs[-1]), w.num_q_heads, w.head_dim), w.q_dtype, w.seed + 11).to(DEV)
+    out = _run(w, eng, torch.from_numpy(qs).to(DEV), q, qs)
+    assert pa.last_device_error()[0] == 0
+    lens = np.array(w.context_lens)
+    pick = []
+    for lo, hi in ((0, 200), (1000, 1100), (8000, 9000)):
+        idx = np.nonzero((lens >= lo) & (lens < hi))[0]
+        pick += idx[[0, -1]].tolist()
+    pick = sorted(set(pick + [int(np.argmax(lens)), w.num_seqs - 1]))
+    kc, vc, bt, L = _compact(eng, pick, w.block_size)
+    rows = [(int(qs[s]) + i, h) for s in pick for i in range(qlens[s]) for h in (0, 13, 27, 39)]
+    ref = oatt.paged_extend(codes_np(q), w.q_dtype, kc, vc, w.kv_dtype, 1.0, 1.0, bt, L, qs, w.scale, rows=rows)
+    idx = tuple(np.array(rows).T)
+    assert_close(out.double().cpu().numpy()[idx], ref[idx], w.kv_dtype, "spec4 mix full size")
+
+
+def test_long_context_many_chunks():
+    """A 256-query chunk at the end of a 20000-token context, GQA 4: few units, so the
+    context is cut into many chunks merged by log-sum-exp."""
+    lens, qlens = [20000], [256]
+    w, eng, qs_dev, q, qs = _setup(lens, qlens, 8, 2, 128, 16, "bf16", 97)
+    _nan_tails(w, eng)
+    out = _run(w, eng, qs_dev, q, qs)
+    assert pa.last_device_error()[0] == 0
+    _check_rows(w, eng, q, qs, out, _sample_rows(qs, 8, 60, 97), "20000-token context")

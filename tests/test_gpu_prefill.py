@@ -113,3 +113,9 @@ def test_prefill_unsupported_shapes_are_refused():
     with pytest.raises(RuntimeError):
         pa.prefill(q, q, q, eng.cache, torch.tensor([0, 10], dtype=torch.int32, device=DEV), eng.bt_dev,
                    eng.lens_dev, eng.max_context_len, w.scale, torch.empty_like(q), ws)
+
+
+def test_prefill_8x2k_full_size():
+    """The benchmarked prefill shapes (8 prompts x 2048 tokens, 32/32 heads, bf16, 16-token
+    blocks): every cache slot bit-exact, sampled output rows against the oracle."""
+    _prefill_case([2048] * 8, 32, 32, 16, "bf16", 4371, 120)
