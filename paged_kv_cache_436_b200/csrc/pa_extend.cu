@@ -222,28 +222,15 @@ __device__ __forceinline__ ExtUnit ext_make_unit(const ExtendParams& p, int u, i
   x.nblk = 0;
   x.bid = 0;
   if (u >= total) return x;
-  const int pair = u / p.num_kv_heads;
+  const int pair = u / p.num_kv_heads;   // the plan kernel's record of (sequence, tile, partition)
   x.hk = u - pair * p.num_kv_heads;
-  int lo = 0, hi = p.num_seqs;
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (p.plan[mid] <= pair) lo = mid; else hi = mid;
-  }
-  x.s = lo;
-  ext_seq(p, lo, x.Q, x.base);
-  x.row0 = p.query_start[lo];
-  int k = pair - p.plan[lo];
-  const int tiles = (x.Q + qpt - 1) / qpt;
-  x.t = 0;
-  for (int t = 0; t < tiles; ++t) {
-    const int P = ext_tile_parts(x.base, x.Q, qpt, t, p.chunk);
-    if (k < P) {
-      x.t = t;
-      break;
-    }
-    k -= P;
-  }
-  x.part = k;
+  const int4 a = __ldg(p.units + 2 * size_t(pair)), b = __ldg(p.units + 2 * size_t(pair) + 1);
+  x.s = a.x;
+  x.t = a.y;
+  x.part = a.z;
+  x.row0 = a.w;
+  x.Q = b.x;
+  x.base = b.y;
   const int last = x.base + min((x.t + 1) * qpt, x.Q) - 1;     // last position the tile sees
   x.last = last;
   x.b0 = x.part * BPP;
@@ -777,10 +764,12 @@ struct ExtWs {
   size_t plan, ml, acc, units, total;
 };
 
-// Pair records of the 128-row path: it runs only when 2 T G >= 128 S, so its tiles are at
-// most T G / 128 + 1 + S <= 3 T Hq / 128 + 1, each with at most max_parts chunks.
+// Unit records: a sequence with Q_s > 0 queries has at most Q_s row tiles (a tile holds at
+// least one query), so there are at most T tiles (tile groups), each with at most
+// max_parts chunks.
 inline size_t ext_units_bound(int T, int Hq, int max_parts) {
-  return (3 * size_t(T) * Hq / 128 + 2) * size_t(max_parts);
+  (void)Hq;
+  return size_t(T > 0 ? T : 1) * size_t(max_parts);
 }
 
 inline ExtWs ext_ws(int S, int T, int Hq, int D, int max_parts) {
@@ -914,7 +903,7 @@ static pa_status extend_impl(const void* q, int32_t q_dtype, int32_t num_seqs, i
   p.plan = reinterpret_cast<int32_t*>(w + ws.plan);
   p.part_ml = reinterpret_cast<float*>(w + ws.ml);
   p.part_acc = reinterpret_cast<float*>(w + ws.acc);
-  p.units = tc ? reinterpret_cast<int4*>(w + ws.units) : nullptr;
+  p.units = reinterpret_cast<int4*>(w + ws.units);
   p.units_cap = (long long)ext_units_bound(num_tokens, num_q_heads, max_parts);
   p.fresh = fresh ? 1 : 0;
   p.num_seqs = num_seqs;
