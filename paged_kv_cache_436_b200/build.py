@@ -22,7 +22,7 @@ LIB = os.path.join(LIB_DIR, "libpa.so")
 
 SOURCES = [os.path.join(CSRC, "pa_lib.cu"), os.path.join(CSRC, "pa_pool.cpp"), os.path.join(CSRC, "pa_engine.cpp"),
            os.path.join(CSRC, "pa_prefix.cpp")]
-DEPENDS = SOURCES + [os.path.join(CSRC, f) for f in ("pa_decode.cu", "pa_cache.cu", "pa_extend.cu", "pa_extend_tc.cu", "pa_device.cuh")] + \
+DEPENDS = SOURCES + [os.path.join(CSRC, f) for f in ("pa_decode.cu", "pa_cache.cu", "pa_extend.cu", "pa_extend_tc.cu", "pa_device.cuh", "pa_tmap.cuh")] + \
     [os.path.join(INCLUDE, "pa.h")]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O3", "-shared",

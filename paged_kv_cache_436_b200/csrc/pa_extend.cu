@@ -24,6 +24,7 @@
 
 #include "pa.h"
 #include "pa_device.cuh"
+#include "pa_tmap.cuh"
 
 namespace pa {
 
@@ -194,12 +195,12 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi, float& lo_r, float
 template <int D, int BS>
 struct ExtCfg {
   static constexpr int kRowBytes = D * 2;
-  static constexpr int kRowPad = kRowBytes + 16;        // padded row: conflict-free ldmatrix
-  static constexpr int kStage = 2 * BS * kRowPad;       // K rows then V rows
+  static constexpr int kHalf = BS * 128;                // one 64-dim half of a block: BS rows of 128 B
+  static constexpr int kStage = 2 * BS * kRowBytes;     // K block then V block, each D / 64 halves
   static constexpr int kStages = 2;
   static constexpr int kWarps = 4;
   static constexpr int kThreads = kWarps * 32;
-  static constexpr int kSmem = kWarps * kStages * kStage + kWarps * kStages * 8;
+  static constexpr int kSmem = kWarps * kStages * kStage + kWarps * kStages * 8 + 1024;   // + alignment
   static constexpr int kBlocksPerPartition = kPartitionTokens / BS;
   static_assert(BS % 16 == 0, "blocks hold whole 16-token slices");
   static_assert(kBlocksPerPartition <= 32, "block ids of a partition fit the lanes");
@@ -247,14 +248,23 @@ __device__ __forceinline__ ExtUnit ext_make_unit(const ExtendParams& p, int u, i
   return x;
 }
 
+// Byte offset of the 16-byte chunk holding dims [8 c, 8 c + 8) of row r in a block tile
+// laid down by the 128B-swizzled 2-D TMA boxes (one per 64-dim half).
+template <int BS>
+__device__ __forceinline__ uint32_t ext_swz(int r, int c) {
+  return uint32_t((c >> 3) * (BS * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+}
+
 template <int QD, int D, int BS, int G>
-__global__ void __launch_bounds__(ExtCfg<D, BS>::kThreads) extend_kernel(const ExtendParams p) {
+__global__ void __launch_bounds__(ExtCfg<D, BS>::kThreads)
+    extend_kernel(const ExtendParams p, const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv) {
   using C = ExtCfg<D, BS>;
   using QT = typename Q<QD>::T;
   constexpr int NS = C::kStages, NW = C::kWarps, KK = D / 16, NT = D / 8;
   constexpr int QPT = kTileRows / G;                      // queries per tile
 
-  extern __shared__ __align__(128) uint8_t smem[];
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + NW * NS * C::kStage);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint8_t* ring = smem + warp * NS * C::kStage;
@@ -263,20 +273,12 @@ __global__ void __launch_bounds__(ExtCfg<D, BS>::kThreads) extend_kernel(const E
     for (int i = 0; i < NS; ++i) mbar_init(&bar[i], 1);
     fence_mbar_init();
   }
-  // rows past a tile's last visible token are never copied: they keep zeros or an
-  // earlier visible row, so a 0-weighted row cannot bring cache bytes beyond the
-  // context (possibly NaN) into P V
-  for (int i = lane; i < NS * C::kStage / 16; i += 32) reinterpret_cast<uint4*>(ring)[i] = make_uint4(0, 0, 0, 0);
-  fence_async_smem();
   __syncwarp();
   grid_dependency_launch_dependents();
   grid_dependency_wait();
 
   const int Hq = p.num_q_heads, Hkv = p.num_kv_heads;
   const int total = p.plan[p.num_seqs] * Hkv;
-  const uint64_t pol = l2_policy_evict_first();
-  const size_t head_stride = size_t(BS) * C::kRowBytes;           // one (block, kv head) chunk
-  const size_t block_stride = size_t(Hkv) * head_stride;
   uint32_t consumed = 0;
 
   // rows of this lane: r0 = lane / 4 and r0 + 8 of the tile
@@ -311,19 +313,20 @@ __global__ void __launch_bounds__(ExtCfg<D, BS>::kThreads) extend_kernel(const E
                                 : 0u;
       }
 
-    auto issue = [&](int i, uint32_t g) {
+    auto issue = [&](int i, uint32_t g) {   // cache block i of the unit: one 2-D box per (K / V, half)
       const int bid = __shfl_sync(kFull, x.bid, i);
       const int st = g % NS;
       uint8_t* dst = ring + st * C::kStage;
-      const int nrows = min(BS, x.last + 1 - (x.b0 + i) * BS);
-      if (lane == 0) mbar_arrive_expect_tx(&bar[st], 2 * nrows * C::kRowBytes);
-      __syncwarp();
-      const size_t off = size_t(bid) * block_stride + size_t(x.hk) * head_stride;
-      for (int j = lane; j < 2 * nrows; j += 32) {
-        const int which = j / nrows, row = j - which * nrows;
-        const uint8_t* src = (which ? p.v_cache : p.k_cache) + off + size_t(row) * C::kRowBytes;
-        bulk_g2s(dst + which * BS * C::kRowPad + row * C::kRowPad, src, C::kRowBytes, &bar[st], pol);
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&bar[st], C::kStage);
+        const int y = (bid * Hkv + x.hk) * BS;
+#pragma unroll
+        for (int h = 0; h < D / 64; ++h) {
+          tma_load_2d(dst + h * C::kHalf, &tk, h * 64, y, &bar[st]);
+          tma_load_2d(dst + BS * C::kRowBytes + h * C::kHalf, &tv, h * 64, y, &bar[st]);
+        }
       }
+      __syncwarp();
     };
     for (int i = 0; i < NS && i < x.nblk; ++i) issue(i, consumed + i);
 
@@ -341,9 +344,18 @@ __global__ void __launch_bounds__(ExtCfg<D, BS>::kThreads) extend_kernel(const E
         failed = true;
         break;
       }
-      const uint8_t* Ks = ring + st * C::kStage;
-      const uint8_t* Vs = Ks + BS * C::kRowPad;
+      uint8_t* Ks = ring + st * C::kStage;
+      uint8_t* Vs = Ks + BS * C::kRowBytes;
       const int tok0 = (x.b0 + i) * BS;
+      // V rows past the tile's last token (cache bytes beyond the context, possibly NaN)
+      // are zeroed: their P is 0, but 0 * NaN would still reach O
+      if (tok0 + BS - 1 > x.last) {
+        const int keep = x.last + 1 - tok0;
+        for (int j = keep * (D / 8) + lane; j < BS * (D / 8); j += 32)
+          *reinterpret_cast<uint4*>(Vs + ext_swz<BS>(j / (D / 8), j % (D / 8))) = make_uint4(0, 0, 0, 0);
+        fence_async_smem();
+        __syncwarp();
+      }
 #pragma unroll
       for (int sb = 0; sb < BS / 16; ++sb) {
         // S = Q K^T for 16 tokens (two n-tiles of 8)
@@ -352,7 +364,7 @@ __global__ void __launch_bounds__(ExtCfg<D, BS>::kThreads) extend_kernel(const E
         for (int kk = 0; kk < KK; ++kk) {
           uint32_t b[4];
           const int trow = sb * 16 + (lane >> 4) * 8 + (lane & 7);
-          ldsm_x4(b, Ks + trow * C::kRowPad + (kk * 16 + ((lane >> 3) & 1) * 8) * 2);
+          ldsm_x4(b, Ks + ext_swz<BS>(trow, kk * 2 + ((lane >> 3) & 1)));
           mma16816<QD>(sc[0], qa[kk], b[0], b[1]);
           mma16816<QD>(sc[1], qa[kk], b[2], b[3]);
         }
@@ -405,7 +417,7 @@ __global__ void __launch_bounds__(ExtCfg<D, BS>::kThreads) extend_kernel(const E
         for (int np = 0; np < NT / 2; ++np) {
           uint32_t b[4];
           const int trow = sb * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
-          ldsm_x4_trans(b, Vs + trow * C::kRowPad + (np * 16 + (lane >> 4) * 8) * 2);
+          ldsm_x4_trans(b, Vs + ext_swz<BS>(trow, np * 2 + (lane >> 4)));
           mma16816<QD>(o[2 * np], pa, b[0], b[1]);
           mma16816<QD>(o[2 * np + 1], pa, b[2], b[3]);
         }
@@ -783,15 +795,18 @@ inline ExtWs ext_ws(int S, int T, int Hq, int D, int max_parts) {
 }
 
 using ExtKernel = void (*)(const ExtendParams);
+using ExtTmapKernel = void (*)(const ExtendParams, const CUtensorMap, const CUtensorMap);
 struct ExtLaunch {
-  ExtKernel fn = nullptr;
+  ExtKernel fn = nullptr;          // the cooperative kernel
+  ExtTmapKernel tfn = nullptr;     // the warp kernel (reads the cache through tensor maps)
   int smem = 0, threads = 0;
+  const void* key() const { return tfn ? reinterpret_cast<const void*>(tfn) : reinterpret_cast<const void*>(fn); }
 };
 
 template <int QD, int D, int BS, int G>
 ExtLaunch ext_get(bool coop) {
-  if (coop) return ExtLaunch{extend_coop_kernel<QD, D, BS, G>, CoopCfg<D, BS>::kSmem, CoopCfg<D, BS>::kThreads};
-  return ExtLaunch{extend_kernel<QD, D, BS, G>, ExtCfg<D, BS>::kSmem, ExtCfg<D, BS>::kThreads};
+  if (coop) return ExtLaunch{extend_coop_kernel<QD, D, BS, G>, nullptr, CoopCfg<D, BS>::kSmem, CoopCfg<D, BS>::kThreads};
+  return ExtLaunch{nullptr, extend_kernel<QD, D, BS, G>, ExtCfg<D, BS>::kSmem, ExtCfg<D, BS>::kThreads};
 }
 template <int QD, int D, int BS>
 ExtLaunch ext_pick_g(int G, bool coop) {
@@ -888,7 +903,7 @@ static pa_status extend_impl(const void* q, int32_t q_dtype, int32_t num_seqs, i
   ExtLaunch k;
   if (!tc) {
     k = q_dtype == PA_BF16 ? ext_pick_d<PA_BF16>(D, BS, G, coop) : ext_pick_d<PA_F16>(D, BS, G, coop);
-    if (!k.fn) return PA_ERR_ARG;
+    if (!k.key()) return PA_ERR_ARG;
   }
 
   ExtendParams p;
@@ -938,7 +953,7 @@ static pa_status extend_impl(const void* q, int32_t q_dtype, int32_t num_seqs, i
   } else {
     int cap = 0;
     Launch as_launch;
-    as_launch.fn = reinterpret_cast<KernelFn>(k.fn);
+    as_launch.fn = reinterpret_cast<KernelFn>(const_cast<void*>(k.key()));
     as_launch.smem = k.smem;
     as_launch.threads = k.threads;
     if (occupancy(as_launch, &cap) != cudaSuccess) return PA_ERR_CUDA;
@@ -954,6 +969,24 @@ static pa_status extend_impl(const void* q, int32_t q_dtype, int32_t num_seqs, i
   if (tc) {
     st = extend_tc_launch(p, c, q_dtype, G, grid, s, k_new, v_new);
     if (st != PA_OK) return st;
+  } else if (k.tfn) {
+    TmapEncodeFn enc = tmap_encoder();
+    CUtensorMap tk, tv;
+    const long long rows = (long long)c->num_blocks * c->num_kv_heads * BS;
+    if (!enc || !cache_tmap(enc, &tk, c->k_cache, q_dtype, rows, BS, D) ||
+        !cache_tmap(enc, &tv, c->v_cache, q_dtype, rows, BS, D))
+      return PA_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(k.threads);
+    cfg.dynamicSmemBytes = k.smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, k.tfn, p, tk, tv) != cudaSuccess) return PA_ERR_CUDA;
   } else if (ext_launch(k.fn, grid, k.threads, k.smem, s, p) != cudaSuccess) {
     return PA_ERR_CUDA;
   }

@@ -34,10 +34,6 @@
 //     writes (max, sum, unnormalised row) for the log-sum-exp merge kernel.
 // Every wait is bounded; on a timeout the kernel records it, every role stops, the MMA
 // and load issuers drain what they issued, and the TMEM is freed.
-#include <cuda.h>
-
-#include <mutex>
-
 namespace pa {
 
 constexpr int kTcRows = 128;            // query rows per unit (TMEM lanes)
@@ -220,15 +216,6 @@ __device__ __forceinline__ uint32_t exp2_pack(float2 a, float2& sum) {
   }
   sum = add2(sum, r);
   return w;
-}
-
-// 2-D tiled TMA load (box given by the tensor map) signalling `bar` with its bytes.
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_addr(dst)),
-      "l"(map), "r"(x), "r"(y), "r"(smem_addr(bar))
-      : "memory");
 }
 
 // 3-D tiled TMA load.
@@ -727,34 +714,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 // --------------------------------------------------------------------------
 // host side: tensor maps over the cache viewed as [blocks * kv heads * block_size][head_dim]
 // --------------------------------------------------------------------------
-typedef CUresult (*TmapEncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-TmapEncodeFn tmap_encoder() {
-  static std::once_flag once;
-  static TmapEncodeFn fn = nullptr;
-  std::call_once(once, [] {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<TmapEncodeFn>(f);
-  });
-  return fn;
-}
-
-bool cache_tmap(TmapEncodeFn enc, CUtensorMap* m, const void* base, int qd, long long rows, int BS) {
-  const cuuint64_t dims[2] = {cuuint64_t(kTcD), cuuint64_t(rows)};
-  const cuuint64_t strides[1] = {cuuint64_t(kTcD) * 2};
-  const cuuint32_t box[2] = {64, cuuint32_t(BS)};
-  const cuuint32_t es[2] = {1, 1};
-  return enc(m, qd == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
-             const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 // q viewed as [tokens][q heads][head_dim]; box = 64 dims x G heads x 128 / G queries,
 // i.e. one 64-column half of a unit's 128 rows in (query, head) order.
 bool q_tmap(TmapEncodeFn enc, CUtensorMap* m, const void* q, int qd, int num_tokens, int Hq, int G) {
@@ -820,8 +779,8 @@ pa_status extend_tc_launch(const ExtendParams& p, const pa_cache_desc* c, int qd
   if (!fn || !enc) return PA_ERR_ARG;
   CUtensorMap tk, tv, tq;
   const long long rows = (long long)c->num_blocks * c->num_kv_heads * c->block_size;
-  if (!cache_tmap(enc, &tk, c->k_cache, qd, rows, c->block_size) ||
-      !cache_tmap(enc, &tv, c->v_cache, qd, rows, c->block_size) ||
+  if (!cache_tmap(enc, &tk, c->k_cache, qd, rows, c->block_size, kTcD) ||
+      !cache_tmap(enc, &tv, c->v_cache, qd, rows, c->block_size, kTcD) ||
       !q_tmap(enc, &tq, p.q, qd, p.num_tokens, p.num_q_heads, G))
     return PA_ERR_ARG;
   CUtensorMap tkn = tk, tvn = tv;   // used only for whole prompts
