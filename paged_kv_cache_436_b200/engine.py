@@ -188,6 +188,13 @@ class HostPipeline:
         self.d2h = torch.cuda.Stream(dev)
         self.free_in = [None, None]     # step that last read buffer b has finished
         self.free_out = [None, None]    # the output copy that last read dout[b] has finished
+        # the previous step's attention kernel has started: its small metadata copy is done,
+        # so the next inputs' large copy cannot delay it on the copy engine
+        self.started = None
+        self._ev = [(torch.cuda.Event(), torch.cuda.Event()) for _ in range(2)]
+        for a, b in self._ev:            # torch creates the CUDA events at their first record
+            a.record(self.compute)
+            b.record(self.compute)
         self.n = 0
 
     def submit(self, hq, hk, hv, hout):
@@ -196,6 +203,8 @@ class HostPipeline:
         with torch.cuda.stream(self.h2d):
             if self.free_in[b] is not None:
                 self.h2d.wait_event(self.free_in[b])
+            if self.started is not None:
+                self.h2d.wait_event(self.started)
             self.dq[b].copy_(hq, non_blocking=True)
             self.dk[b].copy_(hk, non_blocking=True)
             self.dv[b].copy_(hv, non_blocking=True)
@@ -204,7 +213,9 @@ class HostPipeline:
         self.compute.wait_event(landed)
         if self.free_out[b] is not None:
             self.compute.wait_event(self.free_out[b])
-        self.eng.step(self.dq[b], self.dk[b], self.dv[b], self.dout[b], stream=self.compute)
+        ev = self._ev[b]
+        self.eng.step(self.dq[b], self.dk[b], self.dv[b], self.dout[b], stream=self.compute, events=ev)
+        self.started = ev[0]
         done = torch.cuda.Event()
         done.record(self.compute)
         self.free_in[b] = done
