@@ -151,3 +151,56 @@ def run_decode_step(w, sample_heads=None, sample_seqs=None, growth=0, device="cu
     got = out.double().cpu().numpy()
     hs = tuple(np.array(heads).T)
     return assert_close(got[hs], ref[hs], w.kv_dtype, w.name), eng
+
+
+def run_prefill_case(lens, Hq, Hkv, BS, dt, seed, nrows, device="cuda"):
+    """pa_prefill of whole prompts into a NaN-filled cache: every prompt slot bit-exact
+    against the oracle's reshape_and_cache, sampled outputs against its paged_extend."""
+    D = 128
+    w = synthetic.custom(len(lens), Hq, Hkv, D, BS, dt, dt, lens, seed)
+    eng = make_engine(w, device)
+    eng.k_cache.fill_(float("nan"))
+    eng.v_cache.fill_(float("nan"))
+    k0, v0 = codes_np(eng.k_cache), codes_np(eng.v_cache)
+    for s, L in enumerate(lens):
+        eng.extend(s, L)
+    eng.upload_tables()
+    qs = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    T = int(qs[-1])
+    q = synthetic.normal_values((T, Hq, D), dt, seed + 7).to(device)
+    k = synthetic.normal_values((T, Hkv, D), dt, seed + 8).to(device)
+    v = synthetic.normal_values((T, Hkv, D), dt, seed + 9).to(device)
+    out = torch.full_like(q, float("nan"))
+    ws = torch.empty(pa.extend_workspace_size(w.num_seqs, T, Hq, D, eng.max_context_len), dtype=torch.uint8,
+                     device=device)
+    pa.prefill(q, k, v, eng.cache, torch.from_numpy(qs).to(device), eng.bt_dev, eng.lens_dev, eng.max_context_len,
+               w.scale, out, ws)
+    torch.cuda.synchronize()
+    assert pa.last_device_error()[0] == 0
+
+    # the oracle's cache: the same prompt tokens written through its reshape_and_cache
+    bt = eng.bt_host.astype(np.int64)
+    slots = np.concatenate([bt[s, np.arange(L) // BS] * BS + np.arange(L) % BS for s, L in enumerate(lens)])
+    kc, vc = oops.reshape_and_cache(codes_np(k), codes_np(v), dt, slots, k0, v0, dt)
+    gk, gv = codes_np(eng.k_cache), codes_np(eng.v_cache)
+    blk, off = slots // BS, slots % BS
+    assert np.array_equal(gk[blk, :, off, :], kc[blk, :, off, :]), "k slots"
+    assert np.array_equal(gv[blk, :, off, :], vc[blk, :, off, :]), "v slots"
+
+    rng = np.random.default_rng(seed)
+    rows = {(int(t), int(h)) for t, h in zip(rng.integers(0, T, nrows), rng.integers(0, Hq, nrows))}
+    for s in range(len(lens)):
+        for t in (int(qs[s]), int(qs[s + 1]) - 1):
+            rows.update((t, h) for h in range(Hq))
+    rows = sorted(rows)
+    ref = oatt.paged_extend(codes_np(q), dt, kc, vc, dt, 1.0, 1.0, bt, list(lens), qs, w.scale, rows=rows)
+    idx = tuple(np.array(rows).T)
+    got = out.double().cpu().numpy()
+    assert np.isfinite(got[idx]).all()
+    err = assert_close(got[idx], ref[idx], dt, f"prefill {dt} BS{BS} G{Hq // Hkv}")
+    # the first token of every prompt sees itself only: its output is its V row exactly
+    for s in range(len(lens)):
+        t = int(qs[s])
+        for h in range(Hq):
+            assert torch.equal(out[t, h], v[t, h // (Hq // Hkv)])
+    return err

@@ -11,62 +11,10 @@ import torch
 
 import paged_kv_cache_436_b200 as pa
 import synthetic
-from oracle import attention as oatt
-from oracle import cache_ops as ocache
-from tests.gpu_cases import assert_close, codes_np, make_engine
+from tests.gpu_cases import make_engine, run_prefill_case
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
-
-
-def _prefill_case(lens, Hq, Hkv, BS, dt, seed, nrows):
-    D = 128
-    w = synthetic.custom(len(lens), Hq, Hkv, D, BS, dt, dt, lens, seed)
-    eng = make_engine(w, DEV)
-    eng.k_cache.fill_(float("nan"))
-    eng.v_cache.fill_(float("nan"))
-    k0, v0 = codes_np(eng.k_cache), codes_np(eng.v_cache)
-    for s, L in enumerate(lens):
-        eng.extend(s, L)
-    eng.upload_tables()
-    qs = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
-    T = int(qs[-1])
-    q = synthetic.normal_values((T, Hq, D), dt, seed + 7).to(DEV)
-    k = synthetic.normal_values((T, Hkv, D), dt, seed + 8).to(DEV)
-    v = synthetic.normal_values((T, Hkv, D), dt, seed + 9).to(DEV)
-    out = torch.full_like(q, float("nan"))
-    ws = torch.empty(pa.extend_workspace_size(w.num_seqs, T, Hq, D, eng.max_context_len), dtype=torch.uint8,
-                     device=DEV)
-    pa.prefill(q, k, v, eng.cache, torch.from_numpy(qs).to(DEV), eng.bt_dev, eng.lens_dev, eng.max_context_len,
-               w.scale, out, ws)
-    torch.cuda.synchronize()
-    assert pa.last_device_error()[0] == 0
-
-    # the oracle's cache: the same prompt tokens written through its reshape_and_cache
-    bt = eng.bt_host.astype(np.int64)
-    slots = np.concatenate([bt[s, np.arange(L) // BS] * BS + np.arange(L) % BS for s, L in enumerate(lens)])
-    kc, vc = ocache.reshape_and_cache(codes_np(k), codes_np(v), dt, slots, k0, v0, dt)
-    gk, gv = codes_np(eng.k_cache), codes_np(eng.v_cache)
-    blk, off = slots // BS, slots % BS
-    assert np.array_equal(gk[blk, :, off, :], kc[blk, :, off, :]), "k slots"
-    assert np.array_equal(gv[blk, :, off, :], vc[blk, :, off, :]), "v slots"
-
-    rng = np.random.default_rng(seed)
-    rows = {(int(t), int(h)) for t, h in zip(rng.integers(0, T, nrows), rng.integers(0, Hq, nrows))}
-    for s in range(len(lens)):
-        for t in (int(qs[s]), int(qs[s + 1]) - 1):
-            rows.update((t, h) for h in range(Hq))
-    rows = sorted(rows)
-    ref = oatt.paged_extend(codes_np(q), dt, kc, vc, dt, 1.0, 1.0, bt, list(lens), qs, w.scale, rows=rows)
-    idx = tuple(np.array(rows).T)
-    got = out.double().cpu().numpy()
-    assert np.isfinite(got[idx]).all()
-    assert_close(got[idx], ref[idx], dt, f"prefill {dt} BS{BS} G{Hq // Hkv}")
-    # the first token of every prompt sees itself only: its output is its V row exactly
-    for s in range(len(lens)):
-        t = int(qs[s])
-        for h in range(Hq):
-            assert torch.equal(out[t, h], v[t, h // (Hq // Hkv)])
 
 
 @pytest.mark.parametrize("dt,BS,G", [("bf16", 16, 1), ("f16", 32, 2), ("bf16", 32, 4), ("f16", 16, 8),
@@ -76,12 +24,12 @@ def test_prefill_matches_oracle(dt, BS, G):
     chunks) with few units, so contexts are split into chunks and merged."""
     lens = [1, 17, 130, 700, 1025, 257]
     seed = zlib.crc32(repr(("prefill", dt, BS, G)).encode()) % 10000
-    _prefill_case(lens, 2 * G, 2, BS, dt, seed, 160)
+    run_prefill_case(lens, 2 * G, 2, BS, dt, seed, 160)
 
 
 def test_prefill_whole_context_units():
     """Enough row tiles that every unit holds its rows' whole context (no merge)."""
-    _prefill_case([1200, 1100, 1000, 1200], 8, 8, 16, "bf16", 81, 200)
+    run_prefill_case([1200, 1100, 1000, 1200], 8, 8, 16, "bf16", 81, 200)
 
 
 def test_prefill_rejects_context_longer_than_prompt():
@@ -118,4 +66,4 @@ def test_prefill_unsupported_shapes_are_refused():
 def test_prefill_8x2k_full_size():
     """The benchmarked prefill shapes (8 prompts x 2048 tokens, 32/32 heads, bf16, 16-token
     blocks): every cache slot bit-exact, sampled output rows against the oracle."""
-    _prefill_case([2048] * 8, 32, 32, 16, "bf16", 4371, 120)
+    run_prefill_case([2048] * 8, 32, 32, 16, "bf16", 4371, 120)
