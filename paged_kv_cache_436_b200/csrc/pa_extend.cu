@@ -47,6 +47,7 @@ struct ExtendParams {
   int4* units;                  // optional: two int4 per (seq, tile, chunk) pair, written by the plan
                                 //   {s, tile, chunk index, row0}, {Q, base, first token, visible tokens}
   long long units_cap;          // pairs the records can hold
+  int* queue;                   // tcgen05 path: next unit to hand out (zeroed by the plan kernel)
   int fresh;                    // whole prompts (pa_prefill): every L_s must equal Q_s
 };
 
@@ -126,7 +127,7 @@ __global__ void __launch_bounds__(1024) extend_plan_kernel(const ExtendParams p,
         const int row0 = p.query_start[s];
         int idx = before;
         const int tiles = (Q + qpt - 1) / qpt;
-        for (int t = 0; t < tiles; ++t) {
+        for (int t = tiles - 1; t >= 0; --t) {   // longest tile first (dynamic scheduling takes them in order)
           const int last = base + min((t + 1) * qpt, Q) - 1;
           const int P = ext_tile_parts(base, Q, qpt, t, p.chunk);
           for (int part = 0; part < P && idx < p.units_cap; ++part, ++idx) {
@@ -142,6 +143,7 @@ __global__ void __launch_bounds__(1024) extend_plan_kernel(const ExtendParams p,
     __syncthreads();
   }
   if (threadIdx.x == 0) {
+    if (p.queue) *p.queue = 0;   // the tcgen05 kernel's work queue
     // pairs past the records' capacity (only from inconsistent query_start) are dropped
     if (p.units && carry > p.units_cap) record_error(PA_DEV_BAD_CONTEXT_LEN, -1, carry, int(p.units_cap));
     p.plan[p.num_seqs] = p.units && carry > p.units_cap ? int(p.units_cap) : carry;
@@ -773,7 +775,7 @@ __global__ void __launch_bounds__(128) extend_reduce_kernel(const ExtendParams p
 // host side
 // --------------------------------------------------------------------------
 struct ExtWs {
-  size_t plan, ml, acc, units, total;
+  size_t plan, ml, acc, units, queue, total;
 };
 
 // Unit records: a sequence with Q_s > 0 queries has at most Q_s row tiles (a tile holds at
@@ -790,7 +792,8 @@ inline ExtWs ext_ws(int S, int T, int Hq, int D, int max_parts) {
   w.ml = align256(size_t(S + 1) * 4);
   w.acc = w.ml + align256(size_t(T) * Hq * max_parts * 2 * 4);
   w.units = w.acc + align256(size_t(T) * Hq * max_parts * D * 4);
-  w.total = w.units + align256(ext_units_bound(T, Hq, max_parts) * 32);
+  w.queue = w.units + align256(ext_units_bound(T, Hq, max_parts) * 32);
+  w.total = w.queue + 256;
   return w;
 }
 
@@ -919,6 +922,7 @@ static pa_status extend_impl(const void* q, int32_t q_dtype, int32_t num_seqs, i
   p.part_ml = reinterpret_cast<float*>(w + ws.ml);
   p.part_acc = reinterpret_cast<float*>(w + ws.acc);
   p.units = reinterpret_cast<int4*>(w + ws.units);
+  p.queue = tc ? reinterpret_cast<int*>(w + ws.queue) : nullptr;
   p.units_cap = (long long)ext_units_bound(num_tokens, num_q_heads, max_parts);
   p.fresh = fresh ? 1 : 0;
   p.num_seqs = num_seqs;

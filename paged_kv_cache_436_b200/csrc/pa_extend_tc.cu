@@ -303,6 +303,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // per-tile ring barriers (index = tile & 1); per-unit ones (q_full, o_full/o_empty by unit & 1)
   __shared__ uint64_t k_full[2], v_full[2], k_empty[2], pv_done[2], s_full[2], s_empty[2], p_full[2];
   __shared__ uint64_t q_full, q_empty, o_full[2], o_empty[2], bar_fin, grp_bar[4];
+  __shared__ int uq[4];                        // unit ring: unit k of this CTA in slot k % 4
+  __shared__ uint64_t uq_full[4], uq_empty[4];
   __shared__ uint32_t tmem_slot;
   __shared__ int s_abort;
   volatile int* abort = &s_abort;
@@ -328,6 +330,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     mbar_init(&q_full, 1);
     mbar_init(&q_empty, 1);
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&uq_full[i], 1);
+      mbar_init(&uq_empty[i], kTcSoftmaxWarps + 2);   // V producer, MMA warp, softmax warps
+    }
     for (int i = 0; i < 4; ++i) mbar_init(&grp_bar[i], kTcSplit);
     mbar_init(&bar_fin, 1);
     s_abort = 0;
@@ -343,6 +349,30 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int Hq = p.num_q_heads, Hkv = p.num_kv_heads;
   const int total = p.plan[p.num_seqs] * Hkv;
   uint32_t last_load = 0;           // producer: tiles issued (for the drain after an abort)
+  // Dynamic scheduling: the K producer takes unit k of this CTA from the global queue (the
+  // plan kernel lists each sequence's longest row tile first) and publishes it in the
+  // ring; every other role reads the same sequence. -1 ends the work. False on an abort.
+  auto next_unit = [&](uint32_t k, bool taker, int& u) -> bool {
+    const int slot = k & 3;
+    const uint32_t ph = (k >> 2) & 1;
+    if (taker) {
+      if (!tc_wait_warp(&uq_empty[slot], ph ^ 1, abort, 28, int(k))) return false;
+      int v = 0;
+      if (lane == 0) {
+        v = atomicAdd(p.queue, 1);
+        if (v >= total) v = -1;
+        uq[slot] = v;
+        mbar_arrive(&uq_full[slot]);
+      }
+      u = __shfl_sync(kFull, v, 0);
+      return true;
+    }
+    if (!tc_wait_warp(&uq_full[slot], ph, abort, 29, int(k))) return false;
+    u = *reinterpret_cast<volatile int*>(&uq[slot]);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&uq_empty[slot]);
+    return true;
+  };
 
   if (warp > kTcSoftmaxWarps) {
     // ---------------- producers: warp kTcSoftmaxWarps + 1 streams K, the next one V, by 2-D
@@ -368,8 +398,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       pend_g = -1;
       return true;
     };
-    uint32_t g = 0, k = 0;
-    for (int u = blockIdx.x; u < total && !*abort; u += gridDim.x, ++k) {
+    uint32_t g = 0;
+    for (uint32_t k = 0;; ++k) {
+      int u;
+      if (!next_unit(k, !is_v, u) || u < 0) break;
       const TcUnit x = tc_unit(p, u);
       if (is_v) {   // the unit's q rows: box {64 dims, G heads, QPT queries} per 64-dim half
         if (k > 0 && !tc_wait_warp(&q_empty, (k - 1) & 1, abort, 26, u)) break;
@@ -461,7 +493,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       __syncwarp();
       return true;
     };
-    for (int u = blockIdx.x; u < total && !*abort; u += gridDim.x, ++k) {
+    for (;; ++k) {
+      int u;
+      if (!next_unit(k, false, u) || u < 0) break;
       const TcUnit x = tc_unit(p, u);
       const uint32_t ob = k & 1;
       if (!tc_wait_warp(&q_full, k & 1, abort, 14, u)) break;
@@ -519,7 +553,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       return true;
     };
     uint32_t g = 0, k = 0;
-    for (int u = blockIdx.x; u < total; u += gridDim.x, ++k) {
+    for (;; ++k) {
+      int u;
+      if (!next_unit(k, false, u) || u < 0) break;
       const TcUnit x = tc_unit(p, u);
       const uint32_t ob = k & 1, c_o = 256 + ob * 128 + qs_ * kCW;   // this slice of the O buffer
       const int qi = x.t * QPT + row / G;
