@@ -71,6 +71,48 @@ def test_host_argument_checks_launch_nothing():
                        None) == pa.PA_OK
 
 
+def test_extend_and_prefill_argument_checks_launch_nothing():
+    L = pa.lib()
+    bf = pa.CacheDesc(64, 2, 16, 128, pa.PA_BF16, 1.0, 1.0, 256, 256)
+    fp8 = pa.CacheDesc(64, 2, 16, 128, pa.PA_E4M3, 0.05, 0.05, 256, 256)
+    d64 = pa.CacheDesc(64, 2, 16, 64, pa.PA_BF16, 1.0, 1.0, 256, 256)
+    ws = pa.extend_workspace_size(2, 8, 4, 128, 64)
+    assert ws > 0
+
+    def extend(desc, q_dtype=pa.PA_BF16, Hq=4, q=256, scale=0.1, wsb=ws):
+        return L.pa_extend(q, q_dtype, 2, Hq, 256, 8, ctypes.byref(desc), 256, 4, 256, 64, scale, 256, 256, wsb,
+                           None)
+
+    assert extend(fp8) == pa.PA_ERR_ARG                      # E4M3 caches: decode only
+    assert extend(bf, q_dtype=pa.PA_F16) == pa.PA_ERR_ARG    # q dtype must equal the cache's
+    assert extend(bf, Hq=6) == pa.PA_ERR_ARG                 # G = 3
+    assert extend(bf, scale=float("nan")) == pa.PA_ERR_ARG
+    assert extend(bf, q=258) == pa.PA_ERR_ARG                # q not 16-byte aligned
+    assert extend(bf, wsb=64) == pa.PA_ERR_ARG               # workspace too small
+    assert L.pa_extend(None, pa.PA_BF16, 0, 4, None, 0, ctypes.byref(bf), None, 4, None, 0, 0.1, None, None, 0,
+                       None) == pa.PA_OK                      # nothing to do
+
+    def prefill(desc, scale=0.1, k=256):
+        return L.pa_prefill(256, k, k, pa.PA_BF16, 2, 4, 256, 8, ctypes.byref(desc), 256, 4, 256, 64, scale, 256,
+                            256, ws, None)
+
+    assert prefill(d64) == pa.PA_ERR_ARG                      # head_dim 64: no tcgen05 path
+    assert prefill(bf, scale=-0.1) == pa.PA_ERR_ARG           # the tcgen05 path needs scale > 0
+    assert prefill(fp8) == pa.PA_ERR_ARG
+    # the self-test refuses limits out of range before launching anything
+    assert L.pa_selftest_wait_timeout(0, None) == pa.PA_ERR_ARG
+    assert L.pa_selftest_wait_timeout(3000000, None) == pa.PA_ERR_ARG
+
+
+def test_extend_workspace_size_bounds():
+    size = pa.extend_workspace_size
+    assert size(-1, 8, 4, 128, 64) == 0 and size(2, 8, 0, 128, 64) == 0
+    a, b = size(4, 64, 8, 128, 1024), size(4, 64, 8, 128, 4096)
+    assert 0 < a < b                                          # grows with the partitions a row can span
+    assert size(4, 128, 8, 128, 1024) > a                     # and with the query rows
+    assert a % 256 == 0
+
+
 def _oracle_equal(native: pa.Pool, model: BlockPool):
     assert native.num_free() == model.num_free()
     assert native.free_list() == model.free_list()
