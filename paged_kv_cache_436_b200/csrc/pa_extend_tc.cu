@@ -29,7 +29,7 @@
 //     lost). The group's maximum is combined through TMEM columns and a kTcSplit-arrival
 //     mbarrier; P is computed speculatively with the current reference meanwhile and
 //     recomputed only when the reference moves. P goes to a swizzled K-major shared
-//     tile in the query's 16-bit type and the running sum adds those rounded values;
+//     tile in the query's 16-bit type; the running sum adds the binary32 values;
 //   * a unit that covers a row's whole context writes the output row; otherwise it
 //     writes (max, sum, unnormalised row) for the log-sum-exp merge kernel.
 // Every wait is bounded; on a timeout the kernel records it, every role stops, the MMA
@@ -199,22 +199,20 @@ __device__ __forceinline__ float2 add2(float2 a, float2 b) {
 }
 
 // p = 2^a for a pair, rounded to the 16-bit type and packed (lo in the low half); the
-// rounded values are added to `sum` as a pair.
+// binary32 values are added to `sum` as a pair (the weights in P differ from them by at
+// most one 16-bit rounding each).
 template <int QD>
 __device__ __forceinline__ uint32_t exp2_pack(float2 a, float2& sum) {
   const float p0 = ex2(a.x), p1 = ex2(a.y);
   uint32_t w;
-  float2 r;
   if constexpr (QD == PA_BF16) {
     __nv_bfloat162 v = __floats2bfloat162_rn(p0, p1);
     w = *reinterpret_cast<const uint32_t*>(&v);
-    r = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
   } else {
     __half2 v = __floats2half2_rn(p0, p1);
     w = *reinterpret_cast<const uint32_t*>(&v);
-    r = __half22float2(v);
   }
-  sum = add2(sum, r);
+  sum = add2(sum, make_float2(p0, p1));
   return w;
 }
 
