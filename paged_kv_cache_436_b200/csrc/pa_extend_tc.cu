@@ -161,6 +161,13 @@ __device__ __forceinline__ uint32_t pack2_sum(float lo, float hi, float& sum) {
   }
 }
 
+// max(a, b, c) in one instruction (sm_100 three-input max; a NaN operand is ignored as by fmaxf).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // 2^x on the special-function unit (flushes subnormal results to zero).
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -587,9 +594,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
         for (int e = 0; e < 8; ++e) m8[e] = s[e];
 #pragma unroll
-        for (int c = 8; c < kCW; ++c) m8[c & 7] = fmaxf(m8[c & 7], s[c]);
-        const float pm = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+        for (int c = 8; c + 8 < kCW; c += 16)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) m8[e] = fmax3(m8[e], s[c + e], s[c + 8 + e]);
+        if constexpr ((kCW - 8) % 16 != 0) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) m8[e] = fmaxf(m8[e], s[kCW - 8 + e]);
+        }
+        const float pm = fmaxf(fmax3(m8[0], m8[1], m8[2]), fmax3(fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7]));
         publish(c_s, pm);
         // P(g) goes into buffer b once P(g-2) V(g-2) has finished reading it
         if (!(ok = tc_wait_warp(&pv_done[b], ((g >> 1) & 1) ^ 1, abort, 20, u))) break;
