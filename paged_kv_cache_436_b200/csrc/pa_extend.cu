@@ -9,12 +9,16 @@
 //
 // With 16 query rows per K/V byte the work is a real contraction, so it runs on the
 // tensor cores (mma.sync m16n8k16, 16-bit inputs, binary32 accumulation):
-//   * a work unit is (sequence, kv head, tile of 16 rows, 512-token partition); a row
-//     is a (query, q head of the kv head's group) pair, so a tile holds 16 / G queries;
+//   * a work unit is (sequence, kv head, tile of 16 rows, 512-token partition), read
+//     from the record the plan kernel writes for it; a row is a (query, q head of the
+//     kv head's group) pair, so a tile holds 16 / G queries;
 //   * each warp is an independent persistent worker with a 2-stage ring of K/V blocks;
-//     every token row arrives by its own 1-D bulk copy (TMA engine, no multicast) into
-//     a padded shared-memory row (head_dim * 2 + 16 bytes), which keeps the ldmatrix
-//     reads of 8 rows free of bank conflicts without a tensor map;
+//     a cache block arrives as 128B-swizzled 2-D TMA boxes (one per 64-dim half, no
+//     multicast) and ldmatrix reads it at swizzled addresses, free of bank conflicts;
+//     V rows past the tile's last token are zeroed in shared memory;
+//   * the 64-row cooperative kernel (long runs at head_dim 64) streams each token row
+//     by its own 1-D bulk copy into a padded row (head_dim * 2 + 16 bytes) instead;
+//   * long runs at head_dim 128 go to the tcgen05 kernel of pa_extend_tc.cu;
 //   * S = Q K^T and O += P V per 16-token slice; the S accumulators are reused as the
 //     P operand (rounded to the cache's 16-bit type; the running sum adds the same
 //     rounded values); causal mask per row; online softmax in base 2;
