@@ -370,6 +370,9 @@ def time_extend(name, steps, warmup, device, subset=0):
     if name == "spec4_mix":
         base = synthetic.make("llama13b_mix")
         w, qlen = (synthetic.subset(base, subset) if subset else base), 4
+    elif name == "prefill_gqa_8x2k":   # Llama-3-8B attention shapes: 32 q heads over 8 kv heads
+        w = synthetic.custom(8, 32, 8, 128, 16, "bf16", "bf16", [2048] * 8, 4372, pool_factor=1.05)
+        qlen = 2048
     else:
         w = synthetic.custom(8, 32, 32, 128, 16, "bf16", "bf16", [2048] * 8, 4371, pool_factor=1.05)
         qlen = 2048
@@ -403,7 +406,7 @@ def time_extend(name, steps, warmup, device, subset=0):
 
     ms = timed(call)
     prefill = None
-    if name == "prefill_8x2k":
+    if name.startswith("prefill"):
         # the whole prefill step: the prompts' K / V into the cache plus the attention, as
         # one fused pa_prefill and as pa_reshape_and_cache followed by pa_extend
         k_new = synthetic.normal_values((T, w.num_kv_heads, w.head_dim), w.kv_dtype, w.seed + 12, device)
@@ -542,7 +545,7 @@ def workload_config(w, n_gpus):
             "parallelism": f"replicas{n_gpus}" if n_gpus > 1 else "single GPU"}
 
 
-EXTEND_WORKLOADS = ("spec4_mix", "prefill_8x2k")
+EXTEND_WORKLOADS = ("spec4_mix", "prefill_8x2k", "prefill_gqa_8x2k")
 
 
 def extend_roofline(e, hbm_peak):

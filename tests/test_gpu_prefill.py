@@ -67,3 +67,9 @@ def test_prefill_8x2k_full_size():
     """The benchmarked prefill shapes (8 prompts x 2048 tokens, 32/32 heads, bf16, 16-token
     blocks): every cache slot bit-exact, sampled output rows against the oracle."""
     run_prefill_case([2048] * 8, 32, 32, 16, "bf16", 4371, 120)
+
+
+def test_prefill_gqa_8x2k_full_size():
+    """The benchmarked GQA prefill shapes (Llama-3-8B attention: 32 q heads over 8 kv heads,
+    8 prompts x 2048 tokens): every cache slot bit-exact, sampled rows against the oracle."""
+    run_prefill_case([2048] * 8, 32, 8, 16, "bf16", 4372, 120)
