@@ -141,7 +141,10 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+        # the raw samples (the JSON line carries their summary); PA_CLOCKS_DIR keeps them elsewhere
+        import tempfile
+        out_dir = os.environ.get("PA_CLOCKS_DIR") or tempfile.gettempdir()
+        self.path = os.path.join(out_dir, f"pa_clocks_gpu{gpu_index}.csv")
 
     def start(self):
         try:
