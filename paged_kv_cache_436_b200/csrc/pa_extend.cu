@@ -52,6 +52,8 @@ struct ExtendParams {
                                 //   {s, tile, chunk index, row0}, {Q, base, first token, visible tokens}
   long long units_cap;          // pairs the records can hold
   int* queue;                   // tcgen05 path: next unit to hand out (zeroed by the plan kernel)
+  int* row_parts;               // [T] chunks query row t's context spans (0: no valid query);
+                                //   null when no merge pass follows
   int fresh;                    // whole prompts (pa_prefill): every L_s must equal Q_s
 };
 
@@ -80,6 +82,8 @@ __global__ void __launch_bounds__(1024) extend_plan_kernel(const ExtendParams p,
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   grid_dependency_launch_dependents();
   if (threadIdx.x == 0) carry = 0;
+  if (p.row_parts)
+    for (int t = threadIdx.x; t < p.num_tokens; t += blockDim.x) p.row_parts[t] = 0;
   __syncthreads();
   for (int b = 0; b < p.num_seqs; b += blockDim.x) {
     const int s = b + threadIdx.x;
@@ -145,6 +149,13 @@ __global__ void __launch_bounds__(1024) extend_plan_kernel(const ExtendParams p,
     __syncthreads();
     if (threadIdx.x == blockDim.x - 1) carry = before + units;
     __syncthreads();
+  }
+  // chunks each query row spans (the merge kernel reads them): a warp per sequence
+  for (int s = warp; p.row_parts && s < p.num_seqs; s += blockDim.x >> 5) {
+    int Q, base;
+    ext_seq(p, s, Q, base);
+    const int row0 = p.query_start[s];
+    for (int i = lane; i < Q; i += 32) p.row_parts[row0 + i] = (base + i + 1 + p.chunk - 1) / p.chunk;
   }
   if (threadIdx.x == 0) {
     if (p.queue) *p.queue = 0;   // the tcgen05 kernel's work queue
@@ -725,16 +736,7 @@ __global__ void __launch_bounds__(128) extend_reduce_kernel(const ExtendParams p
   grid_dependency_wait();
   const int th = blockIdx.x;
   const int t = th / p.num_q_heads;
-  int lo = 0, hi = p.num_seqs;                        // sequence owning query row t
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (p.query_start[mid] <= t) lo = mid; else hi = mid;
-  }
-  int Qn, base;
-  ext_seq(p, lo, Qn, base);
-  const int qi = t - p.query_start[lo];
-  if (qi < 0 || qi >= Qn) return;
-  const int P = (base + qi + 1 + p.chunk - 1) / p.chunk;
+  const int P = p.row_parts[t];                       // written by the plan kernel
   if (P <= 1) return;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const size_t sbase = size_t(th) * p.max_parts;
@@ -779,7 +781,7 @@ __global__ void __launch_bounds__(128) extend_reduce_kernel(const ExtendParams p
 // host side
 // --------------------------------------------------------------------------
 struct ExtWs {
-  size_t plan, ml, acc, units, queue, total;
+  size_t plan, ml, acc, units, queue, rows, total;
 };
 
 // Unit records: a sequence with Q_s > 0 queries has at most Q_s row tiles (a tile holds at
@@ -797,7 +799,8 @@ inline ExtWs ext_ws(int S, int T, int Hq, int D, int max_parts) {
   w.acc = w.ml + align256(size_t(T) * Hq * max_parts * 2 * 4);
   w.units = w.acc + align256(size_t(T) * Hq * max_parts * D * 4);
   w.queue = w.units + align256(ext_units_bound(T, Hq, max_parts) * 32);
-  w.total = w.queue + 256;
+  w.rows = w.queue + 256;
+  w.total = w.rows + align256(size_t(T > 0 ? T : 1) * 4);
   return w;
 }
 
@@ -927,6 +930,7 @@ static pa_status extend_impl(const void* q, int32_t q_dtype, int32_t num_seqs, i
   p.part_acc = reinterpret_cast<float*>(w + ws.acc);
   p.units = reinterpret_cast<int4*>(w + ws.units);
   p.queue = tc ? reinterpret_cast<int*>(w + ws.queue) : nullptr;
+  p.row_parts = nullptr;   // set below when a merge pass follows
   p.units_cap = (long long)ext_units_bound(num_tokens, num_q_heads, max_parts);
   p.fresh = fresh ? 1 : 0;
   p.num_seqs = num_seqs;
@@ -971,6 +975,8 @@ static pa_status extend_impl(const void* q, int32_t q_dtype, int32_t num_seqs, i
     grid = int(ctas < cap ? ctas : cap);
   }
   if (grid < 1) grid = 1;
+  const bool merge = (long long)max_parts * kPartitionTokens > p.chunk;   // some row spans several chunks
+  if (merge) p.row_parts = reinterpret_cast<int*>(w + ws.rows);
 
   extend_plan_kernel<<<1, 1024, 0, s>>>(p, rows_per_unit / G);
   if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
@@ -998,7 +1004,7 @@ static pa_status extend_impl(const void* q, int32_t q_dtype, int32_t num_seqs, i
   } else if (ext_launch(k.fn, grid, k.threads, k.smem, s, p) != cudaSuccess) {
     return PA_ERR_CUDA;
   }
-  if (max_parts * kPartitionTokens > p.chunk) {   // some row spans several chunks
+  if (merge) {
     const long long rows = (long long)num_tokens * num_q_heads;
     ExtKernel red = q_dtype == PA_BF16 ? (D == 64 ? extend_reduce_kernel<PA_BF16, 64> : extend_reduce_kernel<PA_BF16, 128>)
                                        : (D == 64 ? extend_reduce_kernel<PA_F16, 64> : extend_reduce_kernel<PA_F16, 128>);
