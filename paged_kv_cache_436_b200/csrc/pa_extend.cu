@@ -543,6 +543,11 @@ __global__ void __launch_bounds__(CoopCfg<D, BS>::kThreads) extend_coop_kernel(c
     const uint64_t pol = l2_policy_evict_first();
     uint32_t g = 0;
     volatile int* abort_flag = &s_abort;
+    auto drain = [&]() {   // after an abort: the copies of the last NS stages land before the warp leaves
+      if (lane == 0)
+        for (uint32_t k = g > NS ? g - NS : 0; k < g; ++k) mbar_wait_bounded(&full[k % NS], (k / NS) & 1, 100000000ull);
+      __syncwarp();
+    };
     for (int u = blockIdx.x; u < total && !*abort_flag; u += gridDim.x) {
       const ExtUnit x = ext_make_unit<BS>(p, u, total, QPT, lane);
       for (int i = 0; i < x.nblk; ++i, ++g) {
@@ -553,6 +558,7 @@ __global__ void __launch_bounds__(CoopCfg<D, BS>::kThreads) extend_coop_kernel(c
             record_error(PA_DEV_WAIT_TIMEOUT, 3, u, st);
             s_abort = 1;
           }
+          drain();
           return;
         }
         const int bid = __shfl_sync(kFull, x.bid, i);
@@ -568,6 +574,7 @@ __global__ void __launch_bounds__(CoopCfg<D, BS>::kThreads) extend_coop_kernel(c
         }
       }
     }
+    if (*abort_flag) drain();   // without an abort the consumers wait for every stage themselves
     return;
   }
 

@@ -354,6 +354,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int Hq = p.num_q_heads, Hkv = p.num_kv_heads;
   const int total = p.plan[p.num_seqs] * Hkv;
   uint32_t last_load = 0;           // producer: tiles issued (for the drain after an abort)
+  uint32_t q_loads = 0;             // V producer: Q tiles issued (likewise)
   // Dynamic scheduling: the K producer takes unit k of this CTA from the global queue (the
   // plan kernel lists each sequence's longest row tile first) and publishes it in the
   // ring; every other role reads the same sequence. -1 ends the work. False on an abort.
@@ -416,6 +417,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           tma_load_3d(sQ + kTcRows * 128, &tq, 64, x.hk * G, x.row0 + x.t * QPT, &q_full);
         }
         __syncwarp();
+        q_loads = k + 1;
       }
       const int32_t* trow = p.block_tables + size_t(x.s) * p.max_blocks;
       auto blocks = [&](int j) { return min(BPT, (x.nvis - j * kTcTok + BS - 1) / BS); };
@@ -748,6 +750,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       uint64_t* full = warp == kTcSoftmaxWarps + 2 ? v_full : k_full;
       for (uint32_t h = last_load >= 2 ? last_load - 2 : 0; h < last_load; ++h)
         mbar_wait_bounded(&full[h & 1], (h >> 1) & 1, 100000000ull);
+      if (q_loads > 0) mbar_wait_bounded(&q_full, (q_loads - 1) & 1, 100000000ull);   // V producer only
     }
   }
   tc_fence_before();
