@@ -78,6 +78,18 @@ def test_key_is_the_whole_prefix():
     assert n == 2
 
 
+def test_a_block_repeated_at_another_position_is_not_reused():
+    """Block 0's tokens again as block 1: its KV was computed at positions 0..3 with no
+    context, so only block 0 is reused (a key of the block's own tokens would reuse it
+    for block 1 as well)."""
+    bs = 4
+    pool = BlockPool(20)
+    cache = PrefixCache(bs)
+    first, _ = _serve(pool, cache, [1, 2, 3, 4, 5, 6, 7, 8], bs)
+    row, n = _serve(pool, cache, [1, 2, 3, 4, 1, 2, 3, 4], bs)
+    assert n == 1 and row[0] == first[0] and row[1] not in first
+
+
 def test_evict_and_clear_release_only_unshared_blocks():
     bs = 4
     pool = BlockPool(20)
@@ -97,6 +109,17 @@ def _native_serve(pool, cache, prompt, bs, mb):
     pool.seq_extend(row, n * bs, len(prompt) - n * bs, bs)
     cache.insert(pool, prompt, row)
     return row, n
+
+
+def test_native_index_does_not_reuse_a_block_at_another_position():
+    bs, NB, MB = 4, 20, 4
+    npool = pa.Pool(NB, np.arange(NB))
+    ncache = pa.PrefixCache(bs)
+    first, _ = _native_serve(npool, ncache, [1, 2, 3, 4, 5, 6, 7, 8], bs, MB)
+    row, n = _native_serve(npool, ncache, [1, 2, 3, 4, 1, 2, 3, 4], bs, MB)
+    assert n == 1 and row[0] == first[0] and row[1] not in first[:2]
+    _, n = _native_serve(npool, ncache, [1, 2, 3, 4, 1, 2, 3, 4, 9], bs, MB)
+    assert n == 2                                      # now cached under its own prefix
 
 
 @pytest.mark.parametrize("seed", [0, 1])
