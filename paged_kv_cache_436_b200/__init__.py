@@ -1,8 +1,10 @@
-"""Python binding of libpa: paged KV-cache decode attention for B200 (sm_100a).
+"""Python binding of libpa: paged KV-cache attention for B200 (sm_100a).
 
 Argument marshalling only. Every step of the path -- the block bookkeeping, the
-KV-cache write, the block copy and the decode attention -- runs inside libpa (C++
-on the host, CUDA kernels on the device). PyTorch provides device memory and
+KV-cache write, the block copy, decode attention, multi-query (extend / prefill)
+attention, the prefix-cache index and beam re-selection -- runs inside libpa (C++
+on the host, CUDA kernels on the device). Host buffers are checked for element type,
+contiguity and the extent the C header states before their pointers are passed. PyTorch provides device memory and
 streams; this module passes ``tensor.data_ptr()`` and the current stream.
 
 There is no fallback: if ``lib/libpa.so`` is missing or cannot be loaded every
@@ -145,17 +147,35 @@ def _stream(stream=None):
     return ctypes.c_void_p(s.cuda_stream)
 
 
-def _i32p(a):
+def _host_ptr(a, bits: int, min_size: int, ptr_type):
+    """Pointer to a contiguous host buffer of `bits`-bit integers (numpy array or CPU
+    tensor) with at least `min_size` elements. The native calls trust the extent the
+    header states, so any other buffer is refused here."""
+    if hasattr(a, "ctypes"):                                   # numpy
+        import numpy as np
+        if a.dtype != np.dtype(f"int{bits}") or not a.flags.c_contiguous:
+            raise TypeError(f"expected a C-contiguous int{bits} array, got {a.dtype} "
+                            f"(contiguous={a.flags.c_contiguous})")
+        n, p = a.size, a.ctypes.data_as(ptr_type)
+    else:                                                      # torch
+        import torch
+        want = torch.int32 if bits == 32 else torch.int64
+        if a.dtype != want or a.device.type != "cpu" or not a.is_contiguous():
+            raise TypeError(f"expected a contiguous host {want} tensor, got {a.dtype} on {a.device}")
+        n, p = a.numel(), ctypes.cast(a.data_ptr(), ptr_type)
+    if n < min_size:
+        raise ValueError(f"host buffer of {n} elements, {min_size} needed")
+    return p
+
+
+def _i32p(a, min_size: int = 0):
     """Pointer into a contiguous host int32 buffer (numpy array or CPU tensor)."""
-    if hasattr(a, "ctypes"):
-        return a.ctypes.data_as(_PI32)
-    return ctypes.cast(a.data_ptr(), _PI32)
+    return _host_ptr(a, 32, min_size, _PI32)
 
 
-def _i64p(a):
-    if hasattr(a, "ctypes"):
-        return a.ctypes.data_as(_PI64)
-    return ctypes.cast(a.data_ptr(), _PI64)
+def _i64p(a, min_size: int = 0):
+    """Pointer into a contiguous host int64 buffer (numpy array or CPU tensor)."""
+    return _host_ptr(a, 64, min_size, _PI64)
 
 
 # ---------------------------------------------------------------------------
@@ -177,8 +197,15 @@ class KVCache:
     """K and V caches [num_blocks, num_kv_heads, block_size, head_dim] plus their scales."""
 
     def __init__(self, k_cache, v_cache, kv_dtype: str, k_scale: float = 1.0, v_scale: float = 1.0):
-        assert k_cache.shape == v_cache.shape and k_cache.dim() == 4
-        assert k_cache.is_contiguous() and v_cache.is_contiguous()
+        if kv_dtype not in DTYPES:
+            raise ValueError(f"kv_dtype must be one of {sorted(DTYPES)}, got {kv_dtype!r}")
+        if k_cache.shape != v_cache.shape or k_cache.dim() != 4:
+            raise ValueError(f"K and V caches must share one 4-D shape, got {tuple(k_cache.shape)} "
+                             f"and {tuple(v_cache.shape)}")
+        if not (k_cache.is_contiguous() and v_cache.is_contiguous()):
+            raise ValueError("K and V caches must be contiguous")
+        if dtype_code(k_cache) != DTYPES[kv_dtype] or dtype_code(v_cache) != DTYPES[kv_dtype]:
+            raise TypeError(f"cache tensors of {k_cache.dtype} / {v_cache.dtype} do not hold {kv_dtype}")
         self.k_cache, self.v_cache = k_cache, v_cache
         self.kv_dtype = kv_dtype
         nb, hkv, bs, d = k_cache.shape
@@ -362,30 +389,32 @@ class Pool:
     def seq_extend(self, row, start_pos: int, n_tokens: int, block_size: int, slots=None):
         cs, cd, done = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
         st = lib().pa_seq_extend(self._h, _i32p(row), row.shape[-1], int(start_pos), int(n_tokens),
-                                 int(block_size), _i64p(slots) if slots is not None else None,
+                                 int(block_size), _i64p(slots, int(n_tokens)) if slots is not None else None,
                                  ctypes.byref(cs), ctypes.byref(cd), ctypes.byref(done))
         _check(st, "pa_seq_extend")
         return cs.value, cd.value
 
     def seq_fork(self, row, n_blocks: int):
-        _check(lib().pa_seq_fork(self._h, _i32p(row), int(n_blocks)), "pa_seq_fork")
+        _check(lib().pa_seq_fork(self._h, _i32p(row, int(n_blocks)), int(n_blocks)), "pa_seq_fork")
 
     def seq_free(self, row, n_blocks: int):
-        _check(lib().pa_seq_free(self._h, _i32p(row), int(n_blocks)), "pa_seq_free")
+        _check(lib().pa_seq_free(self._h, _i32p(row, int(n_blocks)), int(n_blocks)), "pa_seq_free")
 
     def batch_reorder(self, block_tables, context_lens, block_size: int, parents):
         """Beam re-selection in place: row i continues old row parents[i] (host int32 arrays)."""
         import numpy as np
         par = np.ascontiguousarray(parents, dtype=np.int32)
-        _check(lib().pa_batch_reorder(self._h, _i32p(block_tables), _i32p(context_lens), block_tables.shape[0],
-                                      block_tables.shape[1], int(block_size), _i32p(par)), "pa_batch_reorder")
+        S, MB = block_tables.shape
+        _check(lib().pa_batch_reorder(self._h, _i32p(block_tables), _i32p(context_lens, S), S, MB, int(block_size),
+                                      _i32p(par, S)), "pa_batch_reorder")
 
     def batch_append(self, block_tables, positions, block_size: int, slots, cow_pairs, updates):
         """One step's bookkeeping. All buffers are contiguous host arrays; returns (n_cow, n_updates)."""
         ncow, nupd, done = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
-        st = lib().pa_batch_append(self._h, _i32p(block_tables), block_tables.shape[0], block_tables.shape[1],
-                                   _i32p(positions), int(block_size), _i64p(slots), _i64p(cow_pairs),
-                                   ctypes.byref(ncow), _i32p(updates), ctypes.byref(nupd), ctypes.byref(done))
+        S, MB = block_tables.shape
+        st = lib().pa_batch_append(self._h, _i32p(block_tables), S, MB, _i32p(positions, S), int(block_size),
+                                   _i64p(slots, S), _i64p(cow_pairs, 2 * S), ctypes.byref(ncow),
+                                   _i32p(updates, 3 * S), ctypes.byref(nupd), ctypes.byref(done))
         _check(st, "pa_batch_append")
         return ncow.value, nupd.value
 
@@ -395,6 +424,7 @@ class PrefixCache:
 
     def __init__(self, block_size: int):
         self._h = ctypes.c_void_p()
+        self.block_size = int(block_size)
         _check(lib().pa_prefix_cache_create(int(block_size), ctypes.byref(self._h)), "pa_prefix_cache_create")
 
     def __len__(self):
@@ -420,7 +450,8 @@ class PrefixCache:
         import numpy as np
         t = np.ascontiguousarray(tokens, dtype=np.int32)
         n = ctypes.c_int32()
-        _check(lib().pa_prefix_cache_insert(self._h, pool._h, _i32p(t), t.size, _i32p(row), ctypes.byref(n)),
+        rp = _i32p(row, t.size // self.block_size if self.block_size > 0 else 0)   # one entry per full block
+        _check(lib().pa_prefix_cache_insert(self._h, pool._h, _i32p(t), t.size, rp, ctypes.byref(n)),
                "pa_prefix_cache_insert")
         return n.value
 

@@ -269,3 +269,54 @@ def test_alloc_free_cost_is_flat_in_pool_size():
     small = min(per_op(4096) for _ in range(3))
     big = min(per_op(1 << 22) for _ in range(3))
     assert big < 4 * small + 2e-8, (small, big)
+
+
+def test_binding_refuses_host_buffers_it_cannot_pass_safely():
+    """The native calls trust the extents the header states; the binding checks element
+    type, contiguity and size first and leaves the pool untouched when it refuses."""
+    import torch
+    p = pa.Pool(8)
+    with pytest.raises(TypeError):
+        p.seq_append(np.zeros(4, np.int64), 0, 16)                     # int64 row read as int32 pairs
+    with pytest.raises(TypeError):
+        p.seq_append(np.zeros((4, 2), np.int32)[:, 0], 0, 16)          # strided view
+    with pytest.raises(TypeError):
+        p.seq_append(torch.zeros(4, dtype=torch.int64), 0, 16)
+    with pytest.raises(ValueError):
+        p.seq_extend(np.zeros(4, np.int32), 0, 20, 16, np.zeros(19, np.int64))   # slots for 19 of 20 tokens
+    with pytest.raises(ValueError):
+        p.seq_free(np.zeros(2, np.int32), 3)
+    S, MB = 3, 4
+    bt = np.zeros((S, MB), np.int32)
+    with pytest.raises(ValueError):
+        p.batch_append(bt, np.zeros(S, np.int32), 16, np.zeros(S, np.int64), np.zeros(2 * S - 1, np.int64),
+                       np.zeros(3 * S, np.int32))
+    with pytest.raises(ValueError):
+        p.batch_reorder(bt, np.zeros(S - 1, np.int32), 16, [0, 0, 0])
+    assert p.num_free() == 8 and p.free_list() == list(range(8))
+    # the same calls with the right buffers go through
+    row = np.zeros(4, np.int32)
+    slots = np.zeros(20, np.int64)
+    assert p.seq_extend(row, 0, 20, 16, slots) == (-1, -1) and slots[19] == row[1] * 16 + 3
+    c = pa.PrefixCache(4)
+    with pytest.raises(ValueError):
+        c.insert(p, list(range(12)), np.zeros(2, np.int32))            # 3 full blocks, 2 entries
+    assert len(c) == 0
+
+
+def test_kv_cache_descriptor_checks_its_tensors():
+    import torch
+    f16 = torch.zeros((2, 1, 16, 64), dtype=torch.float16)
+    assert pa.KVCache(f16, f16.clone(), "f16").desc.head_dim == 64
+    with pytest.raises(ValueError):
+        pa.KVCache(f16, torch.zeros((2, 1, 16, 32), dtype=torch.float16), "f16")
+    with pytest.raises(ValueError):
+        pa.KVCache(f16.transpose(2, 3), f16.transpose(2, 3), "f16")
+    with pytest.raises(TypeError):
+        pa.KVCache(f16, f16.clone(), "bf16")
+    with pytest.raises(TypeError):
+        pa.KVCache(f16, f16.clone(), "e4m3")
+    with pytest.raises(ValueError):
+        pa.KVCache(f16, f16.clone(), "fp8")
+    u8 = torch.zeros((2, 1, 16, 64), dtype=torch.uint8)
+    assert pa.KVCache(u8, u8.clone(), "e4m3", 0.5, 0.25).desc.k_scale == 0.5
