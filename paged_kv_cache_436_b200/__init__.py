@@ -182,6 +182,48 @@ def _i64p(a, min_size: int = 0):
 # device ops
 # ---------------------------------------------------------------------------
 
+def _dev(t, what: str, dtype=None, ndim=None, min_numel=0, contiguous=True):
+    """Refuse, before its pointer reaches a kernel, a tensor that is not on a CUDA device
+    or does not have the element type, rank, layout or size the header states (a host
+    pointer or a short buffer would be read out of bounds on the device)."""
+    if t is None or not t.is_cuda:
+        raise ValueError(f"{what} must be a CUDA tensor")
+    if dtype is not None and t.dtype not in (dtype if isinstance(dtype, tuple) else (dtype,)):
+        raise TypeError(f"{what}: dtype {t.dtype}, expected {dtype}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{what}: {t.dim()}-D, expected {ndim}-D")
+    if contiguous and not t.is_contiguous():
+        raise ValueError(f"{what} must be contiguous")
+    if t.numel() < min_numel:
+        raise ValueError(f"{what}: {t.numel()} elements, at least {min_numel} needed")
+
+
+def _qk_types():
+    import torch
+    return (torch.float16, torch.bfloat16)
+
+
+def _check_cache(cache: "KVCache"):
+    _dev(cache.k_cache, "k_cache")
+    _dev(cache.v_cache, "v_cache")
+
+
+def _check_attention(q, out, cache: "KVCache", block_tables, context_lens, num_seqs: int):
+    """q / out [rows, Hq, D] of one 16-bit type with D the cache's head_dim; int32 block
+    tables with a row per sequence and an int32 length per sequence."""
+    import torch
+    _dev(q, "q", _qk_types(), 3)
+    if q.shape[2] != cache.desc.head_dim:
+        raise ValueError(f"q head_dim {q.shape[2]} != cache head_dim {cache.desc.head_dim}")
+    _dev(out, "out", q.dtype, 3)
+    if out.shape != q.shape:
+        raise ValueError(f"out shape {tuple(out.shape)} != q shape {tuple(q.shape)}")
+    _check_cache(cache)
+    _dev(block_tables, "block_tables", torch.int32, 2)
+    if block_tables.shape[0] < num_seqs:
+        raise ValueError(f"block_tables has {block_tables.shape[0]} rows for {num_seqs} sequences")
+    _dev(context_lens, "context_lens", torch.int32, None, num_seqs)
+
 def dtype_code(t) -> int:
     import torch
     if t.dtype == torch.float16:
@@ -223,7 +265,19 @@ class KVCache:
 
 def reshape_and_cache(k, v, slot_mapping, cache: KVCache, stream=None) -> None:
     """Write each token's K/V rows ([T, Hkv, D], fp16/bf16) into its slot (int64 [T])."""
+    import torch
     T = k.shape[0]
+    for name, x in (("k", k), ("v", v)):
+        _dev(x, name, _qk_types(), 3, contiguous=False)
+        if tuple(x.shape[1:]) != (cache.desc.num_kv_heads, cache.desc.head_dim) or x.shape[0] != T:
+            raise ValueError(f"{name} shape {tuple(x.shape)} is not [{T}, {cache.desc.num_kv_heads}, "
+                             f"{cache.desc.head_dim}]")
+        if x.stride(2) != 1 or x.stride(1) != cache.desc.head_dim:
+            raise ValueError(f"{name}: heads and dims must be contiguous inside a token")
+    if v.dtype != k.dtype:
+        raise TypeError("k and v differ in dtype")
+    _check_cache(cache)
+    _dev(slot_mapping, "slot_mapping", torch.int64, None, T)
     st = lib().pa_reshape_and_cache(_ptr(k), _ptr(v), dtype_code(k), T, k.stride(0), v.stride(0),
                                     _ptr(slot_mapping), ctypes.byref(cache.desc), _stream(stream))
     _check(st, "pa_reshape_and_cache")
@@ -231,7 +285,13 @@ def reshape_and_cache(k, v, slot_mapping, cache: KVCache, stream=None) -> None:
 
 def copy_blocks(pairs, cache: KVCache, stream=None) -> None:
     """Copy whole blocks src -> dst for each row of the device int64 [n, 2] ``pairs``."""
+    import torch
     n = 0 if pairs is None else pairs.shape[0]
+    if n:
+        _dev(pairs, "pairs", torch.int64, 2)
+        if pairs.shape[1] != 2:
+            raise ValueError(f"pairs shape {tuple(pairs.shape)} is not [n, 2]")
+        _check_cache(cache)
     st = lib().pa_copy_blocks(_ptr(pairs), n, ctypes.byref(cache.desc), _stream(stream))
     _check(st, "pa_copy_blocks")
 
@@ -249,6 +309,8 @@ def decode(q, cache: KVCache, block_tables, context_lens, max_context_len: int, 
     ``stage`` (0, 1 or 2) runs one of the three launches alone.
     """
     S, Hq, _ = q.shape
+    _check_attention(q, out, cache, block_tables, context_lens, S)
+    _dev(workspace, "workspace")
     args = (_ptr(q), dtype_code(q), S, Hq, ctypes.byref(cache.desc), _ptr(block_tables),
             block_tables.shape[1], _ptr(context_lens), int(max_context_len), float(scale), _ptr(out),
             _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
@@ -265,8 +327,12 @@ def extend_workspace_size(num_seqs, num_tokens, num_q_heads, head_dim, max_conte
 def extend(q, cache: KVCache, query_start, block_tables, context_lens, max_context_len: int, scale: float, out,
            workspace, stream=None) -> None:
     """Multi-query causal attention: q, out [T, Hq, D]; query_start int32 [S + 1] (device)."""
+    import torch
     T, Hq, _ = q.shape
+    _dev(query_start, "query_start", torch.int32, 1, 1)
     S = query_start.shape[0] - 1
+    _check_attention(q, out, cache, block_tables, context_lens, S)
+    _dev(workspace, "workspace")
     st = lib().pa_extend(_ptr(q), dtype_code(q), S, Hq, _ptr(query_start), T, ctypes.byref(cache.desc),
                          _ptr(block_tables), block_tables.shape[1], _ptr(context_lens), int(max_context_len),
                          float(scale), _ptr(out), _ptr(workspace), workspace.numel() * workspace.element_size(),
@@ -278,8 +344,17 @@ def prefill(q, k, v, cache: KVCache, query_start, block_tables, context_lens, ma
             out, workspace, stream=None) -> None:
     """Whole prompts: q, out [T, Hq, D]; k, v [T, Hkv, D] (the prompts' keys and values, written
     into the cache by the same kernel); query_start int32 [S + 1]; context_lens = prompt lengths."""
+    import torch
     T, Hq, _ = q.shape
+    _dev(query_start, "query_start", torch.int32, 1, 1)
     S = query_start.shape[0] - 1
+    _check_attention(q, out, cache, block_tables, context_lens, S)
+    for name, x in (("k", k), ("v", v)):
+        _dev(x, name, q.dtype, 3)
+        if tuple(x.shape) != (T, cache.desc.num_kv_heads, cache.desc.head_dim):
+            raise ValueError(f"{name} shape {tuple(x.shape)} is not [{T}, {cache.desc.num_kv_heads}, "
+                             f"{cache.desc.head_dim}]")
+    _dev(workspace, "workspace")
     st = lib().pa_prefill(_ptr(q), _ptr(k), _ptr(v), dtype_code(q), S, Hq, _ptr(query_start), T,
                           ctypes.byref(cache.desc), _ptr(block_tables), block_tables.shape[1], _ptr(context_lens),
                           int(max_context_len), float(scale), _ptr(out), _ptr(workspace),
@@ -303,6 +378,7 @@ def decode_no_alloc(q, cache: KVCache, block_tables, context_lens, max_context_l
     every call on a device (serialise calls that could overlap); sizes needing more
     raise PaError(PA_ERR_ARG)."""
     S, Hq, _ = q.shape
+    _check_attention(q, out, cache, block_tables, context_lens, S)
     st = lib().pa_decode_no_alloc(_ptr(q), dtype_code(q), S, Hq, ctypes.byref(cache.desc), _ptr(block_tables),
                                   block_tables.shape[1], _ptr(context_lens), int(max_context_len), float(scale),
                                   _ptr(out), _stream(stream))
@@ -311,7 +387,13 @@ def decode_no_alloc(q, cache: KVCache, block_tables, context_lens, max_context_l
 
 def block_table_update(updates, block_tables, stream=None) -> None:
     """Apply (seq, col, block) int32 [n, 3] device updates to the device block tables."""
+    import torch
     n = 0 if updates is None else updates.shape[0]
+    _dev(block_tables, "block_tables", torch.int32, 2)
+    if n:
+        _dev(updates, "updates", torch.int32, 2)
+        if updates.shape[1] != 3:
+            raise ValueError(f"updates shape {tuple(updates.shape)} is not [n, 3]")
     st = lib().pa_block_table_update(_ptr(updates), n, _ptr(block_tables), block_tables.shape[0],
                                      block_tables.shape[1], _stream(stream))
     _check(st, "pa_block_table_update")

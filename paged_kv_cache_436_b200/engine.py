@@ -23,7 +23,7 @@ import ctypes
 import numpy as np
 import torch
 
-from . import (EngineConfig, KVCache, Pool, _check, _stream, decode, decode_workspace_size, dtype_code, lib)
+from . import (EngineConfig, KVCache, Pool, _check, _dev, _stream, decode, decode_workspace_size, dtype_code, lib)
 
 _TORCH = {"f16": torch.float16, "bf16": torch.bfloat16}
 
@@ -142,6 +142,12 @@ class DecodeEngine:
         (they must exist already: torch creates an event at its first record)."""
         if scale is not None and float(scale) != self.scale:
             raise ValueError("the softmax scale is fixed when the engine is created")
+        qt = _TORCH[self.q_dtype]
+        for name, t, shape in (("q", q, (self.S, self.Hq, self.D)), ("k_new", k_new, (self.S, self.Hkv, self.D)),
+                               ("v_new", v_new, (self.S, self.Hkv, self.D)), ("out", out, (self.S, self.Hq, self.D))):
+            _dev(t, name, qt, 3)
+            if tuple(t.shape) != shape:
+                raise ValueError(f"{name} shape {tuple(t.shape)} is not {list(shape)}")
         h = self._engine()
         e0 = ctypes.c_void_p(events[0].cuda_event) if events else None
         e1 = ctypes.c_void_p(events[1].cuda_event) if events else None

@@ -180,6 +180,26 @@ def test_gqa_equals_mha_with_duplicated_kv_heads():
     assert torch.equal(out_g.view(torch.int16), out_m.view(torch.int16))
 
 
+def test_binding_refuses_mismatched_device_arguments_before_any_launch():
+    w = synthetic.custom(2, 4, 4, 128, 16, "bf16", "bf16", [40, 20], 81)
+    eng = make_engine(w, DEV)
+    pa.last_device_error()                      # start from a clear error word
+    q = torch.zeros((2, 4, 128), dtype=torch.bfloat16, device=DEV)
+    out = torch.empty_like(q)
+    q64 = torch.zeros((2, 4, 64), dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(ValueError):             # head_dim 64 against a 128 cache: q would be over-read
+        pa.decode(q64, eng.cache, eng.bt_dev, eng.lens_dev, eng.max_context_len, w.scale, torch.empty_like(q64),
+                  eng.ws)
+    with pytest.raises(TypeError):
+        pa.decode(q, eng.cache, eng.bt_dev.long(), eng.lens_dev, eng.max_context_len, w.scale, out, eng.ws)
+    with pytest.raises(ValueError):
+        pa.decode(q, eng.cache, eng.bt_dev[:1], eng.lens_dev, eng.max_context_len, w.scale, out, eng.ws)
+    with pytest.raises(TypeError):
+        pa.decode(q, eng.cache, eng.bt_dev, eng.lens_dev, eng.max_context_len, w.scale, out.float(), eng.ws)
+    torch.cuda.synchronize()
+    assert pa.last_device_error()[0] == 0
+
+
 def test_bad_block_id_is_recorded_not_faulting():
     w = synthetic.custom(2, 4, 4, 128, 16, "bf16", "bf16", [40, 20], 81)
     eng = make_engine(w, DEV)
