@@ -396,17 +396,21 @@ pa_status pa_prefix_cache_create(int32_t block_size, pa_prefix_cache** out);
 void pa_prefix_cache_destroy(pa_prefix_cache* cache);
 int32_t pa_prefix_cache_size(const pa_prefix_cache* cache);
 /* Walks the prompt's full blocks in order; each hit takes a reference and is written
- * to block_table_row[k]; stops at the first miss. *n_matched = blocks reused. */
+ * to block_table_row[k]; stops at the first miss. *n_matched = blocks reused. If a
+ * reference is refused (PA_ERR_STATE: a listed block was freed behind the index's back)
+ * the hits before it stand and *n_matched counts them. */
 pa_status pa_prefix_cache_match(pa_prefix_cache* cache, pa_pool* pool, const int32_t* tokens, int32_t n_tokens,
                                 int32_t* block_table_row, int32_t max_blocks, int32_t* n_matched);
 /* Lists every full block of a sequence (tokens from position 0, blocks in
- * block_table_row) that the index does not hold yet, taking a reference on each. */
+ * block_table_row, one entry per full block) that the index does not hold yet, taking
+ * a reference on each. On an error the entries added before it stand (*n_inserted). */
 pa_status pa_prefix_cache_insert(pa_prefix_cache* cache, pa_pool* pool, const int32_t* tokens, int32_t n_tokens,
                                  const int32_t* block_table_row, int32_t* n_inserted);
 /* Drops, oldest insertion first, up to max_blocks entries whose block only the index
  * holds (refcount 1); those blocks return to the free list. */
 pa_status pa_prefix_cache_evict(pa_prefix_cache* cache, pa_pool* pool, int32_t max_blocks, int32_t* n_evicted);
-/* Drops every entry and its reference. */
+/* Drops every entry and its reference. On an error the entries released before it
+ * have left the index (*n_released); the rest remain listed. */
 pa_status pa_prefix_cache_clear(pa_prefix_cache* cache, pa_pool* pool, int32_t* n_released);
 
 /* ------------------------------------------------------------------------- */

@@ -84,7 +84,10 @@ pa_status pa_prefix_cache_match(pa_prefix_cache* c, pa_pool* pool, const int32_t
         std::memcmp(it->second.tokens.data(), tk, size_t(bs) * sizeof(int32_t)) != 0)
       break;
     const pa_status st = pa_pool_incref(pool, it->second.block);
-    if (st != PA_OK) return st;
+    if (st != PA_OK) {   // the references taken so far stand and are reported
+      *n_matched = n;
+      return st;
+    }
     block_table_row[k] = it->second.block;
     parent = key;
     ++n;
@@ -105,7 +108,10 @@ pa_status pa_prefix_cache_insert(pa_prefix_cache* c, pa_pool* pool, const int32_
     const uint64_t key = block_key(parent, tk, bs);
     if (c->map.find(key) == c->map.end()) {
       const pa_status st = pa_pool_incref(pool, block_table_row[k]);
-      if (st != PA_OK) return st;
+      if (st != PA_OK) {   // the entries added so far stand and are reported
+        if (n_inserted) *n_inserted = added;
+        return st;
+      }
       Entry e;
       e.parent = parent;
       e.block = block_table_row[k];
@@ -124,34 +130,41 @@ pa_status pa_prefix_cache_evict(pa_prefix_cache* c, pa_pool* pool, int32_t max_b
   if (n_evicted) *n_evicted = 0;
   if (!c || !pool || max_blocks < 0) return PA_ERR_ARG;
   int32_t n = 0;
+  pa_status st = PA_OK;
   std::deque<uint64_t> keep;
   for (const uint64_t key : c->order) {
     auto it = c->map.find(key);
-    if (n < max_blocks && pa_pool_refcount(pool, it->second.block) == 1) {
-      const pa_status st = pa_pool_decref(pool, it->second.block);
-      if (st != PA_OK) return st;
-      c->map.erase(it);
-      ++n;
-    } else {
-      keep.push_back(key);
+    if (st == PA_OK && n < max_blocks && pa_pool_refcount(pool, it->second.block) == 1) {
+      st = pa_pool_decref(pool, it->second.block);
+      if (st == PA_OK) {
+        c->map.erase(it);
+        ++n;
+        continue;
+      }
     }
+    keep.push_back(key);   // also every entry from a failed release on: order and map stay in step
   }
   c->order.swap(keep);
   if (n_evicted) *n_evicted = n;
-  return PA_OK;
+  return st;
 }
 
 pa_status pa_prefix_cache_clear(pa_prefix_cache* c, pa_pool* pool, int32_t* n_released) {
   if (n_released) *n_released = 0;
   if (!c || !pool) return PA_ERR_ARG;
   int32_t n = 0;
-  for (const uint64_t key : c->order) {
-    const pa_status st = pa_pool_decref(pool, c->map[key].block);
-    if (st != PA_OK) return st;
+  while (!c->order.empty()) {   // entries leave the index as their reference is returned
+    const uint64_t key = c->order.front();
+    auto it = c->map.find(key);
+    const pa_status st = pa_pool_decref(pool, it->second.block);
+    if (st != PA_OK) {
+      if (n_released) *n_released = n;
+      return st;
+    }
+    c->map.erase(it);
+    c->order.pop_front();
     ++n;
   }
-  c->map.clear();
-  c->order.clear();
   if (n_released) *n_released = n;
   return PA_OK;
 }

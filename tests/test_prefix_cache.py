@@ -122,6 +122,31 @@ def test_native_index_does_not_reuse_a_block_at_another_position():
     assert n == 2                                      # now cached under its own prefix
 
 
+def test_native_index_reports_partial_progress_and_stays_consistent():
+    """A block freed behind the index's back: match keeps and reports the hits before
+    it; clear releases what it can and keeps listing the rest, so a second clear
+    neither crashes nor drops a reference twice."""
+    import ctypes
+    bs = 4
+    p = pa.Pool(8, np.arange(8))
+    c = pa.PrefixCache(bs)
+    toks = np.arange(8, dtype=np.int32)
+    row = np.zeros(4, np.int32)
+    p.seq_extend(row, 0, 8, bs)                              # blocks 0, 1
+    assert c.insert(p, toks, row) == 2
+    p.seq_free(row, 2)                                       # the index holds them alone
+    p.decref(1)                                              # ... until block 1 is freed anyway
+    L, n = pa.lib(), ctypes.c_int32(-1)
+    row2 = np.full(4, -1, np.int32)
+    st = L.pa_prefix_cache_match(c._h, p._h, pa._i32p(toks), 8, pa._i32p(row2), 4, ctypes.byref(n))
+    assert st == pa.PA_ERR_STATE and n.value == 1 and row2[0] == 0 and p.refcount(0) == 2
+    assert c.evict(p, 10) == 0 and len(c) == 2               # block 0 is in use, block 1 is not 1-held
+    st = L.pa_prefix_cache_clear(c._h, p._h, ctypes.byref(n))
+    assert st == pa.PA_ERR_STATE and n.value == 1 and len(c) == 1 and p.refcount(0) == 1
+    st = L.pa_prefix_cache_clear(c._h, p._h, ctypes.byref(n))
+    assert st == pa.PA_ERR_STATE and n.value == 0 and len(c) == 1 and p.refcount(0) == 1
+
+
 @pytest.mark.parametrize("seed", [0, 1])
 def test_native_prefix_cache_matches_oracle(seed):
     rng = np.random.default_rng(200 + seed)
