@@ -357,7 +357,9 @@ pa_status pa_seq_extend(pa_pool* pool, int32_t* block_table_row, int32_t max_blo
  * more reference; the caller copies the row. */
 pa_status pa_seq_fork(pa_pool* pool, const int32_t* block_table_row, int32_t n_blocks);
 
-/* pa_seq_free -- a finished sequence drops one reference of each of its n_blocks blocks. */
+/* pa_seq_free -- a finished sequence drops one reference of each of its n_blocks blocks.
+ * The blocks are checked first: one out of range (PA_ERR_ARG) or already free
+ * (PA_ERR_STATE) drops nothing. */
 pa_status pa_seq_free(pa_pool* pool, const int32_t* block_table_row, int32_t n_blocks);
 
 /*
@@ -492,8 +494,8 @@ pa_status pa_engine_last_step(const pa_engine* engine, int32_t* num_cow, int32_t
  * k times holds its blocks k times and a beam chosen 0 times frees its private
  * blocks. The next pa_seq_append / pa_batch_append into a shared partial block then
  * reports the copy-on-write pair. O(total blocks). The caller refreshes the device
- * mirror of the tables (e.g. a full upload). PA_ERR_ARG / PA_ERR_STATE leave
- * everything unchanged.
+ * mirror of the tables (e.g. a full upload). Every old row's blocks are checked first
+ * (in range and held); PA_ERR_ARG / PA_ERR_STATE leave everything unchanged.
  */
 pa_status pa_batch_reorder(pa_pool* pool, int32_t* block_tables, int32_t* context_lens, int32_t num_seqs,
                            int32_t max_blocks, int32_t block_size, const int32_t* parents);

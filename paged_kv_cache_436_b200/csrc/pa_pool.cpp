@@ -4,6 +4,7 @@
 // are O(1); blocks shared between sequences through reference counts; blocks taken
 // only as a sequence grows. Every operation here is O(1) per block and touches no
 // device memory.
+#include <cstdint>
 #include <cstdlib>
 #include <cstring>
 #include <new>
@@ -38,7 +39,7 @@ inline void push(pa_pool* p, int32_t b) {
   ++p->num_free;
 }
 
-inline int32_t ceil_div(int32_t a, int32_t b) { return (a + b - 1) / b; }
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 }  // namespace
 
@@ -140,7 +141,8 @@ pa_status pa_seq_extend(pa_pool* pool, int32_t* row, int32_t max_blocks, int32_t
   if (n_done) *n_done = 0;
   if (!pool || !row || !cow_src || !cow_dst || n_tokens < 0 || start_pos < 0 || block_size <= 0)
     return PA_ERR_ARG;
-  if (n_tokens > 0 && ceil_div(start_pos + n_tokens, block_size) > max_blocks) return PA_ERR_ARG;
+  if (n_tokens > 0 && ceil_div(int64_t(start_pos) + n_tokens, block_size) > max_blocks) return PA_ERR_ARG;
+  if (int64_t(start_pos) + n_tokens > INT32_MAX) return PA_ERR_ARG;
   *cow_src = *cow_dst = -1;
   for (int32_t i = 0; i < n_tokens; ++i) {
     int64_t slot;
@@ -169,9 +171,13 @@ pa_status pa_seq_fork(pa_pool* pool, const int32_t* row, int32_t n_blocks) {
 
 pa_status pa_seq_free(pa_pool* pool, const int32_t* row, int32_t n_blocks) {
   if (!pool || (!row && n_blocks > 0) || n_blocks < 0) return PA_ERR_ARG;
+  for (int32_t i = 0; i < n_blocks; ++i) {   // checked first: a refused call drops nothing
+    if (!in_range(pool, row[i])) return PA_ERR_ARG;
+    if (pool->refcnt[row[i]] == 0) return PA_ERR_STATE;
+  }
   for (int32_t i = 0; i < n_blocks; ++i) {
     pa_status st = pa_pool_decref(pool, row[i]);
-    if (st != PA_OK) return st;
+    if (st != PA_OK) return st;   // only if a block is listed more often than it is held
   }
   return PA_OK;
 }
@@ -220,25 +226,25 @@ pa_status pa_batch_reorder(pa_pool* pool, int32_t* block_tables, int32_t* contex
   const size_t n = size_t(num_seqs) * max_blocks;
   std::vector<int32_t> old_tables(block_tables, block_tables + n);
   std::vector<int32_t> old_lens(context_lens, context_lens + num_seqs);
+  // every old row's blocks (not only the parents'): each of them loses a reference below
   for (int32_t i = 0; i < num_seqs; ++i) {
-    const int32_t p = parents[i];
-    const int32_t nb = ceil_div(old_lens[p], block_size);
+    const int32_t nb = int32_t(ceil_div(old_lens[i], block_size));
     for (int32_t k = 0; k < nb; ++k)
-      if (!in_range(pool, old_tables[size_t(p) * max_blocks + k]) ||
-          pool->refcnt[old_tables[size_t(p) * max_blocks + k]] == 0)
+      if (!in_range(pool, old_tables[size_t(i) * max_blocks + k]) ||
+          pool->refcnt[old_tables[size_t(i) * max_blocks + k]] == 0)
         return PA_ERR_STATE;
   }
   // every new row takes its references before any old row drops its own
   for (int32_t i = 0; i < num_seqs; ++i) {
     const int32_t p = parents[i];
-    const int32_t nb = ceil_div(old_lens[p], block_size);
+    const int32_t nb = int32_t(ceil_div(old_lens[p], block_size));
     std::memcpy(block_tables + size_t(i) * max_blocks, old_tables.data() + size_t(p) * max_blocks,
                 size_t(max_blocks) * sizeof(int32_t));
     context_lens[i] = old_lens[p];
     for (int32_t k = 0; k < nb; ++k) ++pool->refcnt[old_tables[size_t(p) * max_blocks + k]];
   }
   for (int32_t i = 0; i < num_seqs; ++i) {
-    const int32_t nb = ceil_div(old_lens[i], block_size);
+    const int32_t nb = int32_t(ceil_div(old_lens[i], block_size));
     for (int32_t k = 0; k < nb; ++k) {
       const int32_t b = old_tables[size_t(i) * max_blocks + k];
       if (--pool->refcnt[b] == 0) push(pool, b);

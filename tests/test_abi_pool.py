@@ -320,3 +320,31 @@ def test_kv_cache_descriptor_checks_its_tensors():
         pa.KVCache(f16, f16.clone(), "fp8")
     u8 = torch.zeros((2, 1, 16, 64), dtype=torch.uint8)
     assert pa.KVCache(u8, u8.clone(), "e4m3", 0.5, 0.25).desc.k_scale == 0.5
+
+
+def test_refused_pool_calls_change_nothing():
+    """seq_free and batch_reorder check every block before touching a count; seq_extend
+    refuses positions whose end does not fit in int32."""
+    p = pa.Pool(8, np.arange(8))
+    row = np.zeros(4, np.int32)
+    p.seq_extend(row, 0, 40, 16)                          # blocks 0, 1, 2
+    p.decref(1)                                           # block 1 freed behind the row's back
+    with pytest.raises(pa.PaError) as e:
+        p.seq_free(row, 3)
+    assert e.value.status == pa.PA_ERR_STATE
+    assert [p.refcount(b) for b in range(3)] == [1, 0, 1] and p.num_free() == 6
+    # beam reorder: row 1 is dropped (nobody continues it) and lists an out-of-range id
+    bt = np.array([[0, 2, 0, 0], [7, 99, 0, 0]], np.int32)
+    lens = np.array([20, 20], np.int32)
+    p2 = pa.Pool(8, np.arange(8))
+    for _ in range(3):
+        p2.alloc()                                        # blocks 0, 1, 2 held once
+    with pytest.raises(pa.PaError) as e:
+        p2.batch_reorder(bt, lens, 16, [0, 0])
+    assert e.value.status == pa.PA_ERR_STATE
+    assert bt.tolist() == [[0, 2, 0, 0], [7, 99, 0, 0]] and lens.tolist() == [20, 20]
+    assert [p2.refcount(b) for b in range(8)] == [1, 1, 1, 0, 0, 0, 0, 0]
+    big = np.zeros(4, np.int32)
+    with pytest.raises(pa.PaError) as e:
+        p.seq_extend(big, 2**31 - 10, 20, 16)
+    assert e.value.status == pa.PA_ERR_ARG and p.num_free() == 6
