@@ -1,0 +1,88 @@
+"""The JSON line `bench.py` prints, checked on the CPU: `main()` runs with its GPU timing
+legs replaced by fixed numbers, so the assembly of the line (keys, units, derived values,
+the warm-up floor, the nested roofline / e2e / cpu_baseline / clocks objects) is tested
+without a device. The timing legs themselves run only on a GPU."""
+
+import json
+import os
+
+import pytest
+import torch
+
+import bench
+
+STEPS = 10
+BYTES_PER_STEP = 5.0e9
+MS_PER_STEP = 1.0
+
+
+def _fake_time_ours(w, steps, warmup, device, dist, e2e=True, clocks=True, local_rank=0):
+    res = {"ms_total": MS_PER_STEP * steps, "bytes": BYTES_PER_STEP * steps, "launches": 5 * steps,
+           "seq_tokens": 1000 * steps, "kernel_ms_mean": 0.9, "kernel_bytes_mean": BYTES_PER_STEP,
+           "clocks": {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": [], "samples": 3} if clocks else None,
+           "num_cow": 0, "prefix_report": None}
+    if e2e:
+        res["e2e"] = {"ms_total": 1.1 * steps, "bytes": BYTES_PER_STEP * steps, "h2d": 7, "d2h": 3,
+                      "steps": steps}
+    return res
+
+
+def _fake_time_extend(name, steps, warmup, device, subset=0):
+    return {"workload": name, "ms_per_call": 0.4, "kv_gbs": 6000.0, "tflops": 700.0, "query_rows": 16,
+            "kv_bytes": 1, "flops": 1}
+
+
+@pytest.fixture
+def line(monkeypatch, capsys):
+    monkeypatch.setattr(bench, "time_ours", _fake_time_ours)
+    monkeypatch.setattr(bench, "time_extend", _fake_time_extend)
+    monkeypatch.setattr(bench, "cpu_baseline_obj",
+                        lambda w, budget: {"value": 0.07, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                                           "sample": "fixed"})
+    monkeypatch.setattr(torch.cuda, "is_available", lambda: True)
+    monkeypatch.setattr(torch.cuda, "set_device", lambda d: None)
+    for k in ("WORLD_SIZE", "RANK", "LOCAL_RANK"):
+        monkeypatch.delenv(k, raising=False)
+    assert bench.main(["--steps", str(STEPS), "--warmup", "1", "--also", "long_fp8,prefill_8x2k,spec4_mix"]) == 0
+    out = [l for l in capsys.readouterr().out.splitlines() if l.strip()]
+    assert len(out) == 1, "exactly one JSON line"
+    return json.loads(out[0])
+
+
+def test_top_level_keys_and_values(line):
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+              "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "cpu_baseline", "e2e",
+              "gpu_launches", "clocks"):
+        assert k in line, k
+    assert line["metric"] == bench.METRIC and line["unit"] == "GB/s"
+    assert line["n_gpus"] == 1 and line["steps"] == STEPS
+    assert line["warmup"] == 3                                   # raised to the floor of 3
+    assert line["higher_is_better"] is True and line["scaling"] == "weak" and line["vs_baseline"] is None
+    assert line["data"] == "synthetic" and line["dtype"] == "bf16"
+    assert line["config"]["workload"] == "llama13b_mix"
+    assert line["value"] == pytest.approx(BYTES_PER_STEP / (MS_PER_STEP / 1e3) / 1e9)
+    assert line["ms_per_step"] == pytest.approx(MS_PER_STEP)
+    assert line["gpu_launches"] == 5 * STEPS
+
+
+def test_nested_objects(line):
+    r = line["roofline"]
+    for k in ("bound", "achieved", "peak", "unit", "frac", "traffic"):
+        assert k in r, k
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert r["achieved"] == pytest.approx(BYTES_PER_STEP / 0.9e-3 / 1e9)
+    assert r["frac"] == pytest.approx(r["achieved"] / r["peak"])
+    peaks = json.load(open(os.path.join(bench.ROOT, "MEASURED_PEAKS.json")))
+    assert r["peak"] == pytest.approx(float(peaks["hbm_gbs"]))
+    e = line["e2e"]
+    assert e["unit"] == "GB/s" and e["h2d_bytes_per_step"] == 7 and e["d2h_bytes_per_step"] == 3
+    assert e["value"] == pytest.approx(BYTES_PER_STEP / 1.1e-3 / 1e9)
+    c = line["cpu_baseline"]
+    assert {"value", "unit", "cores", "kind", "sample"} <= set(c) and c["kind"] == "oracle"
+    assert {"sm_mhz", "sm_max_mhz", "reasons"} <= set(line["clocks"])
+    names = [x["workload"] for x in line["extend"]]
+    assert names == ["prefill_8x2k", "spec4_mix"]
+    pre, spec = line["extend"]
+    assert pre["roofline"]["bound"] == "tensor" and pre["roofline"]["unit"] == "TFLOP/s"
+    assert spec["roofline"]["bound"] == "hbm" and spec["roofline"]["frac"] == pytest.approx(6000.0 / r["peak"])
+    assert [x["workload"] for x in line["also"]] == ["long_fp8"]
