@@ -1,19 +1,25 @@
 /*
- * pa.h -- C ABI of libpa: paged KV-cache decode attention for NVIDIA B200 (sm_100a).
+ * pa.h -- C ABI of libpa for NVIDIA B200 (sm_100a): paged KV-cache decode attention,
+ * the cache write and block copy it needs, the host block pool, and on the same cache
+ * multi-query (extend) and whole-prompt (prefill) attention, a prefix-cache index and
+ * beam re-selection.
  *
  * The method (PagedAttention as three web pages describe it):
  *   page 1 "突破GPU内存瓶颈：vLLM与PagedAttention技术深度解析", section
  *          "2. PagedAttention的革命性设计" -- fixed-size blocks, a per-sequence block
  *          table mapping logical to physical blocks, blocks shared between sequences;
+ *          section "5. 高级应用场景" -- parallel sampling and beam search share blocks;
  *   page 2 (untitled; first section "1. 为什么vLLM能实现24倍推理加速"), section
  *          "1.1 PagedAttention的内存管理革命" -- the op
  *          paged_attention(queries, key_cache, value_cache, block_tables); section
+ *          "2.1 核心组件交互流程" -- prefill, decode and extend modes; section
  *          "2.2 关键数据结构剖析" -- the metadata (block_tables, context_lens,
- *          num_heads, head_size); section "3.3 常见问题排查" -- the v2 kernel for long
- *          text; section "4.2 混合精度策略" -- an FP8 KV cache;
+ *          query lengths, num_heads, head_size); section "3.3 常见问题排查" -- the v2
+ *          kernel for long text; section "4.2 混合精度策略" -- an FP8 KV cache;
  *   page 3 "内存优化：KV Cache管理、PagedAttention原理与内存池配置", section
  *          "PagedAttention原理" -- blocks of 16 or 32 tokens, refcounted sharing, a free
- *          list with O(1) alloc/free and no device allocation per request.
+ *          list with O(1) alloc/free and no device allocation per request; section
+ *          "案例与场景" -- a hash index over the blocks of common prefixes.
  *
  * Conventions for every call below.
  *   - Device pointers are plain CUDA device addresses owned by the caller; the
