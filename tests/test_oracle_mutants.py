@@ -28,7 +28,7 @@ def _fails(fn, *args):
     return False
 
 
-def test_dropped_softmax_scale_is_fails(monkeypatch):
+def test_dropped_softmax_scale_is_caught(monkeypatch):
     def mutant(q, K, V, scale):
         x = K @ q
         w = np.exp(x - np.max(x)) if len(x) else x
@@ -37,13 +37,13 @@ def test_dropped_softmax_scale_is_fails(monkeypatch):
     assert _fails(ta.test_paged_equals_contiguous_brute_force, 1)
 
 
-def test_scores_against_values_is_fails(monkeypatch):
+def test_scores_against_values_is_caught(monkeypatch):
     orig = attention.softmax_weighted_sum
     monkeypatch.setattr(attention, "softmax_weighted_sum", lambda q, K, V, s: orig(q, V, V, s))
     assert _fails(ta.test_paged_equals_contiguous_brute_force, 1)
 
 
-def test_interleaved_gqa_mapping_is_fails(monkeypatch):
+def test_interleaved_gqa_mapping_is_caught(monkeypatch):
     orig = attention.gather_sequence
 
     def paged_mutant(q, k_cache, v_cache, block_tables, context_lens, scale, heads=None):
@@ -62,7 +62,7 @@ def test_interleaved_gqa_mapping_is_fails(monkeypatch):
     assert _fails(ta.test_paged_equals_contiguous_brute_force, 2)
 
 
-def test_wrong_in_block_offset_is_fails(monkeypatch):
+def test_wrong_in_block_offset_is_caught(monkeypatch):
     def mutant(cache, row, L, g):
         bs = cache.shape[2]
         rows = [cache[int(row[j // bs]), g, (bs - 1 - j % bs), :] for j in range(L)]
@@ -71,13 +71,35 @@ def test_wrong_in_block_offset_is_fails(monkeypatch):
     assert _fails(ta.test_page1_block_table_gather_order)
 
 
-def test_wrong_e4m3_bias_is_fails(monkeypatch):
+def test_softmax_without_the_maximum_subtracted_is_caught(monkeypatch):
+    def mutant(q, K, V, scale):
+        if K.shape[0] == 0:
+            return np.zeros(V.shape[1])
+        with np.errstate(over="ignore", invalid="ignore"):
+            w = np.exp(scale * (K @ q))                 # overflows for large scores
+            return (w @ V) / np.sum(w)
+    monkeypatch.setattr(attention, "softmax_weighted_sum", mutant)
+    assert _fails(ta.test_huge_scores_stay_finite)
+
+
+def test_wrong_bf16_bias_is_caught(monkeypatch):
+    monkeypatch.setattr(codecs, "decode_bf16", lambda c: codecs._decode_binary(c, 8, 7, 126, True))
+    assert _fails(tc.test_bf16_every_code_matches_torch)
+
+
+def test_e4m3_read_with_ieee_specials_is_caught(monkeypatch):
+    # the all-ones exponent as inf / NaN (E4M3 keeps 256..448 there and has no inf)
+    monkeypatch.setattr(codecs, "decode_e4m3", lambda c: codecs._decode_binary(c, 4, 3, 7, True))
+    assert _fails(tc.test_e4m3_every_code_matches_torch)
+
+
+def test_wrong_e4m3_bias_is_caught(monkeypatch):
     monkeypatch.setattr(codecs, "decode_e4m3",
                         lambda c: codecs._decode_binary(c, 4, 3, 8, False, True))
     assert _fails(tc.test_e4m3_every_code_matches_torch)
 
 
-def test_truncating_encoder_is_fails(monkeypatch):
+def test_truncating_encoder_is_caught(monkeypatch):
     orig_rint = np.rint
     monkeypatch.setattr(codecs.np, "rint", np.floor)
     try:
@@ -117,20 +139,20 @@ def test_extend_mutants_reproduce_the_oracle_when_unmutated(monkeypatch):
         pin()
 
 
-def test_extend_query_not_seeing_itself_is_fails(monkeypatch):
+def test_extend_query_not_seeing_itself_is_caught(monkeypatch):
     monkeypatch.setattr(attention, "paged_extend", _extend_mutant(lambda L, Q, i: L - Q + i))
     assert _fails(te.test_first_prompt_token_returns_its_value_row)
     assert _fails(te.test_brute_force_loops)
 
 
-def test_extend_position_from_context_start_is_fails(monkeypatch):
+def test_extend_position_from_context_start_is_caught(monkeypatch):
     # chunked prefill mistake: query i placed at position i instead of L - Q + i
     monkeypatch.setattr(attention, "paged_extend", _extend_mutant(lambda L, Q, i: i + 1))
     assert _fails(te.test_matches_dense_causal_attention)
     assert _fails(te.test_single_query_is_decode)
 
 
-def test_extend_without_causal_mask_is_fails(monkeypatch):
+def test_extend_without_causal_mask_is_caught(monkeypatch):
     monkeypatch.setattr(attention, "paged_extend", _extend_mutant(lambda L, Q, i: L))
     assert _fails(te.test_matches_dense_causal_attention)
     assert _fails(te.test_first_prompt_token_returns_its_value_row)
@@ -160,19 +182,19 @@ def test_pool_mutant_harness_is_faithful(monkeypatch):
     tp.test_prefix_sharing_cow_count_is_sharers_minus_one()
 
 
-def test_writing_into_a_shared_block_is_fails(monkeypatch):
+def test_writing_into_a_shared_block_is_caught(monkeypatch):
     monkeypatch.setattr(BlockPool, "seq_append", _append_mutant(False, True))
     assert _fails(tp.test_copy_on_write_of_shared_partial_block)
     assert _fails(tp.test_prefix_sharing_cow_count_is_sharers_minus_one)
 
 
-def test_copy_on_write_keeping_the_old_reference_is_fails(monkeypatch):
+def test_copy_on_write_keeping_the_old_reference_is_caught(monkeypatch):
     monkeypatch.setattr(BlockPool, "seq_append", _append_mutant(True, False))
     assert _fails(tp.test_copy_on_write_of_shared_partial_block)
     assert _fails(tp.test_prefix_sharing_cow_count_is_sharers_minus_one)
 
 
-def test_fifo_free_list_is_fails(monkeypatch):
+def test_fifo_free_list_is_caught(monkeypatch):
     def decref(self, b):
         self._check(b)
         if self.refcnt[b] == 0:
@@ -184,7 +206,7 @@ def test_fifo_free_list_is_fails(monkeypatch):
     assert _fails(tp.test_lifo_order_and_errors)
 
 
-def test_reorder_dropping_old_references_first_is_fails(monkeypatch):
+def test_reorder_dropping_old_references_first_is_caught(monkeypatch):
     def reorder(pool, rows, lens, parents):
         for r in rows:
             for b in r:
@@ -200,7 +222,7 @@ def test_reorder_dropping_old_references_first_is_fails(monkeypatch):
 
 # ---- prefix cache -----------------------------------------------------------------
 
-def test_prefix_key_of_the_block_alone_is_fails(monkeypatch):
+def test_prefix_key_of_the_block_alone_is_caught(monkeypatch):
     def key_of_block(self, k, tokens):
         return tuple(tokens[k * self.bs:(k + 1) * self.bs])
 
@@ -231,7 +253,7 @@ def test_prefix_key_of_the_block_alone_is_fails(monkeypatch):
     assert _fails(tpc.test_a_block_repeated_at_another_position_is_not_reused)
 
 
-def test_match_without_a_reference_is_fails(monkeypatch):
+def test_match_without_a_reference_is_caught(monkeypatch):
     orig = PrefixCache.match
 
     def match(self, pool, tokens, row):
