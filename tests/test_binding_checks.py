@@ -75,3 +75,20 @@ def test_check_helper_rules():
     with pytest.raises(ValueError):
         pa._dev(Fake(i32), "x", torch.int32, 2, 13)                     # one element short
     pa._dev(Fake(i32), "x", (torch.float16, torch.int32))
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """No fallback: without libpa.so every entry point raises LibraryMissing."""
+    monkeypatch.setattr(pa, "LIB_PATH", str(tmp_path / "libpa.so"))
+    monkeypatch.setattr(pa, "_lib", None)
+    with pytest.raises(pa.LibraryMissing):
+        pa.lib()
+    with pytest.raises(pa.LibraryMissing):
+        pa.Pool(4)
+    with pytest.raises(pa.LibraryMissing):
+        pa.PrefixCache(16)
+    with pytest.raises(pa.LibraryMissing):
+        pa.decode_workspace_size(1, 1, 128, 16)
+    (tmp_path / "libpa.so").write_bytes(b"not a shared object")
+    with pytest.raises(pa.LibraryMissing):
+        pa.lib()
