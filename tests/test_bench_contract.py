@@ -4,7 +4,6 @@ the warm-up floor, the nested roofline / e2e / cpu_baseline / clocks objects) is
 without a device. The timing legs themselves run only on a GPU."""
 
 import json
-import os
 
 import pytest
 import torch
@@ -72,8 +71,8 @@ def test_nested_objects(line):
     assert r["bound"] == "hbm" and r["unit"] == "GB/s"
     assert r["achieved"] == pytest.approx(BYTES_PER_STEP / 0.9e-3 / 1e9)
     assert r["frac"] == pytest.approx(r["achieved"] / r["peak"])
-    peaks = json.load(open(os.path.join(bench.ROOT, "MEASURED_PEAKS.json")))
-    assert r["peak"] == pytest.approx(float(peaks["hbm_gbs"]))
+    hbm, src = bench.peaks()                      # the measured copy bandwidth, else the fallback
+    assert r["peak"] == pytest.approx(hbm) and r["peak_source"].startswith(src)
     e = line["e2e"]
     assert e["unit"] == "GB/s" and e["h2d_bytes_per_step"] == 7 and e["d2h_bytes_per_step"] == 3
     assert e["value"] == pytest.approx(BYTES_PER_STEP / 1.1e-3 / 1e9)
@@ -84,5 +83,6 @@ def test_nested_objects(line):
     assert names == ["prefill_8x2k", "spec4_mix"]
     pre, spec = line["extend"]
     assert pre["roofline"]["bound"] == "tensor" and pre["roofline"]["unit"] == "TFLOP/s"
+    assert pre["roofline"]["peak"] == pytest.approx(bench.bf16_peak()[0])
     assert spec["roofline"]["bound"] == "hbm" and spec["roofline"]["frac"] == pytest.approx(6000.0 / r["peak"])
     assert [x["workload"] for x in line["also"]] == ["long_fp8"]
