@@ -348,3 +348,17 @@ def test_refused_pool_calls_change_nothing():
     with pytest.raises(pa.PaError) as e:
         p.seq_extend(big, 2**31 - 10, 20, 16)
     assert e.value.status == pa.PA_ERR_ARG and p.num_free() == 6
+
+
+def test_engine_metadata_buffer_holds_every_region():
+    """pa_engine_meta_bytes: slots (8 B), copy pairs (16 B), lengths (4 B) and table updates
+    (12 B) per sequence, each region 16-byte aligned; 0 for a negative count."""
+    L = pa.lib()
+    for S in (1, 2, 3, 7, 20, 255, 256, 1000):
+        n = L.pa_engine_meta_bytes(S)
+        regions = [8 * S, 16 * S, 4 * S, 12 * S]
+        want = 0
+        for r in regions:
+            want = (want + 15) // 16 * 16 + r
+        assert n % 16 == 0 and n == (want + 15) // 16 * 16, (S, n)
+    assert L.pa_engine_meta_bytes(-1) == 0
