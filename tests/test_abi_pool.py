@@ -362,3 +362,34 @@ def test_engine_metadata_buffer_holds_every_region():
             want = (want + 15) // 16 * 16 + r
         assert n % 16 == 0 and n == (want + 15) // 16 * 16, (S, n)
     assert L.pa_engine_meta_bytes(-1) == 0
+
+
+def test_engine_create_checks_its_configuration_before_any_cuda_call():
+    """Every refusal here comes from a host check made before the engine creates its
+    CUDA events; the pointers are placeholders and are never dereferenced."""
+    L = pa.lib()
+    pool = pa.Pool(64)
+    S, Hq, MB, maxlen = 4, 8, 8, 128
+    meta = L.pa_engine_meta_bytes(S)
+    ws = L.pa_decode_workspace_size(S, Hq, 128, maxlen)
+
+    def cfg(**kw):
+        c = pa.EngineConfig()
+        c.pool, c.num_seqs, c.num_q_heads, c.max_blocks_per_seq = pool._h, S, Hq, MB
+        c.max_context_len, c.q_dtype, c.scale = maxlen, pa.PA_BF16, 0.125
+        c.cache = pa.CacheDesc(64, 2, 16, 128, pa.PA_BF16, 1.0, 1.0, 256, 256)
+        c.block_tables_host = c.context_lens_host = c.block_tables_dev = 4096
+        c.meta_host[0], c.meta_host[1] = 4096, 8192
+        c.meta_dev, c.meta_bytes, c.workspace, c.workspace_bytes = 4096, meta, 4096, ws
+        for k, v in kw.items():
+            setattr(c, k, v)
+        return c
+
+    out = ctypes.c_void_p()
+    assert L.pa_engine_create(None, ctypes.byref(out)) == pa.PA_ERR_ARG
+    for bad in (dict(pool=None), dict(num_seqs=0), dict(num_q_heads=0), dict(max_blocks_per_seq=0),
+                dict(max_context_len=-1), dict(meta_bytes=meta - 1), dict(meta_dev=4096 + 8),
+                dict(workspace_bytes=ws - 1), dict(workspace=None), dict(block_tables_dev=None)):
+        assert L.pa_engine_create(ctypes.byref(cfg(**bad)), ctypes.byref(out)) == pa.PA_ERR_ARG, bad
+        assert not out.value
+    assert L.pa_engine_step(None, 256, 256, 256, 256, None, None, None) == pa.PA_ERR_ARG
