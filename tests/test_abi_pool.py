@@ -393,3 +393,15 @@ def test_engine_create_checks_its_configuration_before_any_cuda_call():
         assert L.pa_engine_create(ctypes.byref(cfg(**bad)), ctypes.byref(out)) == pa.PA_ERR_ARG, bad
         assert not out.value
     assert L.pa_engine_step(None, 256, 256, 256, 256, None, None, None) == pa.PA_ERR_ARG
+
+
+def test_no_alloc_decode_refuses_oversized_work_before_any_cuda_call():
+    L = pa.lib()
+    desc = pa.CacheDesc(64, 40, 16, 128, pa.PA_BF16, 1.0, 1.0, 256, 256)
+    big = 8192 + 512                                   # 256 seqs x 40 heads x 17 partitions
+    assert L.pa_decode_workspace_size(256, 40, 128, big) > pa.NO_ALLOC_WORKSPACE_BYTES
+    assert L.pa_decode_no_alloc(256, pa.PA_BF16, 256, 40, ctypes.byref(desc), 256, 1024, 256, big, 0.1,
+                                256, None) == pa.PA_ERR_ARG
+    assert L.pa_decode_no_alloc(256, pa.PA_BF16, 256, 40, None, 256, 1024, 256, 16, 0.1, 256, None) == pa.PA_ERR_ARG
+    assert L.pa_decode_no_alloc(256, pa.PA_BF16, -1, 40, ctypes.byref(desc), 256, 1024, 256, 16, 0.1,
+                                256, None) == pa.PA_ERR_ARG
