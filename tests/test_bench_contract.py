@@ -86,3 +86,39 @@ def test_nested_objects(line):
     assert pre["roofline"]["peak"] == pytest.approx(bench.bf16_peak()[0])
     assert spec["roofline"]["bound"] == "hbm" and spec["roofline"]["frac"] == pytest.approx(6000.0 / r["peak"])
     assert [x["workload"] for x in line["also"]] == ["long_fp8"]
+
+
+def test_clock_samples_inside_the_timed_window(tmp_path, monkeypatch):
+    """ClockSampler.stop: median SM clock, max clock and active throttle reasons of the
+    samples inside the timed window only (nvidia-smi replaced by a prepared CSV)."""
+    import datetime
+    monkeypatch.setenv("PA_CLOCKS_DIR", str(tmp_path))
+    s = bench.ClockSampler(0)
+    t0 = datetime.datetime(2026, 1, 1, 12, 0, 0)
+
+    def row(dt, clk, reasons=("Not Active",) * 4):
+        ts = (t0 + datetime.timedelta(seconds=dt)).strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+        return f"{ts}, 0, {clk}, 1965, 900.0, 0x0, " + ", ".join(reasons) + "\n"
+    with open(s.path, "w") as f:
+        f.write(row(0.0, 1200))                                           # before the window
+        f.write(row(1.0, 1965))
+        f.write(row(1.1, 1950, ("Not Active", "Not Active", "Not Active", "Active")))
+        f.write(row(1.2, 1965))
+        f.write("garbage line\n")
+        f.write(row(3.0, 800, ("Active", "Not Active", "Not Active", "Not Active")))  # after it
+
+    class FakeProc:
+        def terminate(self):
+            pass
+
+        def wait(self, timeout=None):
+            return 0
+
+        def kill(self):
+            pass
+    s.proc, s.f = FakeProc(), open(tmp_path / "unused.csv", "w")
+    w0 = (t0 + datetime.timedelta(seconds=0.9)).timestamp()
+    w1 = (t0 + datetime.timedelta(seconds=1.3)).timestamp()
+    c = s.stop((w0, w1))
+    assert c["samples"] == 3 and c["sm_mhz"] == 1965.0 and c["sm_max_mhz"] == 1965.0
+    assert c["reasons"] == ["sw_power_cap"]
