@@ -4,6 +4,7 @@ the warm-up floor, the nested roofline / e2e / cpu_baseline / clocks objects) is
 without a device. The timing legs themselves run only on a GPU."""
 
 import json
+import os
 
 import pytest
 import torch
@@ -122,3 +123,19 @@ def test_clock_samples_inside_the_timed_window(tmp_path, monkeypatch):
     c = s.stop((w0, w1))
     assert c["samples"] == 3 and c["sm_mhz"] == 1965.0 and c["sm_max_mhz"] == 1965.0
     assert c["reasons"] == ["sw_power_cap"]
+
+
+def test_traffic_is_reported_only_for_the_captured_kernel_source(tmp_path, monkeypatch):
+    import json as _json
+    import shutil
+    rec = _json.load(open(os.path.join(bench.ROOT, "profiles", "partition_kernel_traffic.json")))
+    ratio = rec["traffic_per_algorithmic_byte"]["llama13b_mix"]
+    assert bench.kernel_traffic("llama13b_mix", 1.0e9) == pytest.approx(ratio * 1.0e9)
+    assert bench.kernel_traffic("tiny", 1.0e9) is None                 # no capture for it
+    # a copy of the tree whose partition kernel differs by one byte: no traffic figure
+    for d in ("profiles", os.path.join("paged_kv_cache_436_b200", "csrc")):
+        shutil.copytree(os.path.join(bench.ROOT, d), tmp_path / d)
+    with open(tmp_path / "paged_kv_cache_436_b200" / "csrc" / "pa_decode.cu", "a") as f:
+        f.write("\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.kernel_traffic("llama13b_mix", 1.0e9) is None
