@@ -453,6 +453,9 @@ class Pool:
     def num_free(self) -> int:
         return lib().pa_pool_num_free(self._h)
 
+    def num_blocks(self) -> int:
+        return lib().pa_pool_num_blocks(self._h)
+
     def free_list(self):
         import numpy as np
         n = self.num_free()

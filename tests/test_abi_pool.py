@@ -405,3 +405,15 @@ def test_no_alloc_decode_refuses_oversized_work_before_any_cuda_call():
     assert L.pa_decode_no_alloc(256, pa.PA_BF16, 256, 40, None, 256, 1024, 256, 16, 0.1, 256, None) == pa.PA_ERR_ARG
     assert L.pa_decode_no_alloc(256, pa.PA_BF16, -1, 40, ctypes.byref(desc), 256, 1024, 256, 16, 0.1,
                                 256, None) == pa.PA_ERR_ARG
+
+
+def test_pool_size_and_usage():
+    """The pool's size and free count give the cache-usage fraction (blocks in use / total)."""
+    p = pa.Pool(12)
+    assert p.num_blocks() == 12 and p.num_free() == 12
+    taken = [p.alloc() for _ in range(5)]
+    assert p.num_blocks() == 12 and (p.num_blocks() - p.num_free()) / p.num_blocks() == 5 / 12
+    for b in taken:
+        p.decref(b)
+    assert p.num_free() == 12
+    assert pa.lib().pa_pool_num_blocks(None) == -1 and pa.lib().pa_pool_num_free(None) == -1
