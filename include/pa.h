@@ -174,7 +174,9 @@ pa_status pa_decode(const void* q, int32_t q_dtype, int32_t num_seqs, int32_t nu
                     int32_t max_context_len, float scale, void* out, void* workspace,
                     size_t workspace_bytes, void* stream);
 
-/* Bytes of workspace pa_decode needs for these sizes (0 on invalid sizes). */
+/* Bytes of workspace pa_decode needs for these sizes: 0 for a negative sequence count or
+ * context length and for a non-positive head count or head_dim. A size is returned for any
+ * max_context_len >= 0; pa_decode itself refuses one above 6,291,456 (PA_ERR_ARG). */
 size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,
                                 int32_t max_context_len);
 
@@ -244,6 +246,8 @@ pa_status pa_extend(const void* q, int32_t q_dtype, int32_t num_seqs, int32_t nu
                     const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
                     int32_t max_context_len, float scale, void* out, void* workspace, size_t workspace_bytes,
                     void* stream);
+/* Bytes of workspace pa_extend and pa_prefill need: 0 for negative counts or lengths and for a
+ * non-positive head count or head_dim; the same length limit as pa_decode applies to the calls. */
 size_t pa_extend_workspace_size(int32_t num_seqs, int32_t num_tokens, int32_t num_q_heads, int32_t head_dim,
                                 int32_t max_context_len);
 

@@ -417,3 +417,20 @@ def test_pool_size_and_usage():
         p.decref(b)
     assert p.num_free() == 12
     assert pa.lib().pa_pool_num_blocks(None) == -1 and pa.lib().pa_pool_num_free(None) == -1
+
+
+def test_workspace_sizes_at_the_length_limit():
+    """Sizes grow by one partition's partials at 512-token steps up to the 6,291,456-token
+    limit; invalid counts give 0; calls beyond the limit are refused by the calls."""
+    L = pa.lib()
+    for f in (lambda m: L.pa_decode_workspace_size(8, 32, 128, m),
+              lambda m: L.pa_extend_workspace_size(8, 8, 32, 128, m)):
+        assert f(0) == f(1) == f(512) < f(513)
+        assert f(6291456) > f(6291456 - 512) > 0
+    assert L.pa_decode_workspace_size(-1, 32, 128, 16) == 0 and L.pa_decode_workspace_size(1, 0, 128, 16) == 0
+    assert L.pa_extend_workspace_size(1, -1, 32, 128, 16) == 0 and L.pa_extend_workspace_size(1, 1, 32, 0, 16) == 0
+    desc = pa.CacheDesc(64, 32, 16, 128, pa.PA_BF16, 1.0, 1.0, 256, 256)
+    big = 6291456 + 1
+    ws = L.pa_decode_workspace_size(8, 32, 128, big)
+    assert L.pa_decode(256, pa.PA_BF16, 8, 32, ctypes.byref(desc), 256, 1 << 20, 256, big, 0.1, 256, 256, ws,
+                       None) == pa.PA_ERR_ARG
