@@ -196,6 +196,14 @@ def test_binding_refuses_mismatched_device_arguments_before_any_launch():
         pa.decode(q, eng.cache, eng.bt_dev[:1], eng.lens_dev, eng.max_context_len, w.scale, out, eng.ws)
     with pytest.raises(TypeError):
         pa.decode(q, eng.cache, eng.bt_dev, eng.lens_dev, eng.max_context_len, w.scale, out.float(), eng.ws)
+    qs = torch.tensor([0, 1, 2], dtype=torch.int32, device=DEV)
+    with pytest.raises(ValueError):             # extend / prefill check the same way
+        pa.extend(q64, eng.cache, qs, eng.bt_dev, eng.lens_dev, eng.max_context_len, w.scale,
+                  torch.empty_like(q64), eng.ws)
+    kv_bad = torch.zeros((2, 2, 128), dtype=torch.bfloat16, device=DEV)      # 2 kv heads, the cache has 4
+    with pytest.raises(ValueError):
+        pa.prefill(q, kv_bad, kv_bad, eng.cache, qs, eng.bt_dev, eng.lens_dev, eng.max_context_len, w.scale,
+                   out, eng.ws)
     torch.cuda.synchronize()
     assert pa.last_device_error()[0] == 0
 
