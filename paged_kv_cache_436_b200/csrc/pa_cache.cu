@@ -79,15 +79,28 @@ __global__ void __launch_bounds__(128) reshape_kernel(const uint8_t* __restrict_
 }
 
 // grid (pairs, 2): y = 0 copies K, y = 1 copies V; 16-byte vectors over the block.
-__global__ void __launch_bounds__(256) copy_blocks_kernel(const int64_t* __restrict__ pairs,
+// Pairs run concurrently, so a pair is copied only if no other pair of the batch writes
+// its source or its destination, or reads its destination (the relation is symmetric:
+// both pairs of a clash are skipped and one of them is recorded). Every pair that is
+// copied then reads the cache as it was before the call.
+__global__ void __launch_bounds__(256) copy_blocks_kernel(const int64_t* __restrict__ pairs, int num_pairs,
                                                           uint8_t* kc, uint8_t* vc,
                                                           int64_t block_bytes, int num_blocks) {
   const int i = blockIdx.x;
   const int64_t src = pairs[2 * i], dst = pairs[2 * i + 1];
+  auto clamp32 = [](int64_t x) { return int(x < INT32_MIN ? INT32_MIN : (x > INT32_MAX ? INT32_MAX : x)); };
   if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
-    if (threadIdx.x == 0 && blockIdx.y == 0)
-      record_error(PA_DEV_BAD_COPY_PAIR, i, int(src < INT32_MIN ? INT32_MIN : (src > INT32_MAX ? INT32_MAX : src)),
-                   int(dst < INT32_MIN ? INT32_MIN : (dst > INT32_MAX ? INT32_MAX : dst)));
+    if (threadIdx.x == 0 && blockIdx.y == 0) record_error(PA_DEV_BAD_COPY_PAIR, i, clamp32(src), clamp32(dst));
+    return;
+  }
+  int clash = 0;
+  for (int j = threadIdx.x; j < num_pairs; j += blockDim.x) {
+    if (j == i) continue;
+    const int64_t sj = pairs[2 * j], dj = pairs[2 * j + 1];
+    clash |= (dj == src) | (dj == dst) | (sj == dst);
+  }
+  if (__syncthreads_or(clash)) {
+    if (threadIdx.x == 0 && blockIdx.y == 0) record_error(PA_DEV_BAD_COPY_PAIR, i, clamp32(src), clamp32(dst));
     return;
   }
   uint8_t* base = blockIdx.y ? vc : kc;
@@ -182,7 +195,7 @@ pa_status pa_copy_blocks(const int64_t* pairs, int32_t num_pairs, const pa_cache
   const int eb = c->kv_dtype == PA_E4M3 ? 1 : 2;
   const int64_t block_bytes = int64_t(c->num_kv_heads) * c->block_size * c->head_dim * eb;
   pa::copy_blocks_kernel<<<dim3(num_pairs, 2), 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      pairs, static_cast<uint8_t*>(c->k_cache), static_cast<uint8_t*>(c->v_cache), block_bytes, c->num_blocks);
+      pairs, num_pairs, static_cast<uint8_t*>(c->k_cache), static_cast<uint8_t*>(c->v_cache), block_bytes, c->num_blocks);
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 

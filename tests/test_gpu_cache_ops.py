@@ -102,6 +102,29 @@ def test_copy_blocks_bit_exact(kv, Hkv, BS, D):
     assert np.array_equal(codes_np(kc)[perm[21]], codes_np(kc0)[perm[20]])
 
 
+def test_copy_blocks_refuses_chained_pairs():
+    """Pairs run concurrently, so a batch may not chain copies (a block that one pair
+    writes is read or written by another). Such pairs are skipped and recorded; the
+    other pairs of the batch are copied as the oracle copies them (every pair reads the
+    cache as it was before the call); a source shared by two pairs is allowed."""
+    NB, Hkv, BS, D = 30, 2, 16, 64
+    kc0 = _random_cache((NB, Hkv, BS, D), "bf16", 21)
+    vc0 = _random_cache((NB, Hkv, BS, D), "bf16", 22)
+    kc, vc = kc0.clone().to(DEV), vc0.clone().to(DEV)
+    cache = pa.KVCache(kc, vc, "bf16")
+    pairs = np.array([[1, 2], [2, 3],          # chain: 2 is written by pair 0 and read by pair 1
+                      [4, 5], [6, 5],          # two writers of block 5
+                      [7, 8], [7, 9],          # a shared source: allowed
+                      [10, 11], [12, 10],      # pair 1's destination is pair 0's source
+                      [13, 14]], dtype=np.int64)
+    pa.copy_blocks(torch.from_numpy(pairs).to(DEV), cache)
+    code, info = pa.last_device_error()
+    assert code == 4 and (info[1], info[2]) in {tuple(r) for r in pairs[[0, 1, 2, 3, 6, 7]].tolist()}
+    ok = pairs[[4, 5, 8]]
+    ek, ev = oops.copy_blocks(codes_np(kc0), codes_np(vc0), ok)
+    assert np.array_equal(codes_np(kc), ek) and np.array_equal(codes_np(vc), ev)
+
+
 def test_block_table_update():
     bt = torch.full((5, 7), -1, dtype=torch.int32, device=DEV)
     upd = torch.tensor([[0, 0, 11], [4, 6, 3], [2, 3, 9]], dtype=torch.int32, device=DEV)
