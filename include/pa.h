@@ -23,9 +23,15 @@
  *
  * Conventions for every call below.
  *   - Device pointers are plain CUDA device addresses owned by the caller; the
- *     library never allocates or frees device memory, and the only device memory it
- *     holds is the fixed scratch array of pa_decode_no_alloc. Host pointers are
- *     plain host memory owned by the caller.
+ *     library never allocates or frees device memory. The only device memory it
+ *     holds is part of its own device image: the sticky device error word (below)
+ *     and the fixed scratch array of pa_decode_no_alloc. Host pointers are plain
+ *     host memory owned by the caller.
+ *   - The library keeps per-device state for the life of the process: kernel
+ *     attributes set on first use, occupancy figures, and the device address of the
+ *     pa_decode_no_alloc array. All of it belongs to the device's primary context.
+ *     cudaDeviceReset destroys that context (the array may then sit at another
+ *     address), so do not call the library on a device after resetting it.
  *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
  *     stream). GPU calls only enqueue work and return; results are ready when the
  *     stream reaches them.
@@ -132,9 +138,14 @@ pa_status pa_reshape_and_cache(const void* k, const void* v, int32_t in_dtype, i
  * "PagedAttention原理": blocks shared between requests through reference counts;
  * page 1, section "5. 高级应用场景": parallel sampling and beam search).
  *   src_dst_pairs device int64 [num_pairs][2].
- * Pairs are copied concurrently: no block may be the destination of one pair and
- * the source or destination of another. Out-of-range ids skip the pair and are
- * recorded (PA_DEV_BAD_COPY_PAIR). num_pairs == 0 enqueues nothing.
+ * Pairs are copied concurrently, so a batch must not chain copies: no block may be
+ * the destination of one pair and the source or destination of another (two pairs
+ * may share a source). The kernel checks this: a pair that clashes with another in
+ * this way is not copied, and neither is the other one; a clash, like an out-of-range
+ * id, skips the pair and is recorded (PA_DEV_BAD_COPY_PAIR, info = pair index, src,
+ * dst). Every pair that is copied reads the cache as it was before the call. The
+ * check costs each pair a scan of the batch (num_pairs * 16 bytes, from L2).
+ * num_pairs == 0 enqueues nothing.
  */
 pa_status pa_copy_blocks(const int64_t* src_dst_pairs, int32_t num_pairs,
                          const pa_cache_desc* cache, void* stream);
@@ -207,8 +218,10 @@ pa_status pa_decode_stage(int32_t stage, const void* q, int32_t q_dtype, int32_t
  *     rejected with PA_ERR_ARG before anything is enqueued (e.g. 8 sequences x 32 q
  *     heads x 32K tokens x head_dim 128 fit; 256 x 40 heads x 8K do not).
  *   - The first call on a device looks up the array's device address (once per
- *     device, with that device current); make that first call before any stream
- *     capture.
+ *     device, with that device current, through cudaGetSymbolAddress) and keeps it
+ *     for the life of the process; make that first call before any stream capture.
+ *     The address is that of the device's primary context: after cudaDeviceReset it
+ *     is stale (see the conventions above).
  *   - Every call on a device shares the one array and leaves its contents behind;
  *     nothing in it needs to start at zero. Calls that may overlap on the GPU (on
  *     different streams, or from different host threads) race on it: serialise them.
