@@ -195,6 +195,125 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+# Reads the SM clock, its maximum, the power draw and the clock-event reasons every
+# `interval` seconds through NVML (read-only queries) and prints one CSV line per
+# sample with its wall-clock time; the device is found by the UUID or PCI bus id the
+# parent passes (CUDA and NVML number devices differently).
+_NVML_LOOP = r"""
+import sys, time, pynvml as N
+uuid, bus, interval = sys.argv[1], sys.argv[2], float(sys.argv[3])
+N.nvmlInit()
+h = None
+for cand in (uuid, "GPU-" + uuid):
+    try:
+        h = N.nvmlDeviceGetHandleByUUID(cand); break
+    except Exception:
+        pass
+if h is None:
+    h = N.nvmlDeviceGetHandleByPciBusId(bus)
+cmax = N.nvmlDeviceGetMaxClockInfo(h, N.NVML_CLOCK_SM)
+bits = (N.nvmlClocksEventReasonHwSlowdown, N.nvmlClocksEventReasonHwThermalSlowdown,
+        N.nvmlClocksEventReasonSwThermalSlowdown, N.nvmlClocksEventReasonSwPowerCap)
+print("ready", flush=True)
+while True:
+    t = time.time()
+    clk = N.nvmlDeviceGetClockInfo(h, N.NVML_CLOCK_SM)
+    r = N.nvmlDeviceGetCurrentClocksEventReasons(h)
+    pw = N.nvmlDeviceGetPowerUsage(h) / 1000.0
+    print("%.6f,%d,%d,%.1f,%s" % (t, clk, cmax, pw, ",".join("1" if r & b else "0" for b in bits)), flush=True)
+    time.sleep(max(0.0, interval - (time.time() - t)))
+"""
+
+
+class NvmlClockSampler:
+    """Clock record of the timed region sampled every 2 ms through NVML in a child
+    process (no GIL shared with the timing loop): a region of a few tens of
+    milliseconds still gets a dozen samples. Same summary as ClockSampler.stop."""
+
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+    def __init__(self, device, interval=0.002):
+        import tempfile
+        import torch
+        props = torch.cuda.get_device_properties(device)
+        self.uuid = str(props.uuid)
+        self.bus = "%08X:%02X:%02X.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+        self.interval = interval
+        out_dir = os.environ.get("PA_CLOCKS_DIR") or tempfile.gettempdir()
+        self.path = os.path.join(out_dir, f"pa_clocks_nvml_{os.getpid()}.csv")
+        self.proc = None
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen([sys.executable, "-c", _NVML_LOOP, self.uuid, self.bus, str(self.interval)],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+            t0 = time.time()
+            while time.time() - t0 < 30:             # until the first sample is written
+                time.sleep(0.05)
+                if self.proc.poll() is not None:
+                    raise RuntimeError("NVML sampler exited")
+                with open(self.path) as g:
+                    if len(g.read().splitlines()) >= 2:
+                        return True
+            raise RuntimeError("NVML sampler gave no sample")
+        except Exception:
+            self.stop_proc()
+            self.proc = None
+            return False
+
+    def stop_proc(self):
+        if self.proc is not None and self.proc.poll() is None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        try:
+            self.f.close()
+        except Exception:
+            pass
+
+    def stop(self, window=None):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        time.sleep(0.01)
+        self.stop_proc()
+        sm, smax, pw, reasons = [], [], [], set()
+        for line in open(self.path):
+            parts = line.strip().split(",")
+            if len(parts) != 8:
+                continue
+            try:
+                ts, clk, cmax, p = float(parts[0]), float(parts[1]), float(parts[2]), float(parts[3])
+            except ValueError:
+                continue
+            if window is not None and not (window[0] <= ts <= window[1]):
+                continue
+            sm.append(clk)
+            smax.append(cmax)
+            pw.append(p)
+            for n, v in zip(self.NAMES, parts[4:8]):
+                if v == "1":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm), "sm_mhz_min": min(sm), "power_w_median": statistics.median(pw),
+                "source": "NVML every %g ms in the timed region" % (self.interval * 1e3)}
+
+
+def clock_sampler(device, local_rank):
+    """NVML sampling when it works, else nvidia-smi at 100 ms."""
+    s = NvmlClockSampler(device)
+    if s.start():
+        return s
+    s = ClockSampler(local_rank)
+    s.start()
+    return s
+
+
 # ---------------------------------------------------------------------------
 # our implementation
 # ---------------------------------------------------------------------------
@@ -302,9 +421,7 @@ def time_ours(w, steps, warmup, device, dist, e2e=True, clocks=True, local_rank=
         run.step(i)
     torch.cuda.synchronize(device)
     barrier(dist, device)
-    sampler = ClockSampler(local_rank) if clocks else None
-    if sampler:
-        sampler.start()
+    sampler = clock_sampler(device, local_rank) if clocks else None
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     for a, b in kev:            # torch creates the CUDA events at their first record
@@ -451,35 +568,49 @@ def time_extend(name, steps, warmup, device, subset=0):
 # the oracle on the host cores (cpu_baseline and --impl reference)
 # ---------------------------------------------------------------------------
 
-def _sample_item(w, s, rng):
-    """Blocks of sequence s for the oracle, drawn fresh on the host, laid out 0..n-1."""
+def _sample_item(w, s):
+    """Blocks of sequence s for the oracle, drawn on the host from a per-sequence seed
+    (the same in every process), laid out 0..n-1."""
     import synthetic
     L = w.context_lens[s]
     nbk = -(-L // w.block_size)
     shape = (nbk, w.num_kv_heads, w.block_size, w.head_dim)
+    seed = w.seed * 7919 + 2 * s
     if w.kv_dtype == "e4m3":
+        rng = np.random.default_rng(seed)
         kc = rng.integers(0, 0x7E, size=shape, dtype=np.uint8)
         vc = rng.integers(0, 0x7E, size=shape, dtype=np.uint8)
         ks = vs = 6.0 / 448
     else:
-        kc = synthetic.normal_codes(shape, w.kv_dtype, s + 1).numpy().view(np.uint16)
-        vc = synthetic.normal_codes(shape, w.kv_dtype, s + 2).numpy().view(np.uint16)
+        kc = synthetic.normal_codes(shape, w.kv_dtype, seed + 1).numpy().view(np.uint16)
+        vc = synthetic.normal_codes(shape, w.kv_dtype, seed + 2).numpy().view(np.uint16)
         ks = vs = 1.0
     return (s, L, kc, vc, ks, vs, np.arange(nbk, dtype=np.int64)[None, :])
+
+
+def _oracle_q(w):
+    import synthetic
+    return synthetic.normal_codes((w.num_seqs, w.num_q_heads, w.head_dim), w.q_dtype, w.seed + 9).numpy().view(
+        np.uint16)
+
+
+def _seq_bytes(w, s):
+    kvb = 1 if w.kv_dtype == "e4m3" else 2
+    return decode_bytes([w.context_lens[s]], w.num_kv_heads, w.num_q_heads, w.head_dim, kvb, 2, w.block_size)
+
+
+def _seq_order(w):
+    return [int(s) for s in np.random.default_rng(w.seed + 7).permutation(w.num_seqs)]
 
 
 def oracle_sample_inputs(w, budget_s):
     """A bounded sample of the workload for the float64 oracle: whole sequences (all
     heads) in a seeded order, added one at a time until the oracle has spent about
     `budget_s` seconds of CPU time on them."""
-    import synthetic
-    rng = np.random.default_rng(w.seed + 7)
-    order = rng.permutation(w.num_seqs)
-    q = synthetic.normal_codes((w.num_seqs, w.num_q_heads, w.head_dim), w.q_dtype, w.seed + 9).numpy()
-    q = q.view(np.uint16)
+    q = _oracle_q(w)
     items, spent = [], 0.0
-    for s in order:
-        item = _sample_item(w, int(s), rng)
+    for s in _seq_order(w):
+        item = _sample_item(w, s)
         spent += oracle_run(w, q, [item])[2]
         items.append(item)
         if spent >= budget_s:
@@ -491,13 +622,12 @@ def oracle_run(w, q, items):
     """One pass of the oracle over the sample; returns (bytes, tokens, cpu seconds)."""
     from threadpoolctl import threadpool_limits
     from oracle import attention as oatt
-    kvb = 1 if w.kv_dtype == "e4m3" else 2
     nbytes, ntok = 0, 0
     with threadpool_limits(limits=1):
         t0 = time.process_time()
         for s, L, kc, vc, ks, vs, bt in items:
             oatt.paged_decode(q[s:s + 1], w.q_dtype, kc, vc, w.kv_dtype, ks, vs, bt, [L], w.scale)
-            nbytes += decode_bytes([L], w.num_kv_heads, w.num_q_heads, w.head_dim, kvb, 2, w.block_size)
+            nbytes += _seq_bytes(w, s)
             ntok += L
         dt = time.process_time() - t0
     return nbytes, ntok, dt
@@ -510,31 +640,138 @@ def sample_text(w, items, seconds, passes=1):
             f"{passes} pass(es), {seconds:.1f} s of CPU time")
 
 
-def cpu_baseline_obj(w, budget_s):
-    q, items = oracle_sample_inputs(w, budget_s)
+def _workload_by_name(name, subset):
+    import synthetic
+    w = synthetic.make(name)
+    return synthetic.subset(w, subset) if subset else w
+
+
+def _pool_worker(name, subset, seqs, conn):
+    """One oracle process of the all-cores baseline (started with spawn, BLAS limited to
+    one thread): draws its sequences, then runs one timed pass per "run" command."""
+    for var in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS"):
+        os.environ[var] = "1"
+    sys.path.insert(0, ROOT)
+    w = _workload_by_name(name, subset)
+    q = _oracle_q(w)
+    items = [_sample_item(w, s) for s in seqs]
+    conn.send("ready")
+    while conn.recv() == "run":
+        t0 = time.perf_counter()
+        nb, nt, _ = oracle_run(w, q, items)
+        conn.send((nb, nt, time.perf_counter() - t0))
+    conn.close()
+
+
+class OraclePool:
+    """The float64 oracle on `workers` processes at once (one per host core), each over
+    its share of a sample of whole sequences (longest-first onto the least-loaded
+    process). A pass starts every process together; its time is the slowest process's."""
+
+    def __init__(self, w, workers, budget_s, rate_1t, subset=0):
+        import multiprocessing as mp
+        self.w = w
+        self.workers = max(1, int(workers))
+        # whole sequences in the seeded order while the estimated single-thread time of
+        # the sample stays within budget_s on every process
+        quota = budget_s * rate_1t * self.workers
+        chosen, tot = [], 0
+        for s in _seq_order(w):
+            b = _seq_bytes(w, s)
+            if chosen and tot + b > quota:
+                break
+            chosen.append(s)
+            tot += b
+        loads = [0] * self.workers
+        shares = [[] for _ in range(self.workers)]
+        for s in sorted(chosen, key=lambda x: -_seq_bytes(w, x)):
+            k = min(range(self.workers), key=lambda i: loads[i])
+            shares[k].append(s)
+            loads[k] += _seq_bytes(w, s)
+        self.seqs = chosen
+        ctx = mp.get_context("spawn")
+        self.conns, self.procs = [], []
+        for share in shares:
+            if not share:
+                continue
+            a, b = ctx.Pipe()
+            p = ctx.Process(target=_pool_worker, args=(w.name, subset, share, b), daemon=True)
+            p.start()
+            self.conns.append(a)
+            self.procs.append(p)
+        for c in self.conns:
+            assert c.recv() == "ready"
+
+    def run(self):
+        for c in self.conns:
+            c.send("run")
+        res = [c.recv() for c in self.conns]
+        return sum(r[0] for r in res), sum(r[1] for r in res), max(r[2] for r in res)
+
+    def close(self):
+        for c in self.conns:
+            c.send("stop")
+        for p in self.procs:
+            p.join(timeout=30)
+
+    def describe(self, seconds, passes):
+        lens = [self.w.context_lens[s] for s in self.seqs]
+        whole = len(self.seqs) == self.w.num_seqs
+        return (f"float64 numpy oracle on {len(self.procs)} processes (one per host core, BLAS limited to 1 "
+                f"thread each, started together): {'the whole' if whole else 'a sample of the'} "
+                f"{self.w.name} workload, {len(self.seqs)} whole sequences (context lengths "
+                f"{min(lens)}..{max(lens)}, all {self.w.num_q_heads} q heads), {passes} pass(es), "
+                f"{seconds:.1f} s of wall time")
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline_obj(w, budget, subset=0):
+    """The oracle on every host core (the headline figure) and on one thread (a second field)."""
+    q, items = oracle_sample_inputs(w, budget)
     nb, nt, dt = oracle_run(w, q, items)
-    return {"value": nb / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "seq_tokens_per_s": nt / dt, "sample": sample_text(w, items, dt)}
+    one = {"value": nb / dt / 1e9, "unit": "GB/s", "cores": 1, "seq_tokens_per_s": nt / dt,
+           "sample": sample_text(w, items, dt)}
+    pool = OraclePool(w, host_cores(), budget, nb / dt, subset)
+    try:
+        pb, pt, pdt = pool.run()
+        text = pool.describe(pdt, 1)
+        cores = len(pool.procs)
+    finally:
+        pool.close()
+    return {"value": pb / pdt / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "seq_tokens_per_s": pt / pdt, "sample": text, "single_thread": one}
 
 
 def reference_arm(w, args):
-    """--impl reference: the oracle, each step one pass over a bounded sample."""
+    """--impl reference: the oracle on every host core, each step one pass over a bounded
+    sample (all processes at once; the step time is the slowest process's)."""
     per_step = max(0.2, min(2.0, 120.0 / (args.steps + args.warmup)))
-    q, items = oracle_sample_inputs(w, per_step)
-    for _ in range(args.warmup):
-        oracle_run(w, q, items)
-    tb, tt, ts = 0, 0, 0.0
-    for _ in range(args.steps):
-        nb, nt, dt = oracle_run(w, q, items)
-        tb, tt, ts = tb + nb, tt + nt, ts + dt
+    q, items = oracle_sample_inputs(w, min(per_step, 1.0))
+    nb, _, dt = oracle_run(w, q, items)
+    pool = OraclePool(w, host_cores(), per_step, nb / dt, args.subset)
+    try:
+        for _ in range(args.warmup):
+            pool.run()
+        tb, tt, ts = 0, 0, 0.0
+        for _ in range(args.steps):
+            b, t, d = pool.run()
+            tb, tt, ts = tb + b, tt + t, ts + d
+        text = pool.describe(ts, args.steps) + "; ms_per_step is the time of one pass over this sample"
+        cores = len(pool.procs)
+    finally:
+        pool.close()
     gbs = tb / ts / 1e9
     return {"metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ts / args.steps * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
             "config": workload_config(w, 1), "seq_tokens_per_s": tt / ts,
-            "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                             "sample": sample_text(w, items, ts, args.steps) +
-                             "; ms_per_step is the time of one pass over this sample"},
+            "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": text},
             "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
@@ -701,7 +938,7 @@ def main(argv=None):
             e["roofline"] = extend_roofline(e, peak)
             line.setdefault("extend", []).append(e)
         if rank == 0 and world == 1 and not args.no_cpu:
-            line["cpu_baseline"] = cpu_baseline_obj(w, args.cpu_budget)
+            line["cpu_baseline"] = cpu_baseline_obj(w, args.cpu_budget, args.subset)
         if rank == 0:
             print(json.dumps(line))
     finally:

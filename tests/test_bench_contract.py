@@ -37,8 +37,8 @@ def line(monkeypatch, capsys):
     monkeypatch.setattr(bench, "time_ours", _fake_time_ours)
     monkeypatch.setattr(bench, "time_extend", _fake_time_extend)
     monkeypatch.setattr(bench, "cpu_baseline_obj",
-                        lambda w, budget: {"value": 0.07, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                                           "sample": "fixed"})
+                        lambda w, budget, subset=0: {"value": 0.07, "unit": "GB/s", "cores": 1,
+                                                     "kind": "oracle", "sample": "fixed"})
     monkeypatch.setattr(torch.cuda, "is_available", lambda: True)
     monkeypatch.setattr(torch.cuda, "set_device", lambda d: None)
     for k in ("WORLD_SIZE", "RANK", "LOCAL_RANK"):
@@ -123,6 +123,31 @@ def test_clock_samples_inside_the_timed_window(tmp_path, monkeypatch):
     c = s.stop((w0, w1))
     assert c["samples"] == 3 and c["sm_mhz"] == 1965.0 and c["sm_max_mhz"] == 1965.0
     assert c["reasons"] == ["sw_power_cap"]
+
+
+def test_nvml_clock_samples_inside_the_timed_window(tmp_path):
+    """NvmlClockSampler.stop: the same summary from the NVML child's CSV lines (wall
+    time, SM clock, max clock, power, four reason bits), inside the window only."""
+    class FakeProps:
+        uuid, pci_domain_id, pci_bus_id, pci_device_id = "abc", 0, 0x1b, 0
+
+    s = bench.NvmlClockSampler.__new__(bench.NvmlClockSampler)
+    s.interval, s.path, s.uuid, s.bus = 0.002, str(tmp_path / "n.csv"), FakeProps.uuid, "x"
+    with open(s.path, "w") as f:
+        f.write("ready\n")
+        f.write("99.000,1200,1965,300.0,0,0,0,0\n")                       # before the window
+        for k, clk in enumerate((1965, 1950, 1965, 1965)):
+            f.write(f"{100.0 + 0.002 * k:.6f},{clk},1965,950.0,0,0,0,{1 if k == 1 else 0}\n")
+        f.write("bad,line\n")
+        f.write("200.000,800,1965,100.0,1,0,0,0\n")                        # after it
+
+    class FakeProc:
+        def poll(self):
+            return 0
+    s.proc, s.f = FakeProc(), open(tmp_path / "unused.csv", "w")
+    c = s.stop((99.5, 101.0))
+    assert c["samples"] == 4 and c["sm_mhz"] == 1965.0 and c["sm_max_mhz"] == 1965.0 and c["sm_mhz_min"] == 1950
+    assert c["reasons"] == ["sw_power_cap"] and c["power_w_median"] == 950.0
 
 
 def test_traffic_is_reported_only_for_the_captured_kernel_source(tmp_path, monkeypatch):

@@ -91,6 +91,19 @@ def test_reference_arm_runs_on_cpu():
     assert line["e2e"]["h2d_bytes_per_step"] == 0
 
 
+def test_cpu_baseline_on_every_core_and_on_one_thread():
+    """cpu_baseline: the oracle on one process per host core (spawned, one BLAS thread
+    each, a pass timed by its slowest process) with the one-thread figure beside it."""
+    import bench
+    w = synthetic.make("tiny")
+    c = bench.cpu_baseline_obj(w, 0.2)
+    assert c["kind"] == "oracle" and c["unit"] == "GB/s" and c["value"] > 0
+    assert 1 <= c["cores"] <= bench.host_cores() and c["cores"] <= w.num_seqs
+    assert "processes" in c["sample"] and "the whole tiny workload" in c["sample"]
+    one = c["single_thread"]
+    assert one["cores"] == 1 and one["value"] > 0 and "1 thread" in one["sample"]
+
+
 def test_reference_arm_other_ranks_exit_without_work():
     """Under torchrun only rank 0 runs the oracle and prints; rank 1 exits 0 silently."""
     env = dict(os.environ, RANK="1", LOCAL_RANK="1", WORLD_SIZE="2")
