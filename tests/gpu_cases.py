@@ -109,9 +109,10 @@ def check_tables(eng, mirror):
         assert eng.pool.refcount(b) == mirror.pool.refcnt[b]
 
 
-def run_decode_step(w, sample_heads=None, sample_seqs=None, growth=0, device="cuda"):
+def run_decode_step(w, sample_heads=None, sample_seqs=None, growth=0, device="cuda", nan_tails=False):
     """History of L-1 tokens per sequence, then one full step that appends the
-    last token and decodes over L. Returns (max error, engine)."""
+    last token and decodes over L (with nan_tails, every cache byte past the contexts
+    is NaN before the step). Returns (max error, engine)."""
     eng = make_engine(w, device, growth=growth)
     fill_cache(w, eng)
     mir = OracleMirror(w)
@@ -120,6 +121,8 @@ def run_decode_step(w, sample_heads=None, sample_seqs=None, growth=0, device="cu
         mir.extend(s, L - 1)
     check_tables(eng, mir)
     eng.upload_tables()
+    if nan_tails:
+        nan_past_contexts_(w, eng)
     slots_o, cows_o, _ = mir.step_bookkeeping()
     assert cows_o == []
     seqs = range(w.num_seqs) if sample_seqs is None else sample_seqs
@@ -204,3 +207,172 @@ def run_prefill_case(lens, Hq, Hkv, BS, dt, seed, nrows, device="cuda"):
         for h in range(Hq):
             assert torch.equal(out[t, h], v[t, h // (Hq // Hkv)])
     return err
+
+
+# ---------------------------------------------------------------------------
+# every output row at full size: the oracle on all host cores
+# ---------------------------------------------------------------------------
+# Large caches go to the oracle through shared memory, and the oracle runs in a pool of
+# spawned processes (one per host core, one BLAS thread each) over whole sequences;
+# spawn is safe after CUDA is initialised in this process (a fork is not).
+
+def _shared_codes(shape, itemsize):
+    """A zeroed shared-memory block holding an unsigned code array of `shape`."""
+    from multiprocessing import shared_memory
+    n = int(np.prod(shape)) * itemsize
+    shm = shared_memory.SharedMemory(create=True, size=max(n, 1))
+    arr = np.ndarray(shape, dtype=np.uint8 if itemsize == 1 else np.uint16, buffer=shm.buf)
+    return shm, arr
+
+
+def _device_to_shared(t):
+    """Copy a device tensor's codes into shared memory (no intermediate host copy)."""
+    shm, arr = _shared_codes(tuple(t.shape), t.element_size())
+    dst = torch.from_numpy(arr.view(np.uint8) if t.element_size() == 1 else arr.view(np.int16))
+    src = t.view(torch.uint8) if t.element_size() == 1 else t.view(torch.int16)
+    step = max(1, (1 << 28) // max(1, src[0].numel() * t.element_size()))
+    for i in range(0, t.shape[0], step):
+        dst[i:i + step].copy_(src[i:i + step])
+    return shm, arr
+
+
+def _oracle_worker(task):
+    """One process of the pool: the oracle rows of some sequences, caches read from
+    shared memory. task = (kind, shm names, shapes, itemsize, args, rows)."""
+    import os
+    for var in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS"):
+        os.environ[var] = "1"
+    from multiprocessing import shared_memory
+    from threadpoolctl import threadpool_limits
+    from oracle import attention as oatt_w
+    kind, names, shape, itemsize, args, rows = task
+    dt = np.uint8 if itemsize == 1 else np.uint16
+    shms = [shared_memory.SharedMemory(name=n) for n in names]
+    try:
+        kc, vc = (np.ndarray(shape, dtype=dt, buffer=s.buf) for s in shms)
+        with threadpool_limits(limits=1):
+            if kind == "decode":
+                q, qd, kvd, ks, vs, bt, lens, scale = args
+                out = oatt_w.paged_decode(q, qd, kc, vc, kvd, ks, vs, bt, lens, scale, heads=rows)
+            else:
+                q, qd, kvd, ks, vs, bt, lens, qs, scale = args
+                out = oatt_w.paged_extend(q, qd, kc, vc, kvd, ks, vs, bt, lens, qs, scale, rows=rows)
+        idx = tuple(np.array(rows).T)
+        return rows, out[idx]
+    finally:
+        for s in shms:
+            s.close()
+
+
+def oracle_rows_parallel(kind, shm_k, shm_v, shape, itemsize, args, groups):
+    """The oracle's rows for every group of (row, head) pairs, one group per task, on
+    one spawned process per host core. Returns {(row, head): float64 vector}."""
+    import multiprocessing as mp
+    import os
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except AttributeError:
+        cores = os.cpu_count() or 1
+    tasks = [(kind, (shm_k.name, shm_v.name), shape, itemsize, args, g) for g in groups if g]
+    res = {}
+    with mp.get_context("spawn").Pool(processes=max(1, min(cores, len(tasks)))) as pool:
+        for rows, vals in pool.imap_unordered(_oracle_worker, tasks):
+            for r, v in zip(rows, vals):
+                res[tuple(r)] = v
+    return res
+
+
+def nan_code(kv_dtype):
+    """The code of a NaN in the cache's format (E4M3: S.1111.111)."""
+    return 0x7F if kv_dtype == "e4m3" else 0x7FC0 if kv_dtype == "bf16" else 0x7E00
+
+
+def fill_nan_(t, kv_dtype):
+    """Set every element of a cache slice to NaN."""
+    if t.element_size() == 1:
+        t.view(torch.uint8).fill_(nan_code(kv_dtype))
+    else:
+        t.view(torch.int16).fill_(nan_code(kv_dtype))
+
+
+def nan_past_contexts_(w, eng):
+    """Before a step: the cache bytes past every sequence's context (the rest of its last
+    block) and every block no sequence holds (the step may take one) become NaN. Memory
+    the pool handed out but nothing wrote may hold anything; no output may depend on it."""
+    BS = w.block_size
+    held = np.zeros(w.num_blocks, bool)
+    for s in range(w.num_seqs):
+        n = int(eng.lens[s])
+        held[eng.bt_host[s, :-(-n // BS)]] = True
+        if n % BS:
+            b = int(eng.bt_host[s, (n - 1) // BS])
+            fill_nan_(eng.k_cache[b, :, n % BS:, :], w.kv_dtype)
+            fill_nan_(eng.v_cache[b, :, n % BS:, :], w.kv_dtype)
+    free = torch.from_numpy(np.nonzero(~held)[0]).to(eng.device)
+    if free.numel():
+        for c in (eng.k_cache, eng.v_cache):
+            sub = c.index_select(0, free)
+            fill_nan_(sub, w.kv_dtype)
+            c.index_copy_(0, free, sub)
+
+
+def run_decode_step_all_rows(w, device="cuda", nan_tails=True):
+    """One full decode step of the workload (history of L-1 tokens, then the step that
+    appends the last token and decodes over L) with EVERY (sequence, q head) output row
+    compared against the oracle, which runs on all host cores. Cache bytes past every
+    context (the rest of each last block, and every free block the step may take) are
+    NaN first. The whole cache after the step is compared bit for bit with the oracle's
+    (the pre-step cache plus the oracle's own writes of the new tokens)."""
+    eng = make_engine(w, device)
+    fill_cache(w, eng)
+    mir = OracleMirror(w)
+    for s, L in enumerate(w.context_lens):
+        eng.extend(s, L - 1)
+        mir.extend(s, L - 1)
+    check_tables(eng, mir)
+    eng.upload_tables()
+    BS = w.block_size
+    if nan_tails:
+        nan_past_contexts_(w, eng)
+    torch.cuda.synchronize()
+    # the oracle's copy of the whole cache before the step, in shared memory
+    shm_k, ek = _device_to_shared(eng.k_cache)
+    shm_v, ev = _device_to_shared(eng.v_cache)
+    try:
+        slots_o, cows_o, _ = mir.step_bookkeeping()
+        assert cows_o == []
+        q, k, v = synthetic.step_inputs(w, 0)
+        out = torch.full((w.num_seqs, w.num_q_heads, w.head_dim), float("nan"), dtype=q.dtype, device=device)
+        eng.step(q.to(device), k.to(device), v.to(device), out, w.scale)
+        torch.cuda.synchronize()
+        assert pa.last_device_error()[0] == 0
+        check_tables(eng, mir)
+        ks, vs = eng.cache.desc.k_scale, eng.cache.desc.v_scale
+        # the oracle writes the new tokens into its copy, one block at a time
+        kn, vn = codes_np(k), codes_np(v)
+        for t, slot in enumerate(slots_o):
+            b, off = slot // BS, slot % BS
+            nk, nv = oops.reshape_and_cache(kn[t:t + 1], vn[t:t + 1], w.q_dtype, [off], ek[b:b + 1], ev[b:b + 1],
+                                            w.kv_dtype, ks, vs)
+            ek[b], ev[b] = nk[0], nv[0]
+        # the device cache after the step equals the oracle's, bit for bit
+        step = max(1, (1 << 28) // (ek[0].size * ek.itemsize))
+        for c, e in ((eng.k_cache, ek), (eng.v_cache, ev)):
+            for i in range(0, w.num_blocks, step):
+                assert np.array_equal(codes_np(c[i:i + step]), e[i:i + step]), f"cache blocks {i}.. after the step"
+        bt = mir.table(eng.MB).astype(np.int64)
+        args = (codes_np(q), w.q_dtype, w.kv_dtype, ks, vs, bt, list(mir.lens), w.scale)
+        # one task per sequence (all its heads), longest first
+        order = sorted(range(w.num_seqs), key=lambda s: -mir.lens[s])
+        groups = [[(s, h) for h in range(w.num_q_heads)] for s in order]
+        ref = oracle_rows_parallel("decode", shm_k, shm_v, ek.shape, ek.itemsize, args, groups)
+    finally:
+        for shm in (shm_k, shm_v):
+            shm.close()
+            shm.unlink()
+    got = out.double().cpu().numpy()
+    keys = sorted(ref)
+    want = np.stack([ref[r] for r in keys])
+    idx = tuple(np.array(keys).T)
+    assert len(keys) == w.num_seqs * w.num_q_heads
+    return assert_close(got[idx], want, w.kv_dtype, f"{w.name}: every row"), eng

@@ -200,31 +200,41 @@ def _compact(eng, seqs, BS):
     return kc, vc, bt, lens
 
 
-def test_spec4_mix_full_size_sampled():
+def test_spec4_mix_every_row():
     """The benchmarked speculative-verification shapes: 4 draft tokens per sequence over the
-    13B mixed-length contexts (256 sequences, 40/40 heads, bf16), on sampled rows."""
+    13B mixed-length contexts (256 sequences, 40/40 heads, bf16). EVERY (query, head) row
+    against the oracle on all host cores; NaN past every context."""
+    from tests.gpu_cases import _device_to_shared, nan_past_contexts_, oracle_rows_parallel
     w = synthetic.make("llama13b_mix")
     eng = make_engine(w, DEV)
     fill_cache(w, eng)
     for s, L in enumerate(w.context_lens):
         eng.extend(s, L)
     eng.upload_tables()
+    nan_past_contexts_(w, eng)
     qlens = [min(4, L) for L in w.context_lens]
     qs = np.concatenate([[0], np.cumsum(qlens)]).astype(np.int32)
     q = synthetic.normal_values((int(qs[-1]), w.num_q_heads, w.head_dim), w.q_dtype, w.seed + 11).to(DEV)
     out = _run(w, eng, torch.from_numpy(qs).to(DEV), q, qs)
     assert pa.last_device_error()[0] == 0
-    lens = np.array(w.context_lens)
-    pick = []
-    for lo, hi in ((0, 200), (1000, 1100), (8000, 9000)):
-        idx = np.nonzero((lens >= lo) & (lens < hi))[0]
-        pick += idx[[0, -1]].tolist()
-    pick = sorted(set(pick + [int(np.argmax(lens)), w.num_seqs - 1]))
-    kc, vc, bt, L = _compact(eng, pick, w.block_size)
-    rows = [(int(qs[s]) + i, h) for s in pick for i in range(qlens[s]) for h in (0, 13, 27, 39)]
-    ref = oatt.paged_extend(codes_np(q), w.q_dtype, kc, vc, w.kv_dtype, 1.0, 1.0, bt, L, qs, w.scale, rows=rows)
-    idx = tuple(np.array(rows).T)
-    assert_close(out.double().cpu().numpy()[idx], ref[idx], w.kv_dtype, "spec4 mix full size")
+    shm_k, kc = _device_to_shared(eng.k_cache)
+    shm_v, vc = _device_to_shared(eng.v_cache)
+    try:
+        args = (codes_np(q), w.q_dtype, w.kv_dtype, 1.0, 1.0, eng.bt_host.astype(np.int64), list(eng.lens), qs,
+                w.scale)
+        order = sorted(range(w.num_seqs), key=lambda s_: -int(eng.lens[s_]))
+        groups = [[(t, h) for t in range(int(qs[s_]), int(qs[s_ + 1])) for h in range(w.num_q_heads)]
+                  for s_ in order]
+        ref = oracle_rows_parallel("extend", shm_k, shm_v, kc.shape, kc.itemsize, args, groups)
+    finally:
+        for shm in (shm_k, shm_v):
+            shm.close()
+            shm.unlink()
+    keys = sorted(ref)
+    assert len(keys) == int(qs[-1]) * w.num_q_heads
+    idx = tuple(np.array(keys).T)
+    want = np.stack([ref[r] for r in keys])
+    assert_close(out.double().cpu().numpy()[idx], want, w.kv_dtype, "spec4 mix, every row")
 
 
 def test_long_context_many_chunks():
