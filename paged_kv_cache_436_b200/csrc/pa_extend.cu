@@ -20,8 +20,9 @@
 //     by its own 1-D bulk copy into a padded row (head_dim * 2 + 16 bytes) instead;
 //   * long runs at head_dim 128 go to the tcgen05 kernel of pa_extend_tc.cu;
 //   * S = Q K^T and O += P V per 16-token slice; the S accumulators are reused as the
-//     P operand (rounded to the cache's 16-bit type; the running sum adds the same
-//     rounded values); causal mask per row; online softmax in base 2;
+//     P operand (rounded to the cache's 16-bit type; for bf16 the rounded remainder
+//     p - bf16(p) is a second operand, so P enters P V to within 2^-16; the running sum
+//     adds the same values); causal mask per row; online softmax in base 2;
 //   * one partition writes the output row, several write (max, sum, unnormalised row)
 //     for the log-sum-exp merge kernel, as in decode.
 #include <cuda_runtime.h>
@@ -55,6 +56,8 @@ struct ExtendParams {
   int* row_parts;               // [T] chunks query row t's context spans (0: no valid query);
                                 //   null when no merge pass follows
   int fresh;                    // whole prompts (pa_prefill): every L_s must equal Q_s
+  int lo_mode;                  // tcgen05 path: how the bf16 remainder of P enters P V (kLoNone /
+                                //   kLoAlways / kLoAdaptive in pa_extend_tc.cu)
 };
 
 constexpr int kTileRows = 16;
@@ -207,6 +210,33 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi, float& lo_r, float
   hi_r = Q<QD>::to_float(b);
   const uint16_t ua = *reinterpret_cast<const uint16_t*>(&a), ub = *reinterpret_cast<const uint16_t*>(&b);
   return uint32_t(ua) | (uint32_t(ub) << 16);
+}
+
+// The P operands of one 16-token slice (the S accumulator layout reused as the A
+// fragment): p = 2^(s - m) per element; hi = p rounded to the 16-bit type. For bf16 the
+// rounding (up to 2^-8 of p) can move an output by more than the parity tolerance when a
+// few weights dominate and their V values cancel, so the remainder p - hi (exact in
+// binary32) is rounded again into lo and multiplied as a second operand: hi + lo is p to
+// within 2^-16 of p. For f16 (rounding up to 2^-11 of p) lo is not formed. l adds hi + lo.
+template <int QD>
+__device__ __forceinline__ void make_p_operands(const float (&sc)[2][4], const float (&base_m)[2], uint32_t (&hi)[4],
+                                                uint32_t (&lo)[4], float (&l)[2]) {
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const float p0 = exp2f(sc[nt][2 * h] - base_m[h]), p1 = exp2f(sc[nt][2 * h + 1] - base_m[h]);
+      float r0, r1;
+      hi[nt * 2 + h] = pack2<QD>(p0, p1, r0, r1);
+      if constexpr (QD == PA_BF16) {
+        float e0, e1;
+        lo[nt * 2 + h] = pack2<QD>(p0 - r0, p1 - r1, e0, e1);
+        l[h] += (r0 + e0) + (r1 + e1);
+      } else {
+        lo[nt * 2 + h] = 0u;
+        l[h] += r0 + r1;
+      }
+    }
 }
 
 template <int D, int BS>
@@ -418,17 +448,11 @@ __global__ void __launch_bounds__(ExtCfg<D, BS>::kThreads)
           }
           base_m[h] = m[h] == -INFINITY ? 0.f : m[h];
         }
-        // P (rounded to the 16-bit type) as the A operand of P V; l adds the rounded p
-        uint32_t pa[4];
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            float r_lo, r_hi;
-            pa[nt * 2 + h] = pack2<QD>(exp2f(sc[nt][2 * h] - base_m[h]), exp2f(sc[nt][2 * h + 1] - base_m[h]),
-                                       r_lo, r_hi);
-            l[h] += r_lo + r_hi;
-          }
+        // P as the A operand of P V: p rounded to the 16-bit type, and for bf16 also the
+        // rounded remainder p - bf16(p) as a second operand (hi + lo carries p to about
+        // 2^-16); l adds what enters the products
+        uint32_t pa[4], pl[4];
+        make_p_operands<QD>(sc, base_m, pa, pl, l);
         // O += P V (V rows through ldmatrix.trans: two n-tiles of 8 dims per x4)
 #pragma unroll
         for (int np = 0; np < NT / 2; ++np) {
@@ -437,6 +461,10 @@ __global__ void __launch_bounds__(ExtCfg<D, BS>::kThreads)
           ldsm_x4_trans(b, Vs + ext_swz<BS>(trow, np * 2 + (lane >> 4)));
           mma16816<QD>(o[2 * np], pa, b[0], b[1]);
           mma16816<QD>(o[2 * np + 1], pa, b[2], b[3]);
+          if constexpr (QD == PA_BF16) {
+            mma16816<QD>(o[2 * np], pl, b[0], b[1]);
+            mma16816<QD>(o[2 * np + 1], pl, b[2], b[3]);
+          }
         }
       }
       __syncwarp();
@@ -672,16 +700,8 @@ __global__ void __launch_bounds__(CoopCfg<D, BS>::kThreads) extend_coop_kernel(c
             }
             base_m[h] = m[h] == -INFINITY ? 0.f : m[h];
           }
-          uint32_t pa[4];
-#pragma unroll
-          for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              float r_lo, r_hi;
-              pa[nt * 2 + h] = pack2<QD>(exp2f(sc[nt][2 * h] - base_m[h]), exp2f(sc[nt][2 * h + 1] - base_m[h]),
-                                         r_lo, r_hi);
-              l[h] += r_lo + r_hi;
-            }
+          uint32_t pa[4], pl[4];
+          make_p_operands<QD>(sc, base_m, pa, pl, l);
 #pragma unroll
           for (int np = 0; np < NT / 2; ++np) {
             uint32_t b[4];
@@ -689,6 +709,10 @@ __global__ void __launch_bounds__(CoopCfg<D, BS>::kThreads) extend_coop_kernel(c
             ldsm_x4_trans(b, Vs + trow * C::kRowPad + (np * 16 + (lane >> 4) * 8) * 2);
             mma16816<QD>(o[2 * np], pa, b[0], b[1]);
             mma16816<QD>(o[2 * np + 1], pa, b[2], b[3]);
+            if constexpr (QD == PA_BF16) {
+              mma16816<QD>(o[2 * np], pl, b[0], b[1]);
+              mma16816<QD>(o[2 * np + 1], pl, b[2], b[3]);
+            }
           }
         }
       }
@@ -867,6 +891,7 @@ bool extend_tc_supported(int qd, int D, int BS, int G);
 cudaError_t extend_tc_grid_cap(int qd, int BS, int G, int* cap);
 pa_status extend_tc_launch(const ExtendParams& p, const pa_cache_desc* c, int qd, int G, int grid, cudaStream_t s,
                            const void* k_new, const void* v_new);
+int tc_bf16_lo_mode();
 constexpr int kTcUnitRows = 128;
 
 }  // namespace pa
@@ -940,6 +965,7 @@ static pa_status extend_impl(const void* q, int32_t q_dtype, int32_t num_seqs, i
   p.row_parts = nullptr;   // set below when a merge pass follows
   p.units_cap = (long long)ext_units_bound(num_tokens, num_q_heads, max_parts);
   p.fresh = fresh ? 1 : 0;
+  p.lo_mode = q_dtype == PA_BF16 ? tc_bf16_lo_mode() : 0;
   p.num_seqs = num_seqs;
   p.num_tokens = num_tokens;
   p.num_q_heads = num_q_heads;
@@ -959,12 +985,13 @@ static pa_status extend_impl(const void* q, int32_t q_dtype, int32_t num_seqs, i
   int grid = 1;
   p.chunk = kPartitionTokens;
   if (tc) {
-    // the whole context per unit when that already gives two units per SM; otherwise
-    // the largest multiple of the partition length that does (split-K + merge)
+    // the whole context per unit when that already gives two units to each of a CTA's
+    // two pipelines; otherwise the largest multiple of the partition length that does
+    // (split-K + merge)
     int cap = 0;
     if (extend_tc_grid_cap(q_dtype, BS, G, &cap) != cudaSuccess) return PA_ERR_CUDA;
     int nchunks = 1;
-    while (nchunks < max_parts && tiles * c->num_kv_heads * nchunks < 2LL * cap) ++nchunks;
+    while (nchunks < max_parts && tiles * c->num_kv_heads * nchunks < 4LL * cap) ++nchunks;
     const int parts_per_chunk = (max_parts + nchunks - 1) / nchunks;
     p.chunk = parts_per_chunk * kPartitionTokens;
     const long long units = tiles * c->num_kv_heads * ((max_parts + parts_per_chunk - 1) / parts_per_chunk);

@@ -8,52 +8,62 @@
 //     512-token partition, chosen by the host so that there are enough units to fill
 //     the GPU (the whole context when there are, then no merge pass at all); the plan
 //     kernel writes one record per (sequence, tile, chunk);
-//   * one persistent CTA per SM with warp-specialised roles: 8 softmax warps (warps w and
-//     w + 4 share TMEM lanes 32 (w % 4) .. + 31, i.e. rows of the tile, and split the 128
-//     columns into slices of 64: more slices put more warps in lockstep on the same SM
-//     sub-partition and measured slower), one MMA-issue warp, one K and one V producer warp;
-//   * TMEM: S of two consecutive 128-token K/V tiles in columns [0, 256), the output
-//     accumulators O of two consecutive units in [256, 512);
-//   * the unit's Q rows come by one 3-D TMA box per 64-column half (64 dims x G heads x
-//     128 / G queries: the rows in (query, head) order) into a 128B-swizzled K-major
-//     tile, loaded as soon as the previous unit's last S has completed; K and V tiles
-//     come by 2-D TMA (cp.async.bulk.tensor, 128B swizzle, no multicast) straight from
-//     the paged cache, one box per (cache block, 64-column half), into 2-deep K and V
-//     rings;
-//   * S = Q K^T (both K-major) and O += P V (P K-major; V MN-major, i.e. left in its
-//     [token][dim] cache layout) are issued by one thread; order S(g), P(g-1) V(g-1),
-//     S(g+1), ... so that the next S runs while the softmax works on the current one;
-//   * the softmax reads its half of the S row from TMEM, masks causally and keeps a
-//     reference maximum that moves only when the row maximum passes it by more than 2^8
-//     (O and the running sum are then rescaled; every p stays below 2^8, so nothing is
-//     lost). The group's maximum is combined through TMEM columns and a kTcSplit-arrival
-//     mbarrier; P is computed speculatively with the current reference meanwhile and
-//     recomputed only when the reference moves. P goes to a swizzled K-major shared
-//     tile in the query's 16-bit type; the running sum adds the binary32 values;
+//   * one persistent CTA per SM runs two independent pipelines ("sets") that share the
+//     tensor core: each set takes its own units from the global queue and has its own
+//     Q, K and V buffers in shared memory and its own S and O accumulators in TMEM
+//     (S of set c in columns [128 c, 128 c + 128), O in [256 + 128 c, ...)). While one
+//     set's softmax works on its scores, the tensor core runs the other set's MMAs;
+//   * warps: 4 softmax warps per set (thread = one row of the tile, all 128 columns, so
+//     no two warps ever combine a row), one MMA-issue warp for both sets, and one
+//     producer warp per set that takes its units, loads Q (one 3-D TMA box per 64-dim
+//     half: 64 dims x G heads x 128 / G queries) and streams K and V tiles (2-D TMA,
+//     one box per (cache block, 64-dim half), 128B swizzle, no multicast);
+//   * S = Q K^T (both operands K-major in shared memory). The softmax writes P over its
+//     own scores in TMEM as 16-bit pairs, and O += P V takes P from TMEM (A operand)
+//     and V in its [token][dim] cache layout (MN-major B operand). Per set the issue
+//     order is S(g), P(g) V(g), S(g + 1) (which waits for P(g) V(g): it overwrites the
+//     P it reads); the MMA warp alternates S(set 0), S(set 1), P V(set 0), P V(set 1);
+//   * the softmax keeps a reference maximum that moves only when the row maximum passes
+//     it by more than 2^8 (O and the running sum are then rescaled; every p stays below
+//     2^8). For bf16, p rounded to bf16 can leave the parity tolerance when a few
+//     weights dominate and their V values cancel, so the rounded remainder
+//     p - bf16(p) goes into the other 64 columns of S and a second P V product adds it
+//     (hi + lo carries p to within 2^-16): for every tile, or only for tiles where some
+//     row has a weight above 1/8 of its running sum (a later tile can only lower that
+//     share, so every unadjusted weight ends below 1/8 of the row's total);
 //   * a unit that covers a row's whole context writes the output row; otherwise it
 //     writes (max, sum, unnormalised row) for the log-sum-exp merge kernel.
 // Every wait is bounded; on a timeout the kernel records it, every role stops, the MMA
 // and load issuers drain what they issued, and the TMEM is freed.
+#include <cstdlib>
+#include <cstring>
+
 namespace pa {
 
 constexpr int kTcRows = 128;            // query rows per unit (TMEM lanes)
 constexpr int kTcTok = 128;             // tokens per K/V tile
 constexpr int kTcD = 128;               // head_dim of this path
-constexpr uint32_t kTcTmemCols = 512;   // S double buffer [0, 256), O double buffer [256, 512)
-constexpr int kTcSplit = 2;             // softmax warps per 32-row group (column slices)
-constexpr int kTcSoftmaxWarps = 4 * kTcSplit;   // + an MMA-issue warp + K and V producer warps
-constexpr int kTcThreads = (kTcSoftmaxWarps + 3) * 32;
+constexpr uint32_t kTcTmemCols = 512;   // S of the two sets in [0, 256), their O in [256, 512)
+constexpr int kTcSets = 2;              // independent pipelines sharing the tensor core
+constexpr int kTcSetWarps = 4;          // softmax warps per set: one thread per row
+constexpr int kTcSoftmaxWarps = kTcSets * kTcSetWarps;
+constexpr int kTcMmaWarp = kTcSoftmaxWarps;           // followed by one producer warp per set
+constexpr int kTcThreads = (kTcSoftmaxWarps + 1 + kTcSets) * 32;
 constexpr float kTcRescale = 8.f;       // log2 units
+constexpr float kTcLoShare = 0.125f;    // adaptive remainder: a weight above this share of the running sum
+
+// P V precision modes (ExtendParams::lo_mode)
+constexpr int kLoNone = 0;      // P rounded to the 16-bit type only (f16: rounding up to 2^-11 of p)
+constexpr int kLoAlways = 1;    // the bf16 remainder for every tile
+constexpr int kLoAdaptive = 2;  // the bf16 remainder for tiles with a weight above kTcLoShare
 
 struct TcSmem {
   static constexpr int kTile = kTcRows * kTcD * 2;   // 32 KB: two 64-column halves of 16 KB
-  static constexpr int kQ = 0;
-  static constexpr int kP = kQ + kTile;              // P buffers 0, 1
-  static constexpr int kK = kP + 2 * kTile;          // K buffers 0, 1
-  static constexpr int kV = kK + 2 * kTile;          // V buffers 0, 1
-  static constexpr int kBytes = kV + 2 * kTile + 1024;   // 225 KB with the alignment slack
+  static constexpr int kQ = 0, kK = kTile, kV = 2 * kTile;
+  static constexpr int kSet = 3 * kTile;             // Q, K and V of one set
+  static constexpr int kBytes = kTcSets * kSet + 1024;   // 193 KB with the alignment slack
 };
-static_assert(kTcRows == kTcTok, "Q, P, K and V tiles share one swizzled layout");
+static_assert(kTcRows == kTcTok, "Q, K and V tiles share one swizzled layout");
 
 // Shared-memory matrix descriptor: 128B swizzle, sm_100 descriptor version.
 __device__ __forceinline__ uint64_t tc_desc(uint32_t saddr, uint32_t sbo, uint32_t lbo) {
@@ -144,23 +154,6 @@ __device__ __forceinline__ void tc_st32(uint32_t addr, const float* v) {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-// Two values rounded to the 16-bit type and packed (lo in the low half); `sum` adds the
-// rounded values.
-template <int QD>
-__device__ __forceinline__ uint32_t pack2_sum(float lo, float hi, float& sum) {
-  if constexpr (QD == PA_BF16) {
-    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-    const uint32_t w = *reinterpret_cast<const uint32_t*>(&v);
-    sum += __uint_as_float(w << 16) + __uint_as_float(w & 0xffff0000u);
-    return w;
-  } else {
-    __half2 v = __floats2half2_rn(lo, hi);
-    const float2 f = __half22float2(v);
-    sum += f.x + f.y;
-    return *reinterpret_cast<const uint32_t*>(&v);
-  }
-}
-
 // max(a, b, c) in one instruction (sm_100 three-input max; a NaN operand is ignored as by fmaxf).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;
@@ -173,18 +166,6 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
-}
-
-// One 32-bit column of this warp's 32 lanes (warp-collective), with its wait.
-__device__ __forceinline__ void tc_st1(uint32_t addr, uint32_t v) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(addr), "r"(v) : "memory");
-  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ uint32_t tc_ld1(uint32_t addr) {
-  uint32_t v;
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(v) : "r"(addr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-  return pin_after_wait(v);
 }
 
 // Packed binary32 pairs (sm_100 f32x2 arithmetic): a * b + c and a + b, lane-wise.
@@ -203,24 +184,6 @@ __device__ __forceinline__ float2 add2(float2 a, float2 b) {
       : "=f"(d.x), "=f"(d.y)
       : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
   return d;
-}
-
-// p = 2^a for a pair, rounded to the 16-bit type and packed (lo in the low half); the
-// binary32 values are added to `sum` as a pair (the weights in P differ from them by at
-// most one 16-bit rounding each).
-template <int QD>
-__device__ __forceinline__ uint32_t exp2_pack(float2 a, float2& sum) {
-  const float p0 = ex2(a.x), p1 = ex2(a.y);
-  uint32_t w;
-  if constexpr (QD == PA_BF16) {
-    __nv_bfloat162 v = __floats2bfloat162_rn(p0, p1);
-    w = *reinterpret_cast<const uint32_t*>(&v);
-  } else {
-    __half2 v = __floats2half2_rn(p0, p1);
-    w = *reinterpret_cast<const uint32_t*>(&v);
-  }
-  sum = add2(sum, make_float2(p0, p1));
-  return w;
 }
 
 // 3-D tiled TMA load.
@@ -293,8 +256,114 @@ __device__ __forceinline__ bool tc_wait_warp(uint64_t* bar, uint32_t parity, vol
   return __all_sync(kFull, tc_wait(bar, parity, abort, where, u));
 }
 
+
+// O += P V with P (the A operand) in TMEM: M = 128 lanes, K = 16 per instruction (8
+// columns of bf16 / f16 pairs), B from shared memory.
+__device__ __forceinline__ void tc_mma_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
+// 16 consecutive 32-bit columns of this warp's 32 lanes, without the wait (the registers
+// are read at issue; one tc_wait_st() orders all of them before the next barrier).
+__device__ __forceinline__ void tc_st16(uint32_t addr, const uint32_t* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          addr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+__device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Two values rounded to the 16-bit type and packed (lo in the low half).
+template <int QD>
+__device__ __forceinline__ uint32_t pack16x2(float lo, float hi) {
+  if constexpr (QD == PA_BF16) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&v);
+  } else {
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&v);
+  }
+}
+
+// The binary32 values of a packed bf16 pair (bf16 is the upper half of a binary32).
+__device__ __forceinline__ float2 bf16x2_value(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+// Pass 1 of the softmax: the maximum of one row's 128 scores in TMEM (this thread's lane),
+// columns past `vis` masked when kMask.
+template <bool kMask>
+__device__ __forceinline__ float tc_row_max(uint32_t addr, int vis) {
+  uint32_t r[kTcTok];
+#pragma unroll
+  for (int i = 0; i < kTcTok / 32; ++i) tc_ld32_async(addr + i * 32, r + i * 32);
+  tc_wait_ld();
+  auto at = [&](int i) {
+    const float v = __uint_as_float(pin_after_wait(r[i]));
+    return kMask && i > vis ? -INFINITY : v;
+  };
+  float m8[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) m8[e] = at(e);
+#pragma unroll
+  for (int i = 8; i + 8 < kTcTok; i += 16)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) m8[e] = fmax3(m8[e], at(i + e), at(i + 8 + e));
+  if constexpr ((kTcTok - 8) % 16 != 0) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) m8[e] = fmaxf(m8[e], at(kTcTok - 8 + e));
+  }
+  return fmaxf(fmax3(m8[0], m8[1], m8[2]), fmax3(fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7]));
+}
+
+// Pass 2 of the softmax, 32 columns at a time: p = 2^(s * s_mul + nmb) of one row's 128
+// scores, written over them as 16-bit pairs (the 32 tokens of chunk q: P in columns
+// [32 q, 32 q + 16); with kLo the rounded remainder p - bf16(p) in [32 q + 16, 32 q + 32));
+// the binary32 p are added to l2 (four pair chains).
+template <int QD, bool kMask, bool kLo>
+__device__ __forceinline__ void tc_make_p(uint32_t addr, int vis, float s_mul, float nmb, float2 (&l2)[4]) {
+#pragma unroll
+  for (int q = 0; q < kTcTok / 32; ++q) {
+    uint32_t r[32];
+    tc_ld32_async(addr + q * 32, r);
+    tc_wait_ld();
+    uint32_t wh[16], wl[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const int col = q * 32 + 2 * e;
+      float s0 = __uint_as_float(pin_after_wait(r[2 * e]));
+      float s1 = __uint_as_float(pin_after_wait(r[2 * e + 1]));
+      if (kMask) {
+        s0 = col > vis ? -INFINITY : s0;
+        s1 = col + 1 > vis ? -INFINITY : s1;
+      }
+      const float2 a = fma2(make_float2(s0, s1), s_mul, nmb);
+      const float p0 = ex2(a.x), p1 = ex2(a.y);
+      wh[e] = pack16x2<QD>(p0, p1);
+      l2[e & 3] = add2(l2[e & 3], make_float2(p0, p1));
+      if constexpr (kLo) {
+        const float2 hv = bf16x2_value(wh[e]);
+        wl[e] = pack16x2<QD>(p0 - hv.x, p1 - hv.y);
+      }
+    }
+    tc_st16(addr + q * 32, wh);
+    if constexpr (kLo) tc_st16(addr + q * 32 + 16, wl);
+  }
+}
+
+// 184 registers x 352 threads = 64768 of the SM's 65536: one CTA per SM (a bound of 352
+// threads would let the compiler assume 384 and stop at 168, spilling the softmax rows).
+constexpr int kTcMaxRegs = 184;
+static_assert(kTcMaxRegs * kTcThreads <= 65536, "the register file holds one CTA");
+
 template <int QD, int BS, int G>
-__global__ void __launch_bounds__(kTcThreads, 1)
+__global__ void __maxnreg__(kTcMaxRegs)
     extend_tc_kernel(const ExtendParams p, const __grid_constant__ CUtensorMap tk,
                      const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tq,
                      const __grid_constant__ CUtensorMap tkn, const __grid_constant__ CUtensorMap tvn) {
@@ -304,12 +373,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   constexpr uint32_t kBlockTx = BS * kTcD * 2;        // bytes of one cache block of K (or V)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = sm + TcSmem::kQ;
-  // per-tile ring barriers (index = tile & 1); per-unit ones (q_full, o_full/o_empty by unit & 1)
-  __shared__ uint64_t k_full[2], v_full[2], k_empty[2], pv_done[2], s_full[2], s_empty[2], p_full[2];
-  __shared__ uint64_t q_full, q_empty, o_full[2], o_empty[2], bar_fin, grp_bar[4];
-  __shared__ int uq[4];                        // unit ring: unit k of this CTA in slot k % 4
-  __shared__ uint64_t uq_full[4], uq_empty[4];
+  // per set: S(g) landed, P(g) written (one arrival per softmax warp), P(g) V(g) done;
+  // K(g) / V(g) landed, K buffer free; Q of unit k landed / free; O of unit k complete /
+  // read (one arrival per softmax warp); the unit ring
+  __shared__ uint64_t s_full[kTcSets], p_full[kTcSets], pv_done[kTcSets], k_full[kTcSets], v_full[kTcSets];
+  __shared__ uint64_t k_empty[kTcSets], q_full[kTcSets], q_empty[kTcSets], o_full[kTcSets], o_empty[kTcSets];
+  __shared__ uint64_t uq_full[kTcSets][4], uq_empty[kTcSets][4], bar_fin;
+  __shared__ int uq[kTcSets][4];               // unit k of set c in slot k % 4
+  __shared__ int lo_tile[kTcSets];             // adaptive remainder: the set's latest tile that needs it
   __shared__ uint32_t tmem_slot;
   __shared__ int s_abort;
   volatile int* abort = &s_abort;
@@ -322,24 +393,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
   if (tid == 32) {
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&k_full[b], 1);
-      mbar_init(&v_full[b], 1);
-      mbar_init(&k_empty[b], 1);
-      mbar_init(&pv_done[b], 1);
-      mbar_init(&s_full[b], 1);
-      mbar_init(&s_empty[b], kTcSoftmaxWarps);
-      mbar_init(&p_full[b], kTcSoftmaxWarps);
-      mbar_init(&o_full[b], 1);
-      mbar_init(&o_empty[b], kTcSoftmaxWarps);
+    for (int c = 0; c < kTcSets; ++c) {
+      mbar_init(&s_full[c], 1);
+      mbar_init(&p_full[c], kTcSetWarps);
+      mbar_init(&pv_done[c], 1);
+      mbar_init(&k_full[c], 1);
+      mbar_init(&v_full[c], 1);
+      mbar_init(&k_empty[c], 1);
+      mbar_init(&q_full[c], 1);
+      mbar_init(&q_empty[c], 1);
+      mbar_init(&o_full[c], 1);
+      mbar_init(&o_empty[c], kTcSetWarps);
+      for (int i = 0; i < 4; ++i) {
+        mbar_init(&uq_full[c][i], 1);
+        mbar_init(&uq_empty[c][i], kTcSetWarps + 1);   // the set's softmax warps and the MMA warp
+      }
+      lo_tile[c] = -1;
     }
-    mbar_init(&q_full, 1);
-    mbar_init(&q_empty, 1);
-    for (int i = 0; i < 4; ++i) {
-      mbar_init(&uq_full[i], 1);
-      mbar_init(&uq_empty[i], kTcSoftmaxWarps + 2);   // V producer, MMA warp, softmax warps
-    }
-    for (int i = 0; i < 4; ++i) mbar_init(&grp_bar[i], kTcSplit);
     mbar_init(&bar_fin, 1);
     s_abort = 0;
     fence_mbar_init();
@@ -353,72 +423,55 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t tmem = tmem_slot;
   const int Hq = p.num_q_heads, Hkv = p.num_kv_heads;
   const int total = p.plan[p.num_seqs] * Hkv;
-  uint32_t last_load = 0;           // producer: tiles issued (for the drain after an abort)
-  uint32_t q_loads = 0;             // V producer: Q tiles issued (likewise)
-  // Dynamic scheduling: the K producer takes unit k of this CTA from the global queue (the
-  // plan kernel lists each sequence's longest row tile first) and publishes it in the
-  // ring; every other role reads the same sequence. -1 ends the work. False on an abort.
-  auto next_unit = [&](uint32_t k, bool taker, int& u) -> bool {
+  uint32_t k_loads = 0, v_loads = 0, q_loads = 0;   // producer: loads issued (for the drain after an abort)
+
+  // Dynamic scheduling: each set's producer takes the set's unit k from the global queue
+  // (the plan kernel lists each sequence's longest row tile first) and publishes it in
+  // the set's ring; the set's softmax warps and the MMA warp read the same sequence. -1
+  // ends the set's work. False on an abort.
+  auto next_unit = [&](int c, uint32_t k, bool taker, int& u) -> bool {
     const int slot = k & 3;
     const uint32_t ph = (k >> 2) & 1;
     if (taker) {
-      if (!tc_wait_warp(&uq_empty[slot], ph ^ 1, abort, 28, int(k))) return false;
+      if (!tc_wait_warp(&uq_empty[c][slot], ph ^ 1, abort, 28, int(k))) return false;
       int v = 0;
       if (lane == 0) {
         v = atomicAdd(p.queue, 1);
         if (v >= total) v = -1;
-        uq[slot] = v;
-        mbar_arrive(&uq_full[slot]);
+        uq[c][slot] = v;
+        mbar_arrive(&uq_full[c][slot]);
       }
       u = __shfl_sync(kFull, v, 0);
       return true;
     }
-    if (!tc_wait_warp(&uq_full[slot], ph, abort, 29, int(k))) return false;
-    u = *reinterpret_cast<volatile int*>(&uq[slot]);
+    if (!tc_wait_warp(&uq_full[c][slot], ph, abort, 29, int(k))) return false;
+    u = *reinterpret_cast<volatile int*>(&uq[c][slot]);
     __syncwarp();
-    if (lane == 0) mbar_arrive(&uq_empty[slot]);
+    if (lane == 0) mbar_arrive(&uq_empty[c][slot]);
     return true;
   };
 
-  if (warp > kTcSoftmaxWarps) {
-    // ---------------- producers: warp kTcSoftmaxWarps + 1 streams K, the next one V, by 2-D
-    // TMA, lane i loading cache block i of a tile; separate warps, so that a K tile never
-    // waits behind the V tile before it (which waits for an older P V) ----------------
-    const bool is_v = warp == kTcSoftmaxWarps + 2;
-    uint64_t* full = is_v ? v_full : k_full;
-    uint64_t* empty = is_v ? pv_done : k_empty;   // V(g) after P(g-2) V(g-2); K(g) after S(g-2)
-    const CUtensorMap* map = is_v ? &tv : &tk;
-    uint8_t* ring = sm + (is_v ? TcSmem::kV : TcSmem::kK);
-    const CUtensorMap* in_map = is_v ? &tvn : &tkn;   // whole prompts: the prompt's K or V rows
-    int pend_g = -1, pend_nbw = 0, pend_y = 0;        // a loaded tile still to be written to the cache
-    auto flush_store = [&]() {
-      if (pend_g < 0) return true;
-      const int b = pend_g & 1;
-      if (!tc_wait_warp(&full[b], (uint32_t(pend_g) >> 1) & 1, abort, 27, pend_g)) return false;
-      if (lane < pend_nbw) {
-        const uint8_t* src = ring + b * TcSmem::kTile + lane * (BS * 128);
-        tma_store_2d(map, 0, pend_y, src);
-        tma_store_2d(map, 64, pend_y, src + kTcTok * 128);
-        bulk_commit();
-      }
-      pend_g = -1;
-      return true;
-    };
+  if (warp > kTcMmaWarp) {
+    // ---------------- producer of set c: its units, their Q, K and V tiles ----------------
+    const int c = warp - kTcMmaWarp - 1;
+    uint8_t* sQ = sm + c * TcSmem::kSet + TcSmem::kQ;
+    uint8_t* sK = sm + c * TcSmem::kSet + TcSmem::kK;
+    uint8_t* sV = sm + c * TcSmem::kSet + TcSmem::kV;
     uint32_t g = 0;
-    for (uint32_t k = 0;; ++k) {
+    bool ok = true;
+    for (uint32_t k = 0; ok; ++k) {
       int u;
-      if (!next_unit(k, !is_v, u) || u < 0) break;
+      if (!(ok = next_unit(c, k, true, u)) || u < 0) break;
       const TcUnit x = tc_unit(p, u);
-      if (is_v) {   // the unit's q rows: box {64 dims, G heads, QPT queries} per 64-dim half
-        if (k > 0 && !tc_wait_warp(&q_empty, (k - 1) & 1, abort, 26, u)) break;
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&q_full, TcSmem::kTile);
-          tma_load_3d(sQ, &tq, 0, x.hk * G, x.row0 + x.t * QPT, &q_full);
-          tma_load_3d(sQ + kTcRows * 128, &tq, 64, x.hk * G, x.row0 + x.t * QPT, &q_full);
-        }
-        __syncwarp();
-        q_loads = k + 1;
+      // the unit's q rows, once the last S of the set's previous unit has read the buffer
+      if (!(ok = tc_wait_warp(&q_empty[c], (k & 1) ^ 1, abort, 26, u))) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&q_full[c], TcSmem::kTile);
+        tma_load_3d(sQ, &tq, 0, x.hk * G, x.row0 + x.t * QPT, &q_full[c]);
+        tma_load_3d(sQ + kTcRows * 128, &tq, 64, x.hk * G, x.row0 + x.t * QPT, &q_full[c]);
       }
+      __syncwarp();
+      q_loads = k + 1;
       const int32_t* trow = p.block_tables + size_t(x.s) * p.max_blocks;
       auto blocks = [&](int j) { return min(BPT, (x.nvis - j * kTcTok + BS - 1) / BS); };
       auto fetch = [&](int lb, int n) {   // block id of this lane's block (lane < n), checked
@@ -426,214 +479,192 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (lane < n) {
           id = trow[lb + lane];
           if (id < 0 || id >= p.num_blocks) {
-            if (!is_v) record_error(PA_DEV_BAD_BLOCK_ID, x.s, lb + lane, id);
+            record_error(PA_DEV_BAD_BLOCK_ID, x.s, lb + lane, id);
             id = 0;
           }
         }
         return id;
       };
-      if (p.fresh) {
-        // whole prompts: tiles come from the prompt's own K / V rows, 128 rows per box;
-        // the row tile that sees all of a K/V tile's prompt positions also writes that
-        // tile into its cache blocks (TMA stores, once its load has landed)
-        bool ok = true;
-        for (int j = 0; j < x.ntiles; ++j, ++g) {
-          const int b = g & 1, p0 = x.t0 + j * kTcTok;
-          if (!(ok = tc_wait_warp(&empty[b], ((g >> 1) & 1) ^ 1, abort, is_v ? 11 : 10, u))) break;
-          bulk_wait_read_all();   // the stores that read this buffer two tiles ago
+      for (int j = 0; j < x.ntiles; ++j, ++g) {
+        const int p0 = x.t0 + j * kTcTok;
+        const int nb = blocks(j);
+        const int id = p.fresh ? 0 : fetch(p0 / BS, nb);
+        // K(g) once S(g-1) has read the buffer (and, for whole prompts, once the cache
+        // stores of the previous tile have read both buffers)
+        if (!(ok = tc_wait_warp(&k_empty[c], (g & 1) ^ 1, abort, 10, u))) break;
+        if (p.fresh) bulk_wait_read_all();
+        __syncwarp();
+        if (p.fresh) {   // whole prompts: the prompt's own rows, 128 per box
           if (lane == 0) {
-            mbar_arrive_expect_tx(&full[b], TcSmem::kTile);
-            tma_load_3d(ring + b * TcSmem::kTile, in_map, 0, x.hk, x.row0 + p0, &full[b]);
-            tma_load_3d(ring + b * TcSmem::kTile + kTcTok * 128, in_map, 64, x.hk, x.row0 + p0, &full[b]);
+            mbar_arrive_expect_tx(&k_full[c], TcSmem::kTile);
+            tma_load_3d(sK, &tkn, 0, x.hk, x.row0 + p0, &k_full[c]);
+            tma_load_3d(sK + kTcTok * 128, &tkn, 64, x.hk, x.row0 + p0, &k_full[c]);
+          }
+        } else {
+          if (lane == 0) mbar_arrive_expect_tx(&k_full[c], uint32_t(nb) * kBlockTx);
+          __syncwarp();
+          if (lane < nb) {
+            const int y = (id * Hkv + x.hk) * BS;
+            tma_load_2d(sK + lane * (BS * 128), &tk, 0, y, &k_full[c]);
+            tma_load_2d(sK + kTcTok * 128 + lane * (BS * 128), &tk, 64, y, &k_full[c]);
+          }
+        }
+        __syncwarp();
+        k_loads = g + 1;
+        // V(g) once P(g-1) V(g-1) has read the buffer
+        if (!(ok = tc_wait_warp(&pv_done[c], (g & 1) ^ 1, abort, 11, u))) break;
+        if (p.fresh) {
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&v_full[c], TcSmem::kTile);
+            tma_load_3d(sV, &tvn, 0, x.hk, x.row0 + p0, &v_full[c]);
+            tma_load_3d(sV + kTcTok * 128, &tvn, 64, x.hk, x.row0 + p0, &v_full[c]);
+          }
+        } else {
+          if (lane == 0) mbar_arrive_expect_tx(&v_full[c], uint32_t(nb) * kBlockTx);
+          __syncwarp();
+          if (lane < nb) {
+            const int y = (id * Hkv + x.hk) * BS;
+            tma_load_2d(sV + lane * (BS * 128), &tv, 0, y, &v_full[c]);
+            tma_load_2d(sV + kTcTok * 128 + lane * (BS * 128), &tv, 64, y, &v_full[c]);
+          }
+        }
+        __syncwarp();
+        v_loads = g + 1;
+        // whole prompts: the row tile that sees every prompt position of this K/V tile
+        // writes the tile into its cache blocks, once both loads have landed
+        if (p.fresh && x.t == min((p0 + kTcTok - 1) / QPT, (x.Q - 1) / QPT)) {
+          if (!(ok = tc_wait_warp(&k_full[c], g & 1, abort, 27, u) && tc_wait_warp(&v_full[c], g & 1, abort, 27, u)))
+            break;
+          const int nbw = (min(p0 + kTcTok, x.Q) - p0 + BS - 1) / BS;
+          const int idw = fetch(p0 / BS, nbw);
+          if (lane < nbw) {
+            const int y = (idw * Hkv + x.hk) * BS;
+            tma_store_2d(&tk, 0, y, sK + lane * (BS * 128));
+            tma_store_2d(&tk, 64, y, sK + kTcTok * 128 + lane * (BS * 128));
+            tma_store_2d(&tv, 0, y, sV + lane * (BS * 128));
+            tma_store_2d(&tv, 64, y, sV + kTcTok * 128 + lane * (BS * 128));
+            bulk_commit();
           }
           __syncwarp();
-          last_load = g + 1;
-          if (!(ok = flush_store())) break;
-          if (x.t == min((p0 + kTcTok - 1) / QPT, (x.Q - 1) / QPT)) {
-            pend_nbw = (min(p0 + kTcTok, x.Q) - p0 + BS - 1) / BS;
-            pend_y = (fetch(p0 / BS, pend_nbw) * Hkv + x.hk) * BS;
-            pend_g = int(g);
-          }
         }
-        if (!ok) break;
-        continue;
-      }
-      int id = fetch(x.t0 / BS, blocks(0));
-      for (int j = 0; j < x.ntiles; ++j, ++g) {
-        const int b = g & 1, nb = blocks(j);
-        const int next = j + 1 < x.ntiles ? fetch((x.t0 + (j + 1) * kTcTok) / BS, blocks(j + 1)) : 0;
-        const int y = (id * Hkv + x.hk) * BS;
-        uint8_t* dst = ring + b * TcSmem::kTile + lane * (BS * 128);
-        if (!tc_wait_warp(&empty[b], ((g >> 1) & 1) ^ 1, abort, is_v ? 11 : 10, u)) break;
-        if (lane == 0) mbar_arrive_expect_tx(&full[b], uint32_t(nb) * kBlockTx);
-        __syncwarp();
-        if (lane < nb) {
-          tma_load_2d(dst, map, 0, y, &full[b]);
-          tma_load_2d(dst + kTcTok * 128, map, 64, y, &full[b]);
-        }
-        last_load = g + 1;
-        id = next;
       }
     }
-    if (p.fresh && !*abort) flush_store();
     bulk_wait_all();   // this thread's cache stores are complete before the kernel ends
-  } else if (warp == kTcSoftmaxWarps) {
-    // ---------------- MMA issue: S(g) then O += P(g-1) V(g-1) ----------------
+  } else if (warp == kTcMmaWarp) {
+    // ---------------- MMA issue for both sets: S(0), S(1), P V(0), P V(1), ... ----------------
     const uint32_t idS = tc_idesc<QD>(0), idO = tc_idesc<QD>(1);
-    uint32_t g = 0, k = 0;
-    auto pv = [&](uint32_t h, bool first, uint32_t ob, int u) {
-      const int b = h & 1;
-      if (!tc_wait_warp(&p_full[b], (h >> 1) & 1, abort, 12, u)) return false;
-      if (!tc_wait_warp(&v_full[b], (h >> 1) & 1, abort, 13, u)) return false;
-      if (lane == 0) {
-        tc_fence_after();
-        const uint32_t pa_ = smem_addr(sm + TcSmem::kP + b * TcSmem::kTile);
-        const uint32_t va = smem_addr(sm + TcSmem::kV + b * TcSmem::kTile);
+    TcUnit x[kTcSets];
+    int j[kTcSets];
+    uint32_t g[kTcSets], k[kTcSets];
+    bool live[kTcSets], fresh_unit[kTcSets];
 #pragma unroll
-        for (int kk = 0; kk < kTcTok / 16; ++kk) {
-          const uint32_t aoff = (kk >> 2) * (kTcRows * 128) + (kk & 3) * 32;
-          tc_mma(tmem + 256 + ob * 128, tc_desc(pa_ + aoff, 1024, 16), tc_desc(va + kk * 2048, 1024, kTcTok * 128),
-                 idO, (first && kk == 0) ? 0u : 1u);
+    for (int c = 0; c < kTcSets; ++c) {
+      j[c] = 0;
+      g[c] = k[c] = 0;
+      live[c] = fresh_unit[c] = true;
+    }
+    bool ok = true;
+    while (ok && (live[0] || live[1])) {
+      bool pend[kTcSets] = {false, false};
+#pragma unroll
+      for (int c = 0; c < kTcSets; ++c) {
+        if (!ok || !live[c]) continue;
+        if (fresh_unit[c]) {
+          int u;
+          if (!(ok = next_unit(c, k[c], false, u))) break;
+          if (u < 0) {
+            live[c] = false;
+            continue;
+          }
+          x[c] = tc_unit(p, u);
+          j[c] = 0;
+          fresh_unit[c] = false;
+          if (!(ok = tc_wait_warp(&q_full[c], k[c] & 1, abort, 14, u))) break;
         }
-        tc_commit(&pv_done[b]);
-      }
-      __syncwarp();
-      return true;
-    };
-    for (;; ++k) {
-      int u;
-      if (!next_unit(k, false, u) || u < 0) break;
-      const TcUnit x = tc_unit(p, u);
-      const uint32_t ob = k & 1;
-      if (!tc_wait_warp(&q_full, k & 1, abort, 14, u)) break;
-      if (!tc_wait_warp(&o_empty[ob], ((k >> 1) & 1) ^ 1, abort, 15, u)) break;
-      bool ok = true;
-      for (int j = 0; j < x.ntiles && ok; ++j, ++g) {
-        const int b = g & 1;
-        ok = tc_wait_warp(&k_full[b], (g >> 1) & 1, abort, 16, u) &&
-             tc_wait_warp(&s_empty[b], ((g >> 1) & 1) ^ 1, abort, 17, u);
-        if (!ok) break;
+        // S(g) = Q K(g)^T into the set's S columns, once K(g) has landed and P(g-1) V(g-1)
+        // (which reads P from those columns) has completed
+        if (!(ok = tc_wait_warp(&k_full[c], g[c] & 1, abort, 16, int(g[c])) &&
+                   tc_wait_warp(&pv_done[c], (g[c] & 1) ^ 1, abort, 17, int(g[c]))))
+          break;
         if (lane == 0) {
           tc_fence_after();
-          const uint32_t qa = smem_addr(sQ), ka = smem_addr(sm + TcSmem::kK + b * TcSmem::kTile);
+          const uint32_t qa = smem_addr(sm + c * TcSmem::kSet + TcSmem::kQ);
+          const uint32_t ka = smem_addr(sm + c * TcSmem::kSet + TcSmem::kK);
 #pragma unroll
           for (int kk = 0; kk < kTcD / 16; ++kk) {
             const uint32_t off = (kk >> 2) * (kTcRows * 128) + (kk & 3) * 32;
-            tc_mma(tmem + b * 128, tc_desc(qa + off, 1024, 16), tc_desc(ka + off, 1024, 16), idS, kk > 0);
+            tc_mma(tmem + c * 128, tc_desc(qa + off, 1024, 16), tc_desc(ka + off, 1024, 16), idS, kk > 0);
           }
-          tc_commit(&s_full[b]);
-          tc_commit(&k_empty[b]);
-          if (j + 1 == x.ntiles) tc_commit(&q_empty);   // sQ is free once this S completes
+          tc_commit(&s_full[c]);
+          tc_commit(&k_empty[c]);
+          if (j[c] + 1 == x[c].ntiles) tc_commit(&q_empty[c]);   // the Q buffer is free once this S completes
         }
         __syncwarp();
-        if (j > 0) ok = pv(g - 1, j == 1, ob, u);
+        pend[c] = true;
       }
-      if (!ok || !pv(g - 1, x.ntiles == 1, ob, u)) break;
-      if (lane == 0) tc_commit(&o_full[ob]);
-      __syncwarp();
+#pragma unroll
+      for (int c = 0; c < kTcSets; ++c) {
+        if (!ok || !pend[c]) continue;
+        // O += P(g) V(g) (+ the remainder), once P is in TMEM and V(g) has landed; a unit's
+        // first product overwrites O, so it waits until the previous unit's O was read
+        if (!(ok = tc_wait_warp(&p_full[c], g[c] & 1, abort, 12, int(g[c])) &&
+                   tc_wait_warp(&v_full[c], g[c] & 1, abort, 13, int(g[c]))))
+          break;
+        if (j[c] == 0 && k[c] > 0 && !(ok = tc_wait_warp(&o_empty[c], (k[c] & 1) ^ 1, abort, 15, int(k[c])))) break;
+        const bool lo = p.lo_mode == kLoAlways ||
+                        (p.lo_mode == kLoAdaptive && *reinterpret_cast<volatile int*>(&lo_tile[c]) == int(g[c]));
+        if (lane == 0) {
+          tc_fence_after();
+          const uint32_t va = smem_addr(sm + c * TcSmem::kSet + TcSmem::kV);
+          const uint32_t d = tmem + 256 + c * 128, a = tmem + c * 128;
+#pragma unroll
+          for (int kk = 0; kk < kTcTok / 16; ++kk)   // P of tokens 16 kk .. 16 kk + 15
+            tc_mma_ts(d, a + 32 * (kk >> 1) + 8 * (kk & 1), tc_desc(va + kk * 2048, 1024, kTcTok * 128), idO,
+                      (j[c] > 0 || kk > 0) ? 1u : 0u);
+          if (lo) {
+#pragma unroll
+            for (int kk = 0; kk < kTcTok / 16; ++kk)   // their remainders, 16 columns further
+              tc_mma_ts(d, a + 32 * (kk >> 1) + 8 * (kk & 1) + 16, tc_desc(va + kk * 2048, 1024, kTcTok * 128), idO,
+                        1u);
+          }
+          tc_commit(&pv_done[c]);
+          if (j[c] + 1 == x[c].ntiles) tc_commit(&o_full[c]);
+        }
+        __syncwarp();
+        ++g[c];
+        if (++j[c] == x[c].ntiles) {
+          fresh_unit[c] = true;
+          ++k[c];
+        }
+      }
     }
   } else {
-    // ---------------- softmax warps ----------------
-    // Warps w, w + 4, w + 8, ... share TMEM lanes 32 (w % 4) .. + 31 (rows of the tile) and
-    // split the columns: slice q = w / 4 holds score / P / O columns [kCW q, kCW q + kCW).
-    // The group combines its row maxima and sums through one TMEM column each has already
-    // read (its own first column of the S or O buffer) and a kTcSplit-arrival mbarrier.
-    constexpr int kCW = kTcTok / kTcSplit;             // columns per warp
-    const int qs_ = warp >> 2, rw = warp & 3, row = rw * 32 + lane;
+    // ---------------- softmax warps: set c, rows 32 rw .. 32 rw + 31 of the tile ----------------
+    const int c = warp / kTcSetWarps, rw = warp % kTcSetWarps, row = rw * 32 + lane;
     const uint32_t t_row = tmem + (uint32_t(rw * 32) << 16);
-    uint32_t xc = 0;   // group exchanges so far
-    auto publish = [&](uint32_t col_own, float v) {
-      tc_st1(t_row + col_own, __float_as_uint(v));
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&grp_bar[rw]);
-    };
-    // all slices' values in slice order (identical in every warp of the group)
-    auto gather = [&](uint32_t col0, float own, int u, float* all) {
-      const bool ok = tc_wait_warp(&grp_bar[rw], xc & 1, abort, 23, u);
-      ++xc;
-      if (!ok) return false;
-      tc_fence_after();
-#pragma unroll
-      for (int q = 0; q < kTcSplit; ++q)
-        all[q] = q == qs_ ? own : __uint_as_float(tc_ld1(t_row + col0 + q * kCW));
-      return true;
-    };
-    uint32_t g = 0, k = 0;
-    for (;; ++k) {
+    const uint32_t c_s = c * 128, c_o = 256 + c * 128;
+    uint8_t* sV = sm + c * TcSmem::kSet + TcSmem::kV;
+    uint32_t g = 0;
+    for (uint32_t k = 0;; ++k) {
       int u;
-      if (!next_unit(k, false, u) || u < 0) break;
+      if (!next_unit(c, k, false, u) || u < 0) break;
       const TcUnit x = tc_unit(p, u);
-      const uint32_t ob = k & 1, c_o = 256 + ob * 128 + qs_ * kCW;   // this slice of the O buffer
       const int qi = x.t * QPT + row / G;
       const int head = x.hk * G + row % G;
       const bool has_q = qi < x.Q;
       const int qpos = has_q ? x.base + qi : -1;
       const int tok = has_q ? x.row0 + qi : -1;
-      float m_ref = -INFINITY, l = 0.f;   // l: this slice's share of the row sum
+      float m_ref = -INFINITY, l = 0.f;
       bool ok = true;
       for (int j = 0; j < x.ntiles; ++j, ++g) {
-        const int b = g & 1;
-        const uint32_t c_s = b * 128 + qs_ * kCW;                    // this slice of S(g)
-        if (!(ok = tc_wait_warp(&s_full[b], (g >> 1) & 1, abort, 18, u))) break;
+        if (!(ok = tc_wait_warp(&s_full[c], g & 1, abort, 18, u))) break;
         tc_fence_after();
-        float s[kCW];
-        {
-          uint32_t r[kCW];
-#pragma unroll
-          for (int c = 0; c < kCW / 32; ++c) tc_ld32_async(t_row + c_s + c * 32, r + c * 32);
-          tc_wait_ld();
-#pragma unroll
-          for (int c = 0; c < kCW; ++c) s[c] = __uint_as_float(pin_after_wait(r[c]));
-        }
-        // causal mask, this slice's maximum (8 independent chains)
-        const int tp0 = x.t0 + j * kTcTok + qs_ * kCW;
-        if (tp0 + kCW - 1 > qpos) {
-#pragma unroll
-          for (int c = 0; c < kCW; ++c) s[c] = tp0 + c > qpos ? -INFINITY : s[c];
-        }
-        float m8[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) m8[e] = s[e];
-#pragma unroll
-        for (int c = 8; c + 8 < kCW; c += 16)
-#pragma unroll
-          for (int e = 0; e < 8; ++e) m8[e] = fmax3(m8[e], s[c + e], s[c + 8 + e]);
-        if constexpr ((kCW - 8) % 16 != 0) {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) m8[e] = fmaxf(m8[e], s[kCW - 8 + e]);
-        }
-        const float pm = fmaxf(fmax3(m8[0], m8[1], m8[2]), fmax3(fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7]));
-        publish(c_s, pm);
-        // P(g) goes into buffer b once P(g-2) V(g-2) has finished reading it
-        if (!(ok = tc_wait_warp(&pv_done[b], ((g >> 1) & 1) ^ 1, abort, 20, u))) break;
-        uint8_t* sP = sm + TcSmem::kP + b * TcSmem::kTile;
-        auto make_p = [&](float ref) {   // P = 2^(s * scale - ref) into sP; returns its rounded sum
-          const float nmb = -ref;
-          float2 l2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-#pragma unroll
-          for (int c = 0; c < kCW / 8; ++c) {
-            uint32_t w[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              w[e] = exp2_pack<QD>(fma2(make_float2(s[c * 8 + 2 * e], s[c * 8 + 2 * e + 1]), p.s_mul, nmb), l2[e]);
-            *reinterpret_cast<uint4*>(sP + tc_swz(row, qs_ * (kCW / 8) + c)) = make_uint4(w[0], w[1], w[2], w[3]);
-          }
-          return ((l2[0].x + l2[0].y) + (l2[1].x + l2[1].y)) + ((l2[2].x + l2[2].y) + (l2[3].x + l2[3].y));
-        };
-        // speculatively with the current reference while the others' maxima are in flight:
-        // it stands unless the row maximum passes the reference by more than 2^8
-        const bool spec = m_ref != -INFINITY && pm * p.s_mul <= m_ref + kTcRescale;
-        float lt = spec ? make_p(m_ref) : 0.f;
-        float pms[kTcSplit];
-        if (!(ok = gather(b * 128, pm, u, pms))) break;
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s_empty[b]);
-        float rmax = pms[0];
-#pragma unroll
-        for (int q = 1; q < kTcSplit; ++q) rmax = fmaxf(rmax, pms[q]);
-        const float mx = rmax * p.s_mul;
+        // pass 1: the row maximum of the causally masked scores (8 independent chains); the
+        // mask only costs work in tiles where some row of the warp ends
+        const int tp0 = x.t0 + j * kTcTok;
+        const int vis = qpos - tp0;   // columns 0 .. vis of this tile are visible to the row
+        const bool masked = !__all_sync(kFull, vis >= kTcTok - 1);
+        const float mx = (masked ? tc_row_max<true>(t_row + c_s, vis) : tc_row_max<false>(t_row + c_s, vis)) * p.s_mul;
         const bool up = mx > m_ref + kTcRescale;
         const float corr = up ? ex2(m_ref - mx) : 1.f;   // 0 while nothing was accumulated
         if (up) {
@@ -641,116 +672,102 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           m_ref = mx;
         }
         if (j > 0 && __any_sync(kFull, up)) {
-          // O must hold P(g-1) V(g-1) before it is rescaled
-          if (!(ok = tc_wait_warp(&pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1, abort, 19, u))) break;
-          tc_fence_after();
+          // O holds every earlier P V of the unit: S(g) was issued after P(g-1) V(g-1) completed
 #pragma unroll 1
-          for (int c = 0; c < kCW / 32; ++c) {
+          for (int i = 0; i < kTcD / 32; ++i) {
             float o[32];
-            tc_ld32(t_row + c_o + c * 32, o);
+            tc_ld32(t_row + c_o + i * 32, o);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] *= corr;
-            tc_st32(t_row + c_o + c * 32, o);
+            for (int e = 0; e < 32; ++e) o[e] *= corr;
+            tc_st32(t_row + c_o + i * 32, o);
           }
         }
-        if (!spec || up) lt = make_p(m_ref == -INFINITY ? 0.f : m_ref);
-        l += lt;
-        // V rows past the visible tokens (cache bytes beyond the context, or stale rows
-        // of blocks not loaded) are zeroed, this slice of each, so that 0-weighted rows
-        // cannot bring a NaN into O
+        // pass 2, 32 columns at a time: P = 2^(s * scale - ref) as 16-bit pairs over the
+        // scores it was made from (the 32 tokens of chunk q: P in columns [32 q, 32 q + 16),
+        // for bf16 the rounded remainder p - bf16(p) in [32 q + 16, 32 q + 32))
+        const float nmb = m_ref == -INFINITY ? 0.f : -m_ref;
+        float2 l2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        const bool lo_on = QD == PA_BF16 && p.lo_mode != kLoNone;
+        if (masked) {
+          if (lo_on) tc_make_p<QD, true, true>(t_row + c_s, vis, p.s_mul, nmb, l2);
+          else tc_make_p<QD, true, false>(t_row + c_s, vis, p.s_mul, nmb, l2);
+        } else {
+          if (lo_on) tc_make_p<QD, false, true>(t_row + c_s, vis, p.s_mul, nmb, l2);
+          else tc_make_p<QD, false, false>(t_row + c_s, vis, p.s_mul, nmb, l2);
+        }
+        l += ((l2[0].x + l2[0].y) + (l2[1].x + l2[1].y)) + ((l2[2].x + l2[2].y) + (l2[3].x + l2[3].y));
+        // the remainder's product is issued when some row of the set has a weight above
+        // kTcLoShare of its running sum (adaptive), or always
+        if (p.lo_mode == kLoAdaptive && __any_sync(kFull, ex2(mx + nmb) > kTcLoShare * l) && lane == 0)
+          *reinterpret_cast<volatile int*>(&lo_tile[c]) = int(g);
+        // V rows past the visible tokens (cache bytes beyond the context, or stale rows of
+        // blocks not loaded) are zeroed, so that 0-weighted rows cannot bring a NaN into O
         const int rem = x.nvis - j * kTcTok;
         if (rem < kTcTok) {
-          if (!(ok = tc_wait_warp(&v_full[b], (g >> 1) & 1, abort, 21, u))) break;
+          if (!(ok = tc_wait_warp(&v_full[c], g & 1, abort, 21, u))) break;
           if (row >= rem) {
-            uint8_t* vt = sm + TcSmem::kV + b * TcSmem::kTile;
 #pragma unroll
-            for (int c = 0; c < kCW / 8; ++c)
-              *reinterpret_cast<uint4*>(vt + tc_swz(row, qs_ * (kCW / 8) + c)) = make_uint4(0, 0, 0, 0);
+            for (int i = 0; i < kTcD / 8; ++i) *reinterpret_cast<uint4*>(sV + tc_swz(row, i)) = make_uint4(0, 0, 0, 0);
           }
+          fence_async_smem();
         }
-        fence_async_smem();
+        tc_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[b]);
+        if (lane == 0) mbar_arrive(&p_full[c]);
       }
       if (!ok) break;
-      // this unit's O
-      if (!tc_wait_warp(&o_full[ob], (k >> 1) & 1, abort, 22, u)) break;
+      // this unit's O, 64 columns at a time: the output row (the row's whole context was in
+      // this unit) or the chunk's partial (unnormalised row, then max and sum); the
+      // accumulator is released once all of it is read
+      if (!tc_wait_warp(&o_full[c], k & 1, abort, 22, u)) break;
       tc_fence_after();
-      float o[kCW];
-      {
-        uint32_t r[kCW];
+      const int P = has_q ? (qpos + 1 + p.chunk - 1) / p.chunk : 0;
+      const bool wr = has_q && x.part < P, fin = wr && P == 1;
+      const float inv = fin ? 1.f / l : 0.f;
+      const size_t slot = (size_t(max(tok, 0)) * Hq + head) * p.max_parts + x.part;
+      uint4* orow = reinterpret_cast<uint4*>(static_cast<QT*>(p.out) + (size_t(max(tok, 0)) * Hq + head) * kTcD);
+      float4* acc = reinterpret_cast<float4*>(p.part_acc + slot * kTcD);
 #pragma unroll
-        for (int c = 0; c < kCW / 32; ++c) tc_ld32_async(t_row + c_o + c * 32, r + c * 32);
+      for (int h = 0; h < kTcD / 64; ++h) {
+        uint32_t r[64];
+        tc_ld32_async(t_row + c_o + h * 64, r);
+        tc_ld32_async(t_row + c_o + h * 64 + 32, r + 32);
         tc_wait_ld();
+        auto o = [&](int i) { return __uint_as_float(pin_after_wait(r[i])); };
+        if (fin) {
 #pragma unroll
-        for (int c = 0; c < kCW; ++c) o[c] = __uint_as_float(pin_after_wait(r[c]));
+          for (int i = 0; i < 8; ++i)
+            orow[h * 8 + i] = make_uint4(pack16x2<QD>(o(8 * i) * inv, o(8 * i + 1) * inv),
+                                         pack16x2<QD>(o(8 * i + 2) * inv, o(8 * i + 3) * inv),
+                                         pack16x2<QD>(o(8 * i + 4) * inv, o(8 * i + 5) * inv),
+                                         pack16x2<QD>(o(8 * i + 6) * inv, o(8 * i + 7) * inv));
+        } else if (wr) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) acc[h * 16 + i] = make_float4(o(4 * i), o(4 * i + 1), o(4 * i + 2), o(4 * i + 3));
+        }
       }
-      publish(c_o, l);
-      float ls[kTcSplit];
-      if (!gather(256 + ob * 128, l, u, ls)) break;
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&o_empty[ob]);
-      float lsum = ls[0];   // slice order: the same sum in every warp of the group
-#pragma unroll
-      for (int q = 1; q < kTcSplit; ++q) lsum += ls[q];
-      const int P = has_q ? (qpos + 1 + p.chunk - 1) / p.chunk : 0;
-      const bool wr = has_q && x.part < P;
-      const bool fin = wr && P == 1;
-      if (fin) {   // this slice of the row, rounded, staged in P buffer 0 (every P V has completed)
-        const float inv = 1.f / lsum;
-#pragma unroll
-        for (int i = 0; i < kCW / 8; ++i) {
-          float dummy = 0.f;
-          uint32_t w[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) w[e] = pack2_sum<QD>(o[i * 8 + 2 * e] * inv, o[i * 8 + 2 * e + 1] * inv, dummy);
-          *reinterpret_cast<uint4*>(sm + TcSmem::kP + tc_swz(row, qs_ * (kCW / 8) + i)) =
-              make_uint4(w[0], w[1], w[2], w[3]);
-        }
-      }
-      __syncwarp();
-      {   // coalesced: each store instruction writes (32 / kLPR) rows x kCW * 2 contiguous bytes
-        constexpr int kLPR = kCW / 8;               // lanes per row (16 bytes each)
-        constexpr int kRPI = 32 / kLPR;             // rows per instruction
-#pragma unroll
-        for (int i = 0; i < 32 / kRPI; ++i) {
-          const int rr = rw * 32 + i * kRPI + lane / kLPR, c = lane % kLPR;
-          const int rqi = x.t * QPT + rr / G;
-          if (x.part == 0 && rqi < x.Q && x.base + rqi + 1 <= p.chunk) {   // that row's whole context is here
-            QT* orow =
-                static_cast<QT*>(p.out) + (size_t(x.row0 + rqi) * Hq + x.hk * G + rr % G) * kTcD + qs_ * kCW;
-            *reinterpret_cast<uint4*>(orow + c * 8) =
-                *reinterpret_cast<const uint4*>(sm + TcSmem::kP + tc_swz(rr, qs_ * kLPR + c));
-          }
-        }
-      }
-      __syncwarp();
-      if (wr && !fin) {   // this chunk's partial: unnormalised row slice, (max, sum) once
-        const size_t slot = (size_t(tok) * Hq + head) * p.max_parts + x.part;
-        float4* acc = reinterpret_cast<float4*>(p.part_acc + slot * kTcD + qs_ * kCW);
-#pragma unroll
-        for (int i = 0; i < kCW / 4; ++i) acc[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
-        if (qs_ == 0) {
-          p.part_ml[slot * 2] = m_ref;
-          p.part_ml[slot * 2 + 1] = lsum;
-        }
+      if (lane == 0) mbar_arrive(&o_empty[c]);
+      if (wr && !fin) {
+        p.part_ml[slot * 2] = m_ref;
+        p.part_ml[slot * 2 + 1] = l;
       }
     }
   }
 
   __syncthreads();
-  if (*abort) {   // drain what this CTA issued: MMAs (their thread), then loads (their warp)
-    if (warp == kTcSoftmaxWarps && lane == 0) {
+  if (*abort) {   // drain what this CTA issued: MMAs (their thread), then each set's last loads
+    if (warp == kTcMmaWarp && lane == 0) {
       tc_commit(&bar_fin);
       mbar_wait_bounded(&bar_fin, 0);
     }
-    if (warp > kTcSoftmaxWarps && lane == 0) {
-      uint64_t* full = warp == kTcSoftmaxWarps + 2 ? v_full : k_full;
-      for (uint32_t h = last_load >= 2 ? last_load - 2 : 0; h < last_load; ++h)
-        mbar_wait_bounded(&full[h & 1], (h >> 1) & 1, 100000000ull);
-      if (q_loads > 0) mbar_wait_bounded(&q_full, (q_loads - 1) & 1, 100000000ull);   // V producer only
+    if (warp > kTcMmaWarp && lane == 0) {
+      const int c = warp - kTcMmaWarp - 1;
+      if (k_loads > 0) mbar_wait_bounded(&k_full[c], (k_loads - 1) & 1, 100000000ull);
+      if (v_loads > 0) mbar_wait_bounded(&v_full[c], (v_loads - 1) & 1, 100000000ull);
+      if (q_loads > 0) mbar_wait_bounded(&q_full[c], (q_loads - 1) & 1, 100000000ull);
     }
   }
   tc_fence_before();
@@ -804,6 +821,17 @@ TcKernel tc_pick(int qd, int BS, int G) {
   if (qd == PA_BF16) return BS == 16 ? tc_pick_g<PA_BF16, 16>(G) : BS == 32 ? tc_pick_g<PA_BF16, 32>(G) : nullptr;
   if (qd == PA_F16) return BS == 16 ? tc_pick_g<PA_F16, 16>(G) : BS == 32 ? tc_pick_g<PA_F16, 32>(G) : nullptr;
   return nullptr;
+}
+
+// How the bf16 remainder of P enters P V on this path: for the tiles that need it
+// (default), or for every tile when PA_BF16_REMAINDER=always is set in the environment
+// (read once). Both keep every weight to within the parity tolerance's needs.
+int tc_bf16_lo_mode() {
+  static const int mode = [] {
+    const char* e = std::getenv("PA_BF16_REMAINDER");
+    return (e && std::strcmp(e, "always") == 0) ? kLoAlways : kLoAdaptive;
+  }();
+  return mode;
 }
 
 bool extend_tc_supported(int qd, int D, int BS, int G) {
