@@ -488,8 +488,8 @@ def time_extend(name, steps, warmup, device, subset=0):
     import torch
     import synthetic
     import paged_kv_cache_436_b200 as pa
-    if name == "spec4_mix":
-        base = synthetic.make("llama13b_mix")
+    if name in ("spec4_mix", "spec4_long_fp8"):   # 4 draft tokens over the 13B mix / the 32K E4M3 cache
+        base = synthetic.make("llama13b_mix" if name == "spec4_mix" else "long_fp8")
         w, qlen = (synthetic.subset(base, subset) if subset else base), 4
     elif name == "prefill_gqa_8x2k":   # Llama-3-8B attention shapes: 32 q heads over 8 kv heads
         w = synthetic.custom(8, 32, 8, 128, 16, "bf16", "bf16", [2048] * 8, 4372, pool_factor=1.05)
@@ -547,7 +547,8 @@ def time_extend(name, steps, warmup, device, subset=0):
 
         prefill = {"fused_ms": timed(fused), "reshape_then_extend_ms": timed(two_pass)}
     lens = np.asarray(w.context_lens, dtype=np.int64)
-    kv_bytes = int(2 * lens.sum() * w.num_kv_heads * w.head_dim * 2) + 2 * T * w.num_q_heads * w.head_dim * 2
+    kvb = 1 if w.kv_dtype == "e4m3" else 2
+    kv_bytes = int(2 * lens.sum() * w.num_kv_heads * w.head_dim * kvb) + 2 * T * w.num_q_heads * w.head_dim * 2
     flops = 0
     for L, Qn in zip(lens, qlens):
         pos = L - Qn + np.arange(Qn, dtype=np.int64)
@@ -786,7 +787,7 @@ def workload_config(w, n_gpus):
             "parallelism": f"replicas{n_gpus}" if n_gpus > 1 else "single GPU"}
 
 
-EXTEND_WORKLOADS = ("spec4_mix", "prefill_8x2k", "prefill_gqa_8x2k")
+EXTEND_WORKLOADS = ("spec4_mix", "spec4_long_fp8", "prefill_8x2k", "prefill_gqa_8x2k")
 
 
 def bf16_peak():
@@ -834,7 +835,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="llama13b_mix")
-    ap.add_argument("--also", default="long_fp8,prefill_8x2k,spec4_mix",
+    ap.add_argument("--also", default="long_fp8,prefill_8x2k,spec4_mix,spec4_long_fp8",
                     help="further workloads reported in the same line ('' = none)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)

@@ -246,13 +246,21 @@ pa_status pa_decode_no_alloc(const void* q, int32_t q_dtype, int32_t num_seqs, i
  * Query i of sequence s sits at position L_s - Q_s + i and attends to tokens
  * 0 .. L_s - Q_s + i; out = softmax(scale * q K^T) V over them. Q_s > L_s, or a range
  * outside [0, num_tokens], is recorded (PA_DEV_BAD_CONTEXT_LEN) and its rows are zero.
- * Runs on the tensor cores (16-bit inputs, binary32 accumulation; P rounded to the
- * cache's 16-bit type): mma.sync for short query runs, tcgen05 with TMEM accumulators
- * for long ones (head_dim 128, scale > 0); context chunks (multiples of 512 tokens)
- * merged by a log-sum-exp kernel as in pa_decode. Cache bytes past a context never
- * affect the output.
- * Supported: 16-bit caches with q_dtype == kv_dtype, head_dim 64 or 128, block_size 16
- * or 32, G in {1, 2, 4, 8}. workspace >= pa_extend_workspace_size(...), 256-byte aligned.
+ * Runs on the tensor cores (16-bit inputs, binary32 accumulation): mma.sync for short
+ * query runs, tcgen05 with TMEM accumulators for long ones (16-bit caches, head_dim 128,
+ * scale > 0); context chunks (multiples of 512 tokens) merged by a log-sum-exp kernel as
+ * in pa_decode. P enters P V in the products' 16-bit type; for bf16 its rounded remainder
+ * p - bf16(p) enters as a second product (always on mma.sync; on tcgen05 for every
+ * 128-token tile in which some row has a weight above 1/8 of its running sum), so every
+ * weight is carried to within 2^-16 of its value where that matters. Cache bytes past a
+ * context never affect the output.
+ * E4M3 caches: each cache block is converted to f16 in shared memory (exact) and the
+ * products run in f16 with P in f16; a bf16 q is read as f16 after a 2^-8 scaling (exact
+ * for |q| in [2^-6, 1.6e7], saturating above); k_scale and v_scale multiply the scores
+ * and the output. These take the mma.sync path for runs of any length.
+ * Supported: 16-bit caches with q_dtype == kv_dtype, or E4M3 caches with q_dtype PA_F16
+ * or PA_BF16; head_dim 64 or 128, block_size 16 or 32, G in {1, 2, 4, 8}.
+ * workspace >= pa_extend_workspace_size(...), 256-byte aligned.
  */
 pa_status pa_extend(const void* q, int32_t q_dtype, int32_t num_seqs, int32_t num_q_heads,
                     const int32_t* query_start, int32_t num_tokens, const pa_cache_desc* cache,
@@ -280,12 +288,18 @@ size_t pa_extend_workspace_size(int32_t num_seqs, int32_t num_tokens, int32_t nu
  *   block_tables   device int32 [num_seqs][max_blocks_per_seq]: blocks that belong to the
  *                  sequence alone (freshly allocated), covering its Q_s tokens
  *   out            device [num_tokens][num_q_heads][head_dim], dtype
- * Afterwards cache slot bt[s][i / BS] * BS + i % BS holds k / v of prompt token i, bit for
- * bit, for every i < Q_s; the slots past Q_s in a prompt's last block hold unspecified
- * values. out is as pa_extend computes it with those cache contents.
- * Supported: dtype = the cache's kv_dtype = PA_F16 or PA_BF16, head_dim 128, block_size 16
- * or 32, G in {1, 2, 4, 8}, scale > 0 (the tcgen05 path); PA_ERR_ARG otherwise. workspace
- * >= pa_extend_workspace_size(...), 256-byte aligned; k, v, q and out 16-byte aligned.
+ * Afterwards cache slot bt[s][i / BS] * BS + i % BS holds k / v of prompt token i (bit for
+ * bit for a 16-bit cache; for an E4M3 cache encoded as pa_reshape_and_cache encodes it,
+ * e4m3_rne_satfinite(x / scale)), for every i < Q_s; the slots past Q_s in a prompt's last
+ * block hold unspecified values. out is as pa_extend computes it with those cache contents
+ * (for an E4M3 cache: over the quantised K / V).
+ * 16-bit caches: one tcgen05 kernel loads each K / V tile from the prompt rows, writes it
+ * into the cache and attends to it in the same pass. E4M3 caches: one launch quantises the
+ * prompts into the cache, then pa_extend's E4M3 kernel reads them back.
+ * Supported: dtype = the cache's kv_dtype = PA_F16 or PA_BF16 with head_dim 128 and
+ * scale > 0 (the tcgen05 path), or an E4M3 cache with dtype PA_F16 or PA_BF16 and head_dim
+ * 64 or 128; block_size 16 or 32, G in {1, 2, 4, 8}; PA_ERR_ARG otherwise. workspace >=
+ * pa_extend_workspace_size(...), 256-byte aligned; k, v, q and out 16-byte aligned.
  */
 pa_status pa_prefill(const void* q, const void* k, const void* v, int32_t dtype, int32_t num_seqs,
                      int32_t num_q_heads, const int32_t* query_start, int32_t num_tokens, const pa_cache_desc* cache,

@@ -20,6 +20,28 @@
 
 namespace pa {
 
+// Eight 16-bit values (one 16-byte vector) stored into an E4M3 cache: x / scale in
+// binary32 (round to nearest), then E4M3 round-to-nearest-even, saturating to +-448.
+template <int IN>
+__device__ __forceinline__ uint2 encode_e4m3x8(const uint4& raw, float scale) {
+  using IT = typename Q<IN>::T;
+  const IT* e = reinterpret_cast<const IT*>(&raw);
+  uint32_t packed[2];
+#pragma unroll
+  for (int w = 0; w < 2; ++w) {
+    uint32_t word = 0;
+#pragma unroll
+    for (int pr = 0; pr < 2; ++pr) {
+      const float a = __fdiv_rn(Q<IN>::to_float(e[4 * w + 2 * pr]), scale);
+      const float b = __fdiv_rn(Q<IN>::to_float(e[4 * w + 2 * pr + 1]), scale);
+      const __nv_fp8x2_storage_t two = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+      word |= uint32_t(two) << (16 * pr);
+    }
+    packed[w] = word;
+  }
+  return make_uint2(packed[0], packed[1]);
+}
+
 // grid (tokens, 2, chunks): y = 0 writes K, y = 1 writes V; each thread moves one
 // vector of 8 input elements (16 bytes) of the token's Hkv * D row.
 template <int KV, int IN>
@@ -30,7 +52,6 @@ __global__ void __launch_bounds__(128) reshape_kernel(const uint8_t* __restrict_
                                                       uint8_t* __restrict__ kc, uint8_t* __restrict__ vc,
                                                       int Hkv, int BS, int D, int num_blocks,
                                                       float k_scale, float v_scale) {
-  using IT = typename Q<IN>::T;
   const int t = blockIdx.x, which = blockIdx.y;
   const int i = blockIdx.z * blockDim.x + threadIdx.x;
   const int nvec = Hkv * D / 8;
@@ -56,25 +77,7 @@ __global__ void __launch_bounds__(128) reshape_kernel(const uint8_t* __restrict_
   if constexpr (KV != PA_E4M3) {
     *reinterpret_cast<uint4*>(dst) = raw;
   } else {
-    // x / scale in binary32 (round to nearest), then E4M3 round-to-nearest-even,
-    // saturating to +-448
-    const float sc = which ? v_scale : k_scale;
-    const IT* e = reinterpret_cast<const IT*>(&raw);
-    uint32_t packed[2];
-#pragma unroll
-    for (int w = 0; w < 2; ++w) {
-      uint32_t word = 0;
-#pragma unroll
-      for (int pr = 0; pr < 2; ++pr) {
-        const float a = __fdiv_rn(Q<IN>::to_float(e[4 * w + 2 * pr]), sc);
-        const float b = __fdiv_rn(Q<IN>::to_float(e[4 * w + 2 * pr + 1]), sc);
-        const __nv_fp8x2_storage_t two =
-            __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
-        word |= uint32_t(two) << (16 * pr);
-      }
-      packed[w] = word;
-    }
-    *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
+    *reinterpret_cast<uint2*>(dst) = encode_e4m3x8<IN>(raw, which ? v_scale : k_scale);
   }
 }
 

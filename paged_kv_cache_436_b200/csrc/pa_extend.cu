@@ -58,6 +58,9 @@ struct ExtendParams {
   int fresh;                    // whole prompts (pa_prefill): every L_s must equal Q_s
   int lo_mode;                  // tcgen05 path: how the bf16 remainder of P enters P V (kLoNone /
                                 //   kLoAlways / kLoAdaptive in pa_extend_tc.cu)
+  float k_scale, v_scale;       // E4M3 caches: per-tensor dequantisation scales (1 otherwise)
+  const void* k_new;            // E4M3 prefill: the prompts' K / V rows [T][Hkv][D] of q's type,
+  const void* v_new;            //   quantised into the cache before the attention reads it
 };
 
 constexpr int kTileRows = 16;
@@ -755,6 +758,302 @@ __global__ void __launch_bounds__(CoopCfg<D, BS>::kThreads) extend_coop_kernel(c
   }
 }
 
+// --------------------------------------------------------------------------
+// E4M3 caches: the 16-row warp kernel with each cache block converted in shared memory
+// --------------------------------------------------------------------------
+// Every (cache block, kv head) chunk of K and of V is contiguous in the cache layout and
+// arrives by one 1-D bulk copy (TMA engine, no multicast) into the warp's ring. Before use
+// it is converted to f16 -- the hardware E4M3 -> f16 conversion, exact: every E4M3 value
+// is an f16 value -- into a staging tile laid out as the 16-bit kernel's swizzled boxes, so
+// the same ldmatrix fragment code reads it. The products then run in f16: q is scaled by
+// 2^-8 into f16 when it is bf16 (exact for |q| in [2^-6, 1.6e7], within 2^-25 below,
+// saturating above), P is f16 (rounding up to 2^-11 of p: no remainder term is needed),
+// and the per-tensor scales multiply the scores (k_scale) and the output (v_scale). The K
+// block is converted and every score of the block formed first; then the V block takes
+// the same staging tile (rows past the tile's last token zero) for the P V products.
+template <int D, int BS>
+struct Fp8Cfg {
+  static constexpr int kChunk = BS * D;           // one (block, kv head) chunk of K (or V), bytes
+  static constexpr int kStage = 2 * kChunk;       // K then V
+  static constexpr int kStages = 2;
+  static constexpr int kStaging = BS * D * 2;     // one block of K or V as f16
+  static constexpr int kWarps = 4;
+  static constexpr int kThreads = kWarps * 32;
+  static constexpr int kPerWarp = kStages * kStage + kStaging;
+  static constexpr int kSmem = kWarps * kPerWarp + kWarps * kStages * 8 + 1024;
+  static_assert(BS % 16 == 0, "blocks hold whole 16-token slices");
+};
+
+// Two values to f16, rounded to nearest and saturating to +-65504, packed (lo in the low half).
+__device__ __forceinline__ uint32_t f16x2_satfinite(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Two E4M3 codes (lo in the low byte) as an f16 pair (exact).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two & 0xffffu), __NV_E4M3);
+  return uint32_t(h.x) | (uint32_t(h.y) << 16);
+}
+
+// One block of E4M3 rows (BS x D bytes, row-major) into the f16 staging tile, rows from
+// `keep` on set to zero. Lane-strided 16-byte chunks: conflict-free reads of whole rows.
+template <int D, int BS>
+__device__ __forceinline__ void fp8_block_to_f16(const uint8_t* src, uint8_t* dst, int keep, int lane) {
+  constexpr int CPR = D / 16;   // 16-byte chunks (16 codes) per row
+#pragma unroll
+  for (int idx = lane; idx < BS * CPR; idx += 32) {
+    const int r = idx / CPR, cb = idx - r * CPR;
+    uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
+    if (r < keep) {
+      const uint4 raw = *reinterpret_cast<const uint4*>(src + r * D + cb * 16);
+      a = make_uint4(e4m3x2_to_f16x2(raw.x), e4m3x2_to_f16x2(raw.x >> 16), e4m3x2_to_f16x2(raw.y),
+                     e4m3x2_to_f16x2(raw.y >> 16));
+      b = make_uint4(e4m3x2_to_f16x2(raw.z), e4m3x2_to_f16x2(raw.z >> 16), e4m3x2_to_f16x2(raw.w),
+                     e4m3x2_to_f16x2(raw.w >> 16));
+    }
+    *reinterpret_cast<uint4*>(dst + ext_swz<BS>(r, 2 * cb)) = a;
+    *reinterpret_cast<uint4*>(dst + ext_swz<BS>(r, 2 * cb + 1)) = b;
+  }
+}
+
+template <int QD, int D, int BS, int G>
+__global__ void __launch_bounds__(Fp8Cfg<D, BS>::kThreads) extend_fp8_kernel(const ExtendParams p) {
+  using C = Fp8Cfg<D, BS>;
+  using QT = typename Q<QD>::T;
+  constexpr int NS = C::kStages, NW = C::kWarps, KK = D / 16, NT = D / 8, SB = BS / 16;
+  constexpr int QPT = kTileRows / G;                      // queries per tile
+  constexpr float kQScale = QD == PA_BF16 ? 1.f / 256.f : 1.f;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint8_t* ring = smem + warp * C::kPerWarp;
+  uint8_t* stg = ring + NS * C::kStage;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + NW * C::kPerWarp) + warp * NS;
+  if (lane == 0) {
+    for (int i = 0; i < NS; ++i) mbar_init(&bar[i], 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  grid_dependency_launch_dependents();
+  grid_dependency_wait();
+
+  const int Hq = p.num_q_heads, Hkv = p.num_kv_heads;
+  const int total = p.plan[p.num_seqs] * Hkv;
+  const uint64_t pol = l2_policy_evict_first();
+  const size_t head_stride = size_t(BS) * D, block_stride = size_t(Hkv) * head_stride;
+  const float s_mul = p.s_mul * p.k_scale / kQScale;      // scores: the f16 products times this
+  uint32_t consumed = 0;
+  const int r0 = lane >> 2, cq = (lane & 3) * 2;
+
+  for (int u = blockIdx.x * NW + warp; u < total; u += gridDim.x * NW) {
+    const ExtUnit x = ext_make_unit<BS>(p, u, total, QPT, lane);
+    int qpos[2], tok[2], head[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int r = r0 + 8 * h;
+      const int qi = x.t * QPT + r / G;
+      head[h] = x.hk * G + r % G;
+      if (qi < x.Q) {
+        qpos[h] = x.base + qi;
+        tok[h] = x.row0 + qi;
+      } else {
+        qpos[h] = -1;
+        tok[h] = -1;
+      }
+    }
+    // Q fragments as f16 pairs (scaled by 2^-8 from bf16), zero for missing rows
+    uint32_t qa[KK][4];
+#pragma unroll
+    for (int kk = 0; kk < KK; ++kk)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int h = e & 1, dim = kk * 16 + cq + (e >> 1) * 8;
+        uint32_t v = 0u;
+        if (tok[h] >= 0) {
+          const QT* qp = static_cast<const QT*>(p.q) + (size_t(tok[h]) * Hq + head[h]) * D + dim;
+          if constexpr (QD == PA_F16) v = *reinterpret_cast<const uint32_t*>(qp);
+          else v = f16x2_satfinite(Q<QD>::to_float(qp[0]) * kQScale, Q<QD>::to_float(qp[1]) * kQScale);
+        }
+        qa[kk][e] = v;
+      }
+
+    auto issue = [&](int i, uint32_t g) {   // cache block i of the unit: one bulk copy each of K and V
+      const int bid = __shfl_sync(kFull, x.bid, i);
+      const int st = g % NS;
+      if (lane == 0) {
+        uint8_t* dst = ring + st * C::kStage;
+        const size_t off = size_t(bid) * block_stride + size_t(x.hk) * head_stride;
+        mbar_arrive_expect_tx(&bar[st], C::kStage);
+        bulk_g2s(dst, p.k_cache + off, C::kChunk, &bar[st], pol);
+        bulk_g2s(dst + C::kChunk, p.v_cache + off, C::kChunk, &bar[st], pol);
+      }
+      __syncwarp();
+    };
+    for (int i = 0; i < NS && i < x.nblk; ++i) issue(i, consumed + i);
+
+    float o[NT][4];
+#pragma unroll
+    for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+    float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+    bool failed = false;
+
+    for (int i = 0; i < x.nblk; ++i) {
+      const uint32_t n = consumed;
+      const int st = n % NS;
+      if (!__all_sync(kFull, mbar_wait_bounded(&bar[st], (n / NS) & 1))) {
+        if (lane == 0) record_error(PA_DEV_WAIT_TIMEOUT, 5, u, st);
+        failed = true;
+        break;
+      }
+      const uint8_t* Ke = ring + st * C::kStage;
+      const int tok0 = (x.b0 + i) * BS;
+      // the K block as f16, then every score of the block
+      fp8_block_to_f16<D, BS>(Ke, stg, BS, lane);
+      __syncwarp();
+      float sc[SB][2][4];
+#pragma unroll
+      for (int sb = 0; sb < SB; ++sb) {
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) sc[sb][nt][0] = sc[sb][nt][1] = sc[sb][nt][2] = sc[sb][nt][3] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < KK; ++kk) {
+          uint32_t b[4];
+          const int trow = sb * 16 + (lane >> 4) * 8 + (lane & 7);
+          ldsm_x4(b, stg + ext_swz<BS>(trow, kk * 2 + ((lane >> 3) & 1)));
+          mma16816<PA_F16>(sc[sb][0], qa[kk], b[0], b[1]);
+          mma16816<PA_F16>(sc[sb][1], qa[kk], b[2], b[3]);
+        }
+      }
+      __syncwarp();   // every lane has read K from the staging tile
+      // the V block into the same tile; rows past the tile's last token (cache bytes beyond
+      // the context, possibly NaN codes) are zero
+      fp8_block_to_f16<D, BS>(Ke + C::kChunk, stg, x.last + 1 - tok0, lane);
+      __syncwarp();
+      ++consumed;     // both halves of the stage are read: it can be refilled
+      if (i + NS < x.nblk) issue(i + NS, consumed + NS - 1);
+#pragma unroll
+      for (int sb = 0; sb < SB; ++sb) {
+        float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int h = e >> 1;
+            const int tp = tok0 + sb * 16 + nt * 8 + cq + (e & 1);
+            float v = sc[sb][nt][e] * s_mul;
+            if (tp > qpos[h]) v = -INFINITY;
+            sc[sb][nt][e] = v;
+            mx[h] = fmaxf(mx[h], v);
+          }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          mx[h] = fmaxf(mx[h], __shfl_xor_sync(kFull, mx[h], 1));
+          mx[h] = fmaxf(mx[h], __shfl_xor_sync(kFull, mx[h], 2));
+        }
+        float base_m[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if (mx[h] > m[h]) {
+            const float corr = exp2f(m[h] - mx[h]);     // 0 while nothing was accumulated
+            m[h] = mx[h];
+            l[h] *= corr;
+#pragma unroll
+            for (int nn = 0; nn < NT; ++nn) {
+              o[nn][2 * h] *= corr;
+              o[nn][2 * h + 1] *= corr;
+            }
+          }
+          base_m[h] = m[h] == -INFINITY ? 0.f : m[h];
+        }
+        uint32_t pa[4], pl[4];
+        make_p_operands<PA_F16>(sc[sb], base_m, pa, pl, l);
+#pragma unroll
+        for (int np = 0; np < NT / 2; ++np) {
+          uint32_t b[4];
+          const int trow = sb * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
+          ldsm_x4_trans(b, stg + ext_swz<BS>(trow, np * 2 + (lane >> 4)));
+          mma16816<PA_F16>(o[2 * np], pa, b[0], b[1]);
+          mma16816<PA_F16>(o[2 * np + 1], pa, b[2], b[3]);
+        }
+      }
+      __syncwarp();   // every lane has read V before the next block takes the tile
+    }
+    if (failed) {
+      for (uint32_t k = consumed; k < consumed + NS; ++k) mbar_wait_bounded(&bar[k % NS], (k / NS) & 1, 100000000ull);
+      break;
+    }
+
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      l[h] += __shfl_xor_sync(kFull, l[h], 1);
+      l[h] += __shfl_xor_sync(kFull, l[h], 2);
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      if (tok[h] < 0) continue;
+      const int P = (qpos[h] + 1 + p.chunk - 1) / p.chunk;
+      if (x.part >= P) continue;
+      if (P == 1) {
+        QT* orow = static_cast<QT*>(p.out) + (size_t(tok[h]) * Hq + head[h]) * D;
+        const float inv = p.v_scale / l[h];
+#pragma unroll
+        for (int nn = 0; nn < NT; ++nn) {
+          float a, b2;
+          *reinterpret_cast<uint32_t*>(orow + nn * 8 + cq) = pack2<QD>(o[nn][2 * h] * inv, o[nn][2 * h + 1] * inv, a, b2);
+        }
+      } else {
+        const size_t slot = (size_t(tok[h]) * Hq + head[h]) * p.max_parts + x.part;
+        float* acc = p.part_acc + slot * D;
+#pragma unroll
+        for (int nn = 0; nn < NT; ++nn)
+          *reinterpret_cast<float2*>(acc + nn * 8 + cq) =
+              make_float2(o[nn][2 * h] * p.v_scale, o[nn][2 * h + 1] * p.v_scale);
+        if ((lane & 3) == 0) {
+          p.part_ml[slot * 2] = m[h];
+          p.part_ml[slot * 2 + 1] = l[h];
+        }
+      }
+    }
+  }
+}
+
+// Whole prompts into an E4M3 cache (pa_prefill): token t of sequence s (rows query_start[s]
+// ..) goes to slot bt[s][i / BS] * BS + i % BS, i = t - query_start[s], stored as
+// e4m3_rne_satfinite(x / scale) as pa_reshape_and_cache stores it. Grid (tokens, K / V,
+// 16-byte input chunks / 128).
+template <int IN>
+__global__ void __launch_bounds__(128) prefill_fp8_write_kernel(const ExtendParams p, int BS, int D) {
+  const int t = blockIdx.x, which = blockIdx.y;
+  const int i = blockIdx.z * blockDim.x + threadIdx.x;
+  const int nvec = p.num_kv_heads * D / 8;
+  if (i >= nvec) return;
+  int lo = 0, hi = p.num_seqs;                 // query_start[lo] <= t < query_start[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (p.query_start[mid] <= t) lo = mid; else hi = mid;
+  }
+  const int s = lo;
+  int nq, base;
+  ext_seq(p, s, nq, base);                     // an invalid sequence (recorded by the plan) has none
+  const int pos = t - p.query_start[s];
+  if (pos < 0 || pos >= nq) return;
+  int bid = p.block_tables[size_t(s) * p.max_blocks + pos / BS];
+  if (bid < 0 || bid >= p.num_blocks) {
+    if (i == 0 && which == 0) record_error(PA_DEV_BAD_BLOCK_ID, s, pos / BS, bid);
+    return;
+  }
+  const int e0 = i * 8, h = e0 / D, d = e0 - h * D;
+  using IT = typename Q<IN>::T;
+  const IT* src = static_cast<const IT*>(which ? p.v_new : p.k_new) + (size_t(t) * p.num_kv_heads) * D + e0;
+  const uint4 raw = *reinterpret_cast<const uint4*>(src);
+  uint8_t* dst = const_cast<uint8_t*>(which ? p.v_cache : p.k_cache) +
+                 ((size_t(bid) * p.num_kv_heads + h) * BS + pos % BS) * D + d;
+  *reinterpret_cast<uint2*>(dst) = encode_e4m3x8<IN>(raw, which ? p.v_scale : p.k_scale);
+}
+
 // Log-sum-exp merge of a query row's partitions: one 4-warp CTA per (query row, q head).
 template <int QD, int D>
 __global__ void __launch_bounds__(128) extend_reduce_kernel(const ExtendParams p) {
@@ -872,6 +1171,24 @@ ExtLaunch ext_pick_d(int D, int BS, int G, bool coop) {
   return ExtLaunch{};
 }
 
+template <int QD, int D, int BS>
+ExtLaunch fp8_pick_g(int G) {
+  using C = Fp8Cfg<D, BS>;
+  switch (G) {
+    case 1: return ExtLaunch{extend_fp8_kernel<QD, D, BS, 1>, nullptr, C::kSmem, C::kThreads};
+    case 2: return ExtLaunch{extend_fp8_kernel<QD, D, BS, 2>, nullptr, C::kSmem, C::kThreads};
+    case 4: return ExtLaunch{extend_fp8_kernel<QD, D, BS, 4>, nullptr, C::kSmem, C::kThreads};
+    case 8: return ExtLaunch{extend_fp8_kernel<QD, D, BS, 8>, nullptr, C::kSmem, C::kThreads};
+  }
+  return ExtLaunch{};
+}
+template <int QD>
+ExtLaunch fp8_pick_d(int D, int BS, int G) {
+  if (D == 64) return BS == 16 ? fp8_pick_g<QD, 64, 16>(G) : BS == 32 ? fp8_pick_g<QD, 64, 32>(G) : ExtLaunch{};
+  if (D == 128) return BS == 16 ? fp8_pick_g<QD, 128, 16>(G) : BS == 32 ? fp8_pick_g<QD, 128, 32>(G) : ExtLaunch{};
+  return ExtLaunch{};
+}
+
 cudaError_t ext_launch(ExtKernel fn, int grid, int threads, size_t smem, cudaStream_t s, const ExtendParams& p) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
@@ -918,7 +1235,9 @@ static pa_status extend_impl(const void* q, int32_t q_dtype, int32_t num_seqs, i
                              size_t workspace_bytes, void* stream, const void* k_new, const void* v_new, bool fresh) {
   pa_status st = validate_cache(c);
   if (st != PA_OK) return st;
-  if (c->kv_dtype == PA_E4M3 || q_dtype != c->kv_dtype) return PA_ERR_ARG;   // 16-bit caches only
+  const bool fp8 = c->kv_dtype == PA_E4M3;
+  if (q_dtype != PA_F16 && q_dtype != PA_BF16) return PA_ERR_ARG;
+  if (!fp8 && q_dtype != c->kv_dtype) return PA_ERR_ARG;   // a 16-bit cache holds q's type
   if (c->block_size != 16 && c->block_size != 32) return PA_ERR_ARG;
   if (num_seqs < 0 || num_tokens < 0 || num_q_heads <= 0 || max_blocks_per_seq <= 0 || max_context_len < 0)
     return PA_ERR_ARG;
@@ -936,14 +1255,19 @@ static pa_status extend_impl(const void* q, int32_t q_dtype, int32_t num_seqs, i
   if (workspace_bytes < ws.total) return PA_ERR_ARG;
   // Long query runs (at least half a 128-row tile per sequence on average) go to the
   // tcgen05 kernel (head_dim 128) or, otherwise, the cooperative 64-row kernel; short
-  // ones (speculative drafts, decode) to the 16-row warp kernel.
+  // ones (speculative drafts, decode) to the 16-row warp kernel. E4M3 caches take the
+  // 16-row kernel that converts each block in shared memory, for runs of any length;
+  // whole prompts into an E4M3 cache are first quantised into it by one more launch.
   const long long rows_total = (long long)num_tokens * G;
-  const bool tc = (fresh || rows_total * 2 >= (long long)kTcUnitRows * num_seqs) && scale > 0.f &&
+  const bool tc = !fp8 && (fresh || rows_total * 2 >= (long long)kTcUnitRows * num_seqs) && scale > 0.f &&
                   extend_tc_supported(q_dtype, D, BS, G);
-  if (fresh && (!tc || !k_new || !v_new || !aligned16(k_new) || !aligned16(v_new))) return PA_ERR_ARG;
-  const bool coop = !tc && rows_total > (long long)kTileRows * num_seqs;
+  if (fresh && (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new) || (!tc && !fp8))) return PA_ERR_ARG;
+  const bool coop = !fp8 && !tc && rows_total > (long long)kTileRows * num_seqs;
   ExtLaunch k;
-  if (!tc) {
+  if (fp8) {
+    k = q_dtype == PA_BF16 ? fp8_pick_d<PA_BF16>(D, BS, G) : fp8_pick_d<PA_F16>(D, BS, G);
+    if (!k.key()) return PA_ERR_ARG;
+  } else if (!tc) {
     k = q_dtype == PA_BF16 ? ext_pick_d<PA_BF16>(D, BS, G, coop) : ext_pick_d<PA_F16>(D, BS, G, coop);
     if (!k.key()) return PA_ERR_ARG;
   }
@@ -966,6 +1290,10 @@ static pa_status extend_impl(const void* q, int32_t q_dtype, int32_t num_seqs, i
   p.units_cap = (long long)ext_units_bound(num_tokens, num_q_heads, max_parts);
   p.fresh = fresh ? 1 : 0;
   p.lo_mode = q_dtype == PA_BF16 ? tc_bf16_lo_mode() : 0;
+  p.k_scale = c->k_scale;
+  p.v_scale = c->v_scale;
+  p.k_new = k_new;
+  p.v_new = v_new;
   p.num_seqs = num_seqs;
   p.num_tokens = num_tokens;
   p.num_q_heads = num_q_heads;
@@ -1004,8 +1332,9 @@ static pa_status extend_impl(const void* q, int32_t q_dtype, int32_t num_seqs, i
     as_launch.threads = k.threads;
     if (occupancy(as_launch, &cap) != cudaSuccess) return PA_ERR_CUDA;
     const long long units = tiles * c->num_kv_heads * max_parts;
-    // the warp kernel runs 4 independent units per CTA, the cooperative one a unit per CTA
+    // the warp kernels run 4 independent units per CTA, the cooperative one a unit per CTA
     const long long ctas = coop ? units : (units + ExtCfg<128, 16>::kWarps - 1) / ExtCfg<128, 16>::kWarps;
+    static_assert(ExtCfg<128, 16>::kWarps == Fp8Cfg<128, 16>::kWarps, "both warp kernels run 4 units per CTA");
     grid = int(ctas < cap ? ctas : cap);
   }
   if (grid < 1) grid = 1;
@@ -1014,6 +1343,13 @@ static pa_status extend_impl(const void* q, int32_t q_dtype, int32_t num_seqs, i
 
   extend_plan_kernel<<<1, 1024, 0, s>>>(p, rows_per_unit / G);
   if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+  if (fp8 && fresh) {   // the prompts' K / V into the cache, before the attention reads it
+    const int nvec = c->num_kv_heads * D / 8;
+    const dim3 wgrid(num_tokens, 2, (nvec + 127) / 128);
+    if (q_dtype == PA_BF16) prefill_fp8_write_kernel<PA_BF16><<<wgrid, 128, 0, s>>>(p, BS, D);
+    else prefill_fp8_write_kernel<PA_F16><<<wgrid, 128, 0, s>>>(p, BS, D);
+    if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+  }
   if (tc) {
     st = extend_tc_launch(p, c, q_dtype, G, grid, s, k_new, v_new);
     if (st != PA_OK) return st;

@@ -278,6 +278,21 @@ __device__ __forceinline__ void tc_st16(uint32_t addr, const uint32_t* v) {
       : "memory");
 }
 __device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+// 16 consecutive 32-bit columns of this warp's 32 lanes, without the wait.
+__device__ __forceinline__ void tc_ld16_async(uint32_t addr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(addr));
+}
+
+// 8 consecutive 32-bit columns of this warp's 32 lanes, without the wait.
+__device__ __forceinline__ void tc_st8(uint32_t addr, const uint32_t* v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(addr), "r"(v[0]),
+               "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
+}
 
 // Two values rounded to the 16-bit type and packed (lo in the low half).
 template <int QD>
@@ -300,43 +315,42 @@ __device__ __forceinline__ float2 bf16x2_value(uint32_t w) {
 // columns past `vis` masked when kMask.
 template <bool kMask>
 __device__ __forceinline__ float tc_row_max(uint32_t addr, int vis) {
-  uint32_t r[kTcTok];
-#pragma unroll
-  for (int i = 0; i < kTcTok / 32; ++i) tc_ld32_async(addr + i * 32, r + i * 32);
-  tc_wait_ld();
-  auto at = [&](int i) {
-    const float v = __uint_as_float(pin_after_wait(r[i]));
-    return kMask && i > vis ? -INFINITY : v;
-  };
   float m8[8];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) m8[e] = at(e);
+  for (int e = 0; e < 8; ++e) m8[e] = -INFINITY;
 #pragma unroll
-  for (int i = 8; i + 8 < kTcTok; i += 16)
+  for (int h = 0; h < kTcTok / 64; ++h) {   // 64 columns at a time
+    uint32_t r[64];
+    tc_ld32_async(addr + h * 64, r);
+    tc_ld32_async(addr + h * 64 + 32, r + 32);
+    tc_wait_ld();
+    auto at = [&](int i) {
+      const float v = __uint_as_float(pin_after_wait(r[i]));
+      return kMask && h * 64 + i > vis ? -INFINITY : v;
+    };
 #pragma unroll
-    for (int e = 0; e < 8; ++e) m8[e] = fmax3(m8[e], at(i + e), at(i + 8 + e));
-  if constexpr ((kTcTok - 8) % 16 != 0) {
+    for (int i = 0; i < 64; i += 16)
 #pragma unroll
-    for (int e = 0; e < 8; ++e) m8[e] = fmaxf(m8[e], at(kTcTok - 8 + e));
+      for (int e = 0; e < 8; ++e) m8[e] = fmax3(m8[e], at(i + e), at(i + 8 + e));
   }
   return fmaxf(fmax3(m8[0], m8[1], m8[2]), fmax3(fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7]));
 }
 
-// Pass 2 of the softmax, 32 columns at a time: p = 2^(s * s_mul + nmb) of one row's 128
-// scores, written over them as 16-bit pairs (the 32 tokens of chunk q: P in columns
-// [32 q, 32 q + 16); with kLo the rounded remainder p - bf16(p) in [32 q + 16, 32 q + 32));
+// Pass 2 of the softmax, 16 columns at a time: p = 2^(s * s_mul + nmb) of one row's 128
+// scores, written over them as 16-bit pairs (tokens 16 t .. 16 t + 15: P in columns
+// [16 t, 16 t + 8); with kLo the rounded remainder p - bf16(p) in [16 t + 8, 16 t + 16));
 // the binary32 p are added to l2 (four pair chains).
 template <int QD, bool kMask, bool kLo>
 __device__ __forceinline__ void tc_make_p(uint32_t addr, int vis, float s_mul, float nmb, float2 (&l2)[4]) {
 #pragma unroll
-  for (int q = 0; q < kTcTok / 32; ++q) {
-    uint32_t r[32];
-    tc_ld32_async(addr + q * 32, r);
+  for (int t = 0; t < kTcTok / 16; ++t) {   // tokens 16 t .. 16 t + 15: scores in columns [16 t, 16 t + 16)
+    uint32_t r[16];
+    tc_ld16_async(addr + t * 16, r);
     tc_wait_ld();
-    uint32_t wh[16], wl[16];
+    uint32_t wh[8], wl[8];
 #pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      const int col = q * 32 + 2 * e;
+    for (int e = 0; e < 8; ++e) {
+      const int col = t * 16 + 2 * e;
       float s0 = __uint_as_float(pin_after_wait(r[2 * e]));
       float s1 = __uint_as_float(pin_after_wait(r[2 * e + 1]));
       if (kMask) {
@@ -352,18 +366,16 @@ __device__ __forceinline__ void tc_make_p(uint32_t addr, int vis, float s_mul, f
         wl[e] = pack16x2<QD>(p0 - hv.x, p1 - hv.y);
       }
     }
-    tc_st16(addr + q * 32, wh);
-    if constexpr (kLo) tc_st16(addr + q * 32 + 16, wl);
+    tc_st8(addr + t * 16, wh);
+    if constexpr (kLo) tc_st8(addr + t * 16 + 8, wl);
   }
 }
 
-// 184 registers x 352 threads = 64768 of the SM's 65536: one CTA per SM (a bound of 352
-// threads would let the compiler assume 384 and stop at 168, spilling the softmax rows).
-constexpr int kTcMaxRegs = 184;
-static_assert(kTcMaxRegs * kTcThreads <= 65536, "the register file holds one CTA");
-
+// One CTA per SM. The register file is split between the SM's four sub-partitions and a
+// warp takes its registers from its own: with 11 warps, three share one sub-partition's
+// 16384 registers, so a thread may hold at most 170 (the compiler takes 168).
 template <int QD, int BS, int G>
-__global__ void __maxnreg__(kTcMaxRegs)
+__global__ void __launch_bounds__(kTcThreads, 1)
     extend_tc_kernel(const ExtendParams p, const __grid_constant__ CUtensorMap tk,
                      const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tq,
                      const __grid_constant__ CUtensorMap tkn, const __grid_constant__ CUtensorMap tvn) {
@@ -619,13 +631,11 @@ __global__ void __maxnreg__(kTcMaxRegs)
           const uint32_t d = tmem + 256 + c * 128, a = tmem + c * 128;
 #pragma unroll
           for (int kk = 0; kk < kTcTok / 16; ++kk)   // P of tokens 16 kk .. 16 kk + 15
-            tc_mma_ts(d, a + 32 * (kk >> 1) + 8 * (kk & 1), tc_desc(va + kk * 2048, 1024, kTcTok * 128), idO,
-                      (j[c] > 0 || kk > 0) ? 1u : 0u);
+            tc_mma_ts(d, a + 16 * kk, tc_desc(va + kk * 2048, 1024, kTcTok * 128), idO, (j[c] > 0 || kk > 0) ? 1u : 0u);
           if (lo) {
 #pragma unroll
-            for (int kk = 0; kk < kTcTok / 16; ++kk)   // their remainders, 16 columns further
-              tc_mma_ts(d, a + 32 * (kk >> 1) + 8 * (kk & 1) + 16, tc_desc(va + kk * 2048, 1024, kTcTok * 128), idO,
-                        1u);
+            for (int kk = 0; kk < kTcTok / 16; ++kk)   // their remainders, 8 columns further
+              tc_mma_ts(d, a + 16 * kk + 8, tc_desc(va + kk * 2048, 1024, kTcTok * 128), idO, 1u);
           }
           tc_commit(&pv_done[c]);
           if (j[c] + 1 == x[c].ntiles) tc_commit(&o_full[c]);
@@ -682,9 +692,9 @@ __global__ void __maxnreg__(kTcMaxRegs)
             tc_st32(t_row + c_o + i * 32, o);
           }
         }
-        // pass 2, 32 columns at a time: P = 2^(s * scale - ref) as 16-bit pairs over the
-        // scores it was made from (the 32 tokens of chunk q: P in columns [32 q, 32 q + 16),
-        // for bf16 the rounded remainder p - bf16(p) in [32 q + 16, 32 q + 32))
+        // pass 2, 16 columns at a time: P = 2^(s * scale - ref) as 16-bit pairs over the
+        // scores it was made from (tokens 16 t ..: P in columns [16 t, 16 t + 8), for bf16
+        // the rounded remainder p - bf16(p) in [16 t + 8, 16 t + 16))
         const float nmb = m_ref == -INFINITY ? 0.f : -m_ref;
         float2 l2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
         const bool lo_on = QD == PA_BF16 && p.lo_mode != kLoNone;

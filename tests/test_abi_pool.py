@@ -83,7 +83,9 @@ def test_extend_and_prefill_argument_checks_launch_nothing():
         return L.pa_extend(q, q_dtype, 2, Hq, 256, 8, ctypes.byref(desc), 256, 4, 256, 64, scale, 256, 256, wsb,
                            None)
 
-    assert extend(fp8) == pa.PA_ERR_ARG                      # E4M3 caches: decode only
+    assert extend(fp8, q_dtype=pa.PA_E4M3) == pa.PA_ERR_ARG  # q is f16 or bf16, also over an E4M3 cache
+    fp8_bs8 = pa.CacheDesc(64, 2, 8, 128, pa.PA_E4M3, 0.05, 0.05, 256, 256)
+    assert extend(fp8_bs8) == pa.PA_ERR_ARG                  # extend reads blocks of 16 or 32 tokens
     assert extend(bf, q_dtype=pa.PA_F16) == pa.PA_ERR_ARG    # q dtype must equal the cache's
     assert extend(bf, Hq=6) == pa.PA_ERR_ARG                 # G = 3
     assert extend(bf, scale=float("nan")) == pa.PA_ERR_ARG
@@ -98,7 +100,8 @@ def test_extend_and_prefill_argument_checks_launch_nothing():
 
     assert prefill(d64) == pa.PA_ERR_ARG                      # head_dim 64: no tcgen05 path
     assert prefill(bf, scale=-0.1) == pa.PA_ERR_ARG           # the tcgen05 path needs scale > 0
-    assert prefill(fp8) == pa.PA_ERR_ARG
+    assert prefill(fp8, k=None) == pa.PA_ERR_ARG              # an E4M3 prefill needs the prompts' K / V
+    assert prefill(fp8, k=264) == pa.PA_ERR_ARG               # ... 16-byte aligned
     # the self-test refuses limits out of range before launching anything
     assert L.pa_selftest_wait_timeout(0, None) == pa.PA_ERR_ARG
     assert L.pa_selftest_wait_timeout(3000000, None) == pa.PA_ERR_ARG

@@ -100,14 +100,16 @@ def test_more_queries_than_context_is_recorded_and_zero():
 
 
 def _nan_tails(w, eng):
-    """Cache bytes past each context in its last block set to NaN: memory that was never
-    written may hold anything, and no output may depend on it."""
+    """Cache bytes past each context in its last block set to NaN (the E4M3 NaN code for an
+    E4M3 cache): memory that was never written may hold anything, and no output may
+    depend on it."""
+    from tests.gpu_cases import fill_nan_
     BS = w.block_size
     for s, L in enumerate(eng.lens):
         if L % BS:
             b = int(eng.bt_host[s, (L - 1) // BS])
-            eng.k_cache[b, :, L % BS:, :] = float("nan")
-            eng.v_cache[b, :, L % BS:, :] = float("nan")
+            fill_nan_(eng.k_cache[b, :, L % BS:, :], w.kv_dtype)
+            fill_nan_(eng.v_cache[b, :, L % BS:, :], w.kv_dtype)
 
 
 def _sample_rows(qs, Hq, n, seed):
@@ -246,3 +248,116 @@ def test_long_context_many_chunks():
     out = _run(w, eng, qs_dev, q, qs)
     assert pa.last_device_error()[0] == 0
     _check_rows(w, eng, q, qs, out, _sample_rows(qs, 8, 60, 97), "20000-token context")
+
+
+# ---------------------------------------------------------------------------
+# E4M3 caches
+# ---------------------------------------------------------------------------
+
+def _ref_scaled(w, eng, q, qs_host, rows=None):
+    d = eng.cache.desc
+    bt = eng.bt_host.astype(np.int64)
+    return oatt.paged_extend(codes_np(q), w.q_dtype, codes_np(eng.k_cache), codes_np(eng.v_cache), w.kv_dtype,
+                             d.k_scale, d.v_scale, bt, list(eng.lens), qs_host, w.scale, rows=rows)
+
+
+@pytest.mark.parametrize("qd,D,BS,G", [("bf16", 128, 32, 1), ("f16", 128, 16, 4), ("bf16", 64, 16, 2),
+                                       ("f16", 64, 32, 8), ("bf16", 128, 16, 8)])
+def test_extend_e4m3_cache_matches_oracle(qd, D, BS, G):
+    """Draft runs of 1-16 tokens over an E4M3 cache (codes of N(0, 1) draws with a
+    per-tensor scale), partition edges and NaN codes past every context: every element
+    within 3e-2 + 3e-2 |ref|."""
+    lens = [1, 5, 17, 511, 512, 513, 530, 1030, 1600]
+    qlens = [1, 5, 3, 8, 2, 7, 1, 16, 13]
+    seed = zlib.crc32(repr(("e4m3", qd, D, BS, G)).encode()) % 10000
+    w = synthetic.custom(len(lens), 2 * G, 2, D, BS, "e4m3", qd, lens, seed)
+    eng = make_engine(w, DEV)
+    fill_cache(w, eng)
+    for s, L in enumerate(lens):
+        eng.extend(s, L)
+    eng.upload_tables()
+    _nan_tails(w, eng)
+    qs = np.concatenate([[0], np.cumsum(qlens)]).astype(np.int32)
+    q = synthetic.normal_values((int(qs[-1]), 2 * G, D), qd, seed + 7).to(DEV)
+    out = _run(w, eng, torch.from_numpy(qs).to(DEV), q, qs)
+    assert pa.last_device_error()[0] == 0
+    assert_close(out.double().cpu().numpy(), _ref_scaled(w, eng, q, qs), "e4m3", f"extend e4m3 {qd} D{D} BS{BS} G{G}")
+
+
+def test_extend_e4m3_long_runs_and_chunks():
+    """Long query runs over an E4M3 cache (a whole 700-token prompt, a 300-token chunk over
+    1300 tokens, a 256-token chunk at the end of 6000 tokens): the same kernel, merged
+    across 512-token partitions; sampled rows."""
+    lens, qlens = [700, 1300, 6000], [700, 300, 256]
+    w = synthetic.custom(3, 8, 2, 128, 32, "e4m3", "bf16", lens, 61)
+    eng = make_engine(w, DEV)
+    fill_cache(w, eng)
+    for s, L in enumerate(lens):
+        eng.extend(s, L)
+    eng.upload_tables()
+    _nan_tails(w, eng)
+    qs = np.concatenate([[0], np.cumsum(qlens)]).astype(np.int32)
+    q = synthetic.normal_values((int(qs[-1]), 8, 128), "bf16", 68).to(DEV)
+    out = _run(w, eng, torch.from_numpy(qs).to(DEV), q, qs)
+    assert pa.last_device_error()[0] == 0
+    rows = _sample_rows(qs, 8, 200, 61)
+    ref = _ref_scaled(w, eng, q, qs, rows=rows)
+    idx = tuple(np.array(rows).T)
+    assert_close(out.double().cpu().numpy()[idx], ref[idx], "e4m3", "e4m3 long runs")
+
+
+def test_extend_e4m3_single_query_agrees_with_decode():
+    """One query per sequence over an E4M3 cache: pa_extend and pa_decode compute the same
+    rows (within the E4M3 tolerance of each other)."""
+    lens = [40, 600, 1500, 3]
+    w = synthetic.custom(4, 8, 2, 128, 32, "e4m3", "bf16", lens, 63)
+    eng = make_engine(w, DEV)
+    fill_cache(w, eng)
+    for s, L in enumerate(lens):
+        eng.extend(s, L)
+    eng.upload_tables()
+    qs = np.arange(5, dtype=np.int32)
+    q = synthetic.normal_values((4, 8, 128), "bf16", 64).to(DEV)
+    ext = _run(w, eng, torch.from_numpy(qs).to(DEV), q, qs)
+    dec = torch.empty_like(q)
+    eng.run_decode(q, dec)
+    torch.cuda.synchronize()
+    a, b = ext.double().cpu().numpy(), dec.double().cpu().numpy()
+    assert np.all(np.abs(a - b) <= 3e-2 + 3e-2 * np.abs(b))
+
+
+def test_spec4_long_fp8_every_row():
+    """The benchmarked speculative-verification shape over the 32K E4M3 cache: 4 draft tokens
+    for each of 8 sequences of 32768 tokens (32/32 heads, 32-token blocks). EVERY (query,
+    head) row against the oracle on all host cores, at the E4M3 tolerance."""
+    from tests.gpu_cases import _device_to_shared, oracle_rows_parallel
+    w = synthetic.make("long_fp8")
+    eng = make_engine(w, DEV)
+    fill_cache(w, eng)
+    for s, L in enumerate(w.context_lens):
+        eng.extend(s, L)
+    eng.upload_tables()
+    qlens = [4] * w.num_seqs
+    qs = np.concatenate([[0], np.cumsum(qlens)]).astype(np.int32)
+    q = synthetic.normal_values((int(qs[-1]), w.num_q_heads, w.head_dim), w.q_dtype, w.seed + 11).to(DEV)
+    out = _run(w, eng, torch.from_numpy(qs).to(DEV), q, qs)
+    assert pa.last_device_error()[0] == 0
+    d = eng.cache.desc
+    shm_k, kc = _device_to_shared(eng.k_cache)
+    shm_v, vc = _device_to_shared(eng.v_cache)
+    try:
+        args = (codes_np(q), w.q_dtype, w.kv_dtype, d.k_scale, d.v_scale, eng.bt_host.astype(np.int64),
+                list(eng.lens), qs, w.scale)
+        groups = [[(t, h)] for s_ in range(w.num_seqs) for t in range(int(qs[s_]), int(qs[s_ + 1]))
+                  for h in range(0, w.num_q_heads, 1)]
+        groups = [sum(groups[i:i + 8], []) for i in range(0, len(groups), 8)]
+        ref = oracle_rows_parallel("extend", shm_k, shm_v, kc.shape, kc.itemsize, args, groups)
+    finally:
+        for shm in (shm_k, shm_v):
+            shm.close()
+            shm.unlink()
+    keys = sorted(ref)
+    assert len(keys) == int(qs[-1]) * w.num_q_heads
+    idx = tuple(np.array(keys).T)
+    want = np.stack([ref[r] for r in keys])
+    assert_close(out.double().cpu().numpy()[idx], want, "e4m3", "spec4 long fp8, every row")

@@ -73,3 +73,47 @@ def test_prefill_gqa_8x2k_full_size():
     """The benchmarked GQA prefill shapes (Llama-3-8B attention: 32 q heads over 8 kv heads,
     8 prompts x 2048 tokens): every cache slot bit-exact, sampled rows against the oracle."""
     run_prefill_case([2048] * 8, 32, 8, 16, "bf16", 4372, 120)
+
+
+@pytest.mark.parametrize("dt,BS,G", [("bf16", 32, 1), ("f16", 16, 4)])
+def test_prefill_into_e4m3_cache(dt, BS, G):
+    """Whole prompts into an E4M3 cache: every prompt slot holds the oracle's E4M3 encoding
+    of the prompt's K / V (x / scale, round to nearest even, saturating; scales chosen so
+    that the largest values saturate) and every output element matches the oracle's
+    attention over that cache within 3e-2 + 3e-2 |ref|."""
+    from oracle import attention as oatt
+    from oracle import cache_ops as oops
+    from tests.gpu_cases import assert_close, codes_np
+    lens = [1, 17, 130, 700, 257]
+    D, Hkv = 128, 2
+    Hq = Hkv * G
+    seed = zlib.crc32(repr(("prefill e4m3", dt, BS, G)).encode()) % 10000
+    w = synthetic.custom(len(lens), Hq, Hkv, D, BS, "e4m3", dt, lens, seed)
+    ks, vs = 3.5 / 448, 3.0 / 448
+    eng = make_engine(w, DEV, k_scale=ks, v_scale=vs)
+    eng.k_cache.fill_(0x7F)                     # NaN codes everywhere beforehand
+    eng.v_cache.fill_(0x7F)
+    k0, v0 = codes_np(eng.k_cache), codes_np(eng.v_cache)
+    for s, L in enumerate(lens):
+        eng.extend(s, L)
+    eng.upload_tables()
+    qs = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    T = int(qs[-1])
+    q = synthetic.normal_values((T, Hq, D), dt, seed + 7).to(DEV)
+    k = synthetic.normal_values((T, Hkv, D), dt, seed + 8).to(DEV)
+    v = synthetic.normal_values((T, Hkv, D), dt, seed + 9).to(DEV)
+    out = torch.full_like(q, float("nan"))
+    ws = torch.empty(pa.extend_workspace_size(w.num_seqs, T, Hq, D, eng.max_context_len), dtype=torch.uint8,
+                     device=DEV)
+    pa.prefill(q, k, v, eng.cache, torch.from_numpy(qs).to(DEV), eng.bt_dev, eng.lens_dev, eng.max_context_len,
+               w.scale, out, ws)
+    torch.cuda.synchronize()
+    assert pa.last_device_error()[0] == 0
+    bt = eng.bt_host.astype(np.int64)
+    slots = np.concatenate([bt[s, np.arange(L) // BS] * BS + np.arange(L) % BS for s, L in enumerate(lens)])
+    kc, vc = oops.reshape_and_cache(codes_np(k), codes_np(v), dt, slots, k0, v0, "e4m3", ks, vs)
+    gk, gv = codes_np(eng.k_cache), codes_np(eng.v_cache)
+    assert np.array_equal(gk[slots // BS, :, slots % BS, :], kc[slots // BS, :, slots % BS, :]), "k slots"
+    assert np.array_equal(gv[slots // BS, :, slots % BS, :], vc[slots // BS, :, slots % BS, :]), "v slots"
+    ref = oatt.paged_extend(codes_np(q), dt, kc, vc, "e4m3", ks, vs, bt, lens, qs, w.scale)
+    assert_close(out.double().cpu().numpy(), ref, "e4m3", f"prefill e4m3 {dt} BS{BS} G{G}")
