@@ -62,10 +62,17 @@ def kernel_traffic(workload: str, bytes_per_launch: float):
     try:
         with open(os.path.join(ROOT, "profiles", "partition_kernel_traffic.json")) as f:
             rec = json.load(f)
+        csrc = os.path.join(ROOT, "paged_kv_cache_436_b200", "csrc")
+        with open(os.path.join(csrc, "pa_decode.cu")) as f:
+            dec = f.read()
+        with open(os.path.join(csrc, "pa_device.cuh")) as f:
+            dev = f.read()
+        # the partition kernel's own source (from its banner to the merge kernel's) and the
+        # device helpers it uses: host code around it may change without a recapture
+        a, b = dec.index("// partition kernel"), dec.index("// log-sum-exp merge of partitions")
         h = hashlib.sha256()
-        for name in ("pa_decode.cu", "pa_device.cuh"):
-            with open(os.path.join(ROOT, "paged_kv_cache_436_b200", "csrc", name), "rb") as f:
-                h.update(f.read())
+        h.update(dec[a:b].encode())
+        h.update(dev.encode())
         if h.hexdigest() != rec["source_sha256"]:
             return None
         base = workload.split("[")[0]

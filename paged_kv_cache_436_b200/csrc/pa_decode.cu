@@ -672,6 +672,20 @@ pa_status validate_cache(const pa_cache_desc* c) {
   return PA_OK;
 }
 
+// Grouped query heads on the tensor cores (pa_extend.cu): the 16-row mma.sync kernel with one
+// query row per sequence, and the size of its workspace.
+pa_status decode_grouped_mma(int stage_mask, const void* q, int32_t q_dtype, int32_t num_seqs, int32_t num_q_heads,
+                             const pa_cache_desc* c, const int32_t* block_tables, int32_t max_blocks_per_seq,
+                             const int32_t* context_lens, int32_t max_context_len, float scale, void* out,
+                             void* workspace, size_t workspace_bytes, cudaStream_t s);
+size_t ext_ws_total(int S, int T, int Hq, int D, int max_parts);
+
+// Whether decode runs on the tensor cores: grouped query heads (G >= 4) over a 16-bit cache
+// in blocks of 16 or 32 tokens; otherwise the CUDA-core partition kernel.
+inline bool decode_on_mma(const pa_cache_desc* c, int G) {
+  return c->kv_dtype != PA_E4M3 && G >= 4 && (c->block_size == 16 || c->block_size == 32);
+}
+
 pa_status decode_impl(int stage_mask, const void* q, int32_t q_dtype, int32_t num_seqs,
                       int32_t num_q_heads, const pa_cache_desc* c, const int32_t* block_tables,
                       int32_t max_blocks_per_seq, const int32_t* context_lens,
@@ -693,6 +707,10 @@ pa_status decode_impl(int stage_mask, const void* q, int32_t q_dtype, int32_t nu
   const int D = c->head_dim, BS = c->block_size;
   const int max_parts = max_context_len > 0 ? (max_context_len + kPartitionTokens - 1) / kPartitionTokens : 1;
   if (max_parts > kMaxPartitions) return PA_ERR_ARG;   // merge weights live in 48 KB of smem
+  if (decode_on_mma(c, G))
+    return decode_grouped_mma(stage_mask, q, q_dtype, num_seqs, num_q_heads, c, block_tables, max_blocks_per_seq,
+                              context_lens, max_context_len, scale, out, workspace, workspace_bytes,
+                              static_cast<cudaStream_t>(stream));
   const WsLayout ws = ws_layout(num_seqs, num_q_heads, D, max_parts);
   if (workspace_bytes < ws.total) return PA_ERR_ARG;
   const Launch part = pick_partition(q_dtype, c->kv_dtype, D, BS, G);
@@ -786,7 +804,10 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t h
   if (num_seqs < 0 || num_q_heads <= 0 || head_dim <= 0 || max_context_len < 0) return 0;
   const int max_parts =
       max_context_len > 0 ? (max_context_len + pa::kPartitionTokens - 1) / pa::kPartitionTokens : 1;
-  return pa::ws_layout(num_seqs, num_q_heads, head_dim, max_parts).total;
+  // enough for either kernel: the grouped-head tensor-core path keeps a few more records
+  const size_t a = pa::ws_layout(num_seqs, num_q_heads, head_dim, max_parts).total;
+  const size_t b = pa::ext_ws_total(num_seqs, num_seqs, num_q_heads, head_dim, max_parts);
+  return a > b ? a : b;
 }
 
 pa_status pa_decode(const void* q, int32_t q_dtype, int32_t num_seqs, int32_t num_q_heads,

@@ -311,63 +311,91 @@ __device__ __forceinline__ float2 bf16x2_value(uint32_t w) {
   return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
 }
 
-// Pass 1 of the softmax: the maximum of one row's 128 scores in TMEM (this thread's lane),
-// columns past `vis` masked when kMask.
-template <bool kMask>
+// Keeps the compiler from moving the computation of v past this point (an empty asm that
+// reads it): the work on one TMEM chunk then overlaps the load of the next one.
+__device__ __forceinline__ void keep8(const float (&v)[8]) {
+  asm volatile("" ::"f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+}
+
+// Folds 32 scores (columns c0 .. c0 + 31 of the tile; past `vis` masked) into 8 maxima.
+__device__ __forceinline__ void tc_fold_max(const uint32_t (&r)[32], int c0, int vis, float (&m8)[8]) {
+  auto at = [&](int i) {
+    const float v = __uint_as_float(pin_after_wait(r[i]));
+    return c0 + i > vis ? -INFINITY : v;
+  };
+#pragma unroll
+  for (int i = 0; i < 32; i += 16)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) m8[e] = fmax3(m8[e], at(i + e), at(i + 8 + e));
+}
+
+// Pass 1 of the softmax: the maximum of one row's 128 causally masked scores in TMEM
+// (this thread's lane), 32 columns at a time with the next 32 in flight.
 __device__ __forceinline__ float tc_row_max(uint32_t addr, int vis) {
   float m8[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) m8[e] = -INFINITY;
-#pragma unroll
-  for (int h = 0; h < kTcTok / 64; ++h) {   // 64 columns at a time
-    uint32_t r[64];
-    tc_ld32_async(addr + h * 64, r);
-    tc_ld32_async(addr + h * 64 + 32, r + 32);
-    tc_wait_ld();
-    auto at = [&](int i) {
-      const float v = __uint_as_float(pin_after_wait(r[i]));
-      return kMask && h * 64 + i > vis ? -INFINITY : v;
-    };
-#pragma unroll
-    for (int i = 0; i < 64; i += 16)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) m8[e] = fmax3(m8[e], at(i + e), at(i + 8 + e));
-  }
+  uint32_t ra[32], rb[32];
+  tc_ld32_async(addr, ra);
+  tc_wait_ld();
+  tc_ld32_async(addr + 32, rb);
+  tc_fold_max(ra, 0, vis, m8);
+  keep8(m8);
+  tc_wait_ld();
+  tc_ld32_async(addr + 64, ra);
+  tc_fold_max(rb, 32, vis, m8);
+  keep8(m8);
+  tc_wait_ld();
+  tc_ld32_async(addr + 96, rb);
+  tc_fold_max(ra, 64, vis, m8);
+  keep8(m8);
+  tc_wait_ld();
+  tc_fold_max(rb, 96, vis, m8);
   return fmaxf(fmax3(m8[0], m8[1], m8[2]), fmax3(fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7]));
 }
 
-// Pass 2 of the softmax, 16 columns at a time: p = 2^(s * s_mul + nmb) of one row's 128
-// scores, written over them as 16-bit pairs (tokens 16 t .. 16 t + 15: P in columns
-// [16 t, 16 t + 8); with kLo the rounded remainder p - bf16(p) in [16 t + 8, 16 t + 16));
-// the binary32 p are added to l2 (four pair chains).
-template <int QD, bool kMask, bool kLo>
-__device__ __forceinline__ void tc_make_p(uint32_t addr, int vis, float s_mul, float nmb, float2 (&l2)[4]) {
+// Pass 2 on 16 scores (tokens 16 t .. 16 t + 15 of the tile, columns [16 t, 16 t + 16) of
+// S; past `vis` masked): p = 2^(s * s_mul + nmb) written over them as 16-bit pairs, P in
+// columns [16 t, 16 t + 8) and, with kLo, the rounded remainder p - bf16(p) in
+// [16 t + 8, 16 t + 16); the binary32 p are added to l2 (four pair chains).
+template <int QD, bool kLo>
+__device__ __forceinline__ void tc_make_p16(uint32_t addr, const uint32_t (&r)[16], int t, int vis, float s_mul,
+                                            float nmb, float2 (&l2)[4]) {
+  uint32_t wh[8], wl[8];
 #pragma unroll
-  for (int t = 0; t < kTcTok / 16; ++t) {   // tokens 16 t .. 16 t + 15: scores in columns [16 t, 16 t + 16)
-    uint32_t r[16];
-    tc_ld16_async(addr + t * 16, r);
-    tc_wait_ld();
-    uint32_t wh[8], wl[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int col = t * 16 + 2 * e;
-      float s0 = __uint_as_float(pin_after_wait(r[2 * e]));
-      float s1 = __uint_as_float(pin_after_wait(r[2 * e + 1]));
-      if (kMask) {
-        s0 = col > vis ? -INFINITY : s0;
-        s1 = col + 1 > vis ? -INFINITY : s1;
-      }
-      const float2 a = fma2(make_float2(s0, s1), s_mul, nmb);
-      const float p0 = ex2(a.x), p1 = ex2(a.y);
-      wh[e] = pack16x2<QD>(p0, p1);
-      l2[e & 3] = add2(l2[e & 3], make_float2(p0, p1));
-      if constexpr (kLo) {
-        const float2 hv = bf16x2_value(wh[e]);
-        wl[e] = pack16x2<QD>(p0 - hv.x, p1 - hv.y);
-      }
+  for (int e = 0; e < 8; ++e) {
+    const int col = t * 16 + 2 * e;
+    float s0 = __uint_as_float(pin_after_wait(r[2 * e]));
+    float s1 = __uint_as_float(pin_after_wait(r[2 * e + 1]));
+    s0 = col > vis ? -INFINITY : s0;
+    s1 = col + 1 > vis ? -INFINITY : s1;
+    const float2 a = fma2(make_float2(s0, s1), s_mul, nmb);
+    const float p0 = ex2(a.x), p1 = ex2(a.y);
+    wh[e] = pack16x2<QD>(p0, p1);
+    l2[e & 3] = add2(l2[e & 3], make_float2(p0, p1));
+    if constexpr (kLo) {
+      const float2 hv = bf16x2_value(wh[e]);
+      wl[e] = pack16x2<QD>(p0 - hv.x, p1 - hv.y);
     }
-    tc_st8(addr + t * 16, wh);
-    if constexpr (kLo) tc_st8(addr + t * 16 + 8, wl);
+  }
+  tc_st8(addr + t * 16, wh);
+  if constexpr (kLo) tc_st8(addr + t * 16 + 8, wl);
+}
+
+// Pass 2 over the row's 128 scores, 16 columns at a time with the next 16 in flight.
+template <int QD, bool kLo>
+__device__ __forceinline__ void tc_make_p(uint32_t addr, int vis, float s_mul, float nmb, float2 (&l2)[4]) {
+  uint32_t ra[16], rb[16];
+  tc_ld16_async(addr, ra);
+  tc_wait_ld();
+#pragma unroll 1
+  for (int t = 0; t < kTcTok / 16; t += 2) {
+    tc_ld16_async(addr + (t + 1) * 16, rb);
+    tc_make_p16<QD, kLo>(addr, ra, t, vis, s_mul, nmb, l2);
+    tc_wait_ld();
+    if (t + 2 < kTcTok / 16) tc_ld16_async(addr + (t + 2) * 16, ra);
+    tc_make_p16<QD, kLo>(addr, rb, t + 1, vis, s_mul, nmb, l2);
+    tc_wait_ld();
   }
 }
 
@@ -563,7 +591,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     bulk_wait_all();   // this thread's cache stores are complete before the kernel ends
   } else if (warp == kTcMmaWarp) {
-    // ---------------- MMA issue for both sets: S(0), S(1), P V(0), P V(1), ... ----------------
+    // ---------------- MMA issue for both sets ----------------
+    // Per set the products form a chain S(g), P(g) V(g), S(g + 1), ...: S(g + 1) overwrites
+    // the P that P(g) V(g) reads, so it waits for that product to complete. The sets are
+    // served in turn -- P V(set 0), S(set 0), P V(set 1), S(set 1), ... -- so that each
+    // set's next S follows its own P V as soon as possible while the other set's softmax
+    // runs, and the tensor core alternates between the two chains.
     const uint32_t idS = tc_idesc<QD>(0), idO = tc_idesc<QD>(1);
     TcUnit x[kTcSets];
     int j[kTcSets];
@@ -576,76 +609,81 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       live[c] = fresh_unit[c] = true;
     }
     bool ok = true;
-    while (ok && (live[0] || live[1])) {
-      bool pend[kTcSets] = {false, false};
-#pragma unroll
-      for (int c = 0; c < kTcSets; ++c) {
-        if (!ok || !live[c]) continue;
-        if (fresh_unit[c]) {
-          int u;
-          if (!(ok = next_unit(c, k[c], false, u))) break;
-          if (u < 0) {
-            live[c] = false;
-            continue;
-          }
-          x[c] = tc_unit(p, u);
-          j[c] = 0;
-          fresh_unit[c] = false;
-          if (!(ok = tc_wait_warp(&q_full[c], k[c] & 1, abort, 14, u))) break;
+    // S(g) of set c (taking the set's next unit first when the last one is done); false
+    // when the set has no more work (live[c] cleared) or on an abort (ok cleared)
+    auto issue_s = [&](int c) {
+      if (fresh_unit[c]) {
+        int u;
+        if (!(ok = next_unit(c, k[c], false, u))) return false;
+        if (u < 0) {
+          live[c] = false;
+          return false;
         }
-        // S(g) = Q K(g)^T into the set's S columns, once K(g) has landed and P(g-1) V(g-1)
-        // (which reads P from those columns) has completed
-        if (!(ok = tc_wait_warp(&k_full[c], g[c] & 1, abort, 16, int(g[c])) &&
-                   tc_wait_warp(&pv_done[c], (g[c] & 1) ^ 1, abort, 17, int(g[c]))))
-          break;
-        if (lane == 0) {
-          tc_fence_after();
-          const uint32_t qa = smem_addr(sm + c * TcSmem::kSet + TcSmem::kQ);
-          const uint32_t ka = smem_addr(sm + c * TcSmem::kSet + TcSmem::kK);
-#pragma unroll
-          for (int kk = 0; kk < kTcD / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * (kTcRows * 128) + (kk & 3) * 32;
-            tc_mma(tmem + c * 128, tc_desc(qa + off, 1024, 16), tc_desc(ka + off, 1024, 16), idS, kk > 0);
-          }
-          tc_commit(&s_full[c]);
-          tc_commit(&k_empty[c]);
-          if (j[c] + 1 == x[c].ntiles) tc_commit(&q_empty[c]);   // the Q buffer is free once this S completes
-        }
-        __syncwarp();
-        pend[c] = true;
+        x[c] = tc_unit(p, u);
+        j[c] = 0;
+        fresh_unit[c] = false;
+        if (!(ok = tc_wait_warp(&q_full[c], k[c] & 1, abort, 14, u))) return false;
       }
+      // once K(g) has landed and P(g-1) V(g-1), which reads P from the S columns, completed
+      if (!(ok = tc_wait_warp(&k_full[c], g[c] & 1, abort, 16, int(g[c])) &&
+                 tc_wait_warp(&pv_done[c], (g[c] & 1) ^ 1, abort, 17, int(g[c]))))
+        return false;
+      if (lane == 0) {
+        tc_fence_after();
+        const uint32_t qa = smem_addr(sm + c * TcSmem::kSet + TcSmem::kQ);
+        const uint32_t ka = smem_addr(sm + c * TcSmem::kSet + TcSmem::kK);
+#pragma unroll
+        for (int kk = 0; kk < kTcD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (kTcRows * 128) + (kk & 3) * 32;
+          tc_mma(tmem + c * 128, tc_desc(qa + off, 1024, 16), tc_desc(ka + off, 1024, 16), idS, kk > 0);
+        }
+        tc_commit(&s_full[c]);
+        tc_commit(&k_empty[c]);
+        if (j[c] + 1 == x[c].ntiles) tc_commit(&q_empty[c]);   // the Q buffer is free once this S completes
+      }
+      __syncwarp();
+      return true;
+    };
+    // O += P(g) V(g) (+ the remainder) of set c, once P is in TMEM and V(g) has landed; a
+    // unit's first product overwrites O, so it waits until the previous unit's O was read
+    auto issue_pv = [&](int c) {
+      if (!(ok = tc_wait_warp(&p_full[c], g[c] & 1, abort, 12, int(g[c])) &&
+                 tc_wait_warp(&v_full[c], g[c] & 1, abort, 13, int(g[c]))))
+        return;
+      if (j[c] == 0 && k[c] > 0 && !(ok = tc_wait_warp(&o_empty[c], (k[c] & 1) ^ 1, abort, 15, int(k[c])))) return;
+      const bool lo = p.lo_mode == kLoAlways ||
+                      (p.lo_mode == kLoAdaptive && *reinterpret_cast<volatile int*>(&lo_tile[c]) == int(g[c]));
+      if (lane == 0) {
+        tc_fence_after();
+        const uint32_t va = smem_addr(sm + c * TcSmem::kSet + TcSmem::kV);
+        const uint32_t d = tmem + 256 + c * 128, a = tmem + c * 128;
+#pragma unroll
+        for (int kk = 0; kk < kTcTok / 16; ++kk)   // P of tokens 16 kk .. 16 kk + 15
+          tc_mma_ts(d, a + 16 * kk, tc_desc(va + kk * 2048, 1024, kTcTok * 128), idO, (j[c] > 0 || kk > 0) ? 1u : 0u);
+        if (lo) {
+#pragma unroll
+          for (int kk = 0; kk < kTcTok / 16; ++kk)   // their remainders, 8 columns further
+            tc_mma_ts(d, a + 16 * kk + 8, tc_desc(va + kk * 2048, 1024, kTcTok * 128), idO, 1u);
+        }
+        tc_commit(&pv_done[c]);
+        if (j[c] + 1 == x[c].ntiles) tc_commit(&o_full[c]);
+      }
+      __syncwarp();
+      ++g[c];
+      if (++j[c] == x[c].ntiles) {
+        fresh_unit[c] = true;
+        ++k[c];
+      }
+    };
+    bool pend[kTcSets];
+#pragma unroll
+    for (int c = 0; c < kTcSets; ++c) pend[c] = ok && issue_s(c);
+    while (ok && (pend[0] || pend[1])) {
 #pragma unroll
       for (int c = 0; c < kTcSets; ++c) {
         if (!ok || !pend[c]) continue;
-        // O += P(g) V(g) (+ the remainder), once P is in TMEM and V(g) has landed; a unit's
-        // first product overwrites O, so it waits until the previous unit's O was read
-        if (!(ok = tc_wait_warp(&p_full[c], g[c] & 1, abort, 12, int(g[c])) &&
-                   tc_wait_warp(&v_full[c], g[c] & 1, abort, 13, int(g[c]))))
-          break;
-        if (j[c] == 0 && k[c] > 0 && !(ok = tc_wait_warp(&o_empty[c], (k[c] & 1) ^ 1, abort, 15, int(k[c])))) break;
-        const bool lo = p.lo_mode == kLoAlways ||
-                        (p.lo_mode == kLoAdaptive && *reinterpret_cast<volatile int*>(&lo_tile[c]) == int(g[c]));
-        if (lane == 0) {
-          tc_fence_after();
-          const uint32_t va = smem_addr(sm + c * TcSmem::kSet + TcSmem::kV);
-          const uint32_t d = tmem + 256 + c * 128, a = tmem + c * 128;
-#pragma unroll
-          for (int kk = 0; kk < kTcTok / 16; ++kk)   // P of tokens 16 kk .. 16 kk + 15
-            tc_mma_ts(d, a + 16 * kk, tc_desc(va + kk * 2048, 1024, kTcTok * 128), idO, (j[c] > 0 || kk > 0) ? 1u : 0u);
-          if (lo) {
-#pragma unroll
-            for (int kk = 0; kk < kTcTok / 16; ++kk)   // their remainders, 8 columns further
-              tc_mma_ts(d, a + 16 * kk + 8, tc_desc(va + kk * 2048, 1024, kTcTok * 128), idO, 1u);
-          }
-          tc_commit(&pv_done[c]);
-          if (j[c] + 1 == x[c].ntiles) tc_commit(&o_full[c]);
-        }
-        __syncwarp();
-        ++g[c];
-        if (++j[c] == x[c].ntiles) {
-          fresh_unit[c] = true;
-          ++k[c];
-        }
+        issue_pv(c);
+        pend[c] = ok && issue_s(c);
       }
     }
   } else {
@@ -669,12 +707,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int j = 0; j < x.ntiles; ++j, ++g) {
         if (!(ok = tc_wait_warp(&s_full[c], g & 1, abort, 18, u))) break;
         tc_fence_after();
-        // pass 1: the row maximum of the causally masked scores (8 independent chains); the
-        // mask only costs work in tiles where some row of the warp ends
+        // pass 1: the row maximum of the causally masked scores (8 independent chains)
         const int tp0 = x.t0 + j * kTcTok;
         const int vis = qpos - tp0;   // columns 0 .. vis of this tile are visible to the row
-        const bool masked = !__all_sync(kFull, vis >= kTcTok - 1);
-        const float mx = (masked ? tc_row_max<true>(t_row + c_s, vis) : tc_row_max<false>(t_row + c_s, vis)) * p.s_mul;
+        const float mx = tc_row_max(t_row + c_s, vis) * p.s_mul;
         const bool up = mx > m_ref + kTcRescale;
         const float corr = up ? ex2(m_ref - mx) : 1.f;   // 0 while nothing was accumulated
         if (up) {
@@ -697,14 +733,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // the rounded remainder p - bf16(p) in [16 t + 8, 16 t + 16))
         const float nmb = m_ref == -INFINITY ? 0.f : -m_ref;
         float2 l2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-        const bool lo_on = QD == PA_BF16 && p.lo_mode != kLoNone;
-        if (masked) {
-          if (lo_on) tc_make_p<QD, true, true>(t_row + c_s, vis, p.s_mul, nmb, l2);
-          else tc_make_p<QD, true, false>(t_row + c_s, vis, p.s_mul, nmb, l2);
-        } else {
-          if (lo_on) tc_make_p<QD, false, true>(t_row + c_s, vis, p.s_mul, nmb, l2);
-          else tc_make_p<QD, false, false>(t_row + c_s, vis, p.s_mul, nmb, l2);
-        }
+        tc_make_p<QD, QD == PA_BF16>(t_row + c_s, vis, p.s_mul, nmb, l2);
         l += ((l2[0].x + l2[0].y) + (l2[1].x + l2[1].y)) + ((l2[2].x + l2[2].y) + (l2[3].x + l2[3].y));
         // the remainder's product is issued when some row of the set has a weight above
         // kTcLoShare of its running sum (adaptive), or always

@@ -41,8 +41,12 @@ def test_every_declared_symbol_is_exported():
 
 def test_version_and_sizes():
     assert "sm_100a" in pa.version()
-    # plan (S+1 ints) + (m, l) + acc per (seq, q head, partition), each 256-byte aligned
-    assert pa.decode_workspace_size(8, 32, 128, 32768) == 256 + 8 * 32 * 64 * 2 * 4 + 8 * 32 * 64 * 128 * 4
+    # plan (S+1 ints) + (m, l) + acc per (seq, q head, partition), each 256-byte aligned; the
+    # grouped-head tensor-core decode adds its unit records (32 bytes per sequence and
+    # partition), the work counter and the chunk count per row
+    S, Hq, D, P = 8, 32, 128, 64
+    partials = 256 + S * Hq * P * 2 * 4 + S * Hq * P * D * 4
+    assert pa.decode_workspace_size(S, Hq, D, 512 * P) == partials + S * P * 32 + 256 + 256
     assert pa.decode_workspace_size(-1, 32, 128, 10) == 0
 
 

@@ -157,10 +157,16 @@ def test_traffic_is_reported_only_for_the_captured_kernel_source(tmp_path, monke
     ratio = rec["traffic_per_algorithmic_byte"]["llama13b_mix"]
     assert bench.kernel_traffic("llama13b_mix", 1.0e9) == pytest.approx(ratio * 1.0e9)
     assert bench.kernel_traffic("tiny", 1.0e9) is None                 # no capture for it
-    # a copy of the tree whose partition kernel differs by one byte: no traffic figure
+    # a copy of the tree: host code outside the partition kernel may change (the figure
+    # stays); one byte more inside the kernel's source drops it
     for d in ("profiles", os.path.join("paged_kv_cache_436_b200", "csrc")):
         shutil.copytree(os.path.join(bench.ROOT, d), tmp_path / d)
-    with open(tmp_path / "paged_kv_cache_436_b200" / "csrc" / "pa_decode.cu", "a") as f:
-        f.write("\n")
+    path = tmp_path / "paged_kv_cache_436_b200" / "csrc" / "pa_decode.cu"
+    with open(path, "a") as f:
+        f.write("\n// host code after the kernels\n")
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.kernel_traffic("llama13b_mix", 1.0e9) == pytest.approx(ratio * 1.0e9)
+    src = path.read_text()
+    i = src.index("// partition kernel")
+    path.write_text(src[:i] + "// partition kernel \n" + src[i + len("// partition kernel"):])
     assert bench.kernel_traffic("llama13b_mix", 1.0e9) is None

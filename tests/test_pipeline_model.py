@@ -9,7 +9,8 @@ asynchronous operations (TMA loads and stores, MMAs with their commits):
   through single buffers (and, for whole prompts, stores some tiles to the cache); the
   set's softmax warps, which read S(g) from TMEM, write P(g) over it, zero ragged V rows,
   rescale O, and read O out at the end of each unit;
-* one MMA issuer for both sets, alternating S(set 0), S(set 1), P V(set 0), P V(set 1).
+* one MMA issuer for both sets: S of each set's first tile, then in turn for each set
+  P V(g) and, once that product has completed, S(g + 1).
 
 A random scheduler interleaves the roles; asynchronous operations complete later, in
 issue order per issuer (a commit arrives once everything its thread issued before it is
@@ -171,74 +172,80 @@ def simulate(units, seed, fresh=False, mutant=None, warps=2):
     # ---------------- MMA issuer for both sets ----------------
     def mma():
         st = [{"live": True, "fresh": True, "j": 0, "g": 0, "k": 0, "u": None} for _ in range(SETS)]
-        while st[0]["live"] or st[1]["live"]:
-            pend = [False] * SETS
-            for c in range(SETS):
-                z = st[c]
-                if not z["live"]:
-                    continue
-                if z["fresh"]:
-                    u = yield from next_unit(c, z["k"])
-                    if u < 0:
-                        z["live"] = False
-                        continue
-                    z["u"], z["j"], z["fresh"] = u, 0, False
-                    yield ("wait", f"q_full{c}", z["k"] & 1)
-                g, u = z["g"], z["u"]
-                yield ("wait", f"k_full{c}", g & 1)
-                if mutant != "s_before_pv_done":
-                    yield ("wait", f"pv_done{c}", (g & 1) ^ 1)
 
-                def s_act(c=c, g=g, u=u):
-                    check(Kb[c] == g, f"S of tile {g} reads another K tile")
-                    check(Qb[c] == u, f"S of unit {u} reads the Q tile of unit {Qb[c]}")
-                    check(pv_done_t[c] >= g - 1, f"S({g}) overwrites P({g - 1}) while P V reads it")
+        def issue_s(c):
+            z = st[c]
+            if z["fresh"]:
+                u = yield from next_unit(c, z["k"])
+                if u < 0:
+                    z["live"] = False
+                    return False
+                z["u"], z["j"], z["fresh"] = u, 0, False
+                yield ("wait", f"q_full{c}", z["k"] & 1)
+            g, u = z["g"], z["u"]
+            yield ("wait", f"k_full{c}", g & 1)
+            if mutant != "s_before_pv_done":
+                yield ("wait", f"pv_done{c}", (g & 1) ^ 1)
 
-                def s_land(c=c, g=g):
-                    S[c] = ("S", g)
-                    P_writers[c] = set()
-                    s_done[c] = g
-                yield ("act", s_act)
-                yield ("async", f"s_full{c}", s_land)
-                yield ("async", f"k_empty{c}", None)
-                if z["j"] + 1 == units[u]:
-                    last_s_of_unit[(c, u)] = g
-                    yield ("async", f"q_empty{c}", None)
-                pend[c] = True
+            def s_act(c=c, g=g, u=u):
+                check(Kb[c] == g, f"S of tile {g} reads another K tile")
+                check(Qb[c] == u, f"S of unit {u} reads the Q tile of unit {Qb[c]}")
+                check(pv_done_t[c] >= g - 1, f"S({g}) overwrites P({g - 1}) while P V reads it")
+
+            def s_land(c=c, g=g):
+                S[c] = ("S", g)
+                P_writers[c] = set()
+                s_done[c] = g
+            yield ("act", s_act)
+            yield ("async", f"s_full{c}", s_land)
+            yield ("async", f"k_empty{c}", None)
+            if z["j"] + 1 == units[u]:
+                last_s_of_unit[(c, u)] = g
+                yield ("async", f"q_empty{c}", None)
+            return True
+
+        def issue_pv(c):
+            z = st[c]
+            g, u, j = z["g"], z["u"], z["j"]
+            if mutant != "pv_before_p":
+                yield ("wait", f"p_full{c}", g & 1)
+            yield ("wait", f"v_full{c}", g & 1)
+            if j == 0 and z["k"] > 0 and mutant != "o_overwrite_early":
+                yield ("wait", f"o_empty{c}", (z["k"] & 1) ^ 1)
+
+            def pv_act(c=c, g=g, u=u, j=j):
+                check(S[c] == ("P", g) and len(P_writers[c]) == warps, f"P V of tile {g} reads an unfinished P")
+                check(Vb[c] == g, f"P V of tile {g} reads another V tile")
+                if j == 0:
+                    check(not O_readers[c], f"O of set {c} restarted while unit {O[c]} is read")
+                    O[c] = u
+                else:
+                    check(O[c] == u, "P V into another unit's accumulator")
+                pv_issued[c] = g
+
+            def pv_land(c=c, g=g):
+                pv_done_t[c] = g
+            yield ("act", pv_act)
+            yield ("async", f"pv_done{c}", pv_land)
+            z["g"] += 1
+            z["j"] += 1
+            if z["j"] == units[u]:
+
+                def o_land(c=c):
+                    O_readers[c] = set(range(warps))
+                yield ("async", f"o_full{c}", o_land)
+                z["fresh"] = True
+                z["k"] += 1
+
+        pend = []
+        for c in range(SETS):
+            pend.append((yield from issue_s(c)))
+        while any(pend):
             for c in range(SETS):
                 if not pend[c]:
                     continue
-                z = st[c]
-                g, u, j = z["g"], z["u"], z["j"]
-                if mutant != "pv_before_p":
-                    yield ("wait", f"p_full{c}", g & 1)
-                yield ("wait", f"v_full{c}", g & 1)
-                if j == 0 and z["k"] > 0 and mutant != "o_overwrite_early":
-                    yield ("wait", f"o_empty{c}", (z["k"] & 1) ^ 1)
-
-                def pv_act(c=c, g=g, u=u, j=j):
-                    check(S[c] == ("P", g) and len(P_writers[c]) == warps, f"P V of tile {g} reads an unfinished P")
-                    check(Vb[c] == g, f"P V of tile {g} reads another V tile")
-                    if j == 0:
-                        check(not O_readers[c], f"O of set {c} restarted while unit {O[c]} is read")
-                        O[c] = u
-                    else:
-                        check(O[c] == u, "P V into another unit's accumulator")
-                    pv_issued[c] = g
-
-                def pv_land(c=c, g=g):
-                    pv_done_t[c] = g
-                yield ("act", pv_act)
-                yield ("async", f"pv_done{c}", pv_land)
-                z["g"] += 1
-                z["j"] += 1
-                if z["j"] == units[u]:
-
-                    def o_land(c=c):
-                        O_readers[c] = set(range(warps))
-                    yield ("async", f"o_full{c}", o_land)
-                    z["fresh"] = True
-                    z["k"] += 1
+                yield from issue_pv(c)
+                pend[c] = yield from issue_s(c)
 
     # ---------------- softmax warp w of set c ----------------
     def softmax(c, w):
