@@ -20,9 +20,10 @@
 //     by its own 1-D bulk copy into a padded row (head_dim * 2 + 16 bytes) instead;
 //   * long runs at head_dim 128 go to the tcgen05 kernel of pa_extend_tc.cu;
 //   * S = Q K^T and O += P V per 16-token slice; the S accumulators are reused as the
-//     P operand (rounded to the cache's 16-bit type; for bf16 the rounded remainder
-//     p - bf16(p) is a second operand, so P enters P V to within 2^-16; the running sum
-//     adds the same values); causal mask per row; online softmax in base 2;
+//     P operand (rounded to the cache's 16-bit type; for bf16, in a slice where some
+//     weight exceeds 1/8 of its running sum, the rounded remainder p - bf16(p) is a
+//     second operand, so such weights enter P V to within 2^-16; the running sum adds
+//     what enters the products); causal mask per row; online softmax in base 2;
 //   * one partition writes the output row, several write (max, sum, unnormalised row)
 //     for the log-sum-exp merge kernel, as in decode.
 #include <cuda_runtime.h>
@@ -232,15 +233,25 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi, float& lo_r, float
   return uint32_t(ua) | (uint32_t(ub) << 16);
 }
 
+// The share of a row's running sum above which a weight's bf16 rounding is corrected: a
+// later token can only lower a weight's share, so every weight left uncorrected ends
+// below this share of its row's total, one of many small independent rounding terms.
+constexpr float kLoShare = 0.125f;
+
 // The P operands of one 16-token slice (the S accumulator layout reused as the A
 // fragment): p = 2^(s - m) per element; hi = p rounded to the 16-bit type. For bf16 the
 // rounding (up to 2^-8 of p) can move an output by more than the parity tolerance when a
 // few weights dominate and their V values cancel, so the remainder p - hi (exact in
-// binary32) is rounded again into lo and multiplied as a second operand: hi + lo is p to
-// within 2^-16 of p. For f16 (rounding up to 2^-11 of p) lo is not formed. l adds hi + lo.
+// binary32) is rounded again into lo, a second operand: hi + lo is p to within 2^-16 of
+// p. lo is needed only where some weight exceeds kLoShare of its running sum; each lane
+// tests its own elements against its share of the row's sum (the lane holding a row's
+// largest weight sees at least the true share), and the returned warp-wide answer says
+// whether the caller multiplies lo. For f16 (rounding up to 2^-11 of p) lo is never
+// formed. l adds what enters the products.
 template <int QD>
-__device__ __forceinline__ void make_p_operands(const float (&sc)[2][4], const float (&base_m)[2], uint32_t (&hi)[4],
+__device__ __forceinline__ bool make_p_operands(const float (&sc)[2][4], const float (&base_m)[2], uint32_t (&hi)[4],
                                                 uint32_t (&lo)[4], float (&l)[2]) {
+  float lh[2] = {0.f, 0.f}, ll[2] = {0.f, 0.f}, pm[2] = {0.f, 0.f};
 #pragma unroll
   for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
@@ -248,15 +259,26 @@ __device__ __forceinline__ void make_p_operands(const float (&sc)[2][4], const f
       const float p0 = exp2f(sc[nt][2 * h] - base_m[h]), p1 = exp2f(sc[nt][2 * h + 1] - base_m[h]);
       float r0, r1;
       hi[nt * 2 + h] = pack2<QD>(p0, p1, r0, r1);
+      lh[h] += r0 + r1;
+      pm[h] = fmaxf(pm[h], fmaxf(p0, p1));
       if constexpr (QD == PA_BF16) {
         float e0, e1;
         lo[nt * 2 + h] = pack2<QD>(p0 - r0, p1 - r1, e0, e1);
-        l[h] += (r0 + e0) + (r1 + e1);
+        ll[h] += e0 + e1;
       } else {
         lo[nt * 2 + h] = 0u;
-        l[h] += r0 + r1;
       }
     }
+  if constexpr (QD != PA_BF16) {
+    l[0] += lh[0];
+    l[1] += lh[1];
+    return false;
+  }
+  const bool need = pm[0] > kLoShare * (l[0] + lh[0] + ll[0]) || pm[1] > kLoShare * (l[1] + lh[1] + ll[1]);
+  const bool any = __any_sync(kFull, need);
+  l[0] += lh[0] + (any ? ll[0] : 0.f);
+  l[1] += lh[1] + (any ? ll[1] : 0.f);
+  return any;
 }
 
 template <int D, int BS>
@@ -472,7 +494,7 @@ __global__ void __launch_bounds__(ExtCfg<D, BS>::kThreads)
         // rounded remainder p - bf16(p) as a second operand (hi + lo carries p to about
         // 2^-16); l adds what enters the products
         uint32_t pa[4], pl[4];
-        make_p_operands<QD>(sc, base_m, pa, pl, l);
+        const bool with_lo = make_p_operands<QD>(sc, base_m, pa, pl, l);
         // O += P V (V rows through ldmatrix.trans: two n-tiles of 8 dims per x4)
 #pragma unroll
         for (int np = 0; np < NT / 2; ++np) {
@@ -481,7 +503,7 @@ __global__ void __launch_bounds__(ExtCfg<D, BS>::kThreads)
           ldsm_x4_trans(b, Vs + ext_swz<BS>(trow, np * 2 + (lane >> 4)));
           mma16816<QD>(o[2 * np], pa, b[0], b[1]);
           mma16816<QD>(o[2 * np + 1], pa, b[2], b[3]);
-          if constexpr (QD == PA_BF16) {
+          if (with_lo) {
             mma16816<QD>(o[2 * np], pl, b[0], b[1]);
             mma16816<QD>(o[2 * np + 1], pl, b[2], b[3]);
           }
@@ -721,7 +743,7 @@ __global__ void __launch_bounds__(CoopCfg<D, BS>::kThreads) extend_coop_kernel(c
             base_m[h] = m[h] == -INFINITY ? 0.f : m[h];
           }
           uint32_t pa[4], pl[4];
-          make_p_operands<QD>(sc, base_m, pa, pl, l);
+          const bool with_lo = make_p_operands<QD>(sc, base_m, pa, pl, l);
 #pragma unroll
           for (int np = 0; np < NT / 2; ++np) {
             uint32_t b[4];
@@ -729,7 +751,7 @@ __global__ void __launch_bounds__(CoopCfg<D, BS>::kThreads) extend_coop_kernel(c
             ldsm_x4_trans(b, Vs + trow * C::kRowPad + (np * 16 + (lane >> 4) * 8) * 2);
             mma16816<QD>(o[2 * np], pa, b[0], b[1]);
             mma16816<QD>(o[2 * np + 1], pa, b[2], b[3]);
-            if constexpr (QD == PA_BF16) {
+            if (with_lo) {
               mma16816<QD>(o[2 * np], pl, b[0], b[1]);
               mma16816<QD>(o[2 * np + 1], pl, b[2], b[3]);
             }

@@ -50,12 +50,11 @@ constexpr int kTcSoftmaxWarps = kTcSets * kTcSetWarps;
 constexpr int kTcMmaWarp = kTcSoftmaxWarps;           // followed by one producer warp per set
 constexpr int kTcThreads = (kTcSoftmaxWarps + 1 + kTcSets) * 32;
 constexpr float kTcRescale = 8.f;       // log2 units
-constexpr float kTcLoShare = 0.125f;    // adaptive remainder: a weight above this share of the running sum
 
 // P V precision modes (ExtendParams::lo_mode)
 constexpr int kLoNone = 0;      // P rounded to the 16-bit type only (f16: rounding up to 2^-11 of p)
 constexpr int kLoAlways = 1;    // the bf16 remainder for every tile
-constexpr int kLoAdaptive = 2;  // the bf16 remainder for tiles with a weight above kTcLoShare
+constexpr int kLoAdaptive = 2;  // the bf16 remainder for tiles with a weight above kLoShare (pa_extend.cu)
 
 struct TcSmem {
   static constexpr int kTile = kTcRows * kTcD * 2;   // 32 KB: two 64-column halves of 16 KB
@@ -317,11 +316,13 @@ __device__ __forceinline__ void keep8(const float (&v)[8]) {
   asm volatile("" ::"f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
 }
 
-// Folds 32 scores (columns c0 .. c0 + 31 of the tile; past `vis` masked) into 8 maxima.
+// Folds 32 scores (columns c0 .. c0 + 31 of the tile; with kMask those past `vis` masked)
+// into 8 maxima.
+template <bool kMask>
 __device__ __forceinline__ void tc_fold_max(const uint32_t (&r)[32], int c0, int vis, float (&m8)[8]) {
   auto at = [&](int i) {
     const float v = __uint_as_float(pin_after_wait(r[i]));
-    return c0 + i > vis ? -INFINITY : v;
+    return kMask && c0 + i > vis ? -INFINITY : v;
   };
 #pragma unroll
   for (int i = 0; i < 32; i += 16)
@@ -329,8 +330,9 @@ __device__ __forceinline__ void tc_fold_max(const uint32_t (&r)[32], int c0, int
     for (int e = 0; e < 8; ++e) m8[e] = fmax3(m8[e], at(i + e), at(i + 8 + e));
 }
 
-// Pass 1 of the softmax: the maximum of one row's 128 causally masked scores in TMEM
-// (this thread's lane), 32 columns at a time with the next 32 in flight.
+// Pass 1 of the softmax: the maximum of one row's 128 scores in TMEM (this thread's lane;
+// with kMask those past `vis` masked), 32 columns at a time with the next 32 in flight.
+template <bool kMask>
 __device__ __forceinline__ float tc_row_max(uint32_t addr, int vis) {
   float m8[8];
 #pragma unroll
@@ -339,26 +341,26 @@ __device__ __forceinline__ float tc_row_max(uint32_t addr, int vis) {
   tc_ld32_async(addr, ra);
   tc_wait_ld();
   tc_ld32_async(addr + 32, rb);
-  tc_fold_max(ra, 0, vis, m8);
+  tc_fold_max<kMask>(ra, 0, vis, m8);
   keep8(m8);
   tc_wait_ld();
   tc_ld32_async(addr + 64, ra);
-  tc_fold_max(rb, 32, vis, m8);
+  tc_fold_max<kMask>(rb, 32, vis, m8);
   keep8(m8);
   tc_wait_ld();
   tc_ld32_async(addr + 96, rb);
-  tc_fold_max(ra, 64, vis, m8);
+  tc_fold_max<kMask>(ra, 64, vis, m8);
   keep8(m8);
   tc_wait_ld();
-  tc_fold_max(rb, 96, vis, m8);
+  tc_fold_max<kMask>(rb, 96, vis, m8);
   return fmaxf(fmax3(m8[0], m8[1], m8[2]), fmax3(fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7]));
 }
 
 // Pass 2 on 16 scores (tokens 16 t .. 16 t + 15 of the tile, columns [16 t, 16 t + 16) of
-// S; past `vis` masked): p = 2^(s * s_mul + nmb) written over them as 16-bit pairs, P in
-// columns [16 t, 16 t + 8) and, with kLo, the rounded remainder p - bf16(p) in
-// [16 t + 8, 16 t + 16); the binary32 p are added to l2 (four pair chains).
-template <int QD, bool kLo>
+// S; with kMask those past `vis` masked): p = 2^(s * s_mul + nmb) written over them as
+// 16-bit pairs, P in columns [16 t, 16 t + 8) and, with kLo, the rounded remainder
+// p - bf16(p) in [16 t + 8, 16 t + 16); the binary32 p are added to l2 (four pair chains).
+template <int QD, bool kMask, bool kLo>
 __device__ __forceinline__ void tc_make_p16(uint32_t addr, const uint32_t (&r)[16], int t, int vis, float s_mul,
                                             float nmb, float2 (&l2)[4]) {
   uint32_t wh[8], wl[8];
@@ -367,8 +369,10 @@ __device__ __forceinline__ void tc_make_p16(uint32_t addr, const uint32_t (&r)[1
     const int col = t * 16 + 2 * e;
     float s0 = __uint_as_float(pin_after_wait(r[2 * e]));
     float s1 = __uint_as_float(pin_after_wait(r[2 * e + 1]));
-    s0 = col > vis ? -INFINITY : s0;
-    s1 = col + 1 > vis ? -INFINITY : s1;
+    if (kMask) {
+      s0 = col > vis ? -INFINITY : s0;
+      s1 = col + 1 > vis ? -INFINITY : s1;
+    }
     const float2 a = fma2(make_float2(s0, s1), s_mul, nmb);
     const float p0 = ex2(a.x), p1 = ex2(a.y);
     wh[e] = pack16x2<QD>(p0, p1);
@@ -383,7 +387,7 @@ __device__ __forceinline__ void tc_make_p16(uint32_t addr, const uint32_t (&r)[1
 }
 
 // Pass 2 over the row's 128 scores, 16 columns at a time with the next 16 in flight.
-template <int QD, bool kLo>
+template <int QD, bool kMask, bool kLo>
 __device__ __forceinline__ void tc_make_p(uint32_t addr, int vis, float s_mul, float nmb, float2 (&l2)[4]) {
   uint32_t ra[16], rb[16];
   tc_ld16_async(addr, ra);
@@ -391,10 +395,10 @@ __device__ __forceinline__ void tc_make_p(uint32_t addr, int vis, float s_mul, f
 #pragma unroll 1
   for (int t = 0; t < kTcTok / 16; t += 2) {
     tc_ld16_async(addr + (t + 1) * 16, rb);
-    tc_make_p16<QD, kLo>(addr, ra, t, vis, s_mul, nmb, l2);
+    tc_make_p16<QD, kMask, kLo>(addr, ra, t, vis, s_mul, nmb, l2);
     tc_wait_ld();
     if (t + 2 < kTcTok / 16) tc_ld16_async(addr + (t + 2) * 16, ra);
-    tc_make_p16<QD, kLo>(addr, rb, t + 1, vis, s_mul, nmb, l2);
+    tc_make_p16<QD, kMask, kLo>(addr, rb, t + 1, vis, s_mul, nmb, l2);
     tc_wait_ld();
   }
 }
@@ -421,6 +425,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __shared__ uint64_t uq_full[kTcSets][4], uq_empty[kTcSets][4], bar_fin;
   __shared__ int uq[kTcSets][4];               // unit k of set c in slot k % 4
   __shared__ int lo_tile[kTcSets];             // adaptive remainder: the set's latest tile that needs it
+  __shared__ uint64_t vote_bar[kTcSets];       // the set's warps agree on the remainder of each tile
+  __shared__ int vote_word[kTcSets][3];        // ... through one word per tile, three in rotation
   __shared__ uint32_t tmem_slot;
   __shared__ int s_abort;
   volatile int* abort = &s_abort;
@@ -449,6 +455,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         mbar_init(&uq_empty[c][i], kTcSetWarps + 1);   // the set's softmax warps and the MMA warp
       }
       lo_tile[c] = -1;
+      mbar_init(&vote_bar[c], kTcSetWarps);
+      vote_word[c][0] = vote_word[c][1] = vote_word[c][2] = 0;
     }
     mbar_init(&bar_fin, 1);
     s_abort = 0;
@@ -707,10 +715,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int j = 0; j < x.ntiles; ++j, ++g) {
         if (!(ok = tc_wait_warp(&s_full[c], g & 1, abort, 18, u))) break;
         tc_fence_after();
-        // pass 1: the row maximum of the causally masked scores (8 independent chains)
+        // pass 1: the row maximum of the causally masked scores (8 independent chains); the
+        // mask costs work only in tiles where some row of the warp ends
         const int tp0 = x.t0 + j * kTcTok;
         const int vis = qpos - tp0;   // columns 0 .. vis of this tile are visible to the row
-        const float mx = tc_row_max(t_row + c_s, vis) * p.s_mul;
+        const bool masked = !__all_sync(kFull, vis >= kTcTok - 1);
+        const float mx = (masked ? tc_row_max<true>(t_row + c_s, vis) : tc_row_max<false>(t_row + c_s, vis)) * p.s_mul;
         const bool up = mx > m_ref + kTcRescale;
         const float corr = up ? ex2(m_ref - mx) : 1.f;   // 0 while nothing was accumulated
         if (up) {
@@ -728,17 +738,40 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             tc_st32(t_row + c_o + i * 32, o);
           }
         }
-        // pass 2, 16 columns at a time: P = 2^(s * scale - ref) as 16-bit pairs over the
-        // scores it was made from (tokens 16 t ..: P in columns [16 t, 16 t + 8), for bf16
-        // the rounded remainder p - bf16(p) in [16 t + 8, 16 t + 16))
         const float nmb = m_ref == -INFINITY ? 0.f : -m_ref;
+        // bf16: does this tile need P's remainder? Adaptive: when some row of the set has a
+        // weight above kLoShare of its running sum -- tested, before the sum of this tile is
+        // known, against the running sum plus the tile's largest weight (a lower bound of the
+        // final sum, so the test flags at least the tiles that need it). The set's four warps
+        // agree through one word and a 4-arrival barrier, since the product covers all rows.
+        bool lo = false;
+        if (QD == PA_BF16 && p.lo_mode == kLoAlways) {
+          lo = true;
+        } else if (QD == PA_BF16 && p.lo_mode == kLoAdaptive) {
+          const float pmax = ex2(mx + nmb);   // the row's largest weight in this tile (0: none visible)
+          const bool need = __any_sync(kFull, pmax > kLoShare * (l + pmax));
+          volatile int* vw = vote_word[c];
+          if (lane == 0) {
+            if (rw == 0) vw[(g + 1) % 3] = 0;   // the next tile's word: every warp read it two tiles ago
+            if (need) atomicOr(const_cast<int*>(&vw[g % 3]), 1);
+            mbar_arrive(&vote_bar[c]);
+          }
+          if (!(ok = tc_wait_warp(&vote_bar[c], g & 1, abort, 24, u))) break;
+          lo = vw[g % 3] != 0;
+          if (lo && rw == 0 && lane == 0) *reinterpret_cast<volatile int*>(&lo_tile[c]) = int(g);
+        }
+        // pass 2, 16 columns at a time: P = 2^(s * scale - ref) as 16-bit pairs over the
+        // scores it was made from (tokens 16 t ..: P in columns [16 t, 16 t + 8), with the
+        // remainder p - bf16(p) in [16 t + 8, 16 t + 16))
         float2 l2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-        tc_make_p<QD, QD == PA_BF16>(t_row + c_s, vis, p.s_mul, nmb, l2);
+        if (masked) {
+          if (lo) tc_make_p<QD, true, QD == PA_BF16>(t_row + c_s, vis, p.s_mul, nmb, l2);
+          else tc_make_p<QD, true, false>(t_row + c_s, vis, p.s_mul, nmb, l2);
+        } else {
+          if (lo) tc_make_p<QD, false, QD == PA_BF16>(t_row + c_s, vis, p.s_mul, nmb, l2);
+          else tc_make_p<QD, false, false>(t_row + c_s, vis, p.s_mul, nmb, l2);
+        }
         l += ((l2[0].x + l2[0].y) + (l2[1].x + l2[1].y)) + ((l2[2].x + l2[2].y) + (l2[3].x + l2[3].y));
-        // the remainder's product is issued when some row of the set has a weight above
-        // kTcLoShare of its running sum (adaptive), or always
-        if (p.lo_mode == kLoAdaptive && __any_sync(kFull, ex2(mx + nmb) > kTcLoShare * l) && lane == 0)
-          *reinterpret_cast<volatile int*>(&lo_tile[c]) = int(g);
         // V rows past the visible tokens (cache bytes beyond the context, or stale rows of
         // blocks not loaded) are zeroed, so that 0-weighted rows cannot bring a NaN into O
         const int rem = x.nvis - j * kTcTok;

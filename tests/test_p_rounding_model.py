@@ -14,7 +14,8 @@ score scales from flat to peaked (scale * sqrt(D) = 1, 4, 12):
   p - bf16(p) as a second product for every tile where some row of the 128 has a weight
   above 1/8 of its running sum -- stays inside for every element;
 * the mma.sync kernels' arithmetic -- 16-token slices, the running maximum, P and its bf16
-  remainder always, the running sum over what enters the products -- stays inside;
+  remainder for every slice where some row has a weight above 1/8 of its running sum,
+  the running sum over what enters the products -- stays inside;
 * f16 P (rounding up to 2^-11 of p) stays inside without a remainder.
 It runs no GPU code.
 """
@@ -60,9 +61,12 @@ def tcgen05_arithmetic(q, K, V, qpos, scale, dt, remainder):
     return _round(O / l[:, None], dt), flagged
 
 
-def mma_sync_arithmetic(q, K, V, qpos, scale, dt):
-    """16-token slices, the running maximum (rescale whenever it grows), P and its bf16
-    remainder, the running sum over what enters the products."""
+def mma_sync_arithmetic(q, K, V, qpos, scale, dt, adaptive=True):
+    """16-token slices, the running maximum (rescale whenever it grows), P and, for a
+    slice where some row's largest weight exceeds 1/8 of its running sum (adaptive) or
+    always, its bf16 remainder; the running sum over what enters the products. (The
+    kernel decides per warp from each lane's share of a row, which flags at least the
+    slices this row-wise rule flags.)"""
     s_mul = np.float32(scale * 1.4426950408889634)
     R, D = q.shape
     m = np.full(R, -np.inf, np.float32)
@@ -80,7 +84,11 @@ def mma_sync_arithmetic(q, K, V, qpos, scale, dt):
         p = np.exp2(S - np.where(m == -np.inf, 0, m)[:, None]).astype(np.float32)
         P = _round(p, dt)
         if dt == "bf16":
-            P = P + _round(p - P, dt)
+            rem = _round(p - P, dt)
+            with np.errstate(invalid="ignore"):
+                need = np.any(p.max(axis=1) > SHARE * (l + (P + rem).sum(axis=1)))
+            if need or not adaptive:
+                P = P + rem
         l = l + P.sum(axis=1)
         O = O + P @ V[lo:hi]
     return _round(O / l[:, None], dt)

@@ -7,8 +7,9 @@ asynchronous operations (TMA loads and stores, MMAs with their commits):
 * per set c (two sets share the tensor core, each working on its own units): a producer
   that takes the set's units from the queue, loads their Q and streams K and V tiles
   through single buffers (and, for whole prompts, stores some tiles to the cache); the
-  set's softmax warps, which read S(g) from TMEM, write P(g) over it, zero ragged V rows,
-  rescale O, and read O out at the end of each unit;
+  set's softmax warps, which read S(g) from TMEM, agree whether the tile needs P's
+  remainder (a word per tile, three in rotation, and a barrier), write P(g) over S, zero
+  ragged V rows, rescale O, and read O out at the end of each unit;
 * one MMA issuer for both sets: S of each set's first tile, then in turn for each set
   P V(g) and, once that product has completed, S(g + 1).
 
@@ -70,7 +71,8 @@ def simulate(units, seed, fresh=False, mutant=None, warps=2):
     B = {}
     for c in range(SETS):
         for n, cnt in (("s_full", 1), ("p_full", warps), ("pv_done", 1), ("k_full", 1), ("v_full", 1),
-                       ("k_empty", 1), ("q_full", 1), ("q_empty", 1), ("o_full", 1), ("o_empty", warps)):
+                       ("k_empty", 1), ("q_full", 1), ("q_empty", 1), ("o_full", 1), ("o_empty", warps),
+                       ("vote", warps)):
             B[f"{n}{c}"] = Bar(f"{n}{c}", cnt)
         for i in range(4):
             B[f"uq_full{c}_{i}"] = Bar(f"uq_full{c}_{i}", 1)
@@ -89,6 +91,9 @@ def simulate(units, seed, fresh=False, mutant=None, warps=2):
     pv_issued = [-1] * SETS
     stores = [0] * SETS               # cache stores still reading the set's K / V buffers
     uq = [[None] * 4 for _ in range(SETS)]
+    vote_word = [[0, 0, 0] for _ in range(SETS)]   # the remainder vote, three words in rotation
+    vote_need = [{} for _ in range(SETS)]          # tile -> OR of the warps' needs
+    vote_seen = [{} for _ in range(SETS)]          # tile -> the answers the warps read
     units_done = []
     queue = {"next": 0}
     n_units = len(units)
@@ -262,6 +267,26 @@ def simulate(units, seed, fresh=False, mutant=None, warps=2):
                     yield ("act", lambda c=c, g=g: check(pv_done_t[c] >= g - 1 and pv_issued[c] == g - 1,
                                                          "O rescaled under a P V"))
 
+                # the remainder vote: warp 0 clears the next tile's word, every warp ORs its
+                # need into this tile's word, arrives, waits for the others, reads the answer
+                need = rng.random() < 0.3
+                if w == 0:
+                    slot = (g + 1) % 3 if mutant != "vote_clear_wrong_word" else g % 3
+                    yield ("act", lambda c=c, slot=slot: vote_word[c].__setitem__(slot, 0))
+
+                def vote(c=c, g=g, need=need):
+                    vote_need[c][g] = vote_need[c].get(g, False) or need
+                    if need:
+                        vote_word[c][g % 3] = 1
+                yield ("act", vote)
+                yield ("arrive", f"vote{c}")
+                if mutant != "vote_not_waited":
+                    yield ("wait", f"vote{c}", g & 1)
+
+                def read_vote(c=c, g=g):
+                    vote_seen[c].setdefault(g, []).append(vote_word[c][g % 3] != 0)
+                yield ("act", read_vote)
+
                 def p_write(c=c, g=g, w=w):
                     check(pv_done_t[c] >= g - 1, f"P({g}) written over P({g - 1}) while P V reads it")
                     S[c] = ("P", g)
@@ -334,6 +359,9 @@ def simulate(units, seed, fresh=False, mutant=None, warps=2):
     else:
         raise Race("no progress bound reached")
     check(sorted(units_done) == list(range(n_units)), "not every unit finished")
+    for c in range(SETS):
+        for g, seen in vote_seen[c].items():
+            check(all(v == vote_need[c][g] for v in seen), f"set {c} disagreed on the remainder of tile {g}")
     check(all(v == 0 for v in stores), "cache stores still in flight at the end")
 
 
@@ -361,6 +389,8 @@ def test_schedule_with_four_softmax_warps_per_set():
     ("pv_before_p", False),          # P V issued before every warp has written P
     ("o_read_early", False),         # O read out before the unit's last P V completed
     ("zero_before_v_lands", False),  # V rows zeroed before the tile's load has landed
+    ("vote_not_waited", False),      # the remainder vote read before every warp has voted
+    ("vote_clear_wrong_word", False),  # warp 0 clears the word of the tile being voted on
     ("store_not_waited", True),      # a K/V buffer reloaded while a cache store still reads it
 ])
 def test_planted_schedule_mistakes_are_caught(mutant, fresh):
