@@ -8,61 +8,77 @@
 //     512-token partition, chosen by the host so that there are enough units to fill
 //     the GPU (the whole context when there are, then no merge pass at all); the plan
 //     kernel writes one record per (sequence, tile, chunk);
-//   * one persistent CTA per SM runs two independent pipelines ("sets") that share the
-//     tensor core: each set takes its own units from the global queue and has its own
-//     Q, K and V buffers in shared memory and its own S and O accumulators in TMEM
-//     (S of set c in columns [128 c, 128 c + 128), O in [256 + 128 c, ...)). While one
-//     set's softmax works on its scores, the tensor core runs the other set's MMAs;
-//   * warps: 4 softmax warps per set (thread = one row of the tile, all 128 columns, so
-//     no two warps ever combine a row), one MMA-issue warp for both sets, and one
-//     producer warp per set that takes its units, loads Q (one 3-D TMA box per 64-dim
-//     half: 64 dims x G heads x 128 / G queries) and streams K and V tiles (2-D TMA,
-//     one box per (cache block, 64-dim half), 128B swizzle, no multicast);
+//   * one persistent CTA per SM takes units from a global queue. Its TMEM holds three S
+//     buffers (tile g of the CTA's sequence of K/V tiles in buffer g % 3, columns
+//     [128 b, 128 b + 128)) and O (columns [384, 512)); shared memory holds the unit's Q
+//     and two buffers each for K and V tiles (tile g in buffer g % 2);
+//   * warps: 8 softmax warps in pairs -- warp w owns the 32 rows of TMEM lane quarter
+//     w % 4 (a warp can only reach its own quarter) and columns [64 h, 64 h + 64) of each
+//     tile, h = w / 4; the two warps of a quarter exchange their row maxima (and running
+//     sums) through shared memory and a two-arrival barrier -- one MMA-issue warp, a K
+//     producer (takes the units, loads Q: one 3-D TMA box per 64-dim half, 64 dims x G
+//     heads x 128 / G queries, and streams K) and a V producer (2-D TMA, one box per
+//     (cache block, 64-dim half), 128B swizzle, no multicast);
 //   * S = Q K^T (both operands K-major in shared memory). The softmax writes P over its
 //     own scores in TMEM as 16-bit pairs, and O += P V takes P from TMEM (A operand)
-//     and V in its [token][dim] cache layout (MN-major B operand). Per set the issue
-//     order is S(g), P(g) V(g), S(g + 1) (which waits for P(g) V(g): it overwrites the
-//     P it reads); the MMA warp alternates S(set 0), S(set 1), P V(set 0), P V(set 1);
+//     and V in its [token][dim] cache layout (MN-major B operand). S(g) is issued once
+//     K(g) has landed and P(g - 3) V(g - 3), which read its buffer, completed, so the
+//     scores of the next tiles are ready while the softmax works on tile g; P(g) V(g) once
+//     the softmax has written P(g). The MMA warp tests the barriers without blocking and
+//     issues each product's 8 MMAs from one block of instructions;
 //   * the softmax keeps a reference maximum that moves only when the row maximum passes
 //     it by more than 2^8 (O and the running sum are then rescaled; every p stays below
 //     2^8). For bf16, p rounded to bf16 can leave the parity tolerance when a few
 //     weights dominate and their V values cancel, so the rounded remainder
-//     p - bf16(p) goes into the other 64 columns of S and a second P V product adds it
-//     (hi + lo carries p to within 2^-16): for every tile, or only for tiles where some
-//     row has a weight above 1/8 of its running sum (a later tile can only lower that
-//     share, so every unadjusted weight ends below 1/8 of the row's total);
-//   * a unit that covers a row's whole context writes the output row; otherwise it
-//     writes (max, sum, unnormalised row) for the log-sum-exp merge kernel.
+//     p - bf16(p) goes into the other 64 columns of each token group of S and a second
+//     P V product adds it (hi + lo carries p to within 2^-16): for every tile, or only
+//     for tiles where some row has a weight above 1/8 of its running sum (a later tile
+//     can only lower that share, so every unadjusted weight ends below 1/8 of the row's
+//     total) -- the warps whose rows do not need it write zeros there;
+//   * a unit that covers a row's whole context writes the output row (staged through
+//     shared memory so that each store covers whole 128-byte row segments); otherwise it
+//     writes (max, sum, unnormalised row) for the log-sum-exp merge kernel. A unit's O is
+//     read after the first tile of the next unit, while the unit's last P V runs, and is
+//     released before the rows are written.
 // Every wait is bounded; on a timeout the kernel records it, every role stops, the MMA
 // and load issuers drain what they issued, and the TMEM is freed.
 #include <cstdlib>
 #include <cstring>
+#include <type_traits>
 
 namespace pa {
 
 constexpr int kTcRows = 128;            // query rows per unit (TMEM lanes)
 constexpr int kTcTok = 128;             // tokens per K/V tile
+constexpr int kTcHalf = kTcTok / 2;     // columns of a tile per softmax warp
 constexpr int kTcD = 128;               // head_dim of this path
-constexpr uint32_t kTcTmemCols = 512;   // S of the two sets in [0, 256), their O in [256, 512)
-constexpr int kTcSets = 2;              // independent pipelines sharing the tensor core
-constexpr int kTcSetWarps = 4;          // softmax warps per set: one thread per row
-constexpr int kTcSoftmaxWarps = kTcSets * kTcSetWarps;
-constexpr int kTcMmaWarp = kTcSoftmaxWarps;           // followed by one producer warp per set
-constexpr int kTcThreads = (kTcSoftmaxWarps + 1 + kTcSets) * 32;
+constexpr int kTcSBufs = 3;             // S buffers in TMEM (tile g in buffer g % 3)
+constexpr int kTcKvBufs = 2;            // K and V buffers in shared memory (tile g in buffer g % 2)
+constexpr uint32_t kTcOCol = kTcSBufs * kTcTok;   // O after the S buffers: 384 + 128 = 512 columns
+constexpr uint32_t kTcTmemCols = 512;
+constexpr int kTcQuarters = 4;          // row groups of 32 (a warp reads the TMEM lanes of its quarter)
+constexpr int kTcSoftmaxWarps = 2 * kTcQuarters;      // warp w: rows of quarter w % 4, column half w / 4
+constexpr int kTcMmaWarp = kTcSoftmaxWarps;           // then the K producer and the V producer
+constexpr int kTcKWarp = kTcMmaWarp + 1, kTcVWarp = kTcMmaWarp + 2;
+constexpr int kTcThreads = (kTcSoftmaxWarps + 3) * 32;
 constexpr float kTcRescale = 8.f;       // log2 units
+static_assert(kTcOCol + kTcD == kTcTmemCols, "three S buffers and O fill the TMEM");
 
 // P V precision modes (ExtendParams::lo_mode)
 constexpr int kLoNone = 0;      // P rounded to the 16-bit type only (f16: rounding up to 2^-11 of p)
 constexpr int kLoAlways = 1;    // the bf16 remainder for every tile
 constexpr int kLoAdaptive = 2;  // the bf16 remainder for tiles with a weight above kLoShare (pa_extend.cu)
 
+// Shared memory: the Q tile and two buffers each for K and V tiles, every tile kept as two
+// 128B-swizzled halves of 64 columns (dims); then the softmax warps' output staging rows.
 struct TcSmem {
-  static constexpr int kTile = kTcRows * kTcD * 2;   // 32 KB: two 64-column halves of 16 KB
-  static constexpr int kQ = 0, kK = kTile, kV = 2 * kTile;
-  static constexpr int kSet = 3 * kTile;             // Q, K and V of one set
-  static constexpr int kBytes = kTcSets * kSet + 1024;   // 193 KB with the alignment slack
+  static constexpr int kQTile = kTcRows * kTcD * 2;    // 32 KB: two halves of 16 KB
+  static constexpr int kKvTile = kTcTok * kTcD * 2;    // 32 KB: two halves of 16 KB
+  static constexpr int kQ = 0, kK = kQTile, kV = kQTile + kTcKvBufs * kKvTile;
+  static constexpr int kStageWarp = 32 * kTcHalf * 2;  // 4 KB: a softmax warp's 32 output rows (its 64 dims)
+  static constexpr int kStage = kV + kTcKvBufs * kKvTile;
+  static constexpr int kBytes = kStage + kTcSoftmaxWarps * kStageWarp + 1024;   // 193 KB with the alignment slack
 };
-static_assert(kTcRows == kTcTok, "Q, K and V tiles share one swizzled layout");
 
 // Shared-memory matrix descriptor: 128B swizzle, sm_100 descriptor version.
 __device__ __forceinline__ uint64_t tc_desc(uint32_t saddr, uint32_t sbo, uint32_t lbo) {
@@ -75,20 +91,68 @@ __device__ __forceinline__ uint64_t tc_desc(uint32_t saddr, uint32_t sbo, uint32
 }
 
 // Instruction descriptor of kind::f16: f32 accumulate, A and B both bf16 or both f16,
-// A K-major, B K-major (b_mn = 0) or MN-major (b_mn = 1), M = N = 128.
+// A K-major, B K-major (b_mn = 0) or MN-major (b_mn = 1), M = 128, N = n.
 template <int QD>
-__device__ __forceinline__ uint32_t tc_idesc(uint32_t b_mn) {
+__device__ __forceinline__ uint32_t tc_idesc(uint32_t b_mn, uint32_t n) {
   constexpr uint32_t fmt = QD == PA_BF16 ? 1u : 0u;
-  return (1u << 4) | (fmt << 7) | (fmt << 10) | (b_mn << 16) | (uint32_t(kTcTok >> 3) << 17) |
-         (uint32_t(kTcRows >> 4) << 24);
+  return (1u << 4) | (fmt << 7) | (fmt << 10) | (b_mn << 16) | ((n >> 3) << 17) | (uint32_t(kTcRows >> 4) << 24);
 }
 
-__device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
-  const uint32_t z = 0;
+// S = Q K^T of one tile: the 8 MMAs of K = 16 over head_dim 128, issued from one block
+// (descriptors advanced by immediates: a separately computed descriptor per MMA costs the
+// issuing thread more time than the MMA takes). a0 / b0 describe dims 0 .. 15 of Q and K;
+// dims 16 k .. lie 32 k bytes into the first 64-column half (k < 4) or one half (16 KB)
+// further -- descriptor addresses count 16-byte units.
+static_assert(kTcRows * 128 / 16 == 1024 && kTcTok * 128 / 16 == 1024, "descriptor steps of tc_mma_s8");
+__device__ __forceinline__ void tc_mma_s8(uint32_t tmem_d, uint64_t a0, uint64_t b0, uint32_t idesc) {
+  const uint32_t zero = 0;
   asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n\t}" ::"r"(tmem_d),
-      "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(z)
+      "{\n\t.reg .pred p;\n\t.reg .b64 a, b;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+      "add.s64 a, %1, 2;\n\tadd.s64 b, %2, 2;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, 1;\n\t"
+      "add.s64 a, %1, 4;\n\tadd.s64 b, %2, 4;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, 1;\n\t"
+      "add.s64 a, %1, 6;\n\tadd.s64 b, %2, 6;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, 1;\n\t"
+      "add.s64 a, %1, 1024;\n\tadd.s64 b, %2, 1024;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, 1;\n\t"
+      "add.s64 a, %1, 1026;\n\tadd.s64 b, %2, 1026;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, 1;\n\t"
+      "add.s64 a, %1, 1028;\n\tadd.s64 b, %2, 1028;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, 1;\n\t"
+      "add.s64 a, %1, 1030;\n\tadd.s64 b, %2, 1030;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, 1;\n\t}" ::"r"(tmem_d),
+      "l"(a0), "l"(b0), "r"(idesc), "r"(zero)
+      : "memory");
+}
+
+// O += P V of one tile with P (the A operand) in TMEM: 8 MMAs of K = 16 tokens, A at TMEM
+// columns tmem_a + 16 t (8 columns of 16-bit pairs each), B = V rows 16 t .. 16 t + 15,
+// 2 KB apart (128 descriptor units). acc0 = 0 makes the first product overwrite O.
+static_assert(kTcTok == 128, "tc_mma_pv8 covers one 128-token tile");
+__device__ __forceinline__ void tc_mma_pv8(uint32_t tmem_d, uint32_t tmem_a, uint64_t b0, uint32_t idesc,
+                                           uint32_t acc0) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 b;\n\t.reg .b32 t;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+      "add.s32 t, %1, 16;\n\tadd.s64 b, %2, 128;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [t], b, %3, 1;\n\t"
+      "add.s32 t, %1, 32;\n\tadd.s64 b, %2, 256;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [t], b, %3, 1;\n\t"
+      "add.s32 t, %1, 48;\n\tadd.s64 b, %2, 384;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [t], b, %3, 1;\n\t"
+      "add.s32 t, %1, 64;\n\tadd.s64 b, %2, 512;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [t], b, %3, 1;\n\t"
+      "add.s32 t, %1, 80;\n\tadd.s64 b, %2, 640;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [t], b, %3, 1;\n\t"
+      "add.s32 t, %1, 96;\n\tadd.s64 b, %2, 768;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [t], b, %3, 1;\n\t"
+      "add.s32 t, %1, 112;\n\tadd.s64 b, %2, 896;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [t], b, %3, 1;\n\t}" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(b0), "r"(idesc), "r"(acc0)
       : "memory");
 }
 
@@ -100,24 +164,9 @@ __device__ __forceinline__ void tc_commit(uint64_t* bar) {
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// 32 consecutive columns of this warp's 32 lanes (warp-collective).
-__device__ __forceinline__ void tc_ld32(uint32_t addr, float* v) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(addr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-// The same load without its wait: issue several, then one tc_wait_ld(), then read the
-// registers through pin_after_wait() so that no use is scheduled before the wait.
+// 32 consecutive columns of this warp's 32 lanes (warp-collective), without the wait:
+// issue several, then one tc_wait_ld(), then read the registers through pin_after_wait()
+// so that no use is scheduled before the wait.
 __device__ __forceinline__ void tc_ld32_async(uint32_t addr, uint32_t* r) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
@@ -132,25 +181,6 @@ __device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sy
 __device__ __forceinline__ uint32_t pin_after_wait(uint32_t x) {
   asm volatile("" : "+r"(x));
   return x;
-}
-
-__device__ __forceinline__ void tc_st32(uint32_t addr, const float* v) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(addr),
-      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
-      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
-      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
-      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
-      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
-      "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
-      "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
-      "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
-      "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
-      "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
-      "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
-      : "memory");
-  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 // max(a, b, c) in one instruction (sm_100 three-input max; a NaN operand is ignored as by fmaxf).
@@ -204,10 +234,10 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
-// Byte offset of 16-byte chunk c (0..15) of row r in a [128 x 128] 16-bit tile kept
-// as two 128B-swizzled K-major halves of 64 columns (8-row atoms of 1 KB).
-__device__ __forceinline__ uint32_t tc_swz(int r, int c) {
-  return uint32_t((c >> 3) * (kTcRows * 128) + (r >> 3) * 1024 + (r & 7) * 128 + (((c & 7) ^ (r & 7)) << 4));
+// Byte offset of 16-byte chunk c (0..15) of row r in a K / V tile ([128 tokens x 128]
+// 16-bit values kept as two 128B-swizzled halves of 64 columns, 8-row atoms of 1 KB).
+__device__ __forceinline__ uint32_t tc_swz_kv(int r, int c) {
+  return uint32_t((c >> 3) * (kTcTok * 128) + (r >> 3) * 1024 + (r & 7) * 128 + (((c & 7) ^ (r & 7)) << 4));
 }
 
 // Geometry of one work unit as every role of the CTA computes it.
@@ -255,16 +285,19 @@ __device__ __forceinline__ bool tc_wait_warp(uint64_t* bar, uint32_t parity, vol
   return __all_sync(kFull, tc_wait(bar, parity, abort, where, u));
 }
 
-
-// O += P V with P (the A operand) in TMEM: M = 128 lanes, K = 16 per instruction (8
-// columns of bf16 / f16 pairs), B from shared memory.
-__device__ __forceinline__ void tc_mma_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t b, uint32_t idesc, uint32_t acc) {
+// Non-blocking test: has the phase with this parity completed (as this thread sees it)?
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
   asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
-      "r"(tmem_a), "l"(b), "r"(idesc), "r"(acc)
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
       : "memory");
+  return ok != 0;
 }
+
 
 // 16 consecutive 32-bit columns of this warp's 32 lanes, without the wait (the registers
 // are read at issue; one tc_wait_st() orders all of them before the next barrier).
@@ -305,11 +338,6 @@ __device__ __forceinline__ uint32_t pack16x2(float lo, float hi) {
   }
 }
 
-// The binary32 values of a packed bf16 pair (bf16 is the upper half of a binary32).
-__device__ __forceinline__ float2 bf16x2_value(uint32_t w) {
-  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
-}
-
 // Keeps the compiler from moving the computation of v past this point (an empty asm that
 // reads it): the work on one TMEM chunk then overlaps the load of the next one.
 __device__ __forceinline__ void keep8(const float (&v)[8]) {
@@ -330,8 +358,10 @@ __device__ __forceinline__ void tc_fold_max(const uint32_t (&r)[32], int c0, int
     for (int e = 0; e < 8; ++e) m8[e] = fmax3(m8[e], at(i + e), at(i + 8 + e));
 }
 
-// Pass 1 of the softmax: the maximum of one row's 128 scores in TMEM (this thread's lane;
-// with kMask those past `vis` masked), 32 columns at a time with the next 32 in flight.
+// Pass 1 of the softmax: the maximum of one row's 64 scores of this warp's half of the
+// tile in TMEM (this thread's lane; with kMask those past `vis` masked), both 32-column
+// loads in flight at once.
+static_assert(kTcHalf == 64, "tc_row_max reads one half tile");
 template <bool kMask>
 __device__ __forceinline__ float tc_row_max(uint32_t addr, int vis) {
   float m8[8];
@@ -339,30 +369,31 @@ __device__ __forceinline__ float tc_row_max(uint32_t addr, int vis) {
   for (int e = 0; e < 8; ++e) m8[e] = -INFINITY;
   uint32_t ra[32], rb[32];
   tc_ld32_async(addr, ra);
-  tc_wait_ld();
   tc_ld32_async(addr + 32, rb);
+  tc_wait_ld();
   tc_fold_max<kMask>(ra, 0, vis, m8);
-  keep8(m8);
-  tc_wait_ld();
-  tc_ld32_async(addr + 64, ra);
   tc_fold_max<kMask>(rb, 32, vis, m8);
-  keep8(m8);
-  tc_wait_ld();
-  tc_ld32_async(addr + 96, rb);
-  tc_fold_max<kMask>(ra, 64, vis, m8);
-  keep8(m8);
-  tc_wait_ld();
-  tc_fold_max<kMask>(rb, 96, vis, m8);
   return fmaxf(fmax3(m8[0], m8[1], m8[2]), fmax3(fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7]));
 }
 
+// The binary32 values of a packed bf16 pair (bf16 is the upper half of a binary32).
+__device__ __forceinline__ float2 bf16x2_value(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+// What pass 2 writes beside P (bf16 only): nothing, the rounded remainder, or zeros (the
+// remainder product may cover these rows because another warp's rows need it).
+constexpr int kRemNone = 0, kRemValue = 1, kRemZero = 2;
+
 // Pass 2 on 16 scores (tokens 16 t .. 16 t + 15 of the tile, columns [16 t, 16 t + 16) of
 // S; with kMask those past `vis` masked): p = 2^(s * s_mul + nmb) written over them as
-// 16-bit pairs, P in columns [16 t, 16 t + 8) and, with kLo, the rounded remainder
-// p - bf16(p) in [16 t + 8, 16 t + 16); the binary32 p are added to l2 (four pair chains).
-template <int QD, bool kMask, bool kLo>
+// 16-bit pairs, P in columns [16 t, 16 t + 8) and, per kRem, the rounded remainder
+// p - bf16(p) (or zeros) in [16 t + 8, 16 t + 16); the binary32 p are added to l2 (four pair
+// chains).
+template <int QD, bool kMask, int kRem>
 __device__ __forceinline__ void tc_make_p16(uint32_t addr, const uint32_t (&r)[16], int t, int vis, float s_mul,
                                             float nmb, float2 (&l2)[4]) {
+  static_assert(kRem == kRemNone || QD == PA_BF16, "the remainder is for bf16 P");
   uint32_t wh[8], wl[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
@@ -377,35 +408,38 @@ __device__ __forceinline__ void tc_make_p16(uint32_t addr, const uint32_t (&r)[1
     const float p0 = ex2(a.x), p1 = ex2(a.y);
     wh[e] = pack16x2<QD>(p0, p1);
     l2[e & 3] = add2(l2[e & 3], make_float2(p0, p1));
-    if constexpr (kLo) {
+    if constexpr (kRem == kRemValue) {
       const float2 hv = bf16x2_value(wh[e]);
       wl[e] = pack16x2<QD>(p0 - hv.x, p1 - hv.y);
+    } else if constexpr (kRem == kRemZero) {
+      wl[e] = 0u;
     }
   }
   tc_st8(addr + t * 16, wh);
-  if constexpr (kLo) tc_st8(addr + t * 16 + 8, wl);
+  if constexpr (kRem != kRemNone) tc_st8(addr + t * 16 + 8, wl);
 }
 
-// Pass 2 over the row's 128 scores, 16 columns at a time with the next 16 in flight.
-template <int QD, bool kMask, bool kLo>
+// Pass 2 over the row's 64 scores of this warp's half, 16 columns at a time with the next
+// 16 in flight.
+template <int QD, bool kMask, int kRem>
 __device__ __forceinline__ void tc_make_p(uint32_t addr, int vis, float s_mul, float nmb, float2 (&l2)[4]) {
   uint32_t ra[16], rb[16];
   tc_ld16_async(addr, ra);
   tc_wait_ld();
 #pragma unroll 1
-  for (int t = 0; t < kTcTok / 16; t += 2) {
+  for (int t = 0; t < kTcHalf / 16; t += 2) {
     tc_ld16_async(addr + (t + 1) * 16, rb);
-    tc_make_p16<QD, kMask, kLo>(addr, ra, t, vis, s_mul, nmb, l2);
+    tc_make_p16<QD, kMask, kRem>(addr, ra, t, vis, s_mul, nmb, l2);
     tc_wait_ld();
-    if (t + 2 < kTcTok / 16) tc_ld16_async(addr + (t + 2) * 16, ra);
-    tc_make_p16<QD, kMask, kLo>(addr, rb, t + 1, vis, s_mul, nmb, l2);
+    if (t + 2 < kTcHalf / 16) tc_ld16_async(addr + (t + 2) * 16, ra);
+    tc_make_p16<QD, kMask, kRem>(addr, rb, t + 1, vis, s_mul, nmb, l2);
     tc_wait_ld();
   }
 }
 
 // One CTA per SM. The register file is split between the SM's four sub-partitions and a
 // warp takes its registers from its own: with 11 warps, three share one sub-partition's
-// 16384 registers, so a thread may hold at most 170 (the compiler takes 168).
+// 16384 registers, so a thread may hold at most 170.
 template <int QD, int BS, int G>
 __global__ void __launch_bounds__(kTcThreads, 1)
     extend_tc_kernel(const ExtendParams p, const __grid_constant__ CUtensorMap tk,
@@ -417,16 +451,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   constexpr uint32_t kBlockTx = BS * kTcD * 2;        // bytes of one cache block of K (or V)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  // per set: S(g) landed, P(g) written (one arrival per softmax warp), P(g) V(g) done;
-  // K(g) / V(g) landed, K buffer free; Q of unit k landed / free; O of unit k complete /
-  // read (one arrival per softmax warp); the unit ring
-  __shared__ uint64_t s_full[kTcSets], p_full[kTcSets], pv_done[kTcSets], k_full[kTcSets], v_full[kTcSets];
-  __shared__ uint64_t k_empty[kTcSets], q_full[kTcSets], q_empty[kTcSets], o_full[kTcSets], o_empty[kTcSets];
-  __shared__ uint64_t uq_full[kTcSets][4], uq_empty[kTcSets][4], bar_fin;
-  __shared__ int uq[kTcSets][4];               // unit k of set c in slot k % 4
-  __shared__ int lo_tile[kTcSets];             // adaptive remainder: the set's latest tile that needs it
-  __shared__ uint64_t vote_bar[kTcSets];       // the set's warps agree on the remainder of each tile
-  __shared__ int vote_word[kTcSets][3];        // ... through one word per tile, three in rotation
+  // tile g: S buffer g % 3 (phase g / 3 of its barriers), K / V buffer g % 2 (phase g / 2).
+  // S(g) landed, P(g) written (one arrival per softmax warp), P(g) V(g) done; K(g) / V(g)
+  // landed; Q of unit k landed / free; O of unit k complete / read (one arrival per
+  // softmax warp); the two warps of a row quarter exchanged; the unit ring.
+  __shared__ uint64_t s_full[kTcSBufs], p_full[kTcSBufs], pv_done[kTcSBufs], k_full[kTcKvBufs], v_full[kTcKvBufs];
+  __shared__ uint64_t q_full, q_empty, o_full, o_empty, xchg[kTcQuarters];
+  __shared__ uint64_t uq_full[4], uq_empty[4], bar_fin;
+  __shared__ int uq[4], uq_nt[4];                                // unit k in slot k % 4, and its K/V tiles
+  __shared__ __align__(8) char lo_need[kTcSBufs][kTcSoftmaxWarps];   // adaptive remainder: the warps' flags
+  __shared__ float2 xval[2][kTcSoftmaxWarps][32];                // row maxima and sums exchanged, two in rotation
   __shared__ uint32_t tmem_slot;
   __shared__ int s_abort;
   volatile int* abort = &s_abort;
@@ -439,24 +473,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
   if (tid == 32) {
-    for (int c = 0; c < kTcSets; ++c) {
-      mbar_init(&s_full[c], 1);
-      mbar_init(&p_full[c], kTcSetWarps);
-      mbar_init(&pv_done[c], 1);
-      mbar_init(&k_full[c], 1);
-      mbar_init(&v_full[c], 1);
-      mbar_init(&k_empty[c], 1);
-      mbar_init(&q_full[c], 1);
-      mbar_init(&q_empty[c], 1);
-      mbar_init(&o_full[c], 1);
-      mbar_init(&o_empty[c], kTcSetWarps);
-      for (int i = 0; i < 4; ++i) {
-        mbar_init(&uq_full[c][i], 1);
-        mbar_init(&uq_empty[c][i], kTcSetWarps + 1);   // the set's softmax warps and the MMA warp
-      }
-      lo_tile[c] = -1;
-      mbar_init(&vote_bar[c], kTcSetWarps);
-      vote_word[c][0] = vote_word[c][1] = vote_word[c][2] = 0;
+    for (int b = 0; b < kTcSBufs; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&p_full[b], kTcSoftmaxWarps);
+      mbar_init(&pv_done[b], 1);
+      for (int w = 0; w < kTcSoftmaxWarps; ++w) lo_need[b][w] = 0;
+    }
+    for (int b = 0; b < kTcKvBufs; ++b) {
+      mbar_init(&k_full[b], 1);
+      mbar_init(&v_full[b], 1);
+    }
+    mbar_init(&q_full, 1);
+    mbar_init(&q_empty, 1);
+    mbar_init(&o_full, 1);
+    mbar_init(&o_empty, kTcSoftmaxWarps);
+    for (int q = 0; q < kTcQuarters; ++q) mbar_init(&xchg[q], 2);
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&uq_full[i], 1);
+      mbar_init(&uq_empty[i], kTcSoftmaxWarps + 2);   // softmax warps, the MMA warp, the V producer
     }
     mbar_init(&bar_fin, 1);
     s_abort = 0;
@@ -471,55 +505,59 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t tmem = tmem_slot;
   const int Hq = p.num_q_heads, Hkv = p.num_kv_heads;
   const int total = p.plan[p.num_seqs] * Hkv;
-  uint32_t k_loads = 0, v_loads = 0, q_loads = 0;   // producer: loads issued (for the drain after an abort)
+  uint32_t kv_loads = 0, q_loads = 0;   // producers: loads issued (for the drain after an abort)
 
-  // Dynamic scheduling: each set's producer takes the set's unit k from the global queue
-  // (the plan kernel lists each sequence's longest row tile first) and publishes it in
-  // the set's ring; the set's softmax warps and the MMA warp read the same sequence. -1
-  // ends the set's work. False on an abort.
-  auto next_unit = [&](int c, uint32_t k, bool taker, int& u) -> bool {
+  // Dynamic scheduling: the K producer takes unit k from the global queue (the plan kernel
+  // lists each sequence's longest row tile first) and publishes it in slot k % 4 of the
+  // ring; the V producer, the softmax warps and the MMA warp read the same sequence. -1
+  // ends the work.
+  auto read_unit = [&](uint32_t k, int& u) -> bool {   // reads slot k % 4 and releases it
     const int slot = k & 3;
-    const uint32_t ph = (k >> 2) & 1;
-    if (taker) {
-      if (!tc_wait_warp(&uq_empty[c][slot], ph ^ 1, abort, 28, int(k))) return false;
-      int v = 0;
-      if (lane == 0) {
-        v = atomicAdd(p.queue, 1);
-        if (v >= total) v = -1;
-        uq[c][slot] = v;
-        mbar_arrive(&uq_full[c][slot]);
-      }
-      u = __shfl_sync(kFull, v, 0);
-      return true;
-    }
-    if (!tc_wait_warp(&uq_full[c][slot], ph, abort, 29, int(k))) return false;
-    u = *reinterpret_cast<volatile int*>(&uq[c][slot]);
+    if (!tc_wait_warp(&uq_full[slot], (k >> 2) & 1, abort, 29, int(k))) return false;
+    u = *reinterpret_cast<volatile int*>(&uq[slot]);
     __syncwarp();
-    if (lane == 0) mbar_arrive(&uq_empty[c][slot]);
+    if (lane == 0) mbar_arrive(&uq_empty[slot]);
     return true;
   };
 
-  if (warp > kTcMmaWarp) {
-    // ---------------- producer of set c: its units, their Q, K and V tiles ----------------
-    const int c = warp - kTcMmaWarp - 1;
-    uint8_t* sQ = sm + c * TcSmem::kSet + TcSmem::kQ;
-    uint8_t* sK = sm + c * TcSmem::kSet + TcSmem::kK;
-    uint8_t* sV = sm + c * TcSmem::kSet + TcSmem::kV;
+  if (warp == kTcKWarp || warp == kTcVWarp) {
+    // ---------------- producers: the K warp takes the units and loads Q and K, the V warp V ----------------
+    const bool isk = warp == kTcKWarp;
+    uint8_t* sQ = sm + TcSmem::kQ;
     uint32_t g = 0;
     bool ok = true;
     for (uint32_t k = 0; ok; ++k) {
-      int u;
-      if (!(ok = next_unit(c, k, true, u)) || u < 0) break;
-      const TcUnit x = tc_unit(p, u);
-      // the unit's q rows, once the last S of the set's previous unit has read the buffer
-      if (!(ok = tc_wait_warp(&q_empty[c], (k & 1) ^ 1, abort, 26, u))) break;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&q_full[c], TcSmem::kTile);
-        tma_load_3d(sQ, &tq, 0, x.hk * G, x.row0 + x.t * QPT, &q_full[c]);
-        tma_load_3d(sQ + kTcRows * 128, &tq, 64, x.hk * G, x.row0 + x.t * QPT, &q_full[c]);
+      int u = -1;
+      if (isk) {
+        const int slot = k & 3;
+        if (!(ok = tc_wait_warp(&uq_empty[slot], ((k >> 2) & 1) ^ 1, abort, 28, int(k)))) break;
+        int v = 0;
+        if (lane == 0) {
+          v = atomicAdd(p.queue, 1);
+          if (v >= total) v = -1;
+        }
+        u = __shfl_sync(kFull, v, 0);
+        if (lane == 0) {
+          uq[slot] = u;
+          uq_nt[slot] = u < 0 ? 0 : tc_unit(p, u).ntiles;
+          mbar_arrive(&uq_full[slot]);
+        }
+      } else if (!(ok = read_unit(k, u))) {
+        break;
       }
-      __syncwarp();
-      q_loads = k + 1;
+      if (u < 0) break;
+      const TcUnit x = tc_unit(p, u);
+      if (isk) {
+        // the unit's q rows, once the last S of the previous unit has read the buffer
+        if (!(ok = tc_wait_warp(&q_empty, (k & 1) ^ 1, abort, 26, u))) break;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&q_full, TcSmem::kQTile);
+          tma_load_3d(sQ, &tq, 0, x.hk * G, x.row0 + x.t * QPT, &q_full);
+          tma_load_3d(sQ + kTcRows * 128, &tq, 64, x.hk * G, x.row0 + x.t * QPT, &q_full);
+        }
+        __syncwarp();
+        q_loads = k + 1;
+      }
       const int32_t* trow = p.block_tables + size_t(x.s) * p.max_blocks;
       auto blocks = [&](int j) { return min(BPT, (x.nvis - j * kTcTok + BS - 1) / BS); };
       auto fetch = [&](int lb, int n) {   // block id of this lane's block (lane < n), checked
@@ -533,64 +571,52 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         return id;
       };
+      const CUtensorMap* cache_map = isk ? &tk : &tv;
+      const CUtensorMap* new_map = isk ? &tkn : &tvn;
       for (int j = 0; j < x.ntiles; ++j, ++g) {
+        const int xb = g & 1;
+        uint64_t* full = isk ? &k_full[xb] : &v_full[xb];
+        uint8_t* dst = sm + (isk ? TcSmem::kK : TcSmem::kV) + xb * TcSmem::kKvTile;
         const int p0 = x.t0 + j * kTcTok;
         const int nb = blocks(j);
         const int id = p.fresh ? 0 : fetch(p0 / BS, nb);
-        // K(g) once S(g-1) has read the buffer (and, for whole prompts, once the cache
-        // stores of the previous tile have read both buffers)
-        if (!(ok = tc_wait_warp(&k_empty[c], (g & 1) ^ 1, abort, 10, u))) break;
+        // K(g) once S(g - 2), V(g) once P(g - 2) V(g - 2) has read the buffer (and, for
+        // whole prompts, once this warp's cache stores have read theirs)
+        if (g >= 2) {
+          const uint32_t gr = g - 2;
+          if (!(ok = tc_wait_warp(isk ? &s_full[gr % kTcSBufs] : &pv_done[gr % kTcSBufs], (gr / kTcSBufs) & 1, abort,
+                                  isk ? 10 : 11, u)))
+            break;
+        }
         if (p.fresh) bulk_wait_read_all();
         __syncwarp();
         if (p.fresh) {   // whole prompts: the prompt's own rows, 128 per box
           if (lane == 0) {
-            mbar_arrive_expect_tx(&k_full[c], TcSmem::kTile);
-            tma_load_3d(sK, &tkn, 0, x.hk, x.row0 + p0, &k_full[c]);
-            tma_load_3d(sK + kTcTok * 128, &tkn, 64, x.hk, x.row0 + p0, &k_full[c]);
+            mbar_arrive_expect_tx(full, TcSmem::kKvTile);
+            tma_load_3d(dst, new_map, 0, x.hk, x.row0 + p0, full);
+            tma_load_3d(dst + kTcTok * 128, new_map, 64, x.hk, x.row0 + p0, full);
           }
         } else {
-          if (lane == 0) mbar_arrive_expect_tx(&k_full[c], uint32_t(nb) * kBlockTx);
+          if (lane == 0) mbar_arrive_expect_tx(full, uint32_t(nb) * kBlockTx);
           __syncwarp();
           if (lane < nb) {
             const int y = (id * Hkv + x.hk) * BS;
-            tma_load_2d(sK + lane * (BS * 128), &tk, 0, y, &k_full[c]);
-            tma_load_2d(sK + kTcTok * 128 + lane * (BS * 128), &tk, 64, y, &k_full[c]);
+            tma_load_2d(dst + lane * (BS * 128), cache_map, 0, y, full);
+            tma_load_2d(dst + kTcTok * 128 + lane * (BS * 128), cache_map, 64, y, full);
           }
         }
         __syncwarp();
-        k_loads = g + 1;
-        // V(g) once P(g-1) V(g-1) has read the buffer
-        if (!(ok = tc_wait_warp(&pv_done[c], (g & 1) ^ 1, abort, 11, u))) break;
-        if (p.fresh) {
-          if (lane == 0) {
-            mbar_arrive_expect_tx(&v_full[c], TcSmem::kTile);
-            tma_load_3d(sV, &tvn, 0, x.hk, x.row0 + p0, &v_full[c]);
-            tma_load_3d(sV + kTcTok * 128, &tvn, 64, x.hk, x.row0 + p0, &v_full[c]);
-          }
-        } else {
-          if (lane == 0) mbar_arrive_expect_tx(&v_full[c], uint32_t(nb) * kBlockTx);
-          __syncwarp();
-          if (lane < nb) {
-            const int y = (id * Hkv + x.hk) * BS;
-            tma_load_2d(sV + lane * (BS * 128), &tv, 0, y, &v_full[c]);
-            tma_load_2d(sV + kTcTok * 128 + lane * (BS * 128), &tv, 64, y, &v_full[c]);
-          }
-        }
-        __syncwarp();
-        v_loads = g + 1;
+        kv_loads = g + 1;
         // whole prompts: the row tile that sees every prompt position of this K/V tile
-        // writes the tile into its cache blocks, once both loads have landed
+        // writes the tile into its cache blocks, once the load has landed
         if (p.fresh && x.t == min((p0 + kTcTok - 1) / QPT, (x.Q - 1) / QPT)) {
-          if (!(ok = tc_wait_warp(&k_full[c], g & 1, abort, 27, u) && tc_wait_warp(&v_full[c], g & 1, abort, 27, u)))
-            break;
+          if (!(ok = tc_wait_warp(full, (g >> 1) & 1, abort, 27, u))) break;
           const int nbw = (min(p0 + kTcTok, x.Q) - p0 + BS - 1) / BS;
           const int idw = fetch(p0 / BS, nbw);
           if (lane < nbw) {
             const int y = (idw * Hkv + x.hk) * BS;
-            tma_store_2d(&tk, 0, y, sK + lane * (BS * 128));
-            tma_store_2d(&tk, 64, y, sK + kTcTok * 128 + lane * (BS * 128));
-            tma_store_2d(&tv, 0, y, sV + lane * (BS * 128));
-            tma_store_2d(&tv, 64, y, sV + kTcTok * 128 + lane * (BS * 128));
+            tma_store_2d(cache_map, 0, y, dst + lane * (BS * 128));
+            tma_store_2d(cache_map, 64, y, dst + kTcTok * 128 + lane * (BS * 128));
             bulk_commit();
           }
           __syncwarp();
@@ -599,247 +625,329 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     bulk_wait_all();   // this thread's cache stores are complete before the kernel ends
   } else if (warp == kTcMmaWarp) {
-    // ---------------- MMA issue for both sets ----------------
-    // Per set the products form a chain S(g), P(g) V(g), S(g + 1), ...: S(g + 1) overwrites
-    // the P that P(g) V(g) reads, so it waits for that product to complete. The sets are
-    // served in turn -- P V(set 0), S(set 0), P V(set 1), S(set 1), ... -- so that each
-    // set's next S follows its own P V as soon as possible while the other set's softmax
-    // runs, and the tensor core alternates between the two chains.
-    const uint32_t idS = tc_idesc<QD>(0), idO = tc_idesc<QD>(1);
-    TcUnit x[kTcSets];
-    int j[kTcSets];
-    uint32_t g[kTcSets], k[kTcSets];
-    bool live[kTcSets], fresh_unit[kTcSets];
-#pragma unroll
-    for (int c = 0; c < kTcSets; ++c) {
-      j[c] = 0;
-      g[c] = k[c] = 0;
-      live[c] = fresh_unit[c] = true;
-    }
-    bool ok = true;
-    // S(g) of set c (taking the set's next unit first when the last one is done); false
-    // when the set has no more work (live[c] cleared) or on an abort (ok cleared)
-    auto issue_s = [&](int c) {
-      if (fresh_unit[c]) {
-        int u;
-        if (!(ok = next_unit(c, k[c], false, u))) return false;
+    // ---------------- MMA issue ----------------
+    // S(g) into S buffer g % 3 once its unit's Q and K(g) have landed and P(g - 3) V(g - 3),
+    // which reads the buffer, completed -- so S runs up to three tiles (and units) ahead of
+    // the softmax; P V(g) once the softmax has written P(g) and V(g) has landed. Both
+    // cursors read the units from the ring; the slot is released when the P V cursor is
+    // done with the unit. Lane 0 tests the barriers without blocking and issues whatever
+    // is ready; the other lanes follow its decisions.
+    const uint32_t idS = tc_idesc<QD>(0, kTcTok), idO = tc_idesc<QD>(1, kTcD);
+    const uint64_t dq = tc_desc(smem_addr(sm + TcSmem::kQ), 1024, 16);
+    const uint64_t dk0 = tc_desc(smem_addr(sm + TcSmem::kK), 1024, 16);
+    const uint64_t dv0 = tc_desc(smem_addr(sm + TcSmem::kV), 1024, kTcTok * 128);
+    constexpr uint64_t kKvDesc = TcSmem::kKvTile >> 4;   // one K / V buffer in descriptor units
+    int s_nt = 0, p_nt = 0;   // K/V tiles of the S cursor's and of the P V cursor's unit
+    int js = 0, jp = 0;
+    uint32_t gs = 0, gp = 0, ks = 0, kp = 0;
+    bool s_live = true, s_fresh = true, p_fresh = true;
+    auto lane0 = [&](bool v) { return __shfl_sync(kFull, v ? 1 : 0, 0) != 0; };
+    auto try_s = [&]() -> bool {
+      if (!s_live || gs >= gp + kTcSBufs) return false;
+      if (s_fresh) {
+        const int slot = ks & 3;
+        if (!lane0(lane == 0 && mbar_test(&uq_full[slot], (ks >> 2) & 1))) return false;
+        int u = lane == 0 ? *reinterpret_cast<volatile int*>(&uq[slot]) : 0;
+        u = __shfl_sync(kFull, u, 0);
         if (u < 0) {
-          live[c] = false;
-          return false;
+          s_live = false;
+          return true;
         }
-        x[c] = tc_unit(p, u);
-        j[c] = 0;
-        fresh_unit[c] = false;
-        if (!(ok = tc_wait_warp(&q_full[c], k[c] & 1, abort, 14, u))) return false;
+        s_nt = *reinterpret_cast<volatile int*>(&uq_nt[slot]);
+        js = 0;
+        s_fresh = false;
       }
-      // once K(g) has landed and P(g-1) V(g-1), which reads P from the S columns, completed
-      if (!(ok = tc_wait_warp(&k_full[c], g[c] & 1, abort, 16, int(g[c])) &&
-                 tc_wait_warp(&pv_done[c], (g[c] & 1) ^ 1, abort, 17, int(g[c]))))
+      const int b = gs % kTcSBufs, xb = gs & 1;
+      if (!lane0(lane == 0 && (js > 0 || mbar_test(&q_full, ks & 1)) && mbar_test(&k_full[xb], (gs >> 1) & 1) &&
+                 mbar_test(&pv_done[b], ((gs / kTcSBufs) & 1) ^ 1)))
         return false;
       if (lane == 0) {
         tc_fence_after();
-        const uint32_t qa = smem_addr(sm + c * TcSmem::kSet + TcSmem::kQ);
-        const uint32_t ka = smem_addr(sm + c * TcSmem::kSet + TcSmem::kK);
-#pragma unroll
-        for (int kk = 0; kk < kTcD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (kTcRows * 128) + (kk & 3) * 32;
-          tc_mma(tmem + c * 128, tc_desc(qa + off, 1024, 16), tc_desc(ka + off, 1024, 16), idS, kk > 0);
+        tc_mma_s8(tmem + b * kTcTok, dq, dk0 + xb * kKvDesc, idS);
+        tc_commit(&s_full[b]);
+        if (js + 1 == s_nt) tc_commit(&q_empty);   // the Q buffer is free once this S completes
+      }
+      __syncwarp();
+      ++gs;
+      if (++js == s_nt) {
+        s_fresh = true;
+        ++ks;
+      }
+      return true;
+    };
+    // a unit's first P V overwrites O, so it also waits until the previous unit's O was read
+    auto try_pv = [&]() -> bool {
+      if (gp >= gs) return false;
+      if (p_fresh) {   // the unit of this tile: the S cursor has read its slot already
+        p_nt = *reinterpret_cast<volatile int*>(&uq_nt[kp & 3]);
+        jp = 0;
+        p_fresh = false;
+      }
+      const int b = gp % kTcSBufs, xb = gp & 1;
+      if (!lane0(lane == 0 && mbar_test(&p_full[b], (gp / kTcSBufs) & 1) && mbar_test(&v_full[xb], (gp >> 1) & 1) &&
+                 (jp > 0 || kp == 0 || mbar_test(&o_empty, (kp & 1) ^ 1))))
+        return false;
+      if (lane == 0) {
+        // the remainder product: every tile, or (adaptive) when a softmax warp flagged it
+        const bool lo = p.lo_mode == kLoAlways ||
+                        (p.lo_mode == kLoAdaptive && *reinterpret_cast<volatile unsigned long long*>(lo_need[b]) != 0);
+        tc_fence_after();
+        const uint32_t d = tmem + kTcOCol, a = tmem + b * kTcTok;
+        const uint64_t dv = dv0 + xb * kKvDesc;
+        tc_mma_pv8(d, a, dv, idO, jp > 0 ? 1u : 0u);   // P of tokens 16 t .. 16 t + 15 at a + 16 t
+        if (lo) tc_mma_pv8(d, a + 8, dv, idO, 1u);      // their remainders, 8 columns further
+        tc_commit(&pv_done[b]);
+        if (jp + 1 == p_nt) tc_commit(&o_full);
+      }
+      __syncwarp();
+      ++gp;
+      if (++jp == p_nt) {   // the unit is done: release its ring slot
+        if (lane == 0) mbar_arrive(&uq_empty[kp & 3]);
+        p_fresh = true;
+        ++kp;
+      }
+      return true;
+    };
+    uint64_t t_idle = 0;   // lane 0: since when nothing was ready
+    while (s_live || gp < gs) {
+      bool moved = try_pv();
+      moved |= try_s();
+      if (moved) {
+        t_idle = 0;
+        continue;
+      }
+      // nothing ready: lane 0 sleeps in the blocking test of the barrier the next P V needs
+      // (it returns when the phase completes or after the hardware's time limit), or
+      // briefly when no P V is pending, so that the polling takes no issue slots from the
+      // softmax warps of its sub-partition; it gives up after 2 s without progress, or once
+      // another role aborted
+      bool stop = false;
+      if (lane == 0) {
+        if (gp < gs) mbar_try_wait(&p_full[gp % kTcSBufs], (gp / kTcSBufs) & 1);
+        else __nanosleep(200);
+        const uint64_t now = global_timer_ns();
+        if (t_idle == 0) t_idle = now;
+        if (*abort) {
+          stop = true;
+        } else if (now - t_idle > 2000000000ull) {
+          record_error(PA_DEV_WAIT_TIMEOUT, 30, int(gs), int(gp));
+          *abort = 1;
+          stop = true;
         }
-        tc_commit(&s_full[c]);
-        tc_commit(&k_empty[c]);
-        if (j[c] + 1 == x[c].ntiles) tc_commit(&q_empty[c]);   // the Q buffer is free once this S completes
+      }
+      if (lane0(stop)) break;
+    }
+  } else {
+    // ---------------- softmax warps: rows of quarter rq, columns [64 h, 64 h + 64) of each tile ----------------
+    const int rq = warp % kTcQuarters, h = warp / kTcQuarters, row = rq * 32 + lane;
+    const int partner = warp ^ kTcQuarters;
+    const uint32_t t_row = tmem + (uint32_t(rq * 32) << 16);
+    uint32_t g = 0, xn = 0;
+    // the partner's values for this lane's row, after both wrote theirs (exchange xn)
+    auto exchange = [&](float2 v, float2& other) -> bool {
+      xval[xn & 1][warp][lane] = v;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&xchg[rq]);
+      if (!tc_wait_warp(&xchg[rq], xn & 1, abort, 23, int(xn))) return false;
+      volatile float* o = reinterpret_cast<volatile float*>(&xval[xn & 1][partner][lane]);
+      other = make_float2(o[0], o[1]);
+      ++xn;
+      return true;
+    };
+    // Unit kk's O (this warp's 64 columns), once the unit's last P V completed: the output
+    // row (the row's whole context was in this unit) or the chunk's partial (unnormalised
+    // row, then max and sum). The accumulator is released as soon as it is in registers.
+    // Called after the next unit's first tile, so that the last P V runs meanwhile.
+    auto epilogue = [&](const TcUnit& x, uint32_t kk, float l, float m_ref) -> bool {
+      if (!tc_wait_warp(&o_full, kk & 1, abort, 22, int(kk))) return false;
+      tc_fence_after();
+      float2 other;
+      if (!exchange(make_float2(l, 0.f), other)) return false;
+      l += other.x;   // the row sum
+      // a row whose context reaches into this unit's chunk writes now: its output row when
+      // the chunk is the row's only one (position below the chunk length), else a partial
+      const int qi = x.t * QPT + row / G, qpos = x.base + qi;
+      const bool wr = qi < x.Q && qpos >= x.part * p.chunk, fin = wr && qpos < p.chunk;
+      uint4* stage = reinterpret_cast<uint4*>(sm + TcSmem::kStage + warp * TcSmem::kStageWarp);
+      const size_t slot = (size_t(x.row0 + qi) * Hq + x.hk * G + row % G) * p.max_parts + x.part;
+      float4* acc = reinterpret_cast<float4*>(p.part_acc + slot * kTcD + h * kTcHalf);
+      const float inv = fin ? 1.f / l : 0.f;
+      // 32 columns at a time; the accumulator is released once both halves are in registers
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t r[32];
+        tc_ld32_async(t_row + kTcOCol + h * kTcHalf + hh * 32, r);
+        tc_wait_ld();
+        if (hh == 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&o_empty);
+        }
+        auto o = [&](int i) { return __uint_as_float(pin_after_wait(r[i])); };
+        if (fin) {
+          // the 16-bit row into this warp's staging rows (16-byte chunk c of row `lane` at
+          // chunk c ^ (lane & 7), so that 8 consecutive lanes cover every bank) ...
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int cc = hh * 4 + i;
+            stage[lane * 8 + (cc ^ (lane & 7))] = make_uint4(pack16x2<QD>(o(8 * i) * inv, o(8 * i + 1) * inv),
+                                                             pack16x2<QD>(o(8 * i + 2) * inv, o(8 * i + 3) * inv),
+                                                             pack16x2<QD>(o(8 * i + 4) * inv, o(8 * i + 5) * inv),
+                                                             pack16x2<QD>(o(8 * i + 6) * inv, o(8 * i + 7) * inv));
+          }
+        } else if (wr) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            acc[hh * 8 + i] = make_float4(o(4 * i), o(4 * i + 1), o(4 * i + 2), o(4 * i + 3));
+        }
+      }
+      if (wr && !fin && h == 0) {
+        p.part_ml[slot * 2] = m_ref;
+        p.part_ml[slot * 2 + 1] = l;
+      }
+      __syncwarp();
+      // ... then out, 4 rows of 128 bytes per instruction: lane j writes chunk j % 8 of
+      // staging row 4 i + j / 8
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int rr = 4 * i + (lane >> 3), c = lane & 7;
+        const int row_r = rq * 32 + rr, qi_r = x.t * QPT + row_r / G;
+        if (x.part == 0 && qi_r < x.Q && x.base + qi_r < p.chunk) {   // that row's output row was staged
+          QT* out_r = static_cast<QT*>(p.out) + (size_t(x.row0 + qi_r) * Hq + x.hk * G + row_r % G) * kTcD +
+                      h * kTcHalf;
+          reinterpret_cast<uint4*>(out_r)[c] = stage[rr * 8 + (c ^ (rr & 7))];
+        }
       }
       __syncwarp();
       return true;
     };
-    // O += P(g) V(g) (+ the remainder) of set c, once P is in TMEM and V(g) has landed; a
-    // unit's first product overwrites O, so it waits until the previous unit's O was read
-    auto issue_pv = [&](int c) {
-      if (!(ok = tc_wait_warp(&p_full[c], g[c] & 1, abort, 12, int(g[c])) &&
-                 tc_wait_warp(&v_full[c], g[c] & 1, abort, 13, int(g[c]))))
-        return;
-      if (j[c] == 0 && k[c] > 0 && !(ok = tc_wait_warp(&o_empty[c], (k[c] & 1) ^ 1, abort, 15, int(k[c])))) return;
-      const bool lo = p.lo_mode == kLoAlways ||
-                      (p.lo_mode == kLoAdaptive && *reinterpret_cast<volatile int*>(&lo_tile[c]) == int(g[c]));
-      if (lane == 0) {
-        tc_fence_after();
-        const uint32_t va = smem_addr(sm + c * TcSmem::kSet + TcSmem::kV);
-        const uint32_t d = tmem + 256 + c * 128, a = tmem + c * 128;
-#pragma unroll
-        for (int kk = 0; kk < kTcTok / 16; ++kk)   // P of tokens 16 kk .. 16 kk + 15
-          tc_mma_ts(d, a + 16 * kk, tc_desc(va + kk * 2048, 1024, kTcTok * 128), idO, (j[c] > 0 || kk > 0) ? 1u : 0u);
-        if (lo) {
-#pragma unroll
-          for (int kk = 0; kk < kTcTok / 16; ++kk)   // their remainders, 8 columns further
-            tc_mma_ts(d, a + 16 * kk + 8, tc_desc(va + kk * 2048, 1024, kTcTok * 128), idO, 1u);
-        }
-        tc_commit(&pv_done[c]);
-        if (j[c] + 1 == x[c].ntiles) tc_commit(&o_full[c]);
-      }
-      __syncwarp();
-      ++g[c];
-      if (++j[c] == x[c].ntiles) {
-        fresh_unit[c] = true;
-        ++k[c];
-      }
-    };
-    bool pend[kTcSets];
-#pragma unroll
-    for (int c = 0; c < kTcSets; ++c) pend[c] = ok && issue_s(c);
-    while (ok && (pend[0] || pend[1])) {
-#pragma unroll
-      for (int c = 0; c < kTcSets; ++c) {
-        if (!ok || !pend[c]) continue;
-        issue_pv(c);
-        pend[c] = ok && issue_s(c);
-      }
-    }
-  } else {
-    // ---------------- softmax warps: set c, rows 32 rw .. 32 rw + 31 of the tile ----------------
-    const int c = warp / kTcSetWarps, rw = warp % kTcSetWarps, row = rw * 32 + lane;
-    const uint32_t t_row = tmem + (uint32_t(rw * 32) << 16);
-    const uint32_t c_s = c * 128, c_o = 256 + c * 128;
-    uint8_t* sV = sm + c * TcSmem::kSet + TcSmem::kV;
-    uint32_t g = 0;
-    for (uint32_t k = 0;; ++k) {
+    TcUnit xprev;
+    uint32_t kprev = 0;
+    float lprev = 0.f, mprev = 0.f;
+    bool pend = false, ok = true;   // pend: the previous unit's O is still to be read
+    for (uint32_t k = 0; ok; ++k) {
       int u;
-      if (!next_unit(c, k, false, u) || u < 0) break;
+      if (!(ok = read_unit(k, u)) || u < 0) break;
       const TcUnit x = tc_unit(p, u);
       const int qi = x.t * QPT + row / G;
-      const int head = x.hk * G + row % G;
       const bool has_q = qi < x.Q;
       const int qpos = has_q ? x.base + qi : -1;
-      const int tok = has_q ? x.row0 + qi : -1;
-      float m_ref = -INFINITY, l = 0.f;
-      bool ok = true;
+      float m_ref = -INFINITY, l = 0.f;   // l: this half's share of the row sum
       for (int j = 0; j < x.ntiles; ++j, ++g) {
-        if (!(ok = tc_wait_warp(&s_full[c], g & 1, abort, 18, u))) break;
+        const int b = g % kTcSBufs;
+        const uint32_t c_s = b * kTcTok + h * kTcHalf;   // this half of S(g), then of P(g)
+        if (!(ok = tc_wait_warp(&s_full[b], (g / kTcSBufs) & 1, abort, 18, u))) break;
         tc_fence_after();
-        // pass 1: the row maximum of the causally masked scores (8 independent chains); the
-        // mask costs work only in tiles where some row of the warp ends
-        const int tp0 = x.t0 + j * kTcTok;
-        const int vis = qpos - tp0;   // columns 0 .. vis of this tile are visible to the row
-        const bool masked = !__all_sync(kFull, vis >= kTcTok - 1);
-        const float mx = (masked ? tc_row_max<true>(t_row + c_s, vis) : tc_row_max<false>(t_row + c_s, vis)) * p.s_mul;
+        // pass 1: the maximum of this half's causally masked scores (8 independent chains;
+        // the mask costs work only in tiles where some row of the warp ends), then the
+        // row's maximum from both halves (and the other half's running sum)
+        const int vis = qpos - (x.t0 + j * kTcTok + h * kTcHalf);   // columns 0 .. vis of the half are visible
+        const bool masked = !__all_sync(kFull, vis >= kTcHalf - 1);
+        const float mh = masked ? tc_row_max<true>(t_row + c_s, vis) : tc_row_max<false>(t_row + c_s, vis);
+        float2 other;
+        if (!(ok = exchange(make_float2(mh, l), other))) break;
+        const float mx = fmaxf(mh, other.x) * p.s_mul;
         const bool up = mx > m_ref + kTcRescale;
         const float corr = up ? ex2(m_ref - mx) : 1.f;   // 0 while nothing was accumulated
+        float l_row = l + other.y;                       // the row's running sum
         if (up) {
           l *= corr;
+          l_row *= corr;
           m_ref = mx;
         }
         if (j > 0 && __any_sync(kFull, up)) {
-          // O holds every earlier P V of the unit: S(g) was issued after P(g-1) V(g-1) completed
+          // O holds every earlier P V of the unit once P(g-1) V(g-1) has completed; this
+          // warp rescales its half of the row's O
+          const uint32_t gr = g - 1;
+          if (!(ok = tc_wait_warp(&pv_done[gr % kTcSBufs], (gr / kTcSBufs) & 1, abort, 19, u))) break;
+          tc_fence_after();
 #pragma unroll 1
-          for (int i = 0; i < kTcD / 32; ++i) {
-            float o[32];
-            tc_ld32(t_row + c_o + i * 32, o);
+          for (int i = 0; i < kTcHalf / 16; ++i) {   // 16 columns at a time (the scores stay live)
+            uint32_t o[16];
+            tc_ld16_async(t_row + kTcOCol + h * kTcHalf + i * 16, o);
+            tc_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] *= corr;
-            tc_st32(t_row + c_o + i * 32, o);
+            for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(pin_after_wait(o[e])) * corr);
+            tc_st16(t_row + kTcOCol + h * kTcHalf + i * 16, o);
           }
+          tc_wait_st();
         }
         const float nmb = m_ref == -INFINITY ? 0.f : -m_ref;
-        // bf16: does this tile need P's remainder? Adaptive: when some row of the set has a
-        // weight above kLoShare of its running sum -- tested, before the sum of this tile is
-        // known, against the running sum plus the tile's largest weight (a lower bound of the
-        // final sum, so the test flags at least the tiles that need it). The set's four warps
-        // agree through one word and a 4-arrival barrier, since the product covers all rows.
-        bool lo = false;
-        if (QD == PA_BF16 && p.lo_mode == kLoAlways) {
-          lo = true;
-        } else if (QD == PA_BF16 && p.lo_mode == kLoAdaptive) {
+        // bf16: the remainder p - bf16(p) goes beside P. Adaptive: the MMA issuer multiplies it
+        // only if some softmax warp flags the tile -- when a row has a weight above kLoShare
+        // of its running sum, tested before the sum of this tile is known against the running
+        // sum plus the tile's largest weight (a lower bound of the row's final sum, so the
+        // test flags at least the tiles that need it); a warp that does not flag the tile
+        // writes zeros there. A warp writes its flag before it signals P; the issuer reads all
+        // flags once all have signalled.
+        int rem_mode = kRemNone;   // bf16: the remainder of every tile, or (adaptive) of flagged rows
+        if (QD == PA_BF16 && p.lo_mode == kLoAlways) rem_mode = kRemValue;
+        if (QD == PA_BF16 && p.lo_mode == kLoAdaptive) {
           const float pmax = ex2(mx + nmb);   // the row's largest weight in this tile (0: none visible)
-          const bool need = __any_sync(kFull, pmax > kLoShare * (l + pmax));
-          volatile int* vw = vote_word[c];
-          if (lane == 0) {
-            if (rw == 0) vw[(g + 1) % 3] = 0;   // the next tile's word: every warp read it two tiles ago
-            if (need) atomicOr(const_cast<int*>(&vw[g % 3]), 1);
-            mbar_arrive(&vote_bar[c]);
-          }
-          if (!(ok = tc_wait_warp(&vote_bar[c], g & 1, abort, 24, u))) break;
-          lo = vw[g % 3] != 0;
-          if (lo && rw == 0 && lane == 0) *reinterpret_cast<volatile int*>(&lo_tile[c]) = int(g);
+          const bool need = __any_sync(kFull, pmax > kLoShare * (l_row + pmax));
+          if (lane == 0) reinterpret_cast<volatile char*>(lo_need[b])[warp] = need ? 1 : 0;
+          rem_mode = need ? kRemValue : kRemZero;
         }
         // pass 2, 16 columns at a time: P = 2^(s * scale - ref) as 16-bit pairs over the
         // scores it was made from (tokens 16 t ..: P in columns [16 t, 16 t + 8), with the
-        // remainder p - bf16(p) in [16 t + 8, 16 t + 16))
+        // remainder p - bf16(p), or zeros, in [16 t + 8, 16 t + 16))
         float2 l2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-        if (masked) {
-          if (lo) tc_make_p<QD, true, QD == PA_BF16>(t_row + c_s, vis, p.s_mul, nmb, l2);
-          else tc_make_p<QD, true, false>(t_row + c_s, vis, p.s_mul, nmb, l2);
-        } else {
-          if (lo) tc_make_p<QD, false, QD == PA_BF16>(t_row + c_s, vis, p.s_mul, nmb, l2);
-          else tc_make_p<QD, false, false>(t_row + c_s, vis, p.s_mul, nmb, l2);
-        }
+        auto pass2 = [&](auto mask_c) {
+          constexpr bool kM = decltype(mask_c)::value;
+          if constexpr (QD == PA_BF16) {
+            if (rem_mode == kRemValue) tc_make_p<QD, kM, kRemValue>(t_row + c_s, vis, p.s_mul, nmb, l2);
+            else if (rem_mode == kRemZero) tc_make_p<QD, kM, kRemZero>(t_row + c_s, vis, p.s_mul, nmb, l2);
+            else tc_make_p<QD, kM, kRemNone>(t_row + c_s, vis, p.s_mul, nmb, l2);
+          } else {
+            tc_make_p<QD, kM, kRemNone>(t_row + c_s, vis, p.s_mul, nmb, l2);
+          }
+        };
+        if (masked) pass2(std::true_type{});
+        else pass2(std::false_type{});
         l += ((l2[0].x + l2[0].y) + (l2[1].x + l2[1].y)) + ((l2[2].x + l2[2].y) + (l2[3].x + l2[3].y));
         // V rows past the visible tokens (cache bytes beyond the context, or stale rows of
-        // blocks not loaded) are zeroed, so that 0-weighted rows cannot bring a NaN into O
+        // blocks not loaded) are zeroed by the first-half warps (one V row per thread), so
+        // that 0-weighted rows cannot bring a NaN into O
         const int rem = x.nvis - j * kTcTok;
-        if (rem < kTcTok) {
-          if (!(ok = tc_wait_warp(&v_full[c], g & 1, abort, 21, u))) break;
+        if (h == 0 && rem < kTcTok) {
+          if (!(ok = tc_wait_warp(&v_full[g & 1], (g >> 1) & 1, abort, 21, u))) break;
           if (row >= rem) {
+            uint8_t* sV = sm + TcSmem::kV + (g & 1) * TcSmem::kKvTile;
 #pragma unroll
-            for (int i = 0; i < kTcD / 8; ++i) *reinterpret_cast<uint4*>(sV + tc_swz(row, i)) = make_uint4(0, 0, 0, 0);
+            for (int i = 0; i < kTcD / 8; ++i) *reinterpret_cast<uint4*>(sV + tc_swz_kv(row, i)) = make_uint4(0, 0, 0, 0);
           }
           fence_async_smem();
         }
         tc_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[c]);
-      }
-      if (!ok) break;
-      // this unit's O, 64 columns at a time: the output row (the row's whole context was in
-      // this unit) or the chunk's partial (unnormalised row, then max and sum); the
-      // accumulator is released once all of it is read
-      if (!tc_wait_warp(&o_full[c], k & 1, abort, 22, u)) break;
-      tc_fence_after();
-      const int P = has_q ? (qpos + 1 + p.chunk - 1) / p.chunk : 0;
-      const bool wr = has_q && x.part < P, fin = wr && P == 1;
-      const float inv = fin ? 1.f / l : 0.f;
-      const size_t slot = (size_t(max(tok, 0)) * Hq + head) * p.max_parts + x.part;
-      uint4* orow = reinterpret_cast<uint4*>(static_cast<QT*>(p.out) + (size_t(max(tok, 0)) * Hq + head) * kTcD);
-      float4* acc = reinterpret_cast<float4*>(p.part_acc + slot * kTcD);
-#pragma unroll
-      for (int h = 0; h < kTcD / 64; ++h) {
-        uint32_t r[64];
-        tc_ld32_async(t_row + c_o + h * 64, r);
-        tc_ld32_async(t_row + c_o + h * 64 + 32, r + 32);
-        tc_wait_ld();
-        auto o = [&](int i) { return __uint_as_float(pin_after_wait(r[i])); };
-        if (fin) {
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            orow[h * 8 + i] = make_uint4(pack16x2<QD>(o(8 * i) * inv, o(8 * i + 1) * inv),
-                                         pack16x2<QD>(o(8 * i + 2) * inv, o(8 * i + 3) * inv),
-                                         pack16x2<QD>(o(8 * i + 4) * inv, o(8 * i + 5) * inv),
-                                         pack16x2<QD>(o(8 * i + 6) * inv, o(8 * i + 7) * inv));
-        } else if (wr) {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) acc[h * 16 + i] = make_float4(o(4 * i), o(4 * i + 1), o(4 * i + 2), o(4 * i + 3));
+        if (lane == 0) mbar_arrive(&p_full[b]);
+        if (j == 0 && pend) {
+          pend = false;
+          if (!(ok = epilogue(xprev, kprev, lprev, mprev))) break;
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&o_empty[c]);
-      if (wr && !fin) {
-        p.part_ml[slot * 2] = m_ref;
-        p.part_ml[slot * 2 + 1] = l;
-      }
+      if (!ok) break;
+      xprev = x;
+      kprev = k;
+      lprev = l;
+      mprev = m_ref;
+      pend = true;
     }
+    if (ok && pend) epilogue(xprev, kprev, lprev, mprev);
   }
 
   __syncthreads();
-  if (*abort) {   // drain what this CTA issued: MMAs (their thread), then each set's last loads
+  if (*abort) {   // drain what this CTA issued: MMAs (their thread), then the producers' last loads
     if (warp == kTcMmaWarp && lane == 0) {
       tc_commit(&bar_fin);
       mbar_wait_bounded(&bar_fin, 0);
     }
-    if (warp > kTcMmaWarp && lane == 0) {
-      const int c = warp - kTcMmaWarp - 1;
-      if (k_loads > 0) mbar_wait_bounded(&k_full[c], (k_loads - 1) & 1, 100000000ull);
-      if (v_loads > 0) mbar_wait_bounded(&v_full[c], (v_loads - 1) & 1, 100000000ull);
-      if (q_loads > 0) mbar_wait_bounded(&q_full[c], (q_loads - 1) & 1, 100000000ull);
+    if ((warp == kTcKWarp || warp == kTcVWarp) && lane == 0) {
+      uint64_t* full = warp == kTcKWarp ? k_full : v_full;
+      for (uint32_t i = kv_loads > 2 ? kv_loads - 2 : 0; i < kv_loads; ++i)
+        mbar_wait_bounded(&full[i & 1], (i >> 1) & 1, 100000000ull);
+      if (warp == kTcKWarp && q_loads > 0) mbar_wait_bounded(&q_full, (q_loads - 1) & 1, 100000000ull);
     }
   }
   tc_fence_before();

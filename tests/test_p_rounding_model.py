@@ -9,10 +9,12 @@ score scales from flat to peaked (scale * sqrt(D) = 1, 4, 12):
 * P rounded to bf16 alone (the arithmetic before the fix) leaves the tolerance: a rounding
   of up to 2^-8 of a dominant weight moves the output by up to 2^-8 |v| while cancelling V
   values keep |ref| small. Rows that see few tokens and rows with peaked scores both do;
-* the tcgen05 kernel's arithmetic -- 128-token tiles, a reference maximum that moves only
-  by more than 2^8, the running sum over the binary32 p, and the bf16 remainder
-  p - bf16(p) as a second product for every tile where some row of the 128 has a weight
-  above 1/8 of its running sum -- stays inside for every element;
+* the tcgen05 kernel's arithmetic -- 128-token tiles whose two 64-column halves keep
+  separate running sums, a reference maximum that moves only by more than 2^8, P as p
+  rounded to bf16 and the bf16 remainder p - bf16(p), added as a second product to the
+  rows of every group of 32 (one warp's rows) where some row has a weight above 1/8 of
+  its running sum (the two halves' sums, exchanged with the maxima), zeros to the other
+  rows of the tile -- stays inside for every element;
 * the mma.sync kernels' arithmetic -- 16-token slices, the running maximum, P and its bf16
   remainder for every slice where some row has a weight above 1/8 of its running sum,
   the running sum over what enters the products -- stays inside;
@@ -38,7 +40,7 @@ def tcgen05_arithmetic(q, K, V, qpos, scale, dt, remainder):
     s_mul = np.float32(scale * 1.4426950408889634)
     R, D = q.shape
     m = np.full(R, -np.inf, np.float32)
-    l = np.zeros(R, np.float32)
+    lh = np.zeros((2, R), np.float32)          # running sums of the two 64-column halves
     O = np.zeros((R, D), np.float32)
     flagged = 0
     for j in range(-(-K.shape[0] // TILE)):
@@ -49,16 +51,26 @@ def tcgen05_arithmetic(q, K, V, qpos, scale, dt, remainder):
             mx = S.max(axis=1) * s_mul
             up = mx > m + 8
             corr = np.where(up, np.exp2(m - mx), 1.0).astype(np.float32)
-        l, O, m = np.where(up, l * corr, l), np.where(up[:, None], O * corr[:, None], O), np.where(up, mx, m)
-        p = np.exp2(S * s_mul - np.where(m == -np.inf, 0, m)[:, None]).astype(np.float32)
-        l = l + p.sum(axis=1)
+        lh, O, m = np.where(up, lh * corr, lh), np.where(up[:, None], O * corr[:, None], O), np.where(up, mx, m)
+        ref = np.where(m == -np.inf, 0, m)
+        p = np.exp2(S * s_mul - ref[:, None]).astype(np.float32)
+        with np.errstate(invalid="ignore"):
+            pmax = np.exp2(mx - ref).astype(np.float32)
+        # per group of 32 rows (one warp's rows), before this tile's sums
+        need_row = pmax > SHARE * (lh.sum(axis=0) + pmax)
+        need = np.repeat(need_row.reshape(-1, 32).any(axis=1), 32) if R % 32 == 0 else np.full(R, need_row.any())
+        halves = [p[:, :64], p[:, 64:]]
+        lh = lh + np.stack([np.pad(x, ((0, 0), (0, 64 - x.shape[1]))).sum(axis=1) for x in halves])
         P = _round(p, dt)
-        use = remainder == "always" or (remainder == "adaptive" and bool(np.any(p.max(axis=1) > SHARE * l)))
-        if use:
+        rem = _round(p - P, dt) if dt == "bf16" else None
+        if rem is not None and remainder == "always":
             flagged += 1
-            P = P + _round(p - P, dt)
+            P = P + rem
+        elif rem is not None and remainder == "adaptive" and need.any():
+            flagged += 1
+            P = P + np.where(need[:, None], rem, 0)
         O = O + P @ V[lo:hi]
-    return _round(O / l[:, None], dt), flagged
+    return _round(O / lh.sum(axis=0)[:, None], dt), flagged
 
 
 def mma_sync_arithmetic(q, K, V, qpos, scale, dt, adaptive=True):

@@ -4,24 +4,36 @@ The GPU race checker is not available here, so the kernel's barrier schedule is 
 as a model: every role of one CTA runs as a generator of waits, arrivals and
 asynchronous operations (TMA loads and stores, MMAs with their commits):
 
-* per set c (two sets share the tensor core, each working on its own units): a producer
-  that takes the set's units from the queue, loads their Q and streams K and V tiles
-  through single buffers (and, for whole prompts, stores some tiles to the cache); the
-  set's softmax warps, which read S(g) from TMEM, agree whether the tile needs P's
-  remainder (a word per tile, three in rotation, and a barrier), write P(g) over S, zero
-  ragged V rows, rescale O, and read O out at the end of each unit;
-* one MMA issuer for both sets: S of each set's first tile, then in turn for each set
-  P V(g) and, once that product has completed, S(g + 1).
+* a K producer that takes the units from the queue, publishes them in a ring, loads each
+  unit's Q and streams K tiles through two buffers (tile g in buffer g % 2); a V producer
+  that follows the ring and streams V tiles the same way (for whole prompts each also
+  stores some of its tiles to the cache);
+* softmax warps in pairs: the two warps of a pair own the same rows, one the first 64
+  columns of each tile, the other the last 64. Each reads its half of S(g) from one of
+  three S buffers in TMEM (tile g in buffer g % 3), exchanges its row maxima with its
+  partner (a slot per exchange, two in rotation, and a two-warp barrier), rescales its
+  half of O when the reference maximum moves, flags whether its rows need the tile's
+  remainder product, writes its half of P(g) over S(g), zeroes ragged V rows (first
+  halves); a unit's O is read out (after the row sums are exchanged) once the first tile
+  of the next unit is done, so that the unit's last P V runs meanwhile;
+* one MMA issuer that polls the barriers without blocking and issues whatever is ready:
+  S(g) once K(g) has landed and P(g - 3) V(g - 3), which read the S buffer, completed --
+  so S runs up to three tiles ahead of the softmax -- and P V(g) once P(g) is written and
+  V(g) has landed.
 
 A random scheduler interleaves the roles; asynchronous operations complete later, in
 issue order per issuer (a commit arrives once everything its thread issued before it is
-done). The model asserts on every shared buffer -- the K, V and Q tiles, each set's S
-columns (which hold P after the softmax), each set's O accumulator -- that no write lands
-before the last reader of the previous contents is done and that every read sees the
-contents it expects; it reports a deadlock when no role and no operation can move.
+done). The model asserts on every shared buffer -- the K and V buffers, the Q buffer, the
+three S buffers (which hold P after the softmax), the O accumulator, the exchange slots
+-- that no write lands before the last reader of the previous contents is done and that
+every read sees the contents it expects; it reports a deadlock when no role and no
+operation can move.
 
-Barrier semantics follow the mbarrier's phase parity: a wait on parity p passes once the
-phase with that parity has completed (a fresh barrier passes parity 1). One of the
+Barriers follow the mbarrier's phase parity: a wait names the phase it needs (the kernel
+passes that phase's parity) and passes once the phase has completed -- a fresh barrier
+passes the wait for phase -1. A parity wait is only sound while the barrier is at most
+one phase past the awaited one and not behind it, so the model also fails a wait (or a
+non-blocking test) that the parity would let through at any other phase. One of the
 kernel's waits is implied by another and kept only as a second guard: a unit's first
 P V waits for o_empty, but it also waits for p_full, and the softmax warps write the new
 unit's first P only after they have read the previous unit's O. The planted mistakes are
@@ -35,12 +47,13 @@ import random
 
 import pytest
 
-SETS = 2
+NS = 3          # S buffers
+NKV = 2         # K and V buffers
 
 
 class Bar:
     def __init__(self, name, count):
-        self.name, self.count, self.pending, self.phase = name, count, count, 0
+        self.name, self.count, self.pending, self.phase = name, count, count, 0   # phase: completed phases
 
     def arrive(self):
         assert self.pending > 0, f"over-arrival on {self.name}"
@@ -49,8 +62,9 @@ class Bar:
             self.phase += 1
             self.pending = self.count
 
-    def passed(self, parity):
-        return (self.phase & 1) != parity
+    def parity_passes(self, n):
+        """What the kernel's parity wait for phase n answers."""
+        return (self.phase & 1) != (n & 1)
 
 
 class Race(AssertionError):
@@ -62,266 +76,345 @@ def check(cond, msg):
         raise Race(msg)
 
 
-def simulate(units, seed, fresh=False, mutant=None, warps=2):
+def simulate(units, seed, fresh=False, mutant=None, quarters=1):
     """units: K/V tiles per unit, in the order the queue hands them out.
     fresh: whole-prompt prefill (tiles from the prompt rows, some stored to the cache).
-    warps: softmax warps per set (the kernel has 4; each arrives once per barrier phase)."""
+    quarters: row groups; each has a pair of softmax warps (the kernel has 4 pairs)."""
     rng = random.Random(seed)
     p_complete = rng.uniform(0.05, 0.5)         # how eagerly asynchronous operations land
+    W = 2 * quarters                            # softmax warps: warp w pairs with warp (w + quarters) % W
     B = {}
-    for c in range(SETS):
-        for n, cnt in (("s_full", 1), ("p_full", warps), ("pv_done", 1), ("k_full", 1), ("v_full", 1),
-                       ("k_empty", 1), ("q_full", 1), ("q_empty", 1), ("o_full", 1), ("o_empty", warps),
-                       ("vote", warps)):
-            B[f"{n}{c}"] = Bar(f"{n}{c}", cnt)
-        for i in range(4):
-            B[f"uq_full{c}_{i}"] = Bar(f"uq_full{c}_{i}", 1)
-            B[f"uq_empty{c}_{i}"] = Bar(f"uq_empty{c}_{i}", warps + 1)   # softmax warps and the MMA warp
+    for b in range(NS):
+        for n, cnt in (("s_full", 1), ("p_full", W), ("pv_done", 1)):
+            B[f"{n}.{b}"] = Bar(f"{n}.{b}", cnt)
+    for x in range(NKV):
+        for n in ("k_full", "v_full"):
+            B[f"{n}.{x}"] = Bar(f"{n}.{x}", 1)
+    for n, cnt in (("q_full", 1), ("q_empty", 1), ("o_full", 1), ("o_empty", W)):
+        B[n] = Bar(n, cnt)
+    for q in range(quarters):
+        B[f"xchg.{q}"] = Bar(f"xchg.{q}", 2)
+    for i in range(4):
+        B[f"uq_full_{i}"] = Bar(f"uq_full_{i}", 1)
+        B[f"uq_empty_{i}"] = Bar(f"uq_empty_{i}", W + 2)   # softmax warps, the MMA warp, the V producer
+
+    def partner(w):
+        return w + quarters if w < quarters else w - quarters
 
     # what each shared buffer holds and how far its readers got
-    Kb = [None] * SETS                # tile in the K buffer
-    Vb = [None] * SETS
-    Qb = [None] * SETS                # unit whose q rows are in the Q buffer
-    S = [None] * SETS                 # ("S", g) or ("P", g): the set's S columns
-    P_writers = [set() for _ in range(SETS)]
-    O = [None] * SETS                 # unit accumulating in the set's O
-    O_readers = [set() for _ in range(SETS)]
-    s_done = [-1] * SETS              # last S(g) completed
-    pv_done_t = [-1] * SETS           # last P(g) V(g) completed
-    pv_issued = [-1] * SETS
-    stores = [0] * SETS               # cache stores still reading the set's K / V buffers
-    uq = [[None] * 4 for _ in range(SETS)]
-    vote_word = [[0, 0, 0] for _ in range(SETS)]   # the remainder vote, three words in rotation
-    vote_need = [{} for _ in range(SETS)]          # tile -> OR of the warps' needs
-    vote_seen = [{} for _ in range(SETS)]          # tile -> the answers the warps read
+    Kb = [None] * NKV                   # tile in each K buffer
+    Vb = [None] * NKV
+    Qb = [None]                         # unit whose q rows are in the Q buffer
+    S = [None] * NS                     # ("S", g) or ("P", g)
+    P_writers = [set() for _ in range(NS)]
+    O = [None]                          # unit accumulating in O
+    O_readers = set()
+    s_done = [-1]                       # last S(g) completed (they complete in order)
+    pv_done_t = [-1]                    # last P(g) V(g) completed
+    stores = {"K": 0, "V": 0}           # cache stores still reading the K / V buffers
+    uq = [None] * 4
+    lo_flag = [[(-1, False)] * W for _ in range(NS)]     # (tile, need) per buffer and warp
+    xslot = [[None] * W for _ in range(2)]               # exchange slots: the exchange number written
     units_done = []
     queue = {"next": 0}
     n_units = len(units)
+    last_s_of_unit = {}
 
-    def next_unit(c, k, taker=False):
-        slot, ph = k & 3, (k >> 2) & 1
-        if taker:
-            yield ("wait", f"uq_empty{c}_{slot}", ph ^ 1)
+    def owns(j):                        # whole prompts: this unit stores some of its tiles
+        return fresh and j % 2 == 0
+
+    # ---------------- K producer: units, Q, K tiles ----------------
+    def k_producer():
+        g, k = 0, 0
+        while True:
+            slot = k & 3
+            yield ("wait", f"uq_empty_{slot}", (k >> 2) - 1)
             u = queue["next"] if queue["next"] < n_units else -1
             queue["next"] += 1
-            uq[c][slot] = u
-            yield ("arrive", f"uq_full{c}_{slot}")
-            return u
-        yield ("wait", f"uq_full{c}_{slot}", ph)
-        u = uq[c][slot]
-        yield ("arrive", f"uq_empty{c}_{slot}")
-        return u
-
-    # ---------------- producer of set c ----------------
-    def producer(c):
-        g = 0
-        k = 0
-        while True:
-            u = yield from next_unit(c, k, taker=True)
+            uq[slot] = u
+            yield ("arrive", f"uq_full_{slot}")
             if u < 0:
                 break
             if mutant != "q_reload_early":
-                yield ("wait", f"q_empty{c}", (k & 1) ^ 1)
+                yield ("wait", "q_empty", k - 1)
 
-            def q_issue(c=c):
-                check(Qb[c] is None or s_done[c] >= last_s_of_unit.get((c, Qb[c]), -1),
-                      f"Q buffer of set {c} reloaded before the last S of unit {Qb[c]}")
-                Qb[c] = None
+            def q_issue():
+                check(Qb[0] is None or s_done[0] >= last_s_of_unit.get(Qb[0], -1),
+                      f"Q buffer reloaded before the last S of unit {Qb[0]}")
+                Qb[0] = None
 
-            def q_land(c=c, u=u):
-                Qb[c] = u
+            def q_land(u=u):
+                Qb[0] = u
             yield ("act", q_issue)
-            yield ("async", f"q_full{c}", q_land)
+            yield ("async", "q_full", q_land)
             for j in range(units[u]):
-                if mutant != "k_reload_early":
-                    yield ("wait", f"k_empty{c}", (g & 1) ^ 1)
-                if fresh:
-                    while stores[c] > 0 and mutant != "store_not_waited":
-                        yield ("spin",)
+                x = g % NKV
+                # K(g) once S(g - 2) has read the buffer
+                if g >= NKV and mutant != "k_reload_early":
+                    yield ("wait", f"s_full.{(g - NKV) % NS}", (g - NKV) // NS)
+                while fresh and stores["K"] > 0 and mutant != "store_not_waited":
+                    yield ("spin",)
 
-                def k_issue(c=c, g=g):
-                    check(stores[c] == 0, f"K buffer of set {c} reloaded under a cache store")
-                    check(s_done[c] >= g - 1, f"K buffer of set {c} reloaded before S of tile {g - 1}")
-                    Kb[c] = None
+                def k_issue(g=g, x=x):
+                    check(stores["K"] == 0, "K buffer reloaded under a cache store")
+                    check(s_done[0] >= g - NKV, f"K buffer {x} reloaded before S of tile {g - NKV}")
+                    Kb[x] = None
 
-                def k_land(c=c, g=g):
-                    Kb[c] = g
+                def k_land(g=g, x=x):
+                    Kb[x] = g
                 yield ("act", k_issue)
-                yield ("async", f"k_full{c}", k_land)
-                if mutant != "v_reload_early":
-                    yield ("wait", f"pv_done{c}", (g & 1) ^ 1)
+                yield ("async", f"k_full.{x}", k_land)
+                if owns(j):
+                    yield ("wait", f"k_full.{x}", g // NKV)
+                    stores["K"] += 1
 
-                def v_issue(c=c, g=g):
-                    check(stores[c] == 0, f"V buffer of set {c} reloaded under a cache store")
-                    check(pv_done_t[c] >= g - 1, f"V buffer of set {c} reloaded before P V of tile {g - 1}")
-                    Vb[c] = None
-
-                def v_land(c=c, g=g):
-                    Vb[c] = g
-                yield ("act", v_issue)
-                yield ("async", f"v_full{c}", v_land)
-                if fresh and j % 2 == 0:        # this unit owns some of its tiles: store them
-                    yield ("wait", f"k_full{c}", g & 1)
-                    yield ("wait", f"v_full{c}", g & 1)
-                    stores[c] += 1
-
-                    def store_done(c=c, g=g):
-                        check(Kb[c] == g and Vb[c] == g, f"cache store of tile {g} read a reloaded buffer")
-                        stores[c] -= 1
+                    def store_done(g=g, x=x):
+                        check(Kb[x] == g, f"cache store of K tile {g} read a reloaded buffer")
+                        stores["K"] -= 1
                     yield ("async", None, store_done)
                 g += 1
             k += 1
 
-    last_s_of_unit = {}
-
-    # ---------------- MMA issuer for both sets ----------------
-    def mma():
-        st = [{"live": True, "fresh": True, "j": 0, "g": 0, "k": 0, "u": None} for _ in range(SETS)]
-
-        def issue_s(c):
-            z = st[c]
-            if z["fresh"]:
-                u = yield from next_unit(c, z["k"])
-                if u < 0:
-                    z["live"] = False
-                    return False
-                z["u"], z["j"], z["fresh"] = u, 0, False
-                yield ("wait", f"q_full{c}", z["k"] & 1)
-            g, u = z["g"], z["u"]
-            yield ("wait", f"k_full{c}", g & 1)
-            if mutant != "s_before_pv_done":
-                yield ("wait", f"pv_done{c}", (g & 1) ^ 1)
-
-            def s_act(c=c, g=g, u=u):
-                check(Kb[c] == g, f"S of tile {g} reads another K tile")
-                check(Qb[c] == u, f"S of unit {u} reads the Q tile of unit {Qb[c]}")
-                check(pv_done_t[c] >= g - 1, f"S({g}) overwrites P({g - 1}) while P V reads it")
-
-            def s_land(c=c, g=g):
-                S[c] = ("S", g)
-                P_writers[c] = set()
-                s_done[c] = g
-            yield ("act", s_act)
-            yield ("async", f"s_full{c}", s_land)
-            yield ("async", f"k_empty{c}", None)
-            if z["j"] + 1 == units[u]:
-                last_s_of_unit[(c, u)] = g
-                yield ("async", f"q_empty{c}", None)
-            return True
-
-        def issue_pv(c):
-            z = st[c]
-            g, u, j = z["g"], z["u"], z["j"]
-            if mutant != "pv_before_p":
-                yield ("wait", f"p_full{c}", g & 1)
-            yield ("wait", f"v_full{c}", g & 1)
-            if j == 0 and z["k"] > 0 and mutant != "o_overwrite_early":
-                yield ("wait", f"o_empty{c}", (z["k"] & 1) ^ 1)
-
-            def pv_act(c=c, g=g, u=u, j=j):
-                check(S[c] == ("P", g) and len(P_writers[c]) == warps, f"P V of tile {g} reads an unfinished P")
-                check(Vb[c] == g, f"P V of tile {g} reads another V tile")
-                if j == 0:
-                    check(not O_readers[c], f"O of set {c} restarted while unit {O[c]} is read")
-                    O[c] = u
-                else:
-                    check(O[c] == u, "P V into another unit's accumulator")
-                pv_issued[c] = g
-
-            def pv_land(c=c, g=g):
-                pv_done_t[c] = g
-            yield ("act", pv_act)
-            yield ("async", f"pv_done{c}", pv_land)
-            z["g"] += 1
-            z["j"] += 1
-            if z["j"] == units[u]:
-
-                def o_land(c=c):
-                    O_readers[c] = set(range(warps))
-                yield ("async", f"o_full{c}", o_land)
-                z["fresh"] = True
-                z["k"] += 1
-
-        pend = []
-        for c in range(SETS):
-            pend.append((yield from issue_s(c)))
-        while any(pend):
-            for c in range(SETS):
-                if not pend[c]:
-                    continue
-                yield from issue_pv(c)
-                pend[c] = yield from issue_s(c)
-
-    # ---------------- softmax warp w of set c ----------------
-    def softmax(c, w):
+    # ---------------- V producer: follows the ring ----------------
+    def v_producer():
         g, k = 0, 0
         while True:
-            u = yield from next_unit(c, k)
+            slot = k & 3
+            yield ("wait", f"uq_full_{slot}", k >> 2)
+            u = uq[slot]
+            yield ("arrive", f"uq_empty_{slot}")
             if u < 0:
                 break
-            n = units[u]
-            for j in range(n):
-                yield ("wait", f"s_full{c}", g & 1)
-                yield ("act", lambda c=c, g=g: check(S[c] in (("S", g), ("P", g)), f"softmax read {S[c]}, not S({g})"))
-                if j > 0 and rng.random() < 0.3:   # the reference maximum moved: rescale O
-                    yield ("act", lambda c=c, g=g: check(pv_done_t[c] >= g - 1 and pv_issued[c] == g - 1,
-                                                         "O rescaled under a P V"))
+            for j in range(units[u]):
+                x = g % NKV
+                # V(g) once P(g - 2) V(g - 2) has read the buffer
+                if g >= NKV and mutant != "v_reload_early":
+                    yield ("wait", f"pv_done.{(g - NKV) % NS}", (g - NKV) // NS)
+                while fresh and stores["V"] > 0 and mutant != "store_not_waited":
+                    yield ("spin",)
 
-                # the remainder vote: warp 0 clears the next tile's word, every warp ORs its
-                # need into this tile's word, arrives, waits for the others, reads the answer
-                need = rng.random() < 0.3
-                if w == 0:
-                    slot = (g + 1) % 3 if mutant != "vote_clear_wrong_word" else g % 3
-                    yield ("act", lambda c=c, slot=slot: vote_word[c].__setitem__(slot, 0))
+                def v_issue(g=g, x=x):
+                    check(stores["V"] == 0, "V buffer reloaded under a cache store")
+                    check(pv_done_t[0] >= g - NKV, f"V buffer {x} reloaded before P V of tile {g - NKV}")
+                    Vb[x] = None
 
-                def vote(c=c, g=g, need=need):
-                    vote_need[c][g] = vote_need[c].get(g, False) or need
-                    if need:
-                        vote_word[c][g % 3] = 1
-                yield ("act", vote)
-                yield ("arrive", f"vote{c}")
-                if mutant != "vote_not_waited":
-                    yield ("wait", f"vote{c}", g & 1)
+                def v_land(g=g, x=x):
+                    Vb[x] = g
+                yield ("act", v_issue)
+                yield ("async", f"v_full.{x}", v_land)
+                if owns(j):
+                    yield ("wait", f"v_full.{x}", g // NKV)
+                    stores["V"] += 1
 
-                def read_vote(c=c, g=g):
-                    vote_seen[c].setdefault(g, []).append(vote_word[c][g % 3] != 0)
-                yield ("act", read_vote)
-
-                def p_write(c=c, g=g, w=w):
-                    check(pv_done_t[c] >= g - 1, f"P({g}) written over P({g - 1}) while P V reads it")
-                    S[c] = ("P", g)
-                    P_writers[c].add(w)
-                yield ("act", p_write)
-                if j == n - 1 and rng.random() < 0.5:   # a ragged tile: zero the V rows past the end
-                    if mutant != "zero_before_v_lands":
-                        yield ("wait", f"v_full{c}", g & 1)
-                    yield ("act", lambda c=c, g=g: check(Vb[c] == g, "zeroed rows of another V tile"))
-                yield ("arrive", f"p_full{c}")
+                    def store_done(g=g, x=x):
+                        check(Vb[x] == g, f"cache store of V tile {g} read a reloaded buffer")
+                        stores["V"] -= 1
+                    yield ("async", None, store_done)
                 g += 1
-            if mutant != "o_read_early":
-                yield ("wait", f"o_full{c}", k & 1)
-            yield ("act", lambda c=c, u=u, w=w: check(O[c] == u and w in O_readers[c] and pv_done_t[c] == g - 1,
-                                                      f"read O of unit {O[c]} before unit {u} was complete"))
-            yield ("act", lambda c=c, w=w: O_readers[c].discard(w))
-            yield ("arrive", f"o_empty{c}")
-            if w == 0:
-                units_done.append(u)
             k += 1
 
-    roles = {"MMA": mma()}
-    for c in range(SETS):
-        roles[f"PR{c}"] = producer(c)
-        for w in range(warps):
-            roles[f"SM{c}.{w}"] = softmax(c, w)
+    # ---------------- MMA issuer ----------------
+    def mma():
+        z = {"s_live": True, "s_fresh": True, "s_j": 0, "s_g": 0, "s_k": 0, "s_u": None,
+             "p_fresh": True, "p_j": 0, "p_g": 0, "p_k": 0, "p_u": None}
+        released = set()                # units whose ring slot this warp has released
+
+        def try_s():
+            if not z["s_live"] or z["s_g"] >= z["p_g"] + NS:
+                return False
+            if z["s_fresh"]:
+                slot = z["s_k"] & 3
+                if not (yield ("test", f"uq_full_{slot}", z["s_k"] >> 2)):
+                    return False
+                u = uq[slot]
+                if mutant == "ring_released_early":   # released when the S cursor reads it
+                    released.add(z["s_k"])
+                    yield ("arrive", f"uq_empty_{slot}")
+                if u < 0:
+                    z["s_live"] = False
+                    return True
+                z["s_u"], z["s_j"], z["s_fresh"] = u, 0, False
+            g, u = z["s_g"], z["s_u"]
+            b, x = g % NS, g % NKV
+            if z["s_j"] == 0 and not (yield ("test", "q_full", z["s_k"])):
+                return False
+            if not (yield ("test", f"k_full.{x}", g // NKV)):
+                return False
+            if g >= NS and mutant != "s_before_pv_done" and not (yield ("test", f"pv_done.{b}", g // NS - 1)):
+                return False
+
+            def s_act(g=g, u=u, b=b, x=x):
+                check(Kb[x] == g, f"S of tile {g} reads another K tile")
+                check(Qb[0] == u, f"S of unit {u} reads the Q tile of unit {Qb[0]}")
+                check(pv_done_t[0] >= g - NS, f"S({g}) overwrites P({g - NS}) while P V reads it")
+
+            def s_land(g=g, b=b):
+                S[b] = ("S", g)
+                P_writers[b] = set()
+                s_done[0] = g
+            yield ("act", s_act)
+            yield ("async", f"s_full.{b}", s_land)
+            if z["s_j"] + 1 == units[u]:
+                last_s_of_unit[u] = g
+                yield ("async", "q_empty", None)
+                z["s_fresh"] = True
+                z["s_k"] += 1
+            z["s_j"] += 1
+            z["s_g"] += 1
+            return True
+
+        def try_pv():
+            if z["p_g"] >= z["s_g"]:
+                return False
+            if z["p_fresh"]:
+                check(z["p_k"] not in released, f"the P V cursor reads ring slot of unit {z['p_k']} after releasing it")
+                z["p_u"], z["p_j"], z["p_fresh"] = uq[z["p_k"] & 3], 0, False
+            g, u, j = z["p_g"], z["p_u"], z["p_j"]
+            b, x = g % NS, g % NKV
+            if mutant != "pv_before_p" and not (yield ("test", f"p_full.{b}", g // NS)):
+                return False
+            if not (yield ("test", f"v_full.{x}", g // NKV)):
+                return False
+            if j == 0 and z["p_k"] > 0 and mutant != "o_overwrite_early" and \
+                    not (yield ("test", "o_empty", z["p_k"] - 1)):
+                return False
+
+            def pv_act(g=g, u=u, j=j, b=b, x=x):
+                check(S[b] == ("P", g) and len(P_writers[b]) == W, f"P V of tile {g} reads an unfinished P")
+                check(all(t == g for t, _ in lo_flag[b]), f"remainder flags of tile {g} read as {lo_flag[b]}")
+                check(Vb[x] == g, f"P V of tile {g} reads another V tile")
+                if j == 0:
+                    check(not O_readers, f"O restarted while unit {O[0]} is read")
+                    O[0] = u
+                else:
+                    check(O[0] == u, "P V into another unit's accumulator")
+
+            def pv_land(g=g):
+                check(pv_done_t[0] == g - 1, "P V products completed out of order")
+                pv_done_t[0] = g
+            yield ("act", pv_act)
+            yield ("async", f"pv_done.{b}", pv_land)
+            z["p_g"] += 1
+            z["p_j"] += 1
+            if z["p_j"] == units[u]:
+
+                def o_land():
+                    O_readers.update(range(W))
+                yield ("async", "o_full", o_land)
+                if mutant != "ring_released_early":
+                    released.add(z["p_k"])
+                    yield ("arrive", f"uq_empty_{z['p_k'] & 3}")
+                z["p_fresh"] = True
+                z["p_k"] += 1
+            return True
+
+        while z["s_live"] or z["p_g"] < z["s_g"]:
+            moved = yield from try_pv()
+            moved |= yield from try_s()
+            if not moved:
+                yield ("spin",)
+
+    # ---------------- softmax warp w: row group w % quarters, column half w // quarters ----------------
+    def softmax(w):
+        q, h = w % quarters, w // quarters
+        g, k, xn = 0, 0, 0
+
+        def exchange():
+            nonlocal xn
+            s = xn & 1 if mutant != "xchg_one_slot" else 0
+            n = xn
+            yield ("act", lambda s=s, n=n: xslot[s].__setitem__(w, n))
+            yield ("arrive", f"xchg.{q}")
+            if mutant != "xchg_not_waited":
+                yield ("wait", f"xchg.{q}", n)
+            yield ("act", lambda s=s, n=n: check(xslot[s][partner(w)] == n,
+                                                 f"warp {w} read exchange {xslot[s][partner(w)]}, not {n}"))
+            xn += 1
+
+        def epilogue(kk, uu, gl):
+            """Unit kk's O: the row sums exchanged, O read once the unit's last P V completed."""
+            if mutant != "o_read_early":
+                yield ("wait", "o_full", kk)
+            yield from exchange()              # row sums of the two halves
+            yield ("act", lambda: check(O[0] == uu and w in O_readers and pv_done_t[0] >= gl,
+                                        f"read O of unit {O[0]} before unit {uu} was complete"))
+            yield ("act", lambda: O_readers.discard(w))
+            yield ("arrive", "o_empty")
+            if w == 0:
+                units_done.append(uu)
+
+        pend = None                            # the previous unit, whose O is read after this unit's first tile
+        while True:
+            slot = k & 3
+            yield ("wait", f"uq_full_{slot}", k >> 2)
+            u = uq[slot]
+            yield ("arrive", f"uq_empty_{slot}")
+            if u < 0:
+                break
+            n_t = units[u]
+            for j in range(n_t):
+                b = g % NS
+                yield ("wait", f"s_full.{b}", g // NS)
+                yield ("act", lambda g=g, b=b: check(S[b] in (("S", g), ("P", g)), f"softmax read {S[b]}, not S({g})"))
+                yield from exchange()          # row maxima of the two halves
+                if j > 0 and rng.random() < 0.3:   # the reference maximum moved: rescale O
+                    if mutant != "rescale_before_pv_done":
+                        yield ("wait", f"pv_done.{(g - 1) % NS}", (g - 1) // NS)
+                    yield ("act", lambda g=g: check(pv_done_t[0] >= g - 1, "O rescaled under a P V"))
+                need = rng.random() < 0.3
+
+                def flag(g=g, b=b, need=need):
+                    lo_flag[b][w] = (g, need)
+                if mutant != "flag_after_p_full":
+                    yield ("act", flag)
+
+                def p_write(g=g, b=b):
+                    check(pv_done_t[0] >= g - NS, f"P({g}) written over P({g - NS}) while P V reads it")
+                    S[b] = ("P", g)
+                    P_writers[b].add(w)
+                yield ("act", p_write)
+                if h == 0 and j == n_t - 1 and rng.random() < 0.5:   # a ragged tile: zero the V rows past the end
+                    if mutant != "zero_before_v_lands":
+                        yield ("wait", f"v_full.{g % NKV}", g // NKV)
+                    yield ("act", lambda g=g: check(Vb[g % NKV] == g, "zeroed rows of another V tile"))
+                yield ("arrive", f"p_full.{b}")
+                if mutant == "flag_after_p_full":
+                    yield ("act", flag)
+                g += 1
+                if j == 0 and pend is not None:
+                    yield from epilogue(*pend)
+                    pend = None
+            pend = (k, u, g - 1)
+            k += 1
+        if pend is not None:
+            yield from epilogue(*pend)
+
+    roles = {"MMA": mma(), "KP": k_producer(), "VP": v_producer()}
+    for w in range(W):
+        roles[f"SM{w}"] = softmax(w)
     waiting = {r: None for r in roles}
     resume = {r: None for r in roles}
     done = set()
     pending = []                       # (issuer, seq, bar, callback)
     seq = 0
-    for step in range(4_000_000):
-        ready = [r for r in roles if r not in done and
-                 (waiting[r] is None or (waiting[r][0] == "wait" and B[waiting[r][1]].passed(waiting[r][2]))
-                  or waiting[r][0] == "spin")]
+
+    def parity_state(r, name, n):
+        """The kernel's parity answer for phase n of barrier `name`, checked for soundness."""
+        bar = B[name]
+        if not bar.parity_passes(n):
+            check(bar.phase <= n + 1, f"{r} waits for phase {n} of {name}, already at {bar.phase}")
+            return False
+        check(bar.phase == n + 1, f"{r}: the parity of phase {n} of {name} passes at phase {bar.phase}")
+        return True
+
+    def can_go(r):
+        op = waiting[r]
+        if op is None or op[0] == "spin":
+            return True
+        return parity_state(r, op[1], op[2])
+
+    for step in range(6_000_000):
+        ready = [r for r in roles if r not in done and can_go(r)]
         if not ready and not pending:
             if len(done) == len(roles):
                 break
@@ -346,7 +439,9 @@ def simulate(units, seed, fresh=False, mutant=None, warps=2):
             continue
         resume[r] = None
         kind = op[0]
-        if kind in ("wait", "spin"):
+        if kind == "test":                # non-blocking: the role continues with the answer
+            resume[r] = parity_state(r, op[1], op[2])
+        elif kind in ("wait", "spin"):
             waiting[r] = op
         elif kind == "arrive":
             B[op[1]].arrive()
@@ -359,10 +454,7 @@ def simulate(units, seed, fresh=False, mutant=None, warps=2):
     else:
         raise Race("no progress bound reached")
     check(sorted(units_done) == list(range(n_units)), "not every unit finished")
-    for c in range(SETS):
-        for g, seen in vote_seen[c].items():
-            check(all(v == vote_need[c][g] for v in seen), f"set {c} disagreed on the remainder of tile {g}")
-    check(all(v == 0 for v in stores), "cache stores still in flight at the end")
+    check(stores["K"] == 0 and stores["V"] == 0, "cache stores still in flight at the end")
 
 
 def _workloads(n, seed):
@@ -376,21 +468,24 @@ def test_schedule_has_no_race_and_no_deadlock(fresh):
         simulate(units, seed=i, fresh=fresh)
 
 
-def test_schedule_with_four_softmax_warps_per_set():
+def test_schedule_with_four_warp_pairs():
     for i, units in enumerate(_workloads(60, 21)):
-        simulate(units, seed=i, fresh=i % 2 == 1, warps=4)
+        simulate(units, seed=i, fresh=i % 2 == 1, quarters=4)
 
 
 @pytest.mark.parametrize("mutant,fresh", [
-    ("k_reload_early", False),       # K(g) loaded before S(g-1) has read the buffer
-    ("v_reload_early", False),       # V(g) loaded before P(g-1) V(g-1) has read the buffer
+    ("k_reload_early", False),       # K(g) loaded before S(g-2) has read the buffer
+    ("v_reload_early", False),       # V(g) loaded before P(g-2) V(g-2) has read the buffer
     ("q_reload_early", False),       # the next unit's Q loaded before this unit's last S
-    ("s_before_pv_done", False),     # S(g) written over P(g-1) while P(g-1) V(g-1) reads it
+    ("s_before_pv_done", False),     # S(g) written over P(g-3) while P(g-3) V(g-3) reads it
     ("pv_before_p", False),          # P V issued before every warp has written P
     ("o_read_early", False),         # O read out before the unit's last P V completed
     ("zero_before_v_lands", False),  # V rows zeroed before the tile's load has landed
-    ("vote_not_waited", False),      # the remainder vote read before every warp has voted
-    ("vote_clear_wrong_word", False),  # warp 0 clears the word of the tile being voted on
+    ("rescale_before_pv_done", False),  # O rescaled while the previous tile's P V may run
+    ("flag_after_p_full", False),    # a warp's remainder flag written after it signalled P
+    ("xchg_not_waited", False),      # the partner's maxima read before it wrote them
+    ("xchg_one_slot", False),        # one exchange slot: overwritten before the partner read it
+    ("ring_released_early", False),  # the MMA warp frees a ring slot before its P V cursor read it
     ("store_not_waited", True),      # a K/V buffer reloaded while a cache store still reads it
 ])
 def test_planted_schedule_mistakes_are_caught(mutant, fresh):
