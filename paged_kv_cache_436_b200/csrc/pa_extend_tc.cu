@@ -528,6 +528,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     bool ok = true;
     for (uint32_t k = 0; ok; ++k) {
       int u = -1;
+      TcUnit x{};
       if (isk) {
         const int slot = k & 3;
         if (!(ok = tc_wait_warp(&uq_empty[slot], ((k >> 2) & 1) ^ 1, abort, 28, int(k)))) break;
@@ -537,16 +538,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           if (v >= total) v = -1;
         }
         u = __shfl_sync(kFull, v, 0);
+        if (u >= 0) x = tc_unit(p, u);
         if (lane == 0) {
           uq[slot] = u;
-          uq_nt[slot] = u < 0 ? 0 : tc_unit(p, u).ntiles;
+          uq_nt[slot] = u < 0 ? 0 : x.ntiles;
           mbar_arrive(&uq_full[slot]);
         }
-      } else if (!(ok = read_unit(k, u))) {
-        break;
+      } else {
+        if (!(ok = read_unit(k, u))) break;
+        if (u >= 0) x = tc_unit(p, u);
       }
       if (u < 0) break;
-      const TcUnit x = tc_unit(p, u);
       if (isk) {
         // the unit's q rows, once the last S of the previous unit has read the buffer
         if (!(ok = tc_wait_warp(&q_empty, (k & 1) ^ 1, abort, 26, u))) break;
@@ -832,7 +834,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int qi = x.t * QPT + row / G;
       const bool has_q = qi < x.Q;
       const int qpos = has_q ? x.base + qi : -1;
-      float m_ref = -INFINITY, l = 0.f;   // l: this half's share of the row sum
+      float m_ref = -INFINITY, l = 0.f;   // l: this warp's columns' share of the row sum
       for (int j = 0; j < x.ntiles; ++j, ++g) {
         const int b = g % kTcSBufs;
         const uint32_t c_s = b * kTcTok + h * kTcHalf;   // this half of S(g), then of P(g)
