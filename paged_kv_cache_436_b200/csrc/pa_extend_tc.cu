@@ -24,8 +24,8 @@
 //     and V in its [token][dim] cache layout (MN-major B operand). S(g) is issued once
 //     K(g) has landed and P(g - 3) V(g - 3), which read its buffer, completed, so the
 //     scores of the next tiles are ready while the softmax works on tile g; P(g) V(g) once
-//     the softmax has written P(g). The MMA warp tests the barriers without blocking and
-//     issues each product's 8 MMAs from one block of instructions;
+//     the softmax has written P(g). One thread of the MMA warp tests the barriers without
+//     blocking and issues each product's 8 MMAs from one block of instructions;
 //   * the softmax keeps a reference maximum that moves only when the row maximum passes
 //     it by more than 2^8 (O and the running sum are then rescaled; every p stays below
 //     2^8). For bf16, p rounded to bf16 can leave the parity tolerance when a few
@@ -632,64 +632,59 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // which reads the buffer, completed -- so S runs up to three tiles (and units) ahead of
     // the softmax; P V(g) once the softmax has written P(g) and V(g) has landed. Both
     // cursors read the units from the ring; the slot is released when the P V cursor is
-    // done with the unit. Lane 0 tests the barriers without blocking and issues whatever
-    // is ready; the other lanes follow its decisions.
-    const uint32_t idS = tc_idesc<QD>(0, kTcTok), idO = tc_idesc<QD>(1, kTcD);
-    const uint64_t dq = tc_desc(smem_addr(sm + TcSmem::kQ), 1024, 16);
-    const uint64_t dk0 = tc_desc(smem_addr(sm + TcSmem::kK), 1024, 16);
-    const uint64_t dv0 = tc_desc(smem_addr(sm + TcSmem::kV), 1024, kTcTok * 128);
-    constexpr uint64_t kKvDesc = TcSmem::kKvTile >> 4;   // one K / V buffer in descriptor units
-    int s_nt = 0, p_nt = 0;   // K/V tiles of the S cursor's and of the P V cursor's unit
-    int js = 0, jp = 0;
-    uint32_t gs = 0, gp = 0, ks = 0, kp = 0;
-    bool s_live = true, s_fresh = true, p_fresh = true;
-    auto lane0 = [&](bool v) { return __shfl_sync(kFull, v ? 1 : 0, 0) != 0; };
-    auto try_s = [&]() -> bool {
-      if (!s_live || gs >= gp + kTcSBufs) return false;
-      if (s_fresh) {
-        const int slot = ks & 3;
-        if (!lane0(lane == 0 && mbar_test(&uq_full[slot], (ks >> 2) & 1))) return false;
-        int u = lane == 0 ? *reinterpret_cast<volatile int*>(&uq[slot]) : 0;
-        u = __shfl_sync(kFull, u, 0);
-        if (u < 0) {
-          s_live = false;
-          return true;
+    // done with the unit. One thread (lane 0) runs the issuer: it tests the barriers
+    // without blocking and issues whatever is ready; the other lanes wait for it.
+    if (lane == 0) {
+      const uint32_t idS = tc_idesc<QD>(0, kTcTok), idO = tc_idesc<QD>(1, kTcD);
+      const uint64_t dq = tc_desc(smem_addr(sm + TcSmem::kQ), 1024, 16);
+      const uint64_t dk0 = tc_desc(smem_addr(sm + TcSmem::kK), 1024, 16);
+      const uint64_t dv0 = tc_desc(smem_addr(sm + TcSmem::kV), 1024, kTcTok * 128);
+      constexpr uint64_t kKvDesc = TcSmem::kKvTile >> 4;   // one K / V buffer in descriptor units
+      int s_nt = 0, p_nt = 0;   // K/V tiles of the S cursor's and of the P V cursor's unit
+      int js = 0, jp = 0;
+      uint32_t gs = 0, gp = 0, ks = 0, kp = 0;
+      bool s_live = true, s_fresh = true, p_fresh = true;
+      auto try_s = [&]() -> bool {
+        if (!s_live || gs >= gp + kTcSBufs) return false;
+        if (s_fresh) {
+          const int slot = ks & 3;
+          if (!mbar_test(&uq_full[slot], (ks >> 2) & 1)) return false;
+          const int u = *reinterpret_cast<volatile int*>(&uq[slot]);
+          if (u < 0) {
+            s_live = false;
+            return true;
+          }
+          s_nt = *reinterpret_cast<volatile int*>(&uq_nt[slot]);
+          js = 0;
+          s_fresh = false;
         }
-        s_nt = *reinterpret_cast<volatile int*>(&uq_nt[slot]);
-        js = 0;
-        s_fresh = false;
-      }
-      const int b = gs % kTcSBufs, xb = gs & 1;
-      if (!lane0(lane == 0 && (js > 0 || mbar_test(&q_full, ks & 1)) && mbar_test(&k_full[xb], (gs >> 1) & 1) &&
-                 mbar_test(&pv_done[b], ((gs / kTcSBufs) & 1) ^ 1)))
-        return false;
-      if (lane == 0) {
+        const int b = gs % kTcSBufs, xb = gs & 1;
+        if (!((js > 0 || mbar_test(&q_full, ks & 1)) && mbar_test(&k_full[xb], (gs >> 1) & 1) &&
+              mbar_test(&pv_done[b], ((gs / kTcSBufs) & 1) ^ 1)))
+          return false;
         tc_fence_after();
         tc_mma_s8(tmem + b * kTcTok, dq, dk0 + xb * kKvDesc, idS);
         tc_commit(&s_full[b]);
         if (js + 1 == s_nt) tc_commit(&q_empty);   // the Q buffer is free once this S completes
-      }
-      __syncwarp();
-      ++gs;
-      if (++js == s_nt) {
-        s_fresh = true;
-        ++ks;
-      }
-      return true;
-    };
-    // a unit's first P V overwrites O, so it also waits until the previous unit's O was read
-    auto try_pv = [&]() -> bool {
-      if (gp >= gs) return false;
-      if (p_fresh) {   // the unit of this tile: the S cursor has read its slot already
-        p_nt = *reinterpret_cast<volatile int*>(&uq_nt[kp & 3]);
-        jp = 0;
-        p_fresh = false;
-      }
-      const int b = gp % kTcSBufs, xb = gp & 1;
-      if (!lane0(lane == 0 && mbar_test(&p_full[b], (gp / kTcSBufs) & 1) && mbar_test(&v_full[xb], (gp >> 1) & 1) &&
-                 (jp > 0 || kp == 0 || mbar_test(&o_empty, (kp & 1) ^ 1))))
-        return false;
-      if (lane == 0) {
+        ++gs;
+        if (++js == s_nt) {
+          s_fresh = true;
+          ++ks;
+        }
+        return true;
+      };
+      // a unit's first P V overwrites O, so it also waits until the previous unit's O was read
+      auto try_pv = [&]() -> bool {
+        if (gp >= gs) return false;
+        if (p_fresh) {   // the unit of this tile: the S cursor has read its slot already
+          p_nt = *reinterpret_cast<volatile int*>(&uq_nt[kp & 3]);
+          jp = 0;
+          p_fresh = false;
+        }
+        const int b = gp % kTcSBufs, xb = gp & 1;
+        if (!(mbar_test(&p_full[b], (gp / kTcSBufs) & 1) && mbar_test(&v_full[xb], (gp >> 1) & 1) &&
+              (jp > 0 || kp == 0 || mbar_test(&o_empty, (kp & 1) ^ 1))))
+          return false;
         // the remainder product: every tile, or (adaptive) when a softmax warp flagged it
         const bool lo = p.lo_mode == kLoAlways ||
                         (p.lo_mode == kLoAdaptive && *reinterpret_cast<volatile unsigned long long*>(lo_need[b]) != 0);
@@ -700,45 +695,40 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (lo) tc_mma_pv8(d, a + 8, dv, idO, 1u);      // their remainders, 8 columns further
         tc_commit(&pv_done[b]);
         if (jp + 1 == p_nt) tc_commit(&o_full);
-      }
-      __syncwarp();
-      ++gp;
-      if (++jp == p_nt) {   // the unit is done: release its ring slot
-        if (lane == 0) mbar_arrive(&uq_empty[kp & 3]);
-        p_fresh = true;
-        ++kp;
-      }
-      return true;
-    };
-    uint64_t t_idle = 0;   // lane 0: since when nothing was ready
-    while (s_live || gp < gs) {
-      bool moved = try_pv();
-      moved |= try_s();
-      if (moved) {
-        t_idle = 0;
-        continue;
-      }
-      // nothing ready: lane 0 sleeps in the blocking test of the barrier the next P V needs
-      // (it returns when the phase completes or after the hardware's time limit), or
-      // briefly when no P V is pending, so that the polling takes no issue slots from the
-      // softmax warps of its sub-partition; it gives up after 2 s without progress, or once
-      // another role aborted
-      bool stop = false;
-      if (lane == 0) {
+        ++gp;
+        if (++jp == p_nt) {   // the unit is done: release its ring slot
+          mbar_arrive(&uq_empty[kp & 3]);
+          p_fresh = true;
+          ++kp;
+        }
+        return true;
+      };
+      uint64_t t_idle = 0;   // since when nothing was ready
+      while (s_live || gp < gs) {
+        bool moved = try_pv();
+        moved |= try_s();
+        if (moved) {
+          t_idle = 0;
+          continue;
+        }
+        // nothing ready: sleep in the blocking test of the barrier the next P V needs (it
+        // returns when the phase completes or after the hardware's time limit), or briefly
+        // when no P V is pending, so that the polling takes no issue slots from the softmax
+        // warps of this sub-partition; give up after 2 s without progress, or once another
+        // role aborted
         if (gp < gs) mbar_try_wait(&p_full[gp % kTcSBufs], (gp / kTcSBufs) & 1);
         else __nanosleep(200);
         const uint64_t now = global_timer_ns();
         if (t_idle == 0) t_idle = now;
-        if (*abort) {
-          stop = true;
-        } else if (now - t_idle > 2000000000ull) {
+        if (*abort) break;
+        if (now - t_idle > 2000000000ull) {
           record_error(PA_DEV_WAIT_TIMEOUT, 30, int(gs), int(gp));
           *abort = 1;
-          stop = true;
+          break;
         }
       }
-      if (lane0(stop)) break;
     }
+    __syncwarp();
   } else {
     // ---------------- softmax warps: rows of quarter rq, columns [64 h, 64 h + 64) of each tile ----------------
     const int rq = warp % kTcQuarters, h = warp / kTcQuarters, row = rq * 32 + lane;

@@ -16,7 +16,8 @@ asynchronous operations (TMA loads and stores, MMAs with their commits):
   remainder product, writes its half of P(g) over S(g), zeroes ragged V rows (first
   halves); a unit's O is read out (after the row sums are exchanged) once the first tile
   of the next unit is done, so that the unit's last P V runs meanwhile;
-* one MMA issuer that polls the barriers without blocking and issues whatever is ready:
+* one MMA issuer (one thread) that polls the barriers without blocking and issues whatever
+  is ready:
   S(g) once K(g) has landed and P(g - 3) V(g - 3), which read the S buffer, completed --
   so S runs up to three tiles ahead of the softmax -- and P V(g) once P(g) is written and
   V(g) has landed.
