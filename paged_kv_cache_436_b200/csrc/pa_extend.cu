@@ -837,13 +837,22 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
 }
 
 // One block of E4M3 rows (BS x D bytes, row-major) into the f16 staging tile, rows from
-// `keep` on set to zero. Lane-strided 16-byte chunks: conflict-free reads of whole rows.
+// `keep` on set to zero. Each lane converts 16-byte chunks (16 codes into two 16-byte f16
+// chunks); every 8-lane phase of the reads and of the stores touches all 32 banks once.
 template <int D, int BS>
 __device__ __forceinline__ void fp8_block_to_f16(const uint8_t* src, uint8_t* dst, int keep, int lane) {
   constexpr int CPR = D / 16;   // 16-byte chunks (16 codes) per row
 #pragma unroll
   for (int idx = lane; idx < BS * CPR; idx += 32) {
-    const int r = idx / CPR, cb = idx - r * CPR;
+    int r = idx / CPR, cb = idx - r * CPR;
+    if constexpr (CPR >= 8) {
+      // rows in pairs, each 8-lane phase four chunks of the even row and four of the odd
+      // row, taken from different 64-byte halves: the reads cover all 32 banks and the two
+      // rows' swizzled destinations fill complementary bank groups
+      const int w = idx % (2 * CPR), g = w >> 3, k = w & 7, rb = k >> 2;
+      r = (idx / (2 * CPR)) * 2 + rb;
+      cb = 4 * (g ^ rb) + (k & 3);
+    }
     uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
     if (r < keep) {
       const uint4 raw = *reinterpret_cast<const uint4*>(src + r * D + cb * 16);
