@@ -285,6 +285,20 @@ __device__ __forceinline__ bool tc_wait_warp(uint64_t* bar, uint32_t parity, vol
   return __all_sync(kFull, tc_wait(bar, parity, abort, where, u));
 }
 
+// As mbar_try_wait, with a bound on how long the hardware may suspend the thread while
+// the phase is incomplete (nanoseconds; it resumes earlier when the phase completes).
+__device__ __forceinline__ bool mbar_try_wait_for(uint64_t* bar, uint32_t parity, uint32_t suspend_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity), "r"(suspend_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Non-blocking test: has the phase with this parity completed (as this thread sees it)?
 __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
@@ -712,11 +726,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           continue;
         }
         // nothing ready: sleep in the blocking test of the barrier the next P V needs (it
-        // returns when the phase completes or after the hardware's time limit), or briefly
-        // when no P V is pending, so that the polling takes no issue slots from the softmax
-        // warps of this sub-partition; give up after 2 s without progress, or once another
-        // role aborted
-        if (gp < gs) mbar_try_wait(&p_full[gp % kTcSBufs], (gp / kTcSBufs) & 1);
+        // returns when the phase completes or after at most 20 us), or briefly when no P V
+        // is pending, so that the polling takes no issue slots from the softmax warps of
+        // this sub-partition; give up after 2 s without progress, or once another role
+        // aborted
+        if (gp < gs) mbar_try_wait_for(&p_full[gp % kTcSBufs], (gp / kTcSBufs) & 1, 20000u);
         else __nanosleep(200);
         const uint64_t now = global_timer_ns();
         if (t_idle == 0) t_idle = now;
