@@ -280,6 +280,24 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile
   }
 }
 
+// As tc_wait, polling with the non-blocking test: for the short waits between the two
+// softmax warps of a row quarter, where a suspended thread would wake later than the
+// phase completes.
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity);
+__device__ __forceinline__ bool tc_spin(uint64_t* bar, uint32_t parity, volatile int* abort, int where, int u) {
+  if (mbar_test(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    if (mbar_test(bar, parity)) return true;
+    if (*abort) return false;
+    if (global_timer_ns() - t0 > 2000000000ull) {
+      record_error(PA_DEV_WAIT_TIMEOUT, where, u, int(parity));
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
 // Warp-uniform form: true only if every lane's wait succeeded.
 __device__ __forceinline__ bool tc_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort, int where, int u) {
   return __all_sync(kFull, tc_wait(bar, parity, abort, where, u));
@@ -754,7 +772,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       xval[xn & 1][warp][lane] = v;
       __syncwarp();
       if (lane == 0) mbar_arrive(&xchg[rq]);
-      if (!tc_wait_warp(&xchg[rq], xn & 1, abort, 23, int(xn))) return false;
+      if (!__all_sync(kFull, tc_spin(&xchg[rq], xn & 1, abort, 23, int(xn)))) return false;
       volatile float* o = reinterpret_cast<volatile float*>(&xval[xn & 1][partner][lane]);
       other = make_float2(o[0], o[1]);
       ++xn;
