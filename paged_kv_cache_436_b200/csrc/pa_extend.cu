@@ -866,6 +866,31 @@ __device__ __forceinline__ void fp8_block_to_f16(const uint8_t* src, uint8_t* ds
   }
 }
 
+// P of one 16-token slice as f16 A operands. Rows r0 + 8 (h = 1) only when some row of the
+// tile's upper half is a real query row (else their operands are left zero: those rows'
+// outputs are never read); l adds what enters the products.
+__device__ __forceinline__ void make_p_f16(const float (&sc)[2][4], const float (&base_m)[2], uint32_t (&pa)[4],
+                                           float (&l)[2], bool hi_rows) {
+  float lh[2] = {0.f, 0.f};
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      if (h == 1 && !hi_rows) {
+        pa[nt * 2 + h] = 0u;
+        continue;
+      }
+      float p0, p1;   // 2^x on the special-function unit (results below 2^-126 are 0)
+      asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(p0) : "f"(sc[nt][2 * h] - base_m[h]));
+      asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(p1) : "f"(sc[nt][2 * h + 1] - base_m[h]));
+      float r0, r1;
+      pa[nt * 2 + h] = pack2<PA_F16>(p0, p1, r0, r1);
+      lh[h] += r0 + r1;
+    }
+  l[0] += lh[0];
+  l[1] += lh[1];
+}
+
 template <int QD, int D, int BS, int G>
 __global__ void __launch_bounds__(Fp8Cfg<D, BS>::kThreads) extend_fp8_kernel(const ExtendParams p) {
   using C = Fp8Cfg<D, BS>;
@@ -912,6 +937,9 @@ __global__ void __launch_bounds__(Fp8Cfg<D, BS>::kThreads) extend_fp8_kernel(con
         tok[h] = -1;
       }
     }
+    // whether any of the tile's rows 8 .. 15 is a query row (a warp-uniform skip of their
+    // softmax otherwise: with few queries per tile only the first rows are real)
+    const bool hi = __any_sync(kFull, tok[1] >= 0);
     // Q fragments as f16 pairs (scaled by 2^-8 from bf16), zero for missing rows
     uint32_t qa[KK][4];
 #pragma unroll
@@ -990,6 +1018,7 @@ __global__ void __launch_bounds__(Fp8Cfg<D, BS>::kThreads) extend_fp8_kernel(con
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int h = e >> 1;
+            if (h == 1 && !hi) break;
             const int tp = tok0 + sb * 16 + nt * 8 + cq + (e & 1);
             float v = sc[sb][nt][e] * s_mul;
             if (tp > qpos[h]) v = -INFINITY;
@@ -998,6 +1027,7 @@ __global__ void __launch_bounds__(Fp8Cfg<D, BS>::kThreads) extend_fp8_kernel(con
           }
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
+          if (h == 1 && !hi) break;
           mx[h] = fmaxf(mx[h], __shfl_xor_sync(kFull, mx[h], 1));
           mx[h] = fmaxf(mx[h], __shfl_xor_sync(kFull, mx[h], 2));
         }
@@ -1016,8 +1046,8 @@ __global__ void __launch_bounds__(Fp8Cfg<D, BS>::kThreads) extend_fp8_kernel(con
           }
           base_m[h] = m[h] == -INFINITY ? 0.f : m[h];
         }
-        uint32_t pa[4], pl[4];
-        make_p_operands<PA_F16>(sc[sb], base_m, pa, pl, l);
+        uint32_t pa[4];
+        make_p_f16(sc[sb], base_m, pa, l, hi);
 #pragma unroll
         for (int np = 0; np < NT / 2; ++np) {
           uint32_t b[4];
