@@ -53,7 +53,7 @@ struct ExtendParams {
   int4* units;                  // optional: two int4 per (seq, tile, chunk) pair, written by the plan
                                 //   {s, tile, chunk index, row0}, {Q, base, first token, visible tokens}
   long long units_cap;          // pairs the records can hold
-  int* queue;                   // tcgen05 path: next unit to hand out (zeroed by the plan kernel)
+  int* queue;                   // next unit to hand out (zeroed by the plan kernel); null: round-robin
   int* row_parts;               // [T] chunks query row t's context spans (0: no valid query);
                                 //   null when no merge pass follows
   int fresh;                    // whole prompts (pa_prefill): every L_s must equal Q_s
@@ -182,7 +182,7 @@ __global__ void __launch_bounds__(1024) extend_plan_kernel(const ExtendParams p,
     for (int i = lane; i < Q; i += 32) p.row_parts[row0 + i] = (base + i + 1 + p.chunk - 1) / p.chunk;
   }
   if (threadIdx.x == 0) {
-    if (p.queue) *p.queue = 0;   // the tcgen05 kernel's work queue
+    if (p.queue) *p.queue = 0;   // the extend kernels' work queue
     // pairs past the records' capacity (only from inconsistent query_start) are dropped
     if (p.units && carry > p.units_cap) record_error(PA_DEV_BAD_CONTEXT_LEN, -1, carry, int(p.units_cap));
     p.plan[p.num_seqs] = p.units && carry > p.units_cap ? int(p.units_cap) : carry;
@@ -373,7 +373,14 @@ __global__ void __launch_bounds__(ExtCfg<D, BS>::kThreads)
   // rows of this lane: r0 = lane / 4 and r0 + 8 of the tile
   const int r0 = lane >> 2, cq = (lane & 3) * 2;
 
-  for (int u = blockIdx.x * NW + warp; u < total; u += gridDim.x * NW) {
+  // units from the plan's queue (lane 0 takes the next one), or round-robin without one
+  auto next_unit = [&](int cur) -> int {
+    if (!p.queue) return cur < 0 ? int(blockIdx.x) * NW + warp : cur + int(gridDim.x) * NW;
+    int v = 0;
+    if (lane == 0) v = atomicAdd(p.queue, 1);
+    return __shfl_sync(kFull, v, 0);
+  };
+  for (int u = next_unit(-1); u < total; u = next_unit(u)) {
     const ExtUnit x = ext_make_unit<BS>(p, u, total, QPT, lane);
     // query index, position and output row of the lane's two rows (-1: no such query)
     int qpos[2], tok[2], head[2];
@@ -921,7 +928,14 @@ __global__ void __launch_bounds__(Fp8Cfg<D, BS>::kThreads) extend_fp8_kernel(con
   uint32_t consumed = 0;
   const int r0 = lane >> 2, cq = (lane & 3) * 2;
 
-  for (int u = blockIdx.x * NW + warp; u < total; u += gridDim.x * NW) {
+  // units from the plan's queue (lane 0 takes the next one), or round-robin without one
+  auto next_unit = [&](int cur) -> int {
+    if (!p.queue) return cur < 0 ? int(blockIdx.x) * NW + warp : cur + int(gridDim.x) * NW;
+    int v = 0;
+    if (lane == 0) v = atomicAdd(p.queue, 1);
+    return __shfl_sync(kFull, v, 0);
+  };
+  for (int u = next_unit(-1); u < total; u = next_unit(u)) {
     const ExtUnit x = ext_make_unit<BS>(p, u, total, QPT, lane);
     int qpos[2], tok[2], head[2];
 #pragma unroll
@@ -1363,7 +1377,7 @@ static pa_status extend_impl(const void* q, int32_t q_dtype, int32_t num_seqs, i
   p.part_ml = reinterpret_cast<float*>(w + ws.ml);
   p.part_acc = reinterpret_cast<float*>(w + ws.acc);
   p.units = reinterpret_cast<int4*>(w + ws.units);
-  p.queue = tc ? reinterpret_cast<int*>(w + ws.queue) : nullptr;
+  p.queue = reinterpret_cast<int*>(w + ws.queue);
   p.row_parts = nullptr;   // set below when a merge pass follows
   p.units_cap = (long long)ext_units_bound(num_tokens, num_q_heads, max_parts);
   p.fresh = fresh ? 1 : 0;
