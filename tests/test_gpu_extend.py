@@ -239,6 +239,45 @@ def test_spec4_mix_every_row():
     assert_close(out.double().cpu().numpy()[idx], want, w.kv_dtype, "spec4 mix, every row")
 
 
+@pytest.mark.parametrize("kv", ["bf16", "e4m3"])
+def test_repeated_calls_share_one_workspace(kv):
+    """The short-run kernels' warps take their units from a counter in the workspace that the
+    plan kernel zeroes on every call: three calls with one workspace (and a different draft
+    count in between) give bit-identical outputs, each against the oracle."""
+    lens = [3, 40, 511, 512, 900, 1500, 2100, 64]
+    w = synthetic.custom(len(lens), 4, 4, 128, 16 if kv == "bf16" else 32, kv, "bf16", lens, 91)
+    eng = make_engine(w, DEV)
+    fill_cache(w, eng)   # E4M3: codes with per-tensor scales
+    for s, L in enumerate(lens):
+        eng.extend(s, L)
+    eng.upload_tables()
+    _nan_tails(w, eng)
+    T_max = 4 * len(lens)
+    ws = torch.empty(pa.extend_workspace_size(w.num_seqs, T_max, 4, 128, eng.max_context_len), dtype=torch.uint8,
+                     device=DEV)
+
+    def call(qlens, seed):
+        qs = np.concatenate([[0], np.cumsum(qlens)]).astype(np.int32)
+        q = synthetic.normal_values((int(qs[-1]), 4, 128), "bf16", seed).to(DEV)
+        out = torch.full_like(q, float("nan"))
+        pa.extend(q, eng.cache, torch.from_numpy(qs).to(DEV), eng.bt_dev, eng.lens_dev, eng.max_context_len, w.scale,
+                  out, ws)
+        torch.cuda.synchronize()
+        assert pa.last_device_error()[0] == 0
+        return q, qs, out
+
+    qlens = [min(4, L) for L in lens]
+    q, qs, first = call(qlens, 92)
+    _, _, other = call([1] * len(lens), 93)
+    _, _, again = call(qlens, 92)
+    assert torch.equal(first, again)
+    d = eng.cache.desc
+    want = oatt.paged_extend(codes_np(q), "bf16", codes_np(eng.k_cache), codes_np(eng.v_cache), w.kv_dtype,
+                             d.k_scale, d.v_scale, eng.bt_host.astype(np.int64), list(eng.lens), qs, w.scale)
+    assert_close(again.double().cpu().numpy(), want, w.kv_dtype, f"repeated extend calls, {kv} cache")
+    assert torch.isfinite(other).all()
+
+
 def test_long_context_many_chunks():
     """A 256-query chunk at the end of a 20000-token context, GQA 4: few units, so the
     context is cut into many chunks merged by log-sum-exp."""
