@@ -260,7 +260,8 @@ pa_status pa_decode_no_alloc(const void* q, int32_t q_dtype, int32_t num_seqs, i
  * and the output. These take the mma.sync path for runs of any length.
  * Supported: 16-bit caches with q_dtype == kv_dtype, or E4M3 caches with q_dtype PA_F16
  * or PA_BF16; head_dim 64 or 128, block_size 16 or 32, G in {1, 2, 4, 8}.
- * workspace >= pa_extend_workspace_size(...), 256-byte aligned.
+ * workspace >= pa_extend_workspace_size(...), 256-byte aligned. A call with num_seqs or
+ * num_tokens 0 checks its arguments and launches nothing.
  */
 pa_status pa_extend(const void* q, int32_t q_dtype, int32_t num_seqs, int32_t num_q_heads,
                     const int32_t* query_start, int32_t num_tokens, const pa_cache_desc* cache,

@@ -278,6 +278,24 @@ def test_repeated_calls_share_one_workspace(kv):
     assert torch.isfinite(other).all()
 
 
+def test_ragged_and_empty_batches():
+    """Sequences with no new token between others (ragged query_start), and a call with no
+    token at all: the others' rows match the oracle; the empty call is a no-op."""
+    lens = [9, 600, 33, 1200, 2]
+    qlens = [3, 0, 5, 0, 2]
+    w, eng, qs_dev, q, qs = _setup(lens, qlens, 8, 2, 128, 16, "bf16", 95)
+    out = _run(w, eng, qs_dev, q, qs)
+    assert pa.last_device_error()[0] == 0
+    assert_close(out.double().cpu().numpy(), _ref(w, eng, q, qs), "bf16", "ragged batch")
+    empty_q, empty_out = q[:0], out[:0]   # views: the pointers stay valid
+    qs0 = torch.zeros(len(lens) + 1, dtype=torch.int32, device=DEV)
+    ws = torch.empty(pa.extend_workspace_size(w.num_seqs, 1, 8, 128, eng.max_context_len), dtype=torch.uint8,
+                     device=DEV)
+    pa.extend(empty_q, eng.cache, qs0, eng.bt_dev, eng.lens_dev, eng.max_context_len, w.scale, empty_out, ws)
+    torch.cuda.synchronize()
+    assert pa.last_device_error()[0] == 0
+
+
 def test_long_context_many_chunks():
     """A 256-query chunk at the end of a 20000-token context, GQA 4: few units, so the
     context is cut into many chunks merged by log-sum-exp."""
