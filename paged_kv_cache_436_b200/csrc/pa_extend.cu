@@ -837,10 +837,14 @@ __device__ __forceinline__ uint32_t f16x2_satfinite(float lo, float hi) {
   return r;
 }
 
-// Two E4M3 codes (lo in the low byte) as an f16 pair (exact).
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
-  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two & 0xffffu), __NV_E4M3);
-  return uint32_t(h.x) | (uint32_t(h.y) << 16);
+// Four E4M3 codes (byte i = code i) as two f16 pairs (codes 0, 1 in lo; 2, 3 in hi), exact:
+// the hardware e4m3x2 -> f16x2 conversion on each 16-bit half of the word, the halves
+// taken apart by a register unpack rather than shifts.
+__device__ __forceinline__ void e4m3x4_to_f16x4(uint32_t four, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 c01, c23;\n\tmov.b32 {c01, c23}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, c01;\n\tcvt.rn.f16x2.e4m3x2 %1, c23;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(four));
 }
 
 // One block of E4M3 rows (BS x D bytes, row-major) into the f16 staging tile, rows from
@@ -863,10 +867,10 @@ __device__ __forceinline__ void fp8_block_to_f16(const uint8_t* src, uint8_t* ds
     uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
     if (r < keep) {
       const uint4 raw = *reinterpret_cast<const uint4*>(src + r * D + cb * 16);
-      a = make_uint4(e4m3x2_to_f16x2(raw.x), e4m3x2_to_f16x2(raw.x >> 16), e4m3x2_to_f16x2(raw.y),
-                     e4m3x2_to_f16x2(raw.y >> 16));
-      b = make_uint4(e4m3x2_to_f16x2(raw.z), e4m3x2_to_f16x2(raw.z >> 16), e4m3x2_to_f16x2(raw.w),
-                     e4m3x2_to_f16x2(raw.w >> 16));
+      e4m3x4_to_f16x4(raw.x, a.x, a.y);
+      e4m3x4_to_f16x4(raw.y, a.z, a.w);
+      e4m3x4_to_f16x4(raw.z, b.x, b.y);
+      e4m3x4_to_f16x4(raw.w, b.z, b.w);
     }
     *reinterpret_cast<uint4*>(dst + ext_swz<BS>(r, 2 * cb)) = a;
     *reinterpret_cast<uint4*>(dst + ext_swz<BS>(r, 2 * cb + 1)) = b;
